@@ -1,0 +1,53 @@
+"""Plant plausible mistakes in a copy of the oracle and check that the pins catch them.
+
+Each mutant is a one-line change to a copy of ``oracle/la_oracle.c`` (a dropped term,
+a wrong sign, a swapped operand, a read before the update).  The copy is compiled on
+the CPU into a temporary library and the pin suite is run against it in a child
+process; the pins must FAIL for every mutant.  The real oracle is never modified.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "la_oracle.c")
+
+MUTANTS = {
+    # mode 0
+    "phi_drops_plus_one": ("x > 0.0 ? x + 1.0 : exp(x)", "x > 0.0 ? x : exp(x)"),
+    "mode0_state_uses_query_feature": ("row[j] += v[i] * fk[j];", "row[j] += v[i] * fq[j];"),
+    "mode0_denominator_before_update": ("            z[j] += fk[j];\n            den += z[j] * fq[j];",
+                                        "            den += z[j] * fq[j];\n            z[j] += fk[j];"),
+    # mode 1
+    "mode1_drops_gate": ("row[j] = a * row[j] + v[i] * k[j];", "row[j] = row[j] + v[i] * k[j];"),
+    "mode1_reads_with_key": ("                row[j] = a * row[j] + v[i] * k[j];\n                acc += row[j] * q[j];",
+                             "                row[j] = a * row[j] + v[i] * k[j];\n                acc += row[j] * k[j];"),
+    # mode 2
+    "mode2_wrong_sign": ("row[j] = a * (row[j] - beta * sk[i] * k[j])", "row[j] = a * (row[j] + beta * sk[i] * k[j])"),
+    "mode2_correction_not_decayed": ("row[j] = a * (row[j] - beta * sk[i] * k[j]) + beta * v[i] * k[j];",
+                                     "row[j] = a * row[j] - beta * sk[i] * k[j] + beta * v[i] * k[j];"),
+    "mode2_write_drops_beta": ("- beta * sk[i] * k[j]) + beta * v[i] * k[j];", "- beta * sk[i] * k[j]) + v[i] * k[j];"),
+    "mode2_reads_old_state": ("                row[j] = a * (row[j] - beta * sk[i] * k[j]) + beta * v[i] * k[j];\n                acc += row[j] * q[j];",
+                              "                acc += row[j] * q[j];\n                row[j] = a * (row[j] - beta * sk[i] * k[j]) + beta * v[i] * k[j];"),
+    "mode2_correction_uses_query": ("acc += row[j] * k[j];\n            sk[i] = acc;", "acc += row[j] * q[j];\n            sk[i] = acc;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistakes(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mutant_c = tmp_path / "mutant.c"
+    mutant_c.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", str(mutant_c), "-o", str(lib), "-lm"],
+                   check=True)
+    env = dict(os.environ, LA_ORACLE_LIB_OVERRIDE=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"planted mistake {name} passed every pin:\n{r.stdout[-2000:]}"
+    assert "failed" in r.stdout or "error" in r.stdout.lower()

@@ -1,0 +1,132 @@
+"""Seeded synthetic inputs for the linear-attention workloads.
+
+This module is shared by the tests, the benchmark and the smoke check.  It holds the
+input recipes only -- shapes, distributions, seeds and draw order -- and none of the
+method's arithmetic.  Both the fp64 oracle and the CUDA library receive the tensors it
+returns (the oracle after an exact upcast to fp64).
+
+Draw order is fixed: q, k, v, gate pre-activation x, beta pre-activation y (and, for
+decode, the initial state first).  Gates are stored as values a_t in (0, 1], not logs.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+MODE_ELU1_NORM = 0
+MODE_GATED = 1
+MODE_GATED_DELTA = 2
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    mode: int
+    dtype: torch.dtype          # q, k, v, o; state, z, gate and beta are always fp32
+    B: int                      # batch (prefill) or sequences N (decode)
+    H: int
+    T: int                      # tokens per sequence (prefill) or decode steps
+    dk: int
+    dv: int
+    seed: int
+    chunk: int = 0              # 0 -> the library default
+    qk_scale: float = 1.0       # q, k ~ N(0,1) * qk_scale
+    v_scale: float = 1.0
+    qk_l2norm: bool = False     # L2-normalise q, k rows in fp32 before the cast
+    gate: str = "none"          # "none" | "softplus" (a = exp(-softplus(x + gate_shift)))
+    gate_shift: float = 0.0
+    beta: bool = False          # beta = sigmoid(y), y ~ N(0,1)
+    decode: bool = False
+    state_std: float = 0.0      # decode: initial state ~ N(0, state_std^2)
+
+    @property
+    def tokens(self) -> int:
+        """Tokens processed per step: B*T for prefill, N for one decode step."""
+        return self.B if self.decode else self.B * self.T
+
+
+# The five workloads, restated from the task's configuration list.
+CONFIGS = {
+    "elu1_f32_small": Workload("elu1_f32_small", MODE_ELU1_NORM, torch.float32, B=1, H=2, T=256,
+                               dk=64, dv=64, seed=1),
+    "elu1_bf16_b4h16t4096": Workload("elu1_bf16_b4h16t4096", MODE_ELU1_NORM, torch.bfloat16, B=4,
+                                     H=16, T=4096, dk=128, dv=128, seed=2, chunk=64,
+                                     qk_scale=1 / math.sqrt(128), v_scale=1 / math.sqrt(128)),
+    "gated_bf16_b8h16t8192": Workload("gated_bf16_b8h16t8192", MODE_GATED, torch.bfloat16, B=8,
+                                      H=16, T=8192, dk=128, dv=128, seed=3,
+                                      qk_scale=1 / math.sqrt(128), gate="softplus"),
+    "gdn_bf16_b2h16t32768": Workload("gdn_bf16_b2h16t32768", MODE_GATED_DELTA, torch.bfloat16,
+                                     B=2, H=16, T=32768, dk=128, dv=128, seed=4, qk_l2norm=True,
+                                     gate="softplus", beta=True),
+    "gdn_decode_n256h32": Workload("gdn_decode_n256h32", MODE_GATED_DELTA, torch.bfloat16, B=256,
+                                   H=32, T=1000, dk=128, dv=128, seed=5, qk_l2norm=True,
+                                   gate="softplus", beta=True, decode=True, state_std=0.02),
+}
+
+
+def _qkv(w: Workload, gen: torch.Generator, device, lead):
+    """Draw q, k, v (in that order) with leading shape `lead`."""
+    q = torch.randn(*lead, w.dk, generator=gen, device=device, dtype=torch.float32)
+    k = torch.randn(*lead, w.dk, generator=gen, device=device, dtype=torch.float32)
+    v = torch.randn(*lead, w.dv, generator=gen, device=device, dtype=torch.float32)
+    if w.qk_l2norm:
+        q = q / q.norm(dim=-1, keepdim=True)
+        k = k / k.norm(dim=-1, keepdim=True)
+    else:
+        q = q * w.qk_scale
+        k = k * w.qk_scale
+    v = v * w.v_scale
+    return q.to(w.dtype), k.to(w.dtype), v.to(w.dtype)
+
+
+def _gates(w: Workload, gen: torch.Generator, device, lead):
+    gate = beta = None
+    if w.gate == "softplus":
+        x = torch.randn(*lead, generator=gen, device=device, dtype=torch.float32)
+        # a = exp(-softplus(x)) = sigmoid(-x): a value in (0, 1)
+        gate = torch.exp(-torch.nn.functional.softplus(x + w.gate_shift))
+    elif w.gate != "none":
+        raise ValueError(f"unknown gate recipe {w.gate!r}")
+    if w.beta:
+        y = torch.randn(*lead, generator=gen, device=device, dtype=torch.float32)
+        beta = torch.sigmoid(y)
+    return gate, beta
+
+
+def prefill_inputs(w: Workload, device="cpu", init_state_std: float = 0.0):
+    """q,k [B,H,T,d_k], v [B,H,T,d_v] in w.dtype; gate, beta [B,H,T] fp32 or None;
+    state0 [B,H,d_v,d_k] fp32 (zeros unless init_state_std > 0)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    lead = (w.B, w.H, w.T)
+    q, k, v = _qkv(w, gen, device, lead)
+    gate, beta = _gates(w, gen, device, lead)
+    if init_state_std > 0:
+        state0 = torch.randn(w.B, w.H, w.dv, w.dk, generator=gen, device=device) * init_state_std
+    else:
+        state0 = torch.zeros(w.B, w.H, w.dv, w.dk, device=device)
+    return dict(q=q, k=k, v=v, gate=gate, beta=beta, state0=state0)
+
+
+def decode_inputs(w: Workload, steps: int | None = None, device="cpu", n_seqs: int | None = None):
+    """Initial state [N,H,d_v,d_k] ~ N(0, state_std^2) and per-step inputs stacked over
+    steps: q,k [steps,N,H,d_k], v [steps,N,H,d_v], gate, beta [steps,N,H]."""
+    steps = w.T if steps is None else steps
+    N = w.B if n_seqs is None else n_seqs
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    state0 = torch.randn(N, w.H, w.dv, w.dk, generator=gen, device=device) * w.state_std
+    lead = (steps, N, w.H)
+    q, k, v = _qkv(w, gen, device, lead)
+    gate, beta = _gates(w, gen, device, lead)
+    z0 = None
+    if w.mode == MODE_ELU1_NORM:
+        z0 = torch.rand(N, w.H, w.dk, generator=gen, device=device) + 1.0
+    return dict(state0=state0, z0=z0, q=q, k=k, v=v, gate=gate, beta=beta)
+
+
+def variant(w: Workload, **changes) -> Workload:
+    """A copy of a workload with some fields changed (smaller sizes, weaker decay ...)."""
+    return dataclasses.replace(w, **changes)
