@@ -1,0 +1,590 @@
+"""Benchmark: causal linear attention prefill / decode on B200 through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one call of the hot path over one batch of the workload's synthetic input
+(prefill: la_prefill over B x T tokens; decode: la_decode_step for N sequences).  The
+default workload is the ungated elu+1 prefill (bf16, B=4, H=16, T=4096, d=128, chunk 64);
+``--extras`` (default on at N=1) also measures the other three workloads and reports
+them under "workloads".  Prints ONE JSON line on rank 0.
+
+Under torchrun each rank runs its own copy of the workload on its own GPU (independent
+sequences, no collective on the data path: weak scaling); the timed region is bracketed
+by a barrier and a device synchronise, and the max over ranks is reported.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload
+(the only other place this file runs the oracle is the cpu_baseline leg).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = "elu1_bf16_b4h16t4096"
+METRIC = "prefill tokens/s + % tensor roofline; decode tokens/s + HBM GB/s (1×B200)"
+L2_FLUSH_BYTES = 256 << 20          # > 126 MB L2
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, local, backend="nccl"):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def barrier(dist, device):
+    if dist is not None:
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(dist, x: float, device) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(dist, x: float, device) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------------
+# workload accounting (algorithmic work, not what a kernel happens to do)
+# ----------------------------------------------------------------------------------
+
+def io_bytes(dtype):
+    return 2 if dtype == torch.bfloat16 else 4
+
+
+def prefill_algorithmic(w: W.Workload, C=64):
+    """Bytes that must cross HBM once and flops of the chunked form at chunk C = 64.
+
+    bytes: q, k, v read + o written, gates/beta read, final state (and z) written.
+    flops per token-head: modes 0/1  2C d_k + 2C d_v + 4 d_k d_v;
+                          mode 2     10 C d + 6 d^2 + C^2 / 3  (d = d_k = d_v)."""
+    th = w.B * w.H * w.T
+    e = io_bytes(w.dtype)
+    b = th * e * (2 * w.dk + 2 * w.dv)
+    if w.gate != "none":
+        b += th * 4
+    if w.beta:
+        b += th * 4
+    b += w.B * w.H * (w.dv * w.dk * 4 + (w.dk * 4 if w.mode == 0 else 0))
+    if w.mode == 2:
+        d = w.dk
+        f = 10 * C * d + 6 * d * d + C * C / 3.0
+    else:
+        f = 2 * C * w.dk + 2 * C * w.dv + 4 * w.dk * w.dv
+    return float(b), float(th * f)
+
+
+def decode_algorithmic(w: W.Workload):
+    """Per decode step: state read + write (fp32), q,k,v read, o written, a/beta read."""
+    nh = w.B * w.H
+    e = io_bytes(w.dtype)
+    b = nh * (2 * w.dk * w.dv * 4 + e * (2 * w.dk + 2 * w.dv))
+    if w.gate != "none":
+        b += nh * 4
+    if w.beta:
+        b += nh * 4
+    if w.mode == 0:
+        b += nh * 2 * w.dk * 4
+    f = nh * 8 * w.dk * w.dv
+    return float(b), float(f)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_sources_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_attention_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if it is for these sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t[kernel_key]
+        if e.get("sources_sha") != kernel_sources_sha():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------------
+# clocks during the timed region (NVML, the library nvidia-smi reads)
+# ----------------------------------------------------------------------------------
+
+class ClockSampler:
+    BAD = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+           "hw_power_brake_slowdown": 0x80}
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+             0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+             0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            idx = device_index
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                idx = int(vis.split(",")[device_index])
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thr is not None:
+            self._stop.set()
+            self._thr.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"],
+                    "samples": 0}
+        reasons = [n for bit, n in self.NAMES.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------------
+# one workload on one GPU
+# ----------------------------------------------------------------------------------
+
+class PrefillCase:
+    def __init__(self, la, w: W.Workload, device, rank):
+        self.la, self.w, self.device = la, w, device
+        wr = W.variant(w, seed=w.seed + 1000 * rank)
+        self.inp = W.prefill_inputs(wr, device=device)
+        self.state = torch.empty(w.B, w.H, w.dv, w.dk, device=device)
+        self.z = torch.empty(w.B, w.H, w.dk, device=device) if w.mode == 0 else None
+        self.o = torch.empty(w.B, w.H, w.T, w.dv, device=device, dtype=w.dtype)
+        self.tokens = w.B * w.T
+        self.bytes, self.flops = prefill_algorithmic(w)
+        self.kind = "prefill"
+
+    def step(self):
+        i = self.inp
+        self.la.prefill(i["q"], i["k"], i["v"], mode=self.w.mode, gate=i["gate"], beta=i["beta"],
+                        state=self.state, z=self.z, o=self.o, chunk=self.w.chunk,
+                        init_state=False)
+
+    def e2e_setup(self):
+        pin = lambda t: None if t is None else t.to("cpu").pin_memory()
+        self.h_in = {k: pin(v) for k, v in self.inp.items() if k in ("q", "k", "v", "gate", "beta")}
+        self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.h_state = torch.empty(self.state.shape, dtype=torch.float32).pin_memory()
+        self.h_z = None if self.z is None else torch.empty(self.z.shape).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values() if t is not None)
+        self.d2h = self.h_o.numel() * self.h_o.element_size() + self.h_state.numel() * 4 + (
+            0 if self.h_z is None else self.h_z.numel() * 4)
+
+    def e2e_step(self):
+        """Host buffers in, host buffers out: copies on the stream, then the ABI call."""
+        h = self.h_in
+        d = {k: (None if v is None else self.inp[k]) for k, v in h.items()}
+        for k, v in h.items():
+            if v is not None:
+                d[k].copy_(v, non_blocking=True)
+        self.la.prefill(d["q"], d["k"], d["v"], mode=self.w.mode, gate=d["gate"], beta=d["beta"],
+                        state=self.state, z=self.z, o=self.o, chunk=self.w.chunk, init_state=False)
+        self.h_o.copy_(self.o, non_blocking=True)
+        self.h_state.copy_(self.state, non_blocking=True)
+        if self.h_z is not None:
+            self.h_z.copy_(self.z, non_blocking=True)
+
+
+class DecodeCase:
+    """One step = one la_decode_step over N sequences; the timed loop walks the
+    pre-generated per-token inputs so that every step reads fresh q, k, v, a, beta."""
+
+    def __init__(self, la, w: W.Workload, device, rank, steps_needed):
+        self.la, self.w, self.device = la, w, device
+        wr = W.variant(w, seed=w.seed + 1000 * rank)
+        self.n_inputs = max(1, min(steps_needed, w.T))
+        self.inp = W.decode_inputs(wr, steps=self.n_inputs, device=device)
+        self.state = self.inp["state0"].clone()
+        self.z = None if self.inp["z0"] is None else self.inp["z0"].clone()
+        self.o = torch.empty(w.B, w.H, w.dv, device=device, dtype=w.dtype)
+        self.t = 0
+        self.tokens = w.B
+        self.bytes, self.flops = decode_algorithmic(w)
+        self.kind = "decode"
+
+    def step(self):
+        i, t = self.inp, self.t % self.n_inputs
+        self.t += 1
+        self.la.decode_step(i["q"][t], i["k"][t], i["v"][t], mode=self.w.mode, state=self.state,
+                            gate=None if i["gate"] is None else i["gate"][t],
+                            beta=None if i["beta"] is None else i["beta"][t], z=self.z, o=self.o)
+
+    def e2e_setup(self):
+        t0 = 0
+        pin = lambda t: None if t is None else t[t0].to("cpu").pin_memory()
+        self.h_in = {k: pin(self.inp[k]) for k in ("q", "k", "v", "gate", "beta")}
+        self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values() if t is not None)
+        self.d2h = self.h_o.numel() * self.h_o.element_size()
+        self.d_in = {k: (None if v is None else torch.empty_like(v, device=self.device))
+                     for k, v in self.h_in.items()}
+
+    def e2e_step(self):
+        """Per token: copy q, k, v, a, beta in from pinned host memory, step the resident
+        state, copy o back (the state stays on the device, as in serving)."""
+        for k, v in self.h_in.items():
+            if v is not None:
+                self.d_in[k].copy_(v, non_blocking=True)
+        d = self.d_in
+        self.la.decode_step(d["q"], d["k"], d["v"], mode=self.w.mode, state=self.state,
+                            gate=d["gate"], beta=d["beta"], z=self.z, o=self.o)
+        self.h_o.copy_(self.o, non_blocking=True)
+
+
+def time_steps(case, steps, warmup, dist, device, flush, fn=None, sampler=None):
+    """Device time of `steps` calls of fn (default case.step), each bracketed by CUDA events
+    on the launching stream, with an L2 flush between steps (outside the events)."""
+    fn = fn or case.step
+    stream = torch.cuda.current_stream(device)
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    n0 = case.la.kernel_launches()
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        for i in range(steps):
+            if flush is not None:
+                flush.zero_()
+            starts[i].record(stream)
+            fn()
+            ends[i].record(stream)
+        torch.cuda.synchronize(device)
+    launches = case.la.kernel_launches() - n0
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return ms, launches
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def measure(la, name, args, dist, device, rank, world, flush, with_e2e, sampler=None):
+    w = W.CONFIGS[name]
+    case = (DecodeCase(la, w, device, rank, args.warmup + args.steps) if w.decode
+            else PrefillCase(la, w, device, rank))
+    ms, launches = time_steps(case, args.steps, args.warmup, dist, device, flush, sampler=sampler)
+    la.check_status()
+    total_ms = max_over_ranks(dist, sum(ms), device)
+    tokens_all = sum_over_ranks(dist, case.tokens * args.steps, device)
+    per_launch_ms = statistics.mean(ms) / max(1, launches // max(1, args.steps))
+    peaks, peak_src = load_peaks()
+    achieved_gbs = case.bytes / (statistics.mean(ms) * 1e-3) / 1e9
+    achieved_tflops = case.flops / (statistics.mean(ms) * 1e-3) / 1e12
+    res = {
+        "workload": name,
+        "tokens_per_s": tokens_all / (total_ms * 1e-3),
+        "ms_per_step": total_ms / args.steps,
+        "ms_per_step_median": statistics.median(ms),
+        "launches_per_step": launches / args.steps,
+        "algorithmic_bytes_per_step": case.bytes,
+        "algorithmic_flops_per_step": case.flops,
+        "hbm_gbs": achieved_gbs,
+        "hbm_frac": achieved_gbs / peaks["hbm_gbs"],
+        "tensor_tflops": achieved_tflops,
+        "tensor_frac": achieved_tflops / peaks["bf16_tflops"],
+        "attainable_frac": max(case.bytes / (peaks["hbm_gbs"] * 1e9),
+                               case.flops / (peaks["bf16_tflops"] * 1e12)) / (statistics.mean(ms) * 1e-3),
+        "peak_source": peak_src,
+        "_case": case, "_ms": ms, "_launches": launches, "_per_launch_ms": per_launch_ms,
+    }
+    if with_e2e:
+        case.e2e_setup()
+        e_ms, _ = time_steps(case, max(3, args.steps // 2), 2, dist, device, None, fn=case.e2e_step)
+        e_total = max_over_ranks(dist, sum(e_ms), device)
+        e_tokens = sum_over_ranks(dist, case.tokens * len(e_ms), device)
+        res["e2e"] = {"value": e_tokens / (e_total * 1e-3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": int(case.h2d), "d2h_bytes_per_step": int(case.d2h)}
+    return res
+
+
+# ----------------------------------------------------------------------------------
+# the oracle on host cores
+# ----------------------------------------------------------------------------------
+
+def oracle_sample(name, budget_s=10.0):
+    """Time the fp64 oracle on a bounded sample of the workload.  Returns a dict with
+    tokens/s (in the workload's token unit), the cores used and a description."""
+    import numpy as np
+    import oracle
+    w = W.CONFIGS[name]
+    threads = oracle.max_threads()
+    gen_w = W.variant(w, B=1, H=min(w.H, max(1, threads)), T=min(w.T, 4096) if not w.decode else w.T)
+    if w.decode:
+        inp = W.decode_inputs(w, steps=1, device="cpu", n_seqs=max(1, threads // w.H + 1))
+        f = lambda t: None if t is None else t.to(torch.float64).numpy()
+        q, k, v = f(inp["q"][0]), f(inp["k"][0]), f(inp["v"][0])
+        g, b = f(inp["gate"][0]) if inp["gate"] is not None else None, f(inp["beta"][0]) if inp["beta"] is not None else None
+        S = f(inp["state0"])
+        z = f(inp["z0"]) if inp["z0"] is not None else None
+        n_seq = q.shape[0]
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            oracle.decode_step(w.mode, q, k, v, g, b, S, z)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s or reps >= 10000:
+                break
+        return {"value": reps * n_seq / el, "unit": "tokens/s", "cores": min(threads, n_seq * w.H),
+                "kind": "oracle",
+                "sample": f"{reps} decode steps of {n_seq} sequences x {w.H} heads (fp64 C, OpenMP)"}
+    inp = W.prefill_inputs(gen_w, device="cpu")
+    f = lambda t: None if t is None else t.to(torch.float64).numpy()
+    args = [f(inp[x]) for x in ("q", "k", "v", "gate", "beta")]
+    # time growing prefixes until the budget is reached
+    T = min(256, gen_w.T)
+    el = 0.0
+    while True:
+        sl = [None if a is None else a[:, :, :T] for a in args]
+        t0 = time.perf_counter()
+        oracle.prefill(w.mode, *sl)
+        el = time.perf_counter() - t0
+        if el * 2 > budget_s or T >= gen_w.T:
+            break
+        T = min(gen_w.T, T * 2)
+    heads = gen_w.H
+    token_heads_per_s = heads * T / el
+    return {"value": token_heads_per_s / w.H, "unit": "tokens/s", "cores": min(threads, heads),
+            "kind": "oracle",
+            "sample": f"{heads} heads x {T} tokens of the workload's recipe (fp64 recurrent C, "
+                      f"OpenMP over heads); tokens/s counts all {w.H} heads of a token"}
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    name = args.workload
+    per_step = []
+    res = None
+    for i in range(args.warmup + args.steps):
+        res = oracle_sample(name, budget_s=max(0.5, min(5.0, 120.0 / (args.warmup + args.steps))))
+        if i >= args.warmup:
+            per_step.append(res["value"])
+    value = statistics.mean(per_step)
+    w = W.CONFIGS[name]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": (w.tokens / value) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": name, "mode": w.mode, "B": w.B, "H": w.H, "T": w.T, "d_k": w.dk,
+                   "d_v": w.dv, "io_dtype": str(w.dtype).replace("torch.", ""),
+                   "parallelism": "host cores (OpenMP over heads)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": res["cores"],
+                         "kind": "oracle", "sample": res["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--extras", type=int, default=-1,
+                    help="1: also measure the other workloads (default: on at N=1)")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world, rank, local = dist_env()
+    if world > 1 and args.gpus != world:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    dist = init_dist(world, local)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+
+    import gated_delta_rule_attention_b200 as la
+    la.library()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    sampler = ClockSampler(local)
+    main_res = measure(la, args.workload, args, dist, device, rank, world, flush, True,
+                       sampler=sampler)
+    extras = {}
+    do_extras = (world == 1) if args.extras < 0 else bool(args.extras)
+    if do_extras:
+        for name in ("elu1_bf16_b4h16t4096", "gated_bf16_b8h16t8192", "gdn_bf16_b2h16t32768",
+                     "gdn_decode_n256h32"):
+            if name == args.workload:
+                continue
+            r = measure(la, name, args, dist, device, rank, world, flush, False)
+            extras[name] = {k: v for k, v in r.items() if not k.startswith("_")}
+            del r
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1:
+        try:
+            cpu = oracle_sample(args.workload, budget_s=args.cpu_budget)
+        except Exception as e:  # the oracle is optional context, never the measurement
+            cpu = {"value": None, "error": str(e)[:200], "kind": "oracle"}
+
+    peaks, peak_src = load_peaks()
+    w = W.CONFIGS[args.workload]
+    case = main_res["_case"]
+    mean_ms = statistics.mean(main_res["_ms"])
+    hbm_bound = case.bytes / (peaks["hbm_gbs"] * 1e9) >= case.flops / (peaks["bf16_tflops"] * 1e12)
+    per_launch_s = main_res["_per_launch_ms"] * 1e-3
+    if hbm_bound:
+        achieved = case.bytes / max(1, round(main_res["launches_per_step"])) / per_launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        achieved = case.flops / max(1, round(main_res["launches_per_step"])) / per_launch_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
+    roof["traffic"] = ncu_traffic(args.workload)
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    roof["tensor_frac"] = main_res["tensor_frac"]
+    roof["hbm_frac"] = main_res["hbm_frac"]
+    roof["attainable_frac"] = main_res["attainable_frac"]
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": main_res["tokens_per_s"],
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": main_res["ms_per_step"],
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "mode": w.mode, "B": w.B, "H": w.H, "T": w.T,
+                       "d_k": w.dk, "d_v": w.dv, "chunk": w.chunk or "default",
+                       "global_batch": w.B * world, "seq_len": w.T,
+                       "parallelism": f"dp{world} (independent sequences per GPU)",
+                       "l2": "flushed between timed steps (256 MiB write)",
+                       "state_dtype": "f32", "accum": "f32"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": main_res.get("e2e"),
+            "gpu_launches": int(main_res["_launches"]),
+            "clocks": sampler.summary(),
+            "workloads": extras,
+        }
+        print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

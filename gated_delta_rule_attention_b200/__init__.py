@@ -1,0 +1,262 @@
+"""Causal linear attention for NVIDIA B200 (sm_100a): Python binding of liblinattn.
+
+The compute path is the C ABI declared in ``include/la.h`` and implemented by the CUDA
+kernels under ``csrc/``.  This module only marshals arguments (ctypes): it checks
+shapes and dtypes, allocates outputs with torch when the caller does not pass them,
+and forwards raw device pointers and the current CUDA stream.  Every step of the
+method runs in the library's kernels; there is no Python or CPU fallback, and the
+import fails loudly if the library is missing.
+
+Three modes, named after the variants on the lesson page "Linear attention and hybrids":
+
+* ``MODE_ELU1_NORM`` -- phi(x) = elu(x)+1 with the z normaliser (section "The kernel trick")
+* ``MODE_GATED`` -- scalar decay gate a_t (section "Memory must forget: decay and gates")
+* ``MODE_GATED_DELTA`` -- the Gated DeltaNet update (section "The delta rule and Gated DeltaNet")
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["MODE_ELU1_NORM", "MODE_GATED", "MODE_GATED_DELTA", "FLAG_INIT_STATE", "LaError",
+           "prefill", "decode_step", "check_status", "library", "library_path", "version",
+           "kernel_launches", "workspace_size"]
+
+MODE_ELU1_NORM = 0
+MODE_GATED = 1
+MODE_GATED_DELTA = 2
+FLAG_INIT_STATE = 1
+
+LA_F32 = 0
+LA_BF16 = 1
+_STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_CUDA",
+           4: "LA_ERR_TIMEOUT"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liblinattn.so")
+_lib = None
+
+
+class LaError(RuntimeError):
+    """A non-zero la_status_t from the library."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = library().la_status_string(status).decode()
+        super().__init__(f"{where}: {msg}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library():
+    """Load liblinattn.so (ctypes).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"liblinattn.so is not built ({_LIB_PATH}); run "
+                          "`python -m gated_delta_rule_attention_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, fp = ctypes.c_void_p, ctypes.c_void_p
+    i, u = ctypes.c_int, ctypes.c_uint
+    lib.la_prefill.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, fp, fp, fp, fp, vp, i, u, vp,
+                               ctypes.c_size_t, vp]
+    lib.la_prefill.restype = i
+    lib.la_decode_step.argtypes = [i, i, i, i, i, i, vp, vp, vp, fp, fp, fp, fp, vp, vp]
+    lib.la_decode_step.restype = i
+    lib.la_prefill_workspace_size.argtypes = [i, i, i, i, i, i, i, i]
+    lib.la_prefill_workspace_size.restype = ctypes.c_size_t
+    lib.la_check_status.argtypes = [vp]
+    lib.la_check_status.restype = i
+    lib.la_status_string.argtypes = [i]
+    lib.la_status_string.restype = ctypes.c_char_p
+    lib.la_version.argtypes = []
+    lib.la_version.restype = i
+    lib.la_kernel_launches.argtypes = []
+    lib.la_kernel_launches.restype = ctypes.c_ulonglong
+    _lib = lib
+    return lib
+
+
+def version() -> int:
+    return int(library().la_version())
+
+
+def kernel_launches() -> int:
+    """Kernels the library has enqueued in this process so far."""
+    return int(library().la_kernel_launches())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _io_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return LA_BF16
+    if t.dtype == torch.float32:
+        return LA_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _stream_handle(device: torch.device, stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise LaError(status, where)
+
+
+def _need(t, shape, dtype, name):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+_workspaces: dict = {}
+
+
+def workspace_size(mode: int, dtype: torch.dtype, B: int, H: int, T: int, d_k: int, d_v: int,
+                   chunk: int = 0) -> int:
+    """Bytes of scratch ``la_prefill`` can use for these sizes (0 if none)."""
+    dt = LA_BF16 if dtype == torch.bfloat16 else LA_F32
+    return int(library().la_prefill_workspace_size(int(mode), dt, B, H, T, d_k, d_v, int(chunk)))
+
+
+def _workspace(device: torch.device, nbytes: int):
+    """A per-device scratch buffer (torch allocation), grown on demand and reused.
+    Calls on different streams of one device must pass their own workspace."""
+    if nbytes <= 0:
+        return None
+    buf = _workspaces.get(device)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _workspaces[device] = buf
+    return buf
+
+
+def prefill(q, k, v, *, mode: int, gate=None, beta=None, state=None, z=None, o=None,
+            chunk: int = 0, init_state: bool | None = None, stream=None, workspace="auto"):
+    """Chunked prefill over whole sequences (``la_prefill``).
+
+    q, k: [B,H,T,d_k]; v: [B,H,T,d_v] (bf16 or fp32, one dtype); gate, beta: [B,H,T] fp32;
+    state: [B,H,d_v,d_k] fp32 (read as S_0 when ``init_state``, default: when given);
+    z: [B,H,d_k] fp32 (mode 0).  Returns (o, state, z).
+
+    CUDA tensors run in place on the current stream.  If the inputs are CPU tensors they
+    are copied to the current CUDA device, the call runs there, and the outputs are
+    copied back to the CPU (the end-to-end path); the computation is still the kernel's.
+    """
+    host = q.device.type == "cpu"
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        move = (lambda t: None if t is None else t.to(dev, non_blocking=True))
+        res = prefill(move(q), move(k), move(v), mode=mode, gate=move(gate), beta=move(beta),
+                      state=move(state), z=move(z), o=None, chunk=chunk,
+                      init_state=init_state if init_state is not None else state is not None,
+                      stream=stream)
+        back = tuple(None if t is None else t.to("cpu") for t in res)
+        if o is not None:
+            o.copy_(back[0])
+            back = (o,) + back[1:]
+        return back
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    dtype = _io_dtype(q)
+    _need(q, (B, H, T, dk), dt, "q")
+    _need(k, (B, H, T, dk), dt, "k")
+    _need(v, (B, H, T, dv), dt, "v")
+    if gate is not None:
+        _need(gate, (B, H, T), torch.float32, "gate")
+    if beta is not None:
+        _need(beta, (B, H, T), torch.float32, "beta")
+    if init_state is None:
+        init_state = state is not None
+    if state is None:
+        state = torch.empty(B, H, dv, dk, device=q.device, dtype=torch.float32)
+    _need(state, (B, H, dv, dk), torch.float32, "state")
+    if mode == MODE_ELU1_NORM:
+        if z is None:
+            if init_state:
+                raise ValueError("mode 0 with init_state needs z")
+            z = torch.empty(B, H, dk, device=q.device, dtype=torch.float32)
+        _need(z, (B, H, dk), torch.float32, "z")
+    if o is None:
+        o = torch.empty(B, H, T, dv, device=q.device, dtype=dt)
+    _need(o, (B, H, T, dv), dt, "o")
+    if isinstance(workspace, str):
+        ws = _workspace(q.device, workspace_size(mode, dt, B, H, T, dk, dv, chunk)) \
+            if workspace == "auto" else None
+    else:
+        ws = workspace
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    st = library().la_prefill(int(mode), dtype, B, H, T, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                              _ptr(gate), _ptr(beta), _ptr(state), _ptr(z), _ptr(o), int(chunk),
+                              FLAG_INIT_STATE if init_state else 0, _ptr(ws), ws_bytes,
+                              _stream_handle(q.device, stream))
+    _check(st, "la_prefill")
+    return o, state, (z if mode == MODE_ELU1_NORM else None)
+
+
+def decode_step(q, k, v, *, mode: int, state, gate=None, beta=None, z=None, o=None,
+                stream=None):
+    """One token for N sequences (``la_decode_step``), state updated in place.
+
+    q, k: [N,H,d_k]; v: [N,H,d_v]; gate, beta: [N,H] fp32; state: [N,H,d_v,d_k] fp32;
+    z: [N,H,d_k] fp32 (mode 0).  Returns (o, state, z).  CPU inputs take the end-to-end
+    path of ``prefill`` (copy in, run on the GPU, copy o, state and z back).
+    """
+    if q.device.type == "cpu":
+        dev = torch.device("cuda", torch.cuda.current_device())
+        move = (lambda t: None if t is None else t.to(dev, non_blocking=True))
+        s_dev, z_dev = move(state), move(z)
+        res = decode_step(move(q), move(k), move(v), mode=mode, state=s_dev, gate=move(gate),
+                          beta=move(beta), z=z_dev, stream=stream)
+        state.copy_(res[1].to("cpu"))
+        if z is not None:
+            z.copy_(res[2].to("cpu"))
+        o_host = res[0].to("cpu")
+        if o is not None:
+            o.copy_(o_host)
+            o_host = o
+        return o_host, state, z
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    dtype = _io_dtype(q)
+    _need(q, (N, H, dk), dt, "q")
+    _need(k, (N, H, dk), dt, "k")
+    _need(v, (N, H, dv), dt, "v")
+    _need(state, (N, H, dv, dk), torch.float32, "state")
+    if gate is not None:
+        _need(gate, (N, H), torch.float32, "gate")
+    if beta is not None:
+        _need(beta, (N, H), torch.float32, "beta")
+    if mode == MODE_ELU1_NORM:
+        _need(z, (N, H, dk), torch.float32, "z")
+    if o is None:
+        o = torch.empty(N, H, dv, device=q.device, dtype=dt)
+    _need(o, (N, H, dv), dt, "o")
+    st = library().la_decode_step(int(mode), dtype, N, H, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(gate), _ptr(beta), _ptr(state), _ptr(z), _ptr(o),
+                                  _stream_handle(q.device, stream))
+    _check(st, "la_decode_step")
+    return o, state, z
+
+
+def check_status(stream=None):
+    """Synchronise the stream and raise LaError if a kernel recorded a device failure."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(library().la_check_status(_stream_handle(dev, stream)), "la_check_status")

@@ -1,0 +1,189 @@
+// abi.cu -- the extern "C" boundary of liblinattn (declared in include/la.h).
+//
+// Host-side only: argument validation, chunk resolution, dispatch to a kernel launcher
+// on the caller's stream, and the device failure word.  No entry point allocates
+// device memory or keeps a pointer past its return.
+#include "la_internal.cuh"
+
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+namespace la {
+
+static std::atomic<unsigned long long> g_launches{0};
+void note_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+__device__ unsigned g_device_error;
+
+unsigned *device_error_word() {
+    constexpr int kMaxDevices = 64;
+    static unsigned *addr[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<unsigned *>(p);
+    }
+    return addr[dev];
+}
+
+namespace {
+
+constexpr long long kMaxElems = 1ll << 40;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// True if `p` is memory the current device can address as global memory.
+bool device_pointer(const void *p) {
+    if (!p) return false;
+    cudaPointerAttributes attr;
+    const cudaError_t err = cudaPointerGetAttributes(&attr, p);
+    if (err != cudaSuccess) {
+        (void)cudaGetLastError();  // clear the non-sticky error this query may leave
+        return false;
+    }
+    if (attr.type == cudaMemoryTypeManaged) return true;
+    if (attr.type != cudaMemoryTypeDevice) return false;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    return attr.device == dev;
+}
+
+bool tensor_ok(const void *p, uintptr_t align) { return p && aligned(p, align) && device_pointer(p); }
+
+la_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
+
+bool dims_ok(int dk, int dv) { return (dk == 64 || dk == 128) && (dv == 64 || dv == 128); }
+
+}  // namespace
+}  // namespace la
+
+using namespace la;
+
+extern "C" la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H, int T, int d_k,
+                                  int d_v, const void *q, const void *k, const void *v,
+                                  const float *gate, const float *beta, float *state, float *z,
+                                  void *o, int chunk, unsigned flags, void *workspace,
+                                  size_t workspace_bytes, void *stream) {
+    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_GATED_DELTA) return LA_ERR_INVALID_ARG;
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || T < 0) return LA_ERR_INVALID_ARG;
+    if (flags & ~LA_FLAG_INIT_STATE) return LA_ERR_INVALID_ARG;
+    if (chunk < 0) return LA_ERR_INVALID_ARG;
+    if (!dims_ok(d_k, d_v)) return LA_ERR_UNSUPPORTED;
+    const long long BH = (long long)B * H;
+    if (BH > INT32_MAX || BH * T * (long long)(d_k > d_v ? d_k : d_v) > kMaxElems)
+        return LA_ERR_INVALID_ARG;
+    const bool init = (flags & LA_FLAG_INIT_STATE) != 0;
+    if (!tensor_ok(state, 16)) return LA_ERR_INVALID_ARG;
+    if (mode == LA_MODE_ELU1_NORM && !tensor_ok(z, 16)) return LA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (init) return LA_OK;
+        cudaError_t e = cudaMemsetAsync(state, 0, sizeof(float) * BH * d_v * d_k, st);
+        if (e == cudaSuccess && mode == LA_MODE_ELU1_NORM)
+            e = cudaMemsetAsync(z, 0, sizeof(float) * BH * d_k, st);
+        return from_cuda(e);
+    }
+    if (!tensor_ok(q, 16) || !tensor_ok(k, 16) || !tensor_ok(v, 16) || !tensor_ok(o, 16))
+        return LA_ERR_INVALID_ARG;
+    if (mode != LA_MODE_ELU1_NORM && gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
+    if (mode == LA_MODE_GATED_DELTA && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
+
+    PrefillArgs a;
+    a.mode = mode;
+    a.dtype = dtype;
+    a.B = B; a.H = H; a.T = T; a.dk = d_k; a.dv = d_v;
+    a.q = q; a.k = k; a.v = v;
+    a.gate = (mode == LA_MODE_ELU1_NORM) ? nullptr : gate;
+    a.beta = (mode == LA_MODE_GATED_DELTA) ? beta : nullptr;
+    a.state = state;
+    a.z = (mode == LA_MODE_ELU1_NORM) ? z : nullptr;
+    a.o = o;
+    a.init_state = init;
+    a.stream = st;
+    if (workspace && workspace_bytes && !tensor_ok(workspace, 16)) return LA_ERR_INVALID_ARG;
+    if (prefill_tc_supports(dtype, d_k, d_v, chunk)) {
+        a.chunk = 64;
+        return from_cuda(launch_prefill_tc(a, workspace, workspace ? workspace_bytes : 0));
+    }
+    int resolved = 0;
+    if (!prefill_simt_supports(dtype, d_k, d_v, chunk, &resolved)) return LA_ERR_UNSUPPORTED;
+    a.chunk = resolved;
+    return from_cuda(launch_prefill_simt(a));
+}
+
+extern "C" size_t la_prefill_workspace_size(la_mode_t mode, la_dtype_t dtype, int B, int H, int T,
+                                            int d_k, int d_v, int chunk) {
+    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_GATED_DELTA || B < 1 || H < 1 || T < 1)
+        return 0;
+    if (!prefill_tc_supports(dtype, d_k, d_v, chunk)) return 0;
+    return prefill_tc_workspace_bytes(mode, B, H, T);
+}
+
+extern "C" la_status_t la_decode_step(la_mode_t mode, la_dtype_t dtype, int N, int H, int d_k,
+                                      int d_v, const void *q, const void *k, const void *v,
+                                      const float *gate, const float *beta, float *state,
+                                      float *z, void *o, void *stream) {
+    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_GATED_DELTA) return LA_ERR_INVALID_ARG;
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (N < 1 || H < 1) return LA_ERR_INVALID_ARG;
+    if (!dims_ok(d_k, d_v)) return LA_ERR_UNSUPPORTED;
+    const long long NH = (long long)N * H;
+    if (NH > INT32_MAX) return LA_ERR_INVALID_ARG;
+    const uintptr_t io_align = dtype == LA_BF16 ? 2 : 4;
+    if (!tensor_ok(q, io_align) || !tensor_ok(k, io_align) || !tensor_ok(v, io_align) ||
+        !tensor_ok(o, io_align) || !tensor_ok(state, 16))
+        return LA_ERR_INVALID_ARG;
+    if (mode == LA_MODE_ELU1_NORM && !tensor_ok(z, 16)) return LA_ERR_INVALID_ARG;
+    if (mode != LA_MODE_ELU1_NORM && gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
+    if (mode == LA_MODE_GATED_DELTA && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
+    DecodeArgs a;
+    a.mode = mode;
+    a.dtype = dtype;
+    a.N = N; a.H = H; a.dk = d_k; a.dv = d_v;
+    a.q = q; a.k = k; a.v = v;
+    a.gate = (mode == LA_MODE_ELU1_NORM) ? nullptr : gate;
+    a.beta = (mode == LA_MODE_GATED_DELTA) ? beta : nullptr;
+    a.state = state;
+    a.z = (mode == LA_MODE_ELU1_NORM) ? z : nullptr;
+    a.o = o;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return from_cuda(launch_decode(a));
+}
+
+extern "C" la_status_t la_check_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return LA_ERR_CUDA;
+    unsigned *word = device_error_word();
+    if (!word) return LA_ERR_CUDA;
+    unsigned host = 0;
+    if (cudaMemcpy(&host, word, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return LA_ERR_CUDA;
+    if (host == 0) return LA_OK;
+    const unsigned zero = 0;
+    if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+        return LA_ERR_CUDA;
+    return (host & kErrTimeout) ? LA_ERR_TIMEOUT : LA_ERR_CUDA;
+}
+
+extern "C" const char *la_status_string(la_status_t s) {
+    switch (s) {
+        case LA_OK: return "LA_OK: success";
+        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument (pointer, size, mode or dtype)";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: no kernel for this combination";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA runtime error";
+        case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT: a kernel's bounded wait ran out";
+    }
+    return "unknown la_status_t";
+}
+
+extern "C" int la_version(void) { return 100; }
+
+extern "C" unsigned long long la_kernel_launches(void) {
+    return g_launches.load(std::memory_order_relaxed);
+}

@@ -1,0 +1,65 @@
+// la_internal.cuh -- declarations shared by the translation units of liblinattn.
+// Nothing here is part of the public ABI (include/la.h).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/la.h"
+
+namespace la {
+
+// Device-side failure word.  A kernel whose bounded wait runs out ORs a code into it
+// and returns early; la_check_status() reads and clears it.  Kernels receive its
+// address as an argument (device_error_word()), so no relocatable device code is needed.
+enum : unsigned { kErrTimeout = 1u, kErrBadLaunch = 2u };
+unsigned *device_error_word();   // address on the current device, or nullptr on error
+
+// Counts kernels enqueued by the library (la_kernel_launches()).
+void note_launches(unsigned n);
+
+struct PrefillArgs {
+    int mode;           // la_mode_t
+    int dtype;          // la_dtype_t
+    int B, H, T, dk, dv;
+    const void *q, *k, *v;
+    const float *gate, *beta;
+    float *state, *z;
+    void *o;
+    int chunk;          // resolved (non-zero) chunk size
+    bool init_state;
+    cudaStream_t stream;
+};
+
+struct DecodeArgs {
+    int mode, dtype;
+    int N, H, dk, dv;
+    const void *q, *k, *v;
+    const float *gate, *beta;
+    float *state, *z;
+    void *o;
+    cudaStream_t stream;
+};
+
+// Launchers return cudaSuccess or the launch error.  They assume validated arguments.
+cudaError_t launch_decode(const DecodeArgs &a);
+cudaError_t launch_prefill_simt(const PrefillArgs &a);
+bool prefill_simt_supports(int dtype, int dk, int dv, int chunk, int *resolved_chunk);
+bool prefill_tc_supports(int dtype, int dk, int dv, int chunk);
+size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T);
+cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes);
+
+// fp32 <-> I/O element helpers used by the CUDA-core kernels.
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// phi(x) = elu(x) + 1 (the lesson's feature map), in fp32.
+__device__ __forceinline__ float feature_phi(float x) { return x > 0.f ? x + 1.f : expf(x); }
+
+}  // namespace la

@@ -1,0 +1,262 @@
+// prefill_simt.cu -- chunked prefill on CUDA cores, fp32 arithmetic throughout.
+//
+// This is the kernel for fp32 I/O (where a bf16 tensor-core product could not hold the
+// fp32 tolerance) and for the d = 64 shapes.  It evaluates the chunked form of "Linear
+// attention and hybrids", section "Three forms of one computation": inside a chunk of C
+// tokens the causally masked C x C matrix, across chunks the state carried in shared
+// memory.  With L tokens in the chunk, in-chunk log-gate prefix lam_i = sum_{m<=i} log a_m
+// (so the page's decay-mask entry D_ij = a_{j+1}...a_i is exp(lam_i - lam_j), section
+// "Memory must forget"), g_i = exp(lam_i), and X the chunk's value rows:
+//
+//   A_ij = (q_i . k_j) exp(lam_i - lam_j)  for j <= i   (phi(q), phi(k) in mode 0)
+//   O    = diag(g) Q S^T + A X              (mode 0: divided by den_i = sum_j A_ij + q_i.z)
+//   S   <- g_L S + sum_j exp(lam_L - lam_j) x_j k_j^T,   z <- z + sum_j phi(k_j)
+//
+// Modes 0/1 use X = V.  Mode 2 (the Gated DeltaNet update of section "The delta rule and
+// Gated DeltaNet") replaces V by the write vectors e_t = b_t (v_t - a_t S_{t-1} k_t),
+// which solve a unit lower-triangular system inside the chunk:
+//
+//   (I + Lm) E = diag(b) V - diag(b g) K S^T,   Lm_ij = b_i exp(lam_i - lam_j) (k_i . k_j), j < i
+//
+// solved here by forward substitution as U = (I+Lm)^-1 diag(b) V, W = (I+Lm)^-1 diag(b g) K,
+// E = U - W S^T.  Every exponent is <= 0, so no factor exceeds 1.
+//
+// One CTA (256 threads) per (batch, head) walks the chunks in order; all tiles are fp32
+// in shared memory with one float of row padding so that row-strided reads are
+// bank-conflict free.
+#include "la_internal.cuh"
+
+#include <cfloat>
+
+namespace la {
+namespace {
+
+constexpr int kSimtThreads = 256;
+
+template <int DK, int DV, int C>
+struct SimtSmem {
+    static constexpr int kS = DV * (DK + 1);
+    static constexpr int kQ = C * (DK + 1);
+    static constexpr int kV = C * (DV + 1);
+    static constexpr int kA = C * (C + 1);
+    static constexpr int kFloats = kS + 3 * kQ + kV + 2 * kA + 4 * C + DK;
+    static constexpr size_t kBytes = sizeof(float) * kFloats;
+};
+
+template <int MODE, int DK, int DV, int C, typename IO>
+__global__ void __launch_bounds__(kSimtThreads)
+prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
+                    const IO *__restrict__ v, const float *__restrict__ gate,
+                    const float *__restrict__ beta, float *__restrict__ state,
+                    float *__restrict__ zg, IO *__restrict__ o, int init_state) {
+    using L = SimtSmem<DK, DV, C>;
+    extern __shared__ float smem[];
+    float *S = smem;                 // [DV][DK+1]
+    float *Qs = S + L::kS;           // [C][DK+1]
+    float *Ks = Qs + L::kQ;          // [C][DK+1]
+    float *Ws = Ks + L::kQ;          // [C][DK+1]  mode 2
+    float *Vs = Ws + L::kQ;          // [C][DV+1]  V, then U, then E in mode 2
+    float *A = Vs + L::kV;           // [C][C+1]
+    float *Lm = A + L::kA;           // [C][C+1]   mode 2
+    float *lam = Lm + L::kA;         // [C]
+    float *bet = lam + C;            // [C]
+    float *den = bet + C;            // [C]
+    float *dec = den + C;            // [C]
+    float *zs = dec + C;             // [DK]
+
+    constexpr int SK = DK + 1, SV = DV + 1, SA = C + 1;
+    const int tid = threadIdx.x;
+    const size_t bh = blockIdx.x;
+    const IO *qh = q + bh * (size_t)T * DK;
+    const IO *kh = k + bh * (size_t)T * DK;
+    const IO *vh = v + bh * (size_t)T * DV;
+    IO *oh = o + bh * (size_t)T * DV;
+    const float *gh = gate ? gate + bh * (size_t)T : nullptr;
+    const float *bh_beta = beta ? beta + bh * (size_t)T : nullptr;
+    float *Sg = state + bh * (size_t)DV * DK;
+
+    for (int p = tid; p < DV * DK; p += kSimtThreads)
+        S[(p / DK) * SK + p % DK] = init_state ? Sg[p] : 0.f;
+    if (MODE == 0)
+        for (int p = tid; p < DK; p += kSimtThreads) zs[p] = init_state ? zg[bh * DK + p] : 0.f;
+    __syncthreads();
+
+    for (int t0 = 0; t0 < T; t0 += C) {
+        const int Lc = min(C, T - t0);
+        // ---- load the chunk (phi applied in mode 0) and the gates
+        for (int p = tid; p < Lc * DK; p += kSimtThreads) {
+            const int i = p / DK, j = p % DK;
+            float qv = to_f32(qh[(size_t)(t0 + i) * DK + j]);
+            float kv = to_f32(kh[(size_t)(t0 + i) * DK + j]);
+            if (MODE == 0) { qv = feature_phi(qv); kv = feature_phi(kv); }
+            Qs[i * SK + j] = qv;
+            Ks[i * SK + j] = kv;
+        }
+        for (int p = tid; p < Lc * DV; p += kSimtThreads)
+            Vs[(p / DV) * SV + p % DV] = to_f32(vh[(size_t)(t0 + p / DV) * DV + p % DV]);
+        if (tid < Lc) {
+            lam[tid] = (MODE != 0 && gh) ? logf(fmaxf(gh[t0 + tid], FLT_MIN)) : 0.f;
+            bet[tid] = (MODE == 2) ? bh_beta[t0 + tid] : 0.f;
+        }
+        __syncthreads();
+        if (tid == 0)
+            for (int i = 1; i < Lc; ++i) lam[i] += lam[i - 1];
+        __syncthreads();
+        if (tid < Lc) dec[tid] = expf(lam[Lc - 1] - lam[tid]);
+
+        // ---- intra-chunk scores A (and the delta-rule matrix Lm)
+        for (int p = tid; p < C * C; p += kSimtThreads) {
+            const int i = p / C, j = p % C;
+            float aij = 0.f, lij = 0.f;
+            if (i < Lc && j <= i) {
+                float qk = 0.f, kk = 0.f;
+#pragma unroll 8
+                for (int c = 0; c < DK; ++c) {
+                    qk = fmaf(Qs[i * SK + c], Ks[j * SK + c], qk);
+                    if (MODE == 2) kk = fmaf(Ks[i * SK + c], Ks[j * SK + c], kk);
+                }
+                const float d = (MODE == 0) ? 1.f : expf(lam[i] - lam[j]);
+                aij = qk * d;
+                if (MODE == 2 && j < i) lij = bet[i] * d * kk;
+            }
+            A[i * SA + j] = aij;
+            if (MODE == 2) Lm[i * SA + j] = lij;
+        }
+        __syncthreads();
+
+        if (MODE == 0 && tid < Lc) {
+            float s = 0.f;
+            for (int j = 0; j <= tid; ++j) s += A[tid * SA + j];
+            for (int c = 0; c < DK; ++c) s = fmaf(Qs[tid * SK + c], zs[c], s);
+            den[tid] = s;
+        }
+
+        if (MODE == 2) {
+            // right-hand sides: diag(b) V in Vs, diag(b g) K in Ws
+            for (int p = tid; p < Lc * DV; p += kSimtThreads) Vs[(p / DV) * SV + p % DV] *= bet[p / DV];
+            for (int p = tid; p < Lc * DK; p += kSimtThreads) {
+                const int i = p / DK, c = p % DK;
+                Ws[i * SK + c] = bet[i] * expf(lam[i]) * Ks[i * SK + c];
+            }
+            __syncthreads();
+            // forward substitution, one column of [U | W] per thread
+            for (int r = 1; r < Lc; ++r) {
+                for (int col = tid; col < DV + DK; col += kSimtThreads) {
+                    float *X = col < DV ? Vs + col : Ws + (col - DV);
+                    const int stride = col < DV ? SV : SK;
+                    float acc = X[r * stride];
+                    for (int j = 0; j < r; ++j) acc = fmaf(-Lm[r * SA + j], X[j * stride], acc);
+                    X[r * stride] = acc;
+                }
+                __syncthreads();
+            }
+            // E = U - W S^T, in place over U
+            for (int p = tid; p < Lc * DV; p += kSimtThreads) {
+                const int t = p / DV, i = p % DV;
+                float acc = Vs[t * SV + i];
+#pragma unroll 8
+                for (int c = 0; c < DK; ++c) acc = fmaf(-Ws[t * SK + c], S[i * SK + c], acc);
+                Vs[t * SV + i] = acc;
+            }
+        }
+        __syncthreads();
+
+        // ---- output: O = diag(g) Q S^T + A X   (mode 0: / den)
+        for (int p = tid; p < Lc * DV; p += kSimtThreads) {
+            const int t = p / DV, i = p % DV;
+            float inter = 0.f;
+#pragma unroll 8
+            for (int c = 0; c < DK; ++c) inter = fmaf(Qs[t * SK + c], S[i * SK + c], inter);
+            float intra = 0.f;
+            for (int j = 0; j <= t; ++j) intra = fmaf(A[t * SA + j], Vs[j * SV + i], intra);
+            float out;
+            if (MODE == 0) out = (inter + intra) / den[t];
+            else out = fmaf(expf(lam[t]), inter, intra);
+            oh[(size_t)(t0 + t) * DV + i] = from_f32<IO>(out);
+        }
+        __syncthreads();
+
+        // ---- state update: S <- g_L S + sum_j exp(lam_L - lam_j) x_j k_j^T
+        const float gL = (MODE == 0) ? 1.f : expf(lam[Lc - 1]);
+        for (int p = tid; p < DV * DK; p += kSimtThreads) {
+            const int i = p / DK, c = p % DK;
+            float acc = 0.f;
+            for (int j = 0; j < Lc; ++j) acc = fmaf(dec[j] * Vs[j * SV + i], Ks[j * SK + c], acc);
+            S[i * SK + c] = fmaf(gL, S[i * SK + c], acc);
+        }
+        if (MODE == 0) {
+            for (int c = tid; c < DK; c += kSimtThreads) {
+                float acc = 0.f;
+                for (int j = 0; j < Lc; ++j) acc += Ks[j * SK + c];
+                zs[c] += acc;
+            }
+        }
+        __syncthreads();
+    }
+
+    for (int p = tid; p < DV * DK; p += kSimtThreads) Sg[p] = S[(p / DK) * SK + p % DK];
+    if (MODE == 0)
+        for (int p = tid; p < DK; p += kSimtThreads) zg[bh * DK + p] = zs[p];
+}
+
+template <int MODE, int DK, int DV, int C, typename IO>
+cudaError_t launch_one(const PrefillArgs &a) {
+    using L = SimtSmem<DK, DV, C>;
+    auto kern = prefill_simt_kernel<MODE, DK, DV, C, IO>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)L::kBytes);
+    if (err != cudaSuccess) return err;
+    kern<<<(unsigned)((size_t)a.B * a.H), kSimtThreads, L::kBytes, a.stream>>>(
+        a.T, static_cast<const IO *>(a.q), static_cast<const IO *>(a.k),
+        static_cast<const IO *>(a.v), a.gate, a.beta, a.state, a.z, static_cast<IO *>(a.o),
+        a.init_state ? 1 : 0);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+template <int MODE, int DK, int DV, typename IO>
+cudaError_t launch_chunk(const PrefillArgs &a) {
+    if (a.chunk == 32) return launch_one<MODE, DK, DV, 32, IO>(a);
+    if constexpr (DK == 64 && DV == 64) {
+        if (a.chunk == 64) return launch_one<MODE, DK, DV, 64, IO>(a);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <int MODE, typename IO>
+cudaError_t launch_dims(const PrefillArgs &a) {
+    if (a.dk == 64 && a.dv == 64) return launch_chunk<MODE, 64, 64, IO>(a);
+    if (a.dk == 128 && a.dv == 128) return launch_chunk<MODE, 128, 128, IO>(a);
+    if (a.dk == 64 && a.dv == 128) return launch_chunk<MODE, 64, 128, IO>(a);
+    if (a.dk == 128 && a.dv == 64) return launch_chunk<MODE, 128, 64, IO>(a);
+    return cudaErrorInvalidValue;
+}
+
+template <typename IO>
+cudaError_t launch_io(const PrefillArgs &a) {
+    switch (a.mode) {
+        case LA_MODE_ELU1_NORM: return launch_dims<0, IO>(a);
+        case LA_MODE_GATED: return launch_dims<1, IO>(a);
+        case LA_MODE_GATED_DELTA: return launch_dims<2, IO>(a);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool prefill_simt_supports(int dtype, int dk, int dv, int chunk, int *resolved) {
+    (void)dtype;
+    const bool small = (dk == 64 && dv == 64);
+    const int c = chunk == 0 ? (small ? 64 : 32) : chunk;
+    if (c == 32 || (c == 64 && small)) {
+        *resolved = c;
+        return true;
+    }
+    return false;
+}
+
+cudaError_t launch_prefill_simt(const PrefillArgs &a) {
+    return a.dtype == LA_BF16 ? launch_io<__nv_bfloat16>(a) : launch_io<float>(a);
+}
+
+}  // namespace la

@@ -1,0 +1,946 @@
+// prefill_tc.cu -- chunked prefill on the 5th-generation tensor cores (tcgen05 + TMEM,
+// operands staged by TMA), bf16 I/O, d_k = d_v = 128, chunk C = 64, fp32 state.
+//
+// The method is the chunked form of the lesson page "Linear attention and hybrids",
+// section "Three forms of one computation" (inside a chunk the masked C x C matrix,
+// across chunks the carried state), with the decay mask of section "Memory must forget:
+// decay and gates" and, in mode 2, the Gated DeltaNet update of section "The delta rule
+// and Gated DeltaNet".  Per chunk of L <= 64 tokens, with the in-chunk log-gate prefix
+// lam_t = sum_{m<=t} log a_m, g_t = exp(lam_t), dec_t = exp(lam_{L-1} - lam_t) (all <= 1):
+//
+//   G   = [K; Q] K^T                            (rows 0-63: K K^T, rows 64-127: Q K^T)
+//   A   = (Q K^T) * exp(lam_t - lam_j), j <= t  (mode 0: phi(Q) phi(K)^T, no decay)
+//   modes 0/1:  O^T = diag-scaled  S Q^T  +  V^T A^T          (mode 0: / den_t)
+//               S  <- g_{L-1} S + V^T diag(dec) K
+//   mode 2:     Lm = strictly-lower(diag(b) exp(lam_t - lam_j) K K^T),  T = (I + Lm)^-1
+//               U^T = V^T (T diag(b))^T,  W^T = K^T (T diag(b g))^T
+//               E^T = U^T - S W^T            (the write vectors e_t = b_t(v_t - a_t S_{t-1} k_t))
+//               O^T = diag-scaled S Q^T + E^T A^T,   S <- g_{L-1} S + (E^T diag(dec)) K
+//
+// Every product has M = 128 (a d_v or d_k dimension) so each is one tcgen05.mma
+// shape (M=128, N=64 or 128, K=16 steps).  Tensor memory holds the fp32 state S (128
+// columns) and the products G, P = S Q^T, R, U^T, W^T, Y = S W^T (64 columns each):
+// exactly the 512 columns of one SM.  The state never leaves the chip between chunks;
+// each chunk the epilogue reads it once to write a bf16 copy (the MMA operand for
+// the next chunk) and to apply the next chunk's decay in place.
+//
+// Warp roles (256 threads): warp 0 lane 0 issues TMA loads into a 2-stage ring;
+// warp 1 owns TMEM and lane 0 issues every MMA; warps 4-7 (thread e <-> TMEM lane e)
+// do all CUDA-core work: gates, phi, masks, the 64x64 triangular inverse, epilogues.
+// Roles hand off through mbarriers; every wait is bounded (a timeout records an error
+// and the CTA winds down: in-flight copies and MMAs are drained before TMEM is freed).
+//
+// A CTA processes one (batch*head, segment) pair: a contiguous token range of the
+// sequence.  With several segments per sequence, three kinds of CTA run:
+//   LOCAL       the segment's own state contribution from a zero state (no output),
+//   TRANSITION  (mode 2) the segment's state transition matrix, i.e. the same
+//               recurrence started from the identity with v = 0 (no output),
+//   OUTPUT      the outputs, started from the exact state at the segment start.
+// A small combine kernel chains segment starts between the two passes.
+#include "la_internal.cuh"
+#include "ptx.cuh"
+#include "tmap.cuh"
+
+#include <cfloat>
+
+namespace la {
+namespace {
+
+using namespace ptx;
+
+constexpr int kC = 64;         // chunk
+constexpr int kD = 128;        // d_k = d_v
+constexpr int kThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+// TMEM column map
+constexpr uint32_t kColS = 0, kColG = 128, kColP = 192, kColR = 256, kColU = 320, kColW = 384,
+                   kColY = 448;
+
+enum Kind { kOutput = 0, kLocal = 1, kTransition = 2 };
+
+struct TcParams {
+    CUtensorMap tq, tk, tv;      // [BH][T][128] bf16, box 64 x 64
+    const float *gate;           // [BH][T] or nullptr
+    const float *beta;           // [BH][T] (mode 2)
+    __nv_bfloat16 *o;            // [BH][T][128]
+    // initial state: mode 0 zero, 1 from s_in (+ seg * s_in_seg), 2 identity
+    const float *s_in;
+    long long s_in_seg;
+    int s_in_mode;
+    const float *z_in;           // mode 0
+    long long z_in_seg;
+    // where the final state goes (nullptr: not written); out_last_only: only the last
+    // segment writes (OUTPUT kind)
+    float *s_out;
+    long long s_out_seg;
+    float *z_out;
+    long long z_out_seg;
+    float *gam_out;              // LOCAL, modes 0/1: product of the segment's gates
+    int out_last_only;
+    int T, BH, seg_len, nseg;
+    unsigned *err;
+};
+
+// ------------------------------------------------------------------ shared layout
+struct Small {
+    uint64_t full[2], empty[2];
+    uint64_t prep_done, g_done, a_ready, tt_ready, ut_done, w_ready, py_done, e_ready,
+        mma2_done, s_ready, fin;
+    uint32_t tmem_base;
+    int abort;
+    int len[2];
+    float lam[2][kC];
+    float bet[2][kC];
+    float den[kC];
+    float z[kD];
+    float scan_tmp[2];
+    float gsum;
+};
+
+constexpr uint32_t kStageBytes = 49152;           // [K0][Q0][K1][Q1][V0][V1], 8 KB each
+constexpr uint32_t kOffStage0 = 0, kOffStage1 = kStageBytes;
+constexpr uint32_t kOffSbf = 2 * kStageBytes;     // 32 KB bf16 state, K-major [d_v][d_k]
+constexpr uint32_t kOffA = kOffSbf + 32768;       // 8 KB  A [t][j]
+constexpr uint32_t kOffTp = kOffA + 8192;         // 8 KB  T'  | K~ cb0 (mode 1)
+constexpr uint32_t kOffTpp = kOffTp + 8192;       // 8 KB  T'' | K~ cb1 (mode 1)
+constexpr uint32_t kOffX = kOffTpp + 8192;        // 48 KB (mode 2): E | E' | W  or  Lm | Tm | Z
+constexpr uint32_t kOffE = kOffX, kOffEp = kOffX + 16384, kOffW = kOffX + 32768;
+constexpr uint32_t kLmStride = 65;
+
+template <int MODE>
+constexpr uint32_t smem_bytes() {
+    return (MODE == 2 ? kOffX + 49152 : kOffX) + sizeof(Small);
+}
+
+__device__ __forceinline__ void epi_sync() { named_sync(1, 128); }
+
+__device__ __forceinline__ uint64_t dk(uint32_t addr) { return sdesc_sw128(addr, 16, 1024); }
+__device__ __forceinline__ uint64_t dmn(uint32_t addr, uint32_t lbo) {
+    return sdesc_sw128(addr, lbo, 1024);
+}
+
+// Bounded wait that ignores the abort flag (used to drain in-flight work on exit).
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return;
+}
+
+// Load and prefix-sum the gates of chunk `c` into buffer `buf` (64 threads, e < 64).
+template <int MODE>
+__device__ __forceinline__ void load_gates(const TcParams &p, Small *sm, int bh, int tb, int te,
+                                           int c, int buf, int e) {
+    const int t0 = tb + kC * c;
+    const int L = min(kC, te - t0);
+    float g = 0.f;
+    if (MODE != 0 && p.gate && e < L) g = logf(fmaxf(p.gate[(size_t)bh * p.T + t0 + e], FLT_MIN));
+    // inclusive scan across 64 threads (two warps)
+    const int lane = e & 31;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float n = __shfl_up_sync(0xffffffffu, g, off);
+        if (lane >= off) g += n;
+    }
+    if (lane == 31) sm->scan_tmp[e >> 5] = g;
+    named_sync(2, 64);
+    if (e >= 32) g += sm->scan_tmp[0];
+    sm->lam[buf][e] = g;
+    sm->bet[buf][e] = (MODE == 2 && e < L) ? p.beta[(size_t)bh * p.T + t0 + e] : 0.f;
+    if (e == 0) sm->len[buf] = L;
+    named_sync(2, 64);
+}
+
+// 64x64 unit lower-triangular inverse, T = (I + Lm)^-1, by 16x16 blocks (128 threads).
+__device__ void invert_unit_lower(const float *Lm, float *Tm, float *Zs, int e) {
+    constexpr int S = kLmStride;
+    if (e < 64) {
+        const int b = e >> 4, c = e & 15;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int r = 1; r < 16; ++r) {
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < r; ++j) s = fmaf(Lm[(16 * b + r) * S + 16 * b + j], x[j], s);
+            if (r > c) x[r] = -s;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tm[(16 * b + r) * S + 16 * b + c] = x[r];
+    } else {
+        // zero the six blocks above the block diagonal
+        for (int idx = e - 64; idx < 6 * 256; idx += 64) {
+            const int blk = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
+            // (i, j) with j > i: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+            const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            Tm[(16 * bi + r) * S + 16 * bj + cc] = 0.f;
+        }
+    }
+    epi_sync();
+    for (int d = 1; d < 4; ++d) {
+        const int outs = (4 - d) * 256;
+        for (int idx = e; idx < outs; idx += 128) {
+            const int blk = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
+            const int bi = blk + d, bj = blk;
+            float z = 0.f;
+            for (int k = 16 * bj; k < 16 * bi; ++k)
+                z = fmaf(Lm[(16 * bi + r) * S + k], Tm[k * S + 16 * bj + cc], z);
+            Zs[blk * 272 + r * 17 + cc] = z;
+        }
+        epi_sync();
+        for (int idx = e; idx < outs; idx += 128) {
+            const int blk = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
+            const int bi = blk + d, bj = blk;
+            float t = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+                t = fmaf(Tm[(16 * bi + r) * S + 16 * bi + m], Zs[blk * 272 + m * 17 + cc], t);
+            Tm[(16 * bi + r) * S + 16 * bj + cc] = -t;
+        }
+        epi_sync();
+    }
+}
+
+// Write 16 fp32 values as 8 bf16 pairs = two 16-byte chunks (chunk index ch, ch+1) of
+// row `row` in a 128B-swizzled tile at shared address `tile`.
+__device__ __forceinline__ void st_row_bf16x16(uint32_t tile, uint32_t row, uint32_t ch,
+                                               const float *v) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+        w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+        w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+        w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+        sts128(tile + sw128_off(row, ch + q), w);
+    }
+}
+
+template <int MODE, int KIND>
+__global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
+    // 128B-swizzled operand tiles need 1024-byte aligned atoms.  The buffer is declared
+    // with that alignment and never re-aligned by integer arithmetic: pointers derived
+    // from it keep the shared address space.
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *sm8 = smem_raw;
+    const uint32_t sm_base = smem_u32(smem_raw);
+    if (sm_base & 1023u) {
+        if (threadIdx.x == 0 && p.err) atomicOr(p.err, (unsigned)kErrBadLaunch);
+        return;
+    }
+    Small *sm = reinterpret_cast<Small *>(sm8 + (MODE == 2 ? kOffX + 49152 : kOffX));
+    const uint32_t stage_addr[2] = {sm_base + kOffStage0, sm_base + kOffStage1};
+
+    constexpr bool kOut = (KIND == kOutput);
+    constexpr bool kNeedG = (MODE == 2) || kOut;
+    constexpr bool kNeedV = (KIND != kTransition);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bh = blockIdx.x % p.BH;
+    const int seg = blockIdx.x / p.BH;
+    const int tb = seg * p.seg_len;
+    const int te = min(p.T, tb + p.seg_len);
+    const int nch = (te - tb + kC - 1) / kC;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm->full[0], 1);
+        mbar_init(&sm->full[1], 1);
+        mbar_init(&sm->empty[0], 1);
+        mbar_init(&sm->empty[1], 1);
+        mbar_init(&sm->prep_done, 1);
+        mbar_init(&sm->g_done, 1);
+        mbar_init(&sm->a_ready, 1);
+        mbar_init(&sm->tt_ready, 1);
+        mbar_init(&sm->ut_done, 1);
+        mbar_init(&sm->w_ready, 1);
+        mbar_init(&sm->py_done, 1);
+        mbar_init(&sm->e_ready, 1);
+        mbar_init(&sm->mma2_done, 1);
+        mbar_init(&sm->s_ready, 1);
+        mbar_init(&sm->fin, 1);
+        sm->abort = 0;
+        sm->gsum = 0.f;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = sm->tmem_base;
+    volatile int *abort = &sm->abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tk);
+            if (kOut) tma_prefetch_desc(&p.tq);
+            if (kNeedV) tma_prefetch_desc(&p.tv);
+            int issued[2] = {0, 0};
+            for (int c = 0; c < nch; ++c) {
+                const int s = c & 1, u = c >> 1;
+                if (u >= 1 && !mbar_wait(&sm->empty[s], (u - 1) & 1, abort, p.err)) break;
+                const uint32_t st = stage_addr[s];
+                const int t = tb + kC * c;
+                const uint32_t bytes = 16384u * (1u + (kOut ? 1u : 0u) + (kNeedV ? 1u : 0u));
+                mbar_arrive_expect_tx(&sm->full[s], bytes);
+                tma_load_3d(st + 0, &p.tk, 0, t, bh, &sm->full[s]);
+                tma_load_3d(st + 16384, &p.tk, 64, t, bh, &sm->full[s]);
+                if (kOut) {
+                    tma_load_3d(st + 8192, &p.tq, 0, t, bh, &sm->full[s]);
+                    tma_load_3d(st + 24576, &p.tq, 64, t, bh, &sm->full[s]);
+                }
+                if (kNeedV) {
+                    tma_load_3d(st + 32768, &p.tv, 0, t, bh, &sm->full[s]);
+                    tma_load_3d(st + 40960, &p.tv, 64, t, bh, &sm->full[s]);
+                }
+                issued[s] = u + 1;
+            }
+            // make sure no copy is still writing shared memory when the CTA exits
+            for (int s = 0; s < 2; ++s)
+                if (issued[s] > 0) drain_wait(&sm->full[s], (issued[s] - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t sbf = sm_base + kOffSbf;
+            const uint32_t at = sm_base + kOffA;
+            const uint32_t tp = sm_base + kOffTp;
+            const uint32_t tpp = sm_base + kOffTpp;
+            const uint32_t et = sm_base + kOffE;
+            const uint32_t ept = sm_base + kOffEp;
+            const uint32_t wt = sm_base + kOffW;
+            const uint32_t id_n64_kk = idesc_bf16(128, 64, false, false);
+            const uint32_t id_n64_mk = idesc_bf16(128, 64, true, false);
+            const uint32_t id_n64_km = idesc_bf16(128, 64, false, true);
+            const uint32_t id_n128_mm = idesc_bf16(128, 128, true, true);
+            const uint32_t id_n128_km = idesc_bf16(128, 128, false, true);
+            bool ok = true;
+            for (int c = 0; c < nch && ok; ++c) {
+                const int s = c & 1, u = c >> 1;
+                const uint32_t par = c & 1;
+                const uint32_t st = stage_addr[s];
+                if (!mbar_wait(&sm->full[s], u & 1, abort, p.err)) break;
+                if (!mbar_wait(&sm->prep_done, par, abort, p.err)) break;
+                tc_fence_after();
+                if (kNeedG) {
+                    // G = [K; Q] K^T   (M=128, N=64, K=128)
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16_ss(tm + kColG, dk(st + off), dk(st + off), id_n64_kk, ks > 0);
+                    }
+                    mma_commit(&sm->g_done);
+                }
+                if constexpr (MODE == 2) {
+                    if (!mbar_wait(&sm->tt_ready, par, abort, p.err)) break;
+                    tc_fence_after();
+                    if (kNeedV) {
+                        // U^T = V^T (T diag b)^T  (A: V^T MN-major; B: T' K-major)
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_bf16_ss(tm + kColU, dmn(st + 32768 + ks * 2048, 8192),
+                                        dk(tp + ks * 32), id_n64_mk, ks > 0);
+                    }
+                    // W^T = K^T (T diag(b g))^T
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ss(tm + kColW, dmn(st + ks * 2048, 16384), dk(tpp + ks * 32),
+                                    id_n64_mk, ks > 0);
+                    mma_commit(&sm->ut_done);
+                    if (!mbar_wait(&sm->w_ready, par, abort, p.err)) break;
+                    if (!mbar_wait(&sm->s_ready, par, abort, p.err)) break;
+                    tc_fence_after();
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t soff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        if (kOut)   // P = S Q^T
+                            mma_bf16_ss(tm + kColP, dk(sbf + soff), dk(st + 8192 + soff), id_n64_kk,
+                                        ks > 0);
+                        // Y = S W^T  (B: W MN-major [d_k rows][t])
+                        mma_bf16_ss(tm + kColY, dk(sbf + soff), dmn(wt + ks * 2048, 8192),
+                                    id_n64_km, ks > 0);
+                    }
+                    mma_commit(&sm->py_done);
+                    if (!mbar_wait(&sm->e_ready, par, abort, p.err)) break;
+                    tc_fence_after();
+                    for (int ks = 0; ks < 4; ++ks) {
+                        if (kOut)   // R = E^T A^T
+                            mma_bf16_ss(tm + kColR, dk(et + ks * 32), dk(at + ks * 32), id_n64_kk,
+                                        ks > 0);
+                        // S += (E^T diag dec) K   (B: K MN-major)
+                        mma_bf16_ss(tm + kColS, dk(ept + ks * 32), dmn(st + ks * 2048, 16384),
+                                    id_n128_km, true);
+                    }
+                    mma_commit(&sm->mma2_done);
+                } else {
+                    if (!mbar_wait(&sm->s_ready, par, abort, p.err)) break;
+                    tc_fence_after();
+                    if (kOut) {
+                        for (int ks = 0; ks < 8; ++ks) {
+                            const uint32_t soff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                            mma_bf16_ss(tm + kColP, dk(sbf + soff), dk(st + 8192 + soff),
+                                        id_n64_kk, ks > 0);
+                        }
+                    }
+                    if (!mbar_wait(&sm->a_ready, par, abort, p.err)) break;
+                    tc_fence_after();
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t vt = dmn(st + 32768 + ks * 2048, 8192);
+                        if (kOut)   // R = V^T A^T
+                            mma_bf16_ss(tm + kColR, vt, dk(at + ks * 32), id_n64_mk, ks > 0);
+                        // S += V^T diag(dec) K
+                        const uint64_t kb = (MODE == 1) ? dmn(tp + ks * 2048, 8192)
+                                                        : dmn(st + ks * 2048, 16384);
+                        mma_bf16_ss(tm + kColS, vt, kb, id_n128_mm, true);
+                    }
+                    mma_commit(&sm->mma2_done);
+                }
+            }
+            // drain: nothing may still write TMEM when it is freed
+            mma_commit(&sm->fin);
+            drain_wait(&sm->fin, 0);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue warps
+        const int e = threadIdx.x - 128;          // TMEM lane
+        const int wq = e >> 5;                    // lane quarter
+        const uint32_t trow = tm + ((uint32_t)(wq * 32) << 16);
+        const uint32_t sbf = sm_base + kOffSbf;
+        const uint32_t atile = sm_base + kOffA;
+        float *Lm = reinterpret_cast<float *>(sm8 + kOffX);
+        float *Tm = Lm + 64 * kLmStride;
+        float *Zs = Tm + 64 * kLmStride;
+        const size_t o_row0 = (size_t)bh * p.T;
+
+        if (e < 64) load_gates<MODE>(p, sm, bh, tb, te, 0, 0, e);
+        epi_sync();
+        // ---- initial state: row e of S
+        {
+            const float scale0 = (MODE == 0) ? 1.f : __expf(sm->lam[0][kC - 1]);
+            const float *src = nullptr;
+            if (p.s_in_mode == 1) src = p.s_in + (size_t)seg * p.s_in_seg + (size_t)bh * kD * kD;
+            for (int c0 = 0; c0 < kD; c0 += 16) {
+                float v[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int col = c0 + j;
+                    v[j] = src ? src[(size_t)e * kD + col]
+                               : ((p.s_in_mode == 2 && col == e) ? 1.f : 0.f);
+                }
+                st_row_bf16x16(sbf + (c0 >> 6) * 16384, e, (c0 & 63) >> 3, v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] *= scale0;
+                tmem_st16(trow + kColS + c0, v);
+            }
+            if (MODE == 0) {
+                const float *zs = (p.s_in_mode == 1 && p.z_in)
+                                      ? p.z_in + (size_t)seg * p.z_in_seg + (size_t)bh * kD
+                                      : nullptr;
+                sm->z[e] = zs ? zs[e] : 0.f;
+            }
+            fence_async_smem();
+            tc_fence_before();
+            epi_sync();
+            if (e == 0) mbar_arrive(&sm->s_ready);
+        }
+
+        for (int c = 0; c < nch; ++c) {
+            const int s = c & 1, u = c >> 1, buf = c & 1;
+            const uint32_t par = c & 1;
+            const uint32_t st = stage_addr[s];
+            const int t0 = tb + kC * c;
+            const int L = sm->len[buf];
+            const float *lam = sm->lam[buf];
+            mbar_wait(&sm->full[s], u & 1, abort, p.err);
+            epi_sync();
+            if (*abort) break;
+
+            // ---- prep: phi (mode 0) or K~ = diag(dec) K (mode 1)
+            if (MODE == 0) {
+                const int nreg = kOut ? 4 : 2;
+                for (int n = e; n < nreg * 512; n += 128) {
+                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);   // 0,2 = K; 1,3 = Q
+                    const int row = (n & 511) >> 3;
+                    const uint32_t ptr = st + region * 8192 + (n & 511) * 16;
+                    uint4 w = lds128(ptr);
+                    const bool is_k = (region & 1) == 0;
+                    if (is_k && row >= L) {
+                        w = make_uint4(0, 0, 0, 0);
+                    } else {
+                        uint32_t *wd = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            float2 f = unpack_bf16x2(wd[q]);
+                            wd[q] = pack_bf16x2(feature_phi(f.x), feature_phi(f.y));
+                        }
+                    }
+                    sts128(ptr, w);
+                }
+            } else if (MODE == 1) {
+                const float lamL = lam[kC - 1];
+                for (int n = e; n < 1024; n += 128) {
+                    const int cb = n >> 9;
+                    const int row = (n & 511) >> 3;
+                    const float d = row < L ? __expf(lamL - lam[row]) : 0.f;
+                    uint4 w = lds128(st + cb * 16384 + (n & 511) * 16);
+                    uint32_t *wd = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float2 f = unpack_bf16x2(wd[q]);
+                        wd[q] = pack_bf16x2(f.x * d, f.y * d);
+                    }
+                    sts128(sm_base + kOffTp + cb * 8192 + (n & 511) * 16, w);
+                }
+            }
+            fence_async_smem();
+            epi_sync();
+            if (e == 0) mbar_arrive(&sm->prep_done);
+
+            // ---- G epilogue: A (rows of Q K^T) and, in mode 2, Lm (rows of K K^T)
+            if (kNeedG) {
+                mbar_wait(&sm->g_done, par, abort, p.err);
+                epi_sync();
+                if (*abort) break;
+                tc_fence_after();
+                if (e >= 64 && kOut) {
+                    const int i = e - 64;
+                    float rs = 0.f;
+                    for (int j0 = 0; j0 < kC; j0 += 16) {
+                        float v[16];
+                        tmem_ld16(trow + kColG + j0, v);
+    #pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int jj = j0 + j;
+                            float a = 0.f;
+                            if (jj <= i) a = (MODE == 0) ? v[j] : v[j] * __expf(lam[i] - lam[jj]);
+                            v[j] = __bfloat162float(__float2bfloat16_rn(a));
+                            rs += v[j];
+                        }
+                        st_row_bf16x16(atile, i, j0 >> 3, v);
+                    }
+                    if (MODE == 0) {
+                        // den_i = sum_j A_ij + phi(q_i) . z   (phi(Q) row i in the stage)
+                        float qz = 0.f;
+                        for (int ch = 0; ch < 16; ++ch) {
+                            const uint32_t qb = st + 8192 + (ch >> 3) * 16384;
+                            const uint4 w = lds128(qb + sw128_off(i, ch & 7));
+                            const uint32_t *wd = reinterpret_cast<const uint32_t *>(&w);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float2 f = unpack_bf16x2(wd[q]);
+                                qz = fmaf(f.x, sm->z[ch * 8 + 2 * q], qz);
+                                qz = fmaf(f.y, sm->z[ch * 8 + 2 * q + 1], qz);
+                            }
+                        }
+                        sm->den[i] = rs + qz;
+                    }
+                } else if (e < 64 && MODE == 2) {
+                    const int i = e;
+                    const float bi = sm->bet[buf][i];
+                    for (int j0 = 0; j0 < kC; j0 += 16) {
+                        float v[16];
+                        tmem_ld16(trow + kColG + j0, v);
+    #pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int jj = j0 + j;
+                            Lm[i * kLmStride + jj] =
+                                (jj < i) ? bi * __expf(lam[i] - lam[jj]) * v[j] : 0.f;
+                        }
+                    }
+                }
+                fence_async_smem();
+                tc_fence_before();
+                epi_sync();
+            }
+            if constexpr (MODE != 2) {
+                if (e == 0) mbar_arrive(&sm->a_ready);
+            } else {
+                // ---- T = (I + Lm)^-1, then T' = T diag(b), T'' = T diag(b g) in bf16
+                invert_unit_lower(Lm, Tm, Zs, e);
+                if (e < 64) {
+                    const int t = e;
+                    for (int j0 = 0; j0 < kC; j0 += 16) {
+                        float v1[16], v2[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float tv = Tm[t * kLmStride + j0 + j] * sm->bet[buf][j0 + j];
+                            v1[j] = tv;
+                            v2[j] = tv * __expf(lam[j0 + j]);
+                        }
+                        st_row_bf16x16(sm_base + kOffTp, t, j0 >> 3, v1);
+                        st_row_bf16x16(sm_base + kOffTpp, t, j0 >> 3, v2);
+                    }
+                }
+                fence_async_smem();
+                epi_sync();
+                if (e == 0) mbar_arrive(&sm->tt_ready);
+                // ---- W epilogue: W^T row (d_k index e) -> bf16 MN-major tile row e
+                mbar_wait(&sm->ut_done, par, abort, p.err);
+                epi_sync();
+                if (*abort) break;
+                tc_fence_after();
+                for (int t0c = 0; t0c < kC; t0c += 16) {
+                    float v[16];
+                    tmem_ld16(trow + kColW + t0c, v);
+                    st_row_bf16x16(sm_base + kOffW, e, t0c >> 3, v);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                epi_sync();
+                if (e == 0) mbar_arrive(&sm->w_ready);
+                // ---- E epilogue: E^T = U^T - S W^T (row d_v = e), and E^T diag(dec)
+                mbar_wait(&sm->py_done, par, abort, p.err);
+                epi_sync();
+                if (*abort) break;
+                tc_fence_after();
+                {
+                    const float lamL = lam[kC - 1];
+                    for (int t0c = 0; t0c < kC; t0c += 16) {
+                        float y[16], uu[16], ev[16];
+                        if (kNeedV) tmem_ld16x2(trow + kColY + t0c, y, trow + kColU + t0c, uu);
+                        else tmem_ld16(trow + kColY + t0c, y);
+    #pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int t = t0c + j;
+                            const float ex = (t < L) ? ((kNeedV ? uu[j] : 0.f) - y[j]) : 0.f;
+                            y[j] = ex;
+                            ev[j] = (t < L) ? ex * __expf(lamL - lam[t]) : 0.f;
+                        }
+                        st_row_bf16x16(sm_base + kOffE, e, t0c >> 3, y);
+                        st_row_bf16x16(sm_base + kOffEp, e, t0c >> 3, ev);
+                    }
+                }
+                fence_async_smem();
+                tc_fence_before();
+                epi_sync();
+                if (e == 0) mbar_arrive(&sm->e_ready);
+            }
+
+            // ---- gates of the next chunk
+            if (c + 1 < nch && e < 64) load_gates<MODE>(p, sm, bh, tb, te, c + 1, buf ^ 1, e);
+            if (KIND == kLocal && MODE == 1 && e == 0) sm->gsum += lam[kC - 1];
+
+            mbar_wait(&sm->mma2_done, par, abort, p.err);
+            epi_sync();
+            if (*abort) break;
+            tc_fence_after();
+
+            // ---- outputs: o_t[e] for t < L
+            if (kOut) {
+                __nv_bfloat16 *orow = p.o + (o_row0 + t0) * kD + e;
+                for (int j0 = 0; j0 < kC; j0 += 16) {
+                    float pv[16], rv[16];
+                    tmem_ld16x2(trow + kColP + j0, pv, trow + kColR + j0, rv);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int t = j0 + j;
+                        if (t < L) {
+                            float val;
+                            if (MODE == 0) val = (pv[j] + rv[j]) / sm->den[t];
+                            else val = fmaf(__expf(lam[t]), pv[j], rv[j]);
+                            orow[(size_t)t * kD] = __float2bfloat16_rn(val);
+                        }
+                    }
+                }
+            }
+            if (MODE == 0) {
+                // z += sum_j phi(k_j)   (rows >= L were zeroed in the prep step)
+                const uint32_t kb = st + (e >> 6) * 16384;
+                const int ch = (e & 63) >> 3, wi = e & 7;
+                float zs = 0.f;
+                for (int j = 0; j < kC; ++j) {
+                    const uint32_t bits = lds_u16(kb + j * 128 + ((ch ^ (j & 7)) << 4) + wi * 2);
+                    zs += __uint_as_float(bits << 16);
+                }
+                sm->z[e] += zs;
+            }
+
+            // ---- state: bf16 copy for the next chunk's MMAs, next decay applied in TMEM
+            {
+                const bool last = (c + 1 == nch);
+                const float gnext =
+                    (MODE == 0 || last) ? 1.f : __expf(sm->lam[buf ^ 1][kC - 1]);
+                float *dst = nullptr;
+                if (last && p.s_out && (!p.out_last_only || seg == p.nseg - 1))
+                    dst = p.s_out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
+                          (size_t)e * kD;
+                for (int c0 = 0; c0 < kD; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(trow + kColS + c0, v);
+                    if (dst) {
+#pragma unroll
+                        for (int j = 0; j < 16; j += 4)
+                            *reinterpret_cast<float4 *>(dst + c0 + j) =
+                                make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                    }
+                    if (!last) {
+                        st_row_bf16x16(sbf + (c0 >> 6) * 16384, e, (c0 & 63) >> 3, v);
+                        if (MODE != 0) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) v[j] *= gnext;
+                            tmem_st16(trow + kColS + c0, v);
+                        }
+                    }
+                }
+                if (last && MODE == 0 && p.z_out && (!p.out_last_only || seg == p.nseg - 1))
+                    p.z_out[(size_t)seg * p.z_out_seg + (size_t)bh * kD + e] = sm->z[e];
+                if (last && KIND == kLocal && MODE == 1 && e == 0 && p.gam_out)
+                    p.gam_out[(size_t)seg * p.BH + bh] = __expf(sm->gsum);
+                fence_async_smem();
+                tc_fence_before();
+                epi_sync();
+                if (e == 0) {
+                    mbar_arrive(&sm->s_ready);
+                    mbar_arrive(&sm->empty[s]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tm, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ combine kernels
+// modes 0/1: S_start[s+1] = gam_s S_start[s] + N_s;  z_start[s+1] = z_start[s] + zN_s.
+__global__ void combine_scalar_kernel(int BH, int nseg, const float *s_init, const float *z_init,
+                                      const float *nloc, const float *zloc, const float *gam,
+                                      float *sst, float *zst, int mode) {
+    const size_t per = (size_t)kD * kD;
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t total = (size_t)BH * per;
+    if (idx < total) {
+        const int bh = (int)(idx / per);
+        float sv = s_init ? s_init[idx] : 0.f;
+        sst[idx] = sv;
+        for (int s = 0; s + 1 < nseg; ++s) {
+            const float g = (mode == 1) ? gam[(size_t)s * BH + bh] : 1.f;
+            sv = fmaf(g, sv, nloc[(size_t)s * total + idx]);
+            sst[(size_t)(s + 1) * total + idx] = sv;
+        }
+    }
+    if (mode == 0 && idx < (size_t)BH * kD) {
+        float zv = z_init ? z_init[idx] : 0.f;
+        zst[idx] = zv;
+        for (int s = 0; s + 1 < nseg; ++s) {
+            zv += zloc[(size_t)s * BH * kD + idx];
+            zst[(size_t)(s + 1) * BH * kD + idx] = zv;
+        }
+    }
+}
+
+// mode 2: S_start[s+1] = S_start[s] M_s + N_s (row-parallel; 16 rows of S per CTA).
+constexpr int kCombRows = 16;
+__global__ void __launch_bounds__(256) combine_matrix_kernel(int BH, int nseg, const float *s_init,
+                                                             const float *nloc, const float *mtr,
+                                                             float *sst) {
+    extern __shared__ float csm[];
+    float *Ms = csm;                       // [128][128]
+    float *Ss = Ms + kD * kD;              // [16][128]
+    const int bh = blockIdx.x;
+    const int r0 = blockIdx.y * kCombRows;
+    const size_t per = (size_t)kD * kD;
+    const size_t total = (size_t)BH * per;
+    for (int i = threadIdx.x; i < kCombRows * kD; i += 256) {
+        const size_t g = (size_t)bh * per + (size_t)r0 * kD + i;
+        const float v = s_init ? s_init[g] : 0.f;
+        Ss[i] = v;
+        sst[g] = v;
+    }
+    for (int s = 0; s + 1 < nseg; ++s) {
+        __syncthreads();
+        const float *Mg = mtr + (size_t)s * total + (size_t)bh * per;
+        for (int i = threadIdx.x; i < kD * kD / 4; i += 256)
+            reinterpret_cast<float4 *>(Ms)[i] = reinterpret_cast<const float4 *>(Mg)[i];
+        __syncthreads();
+        float acc[8];
+        const int col = threadIdx.x & 127;
+        const int rb = (threadIdx.x >> 7) * 8;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+        for (int k = 0; k < kD; ++k) {
+            const float m = Ms[k * kD + col];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) acc[r] = fmaf(Ss[(rb + r) * kD + k], m, acc[r]);
+        }
+        __syncthreads();
+        const float *Ng = nloc + (size_t)s * total + (size_t)bh * per;
+        float *dst = sst + (size_t)(s + 1) * total + (size_t)bh * per;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const size_t g = (size_t)(r0 + rb + r) * kD + col;
+            const float v = acc[r] + Ng[g];
+            Ss[(rb + r) * kD + col] = v;
+            dst[g] = v;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ host side
+struct Plan {
+    int nseg, seg_len;
+};
+
+Plan plan_for(int mode, int BH, int T) {
+    const int nchunks = (T + kC - 1) / kC;
+    int nseg = 1;
+    const int sms = 148;
+    if (BH < sms) nseg = sms / BH;
+    nseg = std::max(1, std::min(nseg, nchunks / 4));   // keep segments >= 4 chunks
+    const int chunks_per_seg = (nchunks + nseg - 1) / nseg;
+    Plan pl;
+    pl.seg_len = chunks_per_seg * kC;
+    pl.nseg = (T + pl.seg_len - 1) / pl.seg_len;
+    return pl;
+}
+
+size_t workspace_floats(int mode, int BH, const Plan &pl) {
+    if (pl.nseg <= 1) return 0;
+    const size_t per = (size_t)BH * kD * kD;
+    size_t f = (size_t)pl.nseg * per;                 // segment start states
+    f += (size_t)(pl.nseg - 1) * per;                 // local states
+    if (mode == 2) f += (size_t)(pl.nseg - 1) * per;  // transitions
+    if (mode == 1) f += (size_t)(pl.nseg - 1) * BH;   // gate products
+    if (mode == 0) f += (size_t)(2 * pl.nseg - 1) * BH * kD;   // z starts + z locals
+    return f;
+}
+
+template <int MODE, int KIND>
+cudaError_t launch_kind(const TcParams &p, int grid, cudaStream_t stream) {
+    auto kern = prefill_tc_kernel<MODE, KIND>;
+    const uint32_t bytes = smem_bytes<MODE>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, bytes, stream>>>(p);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl, float *ws) {
+    const int BH = a.B * a.H;
+    const size_t per = (size_t)BH * kD * kD;
+    if (pl.nseg == 1) {
+        TcParams p = base;
+        p.s_in_mode = a.init_state ? 1 : 0;
+        p.s_in = a.state;
+        p.s_in_seg = 0;
+        p.z_in = a.z;
+        p.z_in_seg = 0;
+        p.s_out = a.state;
+        p.s_out_seg = 0;
+        p.z_out = a.z;
+        p.z_out_seg = 0;
+        p.out_last_only = 1;
+        return launch_kind<MODE, kOutput>(p, BH, a.stream);
+    }
+    float *sst = ws;
+    float *nloc = sst + (size_t)pl.nseg * per;
+    float *mtr = nloc + (size_t)(pl.nseg - 1) * per;            // mode 2
+    float *gam = nloc + (size_t)(pl.nseg - 1) * per;            // mode 1
+    float *zst = nloc + (size_t)(pl.nseg - 1) * per;            // mode 0
+    float *zloc = zst + (size_t)pl.nseg * BH * kD;
+    // pass A: local states (and transitions)
+    {
+        TcParams p = base;
+        p.s_in_mode = 0;
+        p.s_out = nloc;
+        p.s_out_seg = (long long)per;
+        p.z_out = (MODE == 0) ? zloc : nullptr;
+        p.z_out_seg = (long long)BH * kD;
+        p.gam_out = (MODE == 1) ? gam : nullptr;
+        p.out_last_only = 0;
+        cudaError_t e = launch_kind<MODE, kLocal>(p, BH * (pl.nseg - 1), a.stream);
+        if (e != cudaSuccess) return e;
+        if constexpr (MODE == 2) {
+            TcParams q = base;
+            q.s_in_mode = 2;
+            q.s_out = mtr;
+            q.s_out_seg = (long long)per;
+            q.out_last_only = 0;
+            e = launch_kind<MODE, kTransition>(q, BH * (pl.nseg - 1), a.stream);
+            if (e != cudaSuccess) return e;
+        }
+    }
+    // combine: segment start states
+    const float *s_init = a.init_state ? a.state : nullptr;
+    if constexpr (MODE == 2) {
+        const size_t bytes = sizeof(float) * (kD * kD + kCombRows * kD);
+        cudaError_t e = cudaFuncSetAttribute(combine_matrix_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (e != cudaSuccess) return e;
+        combine_matrix_kernel<<<dim3(BH, kD / kCombRows), 256, bytes, a.stream>>>(
+            BH, pl.nseg, s_init, nloc, mtr, sst);
+    } else {
+        const size_t total = per;
+        combine_scalar_kernel<<<(unsigned)((total + 255) / 256), 256, 0, a.stream>>>(
+            BH, pl.nseg, s_init, (MODE == 0 && a.init_state) ? a.z : nullptr, nloc, zloc, gam, sst,
+            zst, MODE);
+    }
+    note_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // pass C: outputs from the exact segment starts
+    TcParams p = base;
+    p.s_in_mode = 1;
+    p.s_in = sst;
+    p.s_in_seg = (long long)per;
+    p.z_in = (MODE == 0) ? zst : nullptr;
+    p.z_in_seg = (long long)BH * kD;
+    p.s_out = a.state;
+    p.s_out_seg = 0;
+    p.z_out = a.z;
+    p.z_out_seg = 0;
+    p.out_last_only = 1;
+    return launch_kind<MODE, kOutput>(p, BH * pl.nseg, a.stream);
+}
+
+}  // namespace
+
+bool prefill_tc_supports(int dtype, int dk, int dv, int chunk) {
+    return dtype == LA_BF16 && dk == kD && dv == kD && (chunk == 0 || chunk == kC);
+}
+
+size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T) {
+    const int BH = B * H;
+    return sizeof(float) * workspace_floats(mode, BH, plan_for(mode, BH, T));
+}
+
+cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes) {
+    const int BH = a.B * a.H;
+    Plan pl = plan_for(a.mode, BH, a.T);
+    if (sizeof(float) * workspace_floats(a.mode, BH, pl) > workspace_bytes || !workspace) {
+        pl.nseg = 1;
+        pl.seg_len = ((a.T + kC - 1) / kC) * kC;
+    }
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    const uint64_t row_pitch = kD * 2, head_pitch = (uint64_t)a.T * kD * 2;
+    if (!make_tmap_3d(&p.tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, a.T, BH, row_pitch,
+                      head_pitch, 64, kC, true) ||
+        !make_tmap_3d(&p.tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, a.T, BH, row_pitch,
+                      head_pitch, 64, kC, true) ||
+        !make_tmap_3d(&p.tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, a.T, BH, row_pitch,
+                      head_pitch, 64, kC, true))
+        return cudaErrorInvalidValue;
+    p.gate = a.gate;
+    p.beta = a.beta;
+    p.o = static_cast<__nv_bfloat16 *>(a.o);
+    p.T = a.T;
+    p.BH = BH;
+    p.seg_len = pl.seg_len;
+    p.nseg = pl.nseg;
+    p.err = device_error_word();
+    float *ws = static_cast<float *>(workspace);
+    switch (a.mode) {
+        case LA_MODE_ELU1_NORM: return run_mode<0>(a, p, pl, ws);
+        case LA_MODE_GATED: return run_mode<1>(a, p, pl, ws);
+        case LA_MODE_GATED_DELTA: return run_mode<2>(a, p, pl, ws);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace la

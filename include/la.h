@@ -1,0 +1,158 @@
+/*
+ * la.h -- C ABI of liblinattn: causal linear attention on NVIDIA B200 (sm_100a).
+ *
+ * The operations are those of the lesson page "Линейное внимание и гибриды"
+ * ("Linear attention and hybrids", ai.flicky.cc, stage 5.5), cited by section:
+ *   [kernel trick]  "Ядерный трюк: убираем softmax"  -- phi(x) = elu(x) + 1, S_i, z_i
+ *   [three forms]   "Три формы одного вычисления"    -- recurrent and chunked forms
+ *   [decay/gates]   "Память должна забывать: затухание и гейты" -- gamma, alpha_t gates
+ *   [delta rule]    "Дельта-правило и Gated DeltaNet" -- delta rule, Gated DeltaNet
+ *
+ * Three variants ("modes"), each with a chunked prefill and a one-token decode step.
+ * Per (batch, head), for t = 1..T, the state is updated first and then read:
+ *
+ *   LA_MODE_ELU1_NORM ([kernel trick], [three forms]):
+ *       S_t = S_{t-1} + v_t phi(k_t)^T,  z_t = z_{t-1} + phi(k_t),
+ *       o_t = S_t phi(q_t) / (z_t . phi(q_t)).
+ *   LA_MODE_GATED ([decay/gates]; no feature map, no denominator):
+ *       S_t = a_t S_{t-1} + v_t k_t^T,   o_t = S_t q_t.
+ *   LA_MODE_GATED_DELTA ([delta rule], the Gated DeltaNet equation):
+ *       S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S_t q_t.
+ *
+ * No 1/sqrt(d) scale is applied inside the attention; callers scale q and k.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers: every tensor argument is a DEVICE pointer (memory the current CUDA device
+ *   can address: cudaMalloc, torch CUDA tensors, managed memory).  Host pointers are
+ *   rejected with LA_ERR_INVALID_ARG before anything is launched.  The caller owns all
+ *   buffers; the library allocates no device memory and keeps no pointer after the call
+ *   returns.  Tensors are dense, row-major, and 16-byte aligned (gate and beta: 4-byte).
+ * Dtypes: q, k, v, o have the I/O dtype (LA_F32 or LA_BF16).  state, z, gate and beta
+ *   are always fp32; all accumulation is fp32.
+ * Sizes: d_k and d_v are each 64 or 128.  B, H, N >= 1.  T >= 0.
+ * Gates: gate holds the decay values a_t in [0, 1] (not their logarithms); NULL means
+ *   a_t = 1.  beta holds b_t in [0, 1].  Mode 0 ignores gate and beta; mode 1 ignores
+ *   beta; mode 2 requires beta.
+ * State layout: S is d_v x d_k per head, exactly the page's S ([three forms]), stored
+ *   [.., d_v, d_k] row-major; z is [.., d_k].  A state written by la_prefill is the
+ *   input of la_decode_step, and vice versa.
+ * Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).  Argument
+ *   checks run on the host and finish before anything is enqueued; the work itself
+ *   runs asynchronously on `stream`.  LA_OK means "enqueued"; device-side failures are
+ *   reported by la_check_status().
+ * Thread safety: the entry points keep no per-call state and may be called from
+ *   several host threads.
+ */
+#ifndef LINATTN_LA_H
+#define LINATTN_LA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LA_MODE_ELU1_NORM = 0,   /* phi = elu+1, z-normalised                 */
+    LA_MODE_GATED = 1,       /* scalar gate a_t, identity feature map     */
+    LA_MODE_GATED_DELTA = 2  /* Gated DeltaNet: gate a_t and delta rate b_t */
+} la_mode_t;
+
+typedef enum {
+    LA_F32 = 0,              /* q, k, v, o in fp32 */
+    LA_BF16 = 1              /* q, k, v, o in bf16 (round-to-nearest-even on output) */
+} la_dtype_t;
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = 1,  /* a NULL / host / misaligned pointer, a bad size, mode or dtype */
+    LA_ERR_UNSUPPORTED = 2,  /* a valid request this build has no kernel for */
+    LA_ERR_CUDA = 3,         /* a CUDA runtime error at launch or while checking status */
+    LA_ERR_TIMEOUT = 4       /* a kernel's bounded wait ran out; its outputs are invalid */
+} la_status_t;
+
+/* la_prefill flag: read `state` (and `z`) as the initial state S_0 (z_0).  Without it
+ * S_0 = 0 and z_0 = 0, and `state` / `z` are only written. */
+#define LA_FLAG_INIT_STATE 1u
+
+/*
+ * la_prefill -- the chunkwise-parallel ("chunked") form of [three forms] over a whole
+ * sequence per (batch, head): inside a chunk of C tokens the masked C x C matrix, across
+ * chunks the carried state; with the decay mask of [decay/gates] in mode 1 and the
+ * delta-rule correction of [delta rule] in mode 2.  The result equals the recurrent
+ * form above up to rounding.
+ *
+ *   q, k   [B, H, T, d_k]  I/O dtype
+ *   v      [B, H, T, d_v]  I/O dtype
+ *   gate   [B, H, T] fp32 or NULL      beta [B, H, T] fp32 (mode 2) or NULL
+ *   state  [B, H, d_v, d_k] fp32       in (if LA_FLAG_INIT_STATE) and out: S_T
+ *   z      [B, H, d_k] fp32            mode 0 only (else ignored, may be NULL): in/out z_T
+ *   o      [B, H, T, d_v]  I/O dtype   out: o_1..o_T
+ *   chunk  tokens per chunk; 0 picks the kernel's default.  bf16 with d_k = d_v = 128
+ *          accepts 0 and 64; every other case accepts 0, 32 and 64 (64 only when
+ *          d_k = d_v = 64).  Other values return LA_ERR_UNSUPPORTED.
+ *   flags  0 or LA_FLAG_INIT_STATE.
+ *   workspace, workspace_bytes
+ *          optional device scratch owned by the caller (NULL / 0 allowed).  With at least
+ *          la_prefill_workspace_size() bytes the tensor-core kernel splits each sequence
+ *          into segments processed in parallel and chains their states exactly; with
+ *          less it runs each sequence in one pass (same result up to rounding, less
+ *          parallelism when B*H is small).  Calls that share a workspace must not
+ *          overlap on the device.
+ * T = 0 is allowed: nothing is read from q, k, v, o; the state is left as given (with
+ * LA_FLAG_INIT_STATE) or zeroed.  q, k, v, o may then be NULL.
+ * o must not overlap q, k, v or the state.
+ */
+la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H, int T, int d_k, int d_v,
+                       const void *q, const void *k, const void *v,
+                       const float *gate, const float *beta,
+                       float *state, float *z, void *o,
+                       int chunk, unsigned flags, void *workspace, size_t workspace_bytes,
+                       void *stream);
+
+/*
+ * la_prefill_workspace_size -- bytes of workspace la_prefill can use for these sizes
+ * (0 when the kernel for them needs none).  Host-only; touches no device.
+ */
+size_t la_prefill_workspace_size(la_mode_t mode, la_dtype_t dtype, int B, int H, int T, int d_k,
+                                 int d_v, int chunk);
+
+/*
+ * la_decode_step -- one token of the recurrent form ([three forms] "recurrent form",
+ * [decay/gates], [delta rule]) for N independent sequences, updating the state in place:
+ * the per-token cost is O(d_k d_v) and independent of how many tokens came before.
+ *
+ *   q, k   [N, H, d_k]  I/O dtype       v [N, H, d_v]  I/O dtype
+ *   gate   [N, H] fp32 or NULL          beta [N, H] fp32 (mode 2) or NULL
+ *   state  [N, H, d_v, d_k] fp32 in/out z [N, H, d_k] fp32 in/out (mode 0 only)
+ *   o      [N, H, d_v] I/O dtype out
+ */
+la_status_t la_decode_step(la_mode_t mode, la_dtype_t dtype, int N, int H, int d_k, int d_v,
+                           const void *q, const void *k, const void *v,
+                           const float *gate, const float *beta,
+                           float *state, float *z, void *o, void *stream);
+
+/*
+ * la_check_status -- synchronise `stream`, then report the first device-side failure
+ * since the last call: LA_ERR_CUDA for a CUDA error, LA_ERR_TIMEOUT if a kernel's
+ * bounded wait ran out (the kernel then returned early and its outputs are invalid).
+ * Clears the recorded failure.  Returns LA_OK if nothing failed.
+ */
+la_status_t la_check_status(void *stream);
+
+/* A static, human-readable description of a status code. */
+const char *la_status_string(la_status_t status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int la_version(void);
+
+/* Number of kernels this library has enqueued in this process (all devices, all
+ * threads), a monotonically increasing diagnostic counter. */
+unsigned long long la_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LINATTN_LA_H */

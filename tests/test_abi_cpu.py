@@ -1,0 +1,106 @@
+"""The C-ABI library loads on a machine without a GPU and exports what include/la.h declares.
+
+No compute call is made here: only symbol lookup, status strings, and argument checks
+that the library answers on the host before touching the device.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_attention_b200 import build
+    build.build()
+    import gated_delta_rule_attention_b200 as la
+    return la.library()
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if fn.endswith(".h"):
+            text = open(os.path.join(HEADER_DIR, fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(la_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("la_prefill", "la_decode_step", "la_check_status", "la_status_string",
+                     "la_version", "la_prefill_workspace_size", "la_kernel_launches"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    from gated_delta_rule_attention_b200 import library_path
+    out = subprocess.run(["nm", "-D", "--defined-only", library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(la_[a-z0-9_]+)$", out, flags=re.M))
+    assert set(declared_functions()) <= exported
+
+
+def test_library_does_not_need_libcuda(lib):
+    from gated_delta_rule_attention_b200 import library_path
+    out = subprocess.run(["readelf", "-d", library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    assert "libcuda.so" not in out
+
+
+def test_status_strings_and_version(lib):
+    for code, tag in enumerate(["LA_OK", "LA_ERR_INVALID_ARG", "LA_ERR_UNSUPPORTED",
+                                "LA_ERR_CUDA", "LA_ERR_TIMEOUT"]):
+        assert lib.la_status_string(code).decode().startswith(tag)
+    assert lib.la_status_string(99).decode() == "unknown la_status_t"
+    assert lib.la_version() >= 100
+
+
+def _prefill(lib, mode=2, dtype=1, B=1, H=1, T=8, dk=128, dv=128, chunk=0, flags=0):
+    null = None
+    return lib.la_prefill(mode, dtype, B, H, T, dk, dv, null, null, null, null, null, null, null,
+                          null, chunk, flags, null, 0, null)
+
+
+def test_host_side_argument_checks(lib):
+    INVALID, UNSUPPORTED = 1, 2
+    assert _prefill(lib, mode=3) == INVALID
+    assert _prefill(lib, mode=-1) == INVALID
+    assert _prefill(lib, dtype=2) == INVALID
+    assert _prefill(lib, B=0) == INVALID
+    assert _prefill(lib, H=0) == INVALID
+    assert _prefill(lib, T=-1) == INVALID
+    assert _prefill(lib, flags=4) == INVALID
+    assert _prefill(lib, chunk=-8) == INVALID
+    assert _prefill(lib, dk=96) == UNSUPPORTED
+    assert _prefill(lib, dv=256) == UNSUPPORTED
+    # NULL tensors are rejected before any launch
+    assert _prefill(lib) == INVALID
+    assert lib.la_decode_step(2, 1, 0, 1, 128, 128, *([None] * 9)) == INVALID
+    assert lib.la_decode_step(2, 1, 1, 1, 128, 32, *([None] * 9)) == UNSUPPORTED
+    assert lib.la_decode_step(2, 1, 4, 2, 128, 128, *([None] * 9)) == INVALID
+
+
+def test_workspace_size_query(lib):
+    # bf16, d = 128: the tensor-core kernel; few heads and a long sequence -> segments
+    assert lib.la_prefill_workspace_size(2, 1, 2, 16, 32768, 128, 128, 0) > 0
+    assert lib.la_prefill_workspace_size(1, 1, 8, 16, 8192, 128, 128, 0) == 0   # 128 heads
+    assert lib.la_prefill_workspace_size(0, 0, 1, 2, 256, 64, 64, 0) == 0       # fp32 path
+    assert lib.la_prefill_workspace_size(3, 1, 1, 1, 64, 128, 128, 0) == 0
+
+
+def test_host_pointers_are_rejected(lib):
+    """A host buffer is never handed to a kernel: the pointer check runs first."""
+    import numpy as np
+    buf = np.zeros(1 << 16, dtype=np.float32)
+    p = buf.ctypes.data_as(ctypes.c_void_p)
+    st = lib.la_decode_step(1, 0, 1, 1, 64, 64, p, p, p, None, None, p, None, p, None)
+    assert st == 1

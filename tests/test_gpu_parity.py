@@ -1,0 +1,177 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Element-by-element comparison on seeded inputs at sizes that span several chunks and a
+ragged tail, the edge cases (T = 1, T = 0, a chunk-aligned T, weak decay, gate = 1,
+beta -> 0/1, an initial state, split prefill, prefill followed by decode), and the
+full-size workloads in the launch configuration the benchmark times, checked on
+sampled heads the oracle can compute.  Tolerance: max relative error per (batch, head)
+slice of 2e-3 for fp32 I/O and 2e-2 for bf16 I/O (fp32 accumulation).
+"""
+import itertools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from parity_util import TOL, f64, oracle_prefill_slices, pick, slice_rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def la():
+    import gated_delta_rule_attention_b200 as m
+    m.library()
+    return m
+
+
+def small(mode, dtype, d, T, B=2, H=3, gate="softplus", gate_shift=0.0, seed=100):
+    return W.Workload(f"m{mode}", mode, dtype, B=B, H=H, T=T, dk=d, dv=d, seed=seed,
+                      qk_scale=1 / np.sqrt(d), qk_l2norm=(mode == 2),
+                      gate="none" if mode == 0 else gate, gate_shift=gate_shift,
+                      beta=(mode == 2))
+
+
+def run_and_compare(la, w, init_std=0.0, chunk=0, heads=None):
+    inp = W.prefill_inputs(w, device="cuda", init_state_std=init_std)
+    init = init_std > 0
+    z0 = None
+    if w.mode == 0 and init:
+        z0 = torch.rand(w.B, w.H, w.dk, device="cuda") * 10 + 1
+    state = inp["state0"].clone()
+    z = z0.clone() if z0 is not None else None
+    o, S, zz = la.prefill(inp["q"], inp["k"], inp["v"], mode=w.mode, gate=inp["gate"],
+                          beta=inp["beta"], state=state, z=z, chunk=chunk, init_state=init)
+    la.check_status()
+    if heads is None:
+        heads = list(itertools.product(range(w.B), range(w.H)))
+    ro, rS, rz = oracle_prefill_slices(w.mode, inp, heads, init_state=init, z0=z0)
+    tol = TOL[w.dtype]
+    eo = slice_rel_err(pick(o, heads), ro, lead=1)
+    eS = slice_rel_err(pick(S, heads), rS, lead=1)
+    assert eo <= tol, f"output rel err {eo:.3e} > {tol}"
+    assert eS <= tol, f"state rel err {eS:.3e} > {tol}"
+    if w.mode == 0:
+        ez = slice_rel_err(pick(zz, heads), rz, lead=1)
+        assert ez <= tol, f"z rel err {ez:.3e}"
+    return eo, eS
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T", [1, 64, 200])
+def test_prefill_small(la, mode, dtype, d, T):
+    run_and_compare(la, small(mode, dtype, d, T))
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("gate,shift", [("softplus", -4.0), ("none", 0.0)])
+def test_prefill_weak_decay_exercises_the_carried_state(la, mode, dtype, gate, shift):
+    """With a ~ 0.98 or a = 1 the state from earlier chunks dominates the output."""
+    run_and_compare(la, small(mode, dtype, 128, 333, gate=gate, gate_shift=shift))
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_prefill_initial_state(la, mode, dtype):
+    run_and_compare(la, small(mode, dtype, 128, 150, gate_shift=-3.0), init_std=0.05)
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_prefill_empty_sequence(la, mode):
+    w = small(mode, torch.bfloat16, 128, 0)
+    inp = W.prefill_inputs(w, device="cuda", init_state_std=0.1)
+    state = inp["state0"].clone()
+    z = torch.ones(w.B, w.H, w.dk, device="cuda") if mode == 0 else None
+    o, S, zz = la.prefill(inp["q"], inp["k"], inp["v"], mode=mode, gate=inp["gate"],
+                          beta=inp["beta"], state=state, z=z, init_state=True)
+    la.check_status()
+    assert o.shape[2] == 0 and torch.equal(S, inp["state0"])
+    S2 = torch.full_like(state, 7.0)
+    z2 = torch.full_like(z, 7.0) if mode == 0 else None
+    la.prefill(inp["q"], inp["k"], inp["v"], mode=mode, gate=inp["gate"], beta=inp["beta"],
+               state=S2, z=z2, init_state=False)
+    la.check_status()
+    assert torch.count_nonzero(S2) == 0
+    if mode == 0:
+        assert torch.count_nonzero(z2) == 0
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_split_prefill_then_decode_continues(la, mode):
+    """prefill(T1) ; prefill(T2 from that state) ; n decode steps == oracle over T1+T2+n."""
+    dtype = torch.bfloat16
+    w = small(mode, dtype, 128, 180, B=1, H=4, gate_shift=-3.0)
+    inp = W.prefill_inputs(w, device="cuda")
+    T1, T2 = 77, 70
+    sl = lambda t, a, b: None if t is None else t[:, :, a:b].contiguous()
+    o1, S, z = la.prefill(sl(inp["q"], 0, T1), sl(inp["k"], 0, T1), sl(inp["v"], 0, T1),
+                          mode=mode, gate=sl(inp["gate"], 0, T1), beta=sl(inp["beta"], 0, T1))
+    o2, S, z = la.prefill(sl(inp["q"], T1, T1 + T2), sl(inp["k"], T1, T1 + T2),
+                          sl(inp["v"], T1, T1 + T2), mode=mode, gate=sl(inp["gate"], T1, T1 + T2),
+                          beta=sl(inp["beta"], T1, T1 + T2), state=S, z=z, init_state=True)
+    outs = [o1, o2]
+    for t in range(T1 + T2, w.T):
+        g = None if inp["gate"] is None else inp["gate"][:, :, t].contiguous()
+        b = None if inp["beta"] is None else inp["beta"][:, :, t].contiguous()
+        od, S, z = la.decode_step(inp["q"][:, :, t].contiguous(), inp["k"][:, :, t].contiguous(),
+                                  inp["v"][:, :, t].contiguous(), mode=mode, state=S, gate=g,
+                                  beta=b, z=z)
+        outs.append(od[:, :, None])
+    la.check_status()
+    o = torch.cat(outs, dim=2)
+    heads = [(0, h) for h in range(w.H)]
+    ro, rS, _ = oracle_prefill_slices(mode, inp, heads)
+    assert slice_rel_err(pick(o, heads), ro, lead=1) <= TOL[dtype]
+    assert slice_rel_err(pick(S, heads), rS, lead=1) <= TOL[dtype]
+
+
+def test_heads_batches_independent(la):
+    """Changing one head's inputs changes only that head's outputs."""
+    w = small(2, torch.bfloat16, 128, 130)
+    inp = W.prefill_inputs(w, device="cuda")
+    o1, S1, _ = la.prefill(inp["q"], inp["k"], inp["v"], mode=2, gate=inp["gate"], beta=inp["beta"])
+    v2 = inp["v"].clone()
+    v2[1, 2] = -v2[1, 2]
+    o2, S2, _ = la.prefill(inp["q"], inp["k"], v2, mode=2, gate=inp["gate"], beta=inp["beta"])
+    la.check_status()
+    mask = torch.ones(w.B, w.H, dtype=torch.bool)
+    mask[1, 2] = False
+    assert torch.equal(o1[mask], o2[mask]) and torch.equal(S1[mask], S2[mask])
+    assert torch.allclose(o1[1, 2].float(), -o2[1, 2].float(), atol=1e-2)
+
+
+# ----------------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_steps(la, mode, dtype, d):
+    w = W.Workload("dec", mode, dtype, B=6, H=3, T=12, dk=d, dv=d, seed=7,
+                   qk_scale=1 / np.sqrt(d), qk_l2norm=(mode == 2),
+                   gate="none" if mode == 0 else "softplus", gate_shift=-2.0, beta=(mode == 2),
+                   decode=True, state_std=0.02)
+    inp = W.decode_inputs(w, device="cuda")
+    S = inp["state0"].clone()
+    z = inp["z0"].clone() if mode == 0 else None
+    Sr = f64(inp["state0"])
+    zr = f64(inp["z0"]) if mode == 0 else None
+    for t in range(w.T):
+        g = None if inp["gate"] is None else inp["gate"][t]
+        b = None if inp["beta"] is None else inp["beta"][t]
+        o, S, z = la.decode_step(inp["q"][t], inp["k"][t], inp["v"][t], mode=mode, state=S,
+                                 gate=g, beta=b, z=z)
+        ro, Sr, zr = oracle.decode_step(mode, f64(inp["q"][t]), f64(inp["k"][t]), f64(inp["v"][t]),
+                                        None if g is None else f64(g),
+                                        None if b is None else f64(b), Sr, zr)
+        la.check_status()
+        assert slice_rel_err(f64(o), ro) <= TOL[dtype], t
+        assert slice_rel_err(f64(S), Sr) <= TOL[dtype], t
+        if mode == 0:
+            assert slice_rel_err(f64(z), zr) <= TOL[dtype]
