@@ -10,23 +10,27 @@
 //
 //   G   = [K; Q] K^T                            (rows 0-63: K K^T, rows 64-127: Q K^T)
 //   A   = (Q K^T) * exp(lam_t - lam_j), j <= t  (mode 0: phi(Q) phi(K)^T, no decay)
-//   modes 0/1:  O^T = diag-scaled  S Q^T  +  V^T A^T          (mode 0: / den_t)
-//               S  <- g_{L-1} S + V^T diag(dec) K
+//   modes 0/1:  O  = diag(g) Q S^T + A V          (mode 0: divided by den_t)
+//               S <- g_{L-1} S + V^T diag(dec) K
 //   mode 2:     Lm = strictly-lower(diag(b) exp(lam_t - lam_j) K K^T),  T = (I + Lm)^-1
 //               U^T = V^T (T diag(b))^T,  W^T = K^T (T diag(b g))^T
-//               E^T = U^T - S W^T            (the write vectors e_t = b_t(v_t - a_t S_{t-1} k_t))
-//               O^T = diag-scaled S Q^T + E^T A^T,   S <- g_{L-1} S + (E^T diag(dec)) K
+//               E^T = U^T - S W^T   (the write vectors e_t = b_t (v_t - a_t S_{t-1} k_t))
+//               O  = diag(g) Q S^T + A E,   S <- g_{L-1} S + (E^T diag(dec)) K
 //
-// Every product has M = 128 (a d_v or d_k dimension) so each is one tcgen05.mma
-// shape (M=128, N=64 or 128, K=16 steps).  Tensor memory holds the fp32 state S (128
-// columns) and the products G, P = S Q^T, R, U^T, W^T, Y = S W^T (64 columns each):
-// exactly the 512 columns of one SM.  The state never leaves the chip between chunks;
-// each chunk the epilogue reads it once to write a bf16 copy (the MMA operand for
-// the next chunk) and to apply the next chunk's decay in place.
+// Products and where they live (M x N x K, tcgen05.mma kind::f16, fp32 accumulators
+// in tensor memory):  G 128x64x128, U^T and W^T 128x64x64, Y = S W^T 128x64x128,
+// dS = V^T K~ (or E'^T K) 128x128x64, O = Q~ S^T + A V (or A E) 64x128x(128+64).  The
+// fp32 state S itself stays in the epilogue threads' registers across chunks (each
+// thread owns half a row); each chunk adds dS to it and writes a bf16 copy to shared
+// memory as the operand of the next chunk's products.  diag(g) and diag(dec) are folded
+// into the operands by scaling the Q and K tiles in shared memory (mode 1) or the E
+// tile (mode 2), after K K^T / Q K^T have been formed from the unscaled tiles.
 //
-// Warp roles (256 threads): warp 0 lane 0 issues TMA loads into a 2-stage ring;
-// warp 1 owns TMEM and lane 0 issues every MMA; warps 4-7 (thread e <-> TMEM lane e)
-// do all CUDA-core work: gates, phi, masks, the 64x64 triangular inverse, epilogues.
+// Warp roles (320 threads): warp 0 lane 0 issues TMA loads into a ring of stages;
+// warp 1 owns TMEM and lane 0 issues every MMA; warps 2-9 are the epilogue: two warps
+// per TMEM lane quarter, each taking one half of the columns.  The schedule per chunk c
+// (epilogue: A-epilogue(c), prologue of c+1, state(c), output(c)) lets the tensor core
+// form G(c+1) and O(c), dS(c) while the epilogue works on the neighbouring chunk.
 // Roles hand off through mbarriers; every wait is bounded (a timeout records an error
 // and the CTA winds down: in-flight copies and MMAs are drained before TMEM is freed).
 //
@@ -41,6 +45,7 @@
 #include "ptx.cuh"
 #include "tmap.cuh"
 
+#include <algorithm>
 #include <cfloat>
 
 namespace la {
@@ -50,11 +55,12 @@ using namespace ptx;
 
 constexpr int kC = 64;         // chunk
 constexpr int kD = 128;        // d_k = d_v
-constexpr int kThreads = 256;
+constexpr int kThreads = 320;  // 10 warps
+constexpr int kEpi = 256;      // epilogue threads (warps 2-9)
 constexpr uint32_t kTmemCols = 512;
 // TMEM column map
-constexpr uint32_t kColS = 0, kColG = 128, kColP = 192, kColR = 256, kColU = 320, kColW = 384,
-                   kColY = 448;
+constexpr uint32_t kColDS = 0, kColG = 128, kColU = 192, kColW = 256, kColY = 320, kColO = 384;
+constexpr float kLog2e = 1.4426950408889634f;
 
 enum Kind { kOutput = 0, kLocal = 1, kTransition = 2 };
 
@@ -75,49 +81,60 @@ struct TcParams {
     long long s_out_seg;
     float *z_out;
     long long z_out_seg;
-    float *gam_out;              // LOCAL, modes 0/1: product of the segment's gates
+    float *gam_out;              // LOCAL, mode 1: product of the segment's gates
     int out_last_only;
     int T, BH, seg_len, nseg;
     unsigned *err;
 };
 
-// ------------------------------------------------------------------ shared layout
 struct Small {
-    uint64_t full[2], empty[2];
+    uint64_t full[3], empty[3];
     uint64_t prep_done, g_done, a_ready, tt_ready, ut_done, w_ready, py_done, e_ready,
         mma2_done, s_ready, fin;
     uint32_t tmem_base;
     int abort;
     int len[2];
-    float lam[2][kC];
+    float lam[2][kC];    // in-chunk inclusive prefix of log2(a), per chunk parity
     float bet[2][kC];
-    float den[kC];
+    float part[4][kC];   // mode 0: row-sum halves, phi(q).z halves
     float z[kD];
     float scan_tmp[2];
     float gsum;
 };
 
-constexpr uint32_t kStageBytes = 49152;           // [K0][Q0][K1][Q1][V0][V1], 8 KB each
-constexpr uint32_t kOffStage0 = 0, kOffStage1 = kStageBytes;
-constexpr uint32_t kOffSbf = 2 * kStageBytes;     // 32 KB bf16 state, K-major [d_v][d_k]
-constexpr uint32_t kOffA = kOffSbf + 32768;       // 8 KB  A [t][j]
-constexpr uint32_t kOffTp = kOffA + 8192;         // 8 KB  T'  | K~ cb0 (mode 1)
-constexpr uint32_t kOffTpp = kOffTp + 8192;       // 8 KB  T'' | K~ cb1 (mode 1)
-constexpr uint32_t kOffX = kOffTpp + 8192;        // 48 KB (mode 2): E | E' | W  or  Lm | Tm | Z
-constexpr uint32_t kOffE = kOffX, kOffEp = kOffX + 16384, kOffW = kOffX + 32768;
+// Shared-memory layout (bytes from the 1024-aligned base).
+template <int MODE>
+struct Lay {
+    static constexpr int kStages = MODE == 2 ? 2 : 3;
+    static constexpr uint32_t kStage = 49152;          // [K0][Q0][K1][Q1][V0][V1], 8 KB each
+    static constexpr uint32_t kSbf = kStages * kStage; // 32 KB bf16 state, [d_v][d_k]
+    static constexpr uint32_t kA = kSbf + 32768;       // 8 KB  A [t][j]
+    static constexpr uint32_t kTp = kA + 8192;         // 8 KB  T diag(b)      (mode 2)
+    static constexpr uint32_t kTpp = kTp + 8192;       // 8 KB  T diag(b g)    (mode 2)
+    static constexpr uint32_t kX = kTpp + 8192;        // 48 KB E | E' | W  or  Lm | Tm | Zs
+    static constexpr uint32_t kE = kX, kEp = kX + 16384, kW = kX + 32768;
+    static constexpr uint32_t kSmall = MODE == 2 ? kX + 49152 : kA + 8192;
+    static constexpr uint32_t kBytes = kSmall + sizeof(Small);
+};
 constexpr uint32_t kLmStride = 65;
 
-template <int MODE>
-constexpr uint32_t smem_bytes() {
-    return (MODE == 2 ? kOffX + 49152 : kOffX) + sizeof(Small);
-}
-
-__device__ __forceinline__ void epi_sync() { named_sync(1, 128); }
-
+__device__ __forceinline__ void epi_sync() { named_sync(1, kEpi); }
 __device__ __forceinline__ uint64_t dk(uint32_t addr) { return sdesc_sw128(addr, 16, 1024); }
 __device__ __forceinline__ uint64_t dmn(uint32_t addr, uint32_t lbo) {
     return sdesc_sw128(addr, lbo, 1024);
 }
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// phi(x) = elu(x) + 1 = x + 1 for x > 0, e^x otherwise
+__device__ __forceinline__ float phi_fast(float x) { return x > 0.f ? x + 1.f : ex2(x * kLog2e); }
 
 // Bounded wait that ignores the abort flag (used to drain in-flight work on exit).
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
@@ -125,15 +142,39 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
         if (mbar_try_wait(bar, parity)) return;
 }
 
-// Load and prefix-sum the gates of chunk `c` into buffer `buf` (64 threads, e < 64).
+// Write 16 fp32 values as bf16 = two 16-byte chunks (ch, ch+1) of row `row` of the
+// 128B-swizzled tile at shared address `tile`.
+__device__ __forceinline__ void st_row_bf16x16(uint32_t tile, uint32_t row, uint32_t ch,
+                                               const float *v) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+        w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+        w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+        w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+        sts128(tile + sw128_off(row, ch + q), w);
+    }
+}
+// Multiply the 8 bf16 values of a 16-byte chunk by s.
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 w, float s) {
+    uint32_t *wd = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float2 f = unpack_bf16x2(wd[q]);
+        wd[q] = pack_bf16x2(f.x * s, f.y * s);
+    }
+    return w;
+}
+
+// Gates of chunk c into parity buffer `buf`: log2 prefix and beta (64 threads, e < 64).
 template <int MODE>
 __device__ __forceinline__ void load_gates(const TcParams &p, Small *sm, int bh, int tb, int te,
                                            int c, int buf, int e) {
     const int t0 = tb + kC * c;
     const int L = min(kC, te - t0);
     float g = 0.f;
-    if (MODE != 0 && p.gate && e < L) g = logf(fmaxf(p.gate[(size_t)bh * p.T + t0 + e], FLT_MIN));
-    // inclusive scan across 64 threads (two warps)
+    if (MODE != 0 && p.gate && e < L) g = lg2(fmaxf(p.gate[(size_t)bh * p.T + t0 + e], FLT_MIN));
     const int lane = e & 31;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -149,7 +190,7 @@ __device__ __forceinline__ void load_gates(const TcParams &p, Small *sm, int bh,
     named_sync(2, 64);
 }
 
-// 64x64 unit lower-triangular inverse, T = (I + Lm)^-1, by 16x16 blocks (128 threads).
+// 64x64 unit lower-triangular inverse T = (I + Lm)^-1 by 16x16 blocks (256 threads).
 __device__ void invert_unit_lower(const float *Lm, float *Tm, float *Zs, int e) {
     constexpr int S = kLmStride;
     if (e < 64) {
@@ -159,18 +200,19 @@ __device__ void invert_unit_lower(const float *Lm, float *Tm, float *Zs, int e) 
         for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
 #pragma unroll
         for (int r = 1; r < 16; ++r) {
-            float s = 0.f;
+            float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < r; ++j) s = fmaf(Lm[(16 * b + r) * S + 16 * b + j], x[j], s);
-            if (r > c) x[r] = -s;
+            for (int j = 0; j < r; j += 2) {
+                s0 = fmaf(Lm[(16 * b + r) * S + 16 * b + j], x[j], s0);
+                if (j + 1 < r) s1 = fmaf(Lm[(16 * b + r) * S + 16 * b + j + 1], x[j + 1], s1);
+            }
+            if (r > c) x[r] = -(s0 + s1);
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) Tm[(16 * b + r) * S + 16 * b + c] = x[r];
     } else {
-        // zero the six blocks above the block diagonal
-        for (int idx = e - 64; idx < 6 * 256; idx += 64) {
+        for (int idx = e - 64; idx < 6 * 256; idx += kEpi - 64) {
             const int blk = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
-            // (i, j) with j > i: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
             const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
             const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
             Tm[(16 * bi + r) * S + 16 * bj + cc] = 0.f;
@@ -179,61 +221,51 @@ __device__ void invert_unit_lower(const float *Lm, float *Tm, float *Zs, int e) 
     epi_sync();
     for (int d = 1; d < 4; ++d) {
         const int outs = (4 - d) * 256;
-        for (int idx = e; idx < outs; idx += 128) {
+        for (int idx = e; idx < outs; idx += kEpi) {
             const int blk = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
             const int bi = blk + d, bj = blk;
-            float z = 0.f;
-            for (int k = 16 * bj; k < 16 * bi; ++k)
-                z = fmaf(Lm[(16 * bi + r) * S + k], Tm[k * S + 16 * bj + cc], z);
-            Zs[blk * 272 + r * 17 + cc] = z;
+            float z0 = 0.f, z1 = 0.f;
+            for (int k = 16 * bj; k < 16 * bi; k += 2) {
+                z0 = fmaf(Lm[(16 * bi + r) * S + k], Tm[k * S + 16 * bj + cc], z0);
+                z1 = fmaf(Lm[(16 * bi + r) * S + k + 1], Tm[(k + 1) * S + 16 * bj + cc], z1);
+            }
+            Zs[blk * 272 + r * 17 + cc] = z0 + z1;
         }
         epi_sync();
-        for (int idx = e; idx < outs; idx += 128) {
+        for (int idx = e; idx < outs; idx += kEpi) {
             const int blk = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
             const int bi = blk + d, bj = blk;
-            float t = 0.f;
+            float t0 = 0.f, t1 = 0.f;
 #pragma unroll
-            for (int m = 0; m < 16; ++m)
-                t = fmaf(Tm[(16 * bi + r) * S + 16 * bi + m], Zs[blk * 272 + m * 17 + cc], t);
-            Tm[(16 * bi + r) * S + 16 * bj + cc] = -t;
+            for (int m = 0; m < 16; m += 2) {
+                t0 = fmaf(Tm[(16 * bi + r) * S + 16 * bi + m], Zs[blk * 272 + m * 17 + cc], t0);
+                t1 = fmaf(Tm[(16 * bi + r) * S + 16 * bi + m + 1], Zs[blk * 272 + (m + 1) * 17 + cc],
+                          t1);
+            }
+            Tm[(16 * bi + r) * S + 16 * bj + cc] = -(t0 + t1);
         }
         epi_sync();
-    }
-}
-
-// Write 16 fp32 values as 8 bf16 pairs = two 16-byte chunks (chunk index ch, ch+1) of
-// row `row` in a 128B-swizzled tile at shared address `tile`.
-__device__ __forceinline__ void st_row_bf16x16(uint32_t tile, uint32_t row, uint32_t ch,
-                                               const float *v) {
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        uint4 w;
-        w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-        w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-        w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-        w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-        sts128(tile + sw128_off(row, ch + q), w);
     }
 }
 
 template <int MODE, int KIND>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
+    using Y = Lay<MODE>;
+    constexpr int NST = Y::kStages;
+    constexpr bool kOut = (KIND == kOutput);
+    constexpr bool kNeedG = (MODE == 2) || kOut;
+    constexpr bool kNeedV = (KIND != kTransition);
+
     // 128B-swizzled operand tiles need 1024-byte aligned atoms.  The buffer is declared
     // with that alignment and never re-aligned by integer arithmetic: pointers derived
     // from it keep the shared address space.
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *sm8 = smem_raw;
-    const uint32_t sm_base = smem_u32(smem_raw);
-    if (sm_base & 1023u) {
+    const uint32_t sb = smem_u32(smem_raw);
+    if (sb & 1023u) {
         if (threadIdx.x == 0 && p.err) atomicOr(p.err, (unsigned)kErrBadLaunch);
         return;
     }
-    Small *sm = reinterpret_cast<Small *>(sm8 + (MODE == 2 ? kOffX + 49152 : kOffX));
-    const uint32_t stage_addr[2] = {sm_base + kOffStage0, sm_base + kOffStage1};
-
-    constexpr bool kOut = (KIND == kOutput);
-    constexpr bool kNeedG = (MODE == 2) || kOut;
-    constexpr bool kNeedV = (KIND != kTransition);
+    Small *sm = reinterpret_cast<Small *>(smem_raw + Y::kSmall);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -244,10 +276,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     const int nch = (te - tb + kC - 1) / kC;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sm->full[0], 1);
-        mbar_init(&sm->full[1], 1);
-        mbar_init(&sm->empty[0], 1);
-        mbar_init(&sm->empty[1], 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&sm->full[s], 1);
+            mbar_init(&sm->empty[s], 1);
+        }
         mbar_init(&sm->prep_done, 1);
         mbar_init(&sm->g_done, 1);
         mbar_init(&sm->a_ready, 1);
@@ -279,11 +311,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             tma_prefetch_desc(&p.tk);
             if (kOut) tma_prefetch_desc(&p.tq);
             if (kNeedV) tma_prefetch_desc(&p.tv);
-            int issued[2] = {0, 0};
+            int issued[NST];
+            for (int s = 0; s < NST; ++s) issued[s] = 0;
             for (int c = 0; c < nch; ++c) {
-                const int s = c & 1, u = c >> 1;
+                const int s = c % NST, u = c / NST;
                 if (u >= 1 && !mbar_wait(&sm->empty[s], (u - 1) & 1, abort, p.err)) break;
-                const uint32_t st = stage_addr[s];
+                const uint32_t st = sb + s * Y::kStage;
                 const int t = tb + kC * c;
                 const uint32_t bytes = 16384u * (1u + (kOut ? 1u : 0u) + (kNeedV ? 1u : 0u));
                 mbar_arrive_expect_tx(&sm->full[s], bytes);
@@ -299,30 +332,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 }
                 issued[s] = u + 1;
             }
-            // make sure no copy is still writing shared memory when the CTA exits
-            for (int s = 0; s < 2; ++s)
+            // no copy may still be writing shared memory when the CTA exits
+            for (int s = 0; s < NST; ++s)
                 if (issued[s] > 0) drain_wait(&sm->full[s], (issued[s] - 1) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t sbf = sm_base + kOffSbf;
-            const uint32_t at = sm_base + kOffA;
-            const uint32_t tp = sm_base + kOffTp;
-            const uint32_t tpp = sm_base + kOffTpp;
-            const uint32_t et = sm_base + kOffE;
-            const uint32_t ept = sm_base + kOffEp;
-            const uint32_t wt = sm_base + kOffW;
-            const uint32_t id_n64_kk = idesc_bf16(128, 64, false, false);
-            const uint32_t id_n64_mk = idesc_bf16(128, 64, true, false);
-            const uint32_t id_n64_km = idesc_bf16(128, 64, false, true);
-            const uint32_t id_n128_mm = idesc_bf16(128, 128, true, true);
-            const uint32_t id_n128_km = idesc_bf16(128, 128, false, true);
-            bool ok = true;
-            for (int c = 0; c < nch && ok; ++c) {
-                const int s = c & 1, u = c >> 1;
+            const uint32_t sbf = sb + Y::kSbf, at = sb + Y::kA, tp = sb + Y::kTp,
+                           tpp = sb + Y::kTpp, et = sb + Y::kE, ept = sb + Y::kEp,
+                           wt = sb + Y::kW;
+            const uint32_t id_g = idesc_bf16(128, 64, false, false);
+            const uint32_t id_uw = idesc_bf16(128, 64, true, false);
+            const uint32_t id_y = idesc_bf16(128, 64, false, true);
+            const uint32_t id_o1 = idesc_bf16(64, 128, false, false);
+            const uint32_t id_o2 = idesc_bf16(64, 128, false, MODE != 2);
+            const uint32_t id_ds = idesc_bf16(128, 128, MODE != 2, true);
+            for (int c = 0; c < nch; ++c) {
+                const int s = c % NST, u = c / NST;
                 const uint32_t par = c & 1;
-                const uint32_t st = stage_addr[s];
+                const uint32_t st = sb + s * Y::kStage;
                 if (!mbar_wait(&sm->full[s], u & 1, abort, p.err)) break;
                 if (!mbar_wait(&sm->prep_done, par, abort, p.err)) break;
                 tc_fence_after();
@@ -330,285 +359,282 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     // G = [K; Q] K^T   (M=128, N=64, K=128)
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16_ss(tm + kColG, dk(st + off), dk(st + off), id_n64_kk, ks > 0);
+                        mma_bf16_ss(tm + kColG, dk(st + off), dk(st + off), id_g, ks > 0);
                     }
                     mma_commit(&sm->g_done);
                 }
                 if constexpr (MODE == 2) {
                     if (!mbar_wait(&sm->tt_ready, par, abort, p.err)) break;
                     tc_fence_after();
-                    if (kNeedV) {
-                        // U^T = V^T (T diag b)^T  (A: V^T MN-major; B: T' K-major)
-                        for (int ks = 0; ks < 4; ++ks)
+                    for (int ks = 0; ks < 4; ++ks) {
+                        if (kNeedV)   // U^T = V^T (T diag b)^T
                             mma_bf16_ss(tm + kColU, dmn(st + 32768 + ks * 2048, 8192),
-                                        dk(tp + ks * 32), id_n64_mk, ks > 0);
-                    }
-                    // W^T = K^T (T diag(b g))^T
-                    for (int ks = 0; ks < 4; ++ks)
+                                        dk(tp + ks * 32), id_uw, ks > 0);
+                        // W^T = K^T (T diag(b g))^T
                         mma_bf16_ss(tm + kColW, dmn(st + ks * 2048, 16384), dk(tpp + ks * 32),
-                                    id_n64_mk, ks > 0);
+                                    id_uw, ks > 0);
+                    }
                     mma_commit(&sm->ut_done);
                     if (!mbar_wait(&sm->w_ready, par, abort, p.err)) break;
                     if (!mbar_wait(&sm->s_ready, par, abort, p.err)) break;
                     tc_fence_after();
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t soff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        if (kOut)   // P = S Q^T
-                            mma_bf16_ss(tm + kColP, dk(sbf + soff), dk(st + 8192 + soff), id_n64_kk,
-                                        ks > 0);
-                        // Y = S W^T  (B: W MN-major [d_k rows][t])
-                        mma_bf16_ss(tm + kColY, dk(sbf + soff), dmn(wt + ks * 2048, 8192),
-                                    id_n64_km, ks > 0);
-                    }
+                    for (int ks = 0; ks < 8; ++ks)   // Y = S W^T
+                        mma_bf16_ss(tm + kColY, dk(sbf + (ks >> 2) * 16384 + (ks & 3) * 32),
+                                    dmn(wt + ks * 2048, 8192), id_y, ks > 0);
                     mma_commit(&sm->py_done);
                     if (!mbar_wait(&sm->e_ready, par, abort, p.err)) break;
                     tc_fence_after();
-                    for (int ks = 0; ks < 4; ++ks) {
-                        if (kOut)   // R = E^T A^T
-                            mma_bf16_ss(tm + kColR, dk(et + ks * 32), dk(at + ks * 32), id_n64_kk,
-                                        ks > 0);
-                        // S += (E^T diag dec) K   (B: K MN-major)
-                        mma_bf16_ss(tm + kColS, dk(ept + ks * 32), dmn(st + ks * 2048, 16384),
-                                    id_n128_km, true);
-                    }
-                    mma_commit(&sm->mma2_done);
                 } else {
+                    if (!mbar_wait(&sm->a_ready, par, abort, p.err)) break;
                     if (!mbar_wait(&sm->s_ready, par, abort, p.err)) break;
                     tc_fence_after();
-                    if (kOut) {
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const uint32_t soff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                            mma_bf16_ss(tm + kColP, dk(sbf + soff), dk(st + 8192 + soff),
-                                        id_n64_kk, ks > 0);
-                        }
-                    }
-                    if (!mbar_wait(&sm->a_ready, par, abort, p.err)) break;
-                    tc_fence_after();
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t vt = dmn(st + 32768 + ks * 2048, 8192);
-                        if (kOut)   // R = V^T A^T
-                            mma_bf16_ss(tm + kColR, vt, dk(at + ks * 32), id_n64_mk, ks > 0);
-                        // S += V^T diag(dec) K
-                        const uint64_t kb = (MODE == 1) ? dmn(tp + ks * 2048, 8192)
-                                                        : dmn(st + ks * 2048, 16384);
-                        mma_bf16_ss(tm + kColS, vt, kb, id_n128_mm, true);
-                    }
-                    mma_commit(&sm->mma2_done);
                 }
+                if (kOut) {
+                    // O = Q~ S^T (+) A V  or  A E     (M=64, N=128)
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16_ss(tm + kColO, dk(st + 8192 + off), dk(sbf + off), id_o1, ks > 0);
+                    }
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t b2 = (MODE == 2) ? dk(et + ks * 32)
+                                                        : dmn(st + 32768 + ks * 2048, 8192);
+                        mma_bf16_ss(tm + kColO, dk(at + ks * 32), b2, id_o2, true);
+                    }
+                }
+                // dS = V^T K~ (modes 0/1) or (E^T diag dec) K (mode 2)   (M=128, N=128)
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t a2 = (MODE == 2) ? dk(ept + ks * 32)
+                                                    : dmn(st + 32768 + ks * 2048, 8192);
+                    mma_bf16_ss(tm + kColDS, a2, dmn(st + ks * 2048, 16384), id_ds, ks > 0);
+                }
+                mma_commit(&sm->mma2_done);
             }
-            // drain: nothing may still write TMEM when it is freed
+            // nothing may still write TMEM when it is freed
             mma_commit(&sm->fin);
             drain_wait(&sm->fin, 0);
         }
-    } else if (warp >= 4) {
-        // ------------------------------------------------------------ epilogue warps
-        const int e = threadIdx.x - 128;          // TMEM lane
-        const int wq = e >> 5;                    // lane quarter
-        const uint32_t trow = tm + ((uint32_t)(wq * 32) << 16);
-        const uint32_t sbf = sm_base + kOffSbf;
-        const uint32_t atile = sm_base + kOffA;
-        float *Lm = reinterpret_cast<float *>(sm8 + kOffX);
+    } else {
+        // ------------------------------------------------------------ epilogue warps 2-9
+        const int e = threadIdx.x - 64;            // 0..255
+        const int q = warp & 3;                    // TMEM lane quarter of this warp
+        const int h = (warp - 2) >> 2;             // column half
+        const int row = 32 * q + lane;             // TMEM lane = tile row
+        const uint32_t tl = tm + ((uint32_t)(32 * q) << 16);
+        const uint32_t sbf = sb + Y::kSbf;
+        float *Lm = reinterpret_cast<float *>(smem_raw + Y::kX);
         float *Tm = Lm + 64 * kLmStride;
         float *Zs = Tm + 64 * kLmStride;
         const size_t o_row0 = (size_t)bh * p.T;
 
-        if (e < 64) load_gates<MODE>(p, sm, bh, tb, te, 0, 0, e);
-        epi_sync();
-        // ---- initial state: row e of S
+        // ---- initial state: this thread's half row of S in registers, bf16 copy in smem
+        float Sr[64];
         {
-            const float scale0 = (MODE == 0) ? 1.f : __expf(sm->lam[0][kC - 1]);
             const float *src = nullptr;
-            if (p.s_in_mode == 1) src = p.s_in + (size_t)seg * p.s_in_seg + (size_t)bh * kD * kD;
-            for (int c0 = 0; c0 < kD; c0 += 16) {
-                float v[16];
+            if (p.s_in_mode == 1)
+                src = p.s_in + (size_t)seg * p.s_in_seg + (size_t)bh * kD * kD + (size_t)row * kD;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int col = c0 + j;
-                    v[j] = src ? src[(size_t)e * kD + col]
-                               : ((p.s_in_mode == 2 && col == e) ? 1.f : 0.f);
-                }
-                st_row_bf16x16(sbf + (c0 >> 6) * 16384, e, (c0 & 63) >> 3, v);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] *= scale0;
-                tmem_st16(trow + kColS + c0, v);
+            for (int j = 0; j < 64; ++j) {
+                const int col = 64 * h + j;
+                Sr[j] = src ? src[col] : ((p.s_in_mode == 2 && col == row) ? 1.f : 0.f);
             }
-            if (MODE == 0) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
+            if (MODE == 0 && e < kD) {
                 const float *zs = (p.s_in_mode == 1 && p.z_in)
                                       ? p.z_in + (size_t)seg * p.z_in_seg + (size_t)bh * kD
                                       : nullptr;
                 sm->z[e] = zs ? zs[e] : 0.f;
             }
             fence_async_smem();
-            tc_fence_before();
             epi_sync();
             if (e == 0) mbar_arrive(&sm->s_ready);
         }
 
-        for (int c = 0; c < nch; ++c) {
-            const int s = c & 1, u = c >> 1, buf = c & 1;
+        // ---- chunk prologue: gates, phi (mode 0); releases G's inputs to the MMA
+        auto prep = [&](int c) -> bool {
+            const int s = c % NST, u = c / NST;
+            if (e < 64) load_gates<MODE>(p, sm, bh, tb, te, c, c & 1, e);
+            mbar_wait(&sm->full[s], u & 1, abort, p.err);
+            epi_sync();
+            if (*abort) return false;
+            if (MODE == 0) {
+                const uint32_t st = sb + s * Y::kStage;
+                const int L = sm->len[c & 1];
+                const int nreg = kOut ? 4 : 2;
+                for (int n = e; n < nreg * 512; n += kEpi) {
+                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);   // 0,2 = K; 1,3 = Q
+                    const int r = (n & 511) >> 3;
+                    const uint32_t a = st + region * 8192 + (n & 511) * 16;
+                    uint4 w;
+                    if ((region & 1) == 0 && r >= L) {
+                        w = make_uint4(0, 0, 0, 0);
+                    } else {
+                        w = lds128(a);
+                        uint32_t *wd = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 f = unpack_bf16x2(wd[k]);
+                            wd[k] = pack_bf16x2(phi_fast(f.x), phi_fast(f.y));
+                        }
+                    }
+                    sts128(a, w);
+                }
+                fence_async_smem();
+            }
+            epi_sync();
+            if (e == 0) mbar_arrive(&sm->prep_done);
+            return true;
+        };
+
+        bool ok = prep(0);
+        for (int c = 0; c < nch && ok; ++c) {
+            const int s = c % NST, buf = c & 1;
             const uint32_t par = c & 1;
-            const uint32_t st = stage_addr[s];
+            const uint32_t st = sb + s * Y::kStage;
             const int t0 = tb + kC * c;
             const int L = sm->len[buf];
             const float *lam = sm->lam[buf];
-            mbar_wait(&sm->full[s], u & 1, abort, p.err);
-            epi_sync();
-            if (*abort) break;
+            const float lamL = lam[kC - 1];
 
-            // ---- prep: phi (mode 0) or K~ = diag(dec) K (mode 1)
-            if (MODE == 0) {
-                const int nreg = kOut ? 4 : 2;
-                for (int n = e; n < nreg * 512; n += 128) {
-                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);   // 0,2 = K; 1,3 = Q
-                    const int row = (n & 511) >> 3;
-                    const uint32_t ptr = st + region * 8192 + (n & 511) * 16;
-                    uint4 w = lds128(ptr);
-                    const bool is_k = (region & 1) == 0;
-                    if (is_k && row >= L) {
-                        w = make_uint4(0, 0, 0, 0);
-                    } else {
-                        uint32_t *wd = reinterpret_cast<uint32_t *>(&w);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float2 f = unpack_bf16x2(wd[q]);
-                            wd[q] = pack_bf16x2(feature_phi(f.x), feature_phi(f.y));
-                        }
-                    }
-                    sts128(ptr, w);
-                }
-            } else if (MODE == 1) {
-                const float lamL = lam[kC - 1];
-                for (int n = e; n < 1024; n += 128) {
-                    const int cb = n >> 9;
-                    const int row = (n & 511) >> 3;
-                    const float d = row < L ? __expf(lamL - lam[row]) : 0.f;
-                    uint4 w = lds128(st + cb * 16384 + (n & 511) * 16);
-                    uint32_t *wd = reinterpret_cast<uint32_t *>(&w);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float2 f = unpack_bf16x2(wd[q]);
-                        wd[q] = pack_bf16x2(f.x * d, f.y * d);
-                    }
-                    sts128(sm_base + kOffTp + cb * 8192 + (n & 511) * 16, w);
-                }
-            }
-            fence_async_smem();
-            epi_sync();
-            if (e == 0) mbar_arrive(&sm->prep_done);
-
-            // ---- G epilogue: A (rows of Q K^T) and, in mode 2, Lm (rows of K K^T)
+            // ---- A-epilogue: masks and decays of G; operand scaling
             if (kNeedG) {
                 mbar_wait(&sm->g_done, par, abort, p.err);
                 epi_sync();
                 if (*abort) break;
                 tc_fence_after();
-                if (e >= 64 && kOut) {
-                    const int i = e - 64;
-                    float rs = 0.f;
-                    for (int j0 = 0; j0 < kC; j0 += 16) {
-                        float v[16];
-                        tmem_ld16(trow + kColG + j0, v);
-    #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int jj = j0 + j;
-                            float a = 0.f;
-                            if (jj <= i) a = (MODE == 0) ? v[j] : v[j] * __expf(lam[i] - lam[jj]);
-                            v[j] = __bfloat162float(__float2bfloat16_rn(a));
-                            rs += v[j];
-                        }
-                        st_row_bf16x16(atile, i, j0 >> 3, v);
-                    }
-                    if (MODE == 0) {
-                        // den_i = sum_j A_ij + phi(q_i) . z   (phi(Q) row i in the stage)
-                        float qz = 0.f;
-                        for (int ch = 0; ch < 16; ++ch) {
-                            const uint32_t qb = st + 8192 + (ch >> 3) * 16384;
-                            const uint4 w = lds128(qb + sw128_off(i, ch & 7));
-                            const uint32_t *wd = reinterpret_cast<const uint32_t *>(&w);
+            }
+            if (q >= 2 && kOut) {
+                // rows i of Q K^T -> A tile, columns j in [32h, 32h + 32)
+                const int i = row - 64;
+                float rs = 0.f;
+                for (int g = 0; g < 2; ++g) {
+                    const int j0 = 32 * h + 16 * g;
+                    float v[16];
+                    tmem_ld16(tl + kColG + j0, v);
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const float2 f = unpack_bf16x2(wd[q]);
-                                qz = fmaf(f.x, sm->z[ch * 8 + 2 * q], qz);
-                                qz = fmaf(f.y, sm->z[ch * 8 + 2 * q + 1], qz);
-                            }
-                        }
-                        sm->den[i] = rs + qz;
+                    for (int j = 0; j < 16; ++j) {
+                        const int jj = j0 + j;
+                        float a = 0.f;
+                        if (jj <= i) a = (MODE == 0) ? v[j] : v[j] * ex2(lam[i] - lam[jj]);
+                        v[j] = __bfloat162float(__float2bfloat16_rn(a));
+                        rs += v[j];
                     }
-                } else if (e < 64 && MODE == 2) {
-                    const int i = e;
-                    const float bi = sm->bet[buf][i];
-                    for (int j0 = 0; j0 < kC; j0 += 16) {
-                        float v[16];
-                        tmem_ld16(trow + kColG + j0, v);
-    #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int jj = j0 + j;
-                            Lm[i * kLmStride + jj] =
-                                (jj < i) ? bi * __expf(lam[i] - lam[jj]) * v[j] : 0.f;
-                        }
+                    st_row_bf16x16(sb + Y::kA, i, j0 >> 3, v);
+                }
+                if (MODE == 0) sm->part[h][i] = rs;
+            } else if (q < 2 && MODE == 2) {
+                // rows r of K K^T -> Lm (strictly lower), columns j in [32h, 32h + 32)
+                const int r = row;
+                const float br = sm->bet[buf][r];
+                for (int g = 0; g < 2; ++g) {
+                    const int j0 = 32 * h + 16 * g;
+                    float v[16];
+                    tmem_ld16(tl + kColG + j0, v);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int jj = j0 + j;
+                        Lm[r * kLmStride + jj] = (jj < r) ? br * ex2(lam[r] - lam[jj]) * v[j] : 0.f;
                     }
                 }
-                fence_async_smem();
-                tc_fence_before();
-                epi_sync();
+            } else if (q < 2 && MODE == 0 && kOut) {
+                // phi(q_r) . z over d_k half h
+                const int r = row;
+                float qz = 0.f;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 w = lds128(st + 8192 + h * 16384 + sw128_off(r, ch));
+                    const uint32_t *wd = reinterpret_cast<const uint32_t *>(&w);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 f = unpack_bf16x2(wd[k]);
+                        qz = fmaf(f.x, sm->z[64 * h + 8 * ch + 2 * k], qz);
+                        qz = fmaf(f.y, sm->z[64 * h + 8 * ch + 2 * k + 1], qz);
+                    }
+                }
+                sm->part[2 + h][r] = qz;
             }
+            if (MODE == 1) {
+                // after G: Q <- diag(g) Q (output kinds) and K <- diag(dec) K, in place
+                for (int n = e; n < 1024; n += kEpi) {
+                    const int cb = n >> 9, r = (n & 511) >> 3;
+                    const uint32_t ka = st + cb * 16384 + (n & 511) * 16;
+                    const float d = r < L ? ex2(lamL - lam[r]) : 0.f;
+                    sts128(ka, scale_bf16x8(lds128(ka), d));
+                    if (kOut) {
+                        const uint32_t qa = ka + 8192;
+                        sts128(qa, scale_bf16x8(lds128(qa), ex2(lam[r])));
+                    }
+                }
+            }
+            if (MODE == 2 && kOut) {
+                // after G: Q <- diag(g) Q in place
+                for (int n = e; n < 1024; n += kEpi) {
+                    const int cb = n >> 9, r = (n & 511) >> 3;
+                    const uint32_t qa = st + 8192 + cb * 16384 + (n & 511) * 16;
+                    sts128(qa, scale_bf16x8(lds128(qa), ex2(lam[r])));
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            epi_sync();
+
             if constexpr (MODE != 2) {
                 if (e == 0) mbar_arrive(&sm->a_ready);
             } else {
-                // ---- T = (I + Lm)^-1, then T' = T diag(b), T'' = T diag(b g) in bf16
+                // ---- T = (I + Lm)^-1;  T diag(b), T diag(b g) as bf16 MMA operands
                 invert_unit_lower(Lm, Tm, Zs, e);
-                if (e < 64) {
-                    const int t = e;
-                    for (int j0 = 0; j0 < kC; j0 += 16) {
+                if (e < 128) {
+                    const int t = e >> 1, hh = e & 1;
+                    for (int g = 0; g < 2; ++g) {
+                        const int j0 = 32 * hh + 16 * g;
                         float v1[16], v2[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const float tv = Tm[t * kLmStride + j0 + j] * sm->bet[buf][j0 + j];
                             v1[j] = tv;
-                            v2[j] = tv * __expf(lam[j0 + j]);
+                            v2[j] = tv * ex2(lam[j0 + j]);
                         }
-                        st_row_bf16x16(sm_base + kOffTp, t, j0 >> 3, v1);
-                        st_row_bf16x16(sm_base + kOffTpp, t, j0 >> 3, v2);
+                        st_row_bf16x16(sb + Y::kTp, t, j0 >> 3, v1);
+                        st_row_bf16x16(sb + Y::kTpp, t, j0 >> 3, v2);
                     }
                 }
                 fence_async_smem();
                 epi_sync();
                 if (e == 0) mbar_arrive(&sm->tt_ready);
-                // ---- W epilogue: W^T row (d_k index e) -> bf16 MN-major tile row e
+                // ---- W^T (row = d_k index) -> bf16 tile [d_k][t] (MN-major B of S W^T)
                 mbar_wait(&sm->ut_done, par, abort, p.err);
                 epi_sync();
                 if (*abort) break;
                 tc_fence_after();
-                for (int t0c = 0; t0c < kC; t0c += 16) {
+                for (int g = 0; g < 2; ++g) {
+                    const int t0c = 32 * h + 16 * g;
                     float v[16];
-                    tmem_ld16(trow + kColW + t0c, v);
-                    st_row_bf16x16(sm_base + kOffW, e, t0c >> 3, v);
+                    tmem_ld16(tl + kColW + t0c, v);
+                    st_row_bf16x16(sb + Y::kW, row, t0c >> 3, v);
                 }
                 fence_async_smem();
                 tc_fence_before();
                 epi_sync();
                 if (e == 0) mbar_arrive(&sm->w_ready);
-                // ---- E epilogue: E^T = U^T - S W^T (row d_v = e), and E^T diag(dec)
+                // ---- E^T = U^T - S W^T (row = d_v index); E^T diag(dec)
                 mbar_wait(&sm->py_done, par, abort, p.err);
                 epi_sync();
                 if (*abort) break;
                 tc_fence_after();
-                {
-                    const float lamL = lam[kC - 1];
-                    for (int t0c = 0; t0c < kC; t0c += 16) {
-                        float y[16], uu[16], ev[16];
-                        if (kNeedV) tmem_ld16x2(trow + kColY + t0c, y, trow + kColU + t0c, uu);
-                        else tmem_ld16(trow + kColY + t0c, y);
-    #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int t = t0c + j;
-                            const float ex = (t < L) ? ((kNeedV ? uu[j] : 0.f) - y[j]) : 0.f;
-                            y[j] = ex;
-                            ev[j] = (t < L) ? ex * __expf(lamL - lam[t]) : 0.f;
-                        }
-                        st_row_bf16x16(sm_base + kOffE, e, t0c >> 3, y);
-                        st_row_bf16x16(sm_base + kOffEp, e, t0c >> 3, ev);
+                for (int g = 0; g < 2; ++g) {
+                    const int t0c = 32 * h + 16 * g;
+                    float y[16], uu[16], ev[16];
+                    if (kNeedV) tmem_ld16x2(tl + kColY + t0c, y, tl + kColU + t0c, uu);
+                    else tmem_ld16(tl + kColY + t0c, y);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int t = t0c + j;
+                        const float ex = (t < L) ? ((kNeedV ? uu[j] : 0.f) - y[j]) : 0.f;
+                        y[j] = ex;
+                        ev[j] = (t < L) ? ex * ex2(lamL - lam[t]) : 0.f;
                     }
+                    st_row_bf16x16(sb + Y::kE, row, t0c >> 3, y);
+                    st_row_bf16x16(sb + Y::kEp, row, t0c >> 3, ev);
                 }
                 fence_async_smem();
                 tc_fence_before();
@@ -616,83 +642,89 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 if (e == 0) mbar_arrive(&sm->e_ready);
             }
 
-            // ---- gates of the next chunk
-            if (c + 1 < nch && e < 64) load_gates<MODE>(p, sm, bh, tb, te, c + 1, buf ^ 1, e);
-            if (KIND == kLocal && MODE == 1 && e == 0) sm->gsum += lam[kC - 1];
+            // ---- prologue of the next chunk overlaps the products of this one
+            if (c + 1 < nch && !prep(c + 1)) break;
 
+            // ---- state: S <- g_{L-1} S + dS in registers; bf16 copy for the next chunk
             mbar_wait(&sm->mma2_done, par, abort, p.err);
             epi_sync();
             if (*abort) break;
             tc_fence_after();
-
-            // ---- outputs: o_t[e] for t < L
-            if (kOut) {
-                __nv_bfloat16 *orow = p.o + (o_row0 + t0) * kD + e;
-                for (int j0 = 0; j0 < kC; j0 += 16) {
-                    float pv[16], rv[16];
-                    tmem_ld16x2(trow + kColP + j0, pv, trow + kColR + j0, rv);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int t = j0 + j;
-                        if (t < L) {
-                            float val;
-                            if (MODE == 0) val = (pv[j] + rv[j]) / sm->den[t];
-                            else val = fmaf(__expf(lam[t]), pv[j], rv[j]);
-                            orow[(size_t)t * kD] = __float2bfloat16_rn(val);
-                        }
-                    }
-                }
-            }
-            if (MODE == 0) {
-                // z += sum_j phi(k_j)   (rows >= L were zeroed in the prep step)
-                const uint32_t kb = st + (e >> 6) * 16384;
-                const int ch = (e & 63) >> 3, wi = e & 7;
-                float zs = 0.f;
-                for (int j = 0; j < kC; ++j) {
-                    const uint32_t bits = lds_u16(kb + j * 128 + ((ch ^ (j & 7)) << 4) + wi * 2);
-                    zs += __uint_as_float(bits << 16);
-                }
-                sm->z[e] += zs;
-            }
-
-            // ---- state: bf16 copy for the next chunk's MMAs, next decay applied in TMEM
+            const bool last = (c + 1 == nch);
             {
-                const bool last = (c + 1 == nch);
-                const float gnext =
-                    (MODE == 0 || last) ? 1.f : __expf(sm->lam[buf ^ 1][kC - 1]);
-                float *dst = nullptr;
-                if (last && p.s_out && (!p.out_last_only || seg == p.nseg - 1))
-                    dst = p.s_out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
-                          (size_t)e * kD;
-                for (int c0 = 0; c0 < kD; c0 += 16) {
+                const float gC = (MODE == 0) ? 1.f : ex2(lamL);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
                     float v[16];
-                    tmem_ld16(trow + kColS + c0, v);
-                    if (dst) {
+                    tmem_ld16(tl + kColDS + 64 * h + 16 * g, v);
 #pragma unroll
-                        for (int j = 0; j < 16; j += 4)
-                            *reinterpret_cast<float4 *>(dst + c0 + j) =
-                                make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                    for (int j = 0; j < 16; ++j) Sr[16 * g + j] = fmaf(gC, Sr[16 * g + j], v[j]);
+                    if (!last) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
+                }
+                if (MODE == 0 && e < kD) {
+                    // z += sum_j phi(k_j)   (rows >= L of phi(K) were zeroed)
+                    const uint32_t kb = st + (e >> 6) * 16384;
+                    const int ch = (e & 63) >> 3, wi = e & 7;
+                    float zs = 0.f;
+                    for (int j = 0; j < kC; ++j) {
+                        const uint32_t bits =
+                            lds_u16(kb + j * 128 + ((ch ^ (j & 7)) << 4) + wi * 2);
+                        zs += __uint_as_float(bits << 16);
                     }
-                    if (!last) {
-                        st_row_bf16x16(sbf + (c0 >> 6) * 16384, e, (c0 & 63) >> 3, v);
-                        if (MODE != 0) {
+                    sm->z[e] += zs;
+                }
+                if (KIND == kLocal && MODE == 1 && e == 0) sm->gsum += lamL;
+                if (last) {
+                    const bool write = p.s_out && (!p.out_last_only || seg == p.nseg - 1);
+                    if (write) {
+                        float *dst = p.s_out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
+                                     (size_t)row * kD + 64 * h;
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) v[j] *= gnext;
-                            tmem_st16(trow + kColS + c0, v);
+                        for (int j = 0; j < 64; j += 4)
+                            *reinterpret_cast<float4 *>(dst + j) =
+                                make_float4(Sr[j], Sr[j + 1], Sr[j + 2], Sr[j + 3]);
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            epi_sync();
+            if (e == 0) {
+                mbar_arrive(&sm->s_ready);
+                mbar_arrive(&sm->empty[s]);
+            }
+            if (last) {
+                if (MODE == 0 && e < kD && p.z_out && (!p.out_last_only || seg == p.nseg - 1))
+                    p.z_out[(size_t)seg * p.z_out_seg + (size_t)bh * kD + e] = sm->z[e];
+                if (KIND == kLocal && MODE == 1 && e == 0 && p.gam_out)
+                    p.gam_out[(size_t)seg * p.BH + bh] = ex2(sm->gsum);
+            }
+
+            // ---- outputs: row t of O (M=64 layout: lane (t % 16) + 32 (t / 16)), half h
+            if (kOut) {
+                const int t = 16 * q + lane;
+                const bool has = lane < 16 && t < L;
+                float inv = 1.f;
+                if (MODE == 0 && has)
+                    inv = 1.f / (sm->part[0][t] + sm->part[1][t] + sm->part[2][t] + sm->part[3][t]);
+                __nv_bfloat16 *orow = p.o + (o_row0 + t0 + t) * kD + 64 * h;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    float v[16];
+                    tmem_ld16(tl + kColO + 64 * h + 16 * g, v);
+                    if (has) {
+#pragma unroll
+                        for (int k = 0; k < 2; ++k) {
+                            uint4 w;
+                            w.x = pack_bf16x2(v[8 * k + 0] * inv, v[8 * k + 1] * inv);
+                            w.y = pack_bf16x2(v[8 * k + 2] * inv, v[8 * k + 3] * inv);
+                            w.z = pack_bf16x2(v[8 * k + 4] * inv, v[8 * k + 5] * inv);
+                            w.w = pack_bf16x2(v[8 * k + 6] * inv, v[8 * k + 7] * inv);
+                            *reinterpret_cast<uint4 *>(orow + 16 * g + 8 * k) = w;
                         }
                     }
                 }
-                if (last && MODE == 0 && p.z_out && (!p.out_last_only || seg == p.nseg - 1))
-                    p.z_out[(size_t)seg * p.z_out_seg + (size_t)bh * kD + e] = sm->z[e];
-                if (last && KIND == kLocal && MODE == 1 && e == 0 && p.gam_out)
-                    p.gam_out[(size_t)seg * p.BH + bh] = __expf(sm->gsum);
-                fence_async_smem();
                 tc_fence_before();
-                epi_sync();
-                if (e == 0) {
-                    mbar_arrive(&sm->s_ready);
-                    mbar_arrive(&sm->empty[s]);
-                }
             }
         }
     }
@@ -811,7 +843,7 @@ size_t workspace_floats(int mode, int BH, const Plan &pl) {
 template <int MODE, int KIND>
 cudaError_t launch_kind(const TcParams &p, int grid, cudaStream_t stream) {
     auto kern = prefill_tc_kernel<MODE, KIND>;
-    const uint32_t bytes = smem_bytes<MODE>();
+    const uint32_t bytes = Lay<MODE>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, bytes, stream>>>(p);
