@@ -119,6 +119,26 @@ size_t la_prefill_workspace_size(la_mode_t mode, la_dtype_t dtype, int B, int H,
                                  int d_v, int chunk);
 
 /*
+ * la_prefill_noalloc -- la_prefill for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is an interface for such callers, e.g. code that
+ * runs inside another framework's memory pool (a cudaMalloc there bypasses the pool)
+ * or a process that reserves all device memory at start-up.  It takes the same
+ * arguments as la_prefill except the workspace, which it takes from a 24 MiB array
+ * that the library keeps in device memory (every GPU that loads the library holds it
+ * until exit).  It allocates nothing and calls no allocating routine.
+ *   - Returns LA_ERR_UNSUPPORTED when la_prefill_workspace_size() for these sizes
+ *     exceeds 24 MiB; nothing is launched then.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current); make that first call before any stream capture on the device.
+ *   - All calls share the array and it keeps the last call's contents (no result
+ *     depends on them).  Calls that overlap on the GPU race on it: serialise them.
+ */
+la_status_t la_prefill_noalloc(la_mode_t mode, la_dtype_t dtype, int B, int H, int T, int d_k,
+                               int d_v, const void *q, const void *k, const void *v,
+                               const float *gate, const float *beta, float *state, float *z,
+                               void *o, int chunk, unsigned flags, void *stream);
+
+/*
  * la_decode_step -- one token of the recurrent form ([three forms] "recurrent form",
  * [decay/gates], [delta rule]) for N independent sequences, updating the state in place:
  * the per-token cost is O(d_k d_v) and independent of how many tokens came before.
