@@ -235,8 +235,9 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------
 
 class PrefillCase:
-    def __init__(self, la, w: W.Workload, device, rank):
+    def __init__(self, la, w: W.Workload, device, rank, workspace="auto"):
         self.la, self.w, self.device = la, w, device
+        self.ws = workspace
         wr = W.variant(w, seed=w.seed + 1000 * rank)
         self.inp = W.prefill_inputs(wr, device=device)
         self.state = torch.empty(w.B, w.H, w.dv, w.dk, device=device)
@@ -250,7 +251,7 @@ class PrefillCase:
         i = self.inp
         self.la.prefill(i["q"], i["k"], i["v"], mode=self.w.mode, gate=i["gate"], beta=i["beta"],
                         state=self.state, z=self.z, o=self.o, chunk=self.w.chunk,
-                        init_state=False)
+                        init_state=False, workspace=self.ws)
 
     def e2e_setup(self):
         pin = lambda t: None if t is None else t.to("cpu").pin_memory()
@@ -270,7 +271,8 @@ class PrefillCase:
             if v is not None:
                 d[k].copy_(v, non_blocking=True)
         self.la.prefill(d["q"], d["k"], d["v"], mode=self.w.mode, gate=d["gate"], beta=d["beta"],
-                        state=self.state, z=self.z, o=self.o, chunk=self.w.chunk, init_state=False)
+                        state=self.state, z=self.z, o=self.o, chunk=self.w.chunk, init_state=False,
+                        workspace=self.ws)
         self.h_o.copy_(self.o, non_blocking=True)
         self.h_state.copy_(self.state, non_blocking=True)
         if self.h_z is not None:
@@ -363,7 +365,7 @@ class _Null:
 def measure(la, name, args, dist, device, rank, world, flush, with_e2e, sampler=None):
     w = W.CONFIGS[name]
     case = (DecodeCase(la, w, device, rank, args.warmup + args.steps) if w.decode
-            else PrefillCase(la, w, device, rank))
+            else PrefillCase(la, w, device, rank, None if args.no_workspace else "auto"))
     ms, launches = time_steps(case, args.steps, args.warmup, dist, device, flush, sampler=sampler)
     la.check_status()
     total_ms = max_over_ranks(dist, sum(ms), device)
@@ -494,6 +496,8 @@ def main():
     ap.add_argument("--extras", type=int, default=-1,
                     help="1: also measure the other workloads (default: on at N=1)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-workspace", action="store_true",
+                    help="prefill without the segment workspace (one kernel per call)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -60,12 +60,13 @@ constexpr int kEpi = 256;      // epilogue threads (warps 2-9)
 constexpr uint32_t kTmemCols = 512;
 // TMEM column map
 constexpr uint32_t kColDS = 0, kColG = 128, kColU = 192, kColW = 256, kColY = 320, kColO = 384;
+constexpr uint32_t kColP = 256;   // mode 1: Q S^T kept apart from A V (M=64, 128 columns)
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum Kind { kOutput = 0, kLocal = 1, kTransition = 2 };
 
 struct TcParams {
-    CUtensorMap tq, tk, tv;      // [BH][T][128] bf16, box 64 x 64
+    CUtensorMap tq, tk, tv, to;  // [BH][T][128] bf16, box 64 x 64 (to: output, stores)
     const float *gate;           // [BH][T] or nullptr
     const float *beta;           // [BH][T] (mode 2)
     __nv_bfloat16 *o;            // [BH][T][128]
@@ -113,7 +114,8 @@ struct Lay {
     static constexpr uint32_t kTpp = kTp + 8192;       // 8 KB  T diag(b g)    (mode 2)
     static constexpr uint32_t kX = kTpp + 8192;        // 48 KB E | E' | W  or  Lm | Tm | Zs
     static constexpr uint32_t kE = kX, kEp = kX + 16384, kW = kX + 32768;
-    static constexpr uint32_t kSmall = MODE == 2 ? kX + 49152 : kA + 8192;
+    static constexpr uint32_t kOst = MODE == 2 ? kX + 49152 : kA + 8192;   // 16 KB O staging
+    static constexpr uint32_t kSmall = kOst + 16384;
     static constexpr uint32_t kBytes = kSmall + sizeof(Small);
 };
 constexpr uint32_t kLmStride = 65;
@@ -167,14 +169,29 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 w, float s) {
     return w;
 }
 
-// Gates of chunk c into parity buffer `buf`: log2 prefix and beta (64 threads, e < 64).
+// Raw gate a_t and beta_t of token `e` of chunk c (64 threads, e < 64), fetched a chunk
+// ahead of use so that the global-load latency overlaps the previous chunk's epilogue.
+struct GateRaw {
+    float a, b;
+};
 template <int MODE>
-__device__ __forceinline__ void load_gates(const TcParams &p, Small *sm, int bh, int tb, int te,
-                                           int c, int buf, int e) {
+__device__ __forceinline__ GateRaw fetch_gates(const TcParams &p, int bh, int tb, int te, int c,
+                                               int e) {
+    GateRaw r{1.f, 0.f};
     const int t0 = tb + kC * c;
     const int L = min(kC, te - t0);
-    float g = 0.f;
-    if (MODE != 0 && p.gate && e < L) g = lg2(fmaxf(p.gate[(size_t)bh * p.T + t0 + e], FLT_MIN));
+    if (MODE != 0 && p.gate && e < L) r.a = p.gate[(size_t)bh * p.T + t0 + e];
+    if (MODE == 2 && e < L) r.b = p.beta[(size_t)bh * p.T + t0 + e];
+    return r;
+}
+
+// Gates of chunk c into parity buffer `buf`: log2 prefix and beta (64 threads, e < 64).
+template <int MODE>
+__device__ __forceinline__ void load_gates(const TcParams &p, Small *sm, int tb, int te, int c,
+                                           int buf, int e, GateRaw raw) {
+    const int t0 = tb + kC * c;
+    const int L = min(kC, te - t0);
+    float g = (MODE != 0 && e < L) ? lg2(fmaxf(raw.a, FLT_MIN)) : 0.f;
     const int lane = e & 31;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -185,9 +202,25 @@ __device__ __forceinline__ void load_gates(const TcParams &p, Small *sm, int bh,
     named_sync(2, 64);
     if (e >= 32) g += sm->scan_tmp[0];
     sm->lam[buf][e] = g;
-    sm->bet[buf][e] = (MODE == 2 && e < L) ? p.beta[(size_t)bh * p.T + t0 + e] : 0.f;
+    sm->bet[buf][e] = (MODE == 2 && e < L) ? raw.b : 0.f;
     if (e == 0) sm->len[buf] = L;
     named_sync(2, 64);
+    (void)p;
+}
+
+// phi(x) = elu(x) + 1 = max(x, 0) + exp(min(x, 0)) on a packed pair of bf16, in bf16x2
+// arithmetic (the inputs and results are bf16 MMA operands).
+__device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
+    uint32_t r;
+    asm("{\n\t.reg .b32 lo, hi, ex;\n\t"
+        "min.bf16x2 lo, %1, %2;\n\t"
+        "max.bf16x2 hi, %1, %2;\n\t"
+        "mul.rn.bf16x2 lo, lo, %3;\n\t"
+        "ex2.approx.ftz.bf16x2 ex, lo;\n\t"
+        "add.rn.bf16x2 %0, hi, ex;\n\t}"
+        : "=r"(r)
+        : "r"(x), "r"(0u), "r"(0x3FB93FB9u));   // bf16x2 of log2(e) = 1.4453 (0x3FB9)
+    return r;
 }
 
 // 64x64 unit lower-triangular inverse T = (I + Lm)^-1 by 16x16 blocks (256 threads).
@@ -390,15 +423,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     tc_fence_after();
                 }
                 if (kOut) {
-                    // O = Q~ S^T (+) A V  or  A E     (M=64, N=128)
+                    // O = Q~ S^T (+) A V  or  A E     (M=64, N=128); mode 1 keeps Q S^T
+                    // in its own accumulator P and applies diag(g) in the output epilogue
+                    const uint32_t dq = (MODE == 1) ? kColP : kColO;
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16_ss(tm + kColO, dk(st + 8192 + off), dk(sbf + off), id_o1, ks > 0);
+                        mma_bf16_ss(tm + dq, dk(st + 8192 + off), dk(sbf + off), id_o1, ks > 0);
                     }
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint64_t b2 = (MODE == 2) ? dk(et + ks * 32)
                                                         : dmn(st + 32768 + ks * 2048, 8192);
-                        mma_bf16_ss(tm + kColO, dk(at + ks * 32), b2, id_o2, true);
+                        mma_bf16_ss(tm + kColO, dk(at + ks * 32), b2, id_o2, MODE != 1 || ks > 0);
                     }
                 }
                 // dS = V^T K~ (modes 0/1) or (E^T diag dec) K (mode 2)   (M=128, N=128)
@@ -424,7 +459,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         float *Lm = reinterpret_cast<float *>(smem_raw + Y::kX);
         float *Tm = Lm + 64 * kLmStride;
         float *Zs = Tm + 64 * kLmStride;
-        const size_t o_row0 = (size_t)bh * p.T;
 
         // ---- initial state: this thread's half row of S in registers, bf16 copy in smem
         float Sr[64];
@@ -451,33 +485,37 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
 
         // ---- chunk prologue: gates, phi (mode 0); releases G's inputs to the MMA
-        auto prep = [&](int c) -> bool {
+        auto prep = [&](int c, GateRaw raw) -> bool {
             const int s = c % NST, u = c / NST;
-            if (e < 64) load_gates<MODE>(p, sm, bh, tb, te, c, c & 1, e);
+            if (e < 64) load_gates<MODE>(p, sm, tb, te, c, c & 1, e, raw);
             mbar_wait(&sm->full[s], u & 1, abort, p.err);
             epi_sync();
             if (*abort) return false;
             if (MODE == 0) {
                 const uint32_t st = sb + s * Y::kStage;
                 const int L = sm->len[c & 1];
-                const int nreg = kOut ? 4 : 2;
-                for (int n = e; n < nreg * 512; n += kEpi) {
-                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);   // 0,2 = K; 1,3 = Q
-                    const int r = (n & 511) >> 3;
-                    const uint32_t a = st + region * 8192 + (n & 511) * 16;
-                    uint4 w;
-                    if ((region & 1) == 0 && r >= L) {
-                        w = make_uint4(0, 0, 0, 0);
-                    } else {
-                        w = lds128(a);
-                        uint32_t *wd = reinterpret_cast<uint32_t *>(&w);
+                constexpr int kIt = (kOut ? 4 : 2) * 512 / kEpi;   // chunks per thread
+                uint4 w[kIt];
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const float2 f = unpack_bf16x2(wd[k]);
-                            wd[k] = pack_bf16x2(phi_fast(f.x), phi_fast(f.y));
-                        }
+                for (int it = 0; it < kIt; ++it) {
+                    const int n = e + kEpi * it;
+                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);   // 0,2 = K; 1,3 = Q
+                    w[it] = lds128(st + region * 8192 + (n & 511) * 16);
+                }
+#pragma unroll
+                for (int it = 0; it < kIt; ++it) {
+                    const int n = e + kEpi * it;
+                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);
+                    const int r = (n & 511) >> 3;
+                    if ((region & 1) == 0 && r >= L) {
+                        w[it] = make_uint4(0, 0, 0, 0);
+                    } else {
+                        w[it].x = phi_bf16x2(w[it].x);
+                        w[it].y = phi_bf16x2(w[it].y);
+                        w[it].z = phi_bf16x2(w[it].z);
+                        w[it].w = phi_bf16x2(w[it].w);
                     }
-                    sts128(a, w);
+                    sts128(st + region * 8192 + (n & 511) * 16, w[it]);
                 }
                 fence_async_smem();
             }
@@ -486,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             return true;
         };
 
-        bool ok = prep(0);
+        bool ok = prep(0, e < 64 ? fetch_gates<MODE>(p, bh, tb, te, 0, e) : GateRaw{1.f, 0.f});
         for (int c = 0; c < nch && ok; ++c) {
             const int s = c % NST, buf = c & 1;
             const uint32_t par = c & 1;
@@ -495,6 +533,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             const int L = sm->len[buf];
             const float *lam = sm->lam[buf];
             const float lamL = lam[kC - 1];
+            // gates of the next chunk: issue the global loads now, use them in its prologue
+            GateRaw next_raw{1.f, 0.f};
+            if (c + 1 < nch && e < 64) next_raw = fetch_gates<MODE>(p, bh, tb, te, c + 1, e);
 
             // ---- A-epilogue: masks and decays of G; operand scaling
             if (kNeedG) {
@@ -506,35 +547,31 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             if (q >= 2 && kOut) {
                 // rows i of Q K^T -> A tile, columns j in [32h, 32h + 32)
                 const int i = row - 64;
+                float v[32];
+                tmem_ld32(tl + kColG + 32 * h, v);
+                const float li = lam[i];
                 float rs = 0.f;
-                for (int g = 0; g < 2; ++g) {
-                    const int j0 = 32 * h + 16 * g;
-                    float v[16];
-                    tmem_ld16(tl + kColG + j0, v);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int jj = j0 + j;
-                        float a = 0.f;
-                        if (jj <= i) a = (MODE == 0) ? v[j] : v[j] * ex2(lam[i] - lam[jj]);
-                        v[j] = __bfloat162float(__float2bfloat16_rn(a));
-                        rs += v[j];
-                    }
-                    st_row_bf16x16(sb + Y::kA, i, j0 >> 3, v);
+                for (int j = 0; j < 32; ++j) {
+                    const int jj = 32 * h + j;
+                    float a = 0.f;
+                    if (jj <= i) a = (MODE == 0) ? v[j] : v[j] * ex2(li - lam[jj]);
+                    v[j] = __bfloat162float(__float2bfloat16_rn(a));
+                    rs += v[j];
                 }
+                st_row_bf16x16(sb + Y::kA, i, 4 * h, v);
+                st_row_bf16x16(sb + Y::kA, i, 4 * h + 2, v + 16);
                 if (MODE == 0) sm->part[h][i] = rs;
             } else if (q < 2 && MODE == 2) {
                 // rows r of K K^T -> Lm (strictly lower), columns j in [32h, 32h + 32)
                 const int r = row;
-                const float br = sm->bet[buf][r];
-                for (int g = 0; g < 2; ++g) {
-                    const int j0 = 32 * h + 16 * g;
-                    float v[16];
-                    tmem_ld16(tl + kColG + j0, v);
+                const float br = sm->bet[buf][r], lr = lam[r];
+                float v[32];
+                tmem_ld32(tl + kColG + 32 * h, v);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int jj = j0 + j;
-                        Lm[r * kLmStride + jj] = (jj < r) ? br * ex2(lam[r] - lam[jj]) * v[j] : 0.f;
-                    }
+                for (int j = 0; j < 32; ++j) {
+                    const int jj = 32 * h + j;
+                    Lm[r * kLmStride + jj] = (jj < r) ? br * ex2(lr - lam[jj]) * v[j] : 0.f;
                 }
             } else if (q < 2 && MODE == 0 && kOut) {
                 // phi(q_r) . z over d_k half h
@@ -554,24 +591,35 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 sm->part[2 + h][r] = qz;
             }
             if (MODE == 1) {
-                // after G: Q <- diag(g) Q (output kinds) and K <- diag(dec) K, in place
-                for (int n = e; n < 1024; n += kEpi) {
-                    const int cb = n >> 9, r = (n & 511) >> 3;
-                    const uint32_t ka = st + cb * 16384 + (n & 511) * 16;
-                    const float d = r < L ? ex2(lamL - lam[r]) : 0.f;
-                    sts128(ka, scale_bf16x8(lds128(ka), d));
-                    if (kOut) {
-                        const uint32_t qa = ka + 8192;
-                        sts128(qa, scale_bf16x8(lds128(qa), ex2(lam[r])));
-                    }
+                // after G: K <- diag(dec) K in place (operand of dS); each thread owns 4
+                // chunks, loaded together before scaling
+                uint4 wk[4];
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int n = e + kEpi * it;
+                    wk[it] = lds128(st + (n >> 9) * 16384 + (n & 511) * 16);
+                }
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int n = e + kEpi * it;
+                    const int r = (n & 511) >> 3;
+                    sts128(st + (n >> 9) * 16384 + (n & 511) * 16,
+                           scale_bf16x8(wk[it], r < L ? ex2(lamL - lam[r]) : 0.f));
                 }
             }
             if (MODE == 2 && kOut) {
                 // after G: Q <- diag(g) Q in place
-                for (int n = e; n < 1024; n += kEpi) {
-                    const int cb = n >> 9, r = (n & 511) >> 3;
-                    const uint32_t qa = st + 8192 + cb * 16384 + (n & 511) * 16;
-                    sts128(qa, scale_bf16x8(lds128(qa), ex2(lam[r])));
+                uint4 wq[4];
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int n = e + kEpi * it;
+                    wq[it] = lds128(st + 8192 + (n >> 9) * 16384 + (n & 511) * 16);
+                }
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int n = e + kEpi * it;
+                    sts128(st + 8192 + (n >> 9) * 16384 + (n & 511) * 16,
+                           scale_bf16x8(wq[it], ex2(lam[(n & 511) >> 3])));
                 }
             }
             fence_async_smem();
@@ -606,11 +654,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 epi_sync();
                 if (*abort) break;
                 tc_fence_after();
-                for (int g = 0; g < 2; ++g) {
-                    const int t0c = 32 * h + 16 * g;
-                    float v[16];
-                    tmem_ld16(tl + kColW + t0c, v);
-                    st_row_bf16x16(sb + Y::kW, row, t0c >> 3, v);
+                {
+                    float v[32];
+                    tmem_ld32(tl + kColW + 32 * h, v);
+                    st_row_bf16x16(sb + Y::kW, row, 4 * h, v);
+                    st_row_bf16x16(sb + Y::kW, row, 4 * h + 2, v + 16);
                 }
                 fence_async_smem();
                 tc_fence_before();
@@ -621,20 +669,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 epi_sync();
                 if (*abort) break;
                 tc_fence_after();
-                for (int g = 0; g < 2; ++g) {
-                    const int t0c = 32 * h + 16 * g;
-                    float y[16], uu[16], ev[16];
-                    if (kNeedV) tmem_ld16x2(tl + kColY + t0c, y, tl + kColU + t0c, uu);
-                    else tmem_ld16(tl + kColY + t0c, y);
+                {
+                    float y[32], uu[32], ev[32];
+                    tmem_ld32(tl + kColY + 32 * h, y);
+                    if (kNeedV) tmem_ld32(tl + kColU + 32 * h, uu);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int t = t0c + j;
+                    for (int j = 0; j < 32; ++j) {
+                        const int t = 32 * h + j;
                         const float ex = (t < L) ? ((kNeedV ? uu[j] : 0.f) - y[j]) : 0.f;
                         y[j] = ex;
                         ev[j] = (t < L) ? ex * ex2(lamL - lam[t]) : 0.f;
                     }
-                    st_row_bf16x16(sb + Y::kE, row, t0c >> 3, y);
-                    st_row_bf16x16(sb + Y::kEp, row, t0c >> 3, ev);
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        st_row_bf16x16(sb + Y::kE, row, 4 * h + 2 * g, y + 16 * g);
+                        st_row_bf16x16(sb + Y::kEp, row, 4 * h + 2 * g, ev + 16 * g);
+                    }
                 }
                 fence_async_smem();
                 tc_fence_before();
@@ -643,23 +693,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             }
 
             // ---- prologue of the next chunk overlaps the products of this one
-            if (c + 1 < nch && !prep(c + 1)) break;
+            if (c + 1 < nch && !prep(c + 1, next_raw)) break;
 
             // ---- state: S <- g_{L-1} S + dS in registers; bf16 copy for the next chunk
             mbar_wait(&sm->mma2_done, par, abort, p.err);
+            if (kOut && e == 0) tma_store_wait_read<0>();   // O staging free again
             epi_sync();
             if (*abort) break;
             tc_fence_after();
             const bool last = (c + 1 == nch);
             {
                 const float gC = (MODE == 0) ? 1.f : ex2(lamL);
+                {
+                    float v[64];
+                    tmem_ld64(tl + kColDS + 64 * h, v);
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float v[16];
-                    tmem_ld16(tl + kColDS + 64 * h + 16 * g, v);
+                    for (int j = 0; j < 64; ++j) Sr[j] = fmaf(gC, Sr[j], v[j]);
+                }
+                if (!last) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) Sr[16 * g + j] = fmaf(gC, Sr[16 * g + j], v[j]);
-                    if (!last) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
+                    for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
                 }
                 if (MODE == 0 && e < kD) {
                     // z += sum_j phi(k_j)   (rows >= L of phi(K) were zeroed)
@@ -700,34 +753,47 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     p.gam_out[(size_t)seg * p.BH + bh] = ex2(sm->gsum);
             }
 
-            // ---- outputs: row t of O (M=64 layout: lane (t % 16) + 32 (t / 16)), half h
+            // ---- outputs: row t of O (M=64 layout: lane (t % 16) + 32 (t / 16)), half h,
+            // staged as bf16 in shared memory and written by two TMA stores (rows past the
+            // end of the sequence are clipped by the tensor map)
             if (kOut) {
                 const int t = 16 * q + lane;
                 const bool has = lane < 16 && t < L;
-                float inv = 1.f;
+                float scale = 1.f;
                 if (MODE == 0 && has)
-                    inv = 1.f / (sm->part[0][t] + sm->part[1][t] + sm->part[2][t] + sm->part[3][t]);
-                __nv_bfloat16 *orow = p.o + (o_row0 + t0 + t) * kD + 64 * h;
+                    scale = 1.f / (sm->part[0][t] + sm->part[1][t] + sm->part[2][t] + sm->part[3][t]);
+                if (MODE == 1 && has) scale = ex2(lam[t]);
+                const uint32_t ost = sb + Y::kOst + h * 8192;
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float v[16];
-                    tmem_ld16(tl + kColO + 64 * h + 16 * g, v);
+                for (int sub = 0; sub < 2; ++sub) {
+                    float v[32];
+                    tmem_ld32(tl + kColO + 64 * h + 32 * sub, v);
+                    if (MODE == 1) {
+                        float pq[32];
+                        tmem_ld32(tl + kColP + 64 * h + 32 * sub, pq);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = fmaf(scale, pq[j], v[j]);
+                    } else if (MODE == 0) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] *= scale;
+                    }
                     if (has) {
-#pragma unroll
-                        for (int k = 0; k < 2; ++k) {
-                            uint4 w;
-                            w.x = pack_bf16x2(v[8 * k + 0] * inv, v[8 * k + 1] * inv);
-                            w.y = pack_bf16x2(v[8 * k + 2] * inv, v[8 * k + 3] * inv);
-                            w.z = pack_bf16x2(v[8 * k + 4] * inv, v[8 * k + 5] * inv);
-                            w.w = pack_bf16x2(v[8 * k + 6] * inv, v[8 * k + 7] * inv);
-                            *reinterpret_cast<uint4 *>(orow + 16 * g + 8 * k) = w;
-                        }
+                        st_row_bf16x16(ost, t, 4 * sub, v);
+                        st_row_bf16x16(ost, t, 4 * sub + 2, v + 16);
                     }
                 }
+                fence_async_smem();
                 tc_fence_before();
+                epi_sync();
+                if (e == 0) {
+                    tma_store_3d(&p.to, sb + Y::kOst, 0, t0, bh);
+                    tma_store_3d(&p.to, sb + Y::kOst + 8192, 64, t0, bh);
+                    tma_store_commit();
+                }
             }
         }
     }
+    if (kOut && warp >= 2 && threadIdx.x == 64) tma_store_wait_all<0>();   // outputs landed
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -956,6 +1022,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t work
         !make_tmap_3d(&p.tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, a.T, BH, row_pitch,
                       head_pitch, 64, kC, true) ||
         !make_tmap_3d(&p.tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, a.T, BH, row_pitch,
+                      head_pitch, 64, kC, true) ||
+        !make_tmap_3d(&p.to, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, a.T, BH, row_pitch,
                       head_pitch, 64, kC, true))
         return cudaErrorInvalidValue;
     p.gate = a.gate;
