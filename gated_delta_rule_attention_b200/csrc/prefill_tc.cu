@@ -135,8 +135,6 @@ __device__ __forceinline__ float lg2(float x) {
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-// phi(x) = elu(x) + 1 = x + 1 for x > 0, e^x otherwise
-__device__ __forceinline__ float phi_fast(float x) { return x > 0.f ? x + 1.f : ex2(x * kLog2e); }
 
 // Bounded wait that ignores the abort flag (used to drain in-flight work on exit).
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
@@ -223,6 +221,48 @@ __device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
     return r;
 }
 
+// ---- warp-level tf32 products for the 16x16 blocks of the triangular inverse
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// acc (16x16 fp32, two m16n8 fragments) += A (16x16) * B (16x16); A, B fp32 in shared
+// memory with row strides lda, ldb (elements).
+__device__ __forceinline__ void mma16x16x16_tf32(float (&acc)[2][4], const float *A, int lda,
+                                                 const float *B, int ldb, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+        const uint32_t a0 = to_tf32(A[g * lda + 8 * kk + t]);
+        const uint32_t a1 = to_tf32(A[(g + 8) * lda + 8 * kk + t]);
+        const uint32_t a2 = to_tf32(A[g * lda + 8 * kk + t + 4]);
+        const uint32_t a3 = to_tf32(A[(g + 8) * lda + 8 * kk + t + 4]);
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+            const uint32_t b0 = to_tf32(B[(8 * kk + t) * ldb + 8 * nh + g]);
+            const uint32_t b1 = to_tf32(B[(8 * kk + t + 4) * ldb + 8 * nh + g]);
+            asm volatile(
+                "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+                "{%8,%9}, {%0,%1,%2,%3};"
+                : "+f"(acc[nh][0]), "+f"(acc[nh][1]), "+f"(acc[nh][2]), "+f"(acc[nh][3])
+                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+}
+// C (16x16, row stride ldc) = s * acc
+__device__ __forceinline__ void store16_tile(const float (&acc)[2][4], float *C, int ldc, int lane,
+                                             float s) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        C[g * ldc + 8 * nh + 2 * t] = s * acc[nh][0];
+        C[g * ldc + 8 * nh + 2 * t + 1] = s * acc[nh][1];
+        C[(g + 8) * ldc + 8 * nh + 2 * t] = s * acc[nh][2];
+        C[(g + 8) * ldc + 8 * nh + 2 * t + 1] = s * acc[nh][3];
+    }
+}
+
 // 64x64 unit lower-triangular inverse T = (I + Lm)^-1 by 16x16 blocks (256 threads).
 __device__ void invert_unit_lower(const float *Lm, float *Tm, float *Zs, int e) {
     constexpr int S = kLmStride;
@@ -252,30 +292,23 @@ __device__ void invert_unit_lower(const float *Lm, float *Tm, float *Zs, int e) 
         }
     }
     epi_sync();
+    // Off-diagonal blocks, by distance d = i - j:  T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj.
+    // Each block is one warp's job on the legacy warp-level tensor-core path (tf32
+    // m16n8k8, fp32 accumulate): the products are 16x16x16, too small for tcgen05.
+    const int w = e >> 5, lane = e & 31;
     for (int d = 1; d < 4; ++d) {
-        const int outs = (4 - d) * 256;
-        for (int idx = e; idx < outs; idx += kEpi) {
-            const int blk = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
-            const int bi = blk + d, bj = blk;
-            float z0 = 0.f, z1 = 0.f;
-            for (int k = 16 * bj; k < 16 * bi; k += 2) {
-                z0 = fmaf(Lm[(16 * bi + r) * S + k], Tm[k * S + 16 * bj + cc], z0);
-                z1 = fmaf(Lm[(16 * bi + r) * S + k + 1], Tm[(k + 1) * S + 16 * bj + cc], z1);
-            }
-            Zs[blk * 272 + r * 17 + cc] = z0 + z1;
-        }
-        epi_sync();
-        for (int idx = e; idx < outs; idx += kEpi) {
-            const int blk = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
-            const int bi = blk + d, bj = blk;
-            float t0 = 0.f, t1 = 0.f;
-#pragma unroll
-            for (int m = 0; m < 16; m += 2) {
-                t0 = fmaf(Tm[(16 * bi + r) * S + 16 * bi + m], Zs[blk * 272 + m * 17 + cc], t0);
-                t1 = fmaf(Tm[(16 * bi + r) * S + 16 * bi + m + 1], Zs[blk * 272 + (m + 1) * 17 + cc],
-                          t1);
-            }
-            Tm[(16 * bi + r) * S + 16 * bj + cc] = -(t0 + t1);
+        if (w < 4 - d) {
+            const int bi = w + d, bj = w;
+            float acc[2][4] = {};
+            for (int k = bj; k < bi; ++k)
+                mma16x16x16_tf32(acc, Lm + (16 * bi) * S + 16 * k, S, Tm + (16 * k) * S + 16 * bj, S,
+                                 lane);
+            float *Z = Zs + w * 272;
+            store16_tile(acc, Z, 17, lane, 1.f);
+            __syncwarp();
+            float acc2[2][4] = {};
+            mma16x16x16_tf32(acc2, Tm + (16 * bi) * S + 16 * bi, S, Z, 17, lane);
+            store16_tile(acc2, Tm + (16 * bi) * S + 16 * bj, S, lane, -1.f);
         }
         epi_sync();
     }
@@ -802,6 +835,450 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     }
 }
 
+// ------------------------------------------------------------------ modes 0 / 1
+// A software-pipelined variant for the two modes without the delta-rule solve.  The
+// epilogue of iteration c forms the A tile of chunk c+1 while the tensor core computes
+// the outputs and state product of chunk c; the MMA issuer forms Q K^T of chunk c+1
+// before the products of chunk c.  G and the A tile are double-buffered by chunk
+// parity, gate buffers by chunk mod 4, and every hand-off is ordered so that no
+// mbarrier can complete two phases ahead of its waiter.
+struct Small01 {
+    uint64_t full[3], empty[3];
+    uint64_t prep_done, g_done, a_ready, mma2_done, s_ready, fin;
+    uint32_t tmem_base;
+    int abort;
+    int len[4];
+    float lam[4][kC];      // in-chunk inclusive prefix of log2(a), chunk mod 4
+    float part[2][4][kC];  // mode 0: row-sum halves and phi(q).z halves, chunk parity
+    float z[2][kD];        // mode 0: z after chunk j in z[j & 1] (z_in in z[1])
+    float scan_tmp[2];
+    float gsum;
+};
+struct Lay01 {
+    static constexpr int kStages = 3;
+    static constexpr uint32_t kStage = 49152;
+    static constexpr uint32_t kSbf = kStages * kStage;   // 32 KB
+    static constexpr uint32_t kA = kSbf + 32768;          // 2 x 8 KB
+    static constexpr uint32_t kOst = kA + 16384;          // 16 KB
+    static constexpr uint32_t kSmall = kOst + 16384;
+    static constexpr uint32_t kBytes = kSmall + sizeof(Small01);
+};
+constexpr uint32_t kColG2 = 128;   // two 64-column G buffers: 128, 192
+
+__device__ __forceinline__ void load_gates01(Small01 *sm, int tb, int te, int c, int e,
+                                             GateRaw raw, bool gated) {
+    const int t0 = tb + kC * c;
+    const int L = min(kC, te - t0);
+    const int buf = c & 3;
+    float g = (gated && e < L) ? lg2(fmaxf(raw.a, FLT_MIN)) : 0.f;
+    const int lane = e & 31;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float n = __shfl_up_sync(0xffffffffu, g, off);
+        if (lane >= off) g += n;
+    }
+    if (lane == 31) sm->scan_tmp[e >> 5] = g;
+    named_sync(2, 64);
+    if (e >= 32) g += sm->scan_tmp[0];
+    sm->lam[buf][e] = g;
+    if (e == 0) sm->len[buf] = L;
+    named_sync(2, 64);
+}
+
+template <int MODE, int KIND>
+__global__ void __launch_bounds__(kThreads, 1) prefill01_kernel(const __grid_constant__ TcParams p) {
+    using Y = Lay01;
+    constexpr int NST = Y::kStages;
+    constexpr bool kOut = (KIND == kOutput);
+    static_assert(MODE == 0 || MODE == 1, "modes 0 and 1 only");
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sb = smem_u32(smem_raw);
+    if (sb & 1023u) {
+        if (threadIdx.x == 0 && p.err) atomicOr(p.err, (unsigned)kErrBadLaunch);
+        return;
+    }
+    Small01 *sm = reinterpret_cast<Small01 *>(smem_raw + Y::kSmall);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bh = blockIdx.x % p.BH;
+    const int seg = blockIdx.x / p.BH;
+    const int tb = seg * p.seg_len;
+    const int te = min(p.T, tb + p.seg_len);
+    const int nch = (te - tb + kC - 1) / kC;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&sm->full[s], 1);
+            mbar_init(&sm->empty[s], 1);
+        }
+        mbar_init(&sm->prep_done, 1);
+        mbar_init(&sm->g_done, 1);
+        mbar_init(&sm->a_ready, 1);
+        mbar_init(&sm->mma2_done, 1);
+        mbar_init(&sm->s_ready, 1);
+        mbar_init(&sm->fin, 1);
+        sm->abort = 0;
+        sm->gsum = 0.f;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = sm->tmem_base;
+    volatile int *abort = &sm->abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tk);
+            tma_prefetch_desc(&p.tv);
+            if (kOut) tma_prefetch_desc(&p.tq);
+            int issued[NST];
+            for (int s = 0; s < NST; ++s) issued[s] = 0;
+            for (int c = 0; c < nch; ++c) {
+                const int s = c % NST, u = c / NST;
+                if (u >= 1 && !mbar_wait(&sm->empty[s], (u - 1) & 1, abort, p.err)) break;
+                const uint32_t st = sb + s * Y::kStage;
+                const int t = tb + kC * c;
+                mbar_arrive_expect_tx(&sm->full[s], kOut ? 49152u : 32768u);
+                tma_load_3d(st + 0, &p.tk, 0, t, bh, &sm->full[s]);
+                tma_load_3d(st + 16384, &p.tk, 64, t, bh, &sm->full[s]);
+                if (kOut) {
+                    tma_load_3d(st + 8192, &p.tq, 0, t, bh, &sm->full[s]);
+                    tma_load_3d(st + 24576, &p.tq, 64, t, bh, &sm->full[s]);
+                }
+                tma_load_3d(st + 32768, &p.tv, 0, t, bh, &sm->full[s]);
+                tma_load_3d(st + 40960, &p.tv, 64, t, bh, &sm->full[s]);
+                issued[s] = u + 1;
+            }
+            for (int s = 0; s < NST; ++s)
+                if (issued[s] > 0) drain_wait(&sm->full[s], (issued[s] - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t sbf = sb + Y::kSbf;
+            const uint32_t id_g = idesc_bf16(128, 64, false, false);
+            const uint32_t id_o1 = idesc_bf16(64, 128, false, false);
+            const uint32_t id_o2 = idesc_bf16(64, 128, false, true);
+            const uint32_t id_ds = idesc_bf16(128, 128, true, true);
+            // chunk j's operands are loaded and prepared; with outputs, G(j) = [K; Q] K^T
+            // into G[j & 1].  Chunk j+1 is taken before chunk j's products, so every
+            // prologue hand-off is consumed before the next one can be signalled.
+            auto take_chunk = [&](int j) -> bool {
+                const int s = j % NST, u = j / NST;
+                if (!mbar_wait(&sm->full[s], u & 1, abort, p.err)) return false;
+                if (!mbar_wait(&sm->prep_done, j & 1, abort, p.err)) return false;
+                if (kOut) {
+                    tc_fence_after();
+                    const uint32_t st = sb + s * Y::kStage;
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16_ss(tm + kColG2 + 64 * (j & 1), dk(st + off), dk(st + off), id_g,
+                                    ks > 0);
+                    }
+                    mma_commit(&sm->g_done);
+                }
+                return true;
+            };
+            bool ok = take_chunk(0);
+            for (int c = 0; c < nch && ok; ++c) {
+                const int s = c % NST;
+                const uint32_t st = sb + s * Y::kStage;
+                const uint32_t at = sb + Y::kA + (c & 1) * 8192;
+                if (c + 1 < nch && !take_chunk(c + 1)) break;
+                if (!mbar_wait(&sm->a_ready, c & 1, abort, p.err)) break;
+                if (!mbar_wait(&sm->s_ready, c & 1, abort, p.err)) break;
+                tc_fence_after();
+                if (kOut) {
+                    const uint32_t dq = (MODE == 1) ? kColP : kColO;
+                    for (int ks = 0; ks < 8; ++ks) {   // Q S^T
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16_ss(tm + dq, dk(st + 8192 + off), dk(sbf + off), id_o1, ks > 0);
+                    }
+                    for (int ks = 0; ks < 4; ++ks)     // A V
+                        mma_bf16_ss(tm + kColO, dk(at + ks * 32), dmn(st + 32768 + ks * 2048, 8192),
+                                    id_o2, MODE != 1 || ks > 0);
+                }
+                for (int ks = 0; ks < 4; ++ks)         // dS = V^T K~
+                    mma_bf16_ss(tm + kColDS, dmn(st + 32768 + ks * 2048, 8192),
+                                dmn(st + ks * 2048, 16384), id_ds, ks > 0);
+                mma_commit(&sm->mma2_done);
+            }
+            mma_commit(&sm->fin);
+            drain_wait(&sm->fin, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue warps 2-9
+        const int e = threadIdx.x - 64;
+        const int q = warp & 3;
+        const int h = (warp - 2) >> 2;
+        const int row = 32 * q + lane;
+        const uint32_t tl = tm + ((uint32_t)(32 * q) << 16);
+        const uint32_t sbf = sb + Y::kSbf;
+
+        float Sr[64];
+        {
+            const float *src = nullptr;
+            if (p.s_in_mode == 1)
+                src = p.s_in + (size_t)seg * p.s_in_seg + (size_t)bh * kD * kD + (size_t)row * kD;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) Sr[j] = src ? src[64 * h + j] : 0.f;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
+            if (MODE == 0 && e < kD) {
+                const float *zs = (p.s_in_mode == 1 && p.z_in)
+                                      ? p.z_in + (size_t)seg * p.z_in_seg + (size_t)bh * kD
+                                      : nullptr;
+                sm->z[1][e] = zs ? zs[e] : 0.f;   // z "after chunk -1"
+            }
+            fence_async_smem();
+            epi_sync();
+            if (e == 0) mbar_arrive(&sm->s_ready);
+        }
+
+        // chunk prologue: gates; mode 0: phi in place and z after this chunk
+        auto prep = [&](int c, GateRaw raw) -> bool {
+            const int s = c % NST, u = c / NST;
+            if (e < 64) load_gates01(sm, tb, te, c, e, raw, MODE == 1 && p.gate != nullptr);
+            mbar_wait(&sm->full[s], u & 1, abort, p.err);
+            epi_sync();
+            if (*abort) return false;
+            if (MODE == 0) {
+                const uint32_t st = sb + s * Y::kStage;
+                const int L = sm->len[c & 3];
+                constexpr int kIt = (kOut ? 4 : 2) * 512 / kEpi;
+                uint4 w[kIt];
+#pragma unroll
+                for (int it = 0; it < kIt; ++it) {
+                    const int n = e + kEpi * it;
+                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);
+                    w[it] = lds128(st + region * 8192 + (n & 511) * 16);
+                }
+#pragma unroll
+                for (int it = 0; it < kIt; ++it) {
+                    const int n = e + kEpi * it;
+                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);
+                    if ((region & 1) == 0 && ((n & 511) >> 3) >= L) {
+                        w[it] = make_uint4(0, 0, 0, 0);
+                    } else {
+                        w[it].x = phi_bf16x2(w[it].x);
+                        w[it].y = phi_bf16x2(w[it].y);
+                        w[it].z = phi_bf16x2(w[it].z);
+                        w[it].w = phi_bf16x2(w[it].w);
+                    }
+                    sts128(st + region * 8192 + (n & 511) * 16, w[it]);
+                }
+                epi_sync();
+                if (e < kD) {
+                    // z after chunk c = z after chunk c-1 + column sums of phi(K)
+                    const uint32_t kb = st + (e >> 6) * 16384;
+                    const int ch = (e & 63) >> 3, wi = e & 7;
+                    float zs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                    for (int j = 0; j < kC; ++j) {
+                        const uint32_t bits =
+                            lds_u16(kb + j * 128 + ((ch ^ (j & 7)) << 4) + wi * 2);
+                        zs[j & 3] += __uint_as_float(bits << 16);
+                    }
+                    sm->z[c & 1][e] = sm->z[(c + 1) & 1][e] + ((zs[0] + zs[1]) + (zs[2] + zs[3]));
+                }
+                fence_async_smem();
+            }
+            epi_sync();
+            if (e == 0) mbar_arrive(&sm->prep_done);
+            return true;
+        };
+
+        // A-epilogue of chunk j (A tile[j & 1]; mode 0 den parts; mode 1 K <- diag(dec) K)
+        auto aepi = [&](int j) -> bool {
+            const int s = j % NST;
+            const uint32_t st = sb + s * Y::kStage;
+            const int L = sm->len[j & 3];
+            const float *lam = sm->lam[j & 3];
+            if (kOut) {
+                mbar_wait(&sm->g_done, j & 1, abort, p.err);
+                epi_sync();
+                if (*abort) return false;
+                tc_fence_after();
+            }
+            if (q >= 2 && kOut) {
+                const int i = row - 64;
+                float v[32];
+                tmem_ld32(tl + kColG2 + 64 * (j & 1) + 32 * h, v);
+                const float li = lam[i];
+                float rs = 0.f;
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int cj = 32 * h + jj;
+                    float a = 0.f;
+                    if (cj <= i) a = (MODE == 0) ? v[jj] : v[jj] * ex2(li - lam[cj]);
+                    if (MODE == 0) {
+                        a = __bfloat162float(__float2bfloat16_rn(a));
+                        rs += a;
+                    }
+                    v[jj] = a;
+                }
+                const uint32_t at = sb + Y::kA + (j & 1) * 8192;
+                st_row_bf16x16(at, i, 4 * h, v);
+                st_row_bf16x16(at, i, 4 * h + 2, v + 16);
+                if (MODE == 0) sm->part[j & 1][h][i] = rs;
+            } else if (q < 2) {
+                if (MODE == 0 && kOut) {
+                    // phi(q_r) . z_{j-1} over d_k half h
+                    const int r = row;
+                    const float *zz = sm->z[(j + 1) & 1];
+                    uint4 w[8];
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        w[ch] = lds128(st + 8192 + h * 16384 + sw128_off(r, ch));
+                    float qz0 = 0.f, qz1 = 0.f;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint32_t *wd = reinterpret_cast<const uint32_t *>(&w[ch]);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 f = unpack_bf16x2(wd[k]);
+                            qz0 = fmaf(f.x, zz[64 * h + 8 * ch + 2 * k], qz0);
+                            qz1 = fmaf(f.y, zz[64 * h + 8 * ch + 2 * k + 1], qz1);
+                        }
+                    }
+                    sm->part[j & 1][2 + h][r] = qz0 + qz1;
+                }
+                if (MODE == 1) {
+                    // K <- diag(dec) K in place: 128 threads x 8 chunks
+                    const float lamL = lam[kC - 1];
+                    const int tq = (h * 2 + q) * 32 + lane;   // 0..127
+                    uint4 wk[8];
+#pragma unroll
+                    for (int it = 0; it < 8; ++it) {
+                        const int n = tq + 128 * it;
+                        wk[it] = lds128(st + (n >> 9) * 16384 + (n & 511) * 16);
+                    }
+#pragma unroll
+                    for (int it = 0; it < 8; ++it) {
+                        const int n = tq + 128 * it;
+                        const int r = (n & 511) >> 3;
+                        sts128(st + (n >> 9) * 16384 + (n & 511) * 16,
+                               scale_bf16x8(wk[it], r < L ? ex2(lamL - lam[r]) : 0.f));
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            epi_sync();
+            return true;
+        };
+
+        bool ok = prep(0, e < 64 ? fetch_gates<MODE>(p, bh, tb, te, 0, e) : GateRaw{1.f, 0.f});
+        GateRaw raw1{1.f, 0.f}, raw2{1.f, 0.f};
+        if (e < 64 && nch > 1) raw1 = fetch_gates<MODE>(p, bh, tb, te, 1, e);
+        if (ok) ok = aepi(0);
+        if (ok && e == 0) mbar_arrive(&sm->a_ready);
+        if (ok && nch > 1) ok = prep(1, raw1);
+        for (int c = 0; c < nch && ok; ++c) {
+            const int s = c % NST;
+            const int t0 = tb + kC * c;
+            const int L = sm->len[c & 3];
+            const float *lam = sm->lam[c & 3];
+            if (c + 2 < nch && e < 64) raw2 = fetch_gates<MODE>(p, bh, tb, te, c + 2, e);
+            // A-epilogue of the next chunk overlaps this chunk's products
+            if (c + 1 < nch && !aepi(c + 1)) break;
+            mbar_wait(&sm->mma2_done, c & 1, abort, p.err);
+            if (kOut && e == 0) tma_store_wait_read<0>();   // O staging free again
+            epi_sync();
+            if (*abort) break;
+            tc_fence_after();
+            if (c + 1 < nch && e == 0) mbar_arrive(&sm->a_ready);
+            // ---- outputs of chunk c (read O/P before the next products may start)
+            if (kOut) {
+                const int t = 16 * q + lane;
+                const bool has = lane < 16 && t < L;
+                float scale = 1.f;
+                if (MODE == 0 && has) {
+                    const float (*pt)[kC] = sm->part[c & 1];
+                    scale = 1.f / ((pt[0][t] + pt[1][t]) + (pt[2][t] + pt[3][t]));
+                }
+                if (MODE == 1 && has) scale = ex2(lam[t]);
+                const uint32_t ost = sb + Y::kOst + h * 8192;
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {
+                    float v[32];
+                    tmem_ld32(tl + kColO + 64 * h + 32 * sub, v);
+                    if (MODE == 1) {
+                        float pq[32];
+                        tmem_ld32(tl + kColP + 64 * h + 32 * sub, pq);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) v[jj] = fmaf(scale, pq[jj], v[jj]);
+                    } else {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) v[jj] *= scale;
+                    }
+                    if (has) {
+                        st_row_bf16x16(ost, t, 4 * sub, v);
+                        st_row_bf16x16(ost, t, 4 * sub + 2, v + 16);
+                    }
+                }
+            }
+            // ---- state: S <- g S + dS (registers), bf16 copy for the next products
+            const bool last = (c + 1 == nch);
+            {
+                const float gC = (MODE == 0) ? 1.f : ex2(lam[kC - 1]);
+                float v[64];
+                tmem_ld64(tl + kColDS + 64 * h, v);
+#pragma unroll
+                for (int jj = 0; jj < 64; ++jj) Sr[jj] = fmaf(gC, Sr[jj], v[jj]);
+                if (!last) {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
+                }
+                if (KIND == kLocal && MODE == 1 && e == 0) sm->gsum += lam[kC - 1];
+                if (last && p.s_out && (!p.out_last_only || seg == p.nseg - 1)) {
+                    float *dst = p.s_out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
+                                 (size_t)row * kD + 64 * h;
+#pragma unroll
+                    for (int jj = 0; jj < 64; jj += 4)
+                        *reinterpret_cast<float4 *>(dst + jj) =
+                            make_float4(Sr[jj], Sr[jj + 1], Sr[jj + 2], Sr[jj + 3]);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            epi_sync();
+            if (e == 0) {
+                mbar_arrive(&sm->s_ready);
+                mbar_arrive(&sm->empty[s]);
+                if (kOut) {
+                    tma_store_3d(&p.to, sb + Y::kOst, 0, t0, bh);
+                    tma_store_3d(&p.to, sb + Y::kOst + 8192, 64, t0, bh);
+                    tma_store_commit();
+                }
+            }
+            if (last) {
+                if (MODE == 0 && e < kD && p.z_out && (!p.out_last_only || seg == p.nseg - 1))
+                    p.z_out[(size_t)seg * p.z_out_seg + (size_t)bh * kD + e] = sm->z[c & 1][e];
+                if (KIND == kLocal && MODE == 1 && e == 0 && p.gam_out)
+                    p.gam_out[(size_t)seg * p.BH + bh] = ex2(sm->gsum);
+            }
+            // ---- prologue of chunk c+2
+            if (c + 2 < nch && !prep(c + 2, raw2)) break;
+        }
+        if (kOut && e == 0) tma_store_wait_all<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tm, kTmemCols);
+    }
+}
+
 // ------------------------------------------------------------------ combine kernels
 // modes 0/1: S_start[s+1] = gam_s S_start[s] + N_s;  z_start[s+1] = z_start[s] + zN_s.
 __global__ void combine_scalar_kernel(int BH, int nseg, const float *s_init, const float *z_init,
@@ -908,8 +1385,8 @@ size_t workspace_floats(int mode, int BH, const Plan &pl) {
 
 template <int MODE, int KIND>
 cudaError_t launch_kind(const TcParams &p, int grid, cudaStream_t stream) {
-    auto kern = prefill_tc_kernel<MODE, KIND>;
-    const uint32_t bytes = Lay<MODE>::kBytes;
+    auto kern = (MODE == 2) ? prefill_tc_kernel<2, KIND> : prefill01_kernel<MODE == 2 ? 0 : MODE, KIND>;
+    const uint32_t bytes = (MODE == 2) ? Lay<2>::kBytes : Lay01::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, bytes, stream>>>(p);
