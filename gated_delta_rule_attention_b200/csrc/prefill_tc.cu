@@ -836,61 +836,67 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 }
 
 // ------------------------------------------------------------------ modes 0 / 1
-// A software-pipelined variant for the two modes without the delta-rule solve.  The
-// epilogue of iteration c forms the A tile of chunk c+1 while the tensor core computes
-// the outputs and state product of chunk c; the MMA issuer forms Q K^T of chunk c+1
-// before the products of chunk c.  G and the A tile are double-buffered by chunk
-// parity, gate buffers by chunk mod 4, and every hand-off is ordered so that no
-// mbarrier can complete two phases ahead of its waiter.
+// The two modes without the delta-rule solve run a dedicated kernel of 12 warps:
+//   warp 0      TMA producer (a ring of three stages of K, Q, V tiles),
+//   warp 1      owns TMEM; lane 0 issues every MMA,
+//   warps 2-9   epilogue: A tile, outputs, and the fp32 state (in registers),
+//   warps 10-11 chunk preparation, running ahead of the epilogue: the in-chunk gate
+//               prefix (mode 1), the feature map phi = elu + 1 applied in place to the
+//               Q and K tiles, the running normaliser z and phi(q_t).z (mode 0), and,
+//               in the LOCAL pass, the decayed K~ = diag(dec) K (mode 1).
+// Per chunk c of the OUTPUT pass the tensor core forms G(c+1) = Q K^T (M=64) while the
+// epilogue is still on chunk c, then Q S^T, A V (M=64) and dS = V^T K~ (M=128) of chunk c.
+// The epilogue turns G(c+1) into the A tile of chunk c+1 while those products run,
+// then writes the outputs of chunk c and adds dS to its register-resident state.  The
+// LOCAL pass (no outputs) double-buffers dS so that the state update of chunk c
+// overlaps the product of chunk c+1.
+//
+// Every hand-off is an mbarrier whose next phase cannot complete before its waiter has
+// consumed the current one: a stage is released only when both the tensor core (commit)
+// and the epilogue (after its last use of the chunk) are done with it, and the
+// per-chunk barriers that can run ahead are double-buffered by chunk parity.  One
+// thread per role polls each barrier, with a bound; the others meet it at a named
+// barrier that also ORs the abandon decision, so that every thread leaves together.
+constexpr int kThreads01 = 384;                 // 12 warps
+constexpr uint32_t kColG01 = 128;               // two 64-column G buffers (M=64)
+constexpr uint32_t kColO01 = 256, kColP01 = 384;
+
 struct Small01 {
-    uint64_t full[3], empty[3];
-    uint64_t prep_done, g_done, a_ready, mma2_done, s_ready, fin;
+    uint64_t full[3], empty[3], prep_done[3];
+    uint64_t g_done[2], a_ready[2], ds_done[2], ds_free[2];
+    uint64_t s_ready, mma2_done, fin;
     uint32_t tmem_base;
     int abort;
-    int len[4];
-    float lam[4][kC];      // in-chunk inclusive prefix of log2(a), chunk mod 4
-    float part[2][4][kC];  // mode 0: row-sum halves and phi(q).z halves, chunk parity
-    float z[2][kD];        // mode 0: z after chunk j in z[j & 1] (z_in in z[1])
+    int len[8];
+    float lam[8][kC];       // in-chunk inclusive prefix of log2(a), chunk mod 8
+    float part[8][3][kC];   // mode 0 denominators: A row-sum halves [0, 1], phi(q).z [2]
+    alignas(16) float zsm[kD];   // mode 0: z after the previous chunk (float4 reads)
     float scan_tmp[2];
-    float gsum;
 };
 struct Lay01 {
     static constexpr int kStages = 3;
-    static constexpr uint32_t kStage = 49152;
-    static constexpr uint32_t kSbf = kStages * kStage;   // 32 KB
-    static constexpr uint32_t kA = kSbf + 32768;          // 2 x 8 KB
-    static constexpr uint32_t kOst = kA + 16384;          // 16 KB
+    static constexpr uint32_t kStage = 49152;             // [K0][Q0][K1][Q1][V0][V1], 8 KB each
+    static constexpr uint32_t kSbf = kStages * kStage;    // 32 KB bf16 state [d_v][d_k]
+    static constexpr uint32_t kA = kSbf + 32768;          // 2 x 8 KB A tiles [t][j]
+    static constexpr uint32_t kOst = kA + 16384;          // 16 KB output staging
     static constexpr uint32_t kSmall = kOst + 16384;
     static constexpr uint32_t kBytes = kSmall + sizeof(Small01);
 };
-constexpr uint32_t kColG2 = 128;   // two 64-column G buffers: 128, 192
+static_assert(Lay01::kBytes <= 227 * 1024, "shared memory per CTA");
 
-__device__ __forceinline__ void load_gates01(Small01 *sm, int tb, int te, int c, int e,
-                                             GateRaw raw, bool gated) {
-    const int t0 = tb + kC * c;
-    const int L = min(kC, te - t0);
-    const int buf = c & 3;
-    float g = (gated && e < L) ? lg2(fmaxf(raw.a, FLT_MIN)) : 0.f;
-    const int lane = e & 31;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const float n = __shfl_up_sync(0xffffffffu, g, off);
-        if (lane >= off) g += n;
-    }
-    if (lane == 31) sm->scan_tmp[e >> 5] = g;
-    named_sync(2, 64);
-    if (e >= 32) g += sm->scan_tmp[0];
-    sm->lam[buf][e] = g;
-    if (e == 0) sm->len[buf] = L;
-    named_sync(2, 64);
+__device__ __forceinline__ float ld_gate(const TcParams &p, int bh, int t0, int L, int i) {
+    float a = 1.f;
+    if (i < L) asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(a) : "l"(p.gate + (size_t)bh * p.T + t0 + i));
+    return a;
 }
 
 template <int MODE, int KIND>
-__global__ void __launch_bounds__(kThreads, 1) prefill01_kernel(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_constant__ TcParams p) {
     using Y = Lay01;
     constexpr int NST = Y::kStages;
     constexpr bool kOut = (KIND == kOutput);
     static_assert(MODE == 0 || MODE == 1, "modes 0 and 1 only");
+    static_assert(KIND == kOutput || KIND == kLocal, "no transition pass without the delta rule");
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sb = smem_u32(smem_raw);
@@ -911,16 +917,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill01_kernel(const __grid_con
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&sm->full[s], 1);
-            mbar_init(&sm->empty[s], 1);
+            mbar_init(&sm->empty[s], 2);     // tensor-core commit + epilogue
+            mbar_init(&sm->prep_done[s], 1);
         }
-        mbar_init(&sm->prep_done, 1);
-        mbar_init(&sm->g_done, 1);
-        mbar_init(&sm->a_ready, 1);
-        mbar_init(&sm->mma2_done, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm->g_done[b], 1);
+            mbar_init(&sm->a_ready[b], 1);
+            mbar_init(&sm->ds_done[b], 1);
+            mbar_init(&sm->ds_free[b], 1);
+        }
         mbar_init(&sm->s_ready, 1);
+        mbar_init(&sm->mma2_done, 1);
         mbar_init(&sm->fin, 1);
         sm->abort = 0;
-        sm->gsum = 0.f;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -964,64 +973,237 @@ __global__ void __launch_bounds__(kThreads, 1) prefill01_kernel(const __grid_con
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t sbf = sb + Y::kSbf;
-            const uint32_t id_g = idesc_bf16(128, 64, false, false);
+            const uint32_t id_g = idesc_bf16(64, 64, false, false);
             const uint32_t id_o1 = idesc_bf16(64, 128, false, false);
             const uint32_t id_o2 = idesc_bf16(64, 128, false, true);
             const uint32_t id_ds = idesc_bf16(128, 128, true, true);
-            // chunk j's operands are loaded and prepared; with outputs, G(j) = [K; Q] K^T
-            // into G[j & 1].  Chunk j+1 is taken before chunk j's products, so every
-            // prologue hand-off is consumed before the next one can be signalled.
-            auto take_chunk = [&](int j) -> bool {
-                const int s = j % NST, u = j / NST;
-                if (!mbar_wait(&sm->full[s], u & 1, abort, p.err)) return false;
-                if (!mbar_wait(&sm->prep_done, j & 1, abort, p.err)) return false;
-                if (kOut) {
+            if (kOut) {
+                // G(j) = phi(Q) phi(K)^T or Q K^T of chunk j, into G[j & 1]
+                auto take = [&](int j) -> bool {
+                    const int s = j % NST, u = j / NST;
+                    if (!mbar_wait(&sm->full[s], u & 1, abort, p.err)) return false;
+                    if (!mbar_wait(&sm->prep_done[s], u & 1, abort, p.err)) return false;
                     tc_fence_after();
                     const uint32_t st = sb + s * Y::kStage;
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16_ss(tm + kColG2 + 64 * (j & 1), dk(st + off), dk(st + off), id_g,
-                                    ks > 0);
+                        mma_bf16_ss(tm + kColG01 + 64 * (j & 1), dk(st + 8192 + off), dk(st + off),
+                                    id_g, ks > 0);
                     }
-                    mma_commit(&sm->g_done);
-                }
-                return true;
-            };
-            bool ok = take_chunk(0);
-            for (int c = 0; c < nch && ok; ++c) {
-                const int s = c % NST;
-                const uint32_t st = sb + s * Y::kStage;
-                const uint32_t at = sb + Y::kA + (c & 1) * 8192;
-                if (c + 1 < nch && !take_chunk(c + 1)) break;
-                if (!mbar_wait(&sm->a_ready, c & 1, abort, p.err)) break;
-                if (!mbar_wait(&sm->s_ready, c & 1, abort, p.err)) break;
-                tc_fence_after();
-                if (kOut) {
-                    const uint32_t dq = (MODE == 1) ? kColP : kColO;
+                    mma_commit(&sm->g_done[j & 1]);
+                    return true;
+                };
+                bool ok = take(0);
+                for (int c = 0; c < nch && ok; ++c) {
+                    const int s = c % NST;
+                    const uint32_t st = sb + s * Y::kStage;
+                    const uint32_t at = sb + Y::kA + (c & 1) * 8192;
+                    if (c + 1 < nch && !take(c + 1)) break;
+                    if (!mbar_wait(&sm->a_ready[c & 1], (c >> 1) & 1, abort, p.err)) break;
+                    if (!mbar_wait(&sm->s_ready, c & 1, abort, p.err)) break;
+                    tc_fence_after();
+                    const uint32_t dq = (MODE == 1) ? kColP01 : kColO01;
                     for (int ks = 0; ks < 8; ++ks) {   // Q S^T
                         const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
                         mma_bf16_ss(tm + dq, dk(st + 8192 + off), dk(sbf + off), id_o1, ks > 0);
                     }
                     for (int ks = 0; ks < 4; ++ks)     // A V
-                        mma_bf16_ss(tm + kColO, dk(at + ks * 32), dmn(st + 32768 + ks * 2048, 8192),
+                        mma_bf16_ss(tm + kColO01, dk(at + ks * 32), dmn(st + 32768 + ks * 2048, 8192),
                                     id_o2, MODE != 1 || ks > 0);
+                    for (int ks = 0; ks < 4; ++ks)     // dS = V^T K~
+                        mma_bf16_ss(tm + kColDS, dmn(st + 32768 + ks * 2048, 8192),
+                                    dmn(st + ks * 2048, 16384), id_ds, ks > 0);
+                    mma_commit(&sm->mma2_done);
+                    mma_commit(&sm->empty[s]);
                 }
-                for (int ks = 0; ks < 4; ++ks)         // dS = V^T K~
-                    mma_bf16_ss(tm + kColDS, dmn(st + 32768 + ks * 2048, 8192),
-                                dmn(st + ks * 2048, 16384), id_ds, ks > 0);
-                mma_commit(&sm->mma2_done);
+            } else {
+                for (int c = 0; c < nch; ++c) {
+                    const int s = c % NST, u = c / NST, b = c & 1;
+                    const uint32_t st = sb + s * Y::kStage;
+                    if (!mbar_wait(&sm->full[s], u & 1, abort, p.err)) break;
+                    if (!mbar_wait(&sm->prep_done[s], u & 1, abort, p.err)) break;
+                    if (c >= 2 && !mbar_wait(&sm->ds_free[b], ((c >> 1) - 1) & 1, abort, p.err)) break;
+                    tc_fence_after();
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ss(tm + kColDS + 128 * b, dmn(st + 32768 + ks * 2048, 8192),
+                                    dmn(st + ks * 2048, 16384), id_ds, ks > 0);
+                    mma_commit(&sm->ds_done[b]);
+                    mma_commit(&sm->empty[s]);
+                }
             }
             mma_commit(&sm->fin);
             drain_wait(&sm->fin, 0);
         }
+    } else if (warp >= 10) {
+        // ------------------------------------------------------------ chunk preparation
+        const int pe = threadIdx.x - 320;      // 0..63
+        const int pw = pe >> 5;                // K column half of this warp (mode 0)
+        const int cg = lane & 7, rg = lane >> 3;
+        float zr[8];                           // mode 0: z of columns 64 pw + 8 cg + k
+        if (MODE == 0) {
+            const float *zs = (p.s_in_mode == 1 && p.z_in)
+                                  ? p.z_in + (size_t)seg * p.z_in_seg + (size_t)bh * kD
+                                  : nullptr;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) zr[k] = zs ? zs[64 * pw + 8 * cg + k] : 0.f;
+            if (rg == 0)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) sm->zsm[64 * pw + 8 * cg + k] = zr[k];
+        }
+        float gsum = 0.f;
+        const bool gated = (MODE == 1) && p.gate != nullptr;
+        float graw = gated ? ld_gate(p, bh, tb, min(kC, te - tb), pe) : 1.f;
+        for (int j = 0; j < nch; ++j) {
+            const int s = j % NST, u = j / NST;
+            const int t0 = tb + kC * j;
+            const int L = min(kC, te - t0);
+            float gnext = 1.f;
+            if (gated && j + 1 < nch) gnext = ld_gate(p, bh, t0 + kC, min(kC, te - t0 - kC), pe);
+            if (MODE == 1) {
+                float g = (gated && pe < L) ? lg2(fmaxf(graw, FLT_MIN)) : 0.f;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float n = __shfl_up_sync(0xffffffffu, g, off);
+                    if (lane >= off) g += n;
+                }
+                if (lane == 31) sm->scan_tmp[pw] = g;
+                named_sync(2, 64);
+                if (pw == 1) g += sm->scan_tmp[0];
+                sm->lam[j & 7][pe] = g;
+                if (pe == kC - 1) gsum += g;
+            }
+            if (pe == 0) sm->len[j & 7] = L;
+            bool ok = true;
+            if (pe == 0) ok = mbar_wait(&sm->full[s], u & 1, abort, p.err);
+            if (named_sync_any(2, 64, !ok)) break;
+            const uint32_t st = sb + s * Y::kStage;
+            if (MODE == 0) {
+                if (kOut) {
+                    // phi(Q) in place, thread = row; phi(q_r) . z_{j-1}
+                    const int r = pe;
+                    float qz0 = 0.f, qz1 = 0.f;
+#pragma unroll
+                    for (int l4 = 0; l4 < 16; l4 += 4) {
+                        uint4 w[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int lc = l4 + i;
+                            w[i] = lds128(st + 8192 + (lc >> 3) * 16384 + sw128_off(r, lc & 7));
+                        }
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int lc = l4 + i;
+                            w[i].x = phi_bf16x2(w[i].x);
+                            w[i].y = phi_bf16x2(w[i].y);
+                            w[i].z = phi_bf16x2(w[i].z);
+                            w[i].w = phi_bf16x2(w[i].w);
+                            sts128(st + 8192 + (lc >> 3) * 16384 + sw128_off(r, lc & 7), w[i]);
+                            const float4 za = *reinterpret_cast<const float4 *>(&sm->zsm[8 * lc]);
+                            const float4 zb = *reinterpret_cast<const float4 *>(&sm->zsm[8 * lc + 4]);
+                            float2 f = unpack_bf16x2(w[i].x);
+                            qz0 = fmaf(f.x, za.x, qz0);
+                            qz1 = fmaf(f.y, za.y, qz1);
+                            f = unpack_bf16x2(w[i].y);
+                            qz0 = fmaf(f.x, za.z, qz0);
+                            qz1 = fmaf(f.y, za.w, qz1);
+                            f = unpack_bf16x2(w[i].z);
+                            qz0 = fmaf(f.x, zb.x, qz0);
+                            qz1 = fmaf(f.y, zb.y, qz1);
+                            f = unpack_bf16x2(w[i].w);
+                            qz0 = fmaf(f.x, zb.z, qz0);
+                            qz1 = fmaf(f.y, zb.w, qz1);
+                        }
+                    }
+                    sm->part[j & 7][2][r] = qz0 + qz1;
+                    named_sync(2, 64);   // every read of z_{j-1} is done
+                }
+                // phi(K) in place (rows past the chunk end zeroed), column sums into z
+                float cs[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) cs[k] = 0.f;
+#pragma unroll
+                for (int i4 = 0; i4 < 16; i4 += 4) {
+                    uint4 w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = 16 * rg + i4 + i;
+                        w[i] = lds128(st + pw * 16384 + sw128_off(r, cg));
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = 16 * rg + i4 + i;
+                        if (r < L) {
+                            w[i].x = phi_bf16x2(w[i].x);
+                            w[i].y = phi_bf16x2(w[i].y);
+                            w[i].z = phi_bf16x2(w[i].z);
+                            w[i].w = phi_bf16x2(w[i].w);
+                        } else {
+                            w[i] = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                        sts128(st + pw * 16384 + sw128_off(r, cg), w[i]);
+                        const uint32_t *wd = reinterpret_cast<const uint32_t *>(&w[i]);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 f = unpack_bf16x2(wd[k]);
+                            cs[2 * k] += f.x;
+                            cs[2 * k + 1] += f.y;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    cs[k] += __shfl_xor_sync(0xffffffffu, cs[k], 8);
+                    cs[k] += __shfl_xor_sync(0xffffffffu, cs[k], 16);
+                    zr[k] += cs[k];
+                }
+                if (rg == 0)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) sm->zsm[64 * pw + 8 * cg + k] = zr[k];
+            } else if (!kOut) {
+                // LOCAL, mode 1: K~ = diag(dec) K in place, dec_r = 2^(lam_{C-1} - lam_r)
+                named_sync(2, 64);   // the whole prefix is written
+                const float *lam = sm->lam[j & 7];
+                const float lamL = lam[kC - 1];
+#pragma unroll
+                for (int i4 = 0; i4 < 16; i4 += 4) {
+                    uint4 w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int n = pe + 64 * (i4 + i);
+                        w[i] = lds128(st + (n >> 9) * 16384 + (n & 511) * 16);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int n = pe + 64 * (i4 + i);
+                        const int r = (n & 511) >> 3;
+                        sts128(st + (n >> 9) * 16384 + (n & 511) * 16,
+                               scale_bf16x8(w[i], r < L ? ex2(lamL - lam[r]) : 0.f));
+                    }
+                }
+            }
+            fence_async_smem();
+            named_sync(2, 64);
+            if (pe == 0) mbar_arrive(&sm->prep_done[s]);
+            graw = gnext;
+        }
+        if (MODE == 0 && rg == 0 && p.z_out && (!p.out_last_only || seg == p.nseg - 1)) {
+            float *dst = p.z_out + (size_t)seg * p.z_out_seg + (size_t)bh * kD + 64 * pw + 8 * cg;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) dst[k] = zr[k];
+        }
+        if (MODE == 1 && !kOut && pe == kC - 1 && p.gam_out)
+            p.gam_out[(size_t)seg * p.BH + bh] = ex2(gsum);
     } else {
         // ------------------------------------------------------------ epilogue warps 2-9
-        const int e = threadIdx.x - 64;
-        const int q = warp & 3;
-        const int h = (warp - 2) >> 2;
-        const int row = 32 * q + lane;
+        const int e = threadIdx.x - 64;        // 0..255
+        const int q = warp & 3;                // TMEM lane quarter of this warp
+        const int h = (warp - 2) >> 2;         // column half
+        const int row = 32 * q + lane;         // M=128 accumulator row = state row
         const uint32_t tl = tm + ((uint32_t)(32 * q) << 16);
         const uint32_t sbf = sb + Y::kSbf;
+        // M=64 accumulators: row 16 q + (lane & 15); lanes 16-31 take the second column range
+        const int r64 = 16 * q + (lane & 15);
+        const int hi = lane >> 4;
 
         float Sr[64];
         {
@@ -1030,246 +1212,179 @@ __global__ void __launch_bounds__(kThreads, 1) prefill01_kernel(const __grid_con
                 src = p.s_in + (size_t)seg * p.s_in_seg + (size_t)bh * kD * kD + (size_t)row * kD;
 #pragma unroll
             for (int j = 0; j < 64; ++j) Sr[j] = src ? src[64 * h + j] : 0.f;
+            if (kOut) {
 #pragma unroll
-            for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
-            if (MODE == 0 && e < kD) {
-                const float *zs = (p.s_in_mode == 1 && p.z_in)
-                                      ? p.z_in + (size_t)seg * p.z_in_seg + (size_t)bh * kD
-                                      : nullptr;
-                sm->z[1][e] = zs ? zs[e] : 0.f;   // z "after chunk -1"
+                for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
+                fence_async_smem();
+                epi_sync();
+                if (e == 0) mbar_arrive(&sm->s_ready);
             }
-            fence_async_smem();
-            epi_sync();
-            if (e == 0) mbar_arrive(&sm->s_ready);
         }
 
-        // chunk prologue: gates; mode 0: phi in place and z after this chunk
-        auto prep = [&](int c, GateRaw raw) -> bool {
-            const int s = c % NST, u = c / NST;
-            if (e < 64) load_gates01(sm, tb, te, c, e, raw, MODE == 1 && p.gate != nullptr);
-            mbar_wait(&sm->full[s], u & 1, abort, p.err);
-            epi_sync();
-            if (*abort) return false;
-            if (MODE == 0) {
-                const uint32_t st = sb + s * Y::kStage;
-                const int L = sm->len[c & 3];
-                constexpr int kIt = (kOut ? 4 : 2) * 512 / kEpi;
-                uint4 w[kIt];
-#pragma unroll
-                for (int it = 0; it < kIt; ++it) {
-                    const int n = e + kEpi * it;
-                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);
-                    w[it] = lds128(st + region * 8192 + (n & 511) * 16);
+        if (kOut) {
+            // A tile of chunk j from G(j): masks, decays (mode 1) or denominators (mode 0);
+            // mode 1 also scales K to K~ = diag(dec) K once G(j) has consumed it.
+            auto aepi = [&](int j) -> bool {
+                const int s = j % NST, u = j / NST;
+                bool ok = true;
+                if (e == 0) {
+                    ok = mbar_wait(&sm->prep_done[s], u & 1, abort, p.err) &&
+                         mbar_wait(&sm->g_done[j & 1], (j >> 1) & 1, abort, p.err);
+                    if (MODE == 1 && ok) ok = mbar_wait(&sm->full[s], u & 1, abort, p.err);
                 }
-#pragma unroll
-                for (int it = 0; it < kIt; ++it) {
-                    const int n = e + kEpi * it;
-                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);
-                    if ((region & 1) == 0 && ((n & 511) >> 3) >= L) {
-                        w[it] = make_uint4(0, 0, 0, 0);
-                    } else {
-                        w[it].x = phi_bf16x2(w[it].x);
-                        w[it].y = phi_bf16x2(w[it].y);
-                        w[it].z = phi_bf16x2(w[it].z);
-                        w[it].w = phi_bf16x2(w[it].w);
-                    }
-                    sts128(st + region * 8192 + (n & 511) * 16, w[it]);
-                }
-                epi_sync();
-                if (e < kD) {
-                    // z after chunk c = z after chunk c-1 + column sums of phi(K)
-                    const uint32_t kb = st + (e >> 6) * 16384;
-                    const int ch = (e & 63) >> 3, wi = e & 7;
-                    float zs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-                    for (int j = 0; j < kC; ++j) {
-                        const uint32_t bits =
-                            lds_u16(kb + j * 128 + ((ch ^ (j & 7)) << 4) + wi * 2);
-                        zs[j & 3] += __uint_as_float(bits << 16);
-                    }
-                    sm->z[c & 1][e] = sm->z[(c + 1) & 1][e] + ((zs[0] + zs[1]) + (zs[2] + zs[3]));
-                }
-                fence_async_smem();
-            }
-            epi_sync();
-            if (e == 0) mbar_arrive(&sm->prep_done);
-            return true;
-        };
-
-        // A-epilogue of chunk j (A tile[j & 1]; mode 0 den parts; mode 1 K <- diag(dec) K)
-        auto aepi = [&](int j) -> bool {
-            const int s = j % NST;
-            const uint32_t st = sb + s * Y::kStage;
-            const int L = sm->len[j & 3];
-            const float *lam = sm->lam[j & 3];
-            if (kOut) {
-                mbar_wait(&sm->g_done, j & 1, abort, p.err);
-                epi_sync();
-                if (*abort) return false;
+                if (named_sync_any(1, kEpi, !ok)) return false;
                 tc_fence_after();
-            }
-            if (q >= 2 && kOut) {
-                const int i = row - 64;
-                float v[32];
-                tmem_ld32(tl + kColG2 + 64 * (j & 1) + 32 * h, v);
-                const float li = lam[i];
+                const int L = sm->len[j & 7];
+                const float *lam = sm->lam[j & 7];
+                const int i = r64;
+                float v[16];
+                tmem_ld_pair16(tl + kColG01 + 64 * (j & 1) + 32 * h, v);
+                const int c0 = 32 * h + 16 * hi;
+                const float li = (MODE == 1) ? lam[i] : 0.f;
                 float rs = 0.f;
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int cj = 32 * h + jj;
+                for (int k = 0; k < 16; ++k) {
                     float a = 0.f;
-                    if (cj <= i) a = (MODE == 0) ? v[jj] : v[jj] * ex2(li - lam[cj]);
+                    if (c0 + k <= i) a = (MODE == 0) ? v[k] : v[k] * ex2(li - lam[c0 + k]);
                     if (MODE == 0) {
                         a = __bfloat162float(__float2bfloat16_rn(a));
                         rs += a;
                     }
-                    v[jj] = a;
+                    v[k] = a;
                 }
-                const uint32_t at = sb + Y::kA + (j & 1) * 8192;
-                st_row_bf16x16(at, i, 4 * h, v);
-                st_row_bf16x16(at, i, 4 * h + 2, v + 16);
-                if (MODE == 0) sm->part[j & 1][h][i] = rs;
-            } else if (q < 2) {
-                if (MODE == 0 && kOut) {
-                    // phi(q_r) . z_{j-1} over d_k half h
-                    const int r = row;
-                    const float *zz = sm->z[(j + 1) & 1];
-                    uint4 w[8];
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        w[ch] = lds128(st + 8192 + h * 16384 + sw128_off(r, ch));
-                    float qz0 = 0.f, qz1 = 0.f;
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        const uint32_t *wd = reinterpret_cast<const uint32_t *>(&w[ch]);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const float2 f = unpack_bf16x2(wd[k]);
-                            qz0 = fmaf(f.x, zz[64 * h + 8 * ch + 2 * k], qz0);
-                            qz1 = fmaf(f.y, zz[64 * h + 8 * ch + 2 * k + 1], qz1);
-                        }
-                    }
-                    sm->part[j & 1][2 + h][r] = qz0 + qz1;
+                st_row_bf16x16(sb + Y::kA + (j & 1) * 8192, i, c0 >> 3, v);
+                if (MODE == 0) {
+                    rs += __shfl_xor_sync(0xffffffffu, rs, 16);
+                    if (hi == 0) sm->part[j & 7][h][i] = rs;
                 }
                 if (MODE == 1) {
-                    // K <- diag(dec) K in place: 128 threads x 8 chunks
+                    const uint32_t st = sb + s * Y::kStage;
                     const float lamL = lam[kC - 1];
-                    const int tq = (h * 2 + q) * 32 + lane;   // 0..127
-                    uint4 wk[8];
+                    uint4 w[4];
 #pragma unroll
-                    for (int it = 0; it < 8; ++it) {
-                        const int n = tq + 128 * it;
-                        wk[it] = lds128(st + (n >> 9) * 16384 + (n & 511) * 16);
+                    for (int it = 0; it < 4; ++it) {
+                        const int n = e + kEpi * it;
+                        w[it] = lds128(st + (n >> 9) * 16384 + (n & 511) * 16);
                     }
 #pragma unroll
-                    for (int it = 0; it < 8; ++it) {
-                        const int n = tq + 128 * it;
+                    for (int it = 0; it < 4; ++it) {
+                        const int n = e + kEpi * it;
                         const int r = (n & 511) >> 3;
                         sts128(st + (n >> 9) * 16384 + (n & 511) * 16,
-                               scale_bf16x8(wk[it], r < L ? ex2(lamL - lam[r]) : 0.f));
+                               scale_bf16x8(w[it], r < L ? ex2(lamL - lam[r]) : 0.f));
                     }
                 }
-            }
-            fence_async_smem();
-            tc_fence_before();
-            epi_sync();
-            return true;
-        };
-
-        bool ok = prep(0, e < 64 ? fetch_gates<MODE>(p, bh, tb, te, 0, e) : GateRaw{1.f, 0.f});
-        GateRaw raw1{1.f, 0.f}, raw2{1.f, 0.f};
-        if (e < 64 && nch > 1) raw1 = fetch_gates<MODE>(p, bh, tb, te, 1, e);
-        if (ok) ok = aepi(0);
-        if (ok && e == 0) mbar_arrive(&sm->a_ready);
-        if (ok && nch > 1) ok = prep(1, raw1);
-        for (int c = 0; c < nch && ok; ++c) {
-            const int s = c % NST;
-            const int t0 = tb + kC * c;
-            const int L = sm->len[c & 3];
-            const float *lam = sm->lam[c & 3];
-            if (c + 2 < nch && e < 64) raw2 = fetch_gates<MODE>(p, bh, tb, te, c + 2, e);
-            // A-epilogue of the next chunk overlaps this chunk's products
-            if (c + 1 < nch && !aepi(c + 1)) break;
-            mbar_wait(&sm->mma2_done, c & 1, abort, p.err);
-            if (kOut && e == 0) tma_store_wait_read<0>();   // O staging free again
-            epi_sync();
-            if (*abort) break;
-            tc_fence_after();
-            if (c + 1 < nch && e == 0) mbar_arrive(&sm->a_ready);
-            // ---- outputs of chunk c (read O/P before the next products may start)
-            if (kOut) {
-                const int t = 16 * q + lane;
-                const bool has = lane < 16 && t < L;
-                float scale = 1.f;
-                if (MODE == 0 && has) {
-                    const float (*pt)[kC] = sm->part[c & 1];
-                    scale = 1.f / ((pt[0][t] + pt[1][t]) + (pt[2][t] + pt[3][t]));
+                fence_async_smem();
+                tc_fence_before();
+                epi_sync();
+                if (e == 0) {
+                    mbar_arrive(&sm->a_ready[j & 1]);
+                    mbar_arrive(&sm->empty[s]);   // the epilogue is done with this stage
                 }
-                if (MODE == 1 && has) scale = ex2(lam[t]);
-                const uint32_t ost = sb + Y::kOst + h * 8192;
-#pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {
+                return true;
+            };
+
+            bool ok = aepi(0);
+            for (int c = 0; c < nch && ok; ++c) {
+                const int t0 = tb + kC * c;
+                if (c + 1 < nch && !aepi(c + 1)) break;
+                bool w_ok = true;
+                if (e == 0) {
+                    w_ok = mbar_wait(&sm->mma2_done, c & 1, abort, p.err);
+                    tma_store_wait_read<0>();   // output staging free again
+                }
+                if (named_sync_any(1, kEpi, !w_ok)) break;
+                tc_fence_after();
+                const int L = sm->len[c & 7];
+                const float *lam = sm->lam[c & 7];
+                // ---- outputs of chunk c: row t = r64, columns 64 h + 32 hi + [0, 32)
+                {
+                    const int t = r64;
+                    const bool has = t < L;
+                    float scale = 1.f;
+                    if (MODE == 0 && has) {
+                        const float (*pt)[kC] = sm->part[c & 7];
+                        scale = 1.f / ((pt[0][t] + pt[1][t]) + pt[2][t]);
+                    }
+                    if (MODE == 1 && has) scale = ex2(lam[t]);
                     float v[32];
-                    tmem_ld32(tl + kColO + 64 * h + 32 * sub, v);
+                    tmem_ld_pair32(tl + kColO01 + 64 * h, v);
                     if (MODE == 1) {
                         float pq[32];
-                        tmem_ld32(tl + kColP + 64 * h + 32 * sub, pq);
+                        tmem_ld_pair32(tl + kColP01 + 64 * h, pq);
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) v[jj] = fmaf(scale, pq[jj], v[jj]);
+                        for (int k = 0; k < 32; ++k) v[k] = fmaf(scale, pq[k], v[k]);
                     } else {
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) v[jj] *= scale;
+                        for (int k = 0; k < 32; ++k) v[k] *= scale;
                     }
                     if (has) {
-                        st_row_bf16x16(ost, t, 4 * sub, v);
-                        st_row_bf16x16(ost, t, 4 * sub + 2, v + 16);
+                        const uint32_t ost = sb + Y::kOst + h * 8192;
+                        st_row_bf16x16(ost, t, 4 * hi, v);
+                        st_row_bf16x16(ost, t, 4 * hi + 2, v + 16);
                     }
                 }
-            }
-            // ---- state: S <- g S + dS (registers), bf16 copy for the next products
-            const bool last = (c + 1 == nch);
-            {
-                const float gC = (MODE == 0) ? 1.f : ex2(lam[kC - 1]);
-                float v[64];
-                tmem_ld64(tl + kColDS + 64 * h, v);
+                // ---- state: S <- g S + dS (registers), bf16 copy for the next products
+                const bool last = (c + 1 == nch);
+                {
+                    const float gC = (MODE == 0) ? 1.f : ex2(lam[kC - 1]);
+                    float v[64];
+                    tmem_ld64(tl + kColDS + 64 * h, v);
 #pragma unroll
-                for (int jj = 0; jj < 64; ++jj) Sr[jj] = fmaf(gC, Sr[jj], v[jj]);
-                if (!last) {
+                    for (int k = 0; k < 64; ++k) Sr[k] = fmaf(gC, Sr[k], v[k]);
+                    if (!last) {
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
+                        for (int g = 0; g < 4; ++g)
+                            st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
+                    }
                 }
-                if (KIND == kLocal && MODE == 1 && e == 0) sm->gsum += lam[kC - 1];
-                if (last && p.s_out && (!p.out_last_only || seg == p.nseg - 1)) {
-                    float *dst = p.s_out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
-                                 (size_t)row * kD + 64 * h;
-#pragma unroll
-                    for (int jj = 0; jj < 64; jj += 4)
-                        *reinterpret_cast<float4 *>(dst + jj) =
-                            make_float4(Sr[jj], Sr[jj + 1], Sr[jj + 2], Sr[jj + 3]);
-                }
-            }
-            fence_async_smem();
-            tc_fence_before();
-            epi_sync();
-            if (e == 0) {
-                mbar_arrive(&sm->s_ready);
-                mbar_arrive(&sm->empty[s]);
-                if (kOut) {
+                fence_async_smem();
+                tc_fence_before();
+                epi_sync();
+                if (e == 0) {
+                    mbar_arrive(&sm->s_ready);
                     tma_store_3d(&p.to, sb + Y::kOst, 0, t0, bh);
                     tma_store_3d(&p.to, sb + Y::kOst + 8192, 64, t0, bh);
                     tma_store_commit();
                 }
+                if (last && p.s_out && (!p.out_last_only || seg == p.nseg - 1)) {
+                    float *dst = p.s_out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
+                                 (size_t)row * kD + 64 * h;
+#pragma unroll
+                    for (int k = 0; k < 64; k += 4)
+                        *reinterpret_cast<float4 *>(dst + k) =
+                            make_float4(Sr[k], Sr[k + 1], Sr[k + 2], Sr[k + 3]);
+                }
             }
-            if (last) {
-                if (MODE == 0 && e < kD && p.z_out && (!p.out_last_only || seg == p.nseg - 1))
-                    p.z_out[(size_t)seg * p.z_out_seg + (size_t)bh * kD + e] = sm->z[c & 1][e];
-                if (KIND == kLocal && MODE == 1 && e == 0 && p.gam_out)
-                    p.gam_out[(size_t)seg * p.BH + bh] = ex2(sm->gsum);
+            if (e == 0) tma_store_wait_all<0>();
+        } else {
+            for (int c = 0; c < nch; ++c) {
+                const int s = c % NST, u = c / NST, b = c & 1;
+                bool ok = true;
+                if (e == 0)
+                    ok = mbar_wait(&sm->prep_done[s], u & 1, abort, p.err) &&
+                         mbar_wait(&sm->ds_done[b], (c >> 1) & 1, abort, p.err);
+                if (e == 0 && ok) mbar_arrive(&sm->empty[s]);   // stage: only dS(c) reads it
+                if (named_sync_any(1, kEpi, !ok)) break;
+                tc_fence_after();
+                const float gC = (MODE == 0) ? 1.f : ex2(sm->lam[c & 7][kC - 1]);
+                float v[64];
+                tmem_ld64(tl + kColDS + 128 * b + 64 * h, v);
+#pragma unroll
+                for (int k = 0; k < 64; ++k) Sr[k] = fmaf(gC, Sr[k], v[k]);
+                tc_fence_before();
+                epi_sync();
+                if (e == 0) mbar_arrive(&sm->ds_free[b]);
+                if (c + 1 == nch && p.s_out) {
+                    float *dst = p.s_out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
+                                 (size_t)row * kD + 64 * h;
+#pragma unroll
+                    for (int k = 0; k < 64; k += 4)
+                        *reinterpret_cast<float4 *>(dst + k) =
+                            make_float4(Sr[k], Sr[k + 1], Sr[k + 2], Sr[k + 3]);
+                }
             }
-            // ---- prologue of chunk c+2
-            if (c + 2 < nch && !prep(c + 2, raw2)) break;
         }
-        if (kOut && e == 0) tma_store_wait_all<0>();
     }
     tc_fence_before();
     __syncthreads();
@@ -1385,11 +1500,19 @@ size_t workspace_floats(int mode, int BH, const Plan &pl) {
 
 template <int MODE, int KIND>
 cudaError_t launch_kind(const TcParams &p, int grid, cudaStream_t stream) {
-    auto kern = (MODE == 2) ? prefill_tc_kernel<2, KIND> : prefill01_kernel<MODE == 2 ? 0 : MODE, KIND>;
-    const uint32_t bytes = (MODE == 2) ? Lay<2>::kBytes : Lay01::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, bytes, stream>>>(p);
+    cudaError_t e;
+    if constexpr (MODE == 2) {
+        e = cudaFuncSetAttribute(prefill_tc_kernel<2, KIND>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Lay<2>::kBytes);
+        if (e != cudaSuccess) return e;
+        prefill_tc_kernel<2, KIND><<<grid, kThreads, Lay<2>::kBytes, stream>>>(p);
+    } else {
+        static_assert(KIND != kTransition, "the transition pass belongs to the delta rule");
+        e = cudaFuncSetAttribute(prefill01_kernel<MODE, KIND>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Lay01::kBytes);
+        if (e != cudaSuccess) return e;
+        prefill01_kernel<MODE, KIND><<<grid, kThreads01, Lay01::kBytes, stream>>>(p);
+    }
     note_launches(1);
     return cudaGetLastError();
 }
