@@ -1394,6 +1394,489 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
     }
 }
 
+// ------------------------------------------------------------------ mode 0
+// elu(x)+1 linear attention with the z normaliser.  No gate acts on the state, so the
+// fp32 state lives in tensor memory and each chunk's dS = V^T phi(K) is accumulated into
+// it by the MMA itself.  What remains per chunk is dominated by the feature map: 2 x 64 x
+// 128 exponentials, which the special-function units deliver at 16 per clock per SM.
+// Eight preparation warps, two on each SM sub-partition, share that work.  18 warps:
+//   warp 0      TMA producer,
+//   warp 1      owns TMEM; lane 0 issues every MMA,
+//   warps 2-9   epilogue: A tile and denominators, bf16 copy of the state, outputs,
+//   warps 10-17 preparation: phi applied in place to the Q and K tiles, the running
+//               column sums z, and phi(q_t) . z_{chunk start}.
+// TMEM: S 0-127 (M=128), G = phi(Q) phi(K)^T 128-255 (two M=64 buffers), O 256-511 (two
+// M=64 buffers, so that the outputs of chunk c are read while chunk c+1 is computed).
+// Shared memory holds two rings filled by TMA: K and Q tiles, four deep, because the
+// preparation warps and Q K^T need them early; V tiles, two deep, needed only by the
+// products of the chunk.  The outputs of a chunk are staged in the Q tile of its own K/Q
+// slot, dead once the products are done, and written by TMA; the slot is released when
+// that store has read it.  G is formed two chunks ahead, after the products of the
+// current chunk, so that the tensor core runs the state chain products(c) -> state copy
+// -> products(c+1) without waiting behind it.
+// The tensor core commits once after Q S^T and dS (the epilogue may then copy the new
+// state) and once after A V (the outputs are complete).
+constexpr int kThreadsE = 576;
+constexpr int kPrepE = 256;   // preparation threads (warps 10-17)
+constexpr uint32_t kColSE = 0, kColGE = 128, kColOE = 256;
+
+struct SmallE {
+    uint64_t full_kq[4], empty_kq[4], prep_done[4], full_v[2], empty_v[2];
+    uint64_t g_done[2], a_ready[2], o_free[2], mma2_done[2];
+    uint64_t s_ready, s_done, fin;
+    uint32_t tmem_base;
+    int abort;
+    int len[8];
+    float part[8][4][kC];        // denominators: A row-sum halves [0, 1], phi(q).z halves [2, 3]
+    alignas(16) float zsm[kD];   // z after the previous chunk (float4 reads)
+    float zpart[8][64];          // per-warp column sums of phi(K)
+};
+struct LayE {
+    static constexpr int kKQStages = 4, kVStages = 2;
+    static constexpr uint32_t kKQ = 0;                      // 4 x 32 KB [K0][Q0][K1][Q1], 8 KB each
+    static constexpr uint32_t kV = kKQ + kKQStages * 32768;  // 2 x 16 KB [V0][V1]
+    static constexpr uint32_t kSbf = kV + kVStages * 16384;  // 32 KB bf16 state [d_v][d_k]
+    static constexpr uint32_t kA = kSbf + 32768;             // 2 x 8 KB A tiles [t][j]
+    static constexpr uint32_t kSmall = kA + 16384;
+    static constexpr uint32_t kBytes = kSmall + sizeof(SmallE);
+};
+static_assert(LayE::kBytes <= 227 * 1024, "shared memory per CTA");
+
+__device__ __forceinline__ void phi_bf16x8(uint4 &w) {
+    w.x = phi_bf16x2(w.x);
+    w.y = phi_bf16x2(w.y);
+    w.z = phi_bf16x2(w.z);
+    w.w = phi_bf16x2(w.w);
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_constant__ TcParams p) {
+    using Y = LayE;
+    constexpr int NKQ = Y::kKQStages, NV = Y::kVStages;
+    constexpr bool kOut = (KIND == kOutput);
+    static_assert(KIND == kOutput || KIND == kLocal, "output or local pass");
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sb = smem_u32(smem_raw);
+    if (sb & 1023u) {
+        if (threadIdx.x == 0 && p.err) atomicOr(p.err, (unsigned)kErrBadLaunch);
+        return;
+    }
+    SmallE *sm = reinterpret_cast<SmallE *>(smem_raw + Y::kSmall);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bh = blockIdx.x % p.BH;
+    const int seg = blockIdx.x / p.BH;
+    const int tb = seg * p.seg_len;
+    const int te = min(p.T, tb + p.seg_len);
+    const int nch = (te - tb + kC - 1) / kC;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NKQ; ++s) {
+            mbar_init(&sm->full_kq[s], 1);
+            mbar_init(&sm->empty_kq[s], kOut ? 2 : 1);   // tensor core (+ A-epilogue)
+            mbar_init(&sm->prep_done[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm->full_v[b], 1);
+            mbar_init(&sm->empty_v[b], 1);
+            mbar_init(&sm->g_done[b], 1);
+            mbar_init(&sm->a_ready[b], 1);
+            mbar_init(&sm->o_free[b], 1);
+            mbar_init(&sm->mma2_done[b], 1);
+        }
+        mbar_init(&sm->s_ready, 1);
+        mbar_init(&sm->s_done, 1);
+        mbar_init(&sm->fin, 1);
+        sm->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = sm->tmem_base;
+    volatile int *abort = &sm->abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        // Both rings are refilled as soon as their slot is released, whichever comes
+        // first: the K/Q ring runs up to four chunks ahead, the V ring two.
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tk);
+            tma_prefetch_desc(&p.tv);
+            if (kOut) tma_prefetch_desc(&p.tq);
+            int nkq = 0, nv = 0;
+            uint32_t idle = 0;
+            while ((nkq < nch || nv < nch) && !*abort) {
+                bool moved = false;
+                if (nkq < nch && (nkq < NKQ || mbar_try_wait(&sm->empty_kq[nkq % NKQ], ((nkq / NKQ) - 1) & 1))) {
+                    const int s = nkq % NKQ, t = tb + kC * nkq;
+                    const uint32_t st = sb + Y::kKQ + s * 32768;
+                    mbar_arrive_expect_tx(&sm->full_kq[s], kOut ? 32768u : 16384u);
+                    tma_load_3d(st + 0, &p.tk, 0, t, bh, &sm->full_kq[s]);
+                    tma_load_3d(st + 16384, &p.tk, 64, t, bh, &sm->full_kq[s]);
+                    if (kOut) {
+                        tma_load_3d(st + 8192, &p.tq, 0, t, bh, &sm->full_kq[s]);
+                        tma_load_3d(st + 24576, &p.tq, 64, t, bh, &sm->full_kq[s]);
+                    }
+                    ++nkq;
+                    moved = true;
+                }
+                if (nv < nch && (nv < NV || mbar_try_wait(&sm->empty_v[nv % NV], ((nv / NV) - 1) & 1))) {
+                    const int s = nv % NV, t = tb + kC * nv;
+                    const uint32_t sv = sb + Y::kV + s * 16384;
+                    mbar_arrive_expect_tx(&sm->full_v[s], 16384u);
+                    tma_load_3d(sv + 0, &p.tv, 0, t, bh, &sm->full_v[s]);
+                    tma_load_3d(sv + 8192, &p.tv, 64, t, bh, &sm->full_v[s]);
+                    ++nv;
+                    moved = true;
+                }
+                if (moved) {
+                    idle = 0;
+                } else if (++idle > kSpinLimit) {
+                    *abort = 1;
+                    if (p.err) atomicOr(p.err, 1u);
+                }
+            }
+            // wait for the copies in flight before the CTA may exit
+            for (int c = max(0, nkq - NKQ); c < nkq; ++c) drain_wait(&sm->full_kq[c % NKQ], (c / NKQ) & 1);
+            for (int c = max(0, nv - NV); c < nv; ++c) drain_wait(&sm->full_v[c % NV], (c / NV) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t sbf = sb + Y::kSbf;
+            const uint32_t id_g = idesc_bf16(64, 64, false, false);
+            const uint32_t id_o1 = idesc_bf16(64, 128, false, false);
+            const uint32_t id_o2 = idesc_bf16(64, 128, false, true);
+            const uint32_t id_ds = idesc_bf16(128, 128, true, true);
+            if (kOut) {
+                auto take = [&](int j) -> bool {   // G(j) = phi(Q) phi(K)^T into G[j & 1]
+                    const int s = j % NKQ, u = j / NKQ;
+                    if (!mbar_wait(&sm->full_kq[s], u & 1, abort, p.err)) return false;
+                    if (!mbar_wait(&sm->prep_done[s], u & 1, abort, p.err)) return false;
+                    tc_fence_after();
+                    const uint32_t st = sb + Y::kKQ + s * 32768;
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16_ss(tm + kColGE + 64 * (j & 1), dk(st + 8192 + off), dk(st + off),
+                                    id_g, ks > 0);
+                    }
+                    mma_commit(&sm->g_done[j & 1]);
+                    return true;
+                };
+                bool ok = take(0) && (nch < 2 || take(1));
+                for (int c = 0; c < nch && ok; ++c) {
+                    const int s = c % NKQ, b = c & 1, sv = c % NV;
+                    const uint32_t st = sb + Y::kKQ + s * 32768;
+                    const uint32_t vt = sb + Y::kV + sv * 16384;
+                    const uint32_t at = sb + Y::kA + b * 8192;
+                    const uint32_t to = tm + kColOE + 128 * b;
+                    if (!mbar_wait(&sm->a_ready[b], (c >> 1) & 1, abort, p.err)) break;
+                    if (!mbar_wait(&sm->s_ready, c & 1, abort, p.err)) break;
+                    if (c >= 2 && !mbar_wait(&sm->o_free[b], ((c >> 1) - 1) & 1, abort, p.err)) break;
+                    if (!mbar_wait(&sm->full_v[sv], (c / NV) & 1, abort, p.err)) break;
+                    tc_fence_after();
+                    for (int ks = 0; ks < 8; ++ks) {   // phi(Q) S^T
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16_ss(to, dk(st + 8192 + off), dk(sbf + off), id_o1, ks > 0);
+                    }
+                    for (int ks = 0; ks < 4; ++ks)     // S += V^T phi(K)
+                        mma_bf16_ss(tm + kColSE, dmn(vt + ks * 2048, 8192),
+                                    dmn(st + ks * 2048, 16384), id_ds, true);
+                    mma_commit(&sm->s_done);
+                    for (int ks = 0; ks < 4; ++ks)     // + A V
+                        mma_bf16_ss(to, dk(at + ks * 32), dmn(vt + ks * 2048, 8192), id_o2, true);
+                    mma_commit(&sm->mma2_done[b]);
+                    mma_commit(&sm->empty_kq[s]);
+                    mma_commit(&sm->empty_v[sv]);
+                    if (c + 2 < nch && !take(c + 2)) break;
+                }
+            } else {
+                bool ok = mbar_wait(&sm->s_ready, 0, abort, p.err);   // initial state in TMEM
+                for (int c = 0; c < nch && ok; ++c) {
+                    const int s = c % NKQ, u = c / NKQ, sv = c % NV;
+                    const uint32_t st = sb + Y::kKQ + s * 32768;
+                    const uint32_t vt = sb + Y::kV + sv * 16384;
+                    if (!mbar_wait(&sm->full_kq[s], u & 1, abort, p.err)) break;
+                    if (!mbar_wait(&sm->prep_done[s], u & 1, abort, p.err)) break;
+                    if (!mbar_wait(&sm->full_v[sv], (c / NV) & 1, abort, p.err)) break;
+                    tc_fence_after();
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ss(tm + kColSE, dmn(vt + ks * 2048, 8192),
+                                    dmn(st + ks * 2048, 16384), id_ds, true);
+                    mma_commit(&sm->empty_kq[s]);
+                    mma_commit(&sm->empty_v[sv]);
+                }
+                mma_commit(&sm->s_done);
+            }
+            mma_commit(&sm->fin);
+            drain_wait(&sm->fin, 0);
+        }
+    } else if (warp >= 10) {
+        // ------------------------------------------------------------ preparation
+        const int pe = threadIdx.x - 320;      // 0..255
+        const int pw = pe >> 5;                // 0..7
+        const int ch = lane & 7, rg = lane >> 3;
+        float zc = 0.f;                        // z of column pe (pe < 128)
+        if (pe < kD) {
+            const float *zs = (p.s_in_mode == 1 && p.z_in)
+                                  ? p.z_in + (size_t)seg * p.z_in_seg + (size_t)bh * kD
+                                  : nullptr;
+            zc = zs ? zs[pe] : 0.f;
+            sm->zsm[pe] = zc;
+        }
+        // Warp pw takes column half pw >> 2 and rows 16 (pw & 3) + 4 rg + i (i < 4); lane
+        // chunk ch holds columns 8 ch .. 8 ch + 7 of that half.
+        const int hw = pw >> 2;
+        const uint32_t half = (uint32_t)hw * 16384;
+        const int r0 = 16 * (pw & 3) + 4 * rg;
+        for (int j = 0; j < nch; ++j) {
+            const int s = j % NKQ, u = j / NKQ;
+            const int L = min(kC, te - (tb + kC * j));
+            if (pe == 0) sm->len[j & 7] = L;
+            bool ok = true;
+            if (pe == 0) ok = mbar_wait(&sm->full_kq[s], u & 1, abort, p.err);
+            if (named_sync_any(2, kPrepE, !ok)) break;
+            const uint32_t st = sb + Y::kKQ + s * 32768;
+            if (kOut) {
+                // phi(Q) in place, and phi(q_r) . z_{j-1} over this half (shuffle-reduced)
+                const uint32_t qb = st + 8192 + half;
+                const float4 za = *reinterpret_cast<const float4 *>(&sm->zsm[64 * hw + 8 * ch]);
+                const float4 zb = *reinterpret_cast<const float4 *>(&sm->zsm[64 * hw + 8 * ch + 4]);
+                uint4 w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) w[i] = lds128(qb + sw128_off(r0 + i, ch));
+                float d[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    phi_bf16x8(w[i]);
+                    const float2 f0 = unpack_bf16x2(w[i].x), f1 = unpack_bf16x2(w[i].y);
+                    const float2 f2 = unpack_bf16x2(w[i].z), f3 = unpack_bf16x2(w[i].w);
+                    d[i] = fmaf(f0.x, za.x, fmaf(f0.y, za.y, fmaf(f1.x, za.z, f1.y * za.w))) +
+                           fmaf(f2.x, zb.x, fmaf(f2.y, zb.y, fmaf(f3.x, zb.z, f3.y * zb.w)));
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sts128(qb + sw128_off(r0 + i, ch), w[i]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    d[i] += __shfl_xor_sync(0xffffffffu, d[i], 1);
+                    d[i] += __shfl_xor_sync(0xffffffffu, d[i], 2);
+                    d[i] += __shfl_xor_sync(0xffffffffu, d[i], 4);
+                }
+                if (ch == 0)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) sm->part[j & 7][2 + hw][r0 + i] = d[i];
+            }
+            // phi(K) in place (rows past the chunk end zeroed) and its column sums
+            {
+                const uint32_t kb = st + half;
+                uint4 w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) w[i] = lds128(kb + sw128_off(r0 + i, ch));
+                float cs[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) cs[k] = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (r0 + i < L)
+                        phi_bf16x8(w[i]);
+                    else
+                        w[i] = make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t *wd = reinterpret_cast<const uint32_t *>(&w[i]);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 f = unpack_bf16x2(wd[k]);
+                        cs[2 * k] += f.x;
+                        cs[2 * k + 1] += f.y;
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sts128(kb + sw128_off(r0 + i, ch), w[i]);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    cs[k] += __shfl_xor_sync(0xffffffffu, cs[k], 8);
+                    cs[k] += __shfl_xor_sync(0xffffffffu, cs[k], 16);
+                }
+                if (rg == 0)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) sm->zpart[pw][8 * ch + k] = cs[k];
+            }
+            named_sync(2, kPrepE);   // column sums ready; every read of z_{j-1} is done
+            if (pe < kD) {
+                const int w0 = 4 * (pe >> 6), cc = pe & 63;
+                zc += (sm->zpart[w0][cc] + sm->zpart[w0 + 1][cc]) +
+                      (sm->zpart[w0 + 2][cc] + sm->zpart[w0 + 3][cc]);
+                sm->zsm[pe] = zc;
+            }
+            fence_async_smem();
+            named_sync(2, kPrepE);
+            if (pe == 0) mbar_arrive(&sm->prep_done[s]);
+        }
+        if (pe < kD && p.z_out && (!p.out_last_only || seg == p.nseg - 1))
+            p.z_out[(size_t)seg * p.z_out_seg + (size_t)bh * kD + pe] = zc;
+    } else {
+        // ------------------------------------------------------------ epilogue warps 2-9
+        const int e = threadIdx.x - 64;        // 0..255
+        const int q = warp & 3;                // TMEM lane quarter of this warp
+        const int h = (warp - 2) >> 2;         // column half
+        const int row = 32 * q + lane;         // state row (d_v index) = TMEM lane
+        const uint32_t tl = tm + ((uint32_t)(32 * q) << 16);
+        const uint32_t sbf = sb + Y::kSbf;
+        const int r64 = 16 * q + (lane & 15);  // M=64 accumulator row of this thread
+        const int hi = lane >> 4;
+
+        // initial state into TMEM (and its bf16 copy for the first Q S^T)
+        {
+            const float *src = nullptr;
+            if (p.s_in_mode == 1)
+                src = p.s_in + (size_t)seg * p.s_in_seg + (size_t)bh * kD * kD + (size_t)row * kD;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float v[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) v[k] = src ? src[64 * h + 16 * g + k] : 0.f;
+                tmem_st16(tl + kColSE + 64 * h + 16 * g, v);
+                if (kOut) st_row_bf16x16(sbf + h * 16384, row, 2 * g, v);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            epi_sync();
+            if (e == 0) mbar_arrive(&sm->s_ready);
+        }
+
+        if (kOut) {
+            // A tile of chunk j from G(j), with its row sums for the denominators
+            auto aepi = [&](int j) -> bool {
+                const int s = j % NKQ, u = j / NKQ;
+                bool ok = true;
+                if (e == 0)
+                    ok = mbar_wait(&sm->prep_done[s], u & 1, abort, p.err) &&
+                         mbar_wait(&sm->g_done[j & 1], (j >> 1) & 1, abort, p.err);
+                if (named_sync_any(1, kEpi, !ok)) return false;
+                tc_fence_after();
+                const int i = r64;
+                float v[16];
+                tmem_ld_pair16(tl + kColGE + 64 * (j & 1) + 32 * h, v);
+                const int c0 = 32 * h + 16 * hi;
+                float rs = 0.f;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float a = (c0 + k <= i) ? __bfloat162float(__float2bfloat16_rn(v[k])) : 0.f;
+                    rs += a;
+                    v[k] = a;
+                }
+                st_row_bf16x16(sb + Y::kA + (j & 1) * 8192, i, c0 >> 3, v);
+                rs += __shfl_xor_sync(0xffffffffu, rs, 16);
+                if (hi == 0) sm->part[j & 7][h][i] = rs;
+                fence_async_smem();
+                tc_fence_before();
+                epi_sync();
+                if (e == 0) mbar_arrive(&sm->a_ready[j & 1]);
+                return true;
+            };
+
+            bool ok = aepi(0);
+            for (int c = 0; c < nch && ok; ++c) {
+                const int t0 = tb + kC * c;
+                const int b = c & 1;
+                const bool last = (c + 1 == nch);
+                if (c + 1 < nch && !aepi(c + 1)) break;
+                // ---- state after chunk c: bf16 copy for the next products
+                bool w_ok = true;
+                if (e == 0) w_ok = mbar_wait(&sm->s_done, c & 1, abort, p.err);
+                if (named_sync_any(1, kEpi, !w_ok)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {
+                    float v[32];
+                    tmem_ld32(tl + kColSE + 64 * h + 32 * sub, v);
+                    if (!last) {
+                        st_row_bf16x16(sbf + h * 16384, row, 4 * sub, v);
+                        st_row_bf16x16(sbf + h * 16384, row, 4 * sub + 2, v + 16);
+                    } else if (p.s_out && (!p.out_last_only || seg == p.nseg - 1)) {
+                        float *dst = p.s_out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
+                                     (size_t)row * kD + 64 * h + 32 * sub;
+#pragma unroll
+                        for (int k = 0; k < 32; k += 4)
+                            *reinterpret_cast<float4 *>(dst + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+                    }
+                }
+                fence_async_smem();
+                tc_fence_before();
+                epi_sync();
+                if (e == 0) mbar_arrive(&sm->s_ready);
+                // ---- outputs of chunk c: row t = r64, columns 64 h + 32 hi + [0, 32)
+                if (e == 0) {
+                    w_ok = mbar_wait(&sm->mma2_done[b], (c >> 1) & 1, abort, p.err);
+                    if (c > 0) {   // the outputs of chunk c-1 have left their staging tile
+                        tma_store_wait_read<0>();
+                        mbar_arrive(&sm->empty_kq[(c - 1) % NKQ]);
+                    }
+                }
+                if (named_sync_any(1, kEpi, !w_ok)) break;
+                tc_fence_after();
+                {
+                    const int L = sm->len[c & 7];
+                    const int t = r64;
+                    const bool has = t < L;
+                    float scale = 1.f;
+                    if (has) {
+                        const float (*pt)[kC] = sm->part[c & 7];
+                        scale = 1.f / ((pt[0][t] + pt[1][t]) + (pt[2][t] + pt[3][t]));
+                    }
+                    float v[32];
+                    tmem_ld_pair32(tl + kColOE + 128 * b + 64 * h, v);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) v[k] *= scale;
+                    if (has) {   // Q tile of this chunk's K/Q slot: [Q0 | Q1] at +8 KB, +24 KB
+                        const uint32_t ost = sb + Y::kKQ + (c % NKQ) * 32768 + 8192 + h * 16384;
+                        st_row_bf16x16(ost, t, 4 * hi, v);
+                        st_row_bf16x16(ost, t, 4 * hi + 2, v + 16);
+                    }
+                }
+                fence_async_smem();
+                tc_fence_before();
+                epi_sync();
+                if (e == 0) {
+                    mbar_arrive(&sm->o_free[b]);
+                    const uint32_t ost = sb + Y::kKQ + (c % NKQ) * 32768 + 8192;
+                    tma_store_3d(&p.to, ost, 0, t0, bh);
+                    tma_store_3d(&p.to, ost + 16384, 64, t0, bh);
+                    tma_store_commit();
+                }
+            }
+            if (e == 0) tma_store_wait_all<0>();
+        } else {
+            bool ok = true;
+            if (e == 0) ok = mbar_wait(&sm->s_done, 0, abort, p.err);
+            if (!named_sync_any(1, kEpi, !ok)) {
+                tc_fence_after();
+                float v[64];
+                tmem_ld64(tl + kColSE + 64 * h, v);
+                if (p.s_out) {
+                    float *dst = p.s_out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
+                                 (size_t)row * kD + 64 * h;
+#pragma unroll
+                    for (int k = 0; k < 64; k += 4)
+                        *reinterpret_cast<float4 *>(dst + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tm, kTmemCols);
+    }
+}
+
 // ------------------------------------------------------------------ combine kernels
 // modes 0/1: S_start[s+1] = gam_s S_start[s] + N_s;  z_start[s+1] = z_start[s] + zN_s.
 __global__ void combine_scalar_kernel(int BH, int nseg, const float *s_init, const float *z_init,
@@ -1508,10 +1991,17 @@ cudaError_t launch_kind(const TcParams &p, int grid, cudaStream_t stream) {
         prefill_tc_kernel<2, KIND><<<grid, kThreads, Lay<2>::kBytes, stream>>>(p);
     } else {
         static_assert(KIND != kTransition, "the transition pass belongs to the delta rule");
-        e = cudaFuncSetAttribute(prefill01_kernel<MODE, KIND>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Lay01::kBytes);
-        if (e != cudaSuccess) return e;
-        prefill01_kernel<MODE, KIND><<<grid, kThreads01, Lay01::kBytes, stream>>>(p);
+        if constexpr (MODE == 0) {
+            e = cudaFuncSetAttribute(prefill_elu_kernel<KIND>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, LayE::kBytes);
+            if (e != cudaSuccess) return e;
+            prefill_elu_kernel<KIND><<<grid, kThreadsE, LayE::kBytes, stream>>>(p);
+        } else {
+            e = cudaFuncSetAttribute(prefill01_kernel<MODE, KIND>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, Lay01::kBytes);
+            if (e != cudaSuccess) return e;
+            prefill01_kernel<MODE, KIND><<<grid, kThreads01, Lay01::kBytes, stream>>>(p);
+        }
     }
     note_launches(1);
     return cudaGetLastError();
