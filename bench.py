@@ -152,16 +152,17 @@ def kernel_sources_sha():
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key: str):
-    """DRAM bytes per launch from the committed ncu summary, if it is for these sources."""
+def ncu_traffic(workload: str):
+    """The committed ncu launch summary of `workload` (kernels in launch order, each with
+    its DRAM bytes per launch and time share), or None when it was taken on other kernel
+    sources than the ones built here."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
-        e = t[kernel_key]
-        if e.get("sources_sha") != kernel_sources_sha():
+        if t.get("sources_sha") != kernel_sources_sha():
             return None
-        return float(e["dram_bytes_per_launch"])
+        return t["workloads"][workload]
     except Exception:
         return None
 
@@ -354,6 +355,25 @@ def time_steps(case, steps, warmup, dist, device, flush, fn=None, sampler=None):
     return ms, launches
 
 
+def launch_profile(case, steps, flush):
+    """Device duration (ms) of each launch of one call, averaged over `steps` further
+    calls: the library records CUDA events around each of its launches on the launching
+    stream (la_launch_timing).  L2 is flushed between calls as in the timed region."""
+    la = case.la
+    la.launch_timing(True)
+    per = []
+    try:
+        for _ in range(steps):
+            if flush is not None:
+                flush.zero_()
+            case.step()
+            per.append(la.launch_times())
+    finally:
+        la.launch_timing(False)
+    n = min(len(p) for p in per) if per else 0
+    return [statistics.mean(p[i] for p in per) for i in range(n)]
+
+
 class _Null:
     def __enter__(self):
         return self
@@ -362,12 +382,47 @@ class _Null:
         return False
 
 
+def roofline(case, kernel_ms, step_ms, peaks, peak_src, prof):
+    """Roofline of the call's outputs pass (its last launch, the one that reads and writes
+    every token of the call: algorithmic bytes = the whole call's), timed by CUDA events on
+    the launching stream, next to the same figure for the whole call (all launches)."""
+    hbm_bound = case.bytes / (peaks["hbm_gbs"] * 1e9) >= case.flops / (peaks["bf16_tflops"] * 1e12)
+    n = len(kernel_ms)
+    names = ([k["name"] for k in prof["kernels"]] if prof and len(prof["kernels"]) == n
+             else [f"launch {i}" for i in range(n)])
+    t_k = (kernel_ms[-1] if n else step_ms) * 1e-3
+    t_call = (sum(kernel_ms) if n else step_ms) * 1e-3
+    if hbm_bound:
+        unit, peak, work, scale = "GB/s", peaks["hbm_gbs"], case.bytes, 1e9
+    else:
+        unit, peak, work, scale = "TFLOP/s", peaks["bf16_tflops"], case.flops, 1e12
+    ach = work / t_k / scale
+    ach_call = work / t_call / scale
+    traffic = None
+    if prof and len(prof["kernels"]) == n and n:
+        traffic = float(prof["kernels"][-1]["dram_bytes_per_launch"])
+    return {
+        "bound": "hbm" if hbm_bound else "tensor",
+        "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak, "traffic": traffic,
+        "kernel": names[-1] if n else "call",
+        "kernel_ms": kernel_ms[-1] if n else step_ms,
+        "kernel_share": (kernel_ms[-1] / sum(kernel_ms)) if n else 1.0,
+        "algorithmic_bytes": case.bytes, "algorithmic_flops": case.flops,
+        "tensor_frac": case.flops / t_k / 1e12 / peaks["bf16_tflops"],
+        "call": {"launches": n, "kernels": names, "kernel_ms": kernel_ms,
+                 "achieved": ach_call, "frac": ach_call / peak,
+                 "traffic": float(prof["dram_bytes_per_call"]) if prof else None},
+        "peak_source": (f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"),
+    }
+
+
 def measure(la, name, args, dist, device, rank, world, flush, with_e2e, sampler=None):
     w = W.CONFIGS[name]
     case = (DecodeCase(la, w, device, rank, args.warmup + args.steps) if w.decode
             else PrefillCase(la, w, device, rank, None if args.no_workspace else "auto"))
     ms, launches = time_steps(case, args.steps, args.warmup, dist, device, flush, sampler=sampler)
     la.check_status()
+    kernel_ms = launch_profile(case, args.steps, flush)
     total_ms = max_over_ranks(dist, sum(ms), device)
     tokens_all = sum_over_ranks(dist, case.tokens * args.steps, device)
     per_launch_ms = statistics.mean(ms) / max(1, launches // max(1, args.steps))
@@ -389,6 +444,7 @@ def measure(la, name, args, dist, device, rank, world, flush, with_e2e, sampler=
         "attainable_frac": max(case.bytes / (peaks["hbm_gbs"] * 1e9),
                                case.flops / (peaks["bf16_tflops"] * 1e12)) / (statistics.mean(ms) * 1e-3),
         "peak_source": peak_src,
+        "kernel_ms": kernel_ms,
         "_case": case, "_ms": ms, "_launches": launches, "_per_launch_ms": per_launch_ms,
     }
     if with_e2e:
@@ -540,21 +596,7 @@ def main():
     w = W.CONFIGS[args.workload]
     case = main_res["_case"]
     mean_ms = statistics.mean(main_res["_ms"])
-    hbm_bound = case.bytes / (peaks["hbm_gbs"] * 1e9) >= case.flops / (peaks["bf16_tflops"] * 1e12)
-    per_launch_s = main_res["_per_launch_ms"] * 1e-3
-    if hbm_bound:
-        achieved = case.bytes / max(1, round(main_res["launches_per_step"])) / per_launch_s / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"]}
-    else:
-        achieved = case.flops / max(1, round(main_res["launches_per_step"])) / per_launch_s / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
-    roof["traffic"] = ncu_traffic(args.workload)
-    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    roof["tensor_frac"] = main_res["tensor_frac"]
-    roof["hbm_frac"] = main_res["hbm_frac"]
-    roof["attainable_frac"] = main_res["attainable_frac"]
+    roof = roofline(case, main_res["kernel_ms"], mean_ms, peaks, peak_src, ncu_traffic(args.workload))
 
     if rank == 0:
         line = {

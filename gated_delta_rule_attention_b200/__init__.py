@@ -78,6 +78,11 @@ def library():
     lib.la_version.restype = i
     lib.la_kernel_launches.argtypes = []
     lib.la_kernel_launches.restype = ctypes.c_ulonglong
+    if hasattr(lib, "la_launch_timing"):   # diagnostic hook, absent from older builds
+        lib.la_launch_timing.argtypes = [i]
+        lib.la_launch_timing.restype = i
+        lib.la_launch_times.argtypes = [ctypes.POINTER(ctypes.c_float), i]
+        lib.la_launch_times.restype = i
     _lib = lib
     return lib
 
@@ -89,6 +94,21 @@ def version() -> int:
 def kernel_launches() -> int:
     """Kernels the library has enqueued in this process so far."""
     return int(library().la_kernel_launches())
+
+
+def launch_timing(enable: bool) -> None:
+    """Turn per-launch device timing on or off (la_launch_timing)."""
+    _check(library().la_launch_timing(1 if enable else 0), "la_launch_timing")
+
+
+def launch_times(max_n: int = 16) -> list:
+    """Device durations (ms) of the launches of the last call, in launch order
+    (la_launch_times); empty while timing is off."""
+    buf = (ctypes.c_float * max_n)()
+    n = library().la_launch_times(buf, max_n)
+    if n < 0:
+        raise RuntimeError("la_launch_times failed")
+    return [float(buf[j]) for j in range(n)]
 
 
 def _ptr(t):

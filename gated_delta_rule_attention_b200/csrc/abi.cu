@@ -69,6 +69,7 @@ extern "C" la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H
                                   const float *gate, const float *beta, float *state, float *z,
                                   void *o, int chunk, unsigned flags, void *workspace,
                                   size_t workspace_bytes, void *stream) {
+    timer_reset();
     if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_GATED_DELTA) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || T < 0) return LA_ERR_INVALID_ARG;
@@ -129,6 +130,7 @@ extern "C" la_status_t la_decode_step(la_mode_t mode, la_dtype_t dtype, int N, i
                                       int d_v, const void *q, const void *k, const void *v,
                                       const float *gate, const float *beta, float *state,
                                       float *z, void *o, void *stream) {
+    timer_reset();
     if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_GATED_DELTA) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     if (N < 1 || H < 1) return LA_ERR_INVALID_ARG;

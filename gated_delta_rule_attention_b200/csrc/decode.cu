@@ -156,8 +156,10 @@ cudaError_t launch_mode(const DecodeArgs &a) {
     IO *o = static_cast<IO *>(a.o);
 #define LA_DECODE_CASE(DKc, DVc)                                                            \
     if (a.dk == DKc && a.dv == DVc) {                                                       \
+        timer_begin(a.stream);                                                              \
         decode_kernel<MODE, DKc, DVc, IO><<<grid, kDecodeThreads, 0, a.stream>>>(            \
             q, k, v, a.gate, a.beta, a.state, a.z, o);                                      \
+        timer_end(a.stream);                                                                \
         note_launches(1);                                                                   \
         return cudaGetLastError();                                                          \
     }

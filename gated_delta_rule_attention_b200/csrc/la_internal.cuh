@@ -19,6 +19,13 @@ unsigned *device_error_word();   // address on the current device, or nullptr on
 // Counts kernels enqueued by the library (la_kernel_launches()).
 void note_launches(unsigned n);
 
+// Optional per-launch device timing (la_launch_timing()): every kernel launch is
+// bracketed by timer_begin / timer_end on its stream; each entry point calls
+// timer_reset() first.  All three do nothing while timing is disabled.
+void timer_reset();
+void timer_begin(cudaStream_t s);
+void timer_end(cudaStream_t s);
+
 struct PrefillArgs {
     int mode;           // la_mode_t
     int dtype;          // la_dtype_t

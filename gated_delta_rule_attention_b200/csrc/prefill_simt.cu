@@ -206,10 +206,12 @@ cudaError_t launch_one(const PrefillArgs &a) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)L::kBytes);
     if (err != cudaSuccess) return err;
+    timer_begin(a.stream);
     kern<<<(unsigned)((size_t)a.B * a.H), kSimtThreads, L::kBytes, a.stream>>>(
         a.T, static_cast<const IO *>(a.q), static_cast<const IO *>(a.k),
         static_cast<const IO *>(a.v), a.gate, a.beta, a.state, a.z, static_cast<IO *>(a.o),
         a.init_state ? 1 : 0);
+    timer_end(a.stream);
     note_launches(1);
     return cudaGetLastError();
 }

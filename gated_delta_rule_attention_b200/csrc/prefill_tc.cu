@@ -1764,14 +1764,21 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                 float v[16];
                 tmem_ld_pair16(tl + kColGE + 64 * (j & 1) + 32 * h, v);
                 const int c0 = 32 * h + 16 * hi;
+                // pack once to bf16 (the MMA operand) and sum the packed values, so that the
+                // denominators use exactly the weights A V is formed with
+                uint32_t pk[8];
                 float rs = 0.f;
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float a = (c0 + k <= i) ? __bfloat162float(__float2bfloat16_rn(v[k])) : 0.f;
-                    rs += a;
-                    v[k] = a;
+                for (int k = 0; k < 16; k += 2) {
+                    const uint32_t w = pack_bf16x2((c0 + k <= i) ? v[k] : 0.f,
+                                                   (c0 + k + 1 <= i) ? v[k + 1] : 0.f);
+                    pk[k >> 1] = w;
+                    const float2 f = unpack_bf16x2(w);
+                    rs += f.x + f.y;
                 }
-                st_row_bf16x16(sb + Y::kA + (j & 1) * 8192, i, c0 >> 3, v);
+                const uint32_t at = sb + Y::kA + (j & 1) * 8192;
+                sts128(at + sw128_off(i, c0 >> 3), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+                sts128(at + sw128_off(i, (c0 >> 3) + 1), make_uint4(pk[4], pk[5], pk[6], pk[7]));
                 rs += __shfl_xor_sync(0xffffffffu, rs, 16);
                 if (hi == 0) sm->part[j & 7][h][i] = rs;
                 fence_async_smem();
@@ -1988,19 +1995,25 @@ cudaError_t launch_kind(const TcParams &p, int grid, cudaStream_t stream) {
         e = cudaFuncSetAttribute(prefill_tc_kernel<2, KIND>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Lay<2>::kBytes);
         if (e != cudaSuccess) return e;
+        timer_begin(stream);
         prefill_tc_kernel<2, KIND><<<grid, kThreads, Lay<2>::kBytes, stream>>>(p);
+        timer_end(stream);
     } else {
         static_assert(KIND != kTransition, "the transition pass belongs to the delta rule");
         if constexpr (MODE == 0) {
             e = cudaFuncSetAttribute(prefill_elu_kernel<KIND>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, LayE::kBytes);
             if (e != cudaSuccess) return e;
+            timer_begin(stream);
             prefill_elu_kernel<KIND><<<grid, kThreadsE, LayE::kBytes, stream>>>(p);
+            timer_end(stream);
         } else {
             e = cudaFuncSetAttribute(prefill01_kernel<MODE, KIND>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, Lay01::kBytes);
             if (e != cudaSuccess) return e;
+            timer_begin(stream);
             prefill01_kernel<MODE, KIND><<<grid, kThreads01, Lay01::kBytes, stream>>>(p);
+            timer_end(stream);
         }
     }
     note_launches(1);
@@ -2060,13 +2073,17 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
         cudaError_t e = cudaFuncSetAttribute(combine_matrix_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         if (e != cudaSuccess) return e;
+        timer_begin(a.stream);
         combine_matrix_kernel<<<dim3(BH, kD / kCombRows), 256, bytes, a.stream>>>(
             BH, pl.nseg, s_init, nloc, mtr, sst);
+        timer_end(a.stream);
     } else {
         const size_t total = per;
+        timer_begin(a.stream);
         combine_scalar_kernel<<<(unsigned)((total + 255) / 256), 256, 0, a.stream>>>(
             BH, pl.nseg, s_init, (MODE == 0 && a.init_state) ? a.z : nullptr, nloc, zloc, gam, sst,
             zst, MODE);
+        timer_end(a.stream);
     }
     note_launches(1);
     cudaError_t e = cudaGetLastError();

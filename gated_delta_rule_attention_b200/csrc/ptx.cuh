@@ -154,7 +154,6 @@ __device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint
 // tcgen05.wait in the SAME asm statement: the registers are defined (ld) or free (st)
 // only when the statement ends, and the compiler can never reuse them early.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
-    __syncwarp();   // tcgen05.ld / st are warp-collective (.sync.aligned)
     uint32_t *u = reinterpret_cast<uint32_t *>(r);
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32"
@@ -169,7 +168,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
 // Two 16-column loads (e.g. two accumulators) in flight together, one wait.
 __device__ __forceinline__ void tmem_ld16x2(uint32_t ta, float (&a)[16], uint32_t tb,
                                             float (&b)[16]) {
-    __syncwarp();   // tcgen05.ld / st are warp-collective (.sync.aligned)
     uint32_t *u = reinterpret_cast<uint32_t *>(a);
     uint32_t *w = reinterpret_cast<uint32_t *>(b);
     asm volatile(
@@ -188,7 +186,6 @@ __device__ __forceinline__ void tmem_ld16x2(uint32_t ta, float (&a)[16], uint32_
 }
 // 32 and 64 consecutive columns per thread, one wait.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
-    __syncwarp();   // tcgen05.ld / st are warp-collective (.sync.aligned)
     uint32_t *u = reinterpret_cast<uint32_t *>(r);
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
@@ -198,7 +195,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
         : "memory");
 }
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&r)[64]) {
-    __syncwarp();   // tcgen05.ld / st are warp-collective (.sync.aligned)
     uint32_t *u = reinterpret_cast<uint32_t *>(r);
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
@@ -212,7 +208,6 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&r)[64]) {
 // [col+N, col+2N).  This is the natural access to an M=64 accumulator, whose rows sit in
 // lanes 0-15 of each 32-lane quarter: every thread of the warp gets useful data.
 __device__ __forceinline__ void tmem_ld_pair16(uint32_t taddr, float (&r)[16]) {
-    __syncwarp();   // tcgen05.ld / st are warp-collective (.sync.aligned)
     uint32_t *u = reinterpret_cast<uint32_t *>(r);
     asm volatile(
         "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 16;\n\t"
@@ -222,7 +217,6 @@ __device__ __forceinline__ void tmem_ld_pair16(uint32_t taddr, float (&r)[16]) {
         : "memory");
 }
 __device__ __forceinline__ void tmem_ld_pair32(uint32_t taddr, float (&r)[32]) {
-    __syncwarp();   // tcgen05.ld / st are warp-collective (.sync.aligned)
     uint32_t *u = reinterpret_cast<uint32_t *>(r);
     asm volatile(
         "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;\n\t"
@@ -232,7 +226,6 @@ __device__ __forceinline__ void tmem_ld_pair32(uint32_t taddr, float (&r)[32]) {
         : "memory");
 }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&r)[16]) {
-    __syncwarp();   // tcgen05.ld / st are warp-collective (.sync.aligned)
     const uint32_t *u = reinterpret_cast<const uint32_t *>(r);
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32"
@@ -290,9 +283,11 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
         : "memory");
 }
 
-// Named barrier over `count` threads (a multiple of 32) of the CTA.
+// Named barrier over `count` threads (a multiple of 32) of the CTA.  bar.sync and bar.red
+// are warp-aligned, as are tcgen05.ld / st: callers reach them with converged warps (every
+// divergent region before them is a structured if, which the compiler reconverges at its
+// end; an explicit __syncwarp there measured ~10 % slower in the modes-1 prefill).
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
-    __syncwarp();   // bar.sync is warp-aligned: the warp must arrive converged
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
@@ -300,7 +295,6 @@ __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
 // gets the same answer, so a decision taken on it (e.g. to abandon a loop) is uniform.
 __device__ __forceinline__ bool named_sync_any(uint32_t id, uint32_t count, bool pred) {
     uint32_t r;
-    __syncwarp();
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"

@@ -171,6 +171,20 @@ int la_version(void);
  * threads), a monotonically increasing diagnostic counter. */
 unsigned long long la_kernel_launches(void);
 
+/* Per-launch device timing, a measurement aid with no counterpart in the pages.
+ * la_launch_timing(1) makes every later call of la_prefill, la_prefill_noalloc and
+ * la_decode_step bracket each kernel it enqueues with two CUDA events recorded on the
+ * call's stream (at most 16 launches per call are timed); la_launch_timing(0) turns it
+ * off (the default).  Enabling adds two event records per launch.
+ *
+ * la_launch_times(ms, max_n) waits for the last timed launch of the most recent call,
+ * writes the device duration of each of its first max_n launches, in milliseconds and
+ * launch order, to the HOST array ms, and returns how many it wrote: 0 when timing is
+ * off or the call launched nothing, -1 on a null ms, a negative max_n or a CUDA error.
+ * The state is process-wide: calls from several threads at once interleave. */
+la_status_t la_launch_timing(int enable);
+int la_launch_times(float *ms, int max_n);
+
 #ifdef __cplusplus
 }
 #endif

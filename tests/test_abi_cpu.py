@@ -104,3 +104,16 @@ def test_host_pointers_are_rejected(lib):
     p = buf.ctypes.data_as(ctypes.c_void_p)
     st = lib.la_decode_step(1, 0, 1, 1, 64, 64, p, p, p, None, None, p, None, p, None)
     assert st == 1
+
+
+def test_launch_timing_without_launches(lib):
+    """The timing hook answers without touching a device while nothing was launched."""
+    import ctypes
+    lib.la_launch_times.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    buf = (ctypes.c_float * 4)()
+    assert lib.la_launch_timing(1) == 0
+    assert lib.la_launch_times(ctypes.cast(buf, ctypes.c_void_p), 4) == 0
+    assert lib.la_launch_times(None, 4) == -1
+    assert lib.la_launch_times(ctypes.cast(buf, ctypes.c_void_p), -1) == -1
+    assert lib.la_launch_timing(0) == 0
+    assert lib.la_launch_times(ctypes.cast(buf, ctypes.c_void_p), 4) == 0

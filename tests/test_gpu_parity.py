@@ -175,3 +175,28 @@ def test_decode_steps(la, mode, dtype, d):
         assert slice_rel_err(f64(S), Sr) <= TOL[dtype], t
         if mode == 0:
             assert slice_rel_err(f64(z), zr) <= TOL[dtype]
+
+
+# ----------------------------------------------------------------------------------
+# per-launch timing hook
+# ----------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_launch_timing_reports_every_launch(la, mode):
+    """With timing on, one device duration per kernel the call enqueued (the segmented
+    prefill: local pass(es), combine, outputs), all positive; off again, nothing."""
+    w = small(mode, torch.bfloat16, 128, 4096, B=1, H=2)
+    inp = W.prefill_inputs(w, device="cuda")
+    la.launch_timing(True)
+    try:
+        n0 = la.kernel_launches()
+        la.prefill(inp["q"], inp["k"], inp["v"], mode=mode, gate=inp["gate"], beta=inp["beta"])
+        n = la.kernel_launches() - n0
+        times = la.launch_times()
+    finally:
+        la.launch_timing(False)
+    la.check_status()
+    assert n >= 3 and len(times) == n
+    assert all(t > 0 for t in times)
+    la.prefill(inp["q"], inp["k"], inp["v"], mode=mode, gate=inp["gate"], beta=inp["beta"])
+    assert la.launch_times() == []
