@@ -1409,9 +1409,9 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
 // M=64 buffers, so that the outputs of chunk c are read while chunk c+1 is computed).
 // Shared memory holds two rings filled by TMA: K and Q tiles, four deep, because the
 // preparation warps and Q K^T need them early; V tiles, two deep, needed only by the
-// products of the chunk.  The outputs of a chunk are staged in the Q tile of its own K/Q
-// slot, dead once the products are done, and written by TMA; the slot is released when
-// that store has read it.  G is formed two chunks ahead, after the products of the
+// products of the chunk.  The outputs of a chunk are staged in its own V slot, dead once
+// the products are done, and written by TMA; that slot is released when the store has read
+// it, while the K/Q slot is released as soon as the products and the A-epilogue are done.  G is formed two chunks ahead, after the products of the
 // current chunk, so that the tensor core runs the state chain products(c) -> state copy
 // -> products(c+1) without waiting behind it.
 // The tensor core commits once after Q S^T and dS (the epilogue may then copy the new
@@ -1480,7 +1480,7 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm->full_v[b], 1);
-            mbar_init(&sm->empty_v[b], 1);
+            mbar_init(&sm->empty_v[b], kOut ? 2 : 1);   // tensor core (+ output store)
             mbar_init(&sm->g_done[b], 1);
             mbar_init(&sm->a_ready[b], 1);
             mbar_init(&sm->o_free[b], 1);
@@ -1784,7 +1784,10 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                 fence_async_smem();
                 tc_fence_before();
                 epi_sync();
-                if (e == 0) mbar_arrive(&sm->a_ready[j & 1]);
+                if (e == 0) {
+                    mbar_arrive(&sm->a_ready[j & 1]);
+                    mbar_arrive(&sm->empty_kq[s]);   // the epilogue is done with this K/Q slot
+                }
                 return true;
             };
 
@@ -1823,7 +1826,7 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                     w_ok = mbar_wait(&sm->mma2_done[b], (c >> 1) & 1, abort, p.err);
                     if (c > 0) {   // the outputs of chunk c-1 have left their staging tile
                         tma_store_wait_read<0>();
-                        mbar_arrive(&sm->empty_kq[(c - 1) % NKQ]);
+                        mbar_arrive(&sm->empty_v[(c - 1) % NV]);
                     }
                 }
                 if (named_sync_any(1, kEpi, !w_ok)) break;
@@ -1841,8 +1844,8 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                     tmem_ld_pair32(tl + kColOE + 128 * b + 64 * h, v);
 #pragma unroll
                     for (int k = 0; k < 32; ++k) v[k] *= scale;
-                    if (has) {   // Q tile of this chunk's K/Q slot: [Q0 | Q1] at +8 KB, +24 KB
-                        const uint32_t ost = sb + Y::kKQ + (c % NKQ) * 32768 + 8192 + h * 16384;
+                    if (has) {   // this chunk's V slot: [V0 | V1] -> [O0 | O1], 8 KB each
+                        const uint32_t ost = sb + Y::kV + (c % NV) * 16384 + h * 8192;
                         st_row_bf16x16(ost, t, 4 * hi, v);
                         st_row_bf16x16(ost, t, 4 * hi + 2, v + 16);
                     }
@@ -1852,9 +1855,9 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                 epi_sync();
                 if (e == 0) {
                     mbar_arrive(&sm->o_free[b]);
-                    const uint32_t ost = sb + Y::kKQ + (c % NKQ) * 32768 + 8192;
+                    const uint32_t ost = sb + Y::kV + (c % NV) * 16384;
                     tma_store_3d(&p.to, ost, 0, t0, bh);
-                    tma_store_3d(&p.to, ost + 16384, 64, t0, bh);
+                    tma_store_3d(&p.to, ost + 8192, 64, t0, bh);
                     tma_store_commit();
                 }
             }
@@ -1885,29 +1888,33 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
 }
 
 // ------------------------------------------------------------------ combine kernels
-// modes 0/1: S_start[s+1] = gam_s S_start[s] + N_s;  z_start[s+1] = z_start[s] + zN_s.
-__global__ void combine_scalar_kernel(int BH, int nseg, const float *s_init, const float *z_init,
-                                      const float *nloc, const float *zloc, const float *gam,
-                                      float *sst, float *zst, int mode) {
-    const size_t per = (size_t)kD * kD;
+// modes 0/1: the local pass ran on `f` sub-segments per segment; their local states fold
+// in order into the segment starts, S <- gam_j S + N_j (z <- z + zN_j), and after every
+// f-th sub-segment the start of the next segment is written.  float4 per thread.
+__global__ void combine_scalar_kernel(int BH, int nseg, int f, const float *s_init,
+                                      const float *z_init, const float *nloc, const float *zloc,
+                                      const float *gam, float *sst, float *zst, int mode) {
+    const size_t per4 = (size_t)kD * kD / 4;
+    const size_t total4 = (size_t)BH * per4;
     const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const size_t total = (size_t)BH * per;
-    if (idx < total) {
-        const int bh = (int)(idx / per);
-        float sv = s_init ? s_init[idx] : 0.f;
-        sst[idx] = sv;
-        for (int s = 0; s + 1 < nseg; ++s) {
-            const float g = (mode == 1) ? gam[(size_t)s * BH + bh] : 1.f;
-            sv = fmaf(g, sv, nloc[(size_t)s * total + idx]);
-            sst[(size_t)(s + 1) * total + idx] = sv;
+    const int nsub = (nseg - 1) * f;
+    if (idx < total4) {
+        const int bh = (int)(idx / per4);
+        float4 sv = s_init ? reinterpret_cast<const float4 *>(s_init)[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4 *>(sst)[idx] = sv;
+        for (int j = 0; j < nsub; ++j) {
+            const float g = (mode == 1) ? gam[(size_t)j * BH + bh] : 1.f;
+            const float4 n = reinterpret_cast<const float4 *>(nloc)[(size_t)j * total4 + idx];
+            sv = make_float4(fmaf(g, sv.x, n.x), fmaf(g, sv.y, n.y), fmaf(g, sv.z, n.z), fmaf(g, sv.w, n.w));
+            if ((j + 1) % f == 0) reinterpret_cast<float4 *>(sst)[(size_t)((j + 1) / f) * total4 + idx] = sv;
         }
     }
     if (mode == 0 && idx < (size_t)BH * kD) {
         float zv = z_init ? z_init[idx] : 0.f;
         zst[idx] = zv;
-        for (int s = 0; s + 1 < nseg; ++s) {
-            zv += zloc[(size_t)s * BH * kD + idx];
-            zst[(size_t)(s + 1) * BH * kD + idx] = zv;
+        for (int j = 0; j < nsub; ++j) {
+            zv += zloc[(size_t)j * BH * kD + idx];
+            if ((j + 1) % f == 0) zst[(size_t)((j + 1) / f) * BH * kD + idx] = zv;
         }
     }
 }
@@ -1962,6 +1969,7 @@ __global__ void __launch_bounds__(256) combine_matrix_kernel(int BH, int nseg, c
 // ------------------------------------------------------------------ host side
 struct Plan {
     int nseg, seg_len;
+    int sub;   // modes 0/1: the local pass runs on `sub` equal sub-segments per segment
 };
 
 Plan plan_for(int mode, int BH, int T) {
@@ -1974,17 +1982,26 @@ Plan plan_for(int mode, int BH, int T) {
     Plan pl;
     pl.seg_len = chunks_per_seg * kC;
     pl.nseg = (T + pl.seg_len - 1) / pl.seg_len;
+    // The local pass covers segments 0 .. nseg-2 only; split them further so that it too
+    // fills the SMs (sub-segments of at least four chunks, dividing the segment evenly).
+    pl.sub = 1;
+    if (mode != 2 && pl.nseg > 1) {
+        int f = sms / (BH * (pl.nseg - 1));
+        while (f > 1 && (chunks_per_seg % f != 0 || chunks_per_seg / f < 4)) --f;
+        pl.sub = std::max(1, f);
+    }
     return pl;
 }
 
 size_t workspace_floats(int mode, int BH, const Plan &pl) {
     if (pl.nseg <= 1) return 0;
     const size_t per = (size_t)BH * kD * kD;
+    const size_t nloc = (size_t)(pl.nseg - 1) * pl.sub;   // local-pass sub-segments
     size_t f = (size_t)pl.nseg * per;                 // segment start states
-    f += (size_t)(pl.nseg - 1) * per;                 // local states
+    f += nloc * per;                                  // local states
     if (mode == 2) f += (size_t)(pl.nseg - 1) * per;  // transitions
-    if (mode == 1) f += (size_t)(pl.nseg - 1) * BH;   // gate products
-    if (mode == 0) f += (size_t)(2 * pl.nseg - 1) * BH * kD;   // z starts + z locals
+    if (mode == 1) f += nloc * BH;                    // gate products
+    if (mode == 0) f += ((size_t)pl.nseg + nloc) * BH * kD;   // z starts + z locals
     return f;
 }
 
@@ -2038,11 +2055,12 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
         p.out_last_only = 1;
         return launch_kind<MODE, kOutput>(p, BH, a.stream);
     }
+    const int nsub = (pl.nseg - 1) * pl.sub;                     // local-pass CTAs per head
     float *sst = ws;
     float *nloc = sst + (size_t)pl.nseg * per;
-    float *mtr = nloc + (size_t)(pl.nseg - 1) * per;            // mode 2
-    float *gam = nloc + (size_t)(pl.nseg - 1) * per;            // mode 1
-    float *zst = nloc + (size_t)(pl.nseg - 1) * per;            // mode 0
+    float *mtr = nloc + (size_t)nsub * per;                      // mode 2 (sub = 1)
+    float *gam = nloc + (size_t)nsub * per;                      // mode 1
+    float *zst = nloc + (size_t)nsub * per;                      // mode 0
     float *zloc = zst + (size_t)pl.nseg * BH * kD;
     // pass A: local states (and transitions)
     {
@@ -2054,7 +2072,9 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
         p.z_out_seg = (long long)BH * kD;
         p.gam_out = (MODE == 1) ? gam : nullptr;
         p.out_last_only = 0;
-        cudaError_t e = launch_kind<MODE, kLocal>(p, BH * (pl.nseg - 1), a.stream);
+        p.seg_len = pl.seg_len / pl.sub;
+        p.nseg = nsub;
+        cudaError_t e = launch_kind<MODE, kLocal>(p, BH * nsub, a.stream);
         if (e != cudaSuccess) return e;
         if constexpr (MODE == 2) {
             TcParams q = base;
@@ -2078,11 +2098,11 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
             BH, pl.nseg, s_init, nloc, mtr, sst);
         timer_end(a.stream);
     } else {
-        const size_t total = per;
+        const size_t total4 = per / 4;
         timer_begin(a.stream);
-        combine_scalar_kernel<<<(unsigned)((total + 255) / 256), 256, 0, a.stream>>>(
-            BH, pl.nseg, s_init, (MODE == 0 && a.init_state) ? a.z : nullptr, nloc, zloc, gam, sst,
-            zst, MODE);
+        combine_scalar_kernel<<<(unsigned)((total4 + 255) / 256), 256, 0, a.stream>>>(
+            BH, pl.nseg, pl.sub, s_init, (MODE == 0 && a.init_state) ? a.z : nullptr, nloc, zloc, gam,
+            sst, zst, MODE);
         timer_end(a.stream);
     }
     note_launches(1);

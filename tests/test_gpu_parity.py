@@ -200,3 +200,11 @@ def test_launch_timing_reports_every_launch(la, mode):
     assert all(t > 0 for t in times)
     la.prefill(inp["q"], inp["k"], inp["v"], mode=mode, gate=inp["gate"], beta=inp["beta"])
     assert la.launch_times() == []
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_prefill_subsegmented_local_pass(la, mode):
+    """60 heads: two segments per head whose local pass runs on two sub-segments each,
+    folded by the combine kernel; ragged tail in the last segment."""
+    w = small(mode, torch.bfloat16, 128, 2000, B=4, H=15, seed=321)
+    run_and_compare(la, w)
