@@ -86,7 +86,54 @@ struct TcParams {
     int out_last_only;
     int T, BH, seg_len, nseg;
     unsigned *err;
+    // s_in_mode 3 (modes 0/1, outputs pass): the start state of segment `seg` is folded in
+    // the kernel from fold_init (nullable: zero) and the local states of the first
+    // seg * fold_sub sub-segments, S <- gam_j S + N_j (z <- z + zN_j), instead of being
+    // read from a start state that a combine kernel wrote.
+    const float *fold_init, *fold_zinit, *fold_loc, *fold_zloc, *fold_gam;
+    int fold_sub;
 };
+
+// Start state S[row][c0 .. c0 + 15] of segment `seg` of head bh (modes 0/1).
+__device__ __forceinline__ void start_state16(const TcParams &p, int seg, int bh, int row, int c0,
+                                              float (&v)[16]) {
+    const size_t off = (size_t)bh * 128 * 128 + (size_t)row * 128 + c0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = 0.f;
+    const float *src = nullptr;
+    if (p.s_in_mode == 1) src = p.s_in + (size_t)seg * p.s_in_seg + off;
+    if (p.s_in_mode == 3) src = p.fold_init ? p.fold_init + off : nullptr;
+    if (src) {
+#pragma unroll
+        for (int k = 0; k < 16; k += 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(src + k);
+            v[k] = x.x; v[k + 1] = x.y; v[k + 2] = x.z; v[k + 3] = x.w;
+        }
+    }
+    if (p.s_in_mode == 3) {
+        const size_t per = (size_t)p.BH * 128 * 128;
+        for (int j = 0; j < seg * p.fold_sub; ++j) {
+            const float g = p.fold_gam ? p.fold_gam[(size_t)j * p.BH + bh] : 1.f;
+            const float *n = p.fold_loc + (size_t)j * per + off;
+#pragma unroll
+            for (int k = 0; k < 16; k += 4) {
+                const float4 x = *reinterpret_cast<const float4 *>(n + k);
+                v[k] = fmaf(g, v[k], x.x);
+                v[k + 1] = fmaf(g, v[k + 1], x.y);
+                v[k + 2] = fmaf(g, v[k + 2], x.z);
+                v[k + 3] = fmaf(g, v[k + 3], x.w);
+            }
+        }
+    }
+}
+// Start value of z[col] of segment `seg` of head bh (mode 0).
+__device__ __forceinline__ float start_z(const TcParams &p, int seg, int bh, int col) {
+    if (p.s_in_mode == 1) return p.z_in ? p.z_in[(size_t)seg * p.z_in_seg + (size_t)bh * 128 + col] : 0.f;
+    if (p.s_in_mode != 3) return 0.f;
+    float z = p.fold_zinit ? p.fold_zinit[(size_t)bh * 128 + col] : 0.f;
+    for (int j = 0; j < seg * p.fold_sub; ++j) z += p.fold_zloc[((size_t)j * p.BH + bh) * 128 + col];
+    return z;
+}
 
 struct Small {
     uint64_t full[3], empty[3];
@@ -1207,11 +1254,13 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
 
         float Sr[64];
         {
-            const float *src = nullptr;
-            if (p.s_in_mode == 1)
-                src = p.s_in + (size_t)seg * p.s_in_seg + (size_t)bh * kD * kD + (size_t)row * kD;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) Sr[j] = src ? src[64 * h + j] : 0.f;
+            for (int g = 0; g < 4; ++g) {
+                float v[16];
+                start_state16(p, seg, bh, row, 64 * h + 16 * g, v);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) Sr[16 * g + k] = v[k];
+            }
             if (kOut) {
 #pragma unroll
                 for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
@@ -1625,10 +1674,7 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
         const int ch = lane & 7, rg = lane >> 3;
         float zc = 0.f;                        // z of column pe (pe < 128)
         if (pe < kD) {
-            const float *zs = (p.s_in_mode == 1 && p.z_in)
-                                  ? p.z_in + (size_t)seg * p.z_in_seg + (size_t)bh * kD
-                                  : nullptr;
-            zc = zs ? zs[pe] : 0.f;
+            zc = start_z(p, seg, bh, pe);
             sm->zsm[pe] = zc;
         }
         // Warp pw takes column half pw >> 2 and rows 16 (pw & 3) + 4 rg + i (i < 4); lane
@@ -1733,14 +1779,10 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
 
         // initial state into TMEM (and its bf16 copy for the first Q S^T)
         {
-            const float *src = nullptr;
-            if (p.s_in_mode == 1)
-                src = p.s_in + (size_t)seg * p.s_in_seg + (size_t)bh * kD * kD + (size_t)row * kD;
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
                 float v[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) v[k] = src ? src[64 * h + 16 * g + k] : 0.f;
+                start_state16(p, seg, bh, row, 64 * h + 16 * g, v);
                 tmem_st16(tl + kColSE + 64 * h + 16 * g, v);
                 if (kOut) st_row_bf16x16(sbf + h * 16384, row, 2 * g, v);
             }
@@ -2084,6 +2126,28 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
             q.out_last_only = 0;
             e = launch_kind<MODE, kTransition>(q, BH * (pl.nseg - 1), a.stream);
             if (e != cudaSuccess) return e;
+        }
+    }
+    // Outputs pass.  Without an initial state and with few sub-segments per head, each
+    // outputs CTA folds its own start state from the local states (no combine launch).
+    // With an initial state the starts are first copied into the workspace by the combine
+    // kernel: the outputs pass overwrites the caller's state with the final one.
+    if constexpr (MODE != 2) {
+        if (!a.init_state && nsub <= 4) {
+            TcParams p = base;
+            p.s_in_mode = 3;
+            p.fold_init = nullptr;
+            p.fold_zinit = nullptr;
+            p.fold_loc = nloc;
+            p.fold_zloc = (MODE == 0) ? zloc : nullptr;
+            p.fold_gam = (MODE == 1) ? gam : nullptr;
+            p.fold_sub = pl.sub;
+            p.s_out = a.state;
+            p.s_out_seg = 0;
+            p.z_out = a.z;
+            p.z_out_seg = 0;
+            p.out_last_only = 1;
+            return launch_kind<MODE, kOutput>(p, BH * pl.nseg, a.stream);
         }
     }
     // combine: segment start states

@@ -203,8 +203,12 @@ def test_launch_timing_reports_every_launch(la, mode):
 
 
 @pytest.mark.parametrize("mode", [0, 1])
-def test_prefill_subsegmented_local_pass(la, mode):
-    """60 heads: two segments per head whose local pass runs on two sub-segments each,
-    folded by the combine kernel; ragged tail in the last segment."""
-    w = small(mode, torch.bfloat16, 128, 2000, B=4, H=15, seed=321)
-    run_and_compare(la, w)
+@pytest.mark.parametrize("B,H,T", [(4, 15, 2000), (1, 4, 4096)])
+@pytest.mark.parametrize("init", [0.0, 0.05])
+def test_prefill_segment_starts(la, mode, B, H, T, init):
+    """Segmented prefill, both ways of forming segment starts.  60 heads x 2000 tokens:
+    two segments whose local pass runs on two sub-segments each (ragged tail in the last);
+    without an initial state the outputs pass folds the starts itself, with one the
+    combine kernel does.  4 heads x 4096 tokens: 16 segments, always the combine kernel."""
+    w = small(mode, torch.bfloat16, 128, T, B=B, H=H, seed=321)
+    run_and_compare(la, w, init_std=init)
