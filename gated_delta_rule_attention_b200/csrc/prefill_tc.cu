@@ -1829,6 +1829,10 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                 if (e == 0) {
                     mbar_arrive(&sm->a_ready[j & 1]);
                     mbar_arrive(&sm->empty_kq[s]);   // the epilogue is done with this K/Q slot
+                    if (j >= 2) {   // the outputs of chunk j-2, stored a whole A-epilogue ago,
+                        tma_store_wait_read<0>();    // have left their V slot: refill it
+                        mbar_arrive(&sm->empty_v[(j - 2) % NV]);
+                    }
                 }
                 return true;
             };
@@ -1866,10 +1870,7 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                 // ---- outputs of chunk c: row t = r64, columns 64 h + 32 hi + [0, 32)
                 if (e == 0) {
                     w_ok = mbar_wait(&sm->mma2_done[b], (c >> 1) & 1, abort, p.err);
-                    if (c > 0) {   // the outputs of chunk c-1 have left their staging tile
-                        tma_store_wait_read<0>();
-                        mbar_arrive(&sm->empty_v[(c - 1) % NV]);
-                    }
+                    tma_store_wait_read<0>();   // (normally long done) before the next staging
                 }
                 if (named_sync_any(1, kEpi, !w_ok)) break;
                 tc_fence_after();
