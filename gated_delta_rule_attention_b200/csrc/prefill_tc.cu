@@ -172,6 +172,22 @@ __device__ __forceinline__ uint64_t dk(uint32_t addr) { return sdesc_sw128(addr,
 __device__ __forceinline__ uint64_t dmn(uint32_t addr, uint32_t lbo) {
     return sdesc_sw128(addr, lbo, 1024);
 }
+
+// D (+)= A B over NK steps of K = 16, issued back to back.  The operand descriptors are
+// built once; each step adds its offset to the start-address field (16-byte units), a
+// compile-time constant once the loop is unrolled.  A K-major 128B-swizzled operand
+// advances 32 bytes per step inside a 64-column half and jumps to the next half
+// (KHALF bytes further) every four steps; an MN-major one advances 8 K rows = 2048 bytes.
+template <int NK, bool A_KMAJ, bool B_KMAJ, uint32_t A_KHALF = 16384, uint32_t B_KHALF = 16384>
+__device__ __forceinline__ void mma_chain(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, bool accumulate_first) {
+#pragma unroll
+    for (int ks = 0; ks < NK; ++ks) {
+        const uint64_t ao = A_KMAJ ? (((ks >> 2) * A_KHALF + (ks & 3) * 32) >> 4) : (uint64_t)(ks * 128);
+        const uint64_t bo = B_KMAJ ? (((ks >> 2) * B_KHALF + (ks & 3) * 32) >> 4) : (uint64_t)(ks * 128);
+        mma_bf16_ss(d_tmem, a_desc + ao, b_desc + bo, idesc, accumulate_first || ks > 0);
+    }
+}
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -470,30 +486,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 tc_fence_after();
                 if (kNeedG) {
                     // G = [K; Q] K^T   (M=128, N=64, K=128)
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16_ss(tm + kColG, dk(st + off), dk(st + off), id_g, ks > 0);
-                    }
+                    mma_chain<8, true, true>(tm + kColG, dk(st), dk(st), id_g, false);
                     mma_commit(&sm->g_done);
                 }
                 if constexpr (MODE == 2) {
                     if (!mbar_wait(&sm->tt_ready, par, abort, p.err)) break;
                     tc_fence_after();
-                    for (int ks = 0; ks < 4; ++ks) {
-                        if (kNeedV)   // U^T = V^T (T diag b)^T
-                            mma_bf16_ss(tm + kColU, dmn(st + 32768 + ks * 2048, 8192),
-                                        dk(tp + ks * 32), id_uw, ks > 0);
-                        // W^T = K^T (T diag(b g))^T
-                        mma_bf16_ss(tm + kColW, dmn(st + ks * 2048, 16384), dk(tpp + ks * 32),
-                                    id_uw, ks > 0);
-                    }
+                    if (kNeedV)   // U^T = V^T (T diag b)^T
+                        mma_chain<4, false, true>(tm + kColU, dmn(st + 32768, 8192), dk(tp), id_uw, false);
+                    // W^T = K^T (T diag(b g))^T
+                    mma_chain<4, false, true>(tm + kColW, dmn(st, 16384), dk(tpp), id_uw, false);
                     mma_commit(&sm->ut_done);
                     if (!mbar_wait(&sm->w_ready, par, abort, p.err)) break;
                     if (!mbar_wait(&sm->s_ready, par, abort, p.err)) break;
                     tc_fence_after();
-                    for (int ks = 0; ks < 8; ++ks)   // Y = S W^T
-                        mma_bf16_ss(tm + kColY, dk(sbf + (ks >> 2) * 16384 + (ks & 3) * 32),
-                                    dmn(wt + ks * 2048, 8192), id_y, ks > 0);
+                    // Y = S W^T
+                    mma_chain<8, true, false>(tm + kColY, dk(sbf), dmn(wt, 8192), id_y, false);
                     mma_commit(&sm->py_done);
                     if (!mbar_wait(&sm->e_ready, par, abort, p.err)) break;
                     tc_fence_after();
@@ -506,22 +514,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     // O = Q~ S^T (+) A V  or  A E     (M=64, N=128); mode 1 keeps Q S^T
                     // in its own accumulator P and applies diag(g) in the output epilogue
                     const uint32_t dq = (MODE == 1) ? kColP : kColO;
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16_ss(tm + dq, dk(st + 8192 + off), dk(sbf + off), id_o1, ks > 0);
-                    }
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t b2 = (MODE == 2) ? dk(et + ks * 32)
-                                                        : dmn(st + 32768 + ks * 2048, 8192);
-                        mma_bf16_ss(tm + kColO, dk(at + ks * 32), b2, id_o2, MODE != 1 || ks > 0);
-                    }
+                    mma_chain<8, true, true>(tm + dq, dk(st + 8192), dk(sbf), id_o1, false);
+                    if constexpr (MODE == 2)
+                        mma_chain<4, true, true>(tm + kColO, dk(at), dk(et), id_o2, true);
+                    else
+                        mma_chain<4, true, false>(tm + kColO, dk(at), dmn(st + 32768, 8192), id_o2, MODE != 1);
                 }
                 // dS = V^T K~ (modes 0/1) or (E^T diag dec) K (mode 2)   (M=128, N=128)
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t a2 = (MODE == 2) ? dk(ept + ks * 32)
-                                                    : dmn(st + 32768 + ks * 2048, 8192);
-                    mma_bf16_ss(tm + kColDS, a2, dmn(st + ks * 2048, 16384), id_ds, ks > 0);
-                }
+                if constexpr (MODE == 2)
+                    mma_chain<4, true, false>(tm + kColDS, dk(ept), dmn(st, 16384), id_ds, false);
+                else
+                    mma_chain<4, false, false>(tm + kColDS, dmn(st + 32768, 8192), dmn(st, 16384), id_ds, false);
                 mma_commit(&sm->mma2_done);
             }
             // nothing may still write TMEM when it is freed
@@ -1032,11 +1035,7 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                     if (!mbar_wait(&sm->prep_done[s], u & 1, abort, p.err)) return false;
                     tc_fence_after();
                     const uint32_t st = sb + s * Y::kStage;
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16_ss(tm + kColG01 + 64 * (j & 1), dk(st + 8192 + off), dk(st + off),
-                                    id_g, ks > 0);
-                    }
+                    mma_chain<8, true, true>(tm + kColG01 + 64 * (j & 1), dk(st + 8192), dk(st), id_g, false);
                     mma_commit(&sm->g_done[j & 1]);
                     return true;
                 };
@@ -1050,16 +1049,11 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                     if (!mbar_wait(&sm->s_ready, c & 1, abort, p.err)) break;
                     tc_fence_after();
                     const uint32_t dq = (MODE == 1) ? kColP01 : kColO01;
-                    for (int ks = 0; ks < 8; ++ks) {   // Q S^T
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16_ss(tm + dq, dk(st + 8192 + off), dk(sbf + off), id_o1, ks > 0);
-                    }
-                    for (int ks = 0; ks < 4; ++ks)     // A V
-                        mma_bf16_ss(tm + kColO01, dk(at + ks * 32), dmn(st + 32768 + ks * 2048, 8192),
-                                    id_o2, MODE != 1 || ks > 0);
-                    for (int ks = 0; ks < 4; ++ks)     // dS = V^T K~
-                        mma_bf16_ss(tm + kColDS, dmn(st + 32768 + ks * 2048, 8192),
-                                    dmn(st + ks * 2048, 16384), id_ds, ks > 0);
+                    mma_chain<8, true, true>(tm + dq, dk(st + 8192), dk(sbf), id_o1, false);   // Q S^T
+                    mma_chain<4, true, false>(tm + kColO01, dk(at), dmn(st + 32768, 8192), id_o2,
+                                              MODE != 1);                                       // A V
+                    mma_chain<4, false, false>(tm + kColDS, dmn(st + 32768, 8192), dmn(st, 16384), id_ds,
+                                               false);                                          // dS = V^T K~
                     mma_commit(&sm->mma2_done);
                     mma_commit(&sm->empty[s]);
                 }
@@ -1071,9 +1065,8 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                     if (!mbar_wait(&sm->prep_done[s], u & 1, abort, p.err)) break;
                     if (c >= 2 && !mbar_wait(&sm->ds_free[b], ((c >> 1) - 1) & 1, abort, p.err)) break;
                     tc_fence_after();
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16_ss(tm + kColDS + 128 * b, dmn(st + 32768 + ks * 2048, 8192),
-                                    dmn(st + ks * 2048, 16384), id_ds, ks > 0);
+                    mma_chain<4, false, false>(tm + kColDS + 128 * b, dmn(st + 32768, 8192), dmn(st, 16384),
+                                               id_ds, false);
                     mma_commit(&sm->ds_done[b]);
                     mma_commit(&sm->empty[s]);
                 }
@@ -1611,11 +1604,7 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                     if (!mbar_wait(&sm->prep_done[s], u & 1, abort, p.err)) return false;
                     tc_fence_after();
                     const uint32_t st = sb + Y::kKQ + s * 32768;
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16_ss(tm + kColGE + 64 * (j & 1), dk(st + 8192 + off), dk(st + off),
-                                    id_g, ks > 0);
-                    }
+                    mma_chain<8, true, true>(tm + kColGE + 64 * (j & 1), dk(st + 8192), dk(st), id_g, false);
                     mma_commit(&sm->g_done[j & 1]);
                     return true;
                 };
@@ -1631,16 +1620,11 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                     if (c >= 2 && !mbar_wait(&sm->o_free[b], ((c >> 1) - 1) & 1, abort, p.err)) break;
                     if (!mbar_wait(&sm->full_v[sv], (c / NV) & 1, abort, p.err)) break;
                     tc_fence_after();
-                    for (int ks = 0; ks < 8; ++ks) {   // phi(Q) S^T
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16_ss(to, dk(st + 8192 + off), dk(sbf + off), id_o1, ks > 0);
-                    }
-                    for (int ks = 0; ks < 4; ++ks)     // S += V^T phi(K)
-                        mma_bf16_ss(tm + kColSE, dmn(vt + ks * 2048, 8192),
-                                    dmn(st + ks * 2048, 16384), id_ds, true);
+                    mma_chain<8, true, true>(to, dk(st + 8192), dk(sbf), id_o1, false);      // phi(Q) S^T
+                    mma_chain<4, false, false>(tm + kColSE, dmn(vt, 8192), dmn(st, 16384), id_ds,
+                                               true);                                     // S += V^T phi(K)
                     mma_commit(&sm->s_done);
-                    for (int ks = 0; ks < 4; ++ks)     // + A V
-                        mma_bf16_ss(to, dk(at + ks * 32), dmn(vt + ks * 2048, 8192), id_o2, true);
+                    mma_chain<4, true, false>(to, dk(at), dmn(vt, 8192), id_o2, true);      // + A V
                     mma_commit(&sm->mma2_done[b]);
                     mma_commit(&sm->empty_kq[s]);
                     mma_commit(&sm->empty_v[sv]);
@@ -1656,9 +1640,7 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                     if (!mbar_wait(&sm->prep_done[s], u & 1, abort, p.err)) break;
                     if (!mbar_wait(&sm->full_v[sv], (c / NV) & 1, abort, p.err)) break;
                     tc_fence_after();
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16_ss(tm + kColSE, dmn(vt + ks * 2048, 8192),
-                                    dmn(st + ks * 2048, 16384), id_ds, true);
+                    mma_chain<4, false, false>(tm + kColSE, dmn(vt, 8192), dmn(st, 16384), id_ds, true);
                     mma_commit(&sm->empty_kq[s]);
                     mma_commit(&sm->empty_v[sv]);
                 }
