@@ -60,8 +60,6 @@ constexpr int kEpi = 256;      // epilogue threads (warps 2-9)
 constexpr uint32_t kTmemCols = 512;
 // TMEM column map
 constexpr uint32_t kColDS = 0, kColG = 128, kColU = 192, kColW = 256, kColY = 320, kColO = 384;
-constexpr uint32_t kColP = 256;   // mode 1: Q S^T kept apart from A V (M=64, 128 columns)
-constexpr float kLog2e = 1.4426950408889634f;
 
 enum Kind { kOutput = 0, kLocal = 1, kTransition = 2 };
 
@@ -137,17 +135,14 @@ __device__ __forceinline__ float start_z(const TcParams &p, int seg, int bh, int
 
 struct Small {
     uint64_t full[3], empty[3];
-    uint64_t prep_done, g_done, a_ready, tt_ready, ut_done, w_ready, py_done, e_ready,
+    uint64_t prep_done, g_done, tt_ready, ut_done, w_ready, py_done, e_ready,
         mma2_done, s_ready, fin;
     uint32_t tmem_base;
     int abort;
     int len[2];
     float lam[2][kC];    // in-chunk inclusive prefix of log2(a), per chunk parity
     float bet[2][kC];
-    float part[4][kC];   // mode 0: row-sum halves, phi(q).z halves
-    float z[kD];
     float scan_tmp[2];
-    float gsum;
 };
 
 // Shared-memory layout (bytes from the 1024-aligned base).
@@ -379,10 +374,10 @@ __device__ void invert_unit_lower(const float *Lm, float *Tm, float *Zs, int e) 
 
 template <int MODE, int KIND>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
+    static_assert(MODE == 2, "this kernel serves the gated delta rule");
     using Y = Lay<MODE>;
     constexpr int NST = Y::kStages;
     constexpr bool kOut = (KIND == kOutput);
-    constexpr bool kNeedG = (MODE == 2) || kOut;
     constexpr bool kNeedV = (KIND != kTransition);
 
     // 128B-swizzled operand tiles need 1024-byte aligned atoms.  The buffer is declared
@@ -411,7 +406,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         mbar_init(&sm->prep_done, 1);
         mbar_init(&sm->g_done, 1);
-        mbar_init(&sm->a_ready, 1);
         mbar_init(&sm->tt_ready, 1);
         mbar_init(&sm->ut_done, 1);
         mbar_init(&sm->w_ready, 1);
@@ -421,7 +415,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         mbar_init(&sm->s_ready, 1);
         mbar_init(&sm->fin, 1);
         sm->abort = 0;
-        sm->gsum = 0.f;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -484,12 +477,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 if (!mbar_wait(&sm->full[s], u & 1, abort, p.err)) break;
                 if (!mbar_wait(&sm->prep_done, par, abort, p.err)) break;
                 tc_fence_after();
-                if (kNeedG) {
+                {
                     // G = [K; Q] K^T   (M=128, N=64, K=128)
                     mma_chain<8, true, true>(tm + kColG, dk(st), dk(st), id_g, false);
                     mma_commit(&sm->g_done);
                 }
-                if constexpr (MODE == 2) {
+                {
                     if (!mbar_wait(&sm->tt_ready, par, abort, p.err)) break;
                     tc_fence_after();
                     if (kNeedV)   // U^T = V^T (T diag b)^T
@@ -505,26 +498,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     mma_commit(&sm->py_done);
                     if (!mbar_wait(&sm->e_ready, par, abort, p.err)) break;
                     tc_fence_after();
-                } else {
-                    if (!mbar_wait(&sm->a_ready, par, abort, p.err)) break;
-                    if (!mbar_wait(&sm->s_ready, par, abort, p.err)) break;
-                    tc_fence_after();
                 }
                 if (kOut) {
-                    // O = Q~ S^T (+) A V  or  A E     (M=64, N=128); mode 1 keeps Q S^T
-                    // in its own accumulator P and applies diag(g) in the output epilogue
-                    const uint32_t dq = (MODE == 1) ? kColP : kColO;
-                    mma_chain<8, true, true>(tm + dq, dk(st + 8192), dk(sbf), id_o1, false);
-                    if constexpr (MODE == 2)
-                        mma_chain<4, true, true>(tm + kColO, dk(at), dk(et), id_o2, true);
-                    else
-                        mma_chain<4, true, false>(tm + kColO, dk(at), dmn(st + 32768, 8192), id_o2, MODE != 1);
+                    // O = Q~ S^T + A E   (M=64, N=128; Q~ = diag(g) Q was scaled in place)
+                    mma_chain<8, true, true>(tm + kColO, dk(st + 8192), dk(sbf), id_o1, false);
+                    mma_chain<4, true, true>(tm + kColO, dk(at), dk(et), id_o2, true);
                 }
-                // dS = V^T K~ (modes 0/1) or (E^T diag dec) K (mode 2)   (M=128, N=128)
-                if constexpr (MODE == 2)
-                    mma_chain<4, true, false>(tm + kColDS, dk(ept), dmn(st, 16384), id_ds, false);
-                else
-                    mma_chain<4, false, false>(tm + kColDS, dmn(st + 32768, 8192), dmn(st, 16384), id_ds, false);
+                // dS = (E^T diag dec) K   (M=128, N=128)
+                mma_chain<4, true, false>(tm + kColDS, dk(ept), dmn(st, 16384), id_ds, false);
                 mma_commit(&sm->mma2_done);
             }
             // nothing may still write TMEM when it is freed
@@ -556,52 +537,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             }
 #pragma unroll
             for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
-            if (MODE == 0 && e < kD) {
-                const float *zs = (p.s_in_mode == 1 && p.z_in)
-                                      ? p.z_in + (size_t)seg * p.z_in_seg + (size_t)bh * kD
-                                      : nullptr;
-                sm->z[e] = zs ? zs[e] : 0.f;
-            }
             fence_async_smem();
             epi_sync();
             if (e == 0) mbar_arrive(&sm->s_ready);
         }
 
-        // ---- chunk prologue: gates, phi (mode 0); releases G's inputs to the MMA
+        // ---- chunk prologue: gates; releases G's inputs to the MMA
         auto prep = [&](int c, GateRaw raw) -> bool {
             const int s = c % NST, u = c / NST;
             if (e < 64) load_gates<MODE>(p, sm, tb, te, c, c & 1, e, raw);
             mbar_wait(&sm->full[s], u & 1, abort, p.err);
             epi_sync();
             if (*abort) return false;
-            if (MODE == 0) {
-                const uint32_t st = sb + s * Y::kStage;
-                const int L = sm->len[c & 1];
-                constexpr int kIt = (kOut ? 4 : 2) * 512 / kEpi;   // chunks per thread
-                uint4 w[kIt];
-#pragma unroll
-                for (int it = 0; it < kIt; ++it) {
-                    const int n = e + kEpi * it;
-                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);   // 0,2 = K; 1,3 = Q
-                    w[it] = lds128(st + region * 8192 + (n & 511) * 16);
-                }
-#pragma unroll
-                for (int it = 0; it < kIt; ++it) {
-                    const int n = e + kEpi * it;
-                    const int region = kOut ? (n >> 9) : ((n >> 9) * 2);
-                    const int r = (n & 511) >> 3;
-                    if ((region & 1) == 0 && r >= L) {
-                        w[it] = make_uint4(0, 0, 0, 0);
-                    } else {
-                        w[it].x = phi_bf16x2(w[it].x);
-                        w[it].y = phi_bf16x2(w[it].y);
-                        w[it].z = phi_bf16x2(w[it].z);
-                        w[it].w = phi_bf16x2(w[it].w);
-                    }
-                    sts128(st + region * 8192 + (n & 511) * 16, w[it]);
-                }
-                fence_async_smem();
-            }
             epi_sync();
             if (e == 0) mbar_arrive(&sm->prep_done);
             return true;
@@ -621,31 +568,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             if (c + 1 < nch && e < 64) next_raw = fetch_gates<MODE>(p, bh, tb, te, c + 1, e);
 
             // ---- A-epilogue: masks and decays of G; operand scaling
-            if (kNeedG) {
-                mbar_wait(&sm->g_done, par, abort, p.err);
-                epi_sync();
-                if (*abort) break;
-                tc_fence_after();
-            }
+            mbar_wait(&sm->g_done, par, abort, p.err);
+            epi_sync();
+            if (*abort) break;
+            tc_fence_after();
             if (q >= 2 && kOut) {
                 // rows i of Q K^T -> A tile, columns j in [32h, 32h + 32)
                 const int i = row - 64;
                 float v[32];
                 tmem_ld32(tl + kColG + 32 * h, v);
                 const float li = lam[i];
-                float rs = 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int jj = 32 * h + j;
-                    float a = 0.f;
-                    if (jj <= i) a = (MODE == 0) ? v[j] : v[j] * ex2(li - lam[jj]);
-                    v[j] = __bfloat162float(__float2bfloat16_rn(a));
-                    rs += v[j];
+                    v[j] = (jj <= i) ? v[j] * ex2(li - lam[jj]) : 0.f;
                 }
                 st_row_bf16x16(sb + Y::kA, i, 4 * h, v);
                 st_row_bf16x16(sb + Y::kA, i, 4 * h + 2, v + 16);
-                if (MODE == 0) sm->part[h][i] = rs;
-            } else if (q < 2 && MODE == 2) {
+            } else if (q < 2) {
                 // rows r of K K^T -> Lm (strictly lower), columns j in [32h, 32h + 32)
                 const int r = row;
                 const float br = sm->bet[buf][r], lr = lam[r];
@@ -656,41 +596,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     const int jj = 32 * h + j;
                     Lm[r * kLmStride + jj] = (jj < r) ? br * ex2(lr - lam[jj]) * v[j] : 0.f;
                 }
-            } else if (q < 2 && MODE == 0 && kOut) {
-                // phi(q_r) . z over d_k half h
-                const int r = row;
-                float qz = 0.f;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 w = lds128(st + 8192 + h * 16384 + sw128_off(r, ch));
-                    const uint32_t *wd = reinterpret_cast<const uint32_t *>(&w);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float2 f = unpack_bf16x2(wd[k]);
-                        qz = fmaf(f.x, sm->z[64 * h + 8 * ch + 2 * k], qz);
-                        qz = fmaf(f.y, sm->z[64 * h + 8 * ch + 2 * k + 1], qz);
-                    }
-                }
-                sm->part[2 + h][r] = qz;
             }
-            if (MODE == 1) {
-                // after G: K <- diag(dec) K in place (operand of dS); each thread owns 4
-                // chunks, loaded together before scaling
-                uint4 wk[4];
-#pragma unroll
-                for (int it = 0; it < 4; ++it) {
-                    const int n = e + kEpi * it;
-                    wk[it] = lds128(st + (n >> 9) * 16384 + (n & 511) * 16);
-                }
-#pragma unroll
-                for (int it = 0; it < 4; ++it) {
-                    const int n = e + kEpi * it;
-                    const int r = (n & 511) >> 3;
-                    sts128(st + (n >> 9) * 16384 + (n & 511) * 16,
-                           scale_bf16x8(wk[it], r < L ? ex2(lamL - lam[r]) : 0.f));
-                }
-            }
-            if (MODE == 2 && kOut) {
+            if (kOut) {
                 // after G: Q <- diag(g) Q in place
                 uint4 wq[4];
 #pragma unroll
@@ -709,9 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             tc_fence_before();
             epi_sync();
 
-            if constexpr (MODE != 2) {
-                if (e == 0) mbar_arrive(&sm->a_ready);
-            } else {
+            {
                 // ---- T = (I + Lm)^-1;  T diag(b), T diag(b g) as bf16 MMA operands
                 invert_unit_lower(Lm, Tm, Zs, e);
                 if (e < 128) {
@@ -786,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             tc_fence_after();
             const bool last = (c + 1 == nch);
             {
-                const float gC = (MODE == 0) ? 1.f : ex2(lamL);
+                const float gC = ex2(lamL);
                 {
                     float v[64];
                     tmem_ld64(tl + kColDS + 64 * h, v);
@@ -797,19 +702,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
                     for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
                 }
-                if (MODE == 0 && e < kD) {
-                    // z += sum_j phi(k_j)   (rows >= L of phi(K) were zeroed)
-                    const uint32_t kb = st + (e >> 6) * 16384;
-                    const int ch = (e & 63) >> 3, wi = e & 7;
-                    float zs = 0.f;
-                    for (int j = 0; j < kC; ++j) {
-                        const uint32_t bits =
-                            lds_u16(kb + j * 128 + ((ch ^ (j & 7)) << 4) + wi * 2);
-                        zs += __uint_as_float(bits << 16);
-                    }
-                    sm->z[e] += zs;
-                }
-                if (KIND == kLocal && MODE == 1 && e == 0) sm->gsum += lamL;
                 if (last) {
                     const bool write = p.s_out && (!p.out_last_only || seg == p.nseg - 1);
                     if (write) {
@@ -829,12 +721,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 mbar_arrive(&sm->s_ready);
                 mbar_arrive(&sm->empty[s]);
             }
-            if (last) {
-                if (MODE == 0 && e < kD && p.z_out && (!p.out_last_only || seg == p.nseg - 1))
-                    p.z_out[(size_t)seg * p.z_out_seg + (size_t)bh * kD + e] = sm->z[e];
-                if (KIND == kLocal && MODE == 1 && e == 0 && p.gam_out)
-                    p.gam_out[(size_t)seg * p.BH + bh] = ex2(sm->gsum);
-            }
 
             // ---- outputs: row t of O (M=64 layout: lane (t % 16) + 32 (t / 16)), half h,
             // staged as bf16 in shared memory and written by two TMA stores (rows past the
@@ -842,24 +728,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             if (kOut) {
                 const int t = 16 * q + lane;
                 const bool has = lane < 16 && t < L;
-                float scale = 1.f;
-                if (MODE == 0 && has)
-                    scale = 1.f / (sm->part[0][t] + sm->part[1][t] + sm->part[2][t] + sm->part[3][t]);
-                if (MODE == 1 && has) scale = ex2(lam[t]);
                 const uint32_t ost = sb + Y::kOst + h * 8192;
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {
                     float v[32];
                     tmem_ld32(tl + kColO + 64 * h + 32 * sub, v);
-                    if (MODE == 1) {
-                        float pq[32];
-                        tmem_ld32(tl + kColP + 64 * h + 32 * sub, pq);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = fmaf(scale, pq[j], v[j]);
-                    } else if (MODE == 0) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] *= scale;
-                    }
                     if (has) {
                         st_row_bf16x16(ost, t, 4 * sub, v);
                         st_row_bf16x16(ost, t, 4 * sub + 2, v + 16);
@@ -919,8 +792,6 @@ struct Small01 {
     int abort;
     int len[8];
     float lam[8][kC];       // in-chunk inclusive prefix of log2(a), chunk mod 8
-    float part[8][3][kC];   // mode 0 denominators: A row-sum halves [0, 1], phi(q).z [2]
-    alignas(16) float zsm[kD];   // mode 0: z after the previous chunk (float4 reads)
     float scan_tmp[2];
 };
 struct Lay01 {
@@ -945,7 +816,7 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
     using Y = Lay01;
     constexpr int NST = Y::kStages;
     constexpr bool kOut = (KIND == kOutput);
-    static_assert(MODE == 0 || MODE == 1, "modes 0 and 1 only");
+    static_assert(MODE == 1, "this kernel serves the scalar-gated mode");
     static_assert(KIND == kOutput || KIND == kLocal, "no transition pass without the delta rule");
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1048,10 +919,9 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                     if (!mbar_wait(&sm->a_ready[c & 1], (c >> 1) & 1, abort, p.err)) break;
                     if (!mbar_wait(&sm->s_ready, c & 1, abort, p.err)) break;
                     tc_fence_after();
-                    const uint32_t dq = (MODE == 1) ? kColP01 : kColO01;
-                    mma_chain<8, true, true>(tm + dq, dk(st + 8192), dk(sbf), id_o1, false);   // Q S^T
+                    mma_chain<8, true, true>(tm + kColP01, dk(st + 8192), dk(sbf), id_o1, false);   // Q S^T
                     mma_chain<4, true, false>(tm + kColO01, dk(at), dmn(st + 32768, 8192), id_o2,
-                                              MODE != 1);                                       // A V
+                                              false);                                             // A V
                     mma_chain<4, false, false>(tm + kColDS, dmn(st + 32768, 8192), dmn(st, 16384), id_ds,
                                                false);                                          // dS = V^T K~
                     mma_commit(&sm->mma2_done);
@@ -1077,21 +947,9 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
     } else if (warp >= 10) {
         // ------------------------------------------------------------ chunk preparation
         const int pe = threadIdx.x - 320;      // 0..63
-        const int pw = pe >> 5;                // K column half of this warp (mode 0)
-        const int cg = lane & 7, rg = lane >> 3;
-        float zr[8];                           // mode 0: z of columns 64 pw + 8 cg + k
-        if (MODE == 0) {
-            const float *zs = (p.s_in_mode == 1 && p.z_in)
-                                  ? p.z_in + (size_t)seg * p.z_in_seg + (size_t)bh * kD
-                                  : nullptr;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) zr[k] = zs ? zs[64 * pw + 8 * cg + k] : 0.f;
-            if (rg == 0)
-#pragma unroll
-                for (int k = 0; k < 8; ++k) sm->zsm[64 * pw + 8 * cg + k] = zr[k];
-        }
+        const int pw = pe >> 5;
         float gsum = 0.f;
-        const bool gated = (MODE == 1) && p.gate != nullptr;
+        const bool gated = p.gate != nullptr;
         float graw = gated ? ld_gate(p, bh, tb, min(kC, te - tb), pe) : 1.f;
         for (int j = 0; j < nch; ++j) {
             const int s = j % NST, u = j / NST;
@@ -1099,7 +957,7 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
             const int L = min(kC, te - t0);
             float gnext = 1.f;
             if (gated && j + 1 < nch) gnext = ld_gate(p, bh, t0 + kC, min(kC, te - t0 - kC), pe);
-            if (MODE == 1) {
+            {
                 float g = (gated && pe < L) ? lg2(fmaxf(graw, FLT_MIN)) : 0.f;
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
@@ -1117,90 +975,8 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
             if (pe == 0) ok = mbar_wait(&sm->full[s], u & 1, abort, p.err);
             if (named_sync_any(2, 64, !ok)) break;
             const uint32_t st = sb + s * Y::kStage;
-            if (MODE == 0) {
-                if (kOut) {
-                    // phi(Q) in place, thread = row; phi(q_r) . z_{j-1}
-                    const int r = pe;
-                    float qz0 = 0.f, qz1 = 0.f;
-#pragma unroll
-                    for (int l4 = 0; l4 < 16; l4 += 4) {
-                        uint4 w[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int lc = l4 + i;
-                            w[i] = lds128(st + 8192 + (lc >> 3) * 16384 + sw128_off(r, lc & 7));
-                        }
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int lc = l4 + i;
-                            w[i].x = phi_bf16x2(w[i].x);
-                            w[i].y = phi_bf16x2(w[i].y);
-                            w[i].z = phi_bf16x2(w[i].z);
-                            w[i].w = phi_bf16x2(w[i].w);
-                            sts128(st + 8192 + (lc >> 3) * 16384 + sw128_off(r, lc & 7), w[i]);
-                            const float4 za = *reinterpret_cast<const float4 *>(&sm->zsm[8 * lc]);
-                            const float4 zb = *reinterpret_cast<const float4 *>(&sm->zsm[8 * lc + 4]);
-                            float2 f = unpack_bf16x2(w[i].x);
-                            qz0 = fmaf(f.x, za.x, qz0);
-                            qz1 = fmaf(f.y, za.y, qz1);
-                            f = unpack_bf16x2(w[i].y);
-                            qz0 = fmaf(f.x, za.z, qz0);
-                            qz1 = fmaf(f.y, za.w, qz1);
-                            f = unpack_bf16x2(w[i].z);
-                            qz0 = fmaf(f.x, zb.x, qz0);
-                            qz1 = fmaf(f.y, zb.y, qz1);
-                            f = unpack_bf16x2(w[i].w);
-                            qz0 = fmaf(f.x, zb.z, qz0);
-                            qz1 = fmaf(f.y, zb.w, qz1);
-                        }
-                    }
-                    sm->part[j & 7][2][r] = qz0 + qz1;
-                    named_sync(2, 64);   // every read of z_{j-1} is done
-                }
-                // phi(K) in place (rows past the chunk end zeroed), column sums into z
-                float cs[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) cs[k] = 0.f;
-#pragma unroll
-                for (int i4 = 0; i4 < 16; i4 += 4) {
-                    uint4 w[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int r = 16 * rg + i4 + i;
-                        w[i] = lds128(st + pw * 16384 + sw128_off(r, cg));
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int r = 16 * rg + i4 + i;
-                        if (r < L) {
-                            w[i].x = phi_bf16x2(w[i].x);
-                            w[i].y = phi_bf16x2(w[i].y);
-                            w[i].z = phi_bf16x2(w[i].z);
-                            w[i].w = phi_bf16x2(w[i].w);
-                        } else {
-                            w[i] = make_uint4(0u, 0u, 0u, 0u);
-                        }
-                        sts128(st + pw * 16384 + sw128_off(r, cg), w[i]);
-                        const uint32_t *wd = reinterpret_cast<const uint32_t *>(&w[i]);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const float2 f = unpack_bf16x2(wd[k]);
-                            cs[2 * k] += f.x;
-                            cs[2 * k + 1] += f.y;
-                        }
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    cs[k] += __shfl_xor_sync(0xffffffffu, cs[k], 8);
-                    cs[k] += __shfl_xor_sync(0xffffffffu, cs[k], 16);
-                    zr[k] += cs[k];
-                }
-                if (rg == 0)
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) sm->zsm[64 * pw + 8 * cg + k] = zr[k];
-            } else if (!kOut) {
-                // LOCAL, mode 1: K~ = diag(dec) K in place, dec_r = 2^(lam_{C-1} - lam_r)
+            if (!kOut) {
+                // LOCAL pass: K~ = diag(dec) K in place, dec_r = 2^(lam_{C-1} - lam_r)
                 named_sync(2, 64);   // the whole prefix is written
                 const float *lam = sm->lam[j & 7];
                 const float lamL = lam[kC - 1];
@@ -1226,12 +1002,7 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
             if (pe == 0) mbar_arrive(&sm->prep_done[s]);
             graw = gnext;
         }
-        if (MODE == 0 && rg == 0 && p.z_out && (!p.out_last_only || seg == p.nseg - 1)) {
-            float *dst = p.z_out + (size_t)seg * p.z_out_seg + (size_t)bh * kD + 64 * pw + 8 * cg;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) dst[k] = zr[k];
-        }
-        if (MODE == 1 && !kOut && pe == kC - 1 && p.gam_out)
+        if (!kOut && pe == kC - 1 && p.gam_out)
             p.gam_out[(size_t)seg * p.BH + bh] = ex2(gsum);
     } else {
         // ------------------------------------------------------------ epilogue warps 2-9
@@ -1272,7 +1043,7 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                 if (e == 0) {
                     ok = mbar_wait(&sm->prep_done[s], u & 1, abort, p.err) &&
                          mbar_wait(&sm->g_done[j & 1], (j >> 1) & 1, abort, p.err);
-                    if (MODE == 1 && ok) ok = mbar_wait(&sm->full[s], u & 1, abort, p.err);
+                    if (ok) ok = mbar_wait(&sm->full[s], u & 1, abort, p.err);
                 }
                 if (named_sync_any(1, kEpi, !ok)) return false;
                 tc_fence_after();
@@ -1282,24 +1053,11 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                 float v[16];
                 tmem_ld_pair16(tl + kColG01 + 64 * (j & 1) + 32 * h, v);
                 const int c0 = 32 * h + 16 * hi;
-                const float li = (MODE == 1) ? lam[i] : 0.f;
-                float rs = 0.f;
+                const float li = lam[i];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    float a = 0.f;
-                    if (c0 + k <= i) a = (MODE == 0) ? v[k] : v[k] * ex2(li - lam[c0 + k]);
-                    if (MODE == 0) {
-                        a = __bfloat162float(__float2bfloat16_rn(a));
-                        rs += a;
-                    }
-                    v[k] = a;
-                }
+                for (int k = 0; k < 16; ++k) v[k] = (c0 + k <= i) ? v[k] * ex2(li - lam[c0 + k]) : 0.f;
                 st_row_bf16x16(sb + Y::kA + (j & 1) * 8192, i, c0 >> 3, v);
-                if (MODE == 0) {
-                    rs += __shfl_xor_sync(0xffffffffu, rs, 16);
-                    if (hi == 0) sm->part[j & 7][h][i] = rs;
-                }
-                if (MODE == 1) {
+                {   // K <- diag(dec) K in place, now that G(j) has consumed K
                     const uint32_t st = sb + s * Y::kStage;
                     const float lamL = lam[kC - 1];
                     uint4 w[4];
@@ -1343,23 +1101,12 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                 {
                     const int t = r64;
                     const bool has = t < L;
-                    float scale = 1.f;
-                    if (MODE == 0 && has) {
-                        const float (*pt)[kC] = sm->part[c & 7];
-                        scale = 1.f / ((pt[0][t] + pt[1][t]) + pt[2][t]);
-                    }
-                    if (MODE == 1 && has) scale = ex2(lam[t]);
-                    float v[32];
+                    const float scale = has ? ex2(lam[t]) : 1.f;
+                    float v[32], pq[32];
                     tmem_ld_pair32(tl + kColO01 + 64 * h, v);
-                    if (MODE == 1) {
-                        float pq[32];
-                        tmem_ld_pair32(tl + kColP01 + 64 * h, pq);
+                    tmem_ld_pair32(tl + kColP01 + 64 * h, pq);
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) v[k] = fmaf(scale, pq[k], v[k]);
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) v[k] *= scale;
-                    }
+                    for (int k = 0; k < 32; ++k) v[k] = fmaf(scale, pq[k], v[k]);
                     if (has) {
                         const uint32_t ost = sb + Y::kOst + h * 8192;
                         st_row_bf16x16(ost, t, 4 * hi, v);
@@ -1369,7 +1116,7 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                 // ---- state: S <- g S + dS (registers), bf16 copy for the next products
                 const bool last = (c + 1 == nch);
                 {
-                    const float gC = (MODE == 0) ? 1.f : ex2(lam[kC - 1]);
+                    const float gC = ex2(lam[kC - 1]);
                     float v[64];
                     tmem_ld64(tl + kColDS + 64 * h, v);
 #pragma unroll
@@ -1409,7 +1156,7 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                 if (e == 0 && ok) mbar_arrive(&sm->empty[s]);   // stage: only dS(c) reads it
                 if (named_sync_any(1, kEpi, !ok)) break;
                 tc_fence_after();
-                const float gC = (MODE == 0) ? 1.f : ex2(sm->lam[c & 7][kC - 1]);
+                const float gC = ex2(sm->lam[c & 7][kC - 1]);
                 float v[64];
                 tmem_ld64(tl + kColDS + 128 * b + 64 * h, v);
 #pragma unroll
