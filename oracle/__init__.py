@@ -36,6 +36,7 @@ _lib = None
 MODE_ELU1_NORM = 0
 MODE_GATED = 1
 MODE_GATED_DELTA = 2
+MODE_KDA = 3
 
 
 def build(force: bool = False) -> str:
@@ -97,7 +98,8 @@ def max_threads() -> int:
 def prefill(mode, q, k, v, gate=None, beta=None, state=None, z=None, nthreads=0):
     """Recurrent form over a whole sequence.
 
-    q, k: [B,H,T,d_k]; v: [B,H,T,d_v]; gate, beta: [B,H,T] or None;
+    q, k: [B,H,T,d_k]; v: [B,H,T,d_v]; gate, beta: [B,H,T] or None (mode 3: gate
+    [B,H,T,d_k], one decay per channel);
     state: [B,H,d_v,d_k] initial state (None -> zero); z: [B,H,d_k] initial
     normaliser for mode 0 (None -> zero).
     Returns (o [B,H,T,d_v], S [B,H,d_v,d_k], z [B,H,d_k] or None), all fp64.
@@ -109,7 +111,7 @@ def prefill(mode, q, k, v, gate=None, beta=None, state=None, z=None, nthreads=0)
     dv = v.shape[-1]
     if v.shape != (B, H, T, dv):
         raise ValueError("v shape mismatch")
-    gate = _f64(gate, (B, H, T))
+    gate = _f64(gate, (B, H, T, dk) if mode == MODE_KDA else (B, H, T))
     beta = _f64(beta, (B, H, T))
     init = state is not None or (mode == 0 and z is not None)
     S = np.zeros((B, H, dv, dk)) if state is None else _f64(state, (B, H, dv, dk)).copy()
@@ -125,7 +127,8 @@ def prefill(mode, q, k, v, gate=None, beta=None, state=None, z=None, nthreads=0)
 
 
 def decode_step(mode, q, k, v, gate, beta, state, z=None, nthreads=0):
-    """One recurrent token for N sequences: q,k [N,H,d_k]; v [N,H,d_v]; gate, beta [N,H].
+    """One recurrent token for N sequences: q,k [N,H,d_k]; v [N,H,d_v]; gate, beta [N,H]
+    (mode 3: gate [N,H,d_k]).
 
     Returns (o [N,H,d_v], S_new [N,H,d_v,d_k], z_new or None); inputs are not modified.
     """
@@ -134,7 +137,7 @@ def decode_step(mode, q, k, v, gate, beta, state, z=None, nthreads=0):
     k = _f64(k, (N, H, dk))
     v = _f64(v)
     dv = v.shape[-1]
-    gate = _f64(gate, (N, H))
+    gate = _f64(gate, (N, H, dk) if mode == MODE_KDA else (N, H))
     beta = _f64(beta, (N, H))
     S = _f64(state, (N, H, dv, dk)).copy()
     zz = None

@@ -56,13 +56,18 @@ def recurrent_form(mode, Q, K, V, gate=None, beta=None, S0=None, z0=None):
 
     For mode 2 the Gated DeltaNet update of [delta rule] is evaluated literally with
     the d_k x d_k matrix (I - b_t k_t k_t^T): S_t = a_t S_{t-1} (I - b_t k k^T) + b_t v k^T.
+    Mode 3 (Kimi Delta Attention) replaces a_t by the diagonal matrix Diag(a_t) (gate
+    [T, d_k]): S_t = S_{t-1} Diag(a_t) (I - b_t k k^T) + b_t v k^T.
     Returns (O, S_T, z_T).
     """
     T, dk = Q.shape
     dv = V.shape[1]
     S = np.zeros((dv, dk)) if S0 is None else np.array(S0, dtype=np.float64)
     z = np.zeros(dk) if z0 is None else np.array(z0, dtype=np.float64)
-    a = np.ones(T) if gate is None else np.asarray(gate, dtype=np.float64)
+    if mode == 3:
+        a = np.ones((T, dk)) if gate is None else np.asarray(gate, dtype=np.float64)
+    else:
+        a = np.ones(T) if gate is None else np.asarray(gate, dtype=np.float64)
     O = np.zeros((T, dv))
     I = np.eye(dk)
     for t in range(T):
@@ -73,6 +78,10 @@ def recurrent_form(mode, Q, K, V, gate=None, beta=None, S0=None, z0=None):
             O[t] = (S @ fq) / (z @ fq)
         elif mode == 1:
             S = a[t] * S + np.outer(V[t], K[t])
+            O[t] = S @ Q[t]
+        elif mode == 3:
+            b = beta[t]
+            S = S @ np.diag(a[t]) @ (I - b * np.outer(K[t], K[t])) + b * np.outer(V[t], K[t])
             O[t] = S @ Q[t]
         else:
             b = beta[t]
@@ -97,18 +106,40 @@ def chunked_form(mode, Q, K, V, C, gate=None, beta=None, S0=None, z0=None):
     solve the unit lower-triangular system (I + L) E = diag(b) V - diag(b g) K S^T,
     L_ij = b_i D_ij (k_i . k_j) for j < i.  Then
         O = diag(g) Q S^T + ((Q K^T) * D) E,   S_new = g_last S + sum_j D_last,j e_j k_j^T.
+
+    mode 3 (per-channel decay, gate [T, d_k]) is the same derivation with the in-block
+    inclusive products G_i = a_s * ... * a_i taken per channel: the decay of a key j seen
+    from row i is G_i / G_j channel by channel, so
+        L_ij = b_i (k_i * G_i) . (k_j / G_j)  (j < i),   A_ij = (q_i * G_i) . (k_j / G_j)  (j <= i),
+        (I + L) E = diag(b) V - diag(b) (K * G) S^T,
+        O = (Q * G) S^T + A E,   S_new = S Diag(G_last) + E^T (K * G_last / G).
     Returns (O, S, z).
     """
     T, dk = Q.shape
     dv = V.shape[1]
     S = np.zeros((dv, dk)) if S0 is None else np.array(S0, dtype=np.float64)
     z = np.zeros(dk) if z0 is None else np.array(z0, dtype=np.float64)
-    a_all = np.ones(T) if gate is None else np.asarray(gate, dtype=np.float64)
+    if mode == 3:
+        a_all = np.ones((T, dk)) if gate is None else np.asarray(gate, dtype=np.float64)
+    else:
+        a_all = np.ones(T) if gate is None else np.asarray(gate, dtype=np.float64)
     O = np.zeros((T, dv))
     for s in range(0, T, C):
         e = min(s + C, T)
         L = e - s
         q, k, v, a = Q[s:e], K[s:e], V[s:e], a_all[s:e]
+        if mode == 3:
+            b = np.asarray(beta[s:e], dtype=np.float64)
+            G = np.cumprod(a, axis=0)                      # [L, d_k] in-block channel products
+            kg, kin = k * G, k / G
+            Lm = np.tril(b[:, None] * (kg @ kin.T), -1)
+            A = np.tril((q * G) @ kin.T)
+            Tinv = np.linalg.inv(np.eye(L) + Lm)
+            U, W = Tinv @ (b[:, None] * v), Tinv @ (b[:, None] * kg)
+            E = U - W @ S.T
+            O[s:e] = (q * G) @ S.T + A @ E
+            S = S * G[-1][None, :] + E.T @ (k * (G[-1][None, :] / G))
+            continue
         g = np.array([np.prod(a[:i + 1]) for i in range(L)])  # in-block inclusive gate products
         D = decay_mask(a, L)
         if mode == 0:

@@ -26,16 +26,21 @@
  *       S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S_t q_t.
  *     The product S_{t-1}(I - b k k^T) is evaluated as S_{t-1} - b (S_{t-1} k) k^T,
  *     which is the same matrix (distributivity), at O(d_k d_v) per token.
+ *   mode 3 (Kimi Delta Attention of [delta rule]: the scalar a_t of mode 2 becomes the
+ *     diagonal matrix Diag(a_t), each memory channel forgetting at its own rate; the
+ *     channels are the d_k columns of S):
+ *       S_t = S_{t-1} Diag(a_t) (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S_t q_t,
+ *     evaluated as M = S_{t-1} Diag(a_t), S_t = M - b (M k) k^T + b v k^T.
  *
  * S is d_v x d_k (the page's orientation), stored row-major [d_v][d_k]; z has
  * d_k entries.  A NULL gate means a_t = 1.  Mode 0 ignores gate and beta, mode 1
- * ignores beta.  Readings where the page is silent (no 1/sqrt(d) inside the
+ * ignores beta.  In mode 3 the gate holds d_k values per token.  Readings where the page is silent (no 1/sqrt(d) inside the
  * attention, no epsilon in the mode-0 denominator, the gate multiplies the old
  * state before token t is written) are listed in the design notes; this file
  * implements exactly the equations above.
  *
  * Layouts (all dense, row-major, fp64):
- *   q, k [B,H,T,d_k]; v, o [B,H,T,d_v]; gate, beta [B,H,T];
+ *   q, k [B,H,T,d_k]; v, o [B,H,T,d_v]; gate, beta [B,H,T] (mode 3: gate [B,H,T,d_k]);
  *   S [B,H,d_v,d_k]; z [B,H,d_k].
  */
 #include <math.h>
@@ -52,8 +57,8 @@ static double oracle_phi(double x) { return x > 0.0 ? x + 1.0 : exp(x); }
 /* One token of the recurrence on one head.  fq/fk are d_k scratch vectors,
  * sk is d_v scratch. */
 static void oracle_token(int mode, int dk, int dv, const double *q, const double *k,
-                         const double *v, double a, double beta, double *S, double *z,
-                         double *o, double *fq, double *fk, double *sk)
+                         const double *v, double a, const double *av, double beta, double *S,
+                         double *z, double *o, double *fq, double *fk, double *sk)
 {
     if (mode == 0) {
         for (int j = 0; j < dk; ++j) {
@@ -81,6 +86,24 @@ static void oracle_token(int mode, int dk, int dv, const double *q, const double
             double acc = 0.0;
             for (int j = 0; j < dk; ++j) {
                 row[j] = a * row[j] + v[i] * k[j];
+                acc += row[j] * q[j];
+            }
+            o[i] = acc;
+        }
+    } else if (mode == 3) {
+        /* M = S_{t-1} Diag(a_t); (M k)_i */
+        for (int i = 0; i < dv; ++i) {
+            const double *row = S + (size_t)i * dk;
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += row[j] * (av ? av[j] : 1.0) * k[j];
+            sk[i] = acc;
+        }
+        for (int i = 0; i < dv; ++i) {
+            double *row = S + (size_t)i * dk;
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) {
+                /* [M (I - b k k^T)]_{ij} + b v_i k_j */
+                row[j] = row[j] * (av ? av[j] : 1.0) - beta * sk[i] * k[j] + beta * v[i] * k[j];
                 acc += row[j] * q[j];
             }
             o[i] = acc;
@@ -118,10 +141,10 @@ int oracle_prefill(int mode, long B, long H, long T, int dk, int dv,
                    const double *gate, const double *beta,
                    double *S, double *z, double *o, int init_state, int nthreads)
 {
-    if (mode < 0 || mode > 2 || B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return -1;
+    if (mode < 0 || mode > 3 || B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return -1;
     if ((T > 0 && (!q || !k || !v || !o)) || !S) return -1;
     if (mode == 0 && !z) return -1;
-    if (mode == 2 && T > 0 && !beta) return -1;
+    if (mode >= 2 && T > 0 && !beta) return -1;
     const long BH = B * H;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
@@ -147,10 +170,11 @@ int oracle_prefill(int mode, long B, long H, long T, int dk, int dv,
             }
             for (long t = 0; t < T; ++t) {
                 const size_t tok = (size_t)bh * T + t;
-                const double a = gate ? gate[tok] : 1.0;
+                const double a = (gate && mode != 3) ? gate[tok] : 1.0;
+                const double *av = (gate && mode == 3) ? gate + tok * dk : NULL;
                 const double b = beta ? beta[tok] : 0.0;
-                oracle_token(mode, dk, dv, q + tok * dk, k + tok * dk, v + tok * dv, a, b, Sh,
-                             zh, o + tok * dv, scratch, scratch + dk, scratch + 2 * dk);
+                oracle_token(mode, dk, dv, q + tok * dk, k + tok * dk, v + tok * dv, a, av, b,
+                             Sh, zh, o + tok * dv, scratch, scratch + dk, scratch + 2 * dk);
             }
         }
         free(scratch);
@@ -161,7 +185,8 @@ int oracle_prefill(int mode, long B, long H, long T, int dk, int dv,
 /*
  * One decode token for N sequences x H heads: the same single step of the
  * recurrence applied in place to a given state.  Layouts: q,k [N,H,d_k];
- * v, o [N,H,d_v]; gate, beta [N,H]; S [N,H,d_v,d_k]; z [N,H,d_k].
+ * v, o [N,H,d_v]; gate, beta [N,H] (mode 3: gate [N,H,d_k]); S [N,H,d_v,d_k];
+ * z [N,H,d_k].
  */
 int oracle_decode_step(int mode, long N, long H, int dk, int dv,
                        const double *q, const double *k, const double *v,

@@ -372,3 +372,93 @@ def test_gate_zero_forgets_everything():
         o, S, _ = run1(mode, Q, K, V, gate=a, beta=b)
         o_tail, S_tail, _ = run1(mode, Q[6:], K[6:], V[6:], gate=a[6:], beta=b[6:])
         assert np.abs(o[6:] - o_tail).max() < 1e-14 and np.abs(S - S_tail).max() < 1e-14
+
+
+# ----------------------------------------------------------------------------------
+# Kimi Delta Attention (mode 3): the Gated DeltaNet update with Diag(a_t), one decay
+# per channel of the memory (the d_k columns of S)
+# ----------------------------------------------------------------------------------
+
+def kda_inputs(seed, T, dk, dv):
+    Q, K, V, _, b = rng_inputs(seed, T, dk, dv, unit_keys=True)
+    r = np.random.default_rng(seed + 1000)
+    a = 1.0 / (1.0 + np.exp(r.normal(size=(T, dk))))   # per-channel values in (0, 1)
+    return Q, K, V, a, b
+
+
+@pytest.mark.parametrize("T", [1, 5, 17, 64])
+def test_three_forms_agree_mode3(T):
+    """C oracle == literal per-token matrix form S Diag(a)(I - b k k^T) + b v k^T ==
+    the per-channel chunked form derived for it (one chunk and C in {4, 16})."""
+    Q, K, V, a, b = kda_inputs(80 + T, T, 6, 4)
+    S0 = np.random.default_rng(T + 5).normal(size=(4, 6))
+    o, S, _ = run1(3, Q, K, V, gate=a, beta=b, S0=S0)
+    o_r, S_r, _ = forms.recurrent_form(3, Q, K, V, gate=a, beta=b, S0=S0)
+    assert np.abs(o - o_r).max() < 1e-12 and np.abs(S - S_r).max() < 1e-12
+    for C in (T, 4, 16):
+        o_c, S_c, _ = forms.chunked_form(3, Q, K, V, C, gate=a, beta=b, S0=S0)
+        assert np.abs(o - o_c).max() < 1e-11 and np.abs(S - S_c).max() < 1e-11
+
+
+def test_mode3_uniform_channels_is_gated_deltanet():
+    """Diag(a_t) with all channels equal to a_t is the scalar Gated DeltaNet gate."""
+    Q, K, V, a, b = rng_inputs(90, 33, 8, 5, unit_keys=True)
+    S0 = np.random.default_rng(91).normal(size=(5, 8))
+    o2, S2, _ = run1(2, Q, K, V, gate=a, beta=b, S0=S0)
+    o3, S3, _ = run1(3, Q, K, V, gate=np.repeat(a[:, None], 8, axis=1), beta=b, S0=S0)
+    assert np.abs(o3 - o2).max() < 1e-13 and np.abs(S3 - S2).max() < 1e-13
+
+
+def test_mode3_ungated_is_the_delta_rule():
+    Q, K, V, _, b = rng_inputs(92, 21, 6, 4, unit_keys=True)
+    o2, S2, _ = run1(2, Q, K, V, gate=None, beta=b)
+    o3, S3, _ = run1(3, Q, K, V, gate=None, beta=b)
+    assert np.array_equal(o3, o2) and np.array_equal(S3, S2)
+
+
+def test_mode3_beta_zero_decays_each_channel():
+    """b = 0 writes nothing: S_t = S_0 Diag(a_1 ... a_t), so column c of the state decays
+    by its own product and o_t = S_0 Diag(prod) q_t."""
+    Q, K, V, a, _ = kda_inputs(93, 12, 7, 4)
+    S0 = np.random.default_rng(94).normal(size=(4, 7))
+    o, S, _ = run1(3, Q, K, V, gate=a, beta=np.zeros(12), S0=S0)
+    P = np.cumprod(a, axis=0)
+    assert np.abs(S - S0 * P[-1][None, :]).max() < 1e-14
+    assert np.abs(o - (Q * P) @ S0.T).max() < 1e-13
+
+
+def test_mode3_closed_channel_keeps_only_fresh_writes():
+    """A channel whose decay is 0 at every token holds only the latest write in it:
+    column c of S_t is b_t (v_t - (M k_t)) k_t[c] with M the decayed old state."""
+    Q, K, V, a, b = kda_inputs(95, 9, 5, 3)
+    a = a.copy()
+    a[:, 2] = 0.0
+    _, S, _ = run1(3, Q, K, V, gate=a, beta=b)
+    _, S8, _ = run1(3, Q[:8], K[:8], V[:8], gate=a[:8], beta=b[:8])
+    M = S8 * a[8][None, :]
+    col = b[8] * (V[8] - M @ K[8]) * K[8][2]
+    assert np.abs(S[:, 2] - col).max() < 1e-13
+
+
+def test_mode3_split_prefill_and_decode_continue():
+    T, T1 = 30, 17
+    Q, K, V, a, b = kda_inputs(96, T, 6, 5)
+    o, S, _ = run1(3, Q, K, V, gate=a, beta=b)
+    o1, S1, _ = run1(3, Q[:T1], K[:T1], V[:T1], gate=a[:T1], beta=b[:T1])
+    o2, S2, _ = run1(3, Q[T1:], K[T1:], V[T1:], gate=a[T1:], beta=b[T1:], S0=S1)
+    assert np.abs(np.concatenate([o1, o2]) - o).max() < 1e-12 and np.abs(S2 - S).max() < 1e-12
+    St = S1[None, None]
+    for t in range(T1, T):
+        od, St, _ = oracle.decode_step(3, Q[t][None, None], K[t][None, None], V[t][None, None],
+                                       a[t][None, None], np.array([[b[t]]]), St)
+        assert np.abs(od[0, 0] - o[t]).max() < 1e-12
+    assert np.abs(St[0, 0] - S).max() < 1e-12
+
+
+def test_mode3_linear_in_values_from_zero_state():
+    Q, K, V, a, b = kda_inputs(97, 25, 6, 4)
+    V2 = np.random.default_rng(98).normal(size=V.shape)
+    o1, S1, _ = run1(3, Q, K, V, gate=a, beta=b)
+    o2, S2, _ = run1(3, Q, K, V2, gate=a, beta=b)
+    o3, S3, _ = run1(3, Q, K, 2.0 * V - 3.0 * V2, gate=a, beta=b)
+    assert np.abs(o3 - (2 * o1 - 3 * o2)).max() < 1e-12 and np.abs(S3 - (2 * S1 - 3 * S2)).max() < 1e-12

@@ -32,6 +32,12 @@ MUTANTS = {
     "mode2_reads_old_state": ("                row[j] = a * (row[j] - beta * sk[i] * k[j]) + beta * v[i] * k[j];\n                acc += row[j] * q[j];",
                               "                acc += row[j] * q[j];\n                row[j] = a * (row[j] - beta * sk[i] * k[j]) + beta * v[i] * k[j];"),
     "mode2_correction_uses_query": ("acc += row[j] * k[j];\n            sk[i] = acc;", "acc += row[j] * q[j];\n            sk[i] = acc;"),
+    # mode 3
+    "mode3_correction_not_decayed": ("acc += row[j] * (av ? av[j] : 1.0) * k[j];", "acc += row[j] * k[j];"),
+    "mode3_drops_channel_decay": ("row[j] = row[j] * (av ? av[j] : 1.0) - beta * sk[i] * k[j]",
+                                  "row[j] = row[j] - beta * sk[i] * k[j]"),
+    "mode3_reads_old_state": ("                row[j] = row[j] * (av ? av[j] : 1.0) - beta * sk[i] * k[j] + beta * v[i] * k[j];\n                acc += row[j] * q[j];",
+                              "                acc += row[j] * q[j];\n                row[j] = row[j] * (av ? av[j] : 1.0) - beta * sk[i] * k[j] + beta * v[i] * k[j];"),
 }
 
 
