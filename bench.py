@@ -98,18 +98,20 @@ def io_bytes(dtype):
 def prefill_algorithmic(w: W.Workload, C=64):
     """Bytes that must cross HBM once and flops of the chunked form at chunk C = 64.
 
-    bytes: q, k, v read + o written, gates/beta read, final state (and z) written.
+    bytes: q, k, v read + o written, gates/beta read (mode 3: d_k gates per token),
+    final state (and z) written.
     flops per token-head: modes 0/1  2C d_k + 2C d_v + 4 d_k d_v;
-                          mode 2     10 C d + 6 d^2 + C^2 / 3  (d = d_k = d_v)."""
+                          modes 2/3  10 C d + 6 d^2 + C^2 / 3  (d = d_k = d_v; the per-channel
+                          decays of mode 3 are exponentials inside the products, not counted)."""
     th = w.B * w.H * w.T
     e = io_bytes(w.dtype)
     b = th * e * (2 * w.dk + 2 * w.dv)
     if w.gate != "none":
-        b += th * 4
+        b += th * 4 * (w.dk if w.mode == 3 else 1)
     if w.beta:
         b += th * 4
     b += w.B * w.H * (w.dv * w.dk * 4 + (w.dk * 4 if w.mode == 0 else 0))
-    if w.mode == 2:
+    if w.mode >= 2:
         d = w.dk
         f = 10 * C * d + 6 * d * d + C * C / 3.0
     else:
@@ -123,7 +125,7 @@ def decode_algorithmic(w: W.Workload):
     e = io_bytes(w.dtype)
     b = nh * (2 * w.dk * w.dv * 4 + e * (2 * w.dk + 2 * w.dv))
     if w.gate != "none":
-        b += nh * 4
+        b += nh * 4 * (w.dk if w.mode == 3 else 1)
     if w.beta:
         b += nh * 4
     if w.mode == 0:
@@ -577,7 +579,7 @@ def main():
     do_extras = (world == 1) if args.extras < 0 else bool(args.extras)
     if do_extras:
         for name in ("elu1_bf16_b4h16t4096", "gated_bf16_b8h16t8192", "gdn_bf16_b2h16t32768",
-                     "gdn_decode_n256h32"):
+                     "gdn_decode_n256h32", "kda_bf16_b2h16t32768", "kda_decode_n256h32"):
             if name == args.workload:
                 continue
             r = measure(la, name, args, dist, device, rank, world, flush, False)

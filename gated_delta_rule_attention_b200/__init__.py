@@ -7,11 +7,13 @@ and forwards raw device pointers and the current CUDA stream.  Every step of the
 method runs in the library's kernels; there is no Python or CPU fallback, and the
 import fails loudly if the library is missing.
 
-Three modes, named after the variants on the lesson page "Linear attention and hybrids":
+Four modes, named after the variants on the lesson page "Linear attention and hybrids":
 
 * ``MODE_ELU1_NORM`` -- phi(x) = elu(x)+1 with the z normaliser (section "The kernel trick")
 * ``MODE_GATED`` -- scalar decay gate a_t (section "Memory must forget: decay and gates")
 * ``MODE_GATED_DELTA`` -- the Gated DeltaNet update (section "The delta rule and Gated DeltaNet")
+* ``MODE_KDA`` -- Kimi Delta Attention, the same update with one decay per channel (gate
+  [.., d_k] per token; same section)
 """
 from __future__ import annotations
 
@@ -20,13 +22,14 @@ import os
 
 import torch
 
-__all__ = ["MODE_ELU1_NORM", "MODE_GATED", "MODE_GATED_DELTA", "FLAG_INIT_STATE", "LaError",
+__all__ = ["MODE_ELU1_NORM", "MODE_GATED", "MODE_GATED_DELTA", "MODE_KDA", "FLAG_INIT_STATE", "LaError",
            "prefill", "decode_step", "check_status", "library", "library_path", "version",
            "kernel_launches", "workspace_size"]
 
 MODE_ELU1_NORM = 0
 MODE_GATED = 1
 MODE_GATED_DELTA = 2
+MODE_KDA = 3
 FLAG_INIT_STATE = 1
 
 LA_F32 = 0
@@ -170,7 +173,8 @@ def prefill(q, k, v, *, mode: int, gate=None, beta=None, state=None, z=None, o=N
             chunk: int = 0, init_state: bool | None = None, stream=None, workspace="auto"):
     """Chunked prefill over whole sequences (``la_prefill``).
 
-    q, k: [B,H,T,d_k]; v: [B,H,T,d_v] (bf16 or fp32, one dtype); gate, beta: [B,H,T] fp32;
+    q, k: [B,H,T,d_k]; v: [B,H,T,d_v] (bf16 or fp32, one dtype); gate, beta: [B,H,T] fp32
+    (``MODE_KDA``: gate [B,H,T,d_k]);
     state: [B,H,d_v,d_k] fp32 (read as S_0 when ``init_state``, default: when given);
     z: [B,H,d_k] fp32 (mode 0).  Returns (o, state, z).
 
@@ -199,7 +203,7 @@ def prefill(q, k, v, *, mode: int, gate=None, beta=None, state=None, z=None, o=N
     _need(k, (B, H, T, dk), dt, "k")
     _need(v, (B, H, T, dv), dt, "v")
     if gate is not None:
-        _need(gate, (B, H, T), torch.float32, "gate")
+        _need(gate, (B, H, T, dk) if mode == MODE_KDA else (B, H, T), torch.float32, "gate")
     if beta is not None:
         _need(beta, (B, H, T), torch.float32, "beta")
     if init_state is None:
@@ -234,7 +238,8 @@ def decode_step(q, k, v, *, mode: int, state, gate=None, beta=None, z=None, o=No
                 stream=None):
     """One token for N sequences (``la_decode_step``), state updated in place.
 
-    q, k: [N,H,d_k]; v: [N,H,d_v]; gate, beta: [N,H] fp32; state: [N,H,d_v,d_k] fp32;
+    q, k: [N,H,d_k]; v: [N,H,d_v]; gate, beta: [N,H] fp32 (``MODE_KDA``: gate [N,H,d_k]);
+    state: [N,H,d_v,d_k] fp32;
     z: [N,H,d_k] fp32 (mode 0).  Returns (o, state, z).  CPU inputs take the end-to-end
     path of ``prefill`` (copy in, run on the GPU, copy o, state and z back).
     """
@@ -261,7 +266,7 @@ def decode_step(q, k, v, *, mode: int, state, gate=None, beta=None, z=None, o=No
     _need(v, (N, H, dv), dt, "v")
     _need(state, (N, H, dv, dk), torch.float32, "state")
     if gate is not None:
-        _need(gate, (N, H), torch.float32, "gate")
+        _need(gate, (N, H, dk) if mode == MODE_KDA else (N, H), torch.float32, "gate")
     if beta is not None:
         _need(beta, (N, H), torch.float32, "beta")
     if mode == MODE_ELU1_NORM:

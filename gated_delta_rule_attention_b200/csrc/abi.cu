@@ -70,7 +70,7 @@ extern "C" la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H
                                   void *o, int chunk, unsigned flags, void *workspace,
                                   size_t workspace_bytes, void *stream) {
     timer_reset();
-    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_GATED_DELTA) return LA_ERR_INVALID_ARG;
+    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_KDA) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || T < 0) return LA_ERR_INVALID_ARG;
     if (flags & ~LA_FLAG_INIT_STATE) return LA_ERR_INVALID_ARG;
@@ -93,7 +93,7 @@ extern "C" la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H
     if (!tensor_ok(q, 16) || !tensor_ok(k, 16) || !tensor_ok(v, 16) || !tensor_ok(o, 16))
         return LA_ERR_INVALID_ARG;
     if (mode != LA_MODE_ELU1_NORM && gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
-    if (mode == LA_MODE_GATED_DELTA && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
+    if (mode >= LA_MODE_GATED_DELTA && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
 
     PrefillArgs a;
     a.mode = mode;
@@ -101,14 +101,14 @@ extern "C" la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H
     a.B = B; a.H = H; a.T = T; a.dk = d_k; a.dv = d_v;
     a.q = q; a.k = k; a.v = v;
     a.gate = (mode == LA_MODE_ELU1_NORM) ? nullptr : gate;
-    a.beta = (mode == LA_MODE_GATED_DELTA) ? beta : nullptr;
+    a.beta = (mode >= LA_MODE_GATED_DELTA) ? beta : nullptr;
     a.state = state;
     a.z = (mode == LA_MODE_ELU1_NORM) ? z : nullptr;
     a.o = o;
     a.init_state = init;
     a.stream = st;
     if (workspace && workspace_bytes && !tensor_ok(workspace, 16)) return LA_ERR_INVALID_ARG;
-    if (prefill_tc_supports(dtype, d_k, d_v, chunk)) {
+    if (prefill_tc_supports(mode, dtype, d_k, d_v, chunk)) {
         a.chunk = 64;
         return from_cuda(launch_prefill_tc(a, workspace, workspace ? workspace_bytes : 0));
     }
@@ -120,9 +120,9 @@ extern "C" la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H
 
 extern "C" size_t la_prefill_workspace_size(la_mode_t mode, la_dtype_t dtype, int B, int H, int T,
                                             int d_k, int d_v, int chunk) {
-    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_GATED_DELTA || B < 1 || H < 1 || T < 1)
+    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_KDA || B < 1 || H < 1 || T < 1)
         return 0;
-    if (!prefill_tc_supports(dtype, d_k, d_v, chunk)) return 0;
+    if (!prefill_tc_supports(mode, dtype, d_k, d_v, chunk)) return 0;
     return prefill_tc_workspace_bytes(mode, B, H, T);
 }
 
@@ -131,7 +131,7 @@ extern "C" la_status_t la_decode_step(la_mode_t mode, la_dtype_t dtype, int N, i
                                       const float *gate, const float *beta, float *state,
                                       float *z, void *o, void *stream) {
     timer_reset();
-    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_GATED_DELTA) return LA_ERR_INVALID_ARG;
+    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_KDA) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     if (N < 1 || H < 1) return LA_ERR_INVALID_ARG;
     if (!dims_ok(d_k, d_v)) return LA_ERR_UNSUPPORTED;
@@ -143,14 +143,14 @@ extern "C" la_status_t la_decode_step(la_mode_t mode, la_dtype_t dtype, int N, i
         return LA_ERR_INVALID_ARG;
     if (mode == LA_MODE_ELU1_NORM && !tensor_ok(z, 16)) return LA_ERR_INVALID_ARG;
     if (mode != LA_MODE_ELU1_NORM && gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
-    if (mode == LA_MODE_GATED_DELTA && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
+    if (mode >= LA_MODE_GATED_DELTA && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
     DecodeArgs a;
     a.mode = mode;
     a.dtype = dtype;
     a.N = N; a.H = H; a.dk = d_k; a.dv = d_v;
     a.q = q; a.k = k; a.v = v;
     a.gate = (mode == LA_MODE_ELU1_NORM) ? nullptr : gate;
-    a.beta = (mode == LA_MODE_GATED_DELTA) ? beta : nullptr;
+    a.beta = (mode >= LA_MODE_GATED_DELTA) ? beta : nullptr;
     a.state = state;
     a.z = (mode == LA_MODE_ELU1_NORM) ? z : nullptr;
     a.o = o;

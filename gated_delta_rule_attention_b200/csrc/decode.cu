@@ -6,6 +6,8 @@
 // s_j (row j of S, d_k floats) evolves independently of every other row:
 //
 //   mode 2:  e_j = b (v_j - a s_j.k);   s_j <- a s_j + e_j k;   o_j = a (s_j.q) + e_j (k.q)
+//   mode 3:  the same with the row first decayed per channel, s_j <- s_j o a (Kimi Delta
+//            Attention: Diag(a) for the scalar a), then a = 1
 //   mode 1:  s_j <- a s_j + v_j k;                              o_j = a (s_j.q) + v_j (k.q)
 //   mode 0:  s_j <- s_j + v_j phi(k);  z <- z + phi(k);
 //            o_j = (s_j.phi(q) + v_j phi(k).phi(q)) / (z_new . phi(q))
@@ -80,8 +82,12 @@ decode_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__re
             kv[e] = feature_phi(kv[e]);
         }
     }
-    const float a = (MODE == 0 || gate == nullptr) ? 1.f : gate[nh];
-    const float b = (MODE == 2) ? beta[nh] : 0.f;
+    constexpr bool kDelta = (MODE == 2 || MODE == 3);
+    const float a = (MODE == 0 || MODE == 3 || gate == nullptr) ? 1.f : gate[nh];
+    const float b = kDelta ? beta[nh] : 0.f;
+    float av[VEC];   // mode 3: this lane's channel decays
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) av[e] = (MODE == 3 && gate) ? gate[nh * DK + lane * VEC + e] : 1.f;
     float kq = 0.f;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) kq = fmaf(kv[e], qv[e], kq);
@@ -114,6 +120,10 @@ decode_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__re
         for (int j = 0; j < ROWS; ++j) {
             s[j].load(S + (size_t)(row0 + rr + j) * DK + lane * VEC);
             vj[j] = to_f32(vh[row0 + rr + j]);
+            if (MODE == 3) {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) s[j].x[e] *= av[e];
+            }
         }
         float sq[ROWS], sk[ROWS];
 #pragma unroll
@@ -123,17 +133,17 @@ decode_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__re
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
                 sq[j] = fmaf(s[j].x[e], qv[e], sq[j]);
-                if (MODE == 2) sk[j] = fmaf(s[j].x[e], kv[e], sk[j]);
+                if (kDelta) sk[j] = fmaf(s[j].x[e], kv[e], sk[j]);
             }
         }
 #pragma unroll
         for (int j = 0; j < ROWS; ++j) {
-            if (MODE == 2) sk[j] = warp_sum(sk[j]);
+            if (kDelta) sk[j] = warp_sum(sk[j]);
         }
 #pragma unroll
         for (int j = 0; j < ROWS; ++j) {
             float w;  // coefficient of k in the row update
-            if (MODE == 2) w = b * (vj[j] - a * sk[j]);
+            if (kDelta) w = b * (vj[j] - a * sk[j]);
             else w = vj[j];
 #pragma unroll
             for (int e = 0; e < VEC; ++e) s[j].x[e] = fmaf(w, kv[e], a * s[j].x[e]);
@@ -177,6 +187,7 @@ cudaError_t launch_io(const DecodeArgs &a) {
         case LA_MODE_ELU1_NORM: return launch_mode<0, IO>(a);
         case LA_MODE_GATED: return launch_mode<1, IO>(a);
         case LA_MODE_GATED_DELTA: return launch_mode<2, IO>(a);
+        case LA_MODE_KDA: return launch_mode<3, IO>(a);
     }
     return cudaErrorInvalidValue;
 }

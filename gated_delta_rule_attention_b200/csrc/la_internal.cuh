@@ -53,7 +53,7 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs &a);
 cudaError_t launch_prefill_simt(const PrefillArgs &a);
 bool prefill_simt_supports(int dtype, int dk, int dv, int chunk, int *resolved_chunk);
-bool prefill_tc_supports(int dtype, int dk, int dv, int chunk);
+bool prefill_tc_supports(int mode, int dtype, int dk, int dv, int chunk);
 size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T);
 cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes);
 

@@ -21,6 +21,14 @@
 // solved here by forward substitution as U = (I+Lm)^-1 diag(b) V, W = (I+Lm)^-1 diag(b g) K,
 // E = U - W S^T.  Every exponent is <= 0, so no factor exceeds 1.
 //
+// Mode 3 (Kimi Delta Attention, the same section: Diag(a_t) in place of the scalar a_t,
+// one decay per channel c of d_k) takes the in-chunk prefix per channel, lam_ic, and
+// the decay of key j seen from row i becomes exp(lam_ic - lam_jc) inside the dot products:
+//
+//   A_ij = sum_c q_ic k_jc exp(lam_ic - lam_jc),  Lm_ij = b_i sum_c k_ic k_jc exp(lam_ic - lam_jc),
+//   (I + Lm) E = diag(b) V - diag(b) (K o G) S^T,   G_ic = exp(lam_ic),
+//   O = (Q o G) S^T + A E,   S <- S Diag(G_L) + E^T (K o exp(lam_L - lam)).
+//
 // One CTA (256 threads) per (batch, head) walks the chunks in order; all tiles are fp32
 // in shared memory with one float of row padding so that row-strided reads are
 // bank-conflict free.
@@ -33,13 +41,14 @@ namespace {
 
 constexpr int kSimtThreads = 256;
 
-template <int DK, int DV, int C>
+template <int MODE, int DK, int DV, int C>
 struct SimtSmem {
     static constexpr int kS = DV * (DK + 1);
     static constexpr int kQ = C * (DK + 1);
     static constexpr int kV = C * (DV + 1);
     static constexpr int kA = C * (C + 1);
-    static constexpr int kFloats = kS + 3 * kQ + kV + 2 * kA + 4 * C + DK;
+    static constexpr int kLamC = (MODE == 3) ? kQ : 0;   // per-channel log-gate prefix
+    static constexpr int kFloats = kS + 3 * kQ + kV + 2 * kA + 4 * C + DK + kLamC;
     static constexpr size_t kBytes = sizeof(float) * kFloats;
 };
 
@@ -49,7 +58,8 @@ prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
                     const IO *__restrict__ v, const float *__restrict__ gate,
                     const float *__restrict__ beta, float *__restrict__ state,
                     float *__restrict__ zg, IO *__restrict__ o, int init_state) {
-    using L = SimtSmem<DK, DV, C>;
+    using L = SimtSmem<MODE, DK, DV, C>;
+    constexpr bool kDelta = (MODE == 2 || MODE == 3);
     extern __shared__ float smem[];
     float *S = smem;                 // [DV][DK+1]
     float *Qs = S + L::kS;           // [C][DK+1]
@@ -63,6 +73,7 @@ prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
     float *den = bet + C;            // [C]
     float *dec = den + C;            // [C]
     float *zs = dec + C;             // [DK]
+    float *lamC = zs + DK;           // [C][DK+1]  mode 3
 
     constexpr int SK = DK + 1, SV = DV + 1, SA = C + 1;
     const int tid = threadIdx.x;
@@ -71,7 +82,7 @@ prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
     const IO *kh = k + bh * (size_t)T * DK;
     const IO *vh = v + bh * (size_t)T * DV;
     IO *oh = o + bh * (size_t)T * DV;
-    const float *gh = gate ? gate + bh * (size_t)T : nullptr;
+    const float *gh = gate ? gate + bh * (size_t)T * (MODE == 3 ? DK : 1) : nullptr;
     const float *bh_beta = beta ? beta + bh * (size_t)T : nullptr;
     float *Sg = state + bh * (size_t)DV * DK;
 
@@ -95,8 +106,17 @@ prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
         for (int p = tid; p < Lc * DV; p += kSimtThreads)
             Vs[(p / DV) * SV + p % DV] = to_f32(vh[(size_t)(t0 + p / DV) * DV + p % DV]);
         if (tid < Lc) {
-            lam[tid] = (MODE != 0 && gh) ? logf(fmaxf(gh[t0 + tid], FLT_MIN)) : 0.f;
-            bet[tid] = (MODE == 2) ? bh_beta[t0 + tid] : 0.f;
+            lam[tid] = (MODE != 0 && MODE != 3 && gh) ? logf(fmaxf(gh[t0 + tid], FLT_MIN)) : 0.f;
+            bet[tid] = kDelta ? bh_beta[t0 + tid] : 0.f;
+        }
+        if (MODE == 3) {   // per-channel in-chunk prefix of log a, one channel per thread
+            for (int c = tid; c < DK; c += kSimtThreads) {
+                float acc = 0.f;
+                for (int i = 0; i < Lc; ++i) {
+                    acc += gh ? logf(fmaxf(gh[(size_t)(t0 + i) * DK + c], FLT_MIN)) : 0.f;
+                    lamC[i * SK + c] = acc;
+                }
+            }
         }
         __syncthreads();
         if (tid == 0)
@@ -112,15 +132,17 @@ prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
                 float qk = 0.f, kk = 0.f;
 #pragma unroll 8
                 for (int c = 0; c < DK; ++c) {
-                    qk = fmaf(Qs[i * SK + c], Ks[j * SK + c], qk);
-                    if (MODE == 2) kk = fmaf(Ks[i * SK + c], Ks[j * SK + c], kk);
+                    const float kj = (MODE == 3) ? Ks[j * SK + c] * expf(lamC[i * SK + c] - lamC[j * SK + c])
+                                                 : Ks[j * SK + c];
+                    qk = fmaf(Qs[i * SK + c], kj, qk);
+                    if (kDelta) kk = fmaf(Ks[i * SK + c], kj, kk);
                 }
-                const float d = (MODE == 0) ? 1.f : expf(lam[i] - lam[j]);
+                const float d = (MODE == 0 || MODE == 3) ? 1.f : expf(lam[i] - lam[j]);
                 aij = qk * d;
-                if (MODE == 2 && j < i) lij = bet[i] * d * kk;
+                if (kDelta && j < i) lij = bet[i] * d * kk;
             }
             A[i * SA + j] = aij;
-            if (MODE == 2) Lm[i * SA + j] = lij;
+            if (kDelta) Lm[i * SA + j] = lij;
         }
         __syncthreads();
 
@@ -131,12 +153,13 @@ prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
             den[tid] = s;
         }
 
-        if (MODE == 2) {
-            // right-hand sides: diag(b) V in Vs, diag(b g) K in Ws
+        if (kDelta) {
+            // right-hand sides: diag(b) V in Vs, diag(b g) K (mode 3: diag(b) (K o G)) in Ws
             for (int p = tid; p < Lc * DV; p += kSimtThreads) Vs[(p / DV) * SV + p % DV] *= bet[p / DV];
             for (int p = tid; p < Lc * DK; p += kSimtThreads) {
                 const int i = p / DK, c = p % DK;
-                Ws[i * SK + c] = bet[i] * expf(lam[i]) * Ks[i * SK + c];
+                const float g = (MODE == 3) ? expf(lamC[i * SK + c]) : expf(lam[i]);
+                Ws[i * SK + c] = bet[i] * g * Ks[i * SK + c];
             }
             __syncthreads();
             // forward substitution, one column of [U | W] per thread
@@ -160,6 +183,16 @@ prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
             }
         }
         __syncthreads();
+        if (MODE == 3) {
+            // Q <- Q o G (the inter-chunk read) and K <- K o exp(lam_L - lam) (the state
+            // update); the raw tiles are no longer needed
+            for (int p = tid; p < Lc * DK; p += kSimtThreads) {
+                const int i = p / DK, c = p % DK;
+                Qs[i * SK + c] *= expf(lamC[i * SK + c]);
+                Ks[i * SK + c] *= expf(lamC[(Lc - 1) * SK + c] - lamC[i * SK + c]);
+            }
+            __syncthreads();
+        }
 
         // ---- output: O = diag(g) Q S^T + A X   (mode 0: / den)
         for (int p = tid; p < Lc * DV; p += kSimtThreads) {
@@ -171,18 +204,21 @@ prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
             for (int j = 0; j <= t; ++j) intra = fmaf(A[t * SA + j], Vs[j * SV + i], intra);
             float out;
             if (MODE == 0) out = (inter + intra) / den[t];
+            else if (MODE == 3) out = inter + intra;
             else out = fmaf(expf(lam[t]), inter, intra);
             oh[(size_t)(t0 + t) * DV + i] = from_f32<IO>(out);
         }
         __syncthreads();
 
         // ---- state update: S <- g_L S + sum_j exp(lam_L - lam_j) x_j k_j^T
-        const float gL = (MODE == 0) ? 1.f : expf(lam[Lc - 1]);
+        const float gL = (MODE == 0 || MODE == 3) ? 1.f : expf(lam[Lc - 1]);
         for (int p = tid; p < DV * DK; p += kSimtThreads) {
             const int i = p / DK, c = p % DK;
             float acc = 0.f;
-            for (int j = 0; j < Lc; ++j) acc = fmaf(dec[j] * Vs[j * SV + i], Ks[j * SK + c], acc);
-            S[i * SK + c] = fmaf(gL, S[i * SK + c], acc);
+            for (int j = 0; j < Lc; ++j)
+                acc = fmaf((MODE == 3 ? 1.f : dec[j]) * Vs[j * SV + i], Ks[j * SK + c], acc);
+            const float g = (MODE == 3) ? expf(lamC[(Lc - 1) * SK + c]) : gL;
+            S[i * SK + c] = fmaf(g, S[i * SK + c], acc);
         }
         if (MODE == 0) {
             for (int c = tid; c < DK; c += kSimtThreads) {
@@ -201,7 +237,7 @@ prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
 
 template <int MODE, int DK, int DV, int C, typename IO>
 cudaError_t launch_one(const PrefillArgs &a) {
-    using L = SimtSmem<DK, DV, C>;
+    using L = SimtSmem<MODE, DK, DV, C>;
     auto kern = prefill_simt_kernel<MODE, DK, DV, C, IO>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)L::kBytes);
@@ -240,6 +276,7 @@ cudaError_t launch_io(const PrefillArgs &a) {
         case LA_MODE_ELU1_NORM: return launch_dims<0, IO>(a);
         case LA_MODE_GATED: return launch_dims<1, IO>(a);
         case LA_MODE_GATED_DELTA: return launch_dims<2, IO>(a);
+        case LA_MODE_KDA: return launch_dims<3, IO>(a);
     }
     return cudaErrorInvalidValue;
 }

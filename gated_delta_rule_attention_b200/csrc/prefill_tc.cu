@@ -1919,8 +1919,10 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
 
 }  // namespace
 
-bool prefill_tc_supports(int dtype, int dk, int dv, int chunk) {
-    return dtype == LA_BF16 && dk == kD && dv == kD && (chunk == 0 || chunk == kC);
+bool prefill_tc_supports(int mode, int dtype, int dk, int dv, int chunk) {
+    // modes 0-2 in bf16 with d = 128; Kimi Delta Attention runs on CUDA cores
+    return mode != LA_MODE_KDA && dtype == LA_BF16 && dk == kD && dv == kD &&
+           (chunk == 0 || chunk == kC);
 }
 
 size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T) {

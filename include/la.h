@@ -8,7 +8,7 @@
  *   [decay/gates]   "Память должна забывать: затухание и гейты" -- gamma, alpha_t gates
  *   [delta rule]    "Дельта-правило и Gated DeltaNet" -- delta rule, Gated DeltaNet
  *
- * Three variants ("modes"), each with a chunked prefill and a one-token decode step.
+ * Four variants ("modes"), each with a chunked prefill and a one-token decode step.
  * Per (batch, head), for t = 1..T, the state is updated first and then read:
  *
  *   LA_MODE_ELU1_NORM ([kernel trick], [three forms]):
@@ -18,6 +18,9 @@
  *       S_t = a_t S_{t-1} + v_t k_t^T,   o_t = S_t q_t.
  *   LA_MODE_GATED_DELTA ([delta rule], the Gated DeltaNet equation):
  *       S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S_t q_t.
+ *   LA_MODE_KDA ([delta rule], Kimi Delta Attention: the scalar a_t replaced by the
+ *   diagonal matrix Diag(a_t), one decay per memory channel, the d_k columns of S):
+ *       S_t = S_{t-1} Diag(a_t) (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S_t q_t.
  *
  * No 1/sqrt(d) scale is applied inside the attention; callers scale q and k.
  *
@@ -32,8 +35,9 @@
  *   are always fp32; all accumulation is fp32.
  * Sizes: d_k and d_v are each 64 or 128.  B, H, N >= 1.  T >= 0.
  * Gates: gate holds the decay values a_t in [0, 1] (not their logarithms); NULL means
- *   a_t = 1.  beta holds b_t in [0, 1].  Mode 0 ignores gate and beta; mode 1 ignores
- *   beta; mode 2 requires beta.
+ *   a_t = 1.  In mode 3 it holds d_k values per token (one per channel).  beta holds
+ *   b_t in [0, 1].  Mode 0 ignores gate and beta; mode 1 ignores beta; modes 2 and 3
+ *   require beta.
  * State layout: S is d_v x d_k per head, exactly the page's S ([three forms]), stored
  *   [.., d_v, d_k] row-major; z is [.., d_k].  A state written by la_prefill is the
  *   input of la_decode_step, and vice versa.
@@ -56,7 +60,8 @@ extern "C" {
 typedef enum {
     LA_MODE_ELU1_NORM = 0,   /* phi = elu+1, z-normalised                 */
     LA_MODE_GATED = 1,       /* scalar gate a_t, identity feature map     */
-    LA_MODE_GATED_DELTA = 2  /* Gated DeltaNet: gate a_t and delta rate b_t */
+    LA_MODE_GATED_DELTA = 2, /* Gated DeltaNet: gate a_t and delta rate b_t */
+    LA_MODE_KDA = 3          /* Kimi Delta Attention: per-channel gate a_t [d_k], rate b_t */
 } la_mode_t;
 
 typedef enum {
@@ -85,13 +90,15 @@ typedef enum {
  *
  *   q, k   [B, H, T, d_k]  I/O dtype
  *   v      [B, H, T, d_v]  I/O dtype
- *   gate   [B, H, T] fp32 or NULL      beta [B, H, T] fp32 (mode 2) or NULL
+ *   gate   [B, H, T] fp32 or NULL      beta [B, H, T] fp32 (modes 2, 3) or NULL
+ *          (mode 3: gate [B, H, T, d_k])
  *   state  [B, H, d_v, d_k] fp32       in (if LA_FLAG_INIT_STATE) and out: S_T
  *   z      [B, H, d_k] fp32            mode 0 only (else ignored, may be NULL): in/out z_T
  *   o      [B, H, T, d_v]  I/O dtype   out: o_1..o_T
  *   chunk  tokens per chunk; 0 picks the kernel's default.  bf16 with d_k = d_v = 128
- *          accepts 0 and 64; every other case accepts 0, 32 and 64 (64 only when
- *          d_k = d_v = 64).  Other values return LA_ERR_UNSUPPORTED.
+ *          in modes 0-2 runs on the tensor cores and accepts 0 and 64; every other case
+ *          (fp32, d = 64, and mode 3) runs on CUDA cores and accepts 0, 32 and 64 (64 only
+ *          when d_k = d_v = 64).  Other values return LA_ERR_UNSUPPORTED.
  *   flags  0 or LA_FLAG_INIT_STATE.
  *   workspace, workspace_bytes
  *          optional device scratch owned by the caller (NULL / 0 allowed).  With at least
@@ -144,7 +151,8 @@ la_status_t la_prefill_noalloc(la_mode_t mode, la_dtype_t dtype, int B, int H, i
  * the per-token cost is O(d_k d_v) and independent of how many tokens came before.
  *
  *   q, k   [N, H, d_k]  I/O dtype       v [N, H, d_v]  I/O dtype
- *   gate   [N, H] fp32 or NULL          beta [N, H] fp32 (mode 2) or NULL
+ *   gate   [N, H] fp32 or NULL          beta [N, H] fp32 (modes 2, 3) or NULL
+ *          (mode 3: gate [N, H, d_k])
  *   state  [N, H, d_v, d_k] fp32 in/out z [N, H, d_k] fp32 in/out (mode 0 only)
  *   o      [N, H, d_v] I/O dtype out
  */

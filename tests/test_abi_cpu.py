@@ -72,7 +72,7 @@ def _prefill(lib, mode=2, dtype=1, B=1, H=1, T=8, dk=128, dv=128, chunk=0, flags
 
 def test_host_side_argument_checks(lib):
     INVALID, UNSUPPORTED = 1, 2
-    assert _prefill(lib, mode=3) == INVALID
+    assert _prefill(lib, mode=4) == INVALID
     assert _prefill(lib, mode=-1) == INVALID
     assert _prefill(lib, dtype=2) == INVALID
     assert _prefill(lib, B=0) == INVALID

@@ -58,7 +58,12 @@ def test_gdn_bf16_b2h16t32768_sampled(la):
     _check_prefill(la, W.CONFIGS["gdn_bf16_b2h16t32768"], [(0, 0), (1, 9), (1, 15)])
 
 
-@pytest.mark.parametrize("name", ["gated_bf16_b8h16t8192", "gdn_bf16_b2h16t32768"])
+def test_kda_bf16_b2h16t32768_sampled(la):
+    _check_prefill(la, W.CONFIGS["kda_bf16_b2h16t32768"], [(0, 0), (1, 15)])
+
+
+@pytest.mark.parametrize("name", ["gated_bf16_b8h16t8192", "gdn_bf16_b2h16t32768",
+                                  "kda_bf16_b2h16t32768"])
 def test_full_size_weak_decay_state_path(la, name):
     """At the configs' own gate distribution the state decays by ~e^-50 per chunk, so
     the carried state barely matters; a ~0.98 gate at the same sizes (fewer heads)
@@ -67,8 +72,9 @@ def test_full_size_weak_decay_state_path(la, name):
     _check_prefill(la, w, [(0, 0), (0, 3)])
 
 
-def test_gdn_decode_n256h32_sampled(la):
-    w = W.CONFIGS["gdn_decode_n256h32"]
+@pytest.mark.parametrize("name", ["gdn_decode_n256h32", "kda_decode_n256h32"])
+def test_decode_n256h32_sampled(la, name):
+    w = W.CONFIGS[name]
     steps = 12
     inp = W.decode_inputs(w, steps=steps, device="cuda")
     S = inp["state0"].clone()

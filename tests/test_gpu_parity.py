@@ -29,9 +29,9 @@ def la():
 
 def small(mode, dtype, d, T, B=2, H=3, gate="softplus", gate_shift=0.0, seed=100):
     return W.Workload(f"m{mode}", mode, dtype, B=B, H=H, T=T, dk=d, dv=d, seed=seed,
-                      qk_scale=1 / np.sqrt(d), qk_l2norm=(mode == 2),
+                      qk_scale=1 / np.sqrt(d), qk_l2norm=(mode >= 2),
                       gate="none" if mode == 0 else gate, gate_shift=gate_shift,
-                      beta=(mode == 2))
+                      beta=(mode >= 2))
 
 
 def run_and_compare(la, w, init_std=0.0, chunk=0, heads=None):
@@ -59,7 +59,7 @@ def run_and_compare(la, w, init_std=0.0, chunk=0, heads=None):
     return eo, eS
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("T", [1, 64, 200])
@@ -67,7 +67,7 @@ def test_prefill_small(la, mode, dtype, d, T):
     run_and_compare(la, small(mode, dtype, d, T))
 
 
-@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("mode", [1, 2, 3])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("gate,shift", [("softplus", -4.0), ("none", 0.0)])
 def test_prefill_weak_decay_exercises_the_carried_state(la, mode, dtype, gate, shift):
@@ -75,13 +75,13 @@ def test_prefill_weak_decay_exercises_the_carried_state(la, mode, dtype, gate, s
     run_and_compare(la, small(mode, dtype, 128, 333, gate=gate, gate_shift=shift))
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_prefill_initial_state(la, mode, dtype):
     run_and_compare(la, small(mode, dtype, 128, 150, gate_shift=-3.0), init_std=0.05)
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
 def test_prefill_empty_sequence(la, mode):
     w = small(mode, torch.bfloat16, 128, 0)
     inp = W.prefill_inputs(w, device="cuda", init_state_std=0.1)
@@ -101,7 +101,7 @@ def test_prefill_empty_sequence(la, mode):
         assert torch.count_nonzero(z2) == 0
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
 def test_split_prefill_then_decode_continues(la, mode):
     """prefill(T1) ; prefill(T2 from that state) ; n decode steps == oracle over T1+T2+n."""
     dtype = torch.bfloat16
@@ -149,13 +149,13 @@ def test_heads_batches_independent(la):
 # decode
 # ----------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("d", [64, 128])
 def test_decode_steps(la, mode, dtype, d):
     w = W.Workload("dec", mode, dtype, B=6, H=3, T=12, dk=d, dv=d, seed=7,
-                   qk_scale=1 / np.sqrt(d), qk_l2norm=(mode == 2),
-                   gate="none" if mode == 0 else "softplus", gate_shift=-2.0, beta=(mode == 2),
+                   qk_scale=1 / np.sqrt(d), qk_l2norm=(mode >= 2),
+                   gate="none" if mode == 0 else "softplus", gate_shift=-2.0, beta=(mode >= 2),
                    decode=True, state_std=0.02)
     inp = W.decode_inputs(w, device="cuda")
     S = inp["state0"].clone()

@@ -6,7 +6,8 @@ method's arithmetic.  Both the fp64 oracle and the CUDA library receive the tens
 returns (the oracle after an exact upcast to fp64).
 
 Draw order is fixed: q, k, v, gate pre-activation x, beta pre-activation y (and, for
-decode, the initial state first).  Gates are stored as values a_t in (0, 1], not logs.
+decode, the initial state first).  Gates are stored as values a_t in (0, 1], not logs;
+in mode 3 (Kimi Delta Attention) there is one gate per channel, x of shape [.., d_k].
 """
 from __future__ import annotations
 
@@ -18,6 +19,7 @@ import torch
 MODE_ELU1_NORM = 0
 MODE_GATED = 1
 MODE_GATED_DELTA = 2
+MODE_KDA = 3
 
 
 @dataclasses.dataclass(frozen=True)
@@ -63,6 +65,14 @@ CONFIGS = {
     "gdn_decode_n256h32": Workload("gdn_decode_n256h32", MODE_GATED_DELTA, torch.bfloat16, B=256,
                                    H=32, T=1000, dk=128, dv=128, seed=5, qk_l2norm=True,
                                    gate="softplus", beta=True, decode=True, state_std=0.02),
+    # Kimi Delta Attention (per-channel gates): the shapes and recipes of the two
+    # gated-delta workloads above with a_t drawn per channel.
+    "kda_bf16_b2h16t32768": Workload("kda_bf16_b2h16t32768", MODE_KDA, torch.bfloat16, B=2, H=16,
+                                     T=32768, dk=128, dv=128, seed=6, qk_l2norm=True,
+                                     gate="softplus", beta=True),
+    "kda_decode_n256h32": Workload("kda_decode_n256h32", MODE_KDA, torch.bfloat16, B=256, H=32,
+                                   T=1000, dk=128, dv=128, seed=7, qk_l2norm=True,
+                                   gate="softplus", beta=True, decode=True, state_std=0.02),
 }
 
 
@@ -84,7 +94,8 @@ def _qkv(w: Workload, gen: torch.Generator, device, lead):
 def _gates(w: Workload, gen: torch.Generator, device, lead):
     gate = beta = None
     if w.gate == "softplus":
-        x = torch.randn(*lead, generator=gen, device=device, dtype=torch.float32)
+        shape = (*lead, w.dk) if w.mode == MODE_KDA else lead
+        x = torch.randn(*shape, generator=gen, device=device, dtype=torch.float32)
         # a = exp(-softplus(x)) = sigmoid(-x): a value in (0, 1)
         gate = torch.exp(-torch.nn.functional.softplus(x + w.gate_shift))
     elif w.gate != "none":
@@ -96,7 +107,8 @@ def _gates(w: Workload, gen: torch.Generator, device, lead):
 
 
 def prefill_inputs(w: Workload, device="cpu", init_state_std: float = 0.0):
-    """q,k [B,H,T,d_k], v [B,H,T,d_v] in w.dtype; gate, beta [B,H,T] fp32 or None;
+    """q,k [B,H,T,d_k], v [B,H,T,d_v] in w.dtype; gate, beta [B,H,T] fp32 or None (mode 3:
+    gate [B,H,T,d_k]);
     state0 [B,H,d_v,d_k] fp32 (zeros unless init_state_std > 0)."""
     gen = torch.Generator(device=device)
     gen.manual_seed(w.seed)
@@ -112,7 +124,8 @@ def prefill_inputs(w: Workload, device="cpu", init_state_std: float = 0.0):
 
 def decode_inputs(w: Workload, steps: int | None = None, device="cpu", n_seqs: int | None = None):
     """Initial state [N,H,d_v,d_k] ~ N(0, state_std^2) and per-step inputs stacked over
-    steps: q,k [steps,N,H,d_k], v [steps,N,H,d_v], gate, beta [steps,N,H]."""
+    steps: q,k [steps,N,H,d_k], v [steps,N,H,d_v], gate, beta [steps,N,H] (mode 3: gate
+    [steps,N,H,d_k])."""
     steps = w.T if steps is None else steps
     N = w.B if n_seqs is None else n_seqs
     gen = torch.Generator(device=device)
