@@ -57,3 +57,30 @@ def test_pins_catch_planted_mistakes(name, tmp_path):
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"planted mistake {name} passed every pin:\n{r.stdout[-2000:]}"
     assert "failed" in r.stdout or "error" in r.stdout.lower()
+
+
+CONV_SRC = os.path.join(ROOT, "oracle", "conv.py")
+CONV_MUTANTS = {
+    "conv_taps_reversed": ("u += w[:, i] * full[:, i:i + T, :]",
+                           "u += w[:, width - 1 - i] * full[:, i:i + T, :]"),
+    "conv_window_not_carried": ("return y, full[:, T:, :].copy()", "return y, full[:, -(width - 1):, :].copy() * 0"),
+    "conv_silu_sign": ("u = u / (1.0 + np.exp(-u))", "u = u / (1.0 + np.exp(u))"),
+    "conv_norm_over_heads": ("r = u.reshape(B, T, H, C // H)", "r = u.reshape(B, T, C // H, H)"),
+    "conv_head_layout": ("y = y.reshape(B, T, H, d).transpose(0, 2, 1, 3).copy()",
+                         "y = y.reshape(B, H, T, d).copy()"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CONV_MUTANTS))
+def test_conv_pins_catch_planted_mistakes(name, tmp_path):
+    old, new = CONV_MUTANTS[name]
+    src = open(CONV_SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mutant = tmp_path / "conv_mutant.py"
+    mutant.write_text(src.replace(old, new))
+    env = dict(os.environ, LA_ORACLE_CONV_OVERRIDE=str(mutant))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_conv_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"planted mistake {name} passed every pin:\n{r.stdout[-2000:]}"
+    assert "failed" in r.stdout or "error" in r.stdout.lower()
