@@ -328,6 +328,59 @@ class DecodeCase:
         self.h_o.copy_(self.o, non_blocking=True)
 
 
+class ConvCase:
+    """One step = the short convolution prologue of one prefill batch: three
+    la_short_conv calls (q and k with SiLU and the L2 norm, v with SiLU), token-major
+    projections in, head-major attention inputs out."""
+
+    def __init__(self, la, cw: W.ConvWorkload, device, rank):
+        self.la, self.w, self.device = la, cw, device
+        self.dims = [cw.dk, cw.dk, cw.dv]
+        self.x, self.wt, self.y, self.win = [], [], [], []
+        for i, d in enumerate(self.dims):
+            C = cw.H * d
+            x, w, _ = W.conv_inputs(cw.B, cw.T, C, cw.width, cw.dtype,
+                                    seed=cw.seed + 10 * i + 1000 * rank, device=device, window=False)
+            self.x.append(x)
+            self.wt.append(w)
+            self.y.append(torch.empty(cw.B, cw.H, cw.T, d, device=device, dtype=cw.dtype))
+            self.win.append(torch.empty(cw.B, cw.width - 1, C, device=device, dtype=cw.dtype))
+        self.tokens = cw.B * cw.T
+        e = io_bytes(cw.dtype)
+        self.bytes = float(sum(2 * cw.B * cw.T * cw.H * d * e + cw.H * d * cw.width * 4
+                               + cw.B * (cw.width - 1) * cw.H * d * e for d in self.dims))
+        self.flops = float(sum(2 * cw.width * cw.B * cw.T * cw.H * d for d in self.dims))
+        self.kind = "conv"
+
+    def _calls(self, collect=None):
+        for i in range(3):
+            self.la.short_conv(self.x[i], self.wt[i], heads=self.w.H, window_out=self.win[i],
+                               silu=self.w.silu, l2norm=self.w.l2norm_qk and i < 2, y=self.y[i])
+            if collect is not None:
+                collect.extend(self.la.launch_times())
+
+    def step(self):
+        self._calls()
+
+    def step_collect(self):
+        out = []
+        self._calls(out)
+        return out
+
+    def e2e_setup(self):
+        self.h_x = [x.to("cpu").pin_memory() for x in self.x]
+        self.h_y = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in self.y]
+        self.h2d = sum(x.numel() * x.element_size() for x in self.h_x)
+        self.d2h = sum(y.numel() * y.element_size() for y in self.h_y)
+
+    def e2e_step(self):
+        for hx, x in zip(self.h_x, self.x):
+            x.copy_(hx, non_blocking=True)
+        self._calls()
+        for hy, y in zip(self.h_y, self.y):
+            hy.copy_(y, non_blocking=True)
+
+
 def time_steps(case, steps, warmup, dist, device, flush, fn=None, sampler=None):
     """Device time of `steps` calls of fn (default case.step), each bracketed by CUDA events
     on the launching stream, with an L2 flush between steps (outside the events)."""
@@ -368,8 +421,11 @@ def launch_profile(case, steps, flush):
         for _ in range(steps):
             if flush is not None:
                 flush.zero_()
-            case.step()
-            per.append(la.launch_times())
+            if hasattr(case, "step_collect"):
+                per.append(case.step_collect())
+            else:
+                case.step()
+                per.append(la.launch_times())
     finally:
         la.launch_timing(False)
     n = min(len(p) for p in per) if per else 0
@@ -419,9 +475,12 @@ def roofline(case, kernel_ms, step_ms, peaks, peak_src, prof):
 
 
 def measure(la, name, args, dist, device, rank, world, flush, with_e2e, sampler=None):
-    w = W.CONFIGS[name]
-    case = (DecodeCase(la, w, device, rank, args.warmup + args.steps) if w.decode
-            else PrefillCase(la, w, device, rank, None if args.no_workspace else "auto"))
+    if name in W.CONV_CONFIGS:
+        case = ConvCase(la, W.CONV_CONFIGS[name], device, rank)
+    else:
+        w = W.CONFIGS[name]
+        case = (DecodeCase(la, w, device, rank, args.warmup + args.steps) if w.decode
+                else PrefillCase(la, w, device, rank, None if args.no_workspace else "auto"))
     ms, launches = time_steps(case, args.steps, args.warmup, dist, device, flush, sampler=sampler)
     la.check_status()
     kernel_ms = launch_profile(case, args.steps, flush)
@@ -579,7 +638,8 @@ def main():
     do_extras = (world == 1) if args.extras < 0 else bool(args.extras)
     if do_extras:
         for name in ("elu1_bf16_b4h16t4096", "gated_bf16_b8h16t8192", "gdn_bf16_b2h16t32768",
-                     "gdn_decode_n256h32", "kda_bf16_b2h16t32768", "kda_decode_n256h32"):
+                     "gdn_decode_n256h32", "kda_bf16_b2h16t32768", "kda_decode_n256h32",
+                     "conv_bf16_b2h16t32768"):
             if name == args.workload:
                 continue
             r = measure(la, name, args, dist, device, rank, world, flush, False)

@@ -23,14 +23,16 @@ import os
 import torch
 
 __all__ = ["MODE_ELU1_NORM", "MODE_GATED", "MODE_GATED_DELTA", "MODE_KDA", "FLAG_INIT_STATE", "LaError",
-           "prefill", "decode_step", "check_status", "library", "library_path", "version",
-           "kernel_launches", "workspace_size"]
+           "prefill", "decode_step", "short_conv", "short_conv_step", "check_status", "library",
+           "library_path", "version", "kernel_launches", "workspace_size"]
 
 MODE_ELU1_NORM = 0
 MODE_GATED = 1
 MODE_GATED_DELTA = 2
 MODE_KDA = 3
 FLAG_INIT_STATE = 1
+CONV_SILU = 2
+CONV_L2NORM = 4
 
 LA_F32 = 0
 LA_BF16 = 1
@@ -81,6 +83,10 @@ def library():
     lib.la_version.restype = i
     lib.la_kernel_launches.argtypes = []
     lib.la_kernel_launches.restype = ctypes.c_ulonglong
+    lib.la_short_conv.argtypes = [i, i, i, i, i, i, vp, fp, vp, vp, vp, u, vp]
+    lib.la_short_conv.restype = i
+    lib.la_short_conv_step.argtypes = [i, i, i, i, i, vp, fp, vp, vp, u, vp]
+    lib.la_short_conv_step.restype = i
     if hasattr(lib, "la_launch_timing"):   # diagnostic hook, absent from older builds
         lib.la_launch_timing.argtypes = [i]
         lib.la_launch_timing.restype = i
@@ -279,6 +285,69 @@ def decode_step(q, k, v, *, mode: int, state, gate=None, beta=None, z=None, o=No
                                   _stream_handle(q.device, stream))
     _check(st, "la_decode_step")
     return o, state, z
+
+
+def _conv_flags(silu: bool, l2norm: bool) -> int:
+    return (CONV_SILU if silu else 0) | (CONV_L2NORM if l2norm else 0)
+
+
+def short_conv(x, w, *, heads: int, window=None, window_out=None, silu: bool = False,
+               l2norm: bool = False, y=None, stream=None):
+    """Short causal depthwise convolution over time (``la_short_conv``).
+
+    x: [B, T, H*d] token-major (bf16 or fp32); w: [H*d, width] fp32 taps (tap width-1
+    multiplies the current token); window: [B, width-1, H*d] in x's dtype, the inputs
+    before x_0 (None: zeros).  ``silu`` applies u * sigmoid(u), ``l2norm`` normalises
+    every head's d-row.  Returns (y [B, H, T, d], window_out [B, width-1, H*d]);
+    ``window_out`` may be passed (``window`` itself updates the window in place).
+    """
+    B, T, C = x.shape
+    width = w.shape[1]
+    if C % heads:
+        raise ValueError("x's last dimension must be heads * d")
+    d = C // heads
+    dt = x.dtype
+    dtype = _io_dtype(x)
+    _need(x, (B, T, C), dt, "x")
+    _need(w, (C, width), torch.float32, "w")
+    if window is not None:
+        _need(window, (B, width - 1, C), dt, "window")
+    if window_out is None:
+        window_out = torch.empty(B, width - 1, C, device=x.device, dtype=dt)
+    _need(window_out, (B, width - 1, C), dt, "window_out")
+    if y is None:
+        y = torch.empty(B, heads, T, d, device=x.device, dtype=dt)
+    _need(y, (B, heads, T, d), dt, "y")
+    st = library().la_short_conv(dtype, B, T, heads, d, width, _ptr(x), _ptr(w), _ptr(window),
+                                 _ptr(window_out), _ptr(y), _conv_flags(silu, l2norm),
+                                 _stream_handle(x.device, stream))
+    _check(st, "la_short_conv")
+    return y, window_out
+
+
+def short_conv_step(x, w, window, *, heads: int, silu: bool = False, l2norm: bool = False,
+                    y=None, stream=None):
+    """One new token of N sequences (``la_short_conv_step``): x [N, H*d], window
+    [N, width-1, H*d] updated in place.  Returns y [N, H, d]."""
+    N, C = x.shape
+    width = w.shape[1]
+    if C % heads:
+        raise ValueError("x's last dimension must be heads * d")
+    d = C // heads
+    dt = x.dtype
+    dtype = _io_dtype(x)
+    _need(x, (N, C), dt, "x")
+    _need(w, (C, width), torch.float32, "w")
+    if width > 1:
+        _need(window, (N, width - 1, C), dt, "window")
+    if y is None:
+        y = torch.empty(N, heads, d, device=x.device, dtype=dt)
+    _need(y, (N, heads, d), dt, "y")
+    st = library().la_short_conv_step(dtype, N, heads, d, width, _ptr(x), _ptr(w),
+                                      _ptr(window if width > 1 else None), _ptr(y),
+                                      _conv_flags(silu, l2norm), _stream_handle(x.device, stream))
+    _check(st, "la_short_conv_step")
+    return y
 
 
 def check_status(stream=None):

@@ -59,6 +59,12 @@ la_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_
 
 bool dims_ok(int dk, int dv) { return (dk == 64 || dk == 128) && (dv == 64 || dv == 128); }
 
+// True if the byte ranges [p, p + n) and [q, q + m) share a byte.
+bool overlap(const void *p, size_t n, const void *q, size_t m) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+    return p && q && n && m && a < b + m && b < a + n;
+}
+
 }  // namespace
 }  // namespace la
 
@@ -156,6 +162,75 @@ extern "C" la_status_t la_decode_step(la_mode_t mode, la_dtype_t dtype, int N, i
     a.o = o;
     a.stream = static_cast<cudaStream_t>(stream);
     return from_cuda(launch_decode(a));
+}
+
+extern "C" la_status_t la_short_conv(la_dtype_t dtype, int B, int T, int H, int d, int width,
+                                     const void *x, const float *w, const void *window_in,
+                                     void *window_out, void *y, unsigned flags, void *stream) {
+    timer_reset();
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (B < 1 || T < 0 || H < 1 || width < 1 || width > 4) return LA_ERR_INVALID_ARG;
+    if (flags & ~(LA_CONV_SILU | LA_CONV_L2NORM)) return LA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
+    const long long C = (long long)H * d;
+    if (C > INT32_MAX || (long long)B * T * C > kMaxElems) return LA_ERR_INVALID_ARG;
+    if (!tensor_ok(w, 4)) return LA_ERR_INVALID_ARG;
+    const size_t es = dtype == LA_BF16 ? 2 : 4;
+    const size_t win_bytes = (size_t)B * (width - 1) * C * es;
+    const void *win_in = width > 1 ? window_in : nullptr;
+    void *win_out = width > 1 ? window_out : nullptr;
+    if (win_in && !tensor_ok(win_in, 16)) return LA_ERR_INVALID_ARG;
+    if (win_out && !tensor_ok(win_out, 16)) return LA_ERR_INVALID_ARG;
+    if (win_in != win_out && overlap(win_in, win_bytes, win_out, win_bytes)) return LA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (!win_out || win_out == win_in) return LA_OK;
+        return from_cuda(win_in ? cudaMemcpyAsync(win_out, win_in, win_bytes, cudaMemcpyDeviceToDevice, st)
+                                : cudaMemsetAsync(win_out, 0, win_bytes, st));
+    }
+    if (!tensor_ok(x, 16) || !tensor_ok(y, 16)) return LA_ERR_INVALID_ARG;
+    const size_t xy_bytes = (size_t)B * T * C * es;
+    if (overlap(x, xy_bytes, y, xy_bytes) || overlap(y, xy_bytes, win_in, win_bytes) ||
+        overlap(y, xy_bytes, win_out, win_bytes) || overlap(x, xy_bytes, win_out, win_bytes))
+        return LA_ERR_INVALID_ARG;
+    ConvArgs a;
+    a.dtype = dtype;
+    a.B = B; a.T = T; a.H = H; a.d = d; a.width = width;
+    a.step = false;
+    a.silu = (flags & LA_CONV_SILU) != 0;
+    a.l2norm = (flags & LA_CONV_L2NORM) != 0;
+    a.x = x; a.w = w; a.win_in = win_in; a.win_out = win_out; a.y = y;
+    a.stream = st;
+    return from_cuda(launch_short_conv(a));
+}
+
+extern "C" la_status_t la_short_conv_step(la_dtype_t dtype, int N, int H, int d, int width,
+                                          const void *x, const float *w, void *window, void *y,
+                                          unsigned flags, void *stream) {
+    timer_reset();
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (N < 1 || H < 1 || width < 1 || width > 4) return LA_ERR_INVALID_ARG;
+    if (flags & ~(LA_CONV_SILU | LA_CONV_L2NORM)) return LA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
+    const long long C = (long long)H * d;
+    if (C > INT32_MAX || (long long)N * C * width > kMaxElems) return LA_ERR_INVALID_ARG;
+    if (!tensor_ok(w, 4) || !tensor_ok(x, 16) || !tensor_ok(y, 16)) return LA_ERR_INVALID_ARG;
+    void *win = width > 1 ? window : nullptr;
+    if (width > 1 && !tensor_ok(win, 16)) return LA_ERR_INVALID_ARG;
+    const size_t es = dtype == LA_BF16 ? 2 : 4;
+    const size_t xy_bytes = (size_t)N * C * es, win_bytes = (size_t)N * (width - 1) * C * es;
+    if (overlap(x, xy_bytes, y, xy_bytes) || overlap(win, win_bytes, x, xy_bytes) ||
+        overlap(win, win_bytes, y, xy_bytes))
+        return LA_ERR_INVALID_ARG;
+    ConvArgs a;
+    a.dtype = dtype;
+    a.B = N; a.T = 1; a.H = H; a.d = d; a.width = width;
+    a.step = true;
+    a.silu = (flags & LA_CONV_SILU) != 0;
+    a.l2norm = (flags & LA_CONV_L2NORM) != 0;
+    a.x = x; a.w = w; a.win_in = win; a.win_out = win; a.y = y;
+    a.stream = static_cast<cudaStream_t>(stream);
+    return from_cuda(launch_short_conv(a));
 }
 
 extern "C" la_status_t la_check_status(void *stream) {

@@ -49,6 +49,19 @@ struct DecodeArgs {
     cudaStream_t stream;
 };
 
+struct ConvArgs {
+    int dtype;
+    int B, T, H, d, width;   // B: batch rows (prefill) or sequences N (step)
+    bool step;               // one token per sequence, window updated in place (win_out)
+    bool silu, l2norm;
+    const void *x;
+    const float *w;
+    const void *win_in;      // prefill: nullable (zeros)
+    void *win_out;           // prefill: nullable; step: the window, in/out
+    void *y;
+    cudaStream_t stream;
+};
+
 // Launchers return cudaSuccess or the launch error.  They assume validated arguments.
 cudaError_t launch_decode(const DecodeArgs &a);
 cudaError_t launch_prefill_simt(const PrefillArgs &a);
@@ -56,6 +69,7 @@ bool prefill_simt_supports(int dtype, int dk, int dv, int chunk, int *resolved_c
 bool prefill_tc_supports(int mode, int dtype, int dk, int dv, int chunk);
 size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T);
 cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes);
+cudaError_t launch_short_conv(const ConvArgs &a);
 
 // fp32 <-> I/O element helpers used by the CUDA-core kernels.
 __device__ __forceinline__ float to_f32(float x) { return x; }

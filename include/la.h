@@ -161,6 +161,49 @@ la_status_t la_decode_step(la_mode_t mode, la_dtype_t dtype, int N, int H, int d
                            const float *gate, const float *beta,
                            float *state, float *z, void *o, void *stream);
 
+/* Flags of la_short_conv / la_short_conv_step. */
+#define LA_CONV_SILU 2u     /* y = u * sigmoid(u) after the convolution */
+#define LA_CONV_L2NORM 4u   /* then every head's row y /= sqrt(sum_d y^2 + 1e-6) */
+
+/*
+ * la_short_conv -- the short causal depthwise convolution over time that Gated DeltaNet
+ * and KDA layers put in front of q, k and v (section "Hybrids of 2025: Qwen3-Next and
+ * Kimi Linear": kernel width 4, each token mixed with the three before it).  Per
+ * channel c (C = H * d channels), with the carried window x_{-1} .. x_{-(width-1)}:
+ *
+ *   u_t[c] = sum_{i < width} w[c][i] x_{t-(width-1)+i}[c]      (tap width-1: token t)
+ *
+ * then, per flags, SiLU (LA_CONV_SILU) and the L2 norm of every head's d-row
+ * (LA_CONV_L2NORM), in that order; fp32 arithmetic, one rounding to the I/O dtype.
+ * The page fixes only the causal depthwise convolution and its width; the bias-free
+ * taps, the activation and the norm's 1e-6 are this library's reading.
+ *
+ *   x           [B, T, H*d]          I/O dtype, token-major (a projection's output)
+ *   w           [H*d, width]         fp32 taps
+ *   window_in   [B, width-1, H*d]    I/O dtype, the inputs before x_0 (oldest first), or
+ *                                    NULL for zeros
+ *   window_out  [B, width-1, H*d]    I/O dtype, out: the last width-1 rows of
+ *                                    [window_in; x], or NULL.  May be window_in itself
+ *                                    (the window is then updated in place); any other
+ *                                    overlap is LA_ERR_INVALID_ARG.
+ *   y           [B, H, T, d]         I/O dtype, head-major: the q / k / v input of
+ *                                    la_prefill.  Must not overlap x or the windows.
+ *   d in {64, 128}; width in 1..4 (width 1 takes no window); T >= 0 (T = 0 only
+ *   copies the window).  16-byte alignment for x, y and the windows, 4 for w.
+ */
+la_status_t la_short_conv(la_dtype_t dtype, int B, int T, int H, int d, int width,
+                          const void *x, const float *w, const void *window_in,
+                          void *window_out, void *y, unsigned flags, void *stream);
+
+/*
+ * la_short_conv_step -- la_short_conv for one new token of N sequences (decoding):
+ *   x [N, H*d], window [N, width-1, H*d] updated in place (required when width > 1),
+ *   y [N, H, d] (the q / k / v input of la_decode_step); w and flags as above.
+ */
+la_status_t la_short_conv_step(la_dtype_t dtype, int N, int H, int d, int width,
+                               const void *x, const float *w, void *window, void *y,
+                               unsigned flags, void *stream);
+
 /*
  * la_check_status -- synchronise `stream`, then report the first device-side failure
  * since the last call: LA_ERR_CUDA for a CUDA error, LA_ERR_TIMEOUT if a kernel's
@@ -180,10 +223,11 @@ int la_version(void);
 unsigned long long la_kernel_launches(void);
 
 /* Per-launch device timing, a measurement aid with no counterpart in the pages.
- * la_launch_timing(1) makes every later call of la_prefill, la_prefill_noalloc and
- * la_decode_step bracket each kernel it enqueues with two CUDA events recorded on the
- * call's stream (at most 16 launches per call are timed); la_launch_timing(0) turns it
- * off (the default).  Enabling adds two event records per launch.
+ * la_launch_timing(1) makes every later call of la_prefill, la_prefill_noalloc,
+ * la_decode_step, la_short_conv and la_short_conv_step bracket each kernel it enqueues
+ * with two CUDA events recorded on the call's stream (at most 16 launches per call are
+ * timed); la_launch_timing(0) turns it off (the default).  Enabling adds two event
+ * records per launch.
  *
  * la_launch_times(ms, max_n) waits for the last timed launch of the most recent call,
  * writes the device duration of each of its first max_n launches, in milliseconds and

@@ -117,3 +117,25 @@ def test_launch_timing_without_launches(lib):
     assert lib.la_launch_times(ctypes.cast(buf, ctypes.c_void_p), -1) == -1
     assert lib.la_launch_timing(0) == 0
     assert lib.la_launch_times(ctypes.cast(buf, ctypes.c_void_p), 4) == 0
+
+
+def test_short_conv_argument_checks(lib):
+    INVALID, UNSUPPORTED = 1, 2
+    n = [None] * 5
+
+    def conv(dtype=1, B=1, T=8, H=2, d=128, width=4, flags=0):
+        return lib.la_short_conv(dtype, B, T, H, d, width, *n, flags, None)
+
+    assert conv(dtype=2) == INVALID
+    assert conv(B=0) == INVALID
+    assert conv(T=-1) == INVALID
+    assert conv(width=0) == INVALID
+    assert conv(width=5) == INVALID
+    assert conv(flags=1) == INVALID        # LA_FLAG_INIT_STATE is not a conv flag
+    assert conv(flags=8) == INVALID
+    assert conv(d=96) == UNSUPPORTED
+    assert conv() == INVALID               # NULL taps / tensors, before any launch
+    assert conv(flags=2 | 4) == INVALID
+    assert lib.la_short_conv_step(1, 0, 2, 128, 4, None, None, None, None, 0, None) == INVALID
+    assert lib.la_short_conv_step(1, 1, 2, 96, 4, None, None, None, None, 0, None) == UNSUPPORTED
+    assert lib.la_short_conv_step(1, 1, 2, 128, 4, None, None, None, None, 0, None) == INVALID

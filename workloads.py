@@ -143,3 +143,45 @@ def decode_inputs(w: Workload, steps: int | None = None, device="cpu", n_seqs: i
 def variant(w: Workload, **changes) -> Workload:
     """A copy of a workload with some fields changed (smaller sizes, weaker decay ...)."""
     return dataclasses.replace(w, **changes)
+
+
+# ---- the short causal convolution in front of q, k, v
+@dataclasses.dataclass(frozen=True)
+class ConvWorkload:
+    name: str
+    dtype: torch.dtype          # x, y and the carried window
+    B: int
+    T: int
+    H: int
+    dk: int
+    dv: int
+    width: int
+    seed: int
+    silu: bool = True           # SiLU on q, k, v
+    l2norm_qk: bool = True      # per-head L2 norm of q and k
+
+    @property
+    def tokens(self) -> int:
+        return self.B * self.T
+
+
+# The Gated DeltaNet prefill workload's q, k, v (B2 H16 T32768, d = 128) through the
+# width-4 convolution of the page, with SiLU and the q/k L2 norm.
+CONV_CONFIGS = {
+    "conv_bf16_b2h16t32768": ConvWorkload("conv_bf16_b2h16t32768", torch.bfloat16, B=2, T=32768,
+                                          H=16, dk=128, dv=128, width=4, seed=8),
+}
+
+
+def conv_inputs(B, T, C, width, dtype, seed, device="cpu", window=True):
+    """Projection output x [B,T,C] ~ N(0,1), taps w [C,width] ~ N(0,1)/sqrt(width) (fp32),
+    carried window [B,width-1,C] ~ N(0,1) (or None).  Draw order: x, w, window."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    x = torch.randn(B, T, C, generator=gen, device=device, dtype=torch.float32).to(dtype)
+    w = torch.randn(C, width, generator=gen, device=device, dtype=torch.float32) / math.sqrt(width)
+    win = None
+    if window:
+        win = torch.randn(B, width - 1, C, generator=gen, device=device,
+                          dtype=torch.float32).to(dtype)
+    return x, w, win
