@@ -150,3 +150,38 @@ def decode_step(mode, q, k, v, gate, beta, state, z=None, nthreads=0):
     if rc != 0:
         raise ValueError("oracle_decode_step rejected its arguments")
     return o, S, zz
+
+
+def prefill_packed(mode, q, k, v, cu, gate=None, beta=None, state=None, z=None, nthreads=0):
+    """Packed variable-length sequences: the recurrent form run on every sequence of the
+    packed token axis on its own (sequence s = tokens cu[s] .. cu[s+1]).
+
+    q, k: [H,T,d_k]; v: [H,T,d_v]; gate, beta: [H,T] (mode 3: gate [H,T,d_k]) or None;
+    state: [N,H,d_v,d_k] start states (None -> zero); z: [N,H,d_k] (mode 0).
+    Returns (o [H,T,d_v], S [N,H,d_v,d_k], z [N,H,d_k] or None), fp64.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    H, T, dk = q.shape
+    dv = v.shape[-1]
+    cu = [int(x) for x in np.asarray(cu).reshape(-1)]
+    N = len(cu) - 1
+    o = np.zeros((H, T, dv))
+    S = np.zeros((N, H, dv, dk))
+    zz = np.zeros((N, H, dk)) if mode == 0 else None
+    for s in range(N):
+        a, b = cu[s], cu[s + 1]
+        sl = lambda x: None if x is None else _f64(x)[:, a:b][None]
+        st = None if state is None else _f64(state)[s][None]
+        z0 = None if z is None else _f64(z)[s][None]
+        if b > a:
+            os_, Ss, zs = prefill(mode, sl(q), sl(k), sl(v), sl(gate), sl(beta), st, z0, nthreads)
+            o[:, a:b] = os_[0]
+            S[s] = Ss[0]
+            if zz is not None:
+                zz[s] = zs[0]
+        else:   # no tokens: the state is the start state
+            if state is not None:
+                S[s] = _f64(state)[s]
+            if zz is not None and z is not None:
+                zz[s] = _f64(z)[s]
+    return o, S, zz

@@ -462,3 +462,58 @@ def test_mode3_linear_in_values_from_zero_state():
     o2, S2, _ = run1(3, Q, K, V2, gate=a, beta=b)
     o3, S3, _ = run1(3, Q, K, 2.0 * V - 3.0 * V2, gate=a, beta=b)
     assert np.abs(o3 - (2 * o1 - 3 * o2)).max() < 1e-12 and np.abs(S3 - (2 * S1 - 3 * S2)).max() < 1e-12
+
+
+# ---- packed variable-length sequences
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+def test_packed_equal_lengths_match_the_batched_call(mode):
+    """N packed sequences of one length are the batch [N, H, L, d] of the dense call."""
+    r = np.random.default_rng(70 + mode)
+    N, H, L, dk, dv = 3, 2, 9, 4, 3
+    q, k, v = r.normal(size=(N, H, L, dk)), r.normal(size=(N, H, L, dk)), r.normal(size=(N, H, L, dv))
+    gshape = (N, H, L, dk) if mode == 3 else (N, H, L)
+    gate = None if mode == 0 else 1 / (1 + np.exp(r.normal(size=gshape)))
+    beta = 1 / (1 + np.exp(r.normal(size=(N, H, L)))) if mode >= 2 else None
+    S0 = r.normal(size=(N, H, dv, dk)) * 0.1
+    z0 = r.random(size=(N, H, dk)) + 1.0 if mode == 0 else None
+    o, S, z = oracle.prefill(mode, q, k, v, gate, beta, S0, z0)
+    pk = lambda x: None if x is None else np.concatenate(list(x), axis=1)   # [H, N*L, ..]
+    cu = np.arange(N + 1) * L
+    po, pS, pz = oracle.prefill_packed(mode, pk(q), pk(k), pk(v), cu, pk(gate), pk(beta), S0, z0)
+    np.testing.assert_allclose(po, pk(o), rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(pS, S, rtol=1e-13, atol=1e-13)
+    if mode == 0:
+        np.testing.assert_allclose(pz, z, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("mode", [1, 2, 3])
+def test_packed_boundary_is_a_zero_gate(mode):
+    """The page's document boundary: a gate a_t = 0 at the first token of a document
+    forgets everything before it.  So one dense sequence with a = 0 at each boundary
+    gives the packed result of the documents taken separately from zero states."""
+    r = np.random.default_rng(80 + mode)
+    H, T, dk, dv = 2, 23, 4, 3
+    cu = np.array([0, 7, 8, 16, 23])
+    q, k, v = r.normal(size=(H, T, dk)), r.normal(size=(H, T, dk)), r.normal(size=(H, T, dv))
+    gshape = (H, T, dk) if mode == 3 else (H, T)
+    gate = 1 / (1 + np.exp(r.normal(size=gshape)))
+    beta = 1 / (1 + np.exp(r.normal(size=(H, T)))) if mode >= 2 else None
+    po, pS, _ = oracle.prefill_packed(mode, q, k, v, cu, gate, beta)
+    g0 = gate.copy()
+    g0[:, cu[1:-1]] = 0.0
+    o, S, _ = oracle.prefill(mode, q[None], k[None], v[None], g0[None],
+                             None if beta is None else beta[None])
+    np.testing.assert_allclose(po, o[0], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(pS[-1], S[0], rtol=1e-12, atol=1e-12)
+
+
+def test_packed_empty_sequence_keeps_its_start_state():
+    r = np.random.default_rng(90)
+    H, dk, dv = 2, 4, 3
+    cu = np.array([0, 5, 5, 9])
+    q, k, v = r.normal(size=(H, 9, dk)), r.normal(size=(H, 9, dk)), r.normal(size=(H, 9, dv))
+    S0 = r.normal(size=(3, H, dv, dk))
+    _, pS, _ = oracle.prefill_packed(1, q, k, v, cu, None, None, S0)
+    np.testing.assert_array_equal(pS[1], S0[1])
+    _, pS0, _ = oracle.prefill_packed(1, q, k, v, cu)
+    np.testing.assert_array_equal(pS0[1], 0.0)
