@@ -328,6 +328,50 @@ class DecodeCase:
         self.h_o.copy_(self.o, non_blocking=True)
 
 
+class VarlenCase:
+    """One step = one la_prefill_varlen call over a packed serving batch (sequences of
+    mixed lengths, each with its own state)."""
+
+    def __init__(self, la, vw: W.VarlenWorkload, device, rank):
+        self.la, self.vw, self.device = la, vw, device
+        w = W.variant(vw.base, seed=vw.base.seed + 1000 * rank)
+        self.w = w
+        self.L = vw.lengths()
+        self.inp = W.varlen_inputs(w, self.L, device=device)
+        N, T = len(self.L), sum(self.L)
+        self.state = torch.empty(N, w.H, w.dv, w.dk, device=device)
+        self.z = torch.empty(N, w.H, w.dk, device=device) if w.mode == 0 else None
+        self.o = torch.empty(w.H, T, w.dv, device=device, dtype=w.dtype)
+        self.tokens = T
+        b_tok, f_tok = prefill_algorithmic(W.variant(w, B=1, T=T))
+        # prefill_algorithmic counts one final state per (batch, head): add the other N-1
+        self.bytes = b_tok + (N - 1) * w.H * (w.dv * w.dk * 4 + (w.dk * 4 if w.mode == 0 else 0))
+        self.flops = f_tok
+        self.kind = "prefill_varlen"
+
+    def step(self):
+        i = self.inp
+        self.la.prefill_varlen(i["q"], i["k"], i["v"], i["cu"], mode=self.w.mode, gate=i["gate"],
+                               beta=i["beta"], state=self.state, z=self.z, o=self.o,
+                               init_state=False)
+
+    def e2e_setup(self):
+        pin = lambda t: None if t is None else t.to("cpu").pin_memory()
+        self.h_in = {k: pin(self.inp[k]) for k in ("q", "k", "v", "gate", "beta", "cu")}
+        self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.h_state = torch.empty(self.state.shape, dtype=torch.float32).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values() if t is not None)
+        self.d2h = self.h_o.numel() * self.h_o.element_size() + self.h_state.numel() * 4
+
+    def e2e_step(self):
+        for k, v in self.h_in.items():
+            if v is not None:
+                self.inp[k].copy_(v, non_blocking=True)
+        self.step()
+        self.h_o.copy_(self.o, non_blocking=True)
+        self.h_state.copy_(self.state, non_blocking=True)
+
+
 class ConvCase:
     """One step = the short convolution prologue of one prefill batch: three
     la_short_conv calls (q and k with SiLU and the L2 norm, v with SiLU), token-major
@@ -477,6 +521,8 @@ def roofline(case, kernel_ms, step_ms, peaks, peak_src, prof):
 def measure(la, name, args, dist, device, rank, world, flush, with_e2e, sampler=None):
     if name in W.CONV_CONFIGS:
         case = ConvCase(la, W.CONV_CONFIGS[name], device, rank)
+    elif name in W.VARLEN_CONFIGS:
+        case = VarlenCase(la, W.VARLEN_CONFIGS[name], device, rank)
     else:
         w = W.CONFIGS[name]
         case = (DecodeCase(la, w, device, rank, args.warmup + args.steps) if w.decode
@@ -639,7 +685,7 @@ def main():
     if do_extras:
         for name in ("elu1_bf16_b4h16t4096", "gated_bf16_b8h16t8192", "gdn_bf16_b2h16t32768",
                      "gdn_decode_n256h32", "kda_bf16_b2h16t32768", "kda_decode_n256h32",
-                     "conv_bf16_b2h16t32768"):
+                     "conv_bf16_b2h16t32768", "gdn_varlen_bf16_n64h16"):
             if name == args.workload:
                 continue
             r = measure(la, name, args, dist, device, rank, world, flush, False)

@@ -23,7 +23,7 @@ import os
 import torch
 
 __all__ = ["MODE_ELU1_NORM", "MODE_GATED", "MODE_GATED_DELTA", "MODE_KDA", "FLAG_INIT_STATE", "LaError",
-           "prefill", "decode_step", "short_conv", "short_conv_step", "check_status", "library",
+           "prefill", "prefill_varlen", "decode_step", "short_conv", "short_conv_step", "check_status", "library",
            "library_path", "version", "kernel_launches", "workspace_size"]
 
 MODE_ELU1_NORM = 0
@@ -83,6 +83,9 @@ def library():
     lib.la_version.restype = i
     lib.la_kernel_launches.argtypes = []
     lib.la_kernel_launches.restype = ctypes.c_ulonglong
+    lib.la_prefill_varlen.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, vp, fp, fp, fp, fp, vp, i,
+                                      u, vp]
+    lib.la_prefill_varlen.restype = i
     lib.la_short_conv.argtypes = [i, i, i, i, i, i, vp, fp, vp, vp, vp, u, vp]
     lib.la_short_conv.restype = i
     lib.la_short_conv_step.argtypes = [i, i, i, i, i, vp, fp, vp, vp, u, vp]
@@ -237,6 +240,54 @@ def prefill(q, k, v, *, mode: int, gate=None, beta=None, state=None, z=None, o=N
                               FLAG_INIT_STATE if init_state else 0, _ptr(ws), ws_bytes,
                               _stream_handle(q.device, stream))
     _check(st, "la_prefill")
+    return o, state, (z if mode == MODE_ELU1_NORM else None)
+
+
+def prefill_varlen(q, k, v, cu_seqlens, *, mode: int, gate=None, beta=None, state=None, z=None,
+                   o=None, chunk: int = 0, init_state: bool | None = None, stream=None):
+    """Prefill of N packed sequences (``la_prefill_varlen``).
+
+    q, k: [H,T,d_k]; v: [H,T,d_v] with the N sequences packed along T; cu_seqlens: int32
+    [N+1] on the device (sequence s = tokens cu[s]..cu[s+1]); gate, beta: [H,T] fp32
+    (``MODE_KDA``: gate [H,T,d_k]); state: [N,H,d_v,d_k] fp32 (each sequence's start
+    state when ``init_state``, default: when given); z: [N,H,d_k] (mode 0).
+    Returns (o [H,T,d_v], state, z) with each sequence's final state in its slot.
+    """
+    H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    dtype = _io_dtype(q)
+    N = cu_seqlens.numel() - 1
+    if N < 1:
+        raise ValueError("cu_seqlens needs at least two entries")
+    _need(cu_seqlens, (N + 1,), torch.int32, "cu_seqlens")
+    _need(q, (H, T, dk), dt, "q")
+    _need(k, (H, T, dk), dt, "k")
+    _need(v, (H, T, dv), dt, "v")
+    if gate is not None:
+        _need(gate, (H, T, dk) if mode == MODE_KDA else (H, T), torch.float32, "gate")
+    if beta is not None:
+        _need(beta, (H, T), torch.float32, "beta")
+    if init_state is None:
+        init_state = state is not None
+    if state is None:
+        state = torch.empty(N, H, dv, dk, device=q.device, dtype=torch.float32)
+    _need(state, (N, H, dv, dk), torch.float32, "state")
+    if mode == MODE_ELU1_NORM:
+        if z is None:
+            if init_state:
+                raise ValueError("mode 0 with init_state needs z")
+            z = torch.empty(N, H, dk, device=q.device, dtype=torch.float32)
+        _need(z, (N, H, dk), torch.float32, "z")
+    if o is None:
+        o = torch.empty(H, T, dv, device=q.device, dtype=dt)
+    _need(o, (H, T, dv), dt, "o")
+    st = library().la_prefill_varlen(int(mode), dtype, N, H, T, dk, dv, _ptr(cu_seqlens), _ptr(q),
+                                     _ptr(k), _ptr(v), _ptr(gate), _ptr(beta), _ptr(state),
+                                     _ptr(z), _ptr(o), int(chunk),
+                                     FLAG_INIT_STATE if init_state else 0,
+                                     _stream_handle(q.device, stream))
+    _check(st, "la_prefill_varlen")
     return o, state, (z if mode == MODE_ELU1_NORM else None)
 
 

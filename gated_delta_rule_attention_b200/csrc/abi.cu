@@ -124,6 +124,59 @@ extern "C" la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H
     return from_cuda(launch_prefill_simt(a));
 }
 
+extern "C" la_status_t la_prefill_varlen(la_mode_t mode, la_dtype_t dtype, int N, int H, int T,
+                                         int d_k, int d_v, const int *cu_seqlens, const void *q,
+                                         const void *k, const void *v, const float *gate,
+                                         const float *beta, float *state, float *z, void *o,
+                                         int chunk, unsigned flags, void *stream) {
+    timer_reset();
+    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_KDA) return LA_ERR_INVALID_ARG;
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (N < 1 || H < 1 || T < 0) return LA_ERR_INVALID_ARG;
+    if (flags & ~LA_FLAG_INIT_STATE) return LA_ERR_INVALID_ARG;
+    if (chunk < 0) return LA_ERR_INVALID_ARG;
+    if (!dims_ok(d_k, d_v)) return LA_ERR_UNSUPPORTED;
+    if ((long long)N * H > INT32_MAX || (long long)H * T * (d_k > d_v ? d_k : d_v) > kMaxElems)
+        return LA_ERR_INVALID_ARG;
+    const bool init = (flags & LA_FLAG_INIT_STATE) != 0;
+    if (!tensor_ok(cu_seqlens, 4) || !tensor_ok(state, 16)) return LA_ERR_INVALID_ARG;
+    if (mode == LA_MODE_ELU1_NORM && !tensor_ok(z, 16)) return LA_ERR_INVALID_ARG;
+    if (T > 0) {
+        if (!tensor_ok(q, 16) || !tensor_ok(k, 16) || !tensor_ok(v, 16) || !tensor_ok(o, 16))
+            return LA_ERR_INVALID_ARG;
+        if (mode != LA_MODE_ELU1_NORM && gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
+        if (mode >= LA_MODE_GATED_DELTA && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
+    }
+    PrefillArgs a;
+    a.mode = mode;
+    a.dtype = dtype;
+    a.B = 1; a.H = H; a.T = T; a.dk = d_k; a.dv = d_v;
+    a.q = q; a.k = k; a.v = v;
+    a.gate = (mode == LA_MODE_ELU1_NORM) ? nullptr : gate;
+    a.beta = (mode >= LA_MODE_GATED_DELTA) ? beta : nullptr;
+    a.state = state;
+    a.z = (mode == LA_MODE_ELU1_NORM) ? z : nullptr;
+    a.o = o;
+    a.init_state = init;
+    a.stream = static_cast<cudaStream_t>(stream);
+    a.cu = cu_seqlens;
+    a.nseq = N;
+    if (T == 0) {   // every sequence is empty
+        if (init) return LA_OK;
+        return from_cuda(launch_zero_empty_sequences(a));
+    }
+    if (prefill_tc_supports(mode, dtype, d_k, d_v, chunk)) {
+        a.chunk = 64;
+        cudaError_t e = launch_prefill_tc(a, nullptr, 0);
+        if (e == cudaSuccess && !init) e = launch_zero_empty_sequences(a);
+        return from_cuda(e);
+    }
+    int resolved = 0;
+    if (!prefill_simt_supports(dtype, d_k, d_v, chunk, &resolved)) return LA_ERR_UNSUPPORTED;
+    a.chunk = resolved;
+    return from_cuda(launch_prefill_simt(a));
+}
+
 extern "C" size_t la_prefill_workspace_size(la_mode_t mode, la_dtype_t dtype, int B, int H, int T,
                                             int d_k, int d_v, int chunk) {
     if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_KDA || B < 1 || H < 1 || T < 1)
@@ -245,7 +298,9 @@ extern "C" la_status_t la_check_status(void *stream) {
     const unsigned zero = 0;
     if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
         return LA_ERR_CUDA;
-    return (host & kErrTimeout) ? LA_ERR_TIMEOUT : LA_ERR_CUDA;
+    if (host & kErrTimeout) return LA_ERR_TIMEOUT;
+    if (host & kErrBadInput) return LA_ERR_INVALID_ARG;
+    return LA_ERR_CUDA;
 }
 
 extern "C" const char *la_status_string(la_status_t s) {

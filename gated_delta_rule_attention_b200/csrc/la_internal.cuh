@@ -13,7 +13,7 @@ namespace la {
 // Device-side failure word.  A kernel whose bounded wait runs out ORs a code into it
 // and returns early; la_check_status() reads and clears it.  Kernels receive its
 // address as an argument (device_error_word()), so no relocatable device code is needed.
-enum : unsigned { kErrTimeout = 1u, kErrBadLaunch = 2u };
+enum : unsigned { kErrTimeout = 1u, kErrBadLaunch = 2u, kErrBadInput = 4u };
 unsigned *device_error_word();   // address on the current device, or nullptr on error
 
 // Counts kernels enqueued by the library (la_kernel_launches()).
@@ -37,6 +37,11 @@ struct PrefillArgs {
     int chunk;          // resolved (non-zero) chunk size
     bool init_state;
     cudaStream_t stream;
+    // Packed variable-length sequences: nullptr for dense [B, H, T, d] tensors.
+    // Otherwise B = 1, T = total tokens, the tensors are [H, T, d] (gate/beta [H, T]),
+    // sequence s takes tokens [cu[s], cu[s+1]) and owns state slot s of [nseq, H, ..].
+    const int *cu = nullptr;
+    int nseq = 0;
 };
 
 struct DecodeArgs {
@@ -70,6 +75,8 @@ bool prefill_tc_supports(int mode, int dtype, int dk, int dv, int chunk);
 size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T);
 cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes);
 cudaError_t launch_short_conv(const ConvArgs &a);
+// Zero the state (and z) of every packed sequence with no tokens (cu[s+1] <= cu[s]).
+cudaError_t launch_zero_empty_sequences(const PrefillArgs &a);
 
 // fp32 <-> I/O element helpers used by the CUDA-core kernels.
 __device__ __forceinline__ float to_f32(float x) { return x; }

@@ -29,7 +29,8 @@
 //   (I + Lm) E = diag(b) V - diag(b) (K o G) S^T,   G_ic = exp(lam_ic),
 //   O = (Q o G) S^T + A E,   S <- S Diag(G_L) + E^T (K o exp(lam_L - lam)).
 //
-// One CTA (256 threads) per (batch, head) walks the chunks in order; all tiles are fp32
+// One CTA (256 threads) per (batch, head) -- or per (sequence, head) of packed
+// variable-length sequences -- walks the chunks in order; all tiles are fp32
 // in shared memory with one float of row padding so that row-strided reads are
 // bank-conflict free.
 #include "la_internal.cuh"
@@ -54,10 +55,11 @@ struct SimtSmem {
 
 template <int MODE, int DK, int DV, int C, typename IO>
 __global__ void __launch_bounds__(kSimtThreads)
-prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
-                    const IO *__restrict__ v, const float *__restrict__ gate,
-                    const float *__restrict__ beta, float *__restrict__ state,
-                    float *__restrict__ zg, IO *__restrict__ o, int init_state) {
+prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restrict__ q,
+                    const IO *__restrict__ k, const IO *__restrict__ v,
+                    const float *__restrict__ gate, const float *__restrict__ beta,
+                    float *__restrict__ state, float *__restrict__ zg, IO *__restrict__ o,
+                    int init_state, unsigned *err) {
     using L = SimtSmem<MODE, DK, DV, C>;
     constexpr bool kDelta = (MODE == 2 || MODE == 3);
     extern __shared__ float smem[];
@@ -77,13 +79,26 @@ prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
 
     constexpr int SK = DK + 1, SV = DV + 1, SA = C + 1;
     const int tid = threadIdx.x;
+    // The state slot is blockIdx.x: (batch, head) for dense tensors, (sequence, head) for
+    // packed ones.  row0 is the first token row of the CTA in the [rows][d] view of
+    // q, k, v and o, n its token count.
     const size_t bh = blockIdx.x;
-    const IO *qh = q + bh * (size_t)T * DK;
-    const IO *kh = k + bh * (size_t)T * DK;
-    const IO *vh = v + bh * (size_t)T * DV;
-    IO *oh = o + bh * (size_t)T * DV;
-    const float *gh = gate ? gate + bh * (size_t)T * (MODE == 3 ? DK : 1) : nullptr;
-    const float *bh_beta = beta ? beta + bh * (size_t)T : nullptr;
+    size_t row0 = bh * (size_t)T;
+    int n = T;
+    if (cu) {   // packed: sequence blockIdx.x / H of head row blockIdx.x % H
+        const int sq = blockIdx.x / H, hr = blockIdx.x % H;
+        const int a = cu[sq], b = cu[sq + 1];
+        const int tb = min(max(a, 0), T), te = min(max(b, tb), T);
+        if ((a != tb || b != te) && tid == 0 && err) atomicOr(err, (unsigned)kErrBadInput);
+        row0 = (size_t)hr * T + tb;
+        n = te - tb;
+    }
+    const IO *qh = q + row0 * DK;
+    const IO *kh = k + row0 * DK;
+    const IO *vh = v + row0 * DV;
+    IO *oh = o + row0 * DV;
+    const float *gh = gate ? gate + row0 * (MODE == 3 ? DK : 1) : nullptr;
+    const float *bh_beta = beta ? beta + row0 : nullptr;
     float *Sg = state + bh * (size_t)DV * DK;
 
     for (int p = tid; p < DV * DK; p += kSimtThreads)
@@ -92,8 +107,8 @@ prefill_simt_kernel(int T, const IO *__restrict__ q, const IO *__restrict__ k,
         for (int p = tid; p < DK; p += kSimtThreads) zs[p] = init_state ? zg[bh * DK + p] : 0.f;
     __syncthreads();
 
-    for (int t0 = 0; t0 < T; t0 += C) {
-        const int Lc = min(C, T - t0);
+    for (int t0 = 0; t0 < n; t0 += C) {
+        const int Lc = min(C, n - t0);
         // ---- load the chunk (phi applied in mode 0) and the gates
         for (int p = tid; p < Lc * DK; p += kSimtThreads) {
             const int i = p / DK, j = p % DK;
@@ -243,10 +258,11 @@ cudaError_t launch_one(const PrefillArgs &a) {
                                            (int)L::kBytes);
     if (err != cudaSuccess) return err;
     timer_begin(a.stream);
-    kern<<<(unsigned)((size_t)a.B * a.H), kSimtThreads, L::kBytes, a.stream>>>(
-        a.T, static_cast<const IO *>(a.q), static_cast<const IO *>(a.k),
+    const unsigned grid = (unsigned)(a.cu ? (size_t)a.nseq * a.H : (size_t)a.B * a.H);
+    kern<<<grid, kSimtThreads, L::kBytes, a.stream>>>(
+        a.T, a.H, a.cu, static_cast<const IO *>(a.q), static_cast<const IO *>(a.k),
         static_cast<const IO *>(a.v), a.gate, a.beta, a.state, a.z, static_cast<IO *>(a.o),
-        a.init_state ? 1 : 0);
+        a.init_state ? 1 : 0, device_error_word());
     timer_end(a.stream);
     note_launches(1);
     return cudaGetLastError();

@@ -90,7 +90,49 @@ struct TcParams {
     // read from a start state that a combine kernel wrote.
     const float *fold_init, *fold_zinit, *fold_loc, *fold_zloc, *fold_gam;
     int fold_sub;
+    // Packed variable-length sequences (nullptr: dense).  CTA (s, h) takes tokens
+    // [cu[s], cu[s+1]) of head row h of the packed [H][T][128] tensors; its state is
+    // slot s of the s_in / s_out segment stride.
+    const int *cu;
 };
+
+// The token range of this CTA: segment `seg` of head row `bh`, or, for packed sequences,
+// sequence `seg`.  A cu_seqlens entry outside [0, T] or decreasing is clamped (the CTA
+// stays in bounds) and reported in the failure word.
+struct CtaRange {
+    int bh, seg, tb, te;
+};
+__device__ __forceinline__ CtaRange cta_range(const TcParams &p) {
+    CtaRange r;
+    r.bh = blockIdx.x % p.BH;
+    r.seg = blockIdx.x / p.BH;
+    if (p.cu) {
+        const int a = p.cu[r.seg], b = p.cu[r.seg + 1];
+        r.tb = min(max(a, 0), p.T);
+        r.te = min(max(b, r.tb), p.T);
+        if ((a != r.tb || b != r.te) && threadIdx.x == 0 && p.err) atomicOr(p.err, (unsigned)kErrBadInput);
+    } else {
+        r.tb = r.seg * p.seg_len;
+        r.te = min(p.T, r.tb + p.seg_len);
+    }
+    return r;
+}
+
+// Row t of a chunk's output, 32 columns from col, written straight to global memory as
+// bf16 (the last, partial chunk of a packed sequence: a 64-row TMA store would write
+// into the next sequence's rows).
+__device__ __forceinline__ void st_out_row32(const TcParams &p, int bh, int t, int col, const float *v) {
+    uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)bh * p.T + t) * 128 + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+        w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+        w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+        w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+        dst[q] = w;
+    }
+}
 
 // Start state S[row][c0 .. c0 + 15] of segment `seg` of head bh (modes 0/1).
 __device__ __forceinline__ void start_state16(const TcParams &p, int seg, int bh, int row, int c0,
@@ -393,10 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bh = blockIdx.x % p.BH;
-    const int seg = blockIdx.x / p.BH;
-    const int tb = seg * p.seg_len;
-    const int te = min(p.T, tb + p.seg_len);
+    const CtaRange rng = cta_range(p);
+    const int bh = rng.bh, seg = rng.seg, tb = rng.tb, te = rng.te;
+    if (te <= tb) return;   // an empty packed sequence: nothing to read or write
     const int nch = (te - tb + kC - 1) / kC;
 
     if (threadIdx.x == 0) {
@@ -728,12 +769,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             if (kOut) {
                 const int t = 16 * q + lane;
                 const bool has = lane < 16 && t < L;
+                const bool direct = p.cu && L < kC;   // partial chunk of a packed sequence
                 const uint32_t ost = sb + Y::kOst + h * 8192;
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {
                     float v[32];
                     tmem_ld32(tl + kColO + 64 * h + 32 * sub, v);
-                    if (has) {
+                    if (has && direct) {
+                        st_out_row32(p, bh, t0 + t, 64 * h + 32 * sub, v);
+                    } else if (has) {
                         st_row_bf16x16(ost, t, 4 * sub, v);
                         st_row_bf16x16(ost, t, 4 * sub + 2, v + 16);
                     }
@@ -741,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 fence_async_smem();
                 tc_fence_before();
                 epi_sync();
-                if (e == 0) {
+                if (e == 0 && !direct) {
                     tma_store_3d(&p.to, sb + Y::kOst, 0, t0, bh);
                     tma_store_3d(&p.to, sb + Y::kOst + 8192, 64, t0, bh);
                     tma_store_commit();
@@ -829,10 +873,9 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bh = blockIdx.x % p.BH;
-    const int seg = blockIdx.x / p.BH;
-    const int tb = seg * p.seg_len;
-    const int te = min(p.T, tb + p.seg_len);
+    const CtaRange rng = cta_range(p);
+    const int bh = rng.bh, seg = rng.seg, tb = rng.tb, te = rng.te;
+    if (te <= tb) return;   // an empty packed sequence: nothing to read or write
     const int nch = (te - tb + kC - 1) / kC;
 
     if (threadIdx.x == 0) {
@@ -1098,6 +1141,7 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                 const int L = sm->len[c & 7];
                 const float *lam = sm->lam[c & 7];
                 // ---- outputs of chunk c: row t = r64, columns 64 h + 32 hi + [0, 32)
+                const bool direct = p.cu && L < kC;   // partial chunk of a packed sequence
                 {
                     const int t = r64;
                     const bool has = t < L;
@@ -1107,7 +1151,9 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                     tmem_ld_pair32(tl + kColP01 + 64 * h, pq);
 #pragma unroll
                     for (int k = 0; k < 32; ++k) v[k] = fmaf(scale, pq[k], v[k]);
-                    if (has) {
+                    if (has && direct) {
+                        st_out_row32(p, bh, t0 + t, 64 * h + 32 * hi, v);
+                    } else if (has) {
                         const uint32_t ost = sb + Y::kOst + h * 8192;
                         st_row_bf16x16(ost, t, 4 * hi, v);
                         st_row_bf16x16(ost, t, 4 * hi + 2, v + 16);
@@ -1132,9 +1178,11 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
                 epi_sync();
                 if (e == 0) {
                     mbar_arrive(&sm->s_ready);
-                    tma_store_3d(&p.to, sb + Y::kOst, 0, t0, bh);
-                    tma_store_3d(&p.to, sb + Y::kOst + 8192, 64, t0, bh);
-                    tma_store_commit();
+                    if (!direct) {
+                        tma_store_3d(&p.to, sb + Y::kOst, 0, t0, bh);
+                        tma_store_3d(&p.to, sb + Y::kOst + 8192, 64, t0, bh);
+                        tma_store_commit();
+                    }
                 }
                 if (last && p.s_out && (!p.out_last_only || seg == p.nseg - 1)) {
                     float *dst = p.s_out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
@@ -1255,10 +1303,9 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bh = blockIdx.x % p.BH;
-    const int seg = blockIdx.x / p.BH;
-    const int tb = seg * p.seg_len;
-    const int te = min(p.T, tb + p.seg_len);
+    const CtaRange rng = cta_range(p);
+    const int bh = rng.bh, seg = rng.seg, tb = rng.tb, te = rng.te;
+    if (te <= tb) return;   // an empty packed sequence: nothing to read or write
     const int nch = (te - tb + kC - 1) / kC;
 
     if (threadIdx.x == 0) {
@@ -1603,6 +1650,7 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                 }
                 if (named_sync_any(1, kEpi, !w_ok)) break;
                 tc_fence_after();
+                const bool direct = p.cu && sm->len[c & 7] < kC;   // partial packed chunk
                 {
                     const int L = sm->len[c & 7];
                     const int t = r64;
@@ -1616,7 +1664,9 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                     tmem_ld_pair32(tl + kColOE + 128 * b + 64 * h, v);
 #pragma unroll
                     for (int k = 0; k < 32; ++k) v[k] *= scale;
-                    if (has) {   // this chunk's V slot: [V0 | V1] -> [O0 | O1], 8 KB each
+                    if (has && direct) {
+                        st_out_row32(p, bh, t0 + t, 64 * h + 32 * hi, v);
+                    } else if (has) {   // this chunk's V slot: [V0 | V1] -> [O0 | O1], 8 KB each
                         const uint32_t ost = sb + Y::kV + (c % NV) * 16384 + h * 8192;
                         st_row_bf16x16(ost, t, 4 * hi, v);
                         st_row_bf16x16(ost, t, 4 * hi + 2, v + 16);
@@ -1627,10 +1677,12 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
                 epi_sync();
                 if (e == 0) {
                     mbar_arrive(&sm->o_free[b]);
-                    const uint32_t ost = sb + Y::kV + (c % NV) * 16384;
-                    tma_store_3d(&p.to, ost, 0, t0, bh);
-                    tma_store_3d(&p.to, ost + 8192, 64, t0, bh);
-                    tma_store_commit();
+                    if (!direct) {
+                        const uint32_t ost = sb + Y::kV + (c % NV) * 16384;
+                        tma_store_3d(&p.to, ost, 0, t0, bh);
+                        tma_store_3d(&p.to, ost + 8192, 64, t0, bh);
+                        tma_store_commit();
+                    }
                 }
             }
             if (e == 0) tma_store_wait_all<0>();
@@ -1930,6 +1982,26 @@ size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T) {
     return sizeof(float) * workspace_floats(mode, BH, plan_for(mode, BH, T));
 }
 
+// Packed sequences: one outputs-pass CTA per (sequence, head), started from the
+// sequence's own state slot (or zero) and writing its final state there.
+template <int MODE>
+cudaError_t run_packed(const PrefillArgs &a, const TcParams &base) {
+    TcParams p = base;
+    p.cu = a.cu;
+    p.nseg = a.nseq;
+    p.s_in_mode = a.init_state ? 1 : 0;
+    p.s_in = a.state;
+    p.s_in_seg = (long long)a.H * kD * kD;
+    p.z_in = a.z;
+    p.z_in_seg = (long long)a.H * kD;
+    p.s_out = a.state;
+    p.s_out_seg = (long long)a.H * kD * kD;
+    p.z_out = a.z;
+    p.z_out_seg = (long long)a.H * kD;
+    p.out_last_only = 0;
+    return launch_kind<MODE, kOutput>(p, a.nseq * a.H, a.stream);
+}
+
 cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes) {
     const int BH = a.B * a.H;
     Plan pl = plan_for(a.mode, BH, a.T);
@@ -1958,6 +2030,14 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t work
     p.nseg = pl.nseg;
     p.err = device_error_word();
     float *ws = static_cast<float *>(workspace);
+    if (a.cu) {
+        switch (a.mode) {
+            case LA_MODE_ELU1_NORM: return run_packed<0>(a, p);
+            case LA_MODE_GATED: return run_packed<1>(a, p);
+            case LA_MODE_GATED_DELTA: return run_packed<2>(a, p);
+        }
+        return cudaErrorInvalidValue;
+    }
     switch (a.mode) {
         case LA_MODE_ELU1_NORM: return run_mode<0>(a, p, pl, ws);
         case LA_MODE_GATED: return run_mode<1>(a, p, pl, ws);

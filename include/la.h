@@ -119,6 +119,33 @@ la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H, int T, in
                        void *stream);
 
 /*
+ * la_prefill_varlen -- la_prefill over N packed sequences of different lengths, each
+ * with its own state: the batch of a serving step, or a prompt resumed from a cached
+ * prefix state.  Sequence s is tokens [cu_seqlens[s], cu_seqlens[s+1]) of the packed
+ * token axis; nothing crosses from one sequence into the next, exactly as if each were
+ * a separate la_prefill call.  (Inside one sequence, a gate a_t = 0 forgets everything
+ * before token t, the document-boundary reading of [decay/gates].)
+ *
+ *   cu_seqlens  [N + 1] int32, DEVICE memory: non-decreasing offsets within [0, T]
+ *               (cu_seqlens[0] = 0 and cu_seqlens[N] = T in the usual case).  Entries
+ *               outside [0, T] or decreasing are clamped on the device and reported as
+ *               LA_ERR_INVALID_ARG by la_check_status().  Empty sequences are allowed.
+ *   q, k        [H, T, d_k]  I/O dtype (the [1, H, T, d] layout of la_prefill)
+ *   v, o        [H, T, d_v]  I/O dtype
+ *   gate        [H, T] fp32 or NULL (mode 3: [H, T, d_k])     beta [H, T] fp32 (modes 2, 3)
+ *   state       [N, H, d_v, d_k] fp32: in (with LA_FLAG_INIT_STATE: each sequence's
+ *               start state, e.g. a cached prefix's final state) and out (each
+ *               sequence's final state -- the snapshot to cache or to decode from)
+ *   z           [N, H, d_k] fp32, mode 0 only, in/out like state
+ *   chunk, flags as for la_prefill.  No workspace: one CTA per (sequence, head).
+ */
+la_status_t la_prefill_varlen(la_mode_t mode, la_dtype_t dtype, int N, int H, int T, int d_k,
+                              int d_v, const int *cu_seqlens, const void *q, const void *k,
+                              const void *v, const float *gate, const float *beta,
+                              float *state, float *z, void *o, int chunk, unsigned flags,
+                              void *stream);
+
+/*
  * la_prefill_workspace_size -- bytes of workspace la_prefill can use for these sizes
  * (0 when the kernel for them needs none).  Host-only; touches no device.
  */
@@ -207,7 +234,9 @@ la_status_t la_short_conv_step(la_dtype_t dtype, int N, int H, int d, int width,
 /*
  * la_check_status -- synchronise `stream`, then report the first device-side failure
  * since the last call: LA_ERR_CUDA for a CUDA error, LA_ERR_TIMEOUT if a kernel's
- * bounded wait ran out (the kernel then returned early and its outputs are invalid).
+ * bounded wait ran out (the kernel then returned early and its outputs are invalid),
+ * LA_ERR_INVALID_ARG if a kernel met an invalid device-side argument (a cu_seqlens
+ * entry out of range).
  * Clears the recorded failure.  Returns LA_OK if nothing failed.
  */
 la_status_t la_check_status(void *stream);
@@ -224,7 +253,8 @@ unsigned long long la_kernel_launches(void);
 
 /* Per-launch device timing, a measurement aid with no counterpart in the pages.
  * la_launch_timing(1) makes every later call of la_prefill, la_prefill_noalloc,
- * la_decode_step, la_short_conv and la_short_conv_step bracket each kernel it enqueues
+ * la_prefill_varlen, la_decode_step, la_short_conv and la_short_conv_step bracket each
+ * kernel it enqueues
  * with two CUDA events recorded on the call's stream (at most 16 launches per call are
  * timed); la_launch_timing(0) turns it off (the default).  Enabling adds two event
  * records per launch.

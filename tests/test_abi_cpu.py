@@ -139,3 +139,21 @@ def test_short_conv_argument_checks(lib):
     assert lib.la_short_conv_step(1, 0, 2, 128, 4, None, None, None, None, 0, None) == INVALID
     assert lib.la_short_conv_step(1, 1, 2, 96, 4, None, None, None, None, 0, None) == UNSUPPORTED
     assert lib.la_short_conv_step(1, 1, 2, 128, 4, None, None, None, None, 0, None) == INVALID
+
+
+def test_prefill_varlen_argument_checks(lib):
+    INVALID, UNSUPPORTED = 1, 2
+
+    def call(mode=2, dtype=1, N=2, H=2, T=100, dk=128, dv=128, chunk=0, flags=0):
+        return lib.la_prefill_varlen(mode, dtype, N, H, T, dk, dv, *([None] * 9), chunk, flags, None)
+
+    assert call(mode=4) == INVALID
+    assert call(dtype=3) == INVALID
+    assert call(N=0) == INVALID
+    assert call(H=0) == INVALID
+    assert call(T=-1) == INVALID
+    assert call(flags=2) == INVALID
+    assert call(chunk=-1) == INVALID
+    assert call(dk=96) == UNSUPPORTED
+    assert call() == INVALID          # NULL cu_seqlens / tensors, before any launch
+    assert call(T=0) == INVALID       # still needs the offsets and the state

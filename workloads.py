@@ -185,3 +185,61 @@ def conv_inputs(B, T, C, width, dtype, seed, device="cpu", window=True):
         win = torch.randn(B, width - 1, C, generator=gen, device=device,
                           dtype=torch.float32).to(dtype)
     return x, w, win
+
+
+# ---- packed variable-length sequences
+@dataclasses.dataclass(frozen=True)
+class VarlenWorkload:
+    name: str
+    base: Workload              # mode, dtype, H, d, recipes; its B and T are unused
+    N: int                      # sequences
+    min_len: int
+    max_len: int                # lengths log-uniform in [min_len, max_len]
+
+    def lengths(self) -> list:
+        return varlen_lengths(self.N, self.min_len, self.max_len, self.base.seed)
+
+    @property
+    def tokens(self) -> int:
+        return sum(self.lengths())
+
+
+def varlen_lengths(N, lo, hi, seed):
+    """N sequence lengths, log-uniform in [lo, hi] (a serving batch's mix of short and
+    long prompts), drawn from their own generator."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed + 777)
+    u = torch.rand(N, generator=gen, dtype=torch.float64)
+    return [int(round(math.exp(math.log(lo) + float(x) * (math.log(hi) - math.log(lo))))) for x in u]
+
+
+def varlen_inputs(w: Workload, lengths, device="cpu", init_state_std: float = 0.0):
+    """Packed q,k [H,T,d_k], v [H,T,d_v], gate/beta [H,T] (mode 3: gate [H,T,d_k]),
+    cu_seqlens int32 [N+1] and start states [N,H,d_v,d_k] (zeros unless init_state_std),
+    drawn with the recipes of `w` (its B and T are ignored)."""
+    T = int(sum(lengths))
+    wp = dataclasses.replace(w, B=1, T=T)
+    d = prefill_inputs(wp, device=device)
+    out = {k: (None if d[k] is None else d[k][0].contiguous()) for k in ("q", "k", "v", "gate", "beta")}
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + int(n))
+    out["cu"] = torch.tensor(cu, dtype=torch.int32, device=device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed + 4242)
+    N = len(lengths)
+    if init_state_std > 0:
+        out["state0"] = torch.randn(N, w.H, w.dv, w.dk, generator=gen, device=device) * init_state_std
+    else:
+        out["state0"] = torch.zeros(N, w.H, w.dv, w.dk, device=device)
+    return out
+
+
+# A serving-style batch for the Gated DeltaNet recipe: 64 sequences of 64 .. 8192 tokens.
+VARLEN_CONFIGS = {
+    "gdn_varlen_bf16_n64h16": VarlenWorkload(
+        "gdn_varlen_bf16_n64h16",
+        Workload("gdn_varlen_bf16_n64h16", MODE_GATED_DELTA, torch.bfloat16, B=1, H=16, T=0, dk=128,
+                 dv=128, seed=9, qk_l2norm=True, gate="softplus", beta=True),
+        N=64, min_len=64, max_len=8192),
+}
