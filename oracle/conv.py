@@ -71,6 +71,29 @@ def short_conv_step(x, w, window, H=1, silu=False, l2norm=False):
     return y[:, :, 0, :], win_new
 
 
+def short_conv_packed(x, w, cu, window=None, H=1, silu=False, l2norm=False):
+    """Packed variable-length sequences: sequence s = tokens cu[s] .. cu[s+1] of the packed
+    axis, each convolved on its own with its own carried window.
+
+    x: [T, C]; window: [N, width-1, C] or None (zeros).  Returns (y [H, T, d],
+    window_out [N, width-1, C]).
+    """
+    x, w = _f64(x), _f64(w)
+    T, C = x.shape
+    width = w.shape[1]
+    cu = [int(c) for c in np.asarray(cu).reshape(-1)]
+    N = len(cu) - 1
+    y = np.zeros((H, T, C // H))
+    wout = np.zeros((N, width - 1, C))
+    for s in range(N):
+        a, b = cu[s], cu[s + 1]
+        win = None if window is None else _f64(window)[s][None]
+        ys, ws = short_conv(x[a:b][None], w, win, H, silu, l2norm)
+        y[:, a:b] = ys[0]
+        wout[s] = ws[0]
+    return y, wout
+
+
 def _activate(u, H, silu, l2norm):
     if silu:
         u = u / (1.0 + np.exp(-u))

@@ -140,3 +140,31 @@ def test_heads_are_normalised_separately():
     x = np.array([[[3.0, 4.0, 0.0, 2.0]]])
     y, _ = conv.short_conv(x, ident, None, H=H, l2norm=True)
     np.testing.assert_allclose(y[0, :, 0], [[0.6, 0.8], [0.0, 1.0]], rtol=1e-6)
+
+
+def test_packed_equal_lengths_match_the_batched_call():
+    x, w, win = _inputs(12, B=3, T=11)
+    y, wout = conv.short_conv(x, w, win, H=3, silu=True, l2norm=True)
+    B, T, C = x.shape
+    cu = np.arange(B + 1) * T
+    py, pw = conv.short_conv_packed(x.reshape(B * T, C), w, cu, win, H=3, silu=True, l2norm=True)
+    np.testing.assert_allclose(py, np.concatenate(list(y), axis=1), rtol=1e-13, atol=1e-13)
+    np.testing.assert_array_equal(pw, wout)
+
+
+def test_packed_sequences_do_not_mix():
+    """A sequence's first outputs see only its own window, never the previous sequence's
+    last tokens; an empty sequence passes its window through."""
+    r = np.random.default_rng(13)
+    C, width = 8, 4
+    cu = np.array([0, 5, 5, 12])
+    x = r.normal(size=(12, C))
+    w = r.normal(size=(C, width))
+    py, pw = conv.short_conv_packed(x, w, cu, None, H=1)
+    alone, _ = conv.short_conv(x[5:12][None], w, None, H=1)
+    np.testing.assert_array_equal(py[:, 5:12], alone[0])
+    np.testing.assert_array_equal(pw[1], 0.0)
+    win = r.normal(size=(3, width - 1, C))
+    _, pw2 = conv.short_conv_packed(x, w, cu, win, H=1)
+    np.testing.assert_array_equal(pw2[1], win[1])
+    np.testing.assert_array_equal(pw2[2], x[9:12])
