@@ -23,7 +23,7 @@ import os
 import torch
 
 __all__ = ["MODE_ELU1_NORM", "MODE_GATED", "MODE_GATED_DELTA", "MODE_KDA", "FLAG_INIT_STATE", "LaError",
-           "prefill", "prefill_varlen", "decode_step", "short_conv", "short_conv_step", "check_status", "library",
+           "prefill", "prefill_varlen", "decode_step", "short_conv", "short_conv_varlen", "short_conv_step", "check_status", "library",
            "library_path", "version", "kernel_launches", "workspace_size"]
 
 MODE_ELU1_NORM = 0
@@ -88,8 +88,12 @@ def library():
     lib.la_prefill_varlen.restype = i
     lib.la_short_conv.argtypes = [i, i, i, i, i, i, vp, fp, vp, vp, vp, u, vp]
     lib.la_short_conv.restype = i
+    lib.la_short_conv_varlen.argtypes = [i, i, i, i, i, i, vp, vp, fp, vp, vp, vp, u, vp]
+    lib.la_short_conv_varlen.restype = i
     lib.la_short_conv_step.argtypes = [i, i, i, i, i, vp, fp, vp, vp, u, vp]
     lib.la_short_conv_step.restype = i
+    lib.la_selftest_wait_timeout.argtypes = [vp]
+    lib.la_selftest_wait_timeout.restype = i
     if hasattr(lib, "la_launch_timing"):   # diagnostic hook, absent from older builds
         lib.la_launch_timing.argtypes = [i]
         lib.la_launch_timing.restype = i
@@ -376,6 +380,37 @@ def short_conv(x, w, *, heads: int, window=None, window_out=None, silu: bool = F
     return y, window_out
 
 
+def short_conv_varlen(x, w, cu_seqlens, *, heads: int, window=None, window_out=None,
+                      silu: bool = False, l2norm: bool = False, y=None, stream=None):
+    """Packed variable-length sequences (``la_short_conv_varlen``): x [T, H*d] holds N
+    sequences back to back (cu_seqlens int32 [N+1] on the device), window / window_out
+    [N, width-1, H*d].  Returns (y [H, T, d], window_out)."""
+    T, C = x.shape
+    width = w.shape[1]
+    if C % heads:
+        raise ValueError("x's last dimension must be heads * d")
+    d = C // heads
+    N = cu_seqlens.numel() - 1
+    dt = x.dtype
+    dtype = _io_dtype(x)
+    _need(cu_seqlens, (N + 1,), torch.int32, "cu_seqlens")
+    _need(x, (T, C), dt, "x")
+    _need(w, (C, width), torch.float32, "w")
+    if window is not None:
+        _need(window, (N, width - 1, C), dt, "window")
+    if window_out is None:
+        window_out = torch.empty(N, width - 1, C, device=x.device, dtype=dt)
+    _need(window_out, (N, width - 1, C), dt, "window_out")
+    if y is None:
+        y = torch.empty(heads, T, d, device=x.device, dtype=dt)
+    _need(y, (heads, T, d), dt, "y")
+    st = library().la_short_conv_varlen(dtype, N, T, heads, d, width, _ptr(cu_seqlens), _ptr(x),
+                                        _ptr(w), _ptr(window), _ptr(window_out), _ptr(y),
+                                        _conv_flags(silu, l2norm), _stream_handle(x.device, stream))
+    _check(st, "la_short_conv_varlen")
+    return y, window_out
+
+
 def short_conv_step(x, w, window, *, heads: int, silu: bool = False, l2norm: bool = False,
                     y=None, stream=None):
     """One new token of N sequences (``la_short_conv_step``): x [N, H*d], window
@@ -399,6 +434,13 @@ def short_conv_step(x, w, window, *, heads: int, silu: bool = False, l2norm: boo
                                       _conv_flags(silu, l2norm), _stream_handle(x.device, stream))
     _check(st, "la_short_conv_step")
     return y
+
+
+def selftest_wait_timeout(stream=None):
+    """Enqueue the failure-path self-test (``la_selftest_wait_timeout``): the next
+    ``check_status`` raises LaError with LA_ERR_TIMEOUT."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(library().la_selftest_wait_timeout(_stream_handle(dev, stream)), "la_selftest_wait_timeout")
 
 
 def check_status(stream=None):

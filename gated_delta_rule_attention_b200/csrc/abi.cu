@@ -257,6 +257,46 @@ extern "C" la_status_t la_short_conv(la_dtype_t dtype, int B, int T, int H, int 
     return from_cuda(launch_short_conv(a));
 }
 
+extern "C" la_status_t la_short_conv_varlen(la_dtype_t dtype, int N, int T, int H, int d,
+                                            int width, const int *cu_seqlens, const void *x,
+                                            const float *w, const void *window_in,
+                                            void *window_out, void *y, unsigned flags,
+                                            void *stream) {
+    timer_reset();
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (N < 1 || T < 0 || H < 1 || width < 1 || width > 4) return LA_ERR_INVALID_ARG;
+    if (flags & ~(LA_CONV_SILU | LA_CONV_L2NORM)) return LA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
+    const long long C = (long long)H * d;
+    if (C > INT32_MAX || (long long)T * C > kMaxElems || (long long)N * C * width > kMaxElems)
+        return LA_ERR_INVALID_ARG;
+    if (!tensor_ok(w, 4) || !tensor_ok(cu_seqlens, 4)) return LA_ERR_INVALID_ARG;
+    const size_t es = dtype == LA_BF16 ? 2 : 4;
+    const size_t win_bytes = (size_t)N * (width - 1) * C * es;
+    const void *win_in = width > 1 ? window_in : nullptr;
+    void *win_out = width > 1 ? window_out : nullptr;
+    if (win_in && !tensor_ok(win_in, 16)) return LA_ERR_INVALID_ARG;
+    if (win_out && !tensor_ok(win_out, 16)) return LA_ERR_INVALID_ARG;
+    if (win_in != win_out && overlap(win_in, win_bytes, win_out, win_bytes)) return LA_ERR_INVALID_ARG;
+    if (T > 0) {
+        if (!tensor_ok(x, 16) || !tensor_ok(y, 16)) return LA_ERR_INVALID_ARG;
+        const size_t xy_bytes = (size_t)T * C * es;
+        if (overlap(x, xy_bytes, y, xy_bytes) || overlap(y, xy_bytes, win_in, win_bytes) ||
+            overlap(y, xy_bytes, win_out, win_bytes) || overlap(x, xy_bytes, win_out, win_bytes))
+            return LA_ERR_INVALID_ARG;
+    }
+    ConvArgs a;
+    a.dtype = dtype;
+    a.B = N; a.T = T; a.H = H; a.d = d; a.width = width;
+    a.step = false;
+    a.silu = (flags & LA_CONV_SILU) != 0;
+    a.l2norm = (flags & LA_CONV_L2NORM) != 0;
+    a.x = x; a.w = w; a.win_in = win_in; a.win_out = win_out; a.y = y;
+    a.stream = static_cast<cudaStream_t>(stream);
+    a.cu = cu_seqlens;
+    return from_cuda(launch_short_conv(a));
+}
+
 extern "C" la_status_t la_short_conv_step(la_dtype_t dtype, int N, int H, int d, int width,
                                           const void *x, const float *w, void *window, void *y,
                                           unsigned flags, void *stream) {

@@ -188,12 +188,21 @@ __device__ __forceinline__ Vec8 conv_step(const float (&wr)[W][8], Raw<IO> (&win
     return u;
 }
 
+// Offset i of a packed sequence table, clamped to [0, T] (a bad table stays in bounds;
+// the window pass reports it).
+__device__ __forceinline__ int cu_at(const int *cu, int i, int T) { return min(max(cu[i], 0), T); }
+
 // Three CTAs per SM for bf16 (80 registers); fp32 rows take twice the registers.
-template <int W, typename IO, bool SILU, bool L2, int NL>
+// PACKED: x is [T][C] holding N sequences back to back (sequence s = tokens cu[s] ..
+// cu[s+1]); a thread's run may cross sequence starts, where its window restarts from
+// that sequence's carried window.  The windows after the call are written by
+// packed_window_kernel.
+template <int W, typename IO, bool SILU, bool L2, int NL, bool PACKED>
 __global__ void __launch_bounds__(kConvThreads, sizeof(IO) == 2 ? 3 : 2)
 short_conv_kernel(int T, int H, int nrun, long long total, const IO *__restrict__ x,
                   const float *__restrict__ w, const IO *__restrict__ win_in,
-                  IO *__restrict__ win_out, IO *__restrict__ y) {
+                  IO *__restrict__ win_out, IO *__restrict__ y, const int *__restrict__ cu,
+                  int N) {
     constexpr int d = NL * 8;
     constexpr int kVec = sizeof(Raw<IO>) / 16;    // 16-byte pieces per 8 channels
     extern __shared__ uint4 ring[];               // [kDepth][kConvThreads][kVec]
@@ -229,13 +238,47 @@ short_conv_kernel(int T, int H, int nrun, long long total, const IO *__restrict_
     load_taps<W>(w, c0, wr);
     constexpr int WM = W > 1 ? W - 1 : 1;
     Raw<IO> win[WM];
+    // packed: the sequence sq holding the current token, its first token a, and the next
+    // sequence start nb
+    int sq = 0, a = 0, nb = T;
+    // the window in front of token t: rows of the current sequence, else its carried
+    // window (index W-1 + row - a, within [0, W-2] because t >= a), else zeros
+    auto load_window = [&](int t, const IO *wsrc) {
 #pragma unroll
-    for (int i = 0; i < W - 1; ++i) {
-        const int t = t0 - (W - 1) + i;
-        if (t >= 0) win[i].load(xb + (size_t)t * C);
-        else if (win_in) win[i].load(win_in + ((size_t)b * (W - 1) + (W - 1) + t) * C + c0);
-        else win[i].zero();
+        for (int i = 0; i < W - 1; ++i) {
+            const int row = t - (W - 1) + i;
+            if (row >= a) win[i].load(xb + (size_t)row * C);
+            else if (wsrc) win[i].load(wsrc + (size_t)((W - 1) + row - a) * C);
+            else win[i].zero();
+        }
+    };
+    if constexpr (PACKED) {
+        int lo = 0, hi = N - 1;   // the last sequence starting at or before t0
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (cu_at(cu, mid, T) <= t0) lo = mid;
+            else hi = mid - 1;
+        }
+        sq = lo;
+        a = min(cu_at(cu, sq, T), t0);
+        nb = max(cu_at(cu, sq + 1, T), t0 + 1);
+        load_window(t0, win_in ? win_in + (size_t)sq * (W - 1) * C + c0 : nullptr);
+    } else {
+#pragma unroll
+        for (int i = 0; i < W - 1; ++i) {
+            const int t = t0 - (W - 1) + i;
+            if (t >= 0) win[i].load(xb + (size_t)t * C);
+            else if (win_in) win[i].load(win_in + ((size_t)b * (W - 1) + (W - 1) + t) * C + c0);
+            else win[i].zero();
+        }
     }
+    // packed: token t starts a later sequence; move to it and restart the window
+    auto enter = [&](int t) {
+        while (sq + 1 < N && cu_at(cu, sq + 1, T) <= t) ++sq;
+        a = min(cu_at(cu, sq, T), t);
+        nb = (sq + 1 < N) ? max(cu_at(cu, sq + 1, T), t + 1) : T;
+        load_window(t, win_in ? win_in + (size_t)sq * (W - 1) * C + c0 : nullptr);
+    };
     IO *yb = y + (((size_t)b * H + h) * T) * d + dd;
     for (int tb = t0; tb < t1; tb += kDepth) {
 #pragma unroll
@@ -252,7 +295,9 @@ short_conv_kernel(int T, int H, int nrun, long long total, const IO *__restrict_
                 // The second row of a pair past the run's end is stale slot contents:
                 // computed but never stored (a conditional step would cost registers), so
                 // the window registers are not the carried window at the end.
+                if (PACKED && t >= nb) enter(t);
                 Vec8 u0 = conv_step<W, IO>(wr, win, x0);
+                if (PACKED && has1 && t + 1 >= nb) enter(t + 1);
                 Vec8 u1 = conv_step<W, IO>(wr, win, x1);
                 // refill both slots with the rows kDepth further on
                 if (t + kDepth < t1) fetch(k, t + kDepth);
@@ -267,7 +312,7 @@ short_conv_kernel(int T, int H, int nrun, long long total, const IO *__restrict_
     // The carried window after the sequence, the last W-1 rows of [win_in; x]: written
     // by the run-0 thread, the only one that reads win_in, so that win_out may be win_in
     // itself.
-    if (win_out && run == 0) {
+    if (!PACKED && win_out && run == 0) {
 #pragma unroll
         for (int i = 0; i < W - 1; ++i) {
             const int t = T - (W - 1) + i;
@@ -279,6 +324,36 @@ short_conv_kernel(int T, int H, int nrun, long long total, const IO *__restrict_
         }
     }
     cp_async_wait<0>();   // no copy may still target shared memory at exit
+}
+
+// Packed sequences: window_out[s] = the last W-1 rows of [window_in[s]; x[cu[s] ..
+// cu[s+1]]], one thread per (sequence, 8 channels).  Runs after the main pass (stream
+// order), so window_out may be window_in: each thread reads its rows before writing.
+// A decreasing or out-of-range offset is reported in the failure word.
+template <int W, typename IO>
+__global__ void __launch_bounds__(kConvThreads)
+packed_window_kernel(int T, int C, int N, const int *__restrict__ cu, const IO *__restrict__ x,
+                     const IO *__restrict__ win_in, IO *__restrict__ win_out, unsigned *err) {
+    const long long idx = (long long)blockIdx.x * kConvThreads + threadIdx.x;
+    const int G = C >> 3;
+    if (idx >= (long long)N * G) return;
+    const int sq = (int)(idx / G), c0 = 8 * (int)(idx % G);
+    const int ra = cu[sq], rb = cu[sq + 1];
+    const int a = cu_at(cu, sq, T), b = max(cu_at(cu, sq + 1, T), a);
+    if ((ra != a || rb != b) && err) atomicOr(err, (unsigned)kErrBadInput);
+    if (W == 1 || !win_out) return;
+    constexpr int WM = W > 1 ? W - 1 : 1;
+    Raw<IO> r[WM];
+    const IO *wsrc = win_in ? win_in + (size_t)sq * (W - 1) * C + c0 : nullptr;
+#pragma unroll
+    for (int i = 0; i < W - 1; ++i) {
+        const int row = b - (W - 1) + i;
+        if (row >= a) r[i].load(x + (size_t)row * C + c0);
+        else if (wsrc) r[i].load(wsrc + (size_t)((W - 1) + row - a) * C);
+        else r[i].zero();
+    }
+#pragma unroll
+    for (int i = 0; i < W - 1; ++i) r[i].store(win_out + ((size_t)sq * (W - 1) + i) * C + c0);
 }
 
 template <int W, typename IO, bool SILU, bool L2, int NL>
@@ -321,19 +396,48 @@ cudaError_t launch_conv(const ConvArgs &a) {
             a.H, total, static_cast<const IO *>(a.x), a.w, static_cast<IO *>(a.win_out),
             static_cast<IO *>(a.y));
         timer_end(a.stream);
+    } else if (a.cu) {
+        const int nrun = (a.T + kRun - 1) / kRun;
+        const long long total = (long long)nrun * G;
+        const unsigned blocks = (unsigned)((total + kConvThreads - 1) / kConvThreads);
+        const int smem = kDepth * kConvThreads * (int)sizeof(Raw<IO>);
+        auto kern = short_conv_kernel<W, IO, SILU, L2, NL, true>;
+        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (err != cudaSuccess) return err;
+        if (a.T > 0) {
+            timer_begin(a.stream);
+            kern<<<blocks, kConvThreads, smem, a.stream>>>(
+                a.T, a.H, nrun, total, static_cast<const IO *>(a.x), a.w,
+                static_cast<const IO *>(a.win_in), nullptr, static_cast<IO *>(a.y), a.cu, a.B);
+            timer_end(a.stream);
+            note_launches(1);
+            err = cudaGetLastError();
+            if (err != cudaSuccess) return err;
+        }
+        {   // the window pass (also the check of the offsets table)
+            const long long nt = (long long)a.B * G;
+            timer_begin(a.stream);
+            packed_window_kernel<W, IO><<<(unsigned)((nt + kConvThreads - 1) / kConvThreads),
+                                          kConvThreads, 0, a.stream>>>(
+                a.T, C, a.B, a.cu, static_cast<const IO *>(a.x), static_cast<const IO *>(a.win_in),
+                static_cast<IO *>(a.win_out), device_error_word());
+            timer_end(a.stream);
+            note_launches(1);
+        }
+        return cudaGetLastError();
     } else {
         const int nrun = (a.T + kRun - 1) / kRun;
         const long long total = (long long)a.B * nrun * G;
         const unsigned blocks = (unsigned)((total + kConvThreads - 1) / kConvThreads);
         const int smem = kDepth * kConvThreads * (int)sizeof(Raw<IO>);
-        auto kern = short_conv_kernel<W, IO, SILU, L2, NL>;
+        auto kern = short_conv_kernel<W, IO, SILU, L2, NL, false>;
         cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err != cudaSuccess) return err;
         timer_begin(a.stream);
         kern<<<blocks, kConvThreads, smem, a.stream>>>(
             a.T, a.H, nrun, total, static_cast<const IO *>(a.x), a.w,
             static_cast<const IO *>(a.win_in), static_cast<IO *>(a.win_out),
-            static_cast<IO *>(a.y));
+            static_cast<IO *>(a.y), nullptr, 0);
         timer_end(a.stream);
     }
     note_launches(1);

@@ -65,6 +65,9 @@ struct ConvArgs {
     void *win_out;           // prefill: nullable; step: the window, in/out
     void *y;
     cudaStream_t stream;
+    // packed variable-length sequences (prefill only): B = N sequences, T = total tokens,
+    // x [T, H*d], y [H, T, d], windows [N, W-1, H*d]; nullptr for dense
+    const int *cu = nullptr;
 };
 
 // Launchers return cudaSuccess or the launch error.  They assume validated arguments.

@@ -223,6 +223,23 @@ la_status_t la_short_conv(la_dtype_t dtype, int B, int T, int H, int d, int widt
                           void *window_out, void *y, unsigned flags, void *stream);
 
 /*
+ * la_short_conv_varlen -- la_short_conv over N packed sequences of different lengths,
+ * each with its own carried window (sequence s = tokens [cu_seqlens[s],
+ * cu_seqlens[s+1]) of the packed axis; nothing crosses from one sequence into the next).
+ *   cu_seqlens  [N + 1] int32, DEVICE memory, as for la_prefill_varlen (entries outside
+ *               [0, T] or decreasing are clamped and reported by la_check_status())
+ *   x           [T, H*d]             I/O dtype, the packed projection output
+ *   window_in   [N, width-1, H*d]    or NULL (zeros); window_out likewise (may be
+ *                                    window_in itself)
+ *   y           [H, T, d]            I/O dtype: the q / k / v input of la_prefill_varlen
+ * Two launches: the convolution, then the carried windows (and the offsets check).
+ */
+la_status_t la_short_conv_varlen(la_dtype_t dtype, int N, int T, int H, int d, int width,
+                                 const int *cu_seqlens, const void *x, const float *w,
+                                 const void *window_in, void *window_out, void *y,
+                                 unsigned flags, void *stream);
+
+/*
  * la_short_conv_step -- la_short_conv for one new token of N sequences (decoding):
  *   x [N, H*d], window [N, width-1, H*d] updated in place (required when width > 1),
  *   y [N, H, d] (the q / k / v input of la_decode_step); w and flags as above.
@@ -241,6 +258,15 @@ la_status_t la_short_conv_step(la_dtype_t dtype, int N, int H, int d, int width,
  */
 la_status_t la_check_status(void *stream);
 
+/*
+ * la_selftest_wait_timeout -- a diagnostic of the failure path: enqueues one small
+ * kernel that waits, with the bounded wait every pipeline kernel uses, on a barrier
+ * nothing completes.  The wait gives up after its poll limit (well under a second),
+ * records the timeout and returns; the next la_check_status() reports LA_ERR_TIMEOUT
+ * and the device stays usable.  Touches no caller memory.
+ */
+la_status_t la_selftest_wait_timeout(void *stream);
+
 /* A static, human-readable description of a status code. */
 const char *la_status_string(la_status_t status);
 
@@ -253,7 +279,7 @@ unsigned long long la_kernel_launches(void);
 
 /* Per-launch device timing, a measurement aid with no counterpart in the pages.
  * la_launch_timing(1) makes every later call of la_prefill, la_prefill_noalloc,
- * la_prefill_varlen, la_decode_step, la_short_conv and la_short_conv_step bracket each
+ * la_prefill_varlen, la_decode_step and the la_short_conv* entry points bracket each
  * kernel it enqueues
  * with two CUDA events recorded on the call's stream (at most 16 launches per call are
  * timed); la_launch_timing(0) turns it off (the default).  Enabling adds two event

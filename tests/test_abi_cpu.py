@@ -157,3 +157,22 @@ def test_prefill_varlen_argument_checks(lib):
     assert call(dk=96) == UNSUPPORTED
     assert call() == INVALID          # NULL cu_seqlens / tensors, before any launch
     assert call(T=0) == INVALID       # still needs the offsets and the state
+
+
+def test_short_conv_varlen_argument_checks(lib):
+    INVALID, UNSUPPORTED = 1, 2
+
+    def call(dtype=1, N=2, T=10, H=2, d=128, width=4, flags=0):
+        return lib.la_short_conv_varlen(dtype, N, T, H, d, width, *([None] * 6), flags, None)
+
+    assert call(dtype=5) == INVALID
+    assert call(N=0) == INVALID
+    assert call(T=-1) == INVALID
+    assert call(width=5) == INVALID
+    assert call(flags=1) == INVALID
+    assert call(d=32) == UNSUPPORTED
+    assert call() == INVALID          # NULL offsets / taps, before any launch
+
+
+def test_selftest_symbol_is_exported(lib):
+    assert hasattr(lib, "la_selftest_wait_timeout")

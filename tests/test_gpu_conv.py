@@ -143,3 +143,35 @@ def test_conv_full_size_sampled(la):
                                   None if win is None else f64(win), H=cw.H, silu=True, l2norm=True)
         close(y[b:b + 1, :, t0:t0 + n], ref, cw.dtype, True)
     np.testing.assert_array_equal(f64(wout), f64(x[:, -3:]))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("lengths", [[65, 0, 1, 64, 130, 63, 200, 2], [5], [0, 0, 3], [300, 1, 1, 70]])
+@pytest.mark.parametrize("with_window", [False, True])
+def test_conv_varlen_matches_oracle(la, dtype, lengths, with_window):
+    H, d, width = 2, 128 if dtype == torch.bfloat16 else 64, 4
+    C = H * d
+    T = sum(lengths)
+    x, w, _ = W.conv_inputs(1, T, C, width, dtype, seed=T + len(lengths), device="cuda", window=False)
+    x = x[0]
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32, device="cuda")
+    win = None
+    if with_window:
+        win = torch.randn(len(lengths), width - 1, C, device="cuda").to(dtype)
+    keep = None if win is None else win.clone()
+    y, wout = la.short_conv_varlen(x, w, cu, heads=H, window=win, window_out=win, silu=True,
+                                   l2norm=True)
+    la.check_status()
+    ry, rw = oconv.short_conv_packed(f64(x), f64(w), cu.tolist(), None if keep is None else f64(keep),
+                                     H=H, silu=True, l2norm=True)
+    if T:
+        close(y, ry, dtype, True)
+    np.testing.assert_array_equal(f64(wout), rw)
+
+
+def test_conv_varlen_bad_offsets_are_reported(la):
+    x, w, _ = W.conv_inputs(1, 100, 256, 4, torch.bfloat16, seed=1, device="cuda", window=False)
+    bad = torch.tensor([0, 60, 40, 500], dtype=torch.int32, device="cuda")
+    la.short_conv_varlen(x[0], w, bad, heads=2)
+    with pytest.raises(la.LaError, match="INVALID_ARG"):
+        la.check_status()
