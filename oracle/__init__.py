@@ -37,6 +37,8 @@ MODE_ELU1_NORM = 0
 MODE_GATED = 1
 MODE_GATED_DELTA = 2
 MODE_KDA = 3
+MODE_RETNET = 4   # mode 1 with one constant gate per head: gate [H]
+
 
 
 def build(force: bool = False) -> str:
@@ -106,6 +108,9 @@ def prefill(mode, q, k, v, gate=None, beta=None, state=None, z=None, nthreads=0)
     """
     q = _f64(q)
     B, H, T, dk = q.shape
+    if mode == MODE_RETNET:
+        g = np.asarray(gate, dtype=np.float64).reshape(1, H, 1)
+        mode, gate = 1, np.broadcast_to(g, (B, H, T)).copy()
     k = _f64(k, (B, H, T, dk))
     v = _f64(v)
     dv = v.shape[-1]
@@ -134,6 +139,9 @@ def decode_step(mode, q, k, v, gate, beta, state, z=None, nthreads=0):
     """
     q = _f64(q)
     N, H, dk = q.shape
+    if mode == MODE_RETNET:
+        g = np.asarray(gate, dtype=np.float64).reshape(1, H)
+        mode, gate = 1, np.broadcast_to(g, (N, H)).copy()
     k = _f64(k, (N, H, dk))
     v = _f64(v)
     dv = v.shape[-1]
@@ -163,6 +171,9 @@ def prefill_packed(mode, q, k, v, cu, gate=None, beta=None, state=None, z=None, 
     q, k, v = _f64(q), _f64(k), _f64(v)
     H, T, dk = q.shape
     dv = v.shape[-1]
+    if mode == MODE_RETNET:
+        g = np.asarray(gate, dtype=np.float64).reshape(H, 1)
+        mode, gate = 1, np.broadcast_to(g, (H, T)).copy()
     cu = [int(x) for x in np.asarray(cu).reshape(-1)]
     N = len(cu) - 1
     o = np.zeros((H, T, dv))

@@ -517,3 +517,28 @@ def test_packed_empty_sequence_keeps_its_start_state():
     np.testing.assert_array_equal(pS[1], S0[1])
     _, pS0, _ = oracle.prefill_packed(1, q, k, v, cu)
     np.testing.assert_array_equal(pS0[1], 0.0)
+
+
+# ---- constant decay per head (RetNet / Lightning): mode 4
+def test_retnet_mode_matches_the_decay_mask_closed_form():
+    """[decay/gates]: with a constant gamma the decay mask is D_ij = gamma^(i-j); per head
+    o_t = sum_{j<=t} gamma_h^(t-j) (q_t . k_j) v_j and S_T = sum_j gamma_h^(T-1-j) v_j k_j^T."""
+    r = np.random.default_rng(95)
+    B, H, T, dk, dv = 2, 3, 13, 4, 5
+    q, k, v = r.normal(size=(B, H, T, dk)), r.normal(size=(B, H, T, dk)), r.normal(size=(B, H, T, dv))
+    gam = np.array([0.9, 0.5, 0.99])
+    o, S, _ = oracle.prefill(oracle.MODE_RETNET, q, k, v, gam)
+    t = np.arange(T)
+    for h in range(H):
+        D = np.where(t[:, None] >= t[None, :], gam[h] ** (t[:, None] - t[None, :]).clip(min=0), 0.0)
+        for b in range(B):
+            ref_o = (D * (q[b, h] @ k[b, h].T)) @ v[b, h]
+            ref_S = (v[b, h].T * gam[h] ** (T - 1 - t)) @ k[b, h]
+            np.testing.assert_allclose(o[b, h], ref_o, rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(S[b, h], ref_S, rtol=1e-12, atol=1e-12)
+    # the decode step with the same constant gates continues the sequence
+    od, Sd, _ = oracle.decode_step(oracle.MODE_RETNET, q[:, :, -1], k[:, :, -1], v[:, :, -1], gam, None,
+                                   oracle.prefill(oracle.MODE_RETNET, q[:, :, :-1], k[:, :, :-1],
+                                                  v[:, :, :-1], gam)[1])
+    np.testing.assert_allclose(od, o[:, :, -1], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(Sd, S, rtol=1e-12, atol=1e-12)
