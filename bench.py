@@ -106,7 +106,7 @@ def prefill_algorithmic(w: W.Workload, C=64):
     th = w.B * w.H * w.T
     e = io_bytes(w.dtype)
     b = th * e * (2 * w.dk + 2 * w.dv)
-    if w.gate != "none":
+    if w.gate == "softplus":   # per-token gates ("retnet": one constant per head, no stream)
         b += th * 4 * (w.dk if w.mode == 3 else 1)
     if w.beta:
         b += th * 4
@@ -685,7 +685,7 @@ def main():
     if do_extras:
         for name in ("elu1_bf16_b4h16t4096", "gated_bf16_b8h16t8192", "gdn_bf16_b2h16t32768",
                      "gdn_decode_n256h32", "kda_bf16_b2h16t32768", "kda_decode_n256h32",
-                     "conv_bf16_b2h16t32768", "gdn_varlen_bf16_n64h16"):
+                     "conv_bf16_b2h16t32768", "gdn_varlen_bf16_n64h16", "retnet_bf16_b8h16t8192"):
             if name == args.workload:
                 continue
             r = measure(la, name, args, dist, device, rank, world, flush, False)

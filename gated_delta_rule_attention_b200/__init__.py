@@ -14,6 +14,8 @@ Four modes, named after the variants on the lesson page "Linear attention and hy
 * ``MODE_GATED_DELTA`` -- the Gated DeltaNet update (section "The delta rule and Gated DeltaNet")
 * ``MODE_KDA`` -- Kimi Delta Attention, the same update with one decay per channel (gate
   [.., d_k] per token; same section)
+* ``MODE_RETNET`` -- the constant decay of RetNet / Lightning attention: ``MODE_GATED`` with
+  one fixed gate per head (gate [H]; section "Memory must forget: decay and gates")
 """
 from __future__ import annotations
 
@@ -22,7 +24,7 @@ import os
 
 import torch
 
-__all__ = ["MODE_ELU1_NORM", "MODE_GATED", "MODE_GATED_DELTA", "MODE_KDA", "FLAG_INIT_STATE", "LaError",
+__all__ = ["MODE_ELU1_NORM", "MODE_GATED", "MODE_GATED_DELTA", "MODE_KDA", "MODE_RETNET", "FLAG_INIT_STATE", "LaError",
            "prefill", "prefill_varlen", "decode_step", "short_conv", "short_conv_varlen", "short_conv_step", "check_status", "library",
            "library_path", "version", "kernel_launches", "workspace_size"]
 
@@ -30,6 +32,7 @@ MODE_ELU1_NORM = 0
 MODE_GATED = 1
 MODE_GATED_DELTA = 2
 MODE_KDA = 3
+MODE_RETNET = 4
 FLAG_INIT_STATE = 1
 CONV_SILU = 2
 CONV_L2NORM = 4
@@ -160,6 +163,13 @@ def _need(t, shape, dtype, name):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _gate_shape(mode, lead, dk, H):
+    """Shape of the gate tensor: per token, per channel in KDA, one per head in RetNet."""
+    if mode == MODE_RETNET:
+        return (H,)
+    return (*lead, dk) if mode == MODE_KDA else tuple(lead)
+
+
 _workspaces: dict = {}
 
 
@@ -216,7 +226,7 @@ def prefill(q, k, v, *, mode: int, gate=None, beta=None, state=None, z=None, o=N
     _need(k, (B, H, T, dk), dt, "k")
     _need(v, (B, H, T, dv), dt, "v")
     if gate is not None:
-        _need(gate, (B, H, T, dk) if mode == MODE_KDA else (B, H, T), torch.float32, "gate")
+        _need(gate, _gate_shape(mode, (B, H, T), dk, H), torch.float32, "gate")
     if beta is not None:
         _need(beta, (B, H, T), torch.float32, "beta")
     if init_state is None:
@@ -269,7 +279,7 @@ def prefill_varlen(q, k, v, cu_seqlens, *, mode: int, gate=None, beta=None, stat
     _need(k, (H, T, dk), dt, "k")
     _need(v, (H, T, dv), dt, "v")
     if gate is not None:
-        _need(gate, (H, T, dk) if mode == MODE_KDA else (H, T), torch.float32, "gate")
+        _need(gate, _gate_shape(mode, (H, T), dk, H), torch.float32, "gate")
     if beta is not None:
         _need(beta, (H, T), torch.float32, "beta")
     if init_state is None:
@@ -327,7 +337,7 @@ def decode_step(q, k, v, *, mode: int, state, gate=None, beta=None, z=None, o=No
     _need(v, (N, H, dv), dt, "v")
     _need(state, (N, H, dv, dk), torch.float32, "state")
     if gate is not None:
-        _need(gate, (N, H, dk) if mode == MODE_KDA else (N, H), torch.float32, "gate")
+        _need(gate, _gate_shape(mode, (N, H), dk, H), torch.float32, "gate")
     if beta is not None:
         _need(beta, (N, H), torch.float32, "beta")
     if mode == MODE_ELU1_NORM:

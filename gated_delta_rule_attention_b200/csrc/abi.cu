@@ -57,6 +57,11 @@ bool tensor_ok(const void *p, uintptr_t align) { return p && aligned(p, align) &
 
 la_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
 
+// Modes that take beta (the delta rule).
+bool delta_mode(int mode) { return mode == LA_MODE_GATED_DELTA || mode == LA_MODE_KDA; }
+// The RetNet mode is the scalar-gate mode with one constant gate per head.
+int internal_mode(int mode) { return mode == LA_MODE_RETNET ? (int)LA_MODE_GATED : mode; }
+
 bool dims_ok(int dk, int dv) { return (dk == 64 || dk == 128) && (dv == 64 || dv == 128); }
 
 // True if the byte ranges [p, p + n) and [q, q + m) share a byte.
@@ -76,7 +81,8 @@ extern "C" la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H
                                   void *o, int chunk, unsigned flags, void *workspace,
                                   size_t workspace_bytes, void *stream) {
     timer_reset();
-    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_KDA) return LA_ERR_INVALID_ARG;
+    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_RETNET) return LA_ERR_INVALID_ARG;
+    if (mode == LA_MODE_RETNET && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || T < 0) return LA_ERR_INVALID_ARG;
     if (flags & ~LA_FLAG_INIT_STATE) return LA_ERR_INVALID_ARG;
@@ -99,22 +105,23 @@ extern "C" la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H
     if (!tensor_ok(q, 16) || !tensor_ok(k, 16) || !tensor_ok(v, 16) || !tensor_ok(o, 16))
         return LA_ERR_INVALID_ARG;
     if (mode != LA_MODE_ELU1_NORM && gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
-    if (mode >= LA_MODE_GATED_DELTA && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
+    if (delta_mode(mode) && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
 
     PrefillArgs a;
-    a.mode = mode;
+    a.mode = internal_mode(mode);
+    a.gate_heads = (mode == LA_MODE_RETNET) ? H : 0;
     a.dtype = dtype;
     a.B = B; a.H = H; a.T = T; a.dk = d_k; a.dv = d_v;
     a.q = q; a.k = k; a.v = v;
     a.gate = (mode == LA_MODE_ELU1_NORM) ? nullptr : gate;
-    a.beta = (mode >= LA_MODE_GATED_DELTA) ? beta : nullptr;
+    a.beta = delta_mode(mode) ? beta : nullptr;
     a.state = state;
     a.z = (mode == LA_MODE_ELU1_NORM) ? z : nullptr;
     a.o = o;
     a.init_state = init;
     a.stream = st;
     if (workspace && workspace_bytes && !tensor_ok(workspace, 16)) return LA_ERR_INVALID_ARG;
-    if (prefill_tc_supports(mode, dtype, d_k, d_v, chunk)) {
+    if (prefill_tc_supports(internal_mode(mode), dtype, d_k, d_v, chunk)) {
         a.chunk = 64;
         return from_cuda(launch_prefill_tc(a, workspace, workspace ? workspace_bytes : 0));
     }
@@ -130,7 +137,8 @@ extern "C" la_status_t la_prefill_varlen(la_mode_t mode, la_dtype_t dtype, int N
                                          const float *beta, float *state, float *z, void *o,
                                          int chunk, unsigned flags, void *stream) {
     timer_reset();
-    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_KDA) return LA_ERR_INVALID_ARG;
+    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_RETNET) return LA_ERR_INVALID_ARG;
+    if (mode == LA_MODE_RETNET && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     if (N < 1 || H < 1 || T < 0) return LA_ERR_INVALID_ARG;
     if (flags & ~LA_FLAG_INIT_STATE) return LA_ERR_INVALID_ARG;
@@ -145,15 +153,16 @@ extern "C" la_status_t la_prefill_varlen(la_mode_t mode, la_dtype_t dtype, int N
         if (!tensor_ok(q, 16) || !tensor_ok(k, 16) || !tensor_ok(v, 16) || !tensor_ok(o, 16))
             return LA_ERR_INVALID_ARG;
         if (mode != LA_MODE_ELU1_NORM && gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
-        if (mode >= LA_MODE_GATED_DELTA && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
+        if (delta_mode(mode) && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
     }
     PrefillArgs a;
-    a.mode = mode;
+    a.mode = internal_mode(mode);
+    a.gate_heads = (mode == LA_MODE_RETNET) ? H : 0;
     a.dtype = dtype;
     a.B = 1; a.H = H; a.T = T; a.dk = d_k; a.dv = d_v;
     a.q = q; a.k = k; a.v = v;
     a.gate = (mode == LA_MODE_ELU1_NORM) ? nullptr : gate;
-    a.beta = (mode >= LA_MODE_GATED_DELTA) ? beta : nullptr;
+    a.beta = delta_mode(mode) ? beta : nullptr;
     a.state = state;
     a.z = (mode == LA_MODE_ELU1_NORM) ? z : nullptr;
     a.o = o;
@@ -165,7 +174,7 @@ extern "C" la_status_t la_prefill_varlen(la_mode_t mode, la_dtype_t dtype, int N
         if (init) return LA_OK;
         return from_cuda(launch_zero_empty_sequences(a));
     }
-    if (prefill_tc_supports(mode, dtype, d_k, d_v, chunk)) {
+    if (prefill_tc_supports(internal_mode(mode), dtype, d_k, d_v, chunk)) {
         a.chunk = 64;
         cudaError_t e = launch_prefill_tc(a, nullptr, 0);
         if (e == cudaSuccess && !init) e = launch_zero_empty_sequences(a);
@@ -179,10 +188,10 @@ extern "C" la_status_t la_prefill_varlen(la_mode_t mode, la_dtype_t dtype, int N
 
 extern "C" size_t la_prefill_workspace_size(la_mode_t mode, la_dtype_t dtype, int B, int H, int T,
                                             int d_k, int d_v, int chunk) {
-    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_KDA || B < 1 || H < 1 || T < 1)
+    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_RETNET || B < 1 || H < 1 || T < 1)
         return 0;
-    if (!prefill_tc_supports(mode, dtype, d_k, d_v, chunk)) return 0;
-    return prefill_tc_workspace_bytes(mode, B, H, T);
+    if (!prefill_tc_supports(internal_mode(mode), dtype, d_k, d_v, chunk)) return 0;
+    return prefill_tc_workspace_bytes(internal_mode(mode), B, H, T);
 }
 
 extern "C" la_status_t la_decode_step(la_mode_t mode, la_dtype_t dtype, int N, int H, int d_k,
@@ -190,7 +199,8 @@ extern "C" la_status_t la_decode_step(la_mode_t mode, la_dtype_t dtype, int N, i
                                       const float *gate, const float *beta, float *state,
                                       float *z, void *o, void *stream) {
     timer_reset();
-    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_KDA) return LA_ERR_INVALID_ARG;
+    if (mode < LA_MODE_ELU1_NORM || mode > LA_MODE_RETNET) return LA_ERR_INVALID_ARG;
+    if (mode == LA_MODE_RETNET && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     if (N < 1 || H < 1) return LA_ERR_INVALID_ARG;
     if (!dims_ok(d_k, d_v)) return LA_ERR_UNSUPPORTED;
@@ -202,14 +212,15 @@ extern "C" la_status_t la_decode_step(la_mode_t mode, la_dtype_t dtype, int N, i
         return LA_ERR_INVALID_ARG;
     if (mode == LA_MODE_ELU1_NORM && !tensor_ok(z, 16)) return LA_ERR_INVALID_ARG;
     if (mode != LA_MODE_ELU1_NORM && gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
-    if (mode >= LA_MODE_GATED_DELTA && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
+    if (delta_mode(mode) && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
     DecodeArgs a;
-    a.mode = mode;
+    a.mode = internal_mode(mode);
+    a.gate_heads = (mode == LA_MODE_RETNET) ? H : 0;
     a.dtype = dtype;
     a.N = N; a.H = H; a.dk = d_k; a.dv = d_v;
     a.q = q; a.k = k; a.v = v;
     a.gate = (mode == LA_MODE_ELU1_NORM) ? nullptr : gate;
-    a.beta = (mode >= LA_MODE_GATED_DELTA) ? beta : nullptr;
+    a.beta = delta_mode(mode) ? beta : nullptr;
     a.state = state;
     a.z = (mode == LA_MODE_ELU1_NORM) ? z : nullptr;
     a.o = o;

@@ -61,7 +61,8 @@ template <int MODE, int DK, int DV, typename IO>
 __global__ void __launch_bounds__(kDecodeThreads)
 decode_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
               const float *__restrict__ gate, const float *__restrict__ beta,
-              float *__restrict__ state, float *__restrict__ z, IO *__restrict__ o) {
+              float *__restrict__ state, float *__restrict__ z, IO *__restrict__ o,
+              int gate_heads) {
     constexpr int VEC = DK / 32;
     constexpr int RPW = DV / kDecodeWarps;       // rows per warp: 16 or 8
     constexpr int ROWS = RPW < 4 ? RPW : 4;      // rows in flight per warp
@@ -83,7 +84,8 @@ decode_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__re
         }
     }
     constexpr bool kDelta = (MODE == 2 || MODE == 3);
-    const float a = (MODE == 0 || MODE == 3 || gate == nullptr) ? 1.f : gate[nh];
+    const float a = (MODE == 0 || MODE == 3 || gate == nullptr) ? 1.f
+                                                                 : gate[gate_heads ? nh % gate_heads : nh];
     const float b = kDelta ? beta[nh] : 0.f;
     float av[VEC];   // mode 3: this lane's channel decays
 #pragma unroll
@@ -168,7 +170,7 @@ cudaError_t launch_mode(const DecodeArgs &a) {
     if (a.dk == DKc && a.dv == DVc) {                                                       \
         timer_begin(a.stream);                                                              \
         decode_kernel<MODE, DKc, DVc, IO><<<grid, kDecodeThreads, 0, a.stream>>>(            \
-            q, k, v, a.gate, a.beta, a.state, a.z, o);                                      \
+            q, k, v, a.gate, a.beta, a.state, a.z, o, a.gate_heads);                        \
         timer_end(a.stream);                                                                \
         note_launches(1);                                                                   \
         return cudaGetLastError();                                                          \

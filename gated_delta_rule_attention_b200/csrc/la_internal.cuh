@@ -42,6 +42,9 @@ struct PrefillArgs {
     // sequence s takes tokens [cu[s], cu[s+1]) and owns state slot s of [nseq, H, ..].
     const int *cu = nullptr;
     int nseq = 0;
+    // Constant gates (the RetNet decay): gate holds one value per head, [H], used for
+    // every token (0: per-token gates).
+    int gate_heads = 0;
 };
 
 struct DecodeArgs {
@@ -52,6 +55,7 @@ struct DecodeArgs {
     float *state, *z;
     void *o;
     cudaStream_t stream;
+    int gate_heads = 0;   // as in PrefillArgs
 };
 
 struct ConvArgs {

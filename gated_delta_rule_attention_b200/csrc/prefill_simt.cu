@@ -59,7 +59,7 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
                     const IO *__restrict__ k, const IO *__restrict__ v,
                     const float *__restrict__ gate, const float *__restrict__ beta,
                     float *__restrict__ state, float *__restrict__ zg, IO *__restrict__ o,
-                    int init_state, unsigned *err) {
+                    int init_state, unsigned *err, int gate_heads) {
     using L = SimtSmem<MODE, DK, DV, C>;
     constexpr bool kDelta = (MODE == 2 || MODE == 3);
     extern __shared__ float smem[];
@@ -97,7 +97,10 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
     const IO *kh = k + row0 * DK;
     const IO *vh = v + row0 * DV;
     IO *oh = o + row0 * DV;
-    const float *gh = gate ? gate + row0 * (MODE == 3 ? DK : 1) : nullptr;
+    // per-token gates from row0 on, or (gate_heads > 0) one constant gate for the head
+    const float *gh = gate ? (gate_heads ? gate + blockIdx.x % gate_heads : gate + row0 * (MODE == 3 ? DK : 1))
+                           : nullptr;
+    const int gt = gate_heads ? 0 : 1;   // token stride of gh (modes 1, 2)
     const float *bh_beta = beta ? beta + row0 : nullptr;
     float *Sg = state + bh * (size_t)DV * DK;
 
@@ -121,7 +124,7 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
         for (int p = tid; p < Lc * DV; p += kSimtThreads)
             Vs[(p / DV) * SV + p % DV] = to_f32(vh[(size_t)(t0 + p / DV) * DV + p % DV]);
         if (tid < Lc) {
-            lam[tid] = (MODE != 0 && MODE != 3 && gh) ? logf(fmaxf(gh[t0 + tid], FLT_MIN)) : 0.f;
+            lam[tid] = (MODE != 0 && MODE != 3 && gh) ? logf(fmaxf(gh[(t0 + tid) * gt], FLT_MIN)) : 0.f;
             bet[tid] = kDelta ? bh_beta[t0 + tid] : 0.f;
         }
         if (MODE == 3) {   // per-channel in-chunk prefix of log a, one channel per thread
@@ -262,7 +265,7 @@ cudaError_t launch_one(const PrefillArgs &a) {
     kern<<<grid, kSimtThreads, L::kBytes, a.stream>>>(
         a.T, a.H, a.cu, static_cast<const IO *>(a.q), static_cast<const IO *>(a.k),
         static_cast<const IO *>(a.v), a.gate, a.beta, a.state, a.z, static_cast<IO *>(a.o),
-        a.init_state ? 1 : 0, device_error_word());
+        a.init_state ? 1 : 0, device_error_word(), a.gate_heads);
     timer_end(a.stream);
     note_launches(1);
     return cudaGetLastError();

@@ -90,6 +90,9 @@ struct TcParams {
     // read from a start state that a combine kernel wrote.
     const float *fold_init, *fold_zinit, *fold_loc, *fold_zloc, *fold_gam;
     int fold_sub;
+    // Constant per-head gates: gate is [gate_heads], head row bh uses gate[bh % gate_heads]
+    // for every token (0: per-token gates [BH][T]).
+    int gate_heads;
     // Packed variable-length sequences (nullptr: dense).  CTA (s, h) takes tokens
     // [cu[s], cu[s+1]) of head row h of the packed [H][T][128] tensors; its state is
     // slot s of the s_in / s_out segment stride.
@@ -278,7 +281,8 @@ __device__ __forceinline__ GateRaw fetch_gates(const TcParams &p, int bh, int tb
     GateRaw r{1.f, 0.f};
     const int t0 = tb + kC * c;
     const int L = min(kC, te - t0);
-    if (MODE != 0 && p.gate && e < L) r.a = p.gate[(size_t)bh * p.T + t0 + e];
+    if (MODE != 0 && p.gate && e < L)
+        r.a = p.gate[p.gate_heads ? (size_t)(bh % p.gate_heads) : (size_t)bh * p.T + t0 + e];
     if (MODE == 2 && e < L) r.b = p.beta[(size_t)bh * p.T + t0 + e];
     return r;
 }
@@ -851,7 +855,8 @@ static_assert(Lay01::kBytes <= 227 * 1024, "shared memory per CTA");
 
 __device__ __forceinline__ float ld_gate(const TcParams &p, int bh, int t0, int L, int i) {
     float a = 1.f;
-    if (i < L) asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(a) : "l"(p.gate + (size_t)bh * p.T + t0 + i));
+    const size_t off = p.gate_heads ? (size_t)(bh % p.gate_heads) : (size_t)bh * p.T + t0 + i;
+    if (i < L) asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(a) : "l"(p.gate + off));
     return a;
 }
 
@@ -2022,6 +2027,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t work
                       head_pitch, 64, kC, true))
         return cudaErrorInvalidValue;
     p.gate = a.gate;
+    p.gate_heads = a.gate_heads;
     p.beta = a.beta;
     p.o = static_cast<__nv_bfloat16 *>(a.o);
     p.T = a.T;

@@ -21,6 +21,9 @@
  *   LA_MODE_KDA ([delta rule], Kimi Delta Attention: the scalar a_t replaced by the
  *   diagonal matrix Diag(a_t), one decay per memory channel, the d_k columns of S):
  *       S_t = S_{t-1} Diag(a_t) (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S_t q_t.
+ *   LA_MODE_RETNET ([decay/gates], the constant decay gamma of RetNet / Lightning
+ *   attention): S_t = g_h S_{t-1} + v_t k_t^T, o_t = S_t q_t, with one fixed gate g_h per
+ *   head; `gate` is then [H] (required) and no per-token gate tensor is read.
  *
  * No 1/sqrt(d) scale is applied inside the attention; callers scale q and k.
  *
@@ -35,9 +38,9 @@
  *   are always fp32; all accumulation is fp32.
  * Sizes: d_k and d_v are each 64 or 128.  B, H, N >= 1.  T >= 0.
  * Gates: gate holds the decay values a_t in [0, 1] (not their logarithms); NULL means
- *   a_t = 1.  In mode 3 it holds d_k values per token (one per channel).  beta holds
- *   b_t in [0, 1].  Mode 0 ignores gate and beta; mode 1 ignores beta; modes 2 and 3
- *   require beta.
+ *   a_t = 1.  In mode 3 it holds d_k values per token (one per channel); in mode 4 one
+ *   value per head, [H].  beta holds b_t in [0, 1].  Mode 0 ignores gate and beta;
+ *   modes 1 and 4 ignore beta; modes 2 and 3 require beta; mode 4 requires gate.
  * State layout: S is d_v x d_k per head, exactly the page's S ([three forms]), stored
  *   [.., d_v, d_k] row-major; z is [.., d_k].  A state written by la_prefill is the
  *   input of la_decode_step, and vice versa.
@@ -61,7 +64,8 @@ typedef enum {
     LA_MODE_ELU1_NORM = 0,   /* phi = elu+1, z-normalised                 */
     LA_MODE_GATED = 1,       /* scalar gate a_t, identity feature map     */
     LA_MODE_GATED_DELTA = 2, /* Gated DeltaNet: gate a_t and delta rate b_t */
-    LA_MODE_KDA = 3          /* Kimi Delta Attention: per-channel gate a_t [d_k], rate b_t */
+    LA_MODE_KDA = 3,         /* Kimi Delta Attention: per-channel gate a_t [d_k], rate b_t */
+    LA_MODE_RETNET = 4       /* constant decay: mode 1 with one fixed gate per head, [H] */
 } la_mode_t;
 
 typedef enum {

@@ -72,7 +72,7 @@ def _prefill(lib, mode=2, dtype=1, B=1, H=1, T=8, dk=128, dv=128, chunk=0, flags
 
 def test_host_side_argument_checks(lib):
     INVALID, UNSUPPORTED = 1, 2
-    assert _prefill(lib, mode=4) == INVALID
+    assert _prefill(lib, mode=5) == INVALID
     assert _prefill(lib, mode=-1) == INVALID
     assert _prefill(lib, dtype=2) == INVALID
     assert _prefill(lib, B=0) == INVALID
@@ -147,7 +147,7 @@ def test_prefill_varlen_argument_checks(lib):
     def call(mode=2, dtype=1, N=2, H=2, T=100, dk=128, dv=128, chunk=0, flags=0):
         return lib.la_prefill_varlen(mode, dtype, N, H, T, dk, dv, *([None] * 9), chunk, flags, None)
 
-    assert call(mode=4) == INVALID
+    assert call(mode=5) == INVALID
     assert call(dtype=3) == INVALID
     assert call(N=0) == INVALID
     assert call(H=0) == INVALID
@@ -176,3 +176,11 @@ def test_short_conv_varlen_argument_checks(lib):
 
 def test_selftest_symbol_is_exported(lib):
     assert hasattr(lib, "la_selftest_wait_timeout")
+
+
+def test_retnet_mode_needs_its_gate(lib):
+    INVALID = 1
+    # mode 4 without a gate is refused before anything else is looked at
+    assert lib.la_decode_step(4, 1, 1, 1, 128, 128, *([None] * 9)) == INVALID
+    assert lib.la_prefill_workspace_size(4, 1, 1, 16, 32768, 128, 128, 0) > 0   # the mode-1 plan
+    assert lib.la_prefill_workspace_size(5, 1, 1, 16, 32768, 128, 128, 0) == 0

@@ -20,6 +20,7 @@ MODE_ELU1_NORM = 0
 MODE_GATED = 1
 MODE_GATED_DELTA = 2
 MODE_KDA = 3
+MODE_RETNET = 4
 
 
 @dataclasses.dataclass(frozen=True)
@@ -37,7 +38,8 @@ class Workload:
     qk_scale: float = 1.0       # q, k ~ N(0,1) * qk_scale
     v_scale: float = 1.0
     qk_l2norm: bool = False     # L2-normalise q, k rows in fp32 before the cast
-    gate: str = "none"          # "none" | "softplus" (a = exp(-softplus(x + gate_shift)))
+    gate: str = "none"          # "none" | "softplus" (a = exp(-softplus(x + gate_shift))) |
+                                # "retnet" (mode 4: one constant gate per head, no draw)
     gate_shift: float = 0.0
     beta: bool = False          # beta = sigmoid(y), y ~ N(0,1)
     decode: bool = False
@@ -73,6 +75,10 @@ CONFIGS = {
     "kda_decode_n256h32": Workload("kda_decode_n256h32", MODE_KDA, torch.bfloat16, B=256, H=32,
                                    T=1000, dk=128, dv=128, seed=7, qk_l2norm=True,
                                    gate="softplus", beta=True, decode=True, state_std=0.02),
+    # Constant per-head decay (RetNet / Lightning attention) on the scalar-gated shapes.
+    "retnet_bf16_b8h16t8192": Workload("retnet_bf16_b8h16t8192", MODE_RETNET, torch.bfloat16, B=8,
+                                       H=16, T=8192, dk=128, dv=128, seed=10,
+                                       qk_scale=1 / math.sqrt(128), gate="retnet"),
 }
 
 
@@ -93,7 +99,11 @@ def _qkv(w: Workload, gen: torch.Generator, device, lead):
 
 def _gates(w: Workload, gen: torch.Generator, device, lead):
     gate = beta = None
-    if w.gate == "softplus":
+    if w.gate == "retnet":
+        # RetNet's per-head decays: gamma_h = 1 - 2^(-5 - 8 h / H), from 0.969 towards 1
+        h = torch.arange(w.H, device=device, dtype=torch.float64)
+        gate = (1.0 - torch.pow(2.0, -5.0 - 8.0 * h / w.H)).to(torch.float32)
+    elif w.gate == "softplus":
         shape = (*lead, w.dk) if w.mode == MODE_KDA else lead
         x = torch.randn(*shape, generator=gen, device=device, dtype=torch.float32)
         # a = exp(-softplus(x)) = sigmoid(-x): a value in (0, 1)
@@ -221,6 +231,8 @@ def varlen_inputs(w: Workload, lengths, device="cpu", init_state_std: float = 0.
     wp = dataclasses.replace(w, B=1, T=T)
     d = prefill_inputs(wp, device=device)
     out = {k: (None if d[k] is None else d[k][0].contiguous()) for k in ("q", "k", "v", "gate", "beta")}
+    if w.gate == "retnet":
+        out["gate"] = d["gate"]   # one constant per head, [H]: nothing to unpack
     cu = [0]
     for n in lengths:
         cu.append(cu[-1] + int(n))
