@@ -60,6 +60,12 @@ constexpr int kEpi = 256;      // epilogue threads (warps 2-9)
 constexpr uint32_t kTmemCols = 512;
 // TMEM column map
 constexpr uint32_t kColDS = 0, kColG = 128, kColU = 192, kColW = 256, kColY = 320, kColO = 384;
+// Kimi Delta Attention (mode 3): the first-half product G0 (N = 32) borrows the first 32
+// U columns, free until the U^T product of the same chunk.
+constexpr uint32_t kColG0 = kColU;
+// Mode 3 clamps each per-channel log2 gate at -kKdaLog2Clamp (a >= 2^-7.5 = 0.0055), so
+// that no operand factor 2^(lambda_t - lambda_ref) over half a half-chunk exceeds 2^120.
+constexpr float kKdaLog2Clamp = 7.5f;
 
 enum Kind { kOutput = 0, kLocal = 1, kTransition = 2 };
 
@@ -190,10 +196,19 @@ struct Small {
     float scan_tmp[2];
 };
 
+// Mode 3 (KDA): per-channel decay vectors of a chunk (parity buffer) and the exchange
+// between the two token halves of a channel.
+struct SmallKda {
+    float eref[2][2][128];   // 2^lambda at the two reference tokens (15, 47), per channel
+    float edec[2][128];      // 2^(lambda_L - lambda_47): Kb -> K 2^(lambda_L - lambda)
+    float egl[2][128];       // 2^lambda_L: the state's column decay over the chunk
+    float tot0[128], tot1[128], x15b[128];   // half totals and the second half's prefix at 15
+};
+
 // Shared-memory layout (bytes from the 1024-aligned base).
 template <int MODE>
 struct Lay {
-    static constexpr int kStages = MODE == 2 ? 2 : 3;
+    static constexpr int kStages = MODE >= 2 ? 2 : 3;
     static constexpr uint32_t kStage = 49152;          // [K0][Q0][K1][Q1][V0][V1], 8 KB each
     static constexpr uint32_t kSbf = kStages * kStage; // 32 KB bf16 state, [d_v][d_k]
     static constexpr uint32_t kA = kSbf + 32768;       // 8 KB  A [t][j]
@@ -201,10 +216,17 @@ struct Lay {
     static constexpr uint32_t kTpp = kTp + 8192;       // 8 KB  T diag(b g)    (mode 2)
     static constexpr uint32_t kX = kTpp + 8192;        // 48 KB E | E' | W  or  Lm | Tm | Zs
     static constexpr uint32_t kE = kX, kEp = kX + 16384, kW = kX + 32768;
-    static constexpr uint32_t kOst = MODE == 2 ? kX + 49152 : kA + 8192;   // 16 KB O staging
+    static constexpr uint32_t kOst = MODE >= 2 ? kX + 49152 : kA + 8192;   // 16 KB O staging
     static constexpr uint32_t kSmall = kOst + 16384;
-    static constexpr uint32_t kBytes = kSmall + sizeof(Small);
+    // mode 3: T diag(b g) is not needed (the decay sits in the K operand); its slot holds
+    // Kb0 = K 2^(lambda_15 - lambda) (rows 0-31, two 4 KB halves), and the O staging
+    // slot holds Kb = K 2^(lambda_47 - lambda) (then K 2^(lambda_L - lambda)); outputs are
+    // staged in the chunk's V slot instead.
+    static constexpr uint32_t kKb0 = kTpp, kKb = kOst;
+    static constexpr uint32_t kKda = (kSmall + sizeof(Small) + 15) & ~15u;
+    static constexpr uint32_t kBytes = MODE == 3 ? kKda + sizeof(SmallKda) : kSmall + sizeof(Small);
 };
+static_assert(Lay<3>::kBytes <= 227 * 1024, "shared memory per CTA");
 constexpr uint32_t kLmStride = 65;
 
 __device__ __forceinline__ void epi_sync() { named_sync(1, kEpi); }
@@ -270,6 +292,22 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 w, float s) {
     return w;
 }
 
+__device__ __forceinline__ void prefetch_l2(const void *ptr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
+// Multiply the 8 bf16 values of a 16-byte chunk by 8 factors (one per channel).
+__device__ __forceinline__ uint4 scale_bf16x8v(uint4 w, const float4 f0, const float4 f1) {
+    uint32_t *wd = reinterpret_cast<uint32_t *>(&w);
+    const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float2 v = unpack_bf16x2(wd[q]);
+        wd[q] = pack_bf16x2(v.x * f[2 * q], v.y * f[2 * q + 1]);
+    }
+    return w;
+}
+
 // Raw gate a_t and beta_t of token `e` of chunk c (64 threads, e < 64), fetched a chunk
 // ahead of use so that the global-load latency overlaps the previous chunk's epilogue.
 struct GateRaw {
@@ -281,9 +319,9 @@ __device__ __forceinline__ GateRaw fetch_gates(const TcParams &p, int bh, int tb
     GateRaw r{1.f, 0.f};
     const int t0 = tb + kC * c;
     const int L = min(kC, te - t0);
-    if (MODE != 0 && p.gate && e < L)
+    if ((MODE == 1 || MODE == 2) && p.gate && e < L)
         r.a = p.gate[p.gate_heads ? (size_t)(bh % p.gate_heads) : (size_t)bh * p.T + t0 + e];
-    if (MODE == 2 && e < L) r.b = p.beta[(size_t)bh * p.T + t0 + e];
+    if (MODE >= 2 && e < L) r.b = p.beta[(size_t)bh * p.T + t0 + e];
     return r;
 }
 
@@ -293,7 +331,7 @@ __device__ __forceinline__ void load_gates(const TcParams &p, Small *sm, int tb,
                                            int buf, int e, GateRaw raw) {
     const int t0 = tb + kC * c;
     const int L = min(kC, te - t0);
-    float g = (MODE != 0 && e < L) ? lg2(fmaxf(raw.a, FLT_MIN)) : 0.f;
+    float g = ((MODE == 1 || MODE == 2) && e < L) ? lg2(fmaxf(raw.a, FLT_MIN)) : 0.f;
     const int lane = e & 31;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -304,7 +342,7 @@ __device__ __forceinline__ void load_gates(const TcParams &p, Small *sm, int tb,
     named_sync(2, 64);
     if (e >= 32) g += sm->scan_tmp[0];
     sm->lam[buf][e] = g;
-    sm->bet[buf][e] = (MODE == 2 && e < L) ? raw.b : 0.f;
+    sm->bet[buf][e] = (MODE >= 2 && e < L) ? raw.b : 0.f;
     if (e == 0) sm->len[buf] = L;
     named_sync(2, 64);
     (void)p;
@@ -420,7 +458,8 @@ __device__ void invert_unit_lower(const float *Lm, float *Tm, float *Zs, int e) 
 
 template <int MODE, int KIND>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
-    static_assert(MODE == 2, "this kernel serves the gated delta rule");
+    static_assert(MODE == 2 || MODE == 3, "this kernel serves the delta rule (modes 2, 3)");
+    constexpr bool kKda = (MODE == 3);   // per-channel decay: it sits in the K / Q operands
     using Y = Lay<MODE>;
     constexpr int NST = Y::kStages;
     constexpr bool kOut = (KIND == kOutput);
@@ -436,6 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         return;
     }
     Small *sm = reinterpret_cast<Small *>(smem_raw + Y::kSmall);
+    SmallKda *sk = reinterpret_cast<SmallKda *>(smem_raw + (kKda ? Y::kKda : Y::kSmall));   // mode 3
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -510,11 +550,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                            tpp = sb + Y::kTpp, et = sb + Y::kE, ept = sb + Y::kEp,
                            wt = sb + Y::kW;
             const uint32_t id_g = idesc_bf16(128, 64, false, false);
+            const uint32_t id_g0 = idesc_bf16(128, 32, false, false);   // mode 3
+            const uint32_t kb = sb + Y::kKb, kb0 = sb + Y::kKb0;           // mode 3
             const uint32_t id_uw = idesc_bf16(128, 64, true, false);
             const uint32_t id_y = idesc_bf16(128, 64, false, true);
             const uint32_t id_o1 = idesc_bf16(64, 128, false, false);
-            const uint32_t id_o2 = idesc_bf16(64, 128, false, MODE != 2);
-            const uint32_t id_ds = idesc_bf16(128, 128, MODE != 2, true);
+            const uint32_t id_o2 = idesc_bf16(64, 128, false, MODE < 2);
+            const uint32_t id_ds = idesc_bf16(128, 128, MODE < 2, true);
             for (int c = 0; c < nch; ++c) {
                 const int s = c % NST, u = c / NST;
                 const uint32_t par = c & 1;
@@ -522,7 +564,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 if (!mbar_wait(&sm->full[s], u & 1, abort, p.err)) break;
                 if (!mbar_wait(&sm->prep_done, par, abort, p.err)) break;
                 tc_fence_after();
-                {
+                if constexpr (kKda) {
+                    // G1 = [K~; Q~] Kb^T (N=64, rows of the second token half) and
+                    // G0 = [K~; Q~] Kb0^T (N=32, rows of the first half); the operands carry
+                    // the per-channel decays relative to tokens 47 and 15
+                    mma_chain<8, true, true, 16384, 8192>(tm + kColG, dk(st), dk(kb), id_g, false);
+                    mma_chain<8, true, true, 16384, 4096>(tm + kColG0, dk(st), dk(kb0), id_g0, false);
+                    mma_commit(&sm->g_done);
+                } else {
                     // G = [K; Q] K^T   (M=128, N=64, K=128)
                     mma_chain<8, true, true>(tm + kColG, dk(st), dk(st), id_g, false);
                     mma_commit(&sm->g_done);
@@ -532,8 +581,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     tc_fence_after();
                     if (kNeedV)   // U^T = V^T (T diag b)^T
                         mma_chain<4, false, true>(tm + kColU, dmn(st + 32768, 8192), dk(tp), id_uw, false);
-                    // W^T = K^T (T diag(b g))^T
-                    mma_chain<4, false, true>(tm + kColW, dmn(st, 16384), dk(tpp), id_uw, false);
+                    // W^T = K^T (T diag(b g))^T; mode 3: (K o Gamma)^T (T diag b)^T
+                    mma_chain<4, false, true>(tm + kColW, dmn(st, 16384), dk(kKda ? tp : tpp), id_uw, false);
                     mma_commit(&sm->ut_done);
                     if (!mbar_wait(&sm->w_ready, par, abort, p.err)) break;
                     if (!mbar_wait(&sm->s_ready, par, abort, p.err)) break;
@@ -549,8 +598,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     mma_chain<8, true, true>(tm + kColO, dk(st + 8192), dk(sbf), id_o1, false);
                     mma_chain<4, true, true>(tm + kColO, dk(at), dk(et), id_o2, true);
                 }
-                // dS = (E^T diag dec) K   (M=128, N=128)
-                mma_chain<4, true, false>(tm + kColDS, dk(ept), dmn(st, 16384), id_ds, false);
+                // dS = (E^T diag dec) K   (M=128, N=128); mode 3: E^T (K o 2^(lambda_L - lambda))
+                if constexpr (kKda)
+                    mma_chain<4, true, false>(tm + kColDS, dk(et), dmn(kb, 8192), id_ds, false);
+                else
+                    mma_chain<4, true, false>(tm + kColDS, dk(ept), dmn(st, 16384), id_ds, false);
                 mma_commit(&sm->mma2_done);
             }
             // nothing may still write TMEM when it is freed
@@ -587,19 +639,100 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             if (e == 0) mbar_arrive(&sm->s_ready);
         }
 
-        // ---- chunk prologue: gates; releases G's inputs to the MMA
+        // ---- mode 3: thread e owns channel kch for the token half khh of every chunk
+        const int kch = e & 127, khh = e >> 7;
+        float kx[32];            // inclusive prefix of the clamped log2 gates within the half
+        float kx15 = 0.f;        // the prefix at the half's reference token (15 or 47)
+        float kref = 0.f;        // exponent base of Kb: lambda_47 in this thread's prefix units
+        // L2 prefetch of chunk c's gate rows (64 tokens x 512 B: one line per thread)
+        auto kda_prefetch = [&](int c) {
+            const int t0 = tb + kC * c, tok = e >> 2;
+            if (p.gate && tok < min(kC, te - t0))
+                prefetch_l2(p.gate + ((size_t)bh * p.T + t0 + tok) * kD + 32 * (e & 3));
+        };
+        auto kda_load = [&](int c, float (&g)[32]) {
+            const int t0 = tb + kC * c;
+            const int L = min(kC, te - t0);
+            const float *gp = p.gate + ((size_t)bh * p.T + t0 + 32 * khh) * kD + kch;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) g[i] = (p.gate && 32 * khh + i < L) ? gp[(size_t)i * kD] : 1.f;
+        };
+        // prefixes, the exchange between the halves, and the chunk's decay vectors
+        auto kda_prefix = [&](int c, const float (&g)[32]) {
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                acc += fmaxf(lg2(fmaxf(g[i], FLT_MIN)), -kKdaLog2Clamp);
+                kx[i] = acc;
+            }
+            kx15 = kx[15];
+            if (khh == 0) {
+                sk->tot0[kch] = acc;
+            } else {
+                sk->tot1[kch] = acc;
+                sk->x15b[kch] = kx15;
+            }
+            epi_sync();
+            const float tot0 = sk->tot0[kch];
+            kref = (khh == 0) ? tot0 + sk->x15b[kch] : kx15;
+            if (khh == 0) {
+                const int b2 = c & 1;
+                const float lL = tot0 + sk->tot1[kch];
+                sk->eref[b2][0][kch] = ex2(kx15);
+                sk->eref[b2][1][kch] = ex2(kref);
+                sk->edec[b2][kch] = ex2(lL - kref);
+                sk->egl[b2][kch] = ex2(lL);
+            }
+        };
+        // chunk c's operands: K~ = K 2^(lambda - lambda_ref), Q~ likewise (in place; the
+        // reference is token 15 for the first half, 47 for the second), Kb and Kb0.  Runs
+        // once the previous chunk's products are done (Kb is a single buffer); then G may go.
+        auto kda_scale = [&](int c) {
+            const uint32_t st = (c % NST) * Y::kStage;
+            const uint32_t cb = (uint32_t)(kch >> 6), cc = (uint32_t)(kch & 63);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t t = 32 * khh + i;
+                const uint32_t o = sw128_off(t, cc >> 3) + ((cc & 7) << 1);
+                __nv_bfloat16 *kp = reinterpret_cast<__nv_bfloat16 *>(smem_raw + st + cb * 16384 + o);
+                const float kv = __bfloat162float(*kp);
+                const float fa = ex2(kx[i] - kx15);
+                *kp = __float2bfloat16_rn(kv * fa);
+                if (kOut) {
+                    __nv_bfloat16 *qp = kp + 4096;   // the Q tile sits 8 KB after the K tile
+                    *qp = __float2bfloat16_rn(__bfloat162float(*qp) * fa);
+                }
+                *reinterpret_cast<__nv_bfloat16 *>(smem_raw + Y::kKb + cb * 8192 + o) =
+                    __float2bfloat16_rn(kv * ex2(kref - kx[i]));
+                if (khh == 0)
+                    *reinterpret_cast<__nv_bfloat16 *>(smem_raw + Y::kKb0 + cb * 4096 + o) =
+                        __float2bfloat16_rn(kv * ex2(kx15 - kx[i]));
+            }
+            fence_async_smem();
+            epi_sync();
+            if (e == 0) mbar_arrive(&sm->prep_done);
+        };
+        (void)kda_prefetch; (void)kda_load; (void)kda_prefix; (void)kda_scale;
+
+        // ---- chunk prologue: gates; releases G's inputs to the MMA (mode 3: kda_scale does)
         auto prep = [&](int c, GateRaw raw) -> bool {
             const int s = c % NST, u = c / NST;
+            float kg[32];
+            if constexpr (kKda) kda_load(c, kg);
             if (e < 64) load_gates<MODE>(p, sm, tb, te, c, c & 1, e, raw);
             mbar_wait(&sm->full[s], u & 1, abort, p.err);
             epi_sync();
             if (*abort) return false;
+            if constexpr (kKda) kda_prefix(c, kg);
             epi_sync();
-            if (e == 0) mbar_arrive(&sm->prep_done);
+            if (!kKda && e == 0) mbar_arrive(&sm->prep_done);
             return true;
         };
 
         bool ok = prep(0, e < 64 ? fetch_gates<MODE>(p, bh, tb, te, 0, e) : GateRaw{1.f, 0.f});
+        if constexpr (kKda) {
+            if (ok) kda_scale(0);
+        }
         for (int c = 0; c < nch && ok; ++c) {
             const int s = c % NST, buf = c & 1;
             const uint32_t par = c & 1;
@@ -611,13 +744,48 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             // gates of the next chunk: issue the global loads now, use them in its prologue
             GateRaw next_raw{1.f, 0.f};
             if (c + 1 < nch && e < 64) next_raw = fetch_gates<MODE>(p, bh, tb, te, c + 1, e);
+            if (kKda && c + 1 < nch) kda_prefetch(c + 1);
 
             // ---- A-epilogue: masks and decays of G; operand scaling
             mbar_wait(&sm->g_done, par, abort, p.err);
             epi_sync();
             if (*abort) break;
             tc_fence_after();
-            if (q >= 2 && kOut) {
+            if (kKda && kOut && c >= 1 && e == 0) {
+                // chunk c-1's outputs were staged in its V slot: release that stage once
+                // the TMA store has read them
+                tma_store_wait_read<0>();
+                mbar_arrive(&sm->empty[(c - 1) % NST]);
+            }
+            if constexpr (kKda) {
+                // G1 holds the rows of the second token half, G0 (32 columns) those of the
+                // first; entries above the diagonal may be huge or not finite and are dropped
+                const bool second = (q & 1) != 0;
+                float v[32];
+                if (second) {
+                    tmem_ld32(tl + kColG + 32 * h, v);
+                } else if (h == 0) {
+                    tmem_ld32(tl + kColG0, v);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                }
+                if (q >= 2 && kOut) {
+                    const int i = row - 64;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = (32 * h + j <= i) ? v[j] : 0.f;
+                    st_row_bf16x16(sb + Y::kA, i, 4 * h, v);
+                    st_row_bf16x16(sb + Y::kA, i, 4 * h + 2, v + 16);
+                } else if (q < 2) {
+                    const int r = row;
+                    const float br = sm->bet[buf][r];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int jj = 32 * h + j;
+                        Lm[r * kLmStride + jj] = (jj < r) ? br * v[j] : 0.f;
+                    }
+                }
+            } else if (q >= 2 && kOut) {
                 // rows i of Q K^T -> A tile, columns j in [32h, 32h + 32)
                 const int i = row - 64;
                 float v[32];
@@ -642,7 +810,28 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     Lm[r * kLmStride + jj] = (jj < r) ? br * ex2(lr - lam[jj]) * v[j] : 0.f;
                 }
             }
-            if (kOut) {
+            if constexpr (kKda) {
+                // after G: K~ -> K o Gamma (the W^T operand), Q~ -> Q o Gamma (the O
+                // operand), Kb -> K o 2^(lambda_L - lambda) (the dS operand), in place;
+                // Gamma = 2^lambda, every factor <= 1
+                const float *ed = sk->edec[buf];
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int n = e + kEpi * it;   // 16-byte chunk of a 64 x 128 tile
+                    const int half = n >> 9, rr = (n & 511) >> 3, pc = n & 7;
+                    const int c0 = 64 * half + 8 * (pc ^ (rr & 7));
+                    const float *f = sk->eref[buf][rr >= 32 ? 1 : 0];
+                    const float4 f0 = *reinterpret_cast<const float4 *>(f + c0);
+                    const float4 f1 = *reinterpret_cast<const float4 *>(f + c0 + 4);
+                    const uint32_t ka = st + half * 16384 + (n & 511) * 16;
+                    sts128(ka, scale_bf16x8v(lds128(ka), f0, f1));
+                    if (kOut) sts128(ka + 8192, scale_bf16x8v(lds128(ka + 8192), f0, f1));
+                    const float4 d0 = *reinterpret_cast<const float4 *>(ed + c0);
+                    const float4 d1 = *reinterpret_cast<const float4 *>(ed + c0 + 4);
+                    const uint32_t ba = sb + Y::kKb + half * 8192 + (n & 511) * 16;
+                    sts128(ba, scale_bf16x8v(lds128(ba), d0, d1));
+                }
+            } else if (kOut) {
                 // after G: Q <- diag(g) Q in place
                 uint4 wq[4];
 #pragma unroll
@@ -673,10 +862,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                         for (int j = 0; j < 16; ++j) {
                             const float tv = Tm[t * kLmStride + j0 + j] * sm->bet[buf][j0 + j];
                             v1[j] = tv;
-                            v2[j] = tv * ex2(lam[j0 + j]);
+                            v2[j] = kKda ? 0.f : tv * ex2(lam[j0 + j]);
                         }
                         st_row_bf16x16(sb + Y::kTp, t, j0 >> 3, v1);
-                        st_row_bf16x16(sb + Y::kTpp, t, j0 >> 3, v2);
+                        // mode 3 keeps Kb0 in this slot: its W^T uses T diag(b)
+                        if (!kKda) st_row_bf16x16(sb + Y::kTpp, t, j0 >> 3, v2);
                     }
                 }
                 fence_async_smem();
@@ -711,12 +901,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                         const int t = 32 * h + j;
                         const float ex = (t < L) ? ((kNeedV ? uu[j] : 0.f) - y[j]) : 0.f;
                         y[j] = ex;
-                        ev[j] = (t < L) ? ex * ex2(lamL - lam[t]) : 0.f;
+                        ev[j] = (!kKda && t < L) ? ex * ex2(lamL - lam[t]) : 0.f;
                     }
 #pragma unroll
                     for (int g = 0; g < 2; ++g) {
                         st_row_bf16x16(sb + Y::kE, row, 4 * h + 2 * g, y + 16 * g);
-                        st_row_bf16x16(sb + Y::kEp, row, 4 * h + 2 * g, ev + 16 * g);
+                        // mode 3 takes the decay in the K operand of dS (Kb): no E'
+                        if (!kKda) st_row_bf16x16(sb + Y::kEp, row, 4 * h + 2 * g, ev + 16 * g);
                     }
                 }
                 fence_async_smem();
@@ -735,13 +926,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             if (*abort) break;
             tc_fence_after();
             const bool last = (c + 1 == nch);
+            // mode 3: the next chunk's operands now that this chunk's products are done;
+            // G(c+1) runs while this chunk's state and outputs are finished
+            if (kKda && !last) kda_scale(c + 1);
             {
                 const float gC = ex2(lamL);
                 {
                     float v[64];
                     tmem_ld64(tl + kColDS + 64 * h, v);
+                    if constexpr (kKda) {   // S <- S Diag(2^lambda_L) + dS: one decay per column
+                        const float *gl = sk->egl[buf] + 64 * h;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) Sr[j] = fmaf(gC, Sr[j], v[j]);
+                        for (int j = 0; j < 64; ++j) Sr[j] = fmaf(gl[j], Sr[j], v[j]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) Sr[j] = fmaf(gC, Sr[j], v[j]);
+                    }
                 }
                 if (!last) {
 #pragma unroll
@@ -764,7 +964,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             epi_sync();
             if (e == 0) {
                 mbar_arrive(&sm->s_ready);
-                mbar_arrive(&sm->empty[s]);
+                // mode 3 stages the outputs in this stage's V slot: released after the store
+                if (!(kKda && kOut)) mbar_arrive(&sm->empty[s]);
             }
 
             // ---- outputs: row t of O (M=64 layout: lane (t % 16) + 32 (t / 16)), half h,
@@ -774,7 +975,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 const int t = 16 * q + lane;
                 const bool has = lane < 16 && t < L;
                 const bool direct = p.cu && L < kC;   // partial chunk of a packed sequence
-                const uint32_t ost = sb + Y::kOst + h * 8192;
+                // mode 3: the V slot of this chunk's stage (V is dead after U^T)
+                const uint32_t obase = kKda ? st + 32768 : sb + Y::kOst;
+                const uint32_t ost = obase + h * 8192;
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {
                     float v[32];
@@ -790,8 +993,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 tc_fence_before();
                 epi_sync();
                 if (e == 0 && !direct) {
-                    tma_store_3d(&p.to, sb + Y::kOst, 0, t0, bh);
-                    tma_store_3d(&p.to, sb + Y::kOst + 8192, 64, t0, bh);
+                    tma_store_3d(&p.to, obase, 0, t0, bh);
+                    tma_store_3d(&p.to, obase + 8192, 64, t0, bh);
                     tma_store_commit();
                 }
             }
@@ -1814,7 +2017,7 @@ Plan plan_for(int mode, int BH, int T) {
     // The local pass covers segments 0 .. nseg-2 only; split them further so that it too
     // fills the SMs (sub-segments of at least four chunks, dividing the segment evenly).
     pl.sub = 1;
-    if (mode != 2 && pl.nseg > 1) {
+    if (mode < 2 && pl.nseg > 1) {
         int f = sms / (BH * (pl.nseg - 1));
         while (f > 1 && (chunks_per_seg % f != 0 || chunks_per_seg / f < 4)) --f;
         pl.sub = std::max(1, f);
@@ -1828,7 +2031,7 @@ size_t workspace_floats(int mode, int BH, const Plan &pl) {
     const size_t nloc = (size_t)(pl.nseg - 1) * pl.sub;   // local-pass sub-segments
     size_t f = (size_t)pl.nseg * per;                 // segment start states
     f += nloc * per;                                  // local states
-    if (mode == 2) f += (size_t)(pl.nseg - 1) * per;  // transitions
+    if (mode >= 2) f += (size_t)(pl.nseg - 1) * per;  // transitions (delta rule)
     if (mode == 1) f += nloc * BH;                    // gate products
     if (mode == 0) f += ((size_t)pl.nseg + nloc) * BH * kD;   // z starts + z locals
     return f;
@@ -1837,12 +2040,12 @@ size_t workspace_floats(int mode, int BH, const Plan &pl) {
 template <int MODE, int KIND>
 cudaError_t launch_kind(const TcParams &p, int grid, cudaStream_t stream) {
     cudaError_t e;
-    if constexpr (MODE == 2) {
-        e = cudaFuncSetAttribute(prefill_tc_kernel<2, KIND>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Lay<2>::kBytes);
+    if constexpr (MODE >= 2) {
+        e = cudaFuncSetAttribute(prefill_tc_kernel<MODE, KIND>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Lay<MODE>::kBytes);
         if (e != cudaSuccess) return e;
         timer_begin(stream);
-        prefill_tc_kernel<2, KIND><<<grid, kThreads, Lay<2>::kBytes, stream>>>(p);
+        prefill_tc_kernel<MODE, KIND><<<grid, kThreads, Lay<MODE>::kBytes, stream>>>(p);
         timer_end(stream);
     } else {
         static_assert(KIND != kTransition, "the transition pass belongs to the delta rule");
@@ -1905,7 +2108,7 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
         p.nseg = nsub;
         cudaError_t e = launch_kind<MODE, kLocal>(p, BH * nsub, a.stream);
         if (e != cudaSuccess) return e;
-        if constexpr (MODE == 2) {
+        if constexpr (MODE >= 2) {
             TcParams q = base;
             q.s_in_mode = 2;
             q.s_out = mtr;
@@ -1919,7 +2122,7 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
     // outputs CTA folds its own start state from the local states (no combine launch).
     // With an initial state the starts are first copied into the workspace by the combine
     // kernel: the outputs pass overwrites the caller's state with the final one.
-    if constexpr (MODE != 2) {
+    if constexpr (MODE < 2) {
         if (!a.init_state && nsub <= 4) {
             TcParams p = base;
             p.s_in_mode = 3;
@@ -1939,7 +2142,7 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
     }
     // combine: segment start states
     const float *s_init = a.init_state ? a.state : nullptr;
-    if constexpr (MODE == 2) {
+    if constexpr (MODE >= 2) {
         const size_t bytes = sizeof(float) * (kD * kD + kCombRows * kD);
         cudaError_t e = cudaFuncSetAttribute(combine_matrix_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -1977,8 +2180,9 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
 }  // namespace
 
 bool prefill_tc_supports(int mode, int dtype, int dk, int dv, int chunk) {
-    // modes 0-2 in bf16 with d = 128; Kimi Delta Attention runs on CUDA cores
-    return mode != LA_MODE_KDA && dtype == LA_BF16 && dk == kD && dv == kD &&
+    // modes 0-3 in bf16 with d = 128 at chunk 64 (chunk 32 selects the CUDA-core path,
+    // which in mode 3 is exact for every gate value: no clamp)
+    return dtype == LA_BF16 && dk == kD && dv == kD &&
            (chunk == 0 || chunk == kC);
 }
 
@@ -2041,6 +2245,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t work
             case LA_MODE_ELU1_NORM: return run_packed<0>(a, p);
             case LA_MODE_GATED: return run_packed<1>(a, p);
             case LA_MODE_GATED_DELTA: return run_packed<2>(a, p);
+            case LA_MODE_KDA: return run_packed<3>(a, p);
         }
         return cudaErrorInvalidValue;
     }
@@ -2048,6 +2253,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t work
         case LA_MODE_ELU1_NORM: return run_mode<0>(a, p, pl, ws);
         case LA_MODE_GATED: return run_mode<1>(a, p, pl, ws);
         case LA_MODE_GATED_DELTA: return run_mode<2>(a, p, pl, ws);
+        case LA_MODE_KDA: return run_mode<3>(a, p, pl, ws);
     }
     return cudaErrorInvalidValue;
 }

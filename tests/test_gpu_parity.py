@@ -181,7 +181,7 @@ def test_decode_steps(la, mode, dtype, d):
 # per-launch timing hook
 # ----------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
 def test_launch_timing_reports_every_launch(la, mode):
     """With timing on, one device duration per kernel the call enqueued (the segmented
     prefill: local pass(es), combine, outputs), all positive; off again, nothing."""
@@ -212,3 +212,30 @@ def test_prefill_segment_starts(la, mode, B, H, T, init):
     combine kernel does.  4 heads x 4096 tokens: 16 segments, always the combine kernel."""
     w = small(mode, torch.bfloat16, 128, T, B=B, H=H, seed=321)
     run_and_compare(la, w, init_std=init)
+
+
+@pytest.mark.parametrize("mode", [2, 3])
+@pytest.mark.parametrize("init", [0.0, 0.05])
+def test_delta_rule_segments(la, mode, init):
+    """The delta-rule segmented prefill (local and transition passes, the matrix combine,
+    the outputs pass) on 4 heads x 3000 tokens: 11 segments with a ragged last one."""
+    w = small(mode, torch.bfloat16, 128, 3000, B=1, H=4, seed=322)
+    run_and_compare(la, w, init_std=init)
+
+
+@pytest.mark.parametrize("T", [64, 200])
+def test_kda_cuda_core_path(la, T):
+    """chunk 32 selects the CUDA-core KDA kernel (exact for every gate) in bf16 too."""
+    w = small(3, torch.bfloat16, 128, T, seed=323)
+    run_and_compare(la, w, chunk=32)
+
+
+@pytest.mark.parametrize("chunk", [0, 32])
+def test_kda_strong_decay(la, chunk):
+    """Gates near 0.0025 on every channel.  The tensor-core path clamps each per-token,
+    per-channel gate at 2^-7.5 = 0.0055 (its operands carry the decays as factors
+    2^(lambda_t - lambda_ref) that must stay finite); such a gate changes the state by
+    at most 0.55 % of what it forgets, inside the bf16 tolerance.  The CUDA-core path
+    (chunk 32) takes the gates as given."""
+    w = small(3, torch.bfloat16, 128, 200, gate_shift=6.0, seed=324)
+    run_and_compare(la, w, init_std=0.05, chunk=chunk)
