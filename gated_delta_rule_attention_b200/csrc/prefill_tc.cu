@@ -26,6 +26,22 @@
 // into the operands by scaling the Q and K tiles in shared memory (mode 1) or the E
 // tile (mode 2), after K K^T / Q K^T have been formed from the unscaled tiles.
 //
+// Mode 3 (Kimi Delta Attention, same section: Diag(a_t), one decay per column c of S)
+// runs the mode-2 kernel with the decays inside the operands.  With per-channel prefixes
+// lam_tc, the pair decay exp(lam_tc - lam_jc) is split between the two factors of the
+// product around a reference token, one per token half (15 and 47), so that no factor
+// spans more than 16 tokens of decay:
+//   G1 = [K~; Q~] Kb^T  (N = 64, kept for rows 32-63),  Kb  = K 2^(lam_47 - lam_j),
+//   G0 = [K~; Q~] Kb0^T (N = 32, kept for rows 0-31),   Kb0 = K 2^(lam_15 - lam_j),
+//   K~, Q~ = K, Q times 2^(lam_t - lam_ref(t)), in place in the stage;
+// then K~ -> K o Gamma (W^T = (K o Gamma)^T (T diag b)^T), Q~ -> Q o Gamma (the O
+// product), Kb -> K o 2^(lam_L - lam) (dS = E^T Kb), and S <- S Diag(2^lam_L) + dS.
+// Every factor stays within 2^120 because each per-token log2 gate is clamped at -7.5
+// (a >= 0.0055); the CUDA-core kernel (chunk 32) takes gates below that as they are.
+// Kb is written only after the previous chunk's products are done (it is one buffer);
+// T diag(b g) is not needed, and its slot holds Kb0; outputs are staged in the chunk's V
+// slot, so that Kb takes the output staging slot.
+//
 // Warp roles (320 threads): warp 0 lane 0 issues TMA loads into a ring of stages;
 // warp 1 owns TMEM and lane 0 issues every MMA; warps 2-9 are the epilogue: two warps
 // per TMEM lane quarter, each taking one half of the columns.  The schedule per chunk c
@@ -37,7 +53,7 @@
 // A CTA processes one (batch*head, segment) pair: a contiguous token range of the
 // sequence.  With several segments per sequence, three kinds of CTA run:
 //   LOCAL       the segment's own state contribution from a zero state (no output),
-//   TRANSITION  (mode 2) the segment's state transition matrix, i.e. the same
+//   TRANSITION  (modes 2, 3) the segment's state transition matrix, i.e. the same
 //               recurrence started from the identity with v = 0 (no output),
 //   OUTPUT      the outputs, started from the exact state at the segment start.
 // A small combine kernel chains segment starts between the two passes.

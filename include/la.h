@@ -100,9 +100,11 @@ typedef enum {
  *   z      [B, H, d_k] fp32            mode 0 only (else ignored, may be NULL): in/out z_T
  *   o      [B, H, T, d_v]  I/O dtype   out: o_1..o_T
  *   chunk  tokens per chunk; 0 picks the kernel's default.  bf16 with d_k = d_v = 128
- *          in modes 0-2 runs on the tensor cores and accepts 0 and 64; every other case
- *          (fp32, d = 64, and mode 3) runs on CUDA cores and accepts 0, 32 and 64 (64 only
- *          when d_k = d_v = 64).  Other values return LA_ERR_UNSUPPORTED.
+ *          runs on the tensor cores at chunk 0 or 64; bf16 at chunk 32, fp32 and d = 64
+ *          run on CUDA cores and accept 0, 32 and 64 (64 only when d_k = d_v = 64).
+ *          Other values return LA_ERR_UNSUPPORTED.  In mode 3 the tensor-core kernel
+ *          clamps every per-channel gate at 2^-7.5 (0.0055) so that its decay factors
+ *          stay finite; chunk 32 selects the CUDA-core kernel, which takes any gate as is.
  *   flags  0 or LA_FLAG_INIT_STATE.
  *   workspace, workspace_bytes
  *          optional device scratch owned by the caller (NULL / 0 allowed).  With at least
