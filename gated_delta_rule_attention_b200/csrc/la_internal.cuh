@@ -79,7 +79,9 @@ cudaError_t launch_decode(const DecodeArgs &a);
 cudaError_t launch_prefill_simt(const PrefillArgs &a);
 bool prefill_simt_supports(int dtype, int dk, int dv, int chunk, int *resolved_chunk);
 bool prefill_tc_supports(int mode, int dtype, int dk, int dv, int chunk);
-size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T);
+// Workspace of the fastest segment plan, or (minimal) of the smallest segmented plan; the
+// launcher picks the fastest plan that fits the workspace it is given.
+size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T, bool minimal = false);
 cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes);
 cudaError_t launch_short_conv(const ConvArgs &a);
 // Zero the state (and z) of every packed sequence with no tokens (cu[s+1] <= cu[s]).

@@ -53,7 +53,13 @@ extern "C" la_status_t la_prefill_noalloc(la_mode_t mode, la_dtype_t dtype, int 
                                           const void *v, const float *gate, const float *beta,
                                           float *state, float *z, void *o, int chunk,
                                           unsigned flags, void *stream) {
-    const size_t need = la_prefill_workspace_size(mode, dtype, B, H, T, d_k, d_v, chunk);
+    // refuse only when even the smallest segmented plan needs more than the static
+    // buffer; the launcher then takes the fastest plan that fits in it
+    size_t need = la_prefill_workspace_size(mode, dtype, B, H, T, d_k, d_v, chunk);
+    if (need > 0) {
+        const int m = (mode == LA_MODE_RETNET) ? (int)LA_MODE_GATED : (int)mode;
+        need = la::prefill_tc_workspace_bytes(m, B, H, T, true);
+    }
     if (need > la::kStaticWorkspaceBytes) return LA_ERR_UNSUPPORTED;
     void *ws = nullptr;
     if (need > 0) {

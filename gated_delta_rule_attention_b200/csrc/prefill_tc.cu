@@ -83,7 +83,9 @@ constexpr uint32_t kColG0 = kColU;
 // that no operand factor 2^(lambda_t - lambda_ref) over half a half-chunk exceeds 2^120.
 constexpr float kKdaLog2Clamp = 7.5f;
 
-enum Kind { kOutput = 0, kLocal = 1, kTransition = 2 };
+// kLocalTrans (delta rule): one launch of both no-output passes, CTAs [0, split) local,
+// [split, 2 split) transition, so that the two share the SMs' waves.
+enum Kind { kOutput = 0, kLocal = 1, kTransition = 2, kLocalTrans = 3 };
 
 struct TcParams {
     CUtensorMap tq, tk, tv, to;  // [BH][T][128] bf16, box 64 x 64 (to: output, stores)
@@ -115,6 +117,9 @@ struct TcParams {
     // Constant per-head gates: gate is [gate_heads], head row bh uses gate[bh % gate_heads]
     // for every token (0: per-token gates [BH][T]).
     int gate_heads;
+    // kLocalTrans: CTAs from `split` on run the transition pass and write s_out2
+    int split;
+    float *s_out2;
     // Packed variable-length sequences (nullptr: dense).  CTA (s, h) takes tokens
     // [cu[s], cu[s+1]) of head row h of the packed [H][T][128] tensors; its state is
     // slot s of the s_in / s_out segment stride.
@@ -127,10 +132,10 @@ struct TcParams {
 struct CtaRange {
     int bh, seg, tb, te;
 };
-__device__ __forceinline__ CtaRange cta_range(const TcParams &p) {
+__device__ __forceinline__ CtaRange cta_range(const TcParams &p, int idx) {
     CtaRange r;
-    r.bh = blockIdx.x % p.BH;
-    r.seg = blockIdx.x / p.BH;
+    r.bh = idx % p.BH;
+    r.seg = idx / p.BH;
     if (p.cu) {
         const int a = p.cu[r.seg], b = p.cu[r.seg + 1];
         r.tb = min(max(a, 0), p.T);
@@ -479,7 +484,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     using Y = Lay<MODE>;
     constexpr int NST = Y::kStages;
     constexpr bool kOut = (KIND == kOutput);
-    constexpr bool kNeedV = (KIND != kTransition);
+    // transition CTAs: the recurrence from the identity with v = 0 (no V, no outputs)
+    const bool trans = (KIND == kTransition) || (KIND == kLocalTrans && (int)blockIdx.x >= p.split);
+    const bool needV = !trans;
 
     // 128B-swizzled operand tiles need 1024-byte aligned atoms.  The buffer is declared
     // with that alignment and never re-aligned by integer arithmetic: pointers derived
@@ -495,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const CtaRange rng = cta_range(p);
+    const CtaRange rng = cta_range(p, (int)blockIdx.x - (KIND == kLocalTrans && trans ? p.split : 0));
     const int bh = rng.bh, seg = rng.seg, tb = rng.tb, te = rng.te;
     if (te <= tb) return;   // an empty packed sequence: nothing to read or write
     const int nch = (te - tb + kC - 1) / kC;
@@ -533,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (lane == 0) {
             tma_prefetch_desc(&p.tk);
             if (kOut) tma_prefetch_desc(&p.tq);
-            if (kNeedV) tma_prefetch_desc(&p.tv);
+            if (needV) tma_prefetch_desc(&p.tv);
             int issued[NST];
             for (int s = 0; s < NST; ++s) issued[s] = 0;
             for (int c = 0; c < nch; ++c) {
@@ -541,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 if (u >= 1 && !mbar_wait(&sm->empty[s], (u - 1) & 1, abort, p.err)) break;
                 const uint32_t st = sb + s * Y::kStage;
                 const int t = tb + kC * c;
-                const uint32_t bytes = 16384u * (1u + (kOut ? 1u : 0u) + (kNeedV ? 1u : 0u));
+                const uint32_t bytes = 16384u * (1u + (kOut ? 1u : 0u) + (needV ? 1u : 0u));
                 mbar_arrive_expect_tx(&sm->full[s], bytes);
                 tma_load_3d(st + 0, &p.tk, 0, t, bh, &sm->full[s]);
                 tma_load_3d(st + 16384, &p.tk, 64, t, bh, &sm->full[s]);
@@ -549,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     tma_load_3d(st + 8192, &p.tq, 0, t, bh, &sm->full[s]);
                     tma_load_3d(st + 24576, &p.tq, 64, t, bh, &sm->full[s]);
                 }
-                if (kNeedV) {
+                if (needV) {
                     tma_load_3d(st + 32768, &p.tv, 0, t, bh, &sm->full[s]);
                     tma_load_3d(st + 40960, &p.tv, 64, t, bh, &sm->full[s]);
                 }
@@ -595,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 {
                     if (!mbar_wait(&sm->tt_ready, par, abort, p.err)) break;
                     tc_fence_after();
-                    if (kNeedV)   // U^T = V^T (T diag b)^T
+                    if (needV)   // U^T = V^T (T diag b)^T
                         mma_chain<4, false, true>(tm + kColU, dmn(st + 32768, 8192), dk(tp), id_uw, false);
                     // W^T = K^T (T diag(b g))^T; mode 3: (K o Gamma)^T (T diag b)^T
                     mma_chain<4, false, true>(tm + kColW, dmn(st, 16384), dk(kKda ? tp : tpp), id_uw, false);
@@ -641,12 +648,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         float Sr[64];
         {
             const float *src = nullptr;
-            if (p.s_in_mode == 1)
+            const int s_in_mode = trans ? 2 : p.s_in_mode;
+            if (s_in_mode == 1)
                 src = p.s_in + (size_t)seg * p.s_in_seg + (size_t)bh * kD * kD + (size_t)row * kD;
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
                 const int col = 64 * h + j;
-                Sr[j] = src ? src[col] : ((p.s_in_mode == 2 && col == row) ? 1.f : 0.f);
+                Sr[j] = src ? src[col] : ((s_in_mode == 2 && col == row) ? 1.f : 0.f);
             }
 #pragma unroll
             for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
@@ -911,11 +919,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 {
                     float y[32], uu[32], ev[32];
                     tmem_ld32(tl + kColY + 32 * h, y);
-                    if (kNeedV) tmem_ld32(tl + kColU + 32 * h, uu);
+                    if (needV) tmem_ld32(tl + kColU + 32 * h, uu);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int t = 32 * h + j;
-                        const float ex = (t < L) ? ((kNeedV ? uu[j] : 0.f) - y[j]) : 0.f;
+                        const float ex = (t < L) ? ((needV ? uu[j] : 0.f) - y[j]) : 0.f;
                         y[j] = ex;
                         ev[j] = (!kKda && t < L) ? ex * ex2(lamL - lam[t]) : 0.f;
                     }
@@ -964,9 +972,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     for (int g = 0; g < 4; ++g) st_row_bf16x16(sbf + h * 16384, row, 2 * g, Sr + 16 * g);
                 }
                 if (last) {
-                    const bool write = p.s_out && (!p.out_last_only || seg == p.nseg - 1);
+                    float *out = (KIND == kLocalTrans && trans) ? p.s_out2 : p.s_out;
+                    const bool write = out && (!p.out_last_only || seg == p.nseg - 1);
                     if (write) {
-                        float *dst = p.s_out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
+                        float *dst = out + (size_t)seg * p.s_out_seg + (size_t)bh * kD * kD +
                                      (size_t)row * kD + 64 * h;
 #pragma unroll
                         for (int j = 0; j < 64; j += 4)
@@ -1097,7 +1106,7 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const CtaRange rng = cta_range(p);
+    const CtaRange rng = cta_range(p, (int)blockIdx.x);
     const int bh = rng.bh, seg = rng.seg, tb = rng.tb, te = rng.te;
     if (te <= tb) return;   // an empty packed sequence: nothing to read or write
     const int nch = (te - tb + kC - 1) / kC;
@@ -1527,7 +1536,7 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const CtaRange rng = cta_range(p);
+    const CtaRange rng = cta_range(p, (int)blockIdx.x);
     const int bh = rng.bh, seg = rng.seg, tb = rng.tb, te = rng.te;
     if (te <= tb) return;   // an empty packed sequence: nothing to read or write
     const int nch = (te - tb + kC - 1) / kC;
@@ -1967,9 +1976,11 @@ __global__ void combine_scalar_kernel(int BH, int nseg, int f, const float *s_in
     }
 }
 
-// mode 2: S_start[s+1] = S_start[s] M_s + N_s (row-parallel; 16 rows of S per CTA).
+// delta rule: S <- S M_j + N_j over the sub-segments j in order (f per segment), writing
+// the start of segment s+1 after its f-th (row-parallel; 16 rows of S per CTA).
 constexpr int kCombRows = 16;
-__global__ void __launch_bounds__(256) combine_matrix_kernel(int BH, int nseg, const float *s_init,
+__global__ void __launch_bounds__(256) combine_matrix_kernel(int BH, int nseg, int f,
+                                                             const float *s_init,
                                                              const float *nloc, const float *mtr,
                                                              float *sst) {
     extern __shared__ float csm[];
@@ -1985,7 +1996,8 @@ __global__ void __launch_bounds__(256) combine_matrix_kernel(int BH, int nseg, c
         Ss[i] = v;
         sst[g] = v;
     }
-    for (int s = 0; s + 1 < nseg; ++s) {
+    const int nsub = (nseg - 1) * f;
+    for (int s = 0; s < nsub; ++s) {
         __syncthreads();
         const float *Mg = mtr + (size_t)s * total + (size_t)bh * per;
         for (int i = threadIdx.x; i < kD * kD / 4; i += 256)
@@ -2003,13 +2015,14 @@ __global__ void __launch_bounds__(256) combine_matrix_kernel(int BH, int nseg, c
         }
         __syncthreads();
         const float *Ng = nloc + (size_t)s * total + (size_t)bh * per;
-        float *dst = sst + (size_t)(s + 1) * total + (size_t)bh * per;
+        const bool boundary = (s + 1) % f == 0;
+        float *dst = sst + (size_t)((s + 1) / f) * total + (size_t)bh * per;
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
             const size_t g = (size_t)(r0 + rb + r) * kD + col;
             const float v = acc[r] + Ng[g];
             Ss[(rb + r) * kD + col] = v;
-            dst[g] = v;
+            if (boundary) dst[g] = v;
         }
     }
 }
@@ -2020,7 +2033,10 @@ struct Plan {
     int sub;   // modes 0/1: the local pass runs on `sub` equal sub-segments per segment
 };
 
-Plan plan_for(int mode, int BH, int T) {
+// The segment plan for BH heads of T tokens whose workspace fits max_ws bytes (without a
+// segmented plan that fits: one outputs pass over whole sequences).
+size_t workspace_floats(int mode, int BH, const struct Plan &pl);
+Plan plan_for(int mode, int BH, int T, size_t max_ws = SIZE_MAX) {
     const int nchunks = (T + kC - 1) / kC;
     int nseg = 1;
     const int sms = 148;
@@ -2038,6 +2054,31 @@ Plan plan_for(int mode, int BH, int T) {
         while (f > 1 && (chunks_per_seg % f != 0 || chunks_per_seg / f < 4)) --f;
         pl.sub = std::max(1, f);
     }
+    if (mode >= 2 && pl.nseg > 1) {
+        // Delta rule: the local and transition CTAs of the segments 0 .. nseg-2 share one
+        // launch.  Splitting segments into f sub-segments gives more, shorter CTAs; cost
+        // ~ waves x chunks per sub-segment + the combine's matrix steps (about two chunks'
+        // time each), with sub-segments of at least eight chunks that fit the workspace.
+        double best = 0.0;
+        for (int f = 1; f <= 8; f *= 2) {
+            if (f > 1 && (chunks_per_seg % f != 0 || chunks_per_seg / f < 8)) break;
+            Plan t = pl;
+            t.sub = f;
+            if (f > 1 && sizeof(float) * workspace_floats(mode, BH, t) > max_ws) break;
+            const int ctas = 2 * BH * (pl.nseg - 1) * f;
+            const double cost = (double)((ctas + sms - 1) / sms) * (chunks_per_seg / f) +
+                                2.0 * (pl.nseg - 1) * f;
+            if (f == 1 || cost < best) {
+                best = cost;
+                pl.sub = f;
+            }
+        }
+    }
+    if (pl.nseg > 1 && sizeof(float) * workspace_floats(mode, BH, pl) > max_ws) {
+        pl.nseg = 1;
+        pl.sub = 1;
+        pl.seg_len = nchunks * kC;
+    }
     return pl;
 }
 
@@ -2047,7 +2088,7 @@ size_t workspace_floats(int mode, int BH, const Plan &pl) {
     const size_t nloc = (size_t)(pl.nseg - 1) * pl.sub;   // local-pass sub-segments
     size_t f = (size_t)pl.nseg * per;                 // segment start states
     f += nloc * per;                                  // local states
-    if (mode >= 2) f += (size_t)(pl.nseg - 1) * per;  // transitions (delta rule)
+    if (mode >= 2) f += nloc * per;                   // transitions (delta rule)
     if (mode == 1) f += nloc * BH;                    // gate products
     if (mode == 0) f += ((size_t)pl.nseg + nloc) * BH * kD;   // z starts + z locals
     return f;
@@ -2064,7 +2105,8 @@ cudaError_t launch_kind(const TcParams &p, int grid, cudaStream_t stream) {
         prefill_tc_kernel<MODE, KIND><<<grid, kThreads, Lay<MODE>::kBytes, stream>>>(p);
         timer_end(stream);
     } else {
-        static_assert(KIND != kTransition, "the transition pass belongs to the delta rule");
+        static_assert(KIND != kTransition && KIND != kLocalTrans,
+                      "the transition pass belongs to the delta rule");
         if constexpr (MODE == 0) {
             e = cudaFuncSetAttribute(prefill_elu_kernel<KIND>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, LayE::kBytes);
@@ -2110,7 +2152,8 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
     float *gam = nloc + (size_t)nsub * per;                      // mode 1
     float *zst = nloc + (size_t)nsub * per;                      // mode 0
     float *zloc = zst + (size_t)pl.nseg * BH * kD;
-    // pass A: local states (and transitions)
+    // pass A: local states of the sub-segments (and, delta rule, their transitions, in
+    // the same launch)
     {
         TcParams p = base;
         p.s_in_mode = 0;
@@ -2122,17 +2165,15 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
         p.out_last_only = 0;
         p.seg_len = pl.seg_len / pl.sub;
         p.nseg = nsub;
-        cudaError_t e = launch_kind<MODE, kLocal>(p, BH * nsub, a.stream);
-        if (e != cudaSuccess) return e;
+        cudaError_t e;
         if constexpr (MODE >= 2) {
-            TcParams q = base;
-            q.s_in_mode = 2;
-            q.s_out = mtr;
-            q.s_out_seg = (long long)per;
-            q.out_last_only = 0;
-            e = launch_kind<MODE, kTransition>(q, BH * (pl.nseg - 1), a.stream);
-            if (e != cudaSuccess) return e;
+            p.s_out2 = mtr;
+            p.split = BH * nsub;
+            e = launch_kind<MODE, kLocalTrans>(p, 2 * BH * nsub, a.stream);
+        } else {
+            e = launch_kind<MODE, kLocal>(p, BH * nsub, a.stream);
         }
+        if (e != cudaSuccess) return e;
     }
     // Outputs pass.  Without an initial state and with few sub-segments per head, each
     // outputs CTA folds its own start state from the local states (no combine launch).
@@ -2165,7 +2206,7 @@ cudaError_t run_mode(const PrefillArgs &a, const TcParams &base, const Plan &pl,
         if (e != cudaSuccess) return e;
         timer_begin(a.stream);
         combine_matrix_kernel<<<dim3(BH, kD / kCombRows), 256, bytes, a.stream>>>(
-            BH, pl.nseg, s_init, nloc, mtr, sst);
+            BH, pl.nseg, pl.sub, s_init, nloc, mtr, sst);
         timer_end(a.stream);
     } else {
         const size_t total4 = per / 4;
@@ -2202,9 +2243,11 @@ bool prefill_tc_supports(int mode, int dtype, int dk, int dv, int chunk) {
            (chunk == 0 || chunk == kC);
 }
 
-size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T) {
+size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T, bool minimal) {
     const int BH = B * H;
-    return sizeof(float) * workspace_floats(mode, BH, plan_for(mode, BH, T));
+    Plan pl = plan_for(mode, BH, T);
+    if (minimal && mode >= 2) pl.sub = 1;   // the smallest segmented plan
+    return sizeof(float) * workspace_floats(mode, BH, pl);
 }
 
 // Packed sequences: one outputs-pass CTA per (sequence, head), started from the
@@ -2229,11 +2272,7 @@ cudaError_t run_packed(const PrefillArgs &a, const TcParams &base) {
 
 cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes) {
     const int BH = a.B * a.H;
-    Plan pl = plan_for(a.mode, BH, a.T);
-    if (sizeof(float) * workspace_floats(a.mode, BH, pl) > workspace_bytes || !workspace) {
-        pl.nseg = 1;
-        pl.seg_len = ((a.T + kC - 1) / kC) * kC;
-    }
+    const Plan pl = plan_for(a.mode, BH, a.T, workspace ? workspace_bytes : 0);
     TcParams p;
     memset(&p, 0, sizeof(p));
     const uint64_t row_pitch = kD * 2, head_pitch = (uint64_t)a.T * kD * 2;

@@ -110,8 +110,8 @@ typedef enum {
  *          optional device scratch owned by the caller (NULL / 0 allowed).  With at least
  *          la_prefill_workspace_size() bytes the tensor-core kernel splits each sequence
  *          into segments processed in parallel and chains their states exactly; with
- *          less it runs each sequence in one pass (same result up to rounding, less
- *          parallelism when B*H is small).  Calls that share a workspace must not
+ *          less it takes the fastest segment plan that fits, or runs each sequence in
+ *          one pass (same result up to rounding, less parallelism when B*H is small).  Calls that share a workspace must not
  *          overlap on the device.
  * T = 0 is allowed: nothing is read from q, k, v, o; the state is left as given (with
  * LA_FLAG_INIT_STATE) or zeroed.  q, k, v, o may then be NULL.
@@ -166,8 +166,10 @@ size_t la_prefill_workspace_size(la_mode_t mode, la_dtype_t dtype, int B, int H,
  * arguments as la_prefill except the workspace, which it takes from a 24 MiB array
  * that the library keeps in device memory (every GPU that loads the library holds it
  * until exit).  It allocates nothing and calls no allocating routine.
- *   - Returns LA_ERR_UNSUPPORTED when la_prefill_workspace_size() for these sizes
- *     exceeds 24 MiB; nothing is launched then.
+ *   - Returns LA_ERR_UNSUPPORTED when even the smallest segment plan for these sizes
+ *     needs more than 24 MiB (la_prefill_workspace_size() reports the fastest plan's
+ *     need, which may be larger); nothing is launched then.  Otherwise the fastest plan
+ *     that fits in 24 MiB runs.
  *   - The first call on a device looks up the array's device address (with that device
  *     current); make that first call before any stream capture on the device.
  *   - All calls share the array and it keeps the last call's contents (no result
