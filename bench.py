@@ -622,6 +622,9 @@ def run_reference(args):
     if rank != 0:
         return 0
     name = args.workload
+    if name not in W.CONFIGS:
+        print(json.dumps({"impl": "reference", "unavailable": f"no oracle sample for {name}"}))
+        return 0
     per_step = []
     res = None
     for i in range(args.warmup + args.steps):
@@ -649,12 +652,38 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------------
 
+def workload_config(name, world):
+    """(I/O dtype, the JSON line's config) of a workload of any of the three kinds."""
+    common = {"parallelism": f"dp{world} (independent sequences per GPU)",
+              "l2": "flushed between timed steps (256 MiB write)"}
+    if name in W.CONV_CONFIGS:
+        cw = W.CONV_CONFIGS[name]
+        return cw.dtype, {"workload": name, "kind": "short convolution of q, k, v", "B": cw.B,
+                          "H": cw.H, "T": cw.T, "d_k": cw.dk, "d_v": cw.dv, "width": cw.width,
+                          "silu": cw.silu, "l2norm_qk": cw.l2norm_qk, "global_batch": cw.B * world,
+                          "seq_len": cw.T, **common}
+    if name in W.VARLEN_CONFIGS:
+        vw = W.VARLEN_CONFIGS[name]
+        L = vw.lengths()
+        return vw.base.dtype, {"workload": name, "kind": "packed variable-length prefill",
+                               "mode": vw.base.mode, "N": vw.N, "H": vw.base.H, "tokens": sum(L),
+                               "min_len": min(L), "max_len": max(L), "d_k": vw.base.dk,
+                               "d_v": vw.base.dv, "global_batch": vw.N * world,
+                               "seq_len": max(L), "state_dtype": "f32", "accum": "f32", **common}
+    w = W.CONFIGS[name]
+    return w.dtype, {"workload": name, "mode": w.mode, "B": w.B, "H": w.H, "T": w.T,
+                     "d_k": w.dk, "d_v": w.dv, "chunk": w.chunk or "default",
+                     "global_batch": w.B * world, "seq_len": w.T, **common,
+                     "state_dtype": "f32", "accum": "f32"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.CONFIGS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(list(W.CONFIGS) + list(W.CONV_CONFIGS) + list(W.VARLEN_CONFIGS)))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--extras", type=int, default=-1,
                     help="1: also measure the other workloads (default: on at N=1)")
@@ -701,7 +730,7 @@ def main():
             cpu = {"value": None, "error": str(e)[:200], "kind": "oracle"}
 
     peaks, peak_src = load_peaks()
-    w = W.CONFIGS[args.workload]
+    dtype, wconfig = workload_config(args.workload, world)
     case = main_res["_case"]
     mean_ms = statistics.mean(main_res["_ms"])
     roof = roofline(case, main_res["kernel_ms"], mean_ms, peaks, peak_src, ncu_traffic(args.workload))
@@ -718,14 +747,9 @@ def main():
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+            "dtype": "bf16" if dtype == torch.bfloat16 else "f32",
             "data": "synthetic",
-            "config": {"workload": args.workload, "mode": w.mode, "B": w.B, "H": w.H, "T": w.T,
-                       "d_k": w.dk, "d_v": w.dv, "chunk": w.chunk or "default",
-                       "global_batch": w.B * world, "seq_len": w.T,
-                       "parallelism": f"dp{world} (independent sequences per GPU)",
-                       "l2": "flushed between timed steps (256 MiB write)",
-                       "state_dtype": "f32", "accum": "f32"},
+            "config": wconfig,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": main_res.get("e2e"),
