@@ -154,15 +154,29 @@ def kernel_sources_sha():
     return h.hexdigest()[:16]
 
 
+def source_file_shas():
+    """{file: sha} of every kernel source file (csrc/*.cu, *.cuh)."""
+    csrc = os.path.join(ROOT, "gated_delta_rule_attention_b200", "csrc")
+    out = {}
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                out[fn] = hashlib.sha256(f.read()).hexdigest()[:16]
+    return out
+
+
 def ncu_traffic(workload: str):
     """The committed ncu launch summary of `workload` (kernels in launch order, each with
-    its DRAM bytes per launch and time share), or None when it was taken on other kernel
-    sources than the ones built here."""
+    its DRAM bytes per launch and time share), or None when any source file that existed
+    when it was taken has changed since (a file added later cannot change those kernels:
+    every translation unit and header they were built from is among the recorded ones)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
-        if t.get("sources_sha") != kernel_sources_sha():
+        now = source_file_shas()
+        rec = t.get("sources")
+        if not rec or any(now.get(fn) != sha for fn, sha in rec.items()):
             return None
         return t["workloads"][workload]
     except Exception:
