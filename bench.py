@@ -386,6 +386,50 @@ class VarlenCase:
         self.h_state.copy_(self.state, non_blocking=True)
 
 
+class BackwardCase:
+    """One step = one la_prefill_backward call (mode 1): dq, dk, dv and the gate gradient
+    for the default prefill's shape, from output cotangents dO."""
+
+    def __init__(self, la, w: W.Workload, device, rank):
+        self.la, self.w, self.device = la, w, device
+        wr = W.variant(w, seed=w.seed + 1000 * rank)
+        self.inp = W.prefill_inputs(wr, device=device)
+        g = torch.Generator(device=device).manual_seed(wr.seed + 1)
+        self.dO = torch.randn(w.B, w.H, w.T, w.dv, generator=g, device=device).to(w.dtype)
+        self.tokens = w.B * w.T
+        th = w.B * w.H * w.T
+        e = io_bytes(w.dtype)
+        # read q, k, v, dO and the gates; write dq, dk, dv and the gate gradient
+        self.bytes = float(th * (e * (3 * w.dk + 4 * w.dv) + 8))
+        # forward recompute of the states and four d_k x d_v products per token-head, plus
+        # the chunk's score products (C = 32)
+        self.flops = float(th * (10 * w.dk * w.dv + 8 * 32 * (w.dk + w.dv)))
+        self.kind = "backward"
+
+    def step(self):
+        i = self.inp
+        self.la.prefill_backward(i["q"], i["k"], i["v"], self.dO, mode=self.w.mode, gate=i["gate"])
+
+    def e2e_setup(self):
+        pin = lambda t: t.to("cpu").pin_memory()
+        self.h_in = {k: pin(self.inp[k]) for k in ("q", "k", "v", "gate")}
+        self.h_do = pin(self.dO)
+        self.h_out = [torch.empty(self.inp["q"].shape, dtype=self.w.dtype).pin_memory() for _ in range(3)]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values()) + \
+            self.h_do.numel() * self.h_do.element_size()
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+
+    def e2e_step(self):
+        for k, v in self.h_in.items():
+            self.inp[k].copy_(v, non_blocking=True)
+        self.dO.copy_(self.h_do, non_blocking=True)
+        i = self.inp
+        dq, dk, dv, _, _ = self.la.prefill_backward(i["q"], i["k"], i["v"], self.dO, mode=self.w.mode,
+                                                    gate=i["gate"])
+        for h, d in zip(self.h_out, (dq, dk, dv)):
+            h.copy_(d, non_blocking=True)
+
+
 class ConvCase:
     """One step = the short convolution prologue of one prefill batch: three
     la_short_conv calls (q and k with SiLU and the L2 norm, v with SiLU), token-major
@@ -537,6 +581,8 @@ def measure(la, name, args, dist, device, rank, world, flush, with_e2e, sampler=
         case = ConvCase(la, W.CONV_CONFIGS[name], device, rank)
     elif name in W.VARLEN_CONFIGS:
         case = VarlenCase(la, W.VARLEN_CONFIGS[name], device, rank)
+    elif name in W.BACKWARD_CONFIGS:
+        case = BackwardCase(la, W.BACKWARD_CONFIGS[name], device, rank)
     else:
         w = W.CONFIGS[name]
         case = (DecodeCase(la, w, device, rank, args.warmup + args.steps) if w.decode
@@ -684,7 +730,7 @@ def workload_config(name, world):
                                "min_len": min(L), "max_len": max(L), "d_k": vw.base.dk,
                                "d_v": vw.base.dv, "global_batch": vw.N * world,
                                "seq_len": max(L), "state_dtype": "f32", "accum": "f32", **common}
-    w = W.CONFIGS[name]
+    w = W.CONFIGS[name] if name in W.CONFIGS else W.BACKWARD_CONFIGS[name]
     return w.dtype, {"workload": name, "mode": w.mode, "B": w.B, "H": w.H, "T": w.T,
                      "d_k": w.dk, "d_v": w.dv, "chunk": w.chunk or "default",
                      "global_batch": w.B * world, "seq_len": w.T, **common,
@@ -697,7 +743,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=sorted(list(W.CONFIGS) + list(W.CONV_CONFIGS) + list(W.VARLEN_CONFIGS)))
+                    choices=sorted(list(W.CONFIGS) + list(W.CONV_CONFIGS) + list(W.VARLEN_CONFIGS) +
+                                   list(W.BACKWARD_CONFIGS)))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--extras", type=int, default=-1,
                     help="1: also measure the other workloads (default: on at N=1)")
@@ -728,7 +775,8 @@ def main():
     if do_extras:
         for name in ("elu1_bf16_b4h16t4096", "gated_bf16_b8h16t8192", "gdn_bf16_b2h16t32768",
                      "gdn_decode_n256h32", "kda_bf16_b2h16t32768", "kda_decode_n256h32",
-                     "conv_bf16_b2h16t32768", "gdn_varlen_bf16_n64h16", "retnet_bf16_b8h16t8192"):
+                     "conv_bf16_b2h16t32768", "gdn_varlen_bf16_n64h16", "retnet_bf16_b8h16t8192",
+                     "gated_bwd_bf16_b4h16t4096"):
             if name == args.workload:
                 continue
             r = measure(la, name, args, dist, device, rank, world, flush, False)

@@ -257,6 +257,37 @@ la_status_t la_short_conv_step(la_dtype_t dtype, int N, int H, int d, int width,
                                unsigned flags, void *stream);
 
 /*
+ * la_prefill_backward -- gradients of the prefill for the scalar-gate modes (1 and 4):
+ * the derivatives of L = sum_t do_t . o_t + <dS_T, S_T> for the recurrence of
+ * [decay/gates], S_t = a_t S_{t-1} + v_t k_t^T, o_t = S_t q_t, with respect to q, k, v, the
+ * gates and the initial state.  The chunked form ([three forms]) is the one the page uses
+ * for training; it gives no backward formulas, so they are the plain derivatives:
+ *   dQ = diag(g) dO S_c + dP K,  dK = dP^T Q + diag(g_L/g) V G,  dV = P^T dO + diag(g_L/g) K G^T
+ * per chunk (P = (Q K^T) o D, dP = (dO V^T) o D, S_c the chunk-start state, G = dL/dS at
+ * the chunk's end), and d log a_t = sum_{u >= t} (q_u . dq_u - k_u . dk_u) (plus
+ * <dS_T, S_T> at the last token).  CUDA cores, fp32 arithmetic, one CTA per (b, h).
+ *
+ *   mode          LA_MODE_GATED or LA_MODE_RETNET (others: LA_ERR_UNSUPPORTED)
+ *   q, k          [B, H, T, d_k] I/O dtype      v, dO [B, H, T, d_v] I/O dtype
+ *   gate          as for la_prefill (mode 1: [B, H, T] or NULL; mode 4: [H], required)
+ *   state0        [B, H, d_v, d_k] fp32 initial state, or NULL for zero
+ *   dstate        [B, H, d_v, d_k] fp32 cotangent of the final state, or NULL for zero
+ *   dq, dk, dv    out, shapes of q, k, v, I/O dtype
+ *   dgate         out [B, H, T] fp32 (mode 1 with a gate), or NULL; mode 4 takes its
+ *                 gates as fixed and requires NULL.  Gates must be > 0: d a = d log a / a.
+ *   dstate0       out [B, H, d_v, d_k] fp32 (the gradient of state0), or NULL
+ *   workspace     device scratch of at least la_backward_workspace_size() bytes
+ *                 (required: every chunk-start state is kept there)
+ */
+size_t la_backward_workspace_size(la_mode_t mode, int B, int H, int T, int d_k, int d_v);
+la_status_t la_prefill_backward(la_mode_t mode, la_dtype_t dtype, int B, int H, int T, int d_k,
+                                int d_v, const void *q, const void *k, const void *v,
+                                const float *gate, const float *state0, const void *dO,
+                                const float *dstate, void *dq, void *dk, void *dv, float *dgate,
+                                float *dstate0, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/*
  * la_check_status -- synchronise `stream`, then report the first device-side failure
  * since the last call: LA_ERR_CUDA for a CUDA error, LA_ERR_TIMEOUT if a kernel's
  * bounded wait ran out (the kernel then returned early and its outputs are invalid),
@@ -287,7 +318,8 @@ unsigned long long la_kernel_launches(void);
 
 /* Per-launch device timing, a measurement aid with no counterpart in the pages.
  * la_launch_timing(1) makes every later call of la_prefill, la_prefill_noalloc,
- * la_prefill_varlen, la_decode_step and the la_short_conv* entry points bracket each
+ * la_prefill_varlen, la_prefill_backward, la_decode_step and the la_short_conv* entry
+ * points bracket each
  * kernel it enqueues
  * with two CUDA events recorded on the call's stream (at most 16 launches per call are
  * timed); la_launch_timing(0) turns it off (the default).  Enabling adds two event

@@ -184,3 +184,19 @@ def test_retnet_mode_needs_its_gate(lib):
     assert lib.la_decode_step(4, 1, 1, 1, 128, 128, *([None] * 9)) == INVALID
     assert lib.la_prefill_workspace_size(4, 1, 1, 16, 32768, 128, 128, 0) > 0   # the mode-1 plan
     assert lib.la_prefill_workspace_size(5, 1, 1, 16, 32768, 128, 128, 0) == 0
+
+
+def test_prefill_backward_argument_checks(lib):
+    INVALID, UNSUPPORTED = 1, 2
+
+    def call(mode=1, dtype=1, B=1, H=2, T=64, dk=128, dv=128):
+        return lib.la_prefill_backward(mode, dtype, B, H, T, dk, dv, *([None] * 13), 0, None)
+
+    assert call(mode=2) == UNSUPPORTED     # the delta rule's backward is not built
+    assert call(mode=7) == INVALID
+    assert call(T=0) == INVALID
+    assert call(dk=32) == UNSUPPORTED
+    assert call() == INVALID               # NULL tensors, before any launch
+    assert call(mode=4) == INVALID         # mode 4 needs its gate
+    assert lib.la_backward_workspace_size(1, 2, 3, 100, 64, 64) == 4 * 2 * 3 * 5 * 64 * 64
+    assert lib.la_backward_workspace_size(2, 2, 3, 100, 64, 64) == 0

@@ -155,6 +155,15 @@ def variant(w: Workload, **changes) -> Workload:
     return dataclasses.replace(w, **changes)
 
 
+# The backward pass of the scalar-gated prefill (mode 1): the default prefill's shape
+# (B4 H16 T4096, d = 128, bf16) with the gated recipe; output cotangents dO ~ N(0, 1).
+BACKWARD_CONFIGS = {
+    "gated_bwd_bf16_b4h16t4096": Workload("gated_bwd_bf16_b4h16t4096", MODE_GATED, torch.bfloat16,
+                                          B=4, H=16, T=4096, dk=128, dv=128, seed=11,
+                                          qk_scale=1 / math.sqrt(128), gate="softplus"),
+}
+
+
 # ---- the short causal convolution in front of q, k, v
 @dataclasses.dataclass(frozen=True)
 class ConvWorkload:
