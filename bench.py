@@ -100,8 +100,8 @@ def prefill_algorithmic(w: W.Workload, C=64):
 
     bytes: q, k, v read + o written, gates/beta read (mode 3: d_k gates per token),
     final state (and z) written.
-    flops per token-head: modes 0/1  2C d_k + 2C d_v + 4 d_k d_v;
-                          modes 2/3  10 C d + 6 d^2 + C^2 / 3  (d = d_k = d_v; the per-channel
+    flops per token-head: modes 0/1/4  2C d_k + 2C d_v + 4 d_k d_v;
+                          modes 2/3    10 C d + 6 d^2 + C^2 / 3  (d = d_k = d_v; the per-channel
                           decays of mode 3 are exponentials inside the products, not counted)."""
     th = w.B * w.H * w.T
     e = io_bytes(w.dtype)
@@ -111,7 +111,7 @@ def prefill_algorithmic(w: W.Workload, C=64):
     if w.beta:
         b += th * 4
     b += w.B * w.H * (w.dv * w.dk * 4 + (w.dk * 4 if w.mode == 0 else 0))
-    if w.mode >= 2:
+    if w.mode in (2, 3):   # the delta rule (mode 4 is the scalar-gate recurrence)
         d = w.dk
         f = 10 * C * d + 6 * d * d + C * C / 3.0
     else:
