@@ -20,7 +20,9 @@
 //
 // One CTA (256 threads) per (batch, head), fp32 arithmetic on CUDA cores: a forward sweep
 // stores every chunk-start state in the caller's workspace, then a reverse sweep carries G
-// back through the chunks.  Tiles live in shared memory with one float of row padding.
+// back through the chunks.  Tiles live in shared memory with one float of row padding; the
+// products are register-tiled (a thread holds up to 16 x 4 outputs), so that each shared
+// load feeds several FMAs.
 #include "la_internal.cuh"
 
 #include <cfloat>
@@ -37,7 +39,7 @@ struct BwdSmem {
     static constexpr int kQ = kBwdC * (DK + 1);
     static constexpr int kV = kBwdC * (DV + 1);
     static constexpr int kP = kBwdC * (kBwdC + 1);
-    static constexpr int kFloats = 2 * kS + 2 * kQ + 2 * kV + 2 * kP + 4 * kBwdC + 8;
+    static constexpr int kFloats = 2 * kS + 2 * kQ + 2 * kV + 2 * kP + 5 * kBwdC + 8;
     static constexpr size_t kBytes = sizeof(float) * kFloats;
 };
 
@@ -53,6 +55,26 @@ __device__ __forceinline__ float block_sum(float x, float *red) {
     return s;
 }
 
+// Register-tiled products on shared-memory operands.  A thread computes RM rows x RN
+// columns of an M x N output: rows r0 + i (i < RM) and columns lane + 32 n (n < RN), so
+// that the B operand's loads are consecutive across the warp and the A operand's are
+// broadcasts.  acc[i][n] += sum_k A(row, k) B(k, col).
+template <int RM, int RN, int K, typename FA, typename FB>
+__device__ __forceinline__ void tile_mma(float (&acc)[RM][RN], int r0, int lane, FA a, FB b) {
+#pragma unroll 4
+    for (int kk = 0; kk < K; ++kk) {
+        float av[RM], bv[RN];
+#pragma unroll
+        for (int i = 0; i < RM; ++i) av[i] = a(r0 + i, kk);
+#pragma unroll
+        for (int n = 0; n < RN; ++n) bv[n] = b(kk, lane + 32 * n);
+#pragma unroll
+        for (int i = 0; i < RM; ++i)
+#pragma unroll
+            for (int n = 0; n < RN; ++n) acc[i][n] = fmaf(av[i], bv[n], acc[i][n]);
+    }
+}
+
 template <int DK, int DV, typename IO>
 __global__ void __launch_bounds__(kBwdThreads)
 backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__restrict__ k,
@@ -63,6 +85,10 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
                 float *__restrict__ ws) {
     using L = BwdSmem<DK, DV>;
     constexpr int C = kBwdC, SK = DK + 1, SV = DV + 1, SP = C + 1;
+    constexpr int NW = kBwdThreads / 32;       // 8 warps
+    constexpr int RC = C / NW;                 // chunk rows per warp (4)
+    constexpr int RS = DV / NW;                // state rows per warp (16 or 8)
+    constexpr int NK = DK / 32, NV = DV / 32;  // columns per lane
     extern __shared__ float smem[];
     float *S = smem;             // [DV][DK+1]  state (forward) / chunk-start state (reverse)
     float *G = S + L::kS;        // [DV][DK+1]  dL/dS at the chunk's end
@@ -72,13 +98,14 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
     float *dOs = Vs + L::kV;     // [C][DV+1]
     float *P = dOs + L::kV;      // [C][C+1]
     float *dP = P + L::kP;       // [C][C+1]
-    float *lam = dP + L::kP;     // [C]
-    float *dl = lam + C;         // [C]   dlam
-    float *av = dl + C;          // [C]   gate values (clamped)
-    float *dlr = av + C;         // [C]
-    float *red = dlr + C;        // [8]
+    float *lam = dP + L::kP;     // [C]   in-chunk log-gate prefix
+    float *gv = lam + C;         // [C]   g_t = exp(lam_t)
+    float *dec = gv + C;         // [C]   g_L / g_t
+    float *av = dec + C;         // [C]   gate values (clamped)
+    float *dl = av + C;          // [C]   dlam, then its suffix sums
+    float *red = dl + C;         // [8]
 
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t bh = blockIdx.x;
     const int nch = (T + C - 1) / C;
     const size_t row0 = bh * (size_t)T;
@@ -96,12 +123,30 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
         if (tid == 0)
             for (int i = 1; i < C; ++i) lam[i] += lam[i - 1];
         __syncthreads();
+        if (tid < C) {
+            gv[tid] = expf(lam[tid]);
+            dec[tid] = expf(lam[Lc - 1] - lam[tid]);
+        }
+        __syncthreads();
     };
     auto load_rows = [&](const IO *src, float *dst, int t0, int Lc, int d, int stride) {
         for (int p = tid; p < C * d; p += kBwdThreads) {
             const int i = p / d, j = p % d;
             dst[i * stride + j] = i < Lc ? to_f32(src[(row0 + t0 + i) * d + j]) : 0.f;
         }
+    };
+    // S <- gL S + sum_j (dec_j v_j) k_j^T  (this thread's 16 x NK or 8 x NK elements)
+    auto state_step = [&](float *M, float gL) {
+        float acc[RS][NK] = {};
+        tile_mma<RS, NK, C>(acc, RS * warp, lane, [&](int i, int j) { return dec[j] * Vs[j * SV + i]; },
+                            [&](int j, int cc) { return Ks[j * SK + cc]; });
+#pragma unroll
+        for (int i = 0; i < RS; ++i)
+#pragma unroll
+            for (int n = 0; n < NK; ++n) {
+                float &x = M[(RS * warp + i) * SK + lane + 32 * n];
+                x = fmaf(gL, x, acc[i][n]);
+            }
     };
 
     // ---- forward sweep: chunk-start states into the workspace
@@ -113,14 +158,8 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
         const int t0 = c * C, Lc = min(C, T - t0);
         load_rows(k, Ks, t0, Lc, DK, SK);
         load_rows(v, Vs, t0, Lc, DV, SV);
-        load_gates(t0, Lc);
-        const float lL = lam[Lc - 1], gL = expf(lL);
-        for (int p = tid; p < DV * DK; p += kBwdThreads) {
-            const int i = p / DK, cc = p % DK;
-            float acc = 0.f;
-            for (int j = 0; j < Lc; ++j) acc = fmaf(expf(lL - lam[j]) * Vs[j * SV + i], Ks[j * SK + cc], acc);
-            S[i * SK + cc] = fmaf(gL, S[i * SK + cc], acc);
-        }
+        load_gates(t0, Lc);   // (synchronises: every thread has stored S)
+        state_step(S, expf(lam[Lc - 1]));
         __syncthreads();
     }
     __syncthreads();
@@ -129,9 +168,9 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
     // S holds S_T: <dS_T, S_T> enters dlam at the last token
     float part = 0.f;
     for (int p = tid; p < DV * DK; p += kBwdThreads) {
-        const float gv = dST ? dST[bh * DV * DK + p] : 0.f;
-        G[(p / DK) * SK + p % DK] = gv;
-        part = fmaf(gv, S[(p / DK) * SK + p % DK], part);
+        const float g0 = dST ? dST[bh * DV * DK + p] : 0.f;
+        G[(p / DK) * SK + p % DK] = g0;
+        part = fmaf(g0, S[(p / DK) * SK + p % DK], part);
     }
     const float final_dot = block_sum(part, red);
     float R = 0.f;   // sum of dlam over the tokens after this chunk
@@ -144,46 +183,91 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
         for (int p = tid; p < DV * DK; p += kBwdThreads) S[(p / DK) * SK + p % DK] = wsh[(size_t)c * DV * DK + p];
         if (tid < C) dl[tid] = 0.f;
         load_gates(t0, Lc);   // (synchronises)
-        const float lL = lam[Lc - 1], gL = expf(lL);
-        // causal decayed score matrices
+        const float gL = gv[Lc - 1];
+        // causal decayed score matrices P = (Q K^T) o D, dP = (dO V^T) o D
         for (int p = tid; p < C * C; p += kBwdThreads) {
             const int t = p / C, j = p % C;
             float pv = 0.f, dpv = 0.f;
             if (t < Lc && j <= t) {
-                const float dec = expf(lam[t] - lam[j]);
+                const float dd = expf(lam[t] - lam[j]);
                 float a1 = 0.f, a2 = 0.f;
                 for (int cc = 0; cc < DK; ++cc) a1 = fmaf(Qs[t * SK + cc], Ks[j * SK + cc], a1);
                 for (int i = 0; i < DV; ++i) a2 = fmaf(dOs[t * SV + i], Vs[j * SV + i], a2);
-                pv = a1 * dec;
-                dpv = a2 * dec;
+                pv = a1 * dd;
+                dpv = a2 * dd;
             }
             P[t * SP + j] = pv;
             dP[t * SP + j] = dpv;
         }
         __syncthreads();
-        // dQ and dK (rows t, columns cc), with their share of dlam
-        for (int p = tid; p < Lc * DK; p += kBwdThreads) {
-            const int t = p / DK, cc = p % DK;
-            float sd = 0.f, gv = 0.f;
-            for (int i = 0; i < DV; ++i) {
-                sd = fmaf(S[i * SK + cc], dOs[t * SV + i], sd);
-                gv = fmaf(G[i * SK + cc], Vs[t * SV + i], gv);
+        const int r0 = RC * warp;   // this warp's chunk rows
+        {   // dQ = diag(g) dO S_c + dP K
+            float acc[RC][NK] = {};
+            tile_mma<RC, NK, DV>(acc, r0, lane, [&](int t, int i) { return dOs[t * SV + i]; },
+                                 [&](int i, int cc) { return S[i * SK + cc]; });
+#pragma unroll
+            for (int i = 0; i < RC; ++i)
+#pragma unroll
+                for (int n = 0; n < NK; ++n) acc[i][n] *= gv[r0 + i];
+            tile_mma<RC, NK, C>(acc, r0, lane, [&](int t, int j) { return dP[t * SP + j]; },
+                                [&](int j, int cc) { return Ks[j * SK + cc]; });
+#pragma unroll
+            for (int i = 0; i < RC; ++i) {
+                const int t = r0 + i;
+                float qd = 0.f;
+#pragma unroll
+                for (int n = 0; n < NK; ++n) {
+                    const int cc = lane + 32 * n;
+                    qd = fmaf(Qs[t * SK + cc], acc[i][n], qd);
+                    if (t < Lc) dq[(row0 + t0 + t) * DK + cc] = from_f32<IO>(acc[i][n]);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) qd += __shfl_xor_sync(0xffffffffu, qd, off);
+                if (lane == 0 && t < Lc) atomicAdd(&dl[t], qd);
             }
-            float a = expf(lam[t]) * sd, b = expf(lL - lam[t]) * gv;
-            for (int j = 0; j <= t; ++j) a = fmaf(dP[t * SP + j], Ks[j * SK + cc], a);
-            for (int s = t; s < Lc; ++s) b = fmaf(dP[s * SP + t], Qs[s * SK + cc], b);
-            dq[(row0 + t0 + t) * DK + cc] = from_f32<IO>(a);
-            dk[(row0 + t0 + t) * DK + cc] = from_f32<IO>(b);
-            atomicAdd(&dl[t], Qs[t * SK + cc] * a - Ks[t * SK + cc] * b);
         }
-        // dV
-        for (int p = tid; p < Lc * DV; p += kBwdThreads) {
-            const int t = p / DV, i = p % DV;
-            float gk = 0.f;
-            for (int cc = 0; cc < DK; ++cc) gk = fmaf(G[i * SK + cc], Ks[t * SK + cc], gk);
-            float b = expf(lL - lam[t]) * gk;
-            for (int s = t; s < Lc; ++s) b = fmaf(P[s * SP + t], dOs[s * SV + i], b);
-            dv[(row0 + t0 + t) * DV + i] = from_f32<IO>(b);
+        {   // dK = dP^T Q + diag(g_L / g) V G
+            float acc[RC][NK] = {};
+            tile_mma<RC, NK, DV>(acc, r0, lane, [&](int t, int i) { return Vs[t * SV + i]; },
+                                 [&](int i, int cc) { return G[i * SK + cc]; });
+#pragma unroll
+            for (int i = 0; i < RC; ++i)
+#pragma unroll
+                for (int n = 0; n < NK; ++n) acc[i][n] *= dec[r0 + i];
+            tile_mma<RC, NK, C>(acc, r0, lane, [&](int t, int s) { return dP[s * SP + t]; },
+                                [&](int s, int cc) { return Qs[s * SK + cc]; });
+#pragma unroll
+            for (int i = 0; i < RC; ++i) {
+                const int t = r0 + i;
+                float kd = 0.f;
+#pragma unroll
+                for (int n = 0; n < NK; ++n) {
+                    const int cc = lane + 32 * n;
+                    kd = fmaf(Ks[t * SK + cc], acc[i][n], kd);
+                    if (t < Lc) dk[(row0 + t0 + t) * DK + cc] = from_f32<IO>(acc[i][n]);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) kd += __shfl_xor_sync(0xffffffffu, kd, off);
+                if (lane == 0 && t < Lc) atomicAdd(&dl[t], -kd);
+            }
+        }
+        {   // dV = P^T dO + diag(g_L / g) K G^T
+            float acc[RC][NV] = {};
+            tile_mma<RC, NV, DK>(acc, r0, lane, [&](int t, int cc) { return Ks[t * SK + cc]; },
+                                 [&](int cc, int i) { return G[i * SK + cc]; });
+#pragma unroll
+            for (int i = 0; i < RC; ++i)
+#pragma unroll
+                for (int n = 0; n < NV; ++n) acc[i][n] *= dec[r0 + i];
+            tile_mma<RC, NV, C>(acc, r0, lane, [&](int t, int s) { return P[s * SP + t]; },
+                                [&](int s, int i) { return dOs[s * SV + i]; });
+#pragma unroll
+            for (int i = 0; i < RC; ++i) {
+                const int t = r0 + i;
+                if (t < Lc)
+#pragma unroll
+                    for (int n = 0; n < NV; ++n) dv[(row0 + t0 + t) * DV + lane + 32 * n] = from_f32<IO>(acc[i][n]);
+            }
         }
         __syncthreads();
         // gate gradient: suffix sums of dlam
@@ -192,19 +276,24 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
             float run = R;
             for (int t = Lc - 1; t >= 0; --t) {
                 run += dl[t];
-                dlr[t] = run;
+                dl[t] = run;
             }
-            R = run;
         }
         __syncthreads();
-        R = dlr[0];
-        if (dgate && tid < Lc) dgate[row0 + t0 + tid] = dlr[tid] / av[tid];
+        R = dl[0];
+        if (dgate && tid < Lc) dgate[row0 + t0 + tid] = dl[tid] / av[tid];
         // carry G to the chunk start: G <- g_L G + dO^T diag(g) Q
-        for (int p = tid; p < DV * DK; p += kBwdThreads) {
-            const int i = p / DK, cc = p % DK;
-            float acc = 0.f;
-            for (int t = 0; t < Lc; ++t) acc = fmaf(expf(lam[t]) * dOs[t * SV + i], Qs[t * SK + cc], acc);
-            G[i * SK + cc] = fmaf(gL, G[i * SK + cc], acc);
+        {
+            float acc[RS][NK] = {};
+            tile_mma<RS, NK, C>(acc, RS * warp, lane, [&](int i, int t) { return gv[t] * dOs[t * SV + i]; },
+                                [&](int t, int cc) { return Qs[t * SK + cc]; });
+#pragma unroll
+            for (int i = 0; i < RS; ++i)
+#pragma unroll
+                for (int n = 0; n < NK; ++n) {
+                    float &x = G[(RS * warp + i) * SK + lane + 32 * n];
+                    x = fmaf(gL, x, acc[i][n]);
+                }
         }
         __syncthreads();
     }
