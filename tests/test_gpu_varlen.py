@@ -121,3 +121,45 @@ def test_varlen_serving_batch_sampled(la):
                                        sl(inp["beta"]))
             assert slice_rel_err(f64(o[h, a:b])[None], ro[0], lead=1) < TOL[torch.bfloat16]
             assert slice_rel_err(f64(S[s, h])[None], rS[0, 0][None], lead=1) < TOL[torch.bfloat16]
+
+
+def test_serving_chain_conv_prefill_decode(la):
+    """A packed serving step end to end: the short convolution over packed projections
+    (SiLU, q/k L2 norm), the packed Gated DeltaNet prefill from per-sequence start states,
+    then one decode step per sequence from the states it wrote -- against the oracle
+    chain on the same bf16 intermediates."""
+    from oracle import conv as oconv
+    lengths = [40, 1, 97, 64]
+    N, H, d, width = len(lengths), 2, 128, 4
+    T = sum(lengths)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32, device="cuda")
+    ys, refs = [], []
+    for i in range(3):
+        x, w, _ = W.conv_inputs(1, T, H * d, width, torch.bfloat16, seed=500 + i, device="cuda",
+                                window=False)
+        y, _ = la.short_conv_varlen(x[0], w, cu, heads=H, silu=True, l2norm=(i < 2))
+        ys.append(y)
+        refs.append(oconv.short_conv_packed(f64(x[0]), f64(w), cu.tolist(), None, H=H, silu=True,
+                                            l2norm=(i < 2))[0])
+    for y, r in zip(ys, refs):
+        assert slice_rel_err(f64(y), r, lead=1) < 8e-3
+    g = torch.Generator(device="cuda").manual_seed(9)
+    gate = torch.sigmoid(torch.randn(H, T, generator=g, device="cuda") + 3.0)
+    beta = torch.sigmoid(torch.randn(H, T, generator=g, device="cuda"))
+    S0 = torch.randn(N, H, d, d, generator=g, device="cuda") * 0.05
+    o, S, _ = la.prefill_varlen(*ys, cu, mode=2, gate=gate, beta=beta, state=S0.clone())
+    la.check_status()
+    ro, rS, _ = oracle.prefill_packed(2, f64(ys[0]), f64(ys[1]), f64(ys[2]), cu.tolist(), f64(gate),
+                                      f64(beta), f64(S0))
+    assert seq_err(f64(o), ro, cu.tolist()) < TOL[torch.bfloat16]
+    assert slice_rel_err(f64(S), rS) < TOL[torch.bfloat16]
+    # one decode step per sequence from the packed final states
+    q1, k1, v1 = (torch.nn.functional.normalize(torch.randn(N, H, d, generator=g, device="cuda"), dim=-1)
+                  .to(torch.bfloat16) for _ in range(3))
+    a1 = torch.sigmoid(torch.randn(N, H, generator=g, device="cuda") + 3.0)
+    b1 = torch.sigmoid(torch.randn(N, H, generator=g, device="cuda"))
+    od, S2, _ = la.decode_step(q1, k1, v1, mode=2, state=S.clone(), gate=a1, beta=b1)
+    la.check_status()
+    rod, rS2, _ = oracle.decode_step(2, f64(q1), f64(k1), f64(v1), f64(a1), f64(b1), f64(S))
+    assert slice_rel_err(f64(od), rod, lead=1) < TOL[torch.bfloat16]
+    assert slice_rel_err(f64(S2), rS2) < TOL[torch.bfloat16]
