@@ -78,3 +78,21 @@ def test_backward_argument_checks(la):
                                      p(inp["gate"]), None, p(dO), None, p(x[0]), p(x[1]), p(x[2]),
                                      p(dg), None, p(ws), n, None)
         la._check(st, "la_prefill_backward")
+
+
+def test_backward_full_size_sampled(la):
+    """The benchmark's backward workload (mode 1, B4 H16 T4096, d = 128, bf16) in its launch
+    configuration, checked on sampled heads: the oracle runs on each head alone."""
+    w = W.BACKWARD_CONFIGS["gated_bwd_bf16_b4h16t4096"]
+    inp = W.prefill_inputs(w, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(w.seed + 1)
+    dO = torch.randn(w.B, w.H, w.T, w.dv, generator=g, device="cuda").to(w.dtype)
+    dq, dk, dv, dg, _ = la.prefill_backward(inp["q"], inp["k"], inp["v"], dO, mode=1, gate=inp["gate"])
+    la.check_status()
+    for b, h in [(0, 0), (3, 15)]:
+        sl = lambda t: f64(t[b:b + 1, h:h + 1])
+        rq, rk, rv, rg, _ = ob.prefill_backward(1, sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["gate"]),
+                                                sl(dO))
+        for name, x, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv), ("dgate", dg, rg)):
+            e = slice_rel_err(sl(x), r)
+            assert e < TOL[w.dtype], f"{name} head ({b},{h}): {e:.3e}"
