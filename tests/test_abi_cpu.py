@@ -198,5 +198,5 @@ def test_prefill_backward_argument_checks(lib):
     assert call(dk=32) == UNSUPPORTED
     assert call() == INVALID               # NULL tensors, before any launch
     assert call(mode=4) == INVALID         # mode 4 needs its gate
-    assert lib.la_backward_workspace_size(1, 2, 3, 100, 64, 64) == 4 * 2 * 3 * 5 * 64 * 64
+    assert lib.la_backward_workspace_size(1, 2, 3, 100, 64, 64) == 4 * 2 * 3 * (5 * 64 * 64 + 100 * 65)
     assert lib.la_backward_workspace_size(2, 2, 3, 100, 64, 64) == 0
