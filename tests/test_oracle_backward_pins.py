@@ -1,16 +1,36 @@
 """Pins for the fp64 backward oracle (``oracle/backward.py``).
 
 The gradients come from reverse-mode differentiation of the recurrent form; they are tied
-to things other than that machinery: central finite differences of the loss (every input,
-tiny sizes), the closed form of the ungated case, and the decay identity that the CUDA
-kernel uses, d log a_t = sum_{u >= t} (q_u . dq_u - k_u . dk_u) (plus <dS_T, S_T> at the
-last token), which follows from differentiating the decay mask exp(lam_s - lam_j).
+to things other than that machinery: the forward recurrence itself equals the pinned C
+oracle, central finite differences of the loss (every input, tiny sizes), the closed form
+of the ungated case, and the decay identity that the CUDA kernel uses,
+d log a_t = sum_{u >= t} (q_u . dq_u - k_u . dk_u) (plus <dS_T, S_T> at the last token),
+which follows from differentiating the decay mask exp(lam_s - lam_j).
 """
+import importlib.util
+import os
+
 import numpy as np
 import pytest
 import torch
 
-from oracle import backward as ob
+import oracle
+
+
+def _load_backward():
+    # A test that plants a mistake in a copy of oracle/backward.py points this at the copy,
+    # to check that these pins catch it.
+    path = os.environ.get("LA_ORACLE_BACKWARD_OVERRIDE")
+    if not path:
+        from oracle import backward as mod
+        return mod
+    spec = importlib.util.spec_from_file_location("backward_mutant", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+ob = _load_backward()
 
 
 def _inputs(seed, B=1, H=2, T=7, dk=3, dv=2):
@@ -92,3 +112,16 @@ def test_retnet_mode_has_no_gate_gradient_and_matches_mode1():
     assert r4[3] is None
     for x, y in zip(r4[:3] + r4[4:], r1[:3] + r1[4:]):
         np.testing.assert_allclose(x, y, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_forward_recurrence_is_the_pinned_c_oracle(with_state):
+    """The recurrence the gradients differentiate is the scalar-gate mode of the C oracle
+    (pinned on its own to the page's worked examples and closed forms)."""
+    q, k, v, _, a, S0, _ = _inputs(6, B=2, H=3, T=11)
+    if not with_state:
+        S0 = None
+    o, ST = ob.recurrence(*(None if x is None else torch.as_tensor(x) for x in (q, k, v, a, S0)))
+    ro, rS, _ = oracle.prefill(1, q, k, v, a, None, S0)
+    np.testing.assert_allclose(o.numpy(), ro, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ST.numpy(), rS, rtol=1e-12, atol=1e-12)

@@ -84,3 +84,28 @@ def test_conv_pins_catch_planted_mistakes(name, tmp_path):
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"planted mistake {name} passed every pin:\n{r.stdout[-2000:]}"
     assert "failed" in r.stdout or "error" in r.stdout.lower()
+
+
+BWD_SRC = os.path.join(ROOT, "oracle", "backward.py")
+BWD_MUTANTS = {
+    "bwd_gate_after_write": ("        S = S if a is None else a[:, :, t, None, None] * S\n        S = S + v[:, :, t, :, None] * k[:, :, t, None, :]",
+                             "        S = S + v[:, :, t, :, None] * k[:, :, t, None, :]\n        S = S if a is None else a[:, :, t, None, None] * S"),
+    "bwd_reads_before_write": ("        S = S + v[:, :, t, :, None] * k[:, :, t, None, :]\n        outs.append(torch.einsum(\"bhij,bhj->bhi\", S, q[:, :, t]))",
+                               "        outs.append(torch.einsum(\"bhij,bhj->bhi\", S, q[:, :, t]))\n        S = S + v[:, :, t, :, None] * k[:, :, t, None, :]"),
+    "bwd_drops_final_state_term": ("        L = L + (ST * _t(dS_T)).sum()", "        L = L + 0.0 * (ST * _t(dS_T)).sum()"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BWD_MUTANTS))
+def test_backward_pins_catch_planted_mistakes(name, tmp_path):
+    old, new = BWD_MUTANTS[name]
+    src = open(BWD_SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mutant = tmp_path / "backward_mutant.py"
+    mutant.write_text(src.replace(old, new))
+    env = dict(os.environ, LA_ORACLE_BACKWARD_OVERRIDE=str(mutant))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_backward_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"planted mistake {name} passed every pin:\n{r.stdout[-2000:]}"
+    assert "failed" in r.stdout or "error" in r.stdout.lower()
