@@ -83,6 +83,10 @@ bool prefill_tc_supports(int mode, int dtype, int dk, int dv, int chunk);
 // launcher picks the fastest plan that fits the workspace it is given.
 size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T, bool minimal = false);
 cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes);
+// The single-pass gated-delta prefill (d_v split over four CTAs per head, no workspace):
+// whether it serves a call of BH head rows (dense or packed), and its launcher.
+bool prefill_gdn_selected(int mode, int BH, bool packed);
+cudaError_t launch_prefill_gdn(const PrefillArgs &a);
 cudaError_t launch_short_conv(const ConvArgs &a);
 // Zero the state (and z) of every packed sequence with no tokens (cu[s+1] <= cu[s]).
 cudaError_t launch_zero_empty_sequences(const PrefillArgs &a);

@@ -1,0 +1,674 @@
+// prefill_gdn.cu -- single-pass chunked prefill of the gated delta rule (mode 2) on the
+// 5th-generation tensor cores, bf16 I/O, d_k = d_v = 128, chunk C = 64, fp32 state.
+//
+// The update is the Gated DeltaNet equation of the lesson page "Linear attention and
+// hybrids", section "The delta rule and Gated DeltaNet":
+//     S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S_t q_t,
+// evaluated chunk by chunk as in section "Three forms of one computation" (inside a chunk
+// a masked C x C matrix, across chunks the carried state).  Per chunk of L <= 64 tokens,
+// with the in-chunk log2-gate prefix lam_t, g_t = 2^lam_t, dec_t = 2^(lam_{L-1} - lam_t):
+//
+//   G  = [Q; K] K^T                                    (state independent)
+//   A  = (Q K^T) * 2^(lam_t - lam_j), j <= t;   Lm = strictly-lower(diag(b) 2^(lam_t - lam_j) K K^T)
+//   T  = (I + Lm)^-1;   W = T diag(b g) K;   U = T diag(b) V
+//   P  = [diag(g) Q; W] S^T                            (state dependent: the chain)
+//   E  = U - W S^T   (rows t: e_t = b_t (v_t - a_t S_{t-1} k_t), the delta-rule writes)
+//   O  = diag(g) Q S^T + A E,   S^T <- g_{L-1} S^T + K^T diag(dec) E
+//
+// Rows of S evolve independently given the chunk's K, b and gates, so each head's d_v rows
+// are split over kNS = 4 CTAs of 32 rows: the 32 heads of a B2 H16 workload give 128 CTAs,
+// with no segments, transition pass or combine.  Every CTA forms the state-independent
+// half itself (the four slices of a head run side by side and share its tiles through
+// L2) one chunk ahead of the short state chain.  Roles:
+//
+//   warp 0       TMA producer: Q, K (two 64x64 boxes each) and the 64-column half of V
+//                that holds the slice, into a ring of three stages; L2 prefetch ahead
+//   warp 1       owns tensor memory
+//   warp 3       gates: per stage the log2-gate prefix, beta, beta g and the column decay
+//                factors, up to three chunks ahead (it completes the stage with the TMA)
+//   warps 4-11   prep: A and Lm from G (masks, decays), the 64x64 inverse, T diag(b) and
+//                T diag(b g); an elected thread issues G, W and U
+//   warps 12-15  chain: [diag(g) Q; W] into tensor memory (the A operand of P), E from
+//                U - W S^T, the state S^T (fp32, one d_k row of 32 values per thread) and
+//                its bf16 copy, the outputs; elected threads issue P, dS and A E
+//
+// Each group issues its own products right after the named barrier that publishes their
+// operands, so no product waits for a hand-off through another warp.  Product shapes
+// (M x N x K, kind::f16, fp32 accumulators in tensor memory): G 128x64x128,
+// W = [X; T diag(b g)] K 128x128x64 and U = [X; T diag(b)] V 128x64x64 (rows 64-127 are
+// the result; X are the 64 rows of shared memory in front of the operand, whose products
+// land in accumulator rows nobody reads), P 128x32x128 with A in tensor memory,
+// dS^T = K^T E' 128x32x64 and A E 128x32x64 accumulated onto the rows 0-63 of P (again
+// with 64 unused rows after the A tile).  Every wait is bounded; a timeout records an
+// error, every role leaves its loop, in-flight copies and products are drained and the
+// tensor memory is freed.
+#include "la_internal.cuh"
+#include "ptx.cuh"
+#include "tc_util.cuh"
+#include "tmap.cuh"
+
+#include <cfloat>
+#include <cstddef>
+#include <cstring>
+
+namespace la {
+namespace {
+
+using namespace ptx;
+using namespace tc;
+
+constexpr int kC = 64;
+constexpr int kD = 128;
+constexpr int kNS = 4;           // d_v slices per head
+constexpr int kDV = kD / kNS;    // 32 rows of S per CTA
+constexpr int kStages = 3;
+constexpr int kThreads = 512;
+constexpr int kPrepT = 256;      // warps 4-11
+constexpr int kChainT = 128;     // warps 12-15
+// named barriers
+constexpr uint32_t kBarPrep = 1, kBarChain = 3, kBarChainE = 4, kBarChainO = 5;
+// A chunk whose column decay factor 2^(lam_{16b} - lam_j) inside a 16-token block exceeds
+// 2^kFastSpan takes the exact per-element exponentials (no overflow in the fast factors).
+constexpr float kFastSpan = 100.f;
+
+// tensor memory columns
+constexpr uint32_t kColG = 0;      // 64   G (fp32)
+constexpr uint32_t kColW = 64;     // 128  W in lanes 64-127
+constexpr uint32_t kColU = 192;    // 64   U (the V half) in lanes 64-127
+constexpr uint32_t kColQW = 256;   // 2 x 64: [diag(g) Q; W] as bf16 pairs, per chunk parity
+constexpr uint32_t kColP = 384;    // 2 x 32: P (+ A E) per chunk parity
+constexpr uint32_t kColDS = 448;   // 32   dS^T
+constexpr uint32_t kTmemCols = 512;
+
+// shared memory (bytes from the 1024-aligned base)
+constexpr uint32_t kStage = 40960;                 // [Q0 | K0 | Q1 | K1 | V], 8 KB each
+constexpr uint32_t kA0 = kStages * kStage;         // A tile, chunk parity 0 (8 KB)
+constexpr uint32_t kA1 = kA0 + 8192;               // parity 1
+constexpr uint32_t kTbg = kA1 + 8192;              // T diag(b g)   [t][j] bf16
+constexpr uint32_t kTb = kTbg + 8192;              // T diag(b)
+constexpr uint32_t kLm = kTb + 8192;               // fp32 64 x kTStride
+constexpr uint32_t kTm = kLm + 64 * kTStride * 4;
+constexpr uint32_t kZs = kTm + 64 * kTStride * 4;  // 4 x 272 floats
+constexpr uint32_t kS = (kZs + 4 * 272 * 4 + 1023) & ~1023u;   // S^T bf16, 128 rows x 128 B
+constexpr uint32_t kE = kS + 16384;                // E   [t] rows of 128 B (64 B used)
+constexpr uint32_t kEp = kE + 8192;                // E' = diag(dec) E
+constexpr uint32_t kSmall = kEp + 8192;
+
+// Per-stage gate data, written by the gate warp: arrays read as float4 come first.
+struct Gates {
+    float lam[kC];   // inclusive prefix of log2(a) within the chunk
+    float bet[kC];   // beta (0 past the end of the sequence)
+    float bg[kC];    // beta 2^lam
+    float cf[kC];    // 2^(lam_{16 floor(j/16)} - lam_j) >= 1
+    int len;
+    int slow;        // some cf exceeds 2^kFastSpan: exact exponentials for this chunk
+    int pad[2];
+};
+struct Small {
+    Gates gt[kStages];
+    uint64_t full[kStages], empty[kStages];
+    uint64_t g_done, wu_done, w_free, u_free;
+    uint64_t p_done, ds_done;
+    uint64_t ae_done[2];
+    uint32_t tmem_base;
+    int abort;
+};
+static_assert(sizeof(Gates) % 16 == 0 && offsetof(Gates, cf) % 16 == 0, "float4 gate rows");
+static_assert(kSmall % 16 == 0, "gate rows are read as float4");
+constexpr uint32_t kBytes = kSmall + sizeof(Small);
+static_assert(kBytes <= 227 * 1024, "shared memory per CTA");
+
+struct GdnParams {
+    CUtensorMap tq, tk, tv;     // [BH][T][128] bf16, 64 x 64 boxes, 128B swizzle
+    const float *gate;          // [BH][T] or nullptr (a = 1)
+    const float *beta;          // [BH][T]
+    __nv_bfloat16 *o;           // [BH][T][128]
+    const float *s_in;          // nullable: zero start state
+    float *s_out;
+    long long seq_stride;       // state slot stride of a packed sequence (floats)
+    const int *cu;              // packed sequences (nullptr: dense)
+    int T, BH;
+    unsigned *err;
+};
+
+__device__ __forceinline__ void gdn_range(const GdnParams &p, int unit, int &bh, int &seq, int &tb,
+                                          int &te) {
+    bh = unit % p.BH;
+    seq = unit / p.BH;
+    if (p.cu) {
+        const int a = p.cu[seq], b = p.cu[seq + 1];
+        tb = min(max(a, 0), p.T);
+        te = min(max(b, tb), p.T);
+        if ((a != tb || b != te) && threadIdx.x == 0 && p.err) atomicOr(p.err, (unsigned)kErrBadInput);
+    } else {
+        tb = 0;
+        te = p.T;
+    }
+}
+
+// One thread of a group polls `bar` (bounded wait); the group then meets at named barrier
+// `id` of `n` threads, which also makes the decision to abandon uniform.  Waiting at the
+// named barrier costs the other threads no issue slots.  False: abandon.
+__device__ __forceinline__ bool group_wait(uint64_t *bar, uint32_t parity, bool poller, uint32_t id,
+                                           uint32_t n, volatile int *abort, unsigned *err) {
+    if (poller) mbar_wait(bar, parity, abort, err);
+    return !named_sync_any(id, n, *abort != 0);
+}
+
+// D (+)= A B with A in tensor memory (K-major, 8 columns per K = 16 step) and B an
+// MN-major shared-memory operand (rows of 128 bytes, 2048 bytes per step).
+template <int NK>
+__device__ __forceinline__ void mma_chain_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, bool accumulate_first) {
+#pragma unroll
+    for (int ks = 0; ks < NK; ++ks)
+        mma_bf16_ts(d_tmem, a_tmem + 8 * ks, b_desc + (uint64_t)(ks * 128), idesc,
+                    accumulate_first || ks > 0);
+}
+
+// 32 fp32 values as bf16 into the first 64 bytes (4 chunks) of row `row` of a 128B-swizzled
+// MN-major tile.
+__device__ __forceinline__ void st_row32_mn(uint32_t tile, uint32_t row, const float *v) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+        w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+        w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+        w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+        sts128(tile + sw128_off(row, q), w);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_constant__ GdnParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sb = smem_u32(smem_raw);
+    if (sb & 1023u) {
+        if (threadIdx.x == 0 && p.err) atomicOr(p.err, (unsigned)kErrBadLaunch);
+        return;
+    }
+    Small *sm = reinterpret_cast<Small *>(smem_raw + kSmall);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int vs = blockIdx.x % kNS;           // d_v slice: rows [32 vs, 32 vs + 32) of S
+    int bh, seq, tb, te;
+    gdn_range(p, blockIdx.x / kNS, bh, seq, tb, te);
+    if (te <= tb) return;   // an empty packed sequence
+    const int nch = (te - tb + kC - 1) / kC;
+    const size_t slot = (size_t)seq * p.seq_stride + (size_t)bh * kD * kD;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm->full[s], 2);   // the TMA bytes and the gate warp
+            mbar_init(&sm->empty[s], 1);
+        }
+        mbar_init(&sm->g_done, 1);
+        mbar_init(&sm->wu_done, 1);
+        mbar_init(&sm->w_free, 1);
+        mbar_init(&sm->u_free, 1);
+        mbar_init(&sm->p_done, 1);
+        mbar_init(&sm->ds_done, 1);
+        mbar_init(&sm->ae_done[0], 1);
+        mbar_init(&sm->ae_done[1], 1);
+        sm->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = sm->tmem_base;
+    volatile int *abort = &sm->abort;
+    // instruction descriptors
+    const uint32_t id_g = idesc_bf16(128, 64, false, false);
+    const uint32_t id_w = idesc_bf16(128, 128, false, true);
+    const uint32_t id_u = idesc_bf16(128, 64, false, true);
+    const uint32_t id_p = idesc_bf16(128, kDV, false, true);
+    const uint32_t id_ds = idesc_bf16(128, kDV, true, true);
+    const uint32_t id_ae = idesc_bf16(128, kDV, false, true);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tq);
+            tma_prefetch_desc(&p.tk);
+            tma_prefetch_desc(&p.tv);
+            const int vx = 64 * (vs >> 1);
+            int issued[kStages] = {0, 0, 0};
+            for (int c = 0; c < nch; ++c) {
+                const int s = c % kStages, u = c / kStages;
+                if (u >= 1 && !mbar_wait(&sm->empty[s], (u - 1) & 1, abort, p.err)) break;
+                const uint32_t st = sb + s * kStage;
+                const int t = tb + kC * c;
+                mbar_arrive_expect_tx(&sm->full[s], kStage);
+                tma_load_3d(st + 0, &p.tq, 0, t, bh, &sm->full[s]);
+                tma_load_3d(st + 8192, &p.tk, 0, t, bh, &sm->full[s]);
+                tma_load_3d(st + 16384, &p.tq, 64, t, bh, &sm->full[s]);
+                tma_load_3d(st + 24576, &p.tk, 64, t, bh, &sm->full[s]);
+                tma_load_3d(st + 32768, &p.tv, vx, t, bh, &sm->full[s]);
+                issued[s] = u + 1;
+                // the chunk three ahead of this one into L2 (the slices of a head share it)
+                const int tp = t + kStages * kC;
+                if (tp < te) {
+                    tma_prefetch_l2_3d(&p.tq, 0, tp, bh);
+                    tma_prefetch_l2_3d(&p.tq, 64, tp, bh);
+                    tma_prefetch_l2_3d(&p.tk, 0, tp, bh);
+                    tma_prefetch_l2_3d(&p.tk, 64, tp, bh);
+                    tma_prefetch_l2_3d(&p.tv, vx, tp, bh);
+                }
+            }
+            for (int s = 0; s < kStages; ++s)
+                if (issued[s] > 0) drain_wait(&sm->full[s], (issued[s] - 1) & 1);
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ gates
+        // lane l takes tokens 2l, 2l + 1 of the chunk
+        for (int c = 0; c < nch; ++c) {
+            const int s = c % kStages, u = c / kStages;
+            if (u >= 1 && !mbar_wait(&sm->empty[s], (u - 1) & 1, abort, p.err)) break;
+            const int t0 = tb + kC * c;
+            const int L = min(kC, te - t0);
+            float a0 = 1.f, a1 = 1.f, b0 = 0.f, b1 = 0.f;
+            const int i0 = 2 * lane, i1 = 2 * lane + 1;
+            const size_t base = (size_t)bh * p.T + t0;
+            if (i0 < L) {
+                if (p.gate) a0 = p.gate[base + i0];
+                b0 = p.beta[base + i0];
+            }
+            if (i1 < L) {
+                if (p.gate) a1 = p.gate[base + i1];
+                b1 = p.beta[base + i1];
+            }
+            const float g0 = (i0 < L) ? lg2(fmaxf(a0, FLT_MIN)) : 0.f;
+            const float g1 = (i1 < L) ? lg2(fmaxf(a1, FLT_MIN)) : 0.f;
+            float x = g0 + g1;   // inclusive scan of the pair sums over the lanes
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float n = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += n;
+            }
+            const float l1 = x, l0 = x - g1;    // prefixes at tokens 2l + 1 and 2l
+            // lam at the first token of the 16-token block (lane 8 floor(l / 8), token 0)
+            const float lb = __shfl_sync(0xffffffffu, l0, lane & ~7);
+            Gates *G = &sm->gt[s];
+            reinterpret_cast<float2 *>(G->lam)[lane] = make_float2(l0, l1);
+            reinterpret_cast<float2 *>(G->bet)[lane] = make_float2(b0, b1);
+            reinterpret_cast<float2 *>(G->bg)[lane] = make_float2(b0 * ex2(l0), b1 * ex2(l1));
+            reinterpret_cast<float2 *>(G->cf)[lane] = make_float2(ex2(lb - l0), ex2(lb - l1));
+            const bool slow = __any_sync(0xffffffffu, lb - l1 > kFastSpan);
+            if (lane == 0) {
+                G->len = L;
+                G->slow = slow ? 1 : 0;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->full[s]);
+        }
+    } else if (warp >= 4 && warp < 12) {
+        // ------------------------------------------------------------ prep warps 4-11
+        const int pe = threadIdx.x - 128;           // 0..255
+        const int pq = warp & 3;                    // tensor-memory lane quarter
+        const int ph = (warp - 4) >> 2;             // column half of G
+        const int prow = 32 * pq + lane;
+        const uint32_t tl = tm + ((uint32_t)(32 * pq) << 16);
+        float *Lm = reinterpret_cast<float *>(smem_raw + kLm);
+        float *Tm = reinterpret_cast<float *>(smem_raw + kTm);
+        float *Zs = reinterpret_cast<float *>(smem_raw + kZs);
+        // G(c) = [Q; K] K^T once chunk c is loaded (elected thread; the caller made sure G(c-1)
+        // was read)
+        auto issue_g = [&](int c) {
+            const int s = c % kStages;
+            if (!mbar_wait(&sm->full[s], (c / kStages) & 1, abort, p.err)) return;
+            tc_fence_after();
+            const uint32_t st = sb + s * kStage;
+            mma_chain<8, true, true>(tm + kColG, dk(st), dk(st + 8192), id_g, false);
+            mma_commit(&sm->g_done);
+        };
+        if (pe == 0) issue_g(0);
+        for (int c = 0; c < nch; ++c) {
+            const int s = c % kStages;
+            const Gates *G = &sm->gt[s];
+            // chunk c loaded and its gates ready; G(c) formed; the A buffer of this parity
+            // free once A E(c - 2) is done
+            if (pe == 0) {
+                mbar_wait(&sm->full[s], (c / kStages) & 1, abort, p.err);
+                mbar_wait(&sm->g_done, c & 1, abort, p.err);
+                if (c >= 2) mbar_wait(&sm->ae_done[c & 1], ((c >> 1) - 1) & 1, abort, p.err);
+            }
+            if (named_sync_any(kBarPrep, kPrepT, *abort != 0)) break;
+            tc_fence_after();
+            {
+                // rows 0-63 of G: Q K^T -> A tile (j <= t); rows 64-127: K K^T -> Lm (j < t);
+                // columns j in [32 ph, 32 ph + 32).  The pair decay 2^(lam_t - lam_j) is the
+                // row factor 2^(lam_t - lam_{j0}) of the 16-column block j0 times the column
+                // factor cf_j, or (slow chunks) one exponential per element.
+                const bool qrows = pq < 2;
+                const int t = qrows ? prow : prow - 64;
+                const float lt = G->lam[t], bt = qrows ? 1.f : G->bet[t];
+                const bool empty = (pq & 1) == 0 && ph == 1;   // rows 0-31 x columns 32-63
+                float v[32];
+                if (!empty) tmem_ld32(tl + kColG + 32 * ph, v);
+                if (G->slow) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int jj = 32 * ph + j;
+                        const bool keep = !empty && (qrows ? jj <= t : jj < t);
+                        v[j] = keep ? v[j] * bt * ex2(lt - G->lam[jj]) : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int bb = 0; bb < 2; ++bb) {
+                        const int j0 = 32 * ph + 16 * bb;
+                        const float rf = (j0 <= t) ? bt * ex2(lt - G->lam[j0]) : 0.f;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 c4 = *reinterpret_cast<const float4 *>(G->cf + j0 + 4 * q);
+                            const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const int jj = j0 + 4 * q + k, e = 16 * bb + 4 * q + k;
+                                const bool keep = !empty && (qrows ? jj <= t : jj < t);
+                                v[e] = keep ? v[e] * (rf * cc[k]) : 0.f;
+                            }
+                        }
+                    }
+                }
+                if (qrows) {
+                    const uint32_t abuf = sb + ((c & 1) ? kA1 : kA0);
+                    st_row_bf16x16(abuf, t, 4 * ph, v);
+                    st_row_bf16x16(abuf, t, 4 * ph + 2, v + 16);
+                } else {
+                    float4 *lr = reinterpret_cast<float4 *>(Lm + t * kTStride + 32 * ph);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) lr[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            named_sync(kBarPrep, kPrepT);
+            // G is read: the next chunk's G may start
+            if (pe == 0 && c + 1 < nch) issue_g(c + 1);
+            // T = (I + Lm)^-1 (lower triangle)
+            invert_unit_lower_rec<kBarPrep, kPrepT>(Lm, Tm, Zs, pe);
+            // T diag(b), T diag(b g) as bf16 operands once W, U of chunk c - 1 are done
+            if (c >= 1 && pe == 0) mbar_wait(&sm->wu_done, (c - 1) & 1, abort, p.err);
+            if (named_sync_any(kBarPrep, kPrepT, *abort != 0)) break;
+            {
+                const int t = pe >> 2, j0 = 16 * (pe & 3);
+                float v1[16], v2[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 tv = *reinterpret_cast<const float4 *>(Tm + t * kTStride + j0 + 4 * q);
+                    const float4 b4 = *reinterpret_cast<const float4 *>(G->bet + j0 + 4 * q);
+                    const float4 g4 = *reinterpret_cast<const float4 *>(G->bg + j0 + 4 * q);
+                    const float tt[4] = {tv.x, tv.y, tv.z, tv.w}, bb[4] = {b4.x, b4.y, b4.z, b4.w},
+                                gg[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float tj = (j0 + 4 * q + k <= t) ? tt[k] : 0.f;
+                        v1[4 * q + k] = tj * bb[k];
+                        v2[4 * q + k] = tj * gg[k];
+                    }
+                }
+                st_row_bf16x16(sb + kTb, t, j0 >> 3, v1);
+                st_row_bf16x16(sb + kTbg, t, j0 >> 3, v2);
+            }
+            fence_async_smem();
+            named_sync(kBarPrep, kPrepT);
+            if (pe == 0) {
+                // W = T diag(b g) K into rows 64-127;  U = T diag(b) V (the V half) likewise,
+                // once the chain has read W(c - 1) and U(c - 1)
+                bool ok = true;
+                if (c >= 1) {
+                    ok = mbar_wait(&sm->w_free, (c - 1) & 1, abort, p.err) &&
+                         mbar_wait(&sm->u_free, (c - 1) & 1, abort, p.err);
+                }
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t st = sb + s * kStage;
+                    mma_chain<4, true, false>(tm + kColW, dk(sb + kTbg - 8192), dmn(st + 8192, 16384),
+                                              id_w, false);
+                    mma_chain<4, true, false>(tm + kColU, dk(sb + kTb - 8192), dmn(st + 32768, 8192),
+                                              id_u, false);
+                    mma_commit(&sm->wu_done);
+                }
+            }
+        }
+        // nothing this group issued may still write tensor memory when it is freed
+        if (pe == 0) {
+            mma_commit(&sm->g_done);   // completes phase nch (the G products took 0 .. nch-1)
+            drain_wait(&sm->g_done, (uint32_t)nch & 1);
+        }
+    } else if (warp >= 12) {
+        // ------------------------------------------------------------ chain warps 12-15
+        const int ce = threadIdx.x - 384;           // 0..127
+        const int cq = warp & 3;                    // lane quarter
+        const int row = 32 * cq + lane;             // d_k row of S^T; token of P / W / E
+        const uint32_t tl = tm + ((uint32_t)(32 * cq) << 16);
+        float Sr[kDV];   // S^T[row][32 vs + j]
+        {
+            const float *src = p.s_in ? p.s_in + slot + (size_t)(kDV * vs) * kD + row : nullptr;
+#pragma unroll
+            for (int j = 0; j < kDV; ++j) Sr[j] = src ? src[(size_t)j * kD] : 0.f;
+            st_row32_mn(sb + kS, row, Sr);
+            fence_async_smem();
+        }
+        // P(c) = [diag(g) Q; W] S^T  (rows 0-63: inter-chunk outputs, 64-127: W S^T), issued
+        // by the elected thread once the S^T tile and the A operand are published
+        auto issue_p = [&](int c) {
+            tc_fence_after();
+            mma_chain_ts<8>(tm + kColP + kDV * (c & 1), tm + kColQW + 64 * (c & 1), dmn(sb + kS, 8192),
+                            id_p, false);
+            mma_commit(&sm->p_done);
+        };
+        // [diag(g) Q; W] of chunk c into tensor memory as the A operand of P
+        auto qw_step = [&](int c) -> bool {
+            const int s = c % kStages;
+            // the Q tile and the gates are read here: every thread observes the stage
+            mbar_wait(&sm->full[s], (c / kStages) & 1, abort, p.err);
+            if (!group_wait(&sm->wu_done, c & 1, ce == 0, kBarChain, kChainT, abort, p.err)) return false;
+            tc_fence_after();
+            const uint32_t dst = tl + kColQW + 64 * (c & 1);
+            if (cq < 2) {
+                const int t = row;
+                const float gt = ex2(sm->gt[s].lam[t]);
+                const uint32_t st = sb + s * kStage;
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint4 x = scale_bf16x8(lds128(st + 16384 * h + sw128_off(t, ch)), gt);
+                        w[4 * ch + 0] = x.x;
+                        w[4 * ch + 1] = x.y;
+                        w[4 * ch + 2] = x.z;
+                        w[4 * ch + 3] = x.w;
+                    }
+                    tmem_st32(dst + 32 * h, w);
+                }
+            } else {
+#pragma unroll 1
+                for (int h = 0; h < 4; ++h) {
+                    float f[32];
+                    tmem_ld32(tl + kColW + 32 * h, f);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(f[2 * j], f[2 * j + 1]);
+                    tmem_st16u(dst + 16 * h, w);
+                }
+            }
+            tc_fence_before();
+            named_sync(kBarChain, kChainT);
+            if (ce == 0) mbar_arrive(&sm->w_free);
+            return true;
+        };
+        bool ok = qw_step(0);
+        if (ok && ce == 0) issue_p(0);
+        // Iteration c: E of chunk c (lanes 64-127) and the outputs of chunk c - 1 (lanes 0-63);
+        // the A operand of chunk c + 1 while dS(c) is formed; the state update and P(c + 1).
+        // Iteration nch only writes the last outputs.
+        for (int c = 0; c <= nch && ok; ++c) {
+            const int s = c % kStages;
+            const uint32_t par = c & 1;
+            const bool cur = c < nch;
+            // the stage's gates were observed in qw_step(c); read before the barrier below,
+            // which precedes the stage's release (dS(c) is issued after it)
+            const float gL = cur ? ex2(sm->gt[s].lam[kC - 1]) : 1.f;
+            if (cur) {
+                if (!group_wait(&sm->p_done, par, ce == 0, kBarChain, kChainT, abort, p.err)) break;
+                tc_fence_after();
+            }
+            if (cq >= 2) {
+                if (cur) {
+                    // E = U - W S^T; the E tiles are free once A E(c - 1) is done
+                    if (c >= 1 && !group_wait(&sm->ae_done[(c - 1) & 1], ((c - 1) >> 1) & 1, row == 64,
+                                              kBarChainE, 64, abort, p.err))
+                        break;
+                    const int t = row - 64;
+                    const int L = sm->gt[s].len;
+                    const float *lam = sm->gt[s].lam;
+                    float y[32], uu[32];
+                    tmem_ld32(tl + kColP + kDV * par, y);
+                    tmem_ld32(tl + kColU + kDV * (vs & 1), uu);
+                    const float dec = (t < L) ? ex2(lam[kC - 1] - lam[t]) : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float e = (t < L) ? uu[j] - y[j] : 0.f;
+                        y[j] = e;
+                        uu[j] = e * dec;
+                    }
+                    st_row32_mn(sb + kE, t, y);
+                    st_row32_mn(sb + kEp, t, uu);
+                    fence_async_smem();
+                    tc_fence_before();
+                    named_sync(kBarChainE, 64);
+                    if (row == 64) {
+                        mbar_arrive(&sm->u_free);
+                        tc_fence_after();
+                        const uint32_t st = sb + s * kStage;
+                        // dS^T = K^T E'   (E' = diag(dec) E)
+                        mma_chain<4, false, false>(tm + kColDS, dmn(st + 8192, 16384), dmn(sb + kEp, 8192),
+                                                   id_ds, false);
+                        mma_commit(&sm->ds_done);
+                        mma_commit(&sm->empty[s]);
+                        // rows 0-63 of P += A E  (the 64 rows after the A tile multiply into
+                        // rows 64-127, already read)
+                        mma_chain<4, true, false>(tm + kColP + kDV * par, dk(sb + (par ? kA1 : kA0)),
+                                                  dmn(sb + kE, 8192), id_ae, true);
+                        mma_commit(&sm->ae_done[par]);
+                    }
+                }
+            } else if (c >= 1) {
+                // outputs of chunk c - 1: rows 0-63 of P (lanes 0-63), the slice's 32 columns
+                if (!group_wait(&sm->ae_done[(c - 1) & 1], ((c - 1) >> 1) & 1, row == 0, kBarChainO, 64,
+                                abort, p.err))
+                    break;
+                tc_fence_after();
+                const int t = row;
+                const int t0 = tb + kC * (c - 1);
+                const int L = min(kC, te - t0);
+                float v[32];
+                tmem_ld32(tl + kColP + kDV * ((c - 1) & 1), v);
+                if (t < L) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)bh * p.T + t0 + t) * kD + kDV * vs);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 w;
+                        w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+                        w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+                        w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+                        w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+                        dst[q] = w;
+                    }
+                }
+            }
+            if (c + 1 < nch && !qw_step(c + 1)) break;
+            if (!cur) continue;
+            // ---- state: S^T <- g_{L-1} S^T + dS^T; bf16 copy for the next chunk
+            if (!group_wait(&sm->ds_done, par, ce == 0, kBarChain, kChainT, abort, p.err)) break;
+            tc_fence_after();
+            const bool last = (c + 1 == nch);
+            {
+                float d[32];
+                tmem_ld32(tl + kColDS, d);
+#pragma unroll
+                for (int j = 0; j < kDV; ++j) Sr[j] = fmaf(gL, Sr[j], d[j]);
+            }
+            if (last) {
+                if (p.s_out) {
+                    float *dst = p.s_out + slot + (size_t)(kDV * vs) * kD + row;
+#pragma unroll
+                    for (int j = 0; j < kDV; ++j) dst[(size_t)j * kD] = Sr[j];
+                }
+            } else {
+                st_row32_mn(sb + kS, row, Sr);
+                fence_async_smem();
+            }
+            tc_fence_before();
+            named_sync(kBarChain, kChainT);
+            if (ce == 0 && !last) issue_p(c + 1);
+        }
+        // nothing this group issued may still write tensor memory when it is freed
+        if (ce == 0) {
+            mma_commit(&sm->p_done);
+            drain_wait(&sm->p_done, (uint32_t)nch & 1);
+        }
+        if (row == 64) {
+            mma_commit(&sm->ds_done);
+            drain_wait(&sm->ds_done, (uint32_t)nch & 1);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tm, kTmemCols);
+    }
+}
+
+}  // namespace
+
+bool prefill_gdn_selected(int mode, int BH, bool packed) {
+    // Dense calls whose d_v slices fill 64 to 148 SMs (one wave): there the single pass is as
+    // fast as the segmented kernels and moves the algorithmic bytes once (no workspace, no
+    // second pass over k and v).  Fewer heads take the segmented kernels (which split long
+    // sequences over more SMs), more heads one CTA per head; packed sequences take the
+    // per-sequence kernel.
+    return mode == LA_MODE_GATED_DELTA && !packed && BH * kNS >= 64 && BH * kNS <= 148;
+}
+
+cudaError_t launch_prefill_gdn(const PrefillArgs &a) {
+    const int BH = a.cu ? a.H : a.B * a.H;
+    GdnParams p;
+    memset(&p, 0, sizeof(p));
+    const uint64_t row_pitch = kD * 2, head_pitch = (uint64_t)a.T * kD * 2;
+    if (!make_tmap_3d(&p.tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, a.T, BH, row_pitch,
+                      head_pitch, 64, kC, true) ||
+        !make_tmap_3d(&p.tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, a.T, BH, row_pitch,
+                      head_pitch, 64, kC, true) ||
+        !make_tmap_3d(&p.tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, a.T, BH, row_pitch,
+                      head_pitch, 64, kC, true))
+        return cudaErrorInvalidValue;
+    p.gate = a.gate;
+    p.beta = a.beta;
+    p.o = static_cast<__nv_bfloat16 *>(a.o);
+    p.s_in = a.init_state ? a.state : nullptr;
+    p.s_out = a.state;
+    p.seq_stride = a.cu ? (long long)a.H * kD * kD : 0;
+    p.cu = a.cu;
+    p.T = a.T;
+    p.BH = BH;
+    p.err = device_error_word();
+    const int units = a.cu ? a.nseq * a.H : BH;
+    cudaError_t e = cudaFuncSetAttribute(gdn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kBytes);
+    if (e != cudaSuccess) return e;
+    timer_begin(a.stream);
+    gdn_prefill_kernel<<<units * kNS, kThreads, kBytes, a.stream>>>(p);
+    timer_end(a.stream);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace la

@@ -60,6 +60,7 @@
 #include "la_internal.cuh"
 #include "ptx.cuh"
 #include "tmap.cuh"
+#include "tc_util.cuh"
 
 #include <algorithm>
 #include <cfloat>
@@ -68,6 +69,7 @@ namespace la {
 namespace {
 
 using namespace ptx;
+using namespace tc;
 
 constexpr int kC = 64;         // chunk
 constexpr int kD = 128;        // d_k = d_v
@@ -248,87 +250,8 @@ struct Lay {
     static constexpr uint32_t kBytes = MODE == 3 ? kKda + sizeof(SmallKda) : kSmall + sizeof(Small);
 };
 static_assert(Lay<3>::kBytes <= 227 * 1024, "shared memory per CTA");
-constexpr uint32_t kLmStride = 65;
 
 __device__ __forceinline__ void epi_sync() { named_sync(1, kEpi); }
-__device__ __forceinline__ uint64_t dk(uint32_t addr) { return sdesc_sw128(addr, 16, 1024); }
-__device__ __forceinline__ uint64_t dmn(uint32_t addr, uint32_t lbo) {
-    return sdesc_sw128(addr, lbo, 1024);
-}
-
-// D (+)= A B over NK steps of K = 16, issued back to back.  The operand descriptors are
-// built once; each step adds its offset to the start-address field (16-byte units), a
-// compile-time constant once the loop is unrolled.  A K-major 128B-swizzled operand
-// advances 32 bytes per step inside a 64-column half and jumps to the next half
-// (KHALF bytes further) every four steps; an MN-major one advances 8 K rows = 2048 bytes.
-template <int NK, bool A_KMAJ, bool B_KMAJ, uint32_t A_KHALF = 16384, uint32_t B_KHALF = 16384>
-__device__ __forceinline__ void mma_chain(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, bool accumulate_first) {
-#pragma unroll
-    for (int ks = 0; ks < NK; ++ks) {
-        const uint64_t ao = A_KMAJ ? (((ks >> 2) * A_KHALF + (ks & 3) * 32) >> 4) : (uint64_t)(ks * 128);
-        const uint64_t bo = B_KMAJ ? (((ks >> 2) * B_KHALF + (ks & 3) * 32) >> 4) : (uint64_t)(ks * 128);
-        mma_bf16_ss(d_tmem, a_desc + ao, b_desc + bo, idesc, accumulate_first || ks > 0);
-    }
-}
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ float lg2(float x) {
-    float y;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// Bounded wait that ignores the abort flag (used to drain in-flight work on exit).
-__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
-        if (mbar_try_wait(bar, parity)) return;
-}
-
-// Write 16 fp32 values as bf16 = two 16-byte chunks (ch, ch+1) of row `row` of the
-// 128B-swizzled tile at shared address `tile`.
-__device__ __forceinline__ void st_row_bf16x16(uint32_t tile, uint32_t row, uint32_t ch,
-                                               const float *v) {
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        uint4 w;
-        w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-        w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-        w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-        w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-        sts128(tile + sw128_off(row, ch + q), w);
-    }
-}
-// Multiply the 8 bf16 values of a 16-byte chunk by s.
-__device__ __forceinline__ uint4 scale_bf16x8(uint4 w, float s) {
-    uint32_t *wd = reinterpret_cast<uint32_t *>(&w);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float2 f = unpack_bf16x2(wd[q]);
-        wd[q] = pack_bf16x2(f.x * s, f.y * s);
-    }
-    return w;
-}
-
-__device__ __forceinline__ void prefetch_l2(const void *ptr) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
-}
-
-// Multiply the 8 bf16 values of a 16-byte chunk by 8 factors (one per channel).
-__device__ __forceinline__ uint4 scale_bf16x8v(uint4 w, const float4 f0, const float4 f1) {
-    uint32_t *wd = reinterpret_cast<uint32_t *>(&w);
-    const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float2 v = unpack_bf16x2(wd[q]);
-        wd[q] = pack_bf16x2(v.x * f[2 * q], v.y * f[2 * q + 1]);
-    }
-    return w;
-}
-
 // Raw gate a_t and beta_t of token `e` of chunk c (64 threads, e < 64), fetched a chunk
 // ahead of use so that the global-load latency overlaps the previous chunk's epilogue.
 struct GateRaw {
@@ -384,98 +307,6 @@ __device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
     return r;
 }
 
-// ---- warp-level tf32 products for the 16x16 blocks of the triangular inverse
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-// acc (16x16 fp32, two m16n8 fragments) += A (16x16) * B (16x16); A, B fp32 in shared
-// memory with row strides lda, ldb (elements).
-__device__ __forceinline__ void mma16x16x16_tf32(float (&acc)[2][4], const float *A, int lda,
-                                                 const float *B, int ldb, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-        const uint32_t a0 = to_tf32(A[g * lda + 8 * kk + t]);
-        const uint32_t a1 = to_tf32(A[(g + 8) * lda + 8 * kk + t]);
-        const uint32_t a2 = to_tf32(A[g * lda + 8 * kk + t + 4]);
-        const uint32_t a3 = to_tf32(A[(g + 8) * lda + 8 * kk + t + 4]);
-#pragma unroll
-        for (int nh = 0; nh < 2; ++nh) {
-            const uint32_t b0 = to_tf32(B[(8 * kk + t) * ldb + 8 * nh + g]);
-            const uint32_t b1 = to_tf32(B[(8 * kk + t + 4) * ldb + 8 * nh + g]);
-            asm volatile(
-                "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-                "{%8,%9}, {%0,%1,%2,%3};"
-                : "+f"(acc[nh][0]), "+f"(acc[nh][1]), "+f"(acc[nh][2]), "+f"(acc[nh][3])
-                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-        }
-    }
-}
-// C (16x16, row stride ldc) = s * acc
-__device__ __forceinline__ void store16_tile(const float (&acc)[2][4], float *C, int ldc, int lane,
-                                             float s) {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int nh = 0; nh < 2; ++nh) {
-        C[g * ldc + 8 * nh + 2 * t] = s * acc[nh][0];
-        C[g * ldc + 8 * nh + 2 * t + 1] = s * acc[nh][1];
-        C[(g + 8) * ldc + 8 * nh + 2 * t] = s * acc[nh][2];
-        C[(g + 8) * ldc + 8 * nh + 2 * t + 1] = s * acc[nh][3];
-    }
-}
-
-// 64x64 unit lower-triangular inverse T = (I + Lm)^-1 by 16x16 blocks (256 threads).
-__device__ void invert_unit_lower(const float *Lm, float *Tm, float *Zs, int e) {
-    constexpr int S = kLmStride;
-    if (e < 64) {
-        const int b = e >> 4, c = e & 15;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
-#pragma unroll
-        for (int r = 1; r < 16; ++r) {
-            float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-            for (int j = 0; j < r; j += 2) {
-                s0 = fmaf(Lm[(16 * b + r) * S + 16 * b + j], x[j], s0);
-                if (j + 1 < r) s1 = fmaf(Lm[(16 * b + r) * S + 16 * b + j + 1], x[j + 1], s1);
-            }
-            if (r > c) x[r] = -(s0 + s1);
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) Tm[(16 * b + r) * S + 16 * b + c] = x[r];
-    } else {
-        for (int idx = e - 64; idx < 6 * 256; idx += kEpi - 64) {
-            const int blk = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
-            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-            const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            Tm[(16 * bi + r) * S + 16 * bj + cc] = 0.f;
-        }
-    }
-    epi_sync();
-    // Off-diagonal blocks, by distance d = i - j:  T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj.
-    // Each block is one warp's job on the legacy warp-level tensor-core path (tf32
-    // m16n8k8, fp32 accumulate): the products are 16x16x16, too small for tcgen05.
-    const int w = e >> 5, lane = e & 31;
-    for (int d = 1; d < 4; ++d) {
-        if (w < 4 - d) {
-            const int bi = w + d, bj = w;
-            float acc[2][4] = {};
-            for (int k = bj; k < bi; ++k)
-                mma16x16x16_tf32(acc, Lm + (16 * bi) * S + 16 * k, S, Tm + (16 * k) * S + 16 * bj, S,
-                                 lane);
-            float *Z = Zs + w * 272;
-            store16_tile(acc, Z, 17, lane, 1.f);
-            __syncwarp();
-            float acc2[2][4] = {};
-            mma16x16x16_tf32(acc2, Tm + (16 * bi) * S + 16 * bi, S, Z, 17, lane);
-            store16_tile(acc2, Tm + (16 * bi) * S + 16 * bj, S, lane, -1.f);
-        }
-        epi_sync();
-    }
-}
 
 template <int MODE, int KIND>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
@@ -876,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
             {
                 // ---- T = (I + Lm)^-1;  T diag(b), T diag(b g) as bf16 MMA operands
-                invert_unit_lower(Lm, Tm, Zs, e);
+                invert_unit_lower<1, kEpi>(Lm, Tm, Zs, e);
                 if (e < 128) {
                     const int t = e >> 1, hh = e & 1;
                     for (int g = 0; g < 2; ++g) {
@@ -2245,6 +2076,7 @@ bool prefill_tc_supports(int mode, int dtype, int dk, int dv, int chunk) {
 
 size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T, bool minimal) {
     const int BH = B * H;
+    if (prefill_gdn_selected(mode, BH, false)) return 0;
     Plan pl = plan_for(mode, BH, T);
     if (minimal && mode >= 2) pl.sub = 1;   // the smallest segmented plan
     return sizeof(float) * workspace_floats(mode, BH, pl);
@@ -2272,6 +2104,7 @@ cudaError_t run_packed(const PrefillArgs &a, const TcParams &base) {
 
 cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes) {
     const int BH = a.B * a.H;
+    if (prefill_gdn_selected(a.mode, BH, a.cu != nullptr)) return launch_prefill_gdn(a);
     const Plan pl = plan_for(a.mode, BH, a.T, workspace ? workspace_bytes : 0);
     TcParams p;
     memset(&p, 0, sizeof(p));
