@@ -31,11 +31,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 import workloads as W  # noqa: E402
 
-DEFAULT_WORKLOAD = "elu1_bf16_b4h16t4096"
+DEFAULT_WORKLOAD = "gdn_bf16_b2h16t32768"
 METRIC = "prefill tokens/s + % tensor roofline; decode tokens/s + HBM GB/s (1×B200)"
 L2_FLUSH_BYTES = 256 << 20          # > 126 MB L2
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -576,6 +577,29 @@ def roofline(case, kernel_ms, step_ms, peaks, peak_src, prof):
     }
 
 
+def _sig(x, n=3):
+    """x rounded to n significant digits (JSON-compact)."""
+    if x is None or not math.isfinite(x) or x == 0:
+        return x
+    return float(f"{x:.{n}g}")
+
+
+def compact(res, roof, cpu):
+    """One short entry per extra workload (the driver keeps the end of the line): ms per
+    step, tokens/s, the step's roofline fraction (algorithmic bytes or flops over the device
+    time of all its launches), its tensor fraction, DRAM traffic per step over the
+    algorithmic bytes (ncu, null when stale), the oracle's tokens/s on the host cores and
+    the end-to-end tokens/s through host buffers."""
+    tr = roof["call"]["traffic"]
+    t_call = sum(roof["call"]["kernel_ms"]) * 1e-3 if roof["call"]["kernel_ms"] else None
+    tc = res["algorithmic_flops_per_step"] / t_call / 1e12 / load_peaks()[0]["bf16_tflops"] if t_call else None
+    return {"ms": _sig(res["ms_per_step"]), "tok_s": _sig(res["tokens_per_s"]),
+            "frac": _sig(roof["call"]["frac"]), "tc": _sig(tc),
+            "tx": _sig(tr / roof["algorithmic_bytes"]) if tr else None,
+            "cpu": _sig(cpu["value"]) if cpu and cpu.get("value") else None,
+            "e2e": _sig(res["e2e"]["value"]) if res.get("e2e") else None}
+
+
 def measure(la, name, args, dist, device, rank, world, flush, with_e2e, sampler=None):
     if name in W.CONV_CONFIGS:
         case = ConvCase(la, W.CONV_CONFIGS[name], device, rank)
@@ -628,11 +652,69 @@ def measure(la, name, args, dist, device, rank, world, flush, with_e2e, sampler=
 # the oracle on host cores
 # ----------------------------------------------------------------------------------
 
+def _timed_growing(run, n0, n_max, budget_s):
+    """Call run(n) for n = n0, 2 n0, ... until one call takes half the budget or n_max is
+    reached; returns (n, seconds of the last call)."""
+    n = min(n0, n_max)
+    while True:
+        t0 = time.perf_counter()
+        run(n)
+        el = time.perf_counter() - t0
+        if el * 2 > budget_s or n >= n_max:
+            return n, el
+        n = min(n_max, n * 2)
+
+
+def oracle_sample_other(name, budget_s):
+    """The oracle timed on a bounded sample of a convolution, packed-sequence or backward
+    workload (tokens/s in the workload's token unit)."""
+    import oracle
+    f = lambda t: None if t is None else t.to(torch.float64).numpy()
+    if name in W.CONV_CONFIGS:
+        from oracle import conv as oc
+        cw = W.CONV_CONFIGS[name]
+        x, wt, _ = W.conv_inputs(1, min(cw.T, 4096), cw.H * cw.dk, cw.width, cw.dtype, seed=cw.seed,
+                                 window=False)
+        xs, ws_ = f(x), f(wt)
+        T, el = _timed_growing(lambda n: oc.short_conv(xs[:, :n], ws_, H=cw.H, silu=cw.silu,
+                                                       l2norm=cw.l2norm_qk), 256, xs.shape[1], budget_s)
+        # one token = the three projections q, k, v
+        return {"value": T / el / 3, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                "sample": f"1 x {T} tokens of one {cw.H}x{cw.dk} projection (fp64 numpy), /3"}
+    if name in W.VARLEN_CONFIGS:
+        vw = W.VARLEN_CONFIGS[name]
+        L = sorted(vw.lengths())[: max(2, vw.N // 8)]
+        inp = W.varlen_inputs(vw.base, L, device="cpu")
+        a = {k: f(inp[k]) for k in ("q", "k", "v", "gate", "beta")}
+        cu = inp["cu"].numpy()
+        t0 = time.perf_counter()
+        oracle.prefill_packed(vw.base.mode, a["q"], a["k"], a["v"], cu, a["gate"], a["beta"])
+        el = time.perf_counter() - t0
+        return {"value": sum(L) / el, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+                "sample": f"the {len(L)} shortest sequences ({sum(L)} tokens) x {vw.base.H} heads "
+                          f"(fp64 C, OpenMP)"}
+    if name in W.BACKWARD_CONFIGS:
+        from oracle import backward as ob
+        w = W.BACKWARD_CONFIGS[name]
+        inp = W.prefill_inputs(W.variant(w, B=1, H=min(w.H, 4), T=256), device="cpu")
+        a = {k: f(inp[k]) for k in ("q", "k", "v", "gate")}
+        do = np.random.default_rng(0).standard_normal(a["v"].shape)
+        T, el = _timed_growing(lambda n: ob.prefill_backward(w.mode, a["q"][:, :, :n], a["k"][:, :, :n],
+                                                            a["v"][:, :, :n], a["gate"][:, :, :n],
+                                                            do[:, :, :n]), 32, 256, budget_s)
+        hs = a["q"].shape[1]
+        return {"value": hs * T / el / w.H, "unit": "tokens/s", "cores": torch.get_num_threads(),
+                "kind": "oracle", "sample": f"{hs} heads x {T} tokens (fp64 PyTorch autograd on the CPU)"}
+    return None
+
+
 def oracle_sample(name, budget_s=10.0):
     """Time the fp64 oracle on a bounded sample of the workload.  Returns a dict with
     tokens/s (in the workload's token unit), the cores used and a description."""
     import numpy as np
     import oracle
+    if name not in W.CONFIGS:
+        return oracle_sample_other(name, budget_s)
     w = W.CONFIGS[name]
     threads = oracle.max_threads()
     gen_w = W.variant(w, B=1, H=min(w.H, max(1, threads)), T=min(w.T, 4096) if not w.decode else w.T)
@@ -662,7 +744,7 @@ def oracle_sample(name, budget_s=10.0):
     T = min(256, gen_w.T)
     el = 0.0
     while True:
-        sl = [None if a is None else a[:, :, :T] for a in args]
+        sl = [None if a is None else (a if a.ndim == 1 else a[:, :, :T]) for a in args]
         t0 = time.perf_counter()
         oracle.prefill(w.mode, *sl)
         el = time.perf_counter() - t0
@@ -773,14 +855,23 @@ def main():
     extras = {}
     do_extras = (world == 1) if args.extras < 0 else bool(args.extras)
     if do_extras:
-        for name in ("elu1_bf16_b4h16t4096", "gated_bf16_b8h16t8192", "gdn_bf16_b2h16t32768",
-                     "gdn_decode_n256h32", "kda_bf16_b2h16t32768", "kda_decode_n256h32",
-                     "conv_bf16_b2h16t32768", "gdn_varlen_bf16_n64h16", "retnet_bf16_b8h16t8192",
-                     "gated_bwd_bf16_b4h16t4096"):
+        peaks_x, src_x = load_peaks()
+        for name in ("elu1_f32_small", "elu1_bf16_b4h16t4096", "gated_bf16_b8h16t8192",
+                     "gdn_bf16_b2h16t32768", "gdn_decode_n256h32", "kda_bf16_b2h16t32768",
+                     "kda_decode_n256h32", "conv_bf16_b2h16t32768", "gdn_varlen_bf16_n64h16",
+                     "retnet_bf16_b8h16t8192", "gated_bwd_bf16_b4h16t4096"):
             if name == args.workload:
                 continue
-            r = measure(la, name, args, dist, device, rank, world, flush, False)
-            extras[name] = {k: v for k, v in r.items() if not k.startswith("_")}
+            r = measure(la, name, args, dist, device, rank, world, flush, True)
+            rf = roofline(r["_case"], r["kernel_ms"], statistics.mean(r["_ms"]), peaks_x, src_x,
+                          ncu_traffic(name))
+            cpu_x = None
+            if rank == 0 and world == 1:
+                try:
+                    cpu_x = oracle_sample(name, budget_s=1.5)
+                except Exception:
+                    cpu_x = None
+            extras[name] = compact(r, rf, cpu_x)
             del r
             torch.cuda.empty_cache()
 

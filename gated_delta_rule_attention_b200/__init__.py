@@ -185,15 +185,20 @@ def workspace_size(mode: int, dtype: torch.dtype, B: int, H: int, T: int, d_k: i
     return int(library().la_prefill_workspace_size(int(mode), dt, B, H, T, d_k, d_v, int(chunk)))
 
 
-def _workspace(device: torch.device, nbytes: int):
-    """A per-device scratch buffer (torch allocation), grown on demand and reused.
-    Calls on different streams of one device must pass their own workspace."""
+def _workspace(device: torch.device, nbytes: int, stream=None):
+    """A scratch buffer for calls on one stream of one device (torch allocation), grown on
+    demand and reused by later calls on that stream.  Calls on different streams never
+    share a buffer, and each is allocated while its stream is current, so the caching
+    allocator orders the reuse of a replaced buffer after that stream's work."""
     if nbytes <= 0:
         return None
-    buf = _workspaces.get(device)
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    key = (device.index, s.cuda_stream)
+    buf = _workspaces.get(key)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
-        _workspaces[device] = buf
+        with torch.cuda.stream(s):
+            buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _workspaces[key] = buf
     return buf
 
 
@@ -249,7 +254,7 @@ def prefill(q, k, v, *, mode: int, gate=None, beta=None, state=None, z=None, o=N
         o = torch.empty(B, H, T, dv, device=q.device, dtype=dt)
     _need(o, (B, H, T, dv), dt, "o")
     if isinstance(workspace, str):
-        ws = _workspace(q.device, workspace_size(mode, dt, B, H, T, dk, dv, chunk)) \
+        ws = _workspace(q.device, workspace_size(mode, dt, B, H, T, dk, dv, chunk), stream) \
             if workspace == "auto" else None
     else:
         ws = workspace
@@ -343,6 +348,8 @@ def prefill_backward(q, k, v, dO, *, mode: int, gate=None, state0=None, dstate=N
                if need_dstate0 else None)
     nbytes = int(library().la_backward_workspace_size(int(mode), B, H, T, dk_, dv_))
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    if stream is not None:
+        ws.record_stream(stream)   # freed on return: not reused before `stream`'s work is done
     st = library().la_prefill_backward(int(mode), dtype, B, H, T, dk_, dv_, _ptr(q), _ptr(k), _ptr(v),
                                        _ptr(gate), _ptr(state0), _ptr(dO), _ptr(dstate), _ptr(dq),
                                        _ptr(dk), _ptr(dv), _ptr(dgate), _ptr(dstate0), _ptr(ws),

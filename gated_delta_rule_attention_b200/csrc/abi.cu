@@ -7,7 +7,9 @@
 
 #include <atomic>
 #include <cstdint>
+#include <initializer_list>
 #include <mutex>
+#include <utility>
 
 namespace la {
 
@@ -70,6 +72,28 @@ bool overlap(const void *p, size_t n, const void *q, size_t m) {
     return p && q && n && m && a < b + m && b < a + n;
 }
 
+using Span = std::pair<const void *, size_t>;
+
+// True if the buffers a call writes (o, the state, z) share no byte with one another or with
+// any buffer it only reads (null spans are skipped).  The kernels read inputs while they
+// write outputs, so an overlap would be a race, not an in-place update.
+bool writes_disjoint(std::initializer_list<Span> writes, std::initializer_list<Span> reads) {
+    for (auto w = writes.begin(); w != writes.end(); ++w) {
+        for (auto u = w + 1; u != writes.end(); ++u)
+            if (overlap(w->first, w->second, u->first, u->second)) return false;
+        for (const Span &r : reads)
+            if (overlap(w->first, w->second, r.first, r.second)) return false;
+    }
+    return true;
+}
+
+// Bytes of a call's gate tensor: per token (a scalar, or d_k values in the per-channel mode)
+// or one value per head (the constant-decay mode).
+size_t gate_bytes(int mode, long long tokens_x_heads, int H, int d_k) {
+    if (mode == LA_MODE_RETNET) return sizeof(float) * (size_t)H;
+    return sizeof(float) * (size_t)tokens_x_heads * (mode == LA_MODE_KDA ? d_k : 1);
+}
+
 }  // namespace
 }  // namespace la
 
@@ -106,6 +130,17 @@ extern "C" la_status_t la_prefill(la_mode_t mode, la_dtype_t dtype, int B, int H
         return LA_ERR_INVALID_ARG;
     if (mode != LA_MODE_ELU1_NORM && gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
     if (delta_mode(mode) && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
+    {
+        const size_t es = dtype == LA_BF16 ? 2 : 4, th = (size_t)BH * T;
+        const bool z_used = mode == LA_MODE_ELU1_NORM;
+        if (!writes_disjoint({{o, th * d_v * es}, {state, sizeof(float) * BH * d_v * d_k},
+                              {z_used ? z : nullptr, sizeof(float) * BH * d_k}},
+                             {{q, th * d_k * es}, {k, th * d_k * es}, {v, th * d_v * es},
+                              {z_used ? nullptr : gate, gate_bytes(mode, (long long)th, H, d_k)},
+                              {delta_mode(mode) ? beta : nullptr, sizeof(float) * th},
+                              {workspace, workspace ? workspace_bytes : 0}}))
+            return LA_ERR_INVALID_ARG;
+    }
 
     PrefillArgs a;
     a.mode = internal_mode(mode);
@@ -154,6 +189,19 @@ extern "C" la_status_t la_prefill_varlen(la_mode_t mode, la_dtype_t dtype, int N
             return LA_ERR_INVALID_ARG;
         if (mode != LA_MODE_ELU1_NORM && gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
         if (delta_mode(mode) && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
+    }
+    {
+        const size_t es = dtype == LA_BF16 ? 2 : 4, th = (size_t)H * T;
+        const bool z_used = mode == LA_MODE_ELU1_NORM;
+        if (!writes_disjoint({{T > 0 ? o : nullptr, th * d_v * es},
+                              {state, sizeof(float) * N * H * d_v * d_k},
+                              {z_used ? z : nullptr, sizeof(float) * N * H * d_k}},
+                             {{cu_seqlens, sizeof(int) * (N + 1)},
+                              {T > 0 ? q : nullptr, th * d_k * es}, {T > 0 ? k : nullptr, th * d_k * es},
+                              {T > 0 ? v : nullptr, th * d_v * es},
+                              {z_used || T == 0 ? nullptr : gate, gate_bytes(mode, (long long)th, H, d_k)},
+                              {delta_mode(mode) && T > 0 ? beta : nullptr, sizeof(float) * th}}))
+            return LA_ERR_INVALID_ARG;
     }
     PrefillArgs a;
     a.mode = internal_mode(mode);
@@ -213,6 +261,17 @@ extern "C" la_status_t la_decode_step(la_mode_t mode, la_dtype_t dtype, int N, i
     if (mode == LA_MODE_ELU1_NORM && !tensor_ok(z, 16)) return LA_ERR_INVALID_ARG;
     if (mode != LA_MODE_ELU1_NORM && gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
     if (delta_mode(mode) && !tensor_ok(beta, 4)) return LA_ERR_INVALID_ARG;
+    {
+        const size_t es = dtype == LA_BF16 ? 2 : 4;
+        const bool z_used = mode == LA_MODE_ELU1_NORM;
+        if (!writes_disjoint({{o, (size_t)NH * d_v * es}, {state, sizeof(float) * NH * d_v * d_k},
+                              {z_used ? z : nullptr, sizeof(float) * NH * d_k}},
+                             {{q, (size_t)NH * d_k * es}, {k, (size_t)NH * d_k * es},
+                              {v, (size_t)NH * d_v * es},
+                              {z_used ? nullptr : gate, gate_bytes(mode, NH, H, d_k)},
+                              {delta_mode(mode) ? beta : nullptr, sizeof(float) * NH}}))
+            return LA_ERR_INVALID_ARG;
+    }
     DecodeArgs a;
     a.mode = internal_mode(mode);
     a.gate_heads = (mode == LA_MODE_RETNET) ? H : 0;

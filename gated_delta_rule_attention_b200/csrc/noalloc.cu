@@ -53,19 +53,13 @@ extern "C" la_status_t la_prefill_noalloc(la_mode_t mode, la_dtype_t dtype, int 
                                           const void *v, const float *gate, const float *beta,
                                           float *state, float *z, void *o, int chunk,
                                           unsigned flags, void *stream) {
-    // refuse only when even the smallest segmented plan needs more than the static
-    // buffer; the launcher then takes the fastest plan that fits in it
-    size_t need = la_prefill_workspace_size(mode, dtype, B, H, T, d_k, d_v, chunk);
-    if (need > 0) {
-        const int m = (mode == LA_MODE_RETNET) ? (int)LA_MODE_GATED : (int)mode;
-        need = la::prefill_tc_workspace_bytes(m, B, H, T, true);
-    }
-    if (need > la::kStaticWorkspaceBytes) return LA_ERR_UNSUPPORTED;
+    // The launcher runs the fastest segment plan whose workspace fits in the static array,
+    // or, when none fits, the single pass that needs none: every problem la_prefill accepts
+    // runs here too.  Should the array's address be unavailable, the call runs without it
+    // (la_prefill then checks the arguments and picks the single pass).
     void *ws = nullptr;
-    if (need > 0) {
+    if (la_prefill_workspace_size(mode, dtype, B, H, T, d_k, d_v, chunk) > 0)
         ws = la::static_workspace_address();
-        if (!ws) return LA_ERR_CUDA;
-    }
     return la_prefill(mode, dtype, B, H, T, d_k, d_v, q, k, v, gate, beta, state, z, o, chunk,
                       flags, ws, ws ? la::kStaticWorkspaceBytes : 0, stream);
 }

@@ -166,10 +166,10 @@ size_t la_prefill_workspace_size(la_mode_t mode, la_dtype_t dtype, int B, int H,
  * arguments as la_prefill except the workspace, which it takes from a 24 MiB array
  * that the library keeps in device memory (every GPU that loads the library holds it
  * until exit).  It allocates nothing and calls no allocating routine.
- *   - Returns LA_ERR_UNSUPPORTED when even the smallest segment plan for these sizes
- *     needs more than 24 MiB (la_prefill_workspace_size() reports the fastest plan's
- *     need, which may be larger); nothing is launched then.  Otherwise the fastest plan
- *     that fits in 24 MiB runs.
+ *   - Runs the fastest segment plan whose workspace fits in 24 MiB
+ *     (la_prefill_workspace_size() reports the fastest plan's need, which may be larger),
+ *     or, when none fits, the single pass that needs no workspace: it accepts exactly the
+ *     problems la_prefill accepts and returns the same statuses.
  *   - The first call on a device looks up the array's device address (with that device
  *     current); make that first call before any stream capture on the device.
  *   - All calls share the array and it keeps the last call's contents (no result

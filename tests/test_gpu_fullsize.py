@@ -92,6 +92,46 @@ def test_decode_n256h32_sampled(la, name):
     assert slice_rel_err(f64(S[seqs]), Sr) <= TOL[w.dtype]
 
 
+def _decode_oracle(mode, inp, seqs):
+    """The oracle over the decode steps of the listed sequences: the same tokens as one
+    recurrent prefill from the seeded state gives every step's output and the final state.
+    Returns (o [n, H, steps, d_v], S [n, H, d_v, d_k])."""
+    sel = lambda t: None if t is None else f64(t[:, seqs].movedim(0, 2).contiguous())
+    o, S, _ = oracle.prefill(mode, sel(inp["q"]), sel(inp["k"]), sel(inp["v"]), sel(inp["gate"]),
+                             sel(inp["beta"]), f64(inp["state0"][seqs]))
+    return o, S
+
+
+@pytest.mark.parametrize("shift", [0.0, -4.0])
+def test_decode_n256h32_1000_steps(la, shift):
+    """The configured decode workload over its full length: 1000 sequential
+    ``decode_step`` calls on 256 sequences x 32 heads (the launch the benchmark times).
+    Every step's output of 16 sequences is compared with the oracle; at the configured
+    gates also the final state of all 256 sequences.  With weak decay (a ~ 0.98) the state
+    carries ~50 steps of history, so rounding in the fp32 state could accumulate there."""
+    w = W.variant(W.CONFIGS["gdn_decode_n256h32"], gate_shift=shift)
+    steps = w.T
+    assert steps == 1000
+    inp = W.decode_inputs(w, steps=steps, device="cuda")
+    S = inp["state0"].clone()
+    o = torch.empty(w.B, w.H, w.dv, device="cuda", dtype=w.dtype)
+    seqs = list(range(0, w.B, 16))
+    outs = torch.empty(len(seqs), w.H, steps, w.dv, device="cuda", dtype=w.dtype)
+    for t in range(steps):
+        la.decode_step(inp["q"][t], inp["k"][t], inp["v"][t], mode=w.mode, state=S,
+                       gate=inp["gate"][t], beta=inp["beta"][t], o=o)
+        outs[:, :, t] = o[seqs]
+    la.check_status()
+    ro, rS = _decode_oracle(w.mode, inp, seqs)
+    assert slice_rel_err(f64(outs), ro) <= TOL[w.dtype]
+    assert slice_rel_err(f64(S[seqs]), rS) <= TOL[w.dtype]
+    if shift == 0.0:
+        for g in range(0, w.B, 32):
+            grp = list(range(g, g + 32))
+            _, rS = _decode_oracle(w.mode, inp, grp)
+            assert slice_rel_err(f64(S[grp]), rS) <= TOL[w.dtype], g
+
+
 @pytest.mark.parametrize("mode", [0, 1, 2])
 def test_segmented_equals_single_pass(la, mode):
     """The workspace (parallel segments chained by the combine kernel) and the
