@@ -109,3 +109,32 @@ def test_backward_pins_catch_planted_mistakes(name, tmp_path):
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"planted mistake {name} passed every pin:\n{r.stdout[-2000:]}"
     assert "failed" in r.stdout or "error" in r.stdout.lower()
+
+
+DELTA_BWD_MUTANTS = {
+    "delta_correction_sign": ("S = S - b * Sk[..., :, None] * kt[..., None, :]",
+                              "S = S + b * Sk[..., :, None] * kt[..., None, :]"),
+    "delta_correction_uses_query": ('Sk = torch.einsum("bhij,bhj->bhi", S, kt)',
+                                    'Sk = torch.einsum("bhij,bhj->bhi", S, q[:, :, t])'),
+    "delta_write_drops_rate": ("+ b * v[:, :, t, :, None] * kt[..., None, :]",
+                               "+ v[:, :, t, :, None] * kt[..., None, :]"),
+    "kda_decays_rows": ("a[:, :, t, None, :] if mode == MODE_KDA", "a[:, :, t, None, :1] if mode == MODE_KDA"),
+    "delta_drops_final_state_term": ("L = L + (_t(dS_T) * ST).sum()", "L = L + 0.0 * (_t(dS_T) * ST).sum()"),
+    "delta_rate_gradient_misrouted": ("dq, dk, dv, db = (x.detach().numpy() for x in grads[:4])",
+                                      "dq, dk, db, dv = (x.detach().numpy() for x in grads[:4])"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(DELTA_BWD_MUTANTS))
+def test_delta_backward_pins_catch_planted_mistakes(name, tmp_path):
+    old, new = DELTA_BWD_MUTANTS[name]
+    src = open(BWD_SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mutant = tmp_path / "backward_mutant.py"
+    mutant.write_text(src.replace(old, new))
+    env = dict(os.environ, LA_ORACLE_BACKWARD_OVERRIDE=str(mutant))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_delta_backward_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"planted mistake {name} passed every pin:\n{r.stdout[-2000:]}"
+    assert "failed" in r.stdout or "error" in r.stdout.lower()
