@@ -388,8 +388,9 @@ class VarlenCase:
 
 
 class BackwardCase:
-    """One step = one la_prefill_backward call (mode 1): dq, dk, dv and the gate gradient
-    for the default prefill's shape, from output cotangents dO."""
+    """One step = one backward call: la_prefill_backward (mode 1) or
+    la_prefill_backward_delta (modes 2, 3): dq, dk, dv, the gate gradient (and the rate
+    gradient of the delta rule) from output cotangents dO."""
 
     def __init__(self, la, w: W.Workload, device, rank):
         self.la, self.w, self.device = la, w, device
@@ -400,20 +401,37 @@ class BackwardCase:
         self.tokens = w.B * w.T
         th = w.B * w.H * w.T
         e = io_bytes(w.dtype)
-        # read q, k, v, dO and the gates; write dq, dk, dv and the gate gradient
-        self.bytes = float(th * (e * (3 * w.dk + 4 * w.dv) + 8))
-        # forward recompute of the states and four d_k x d_v products per token-head, plus
-        # the chunk's score products (C = 32)
-        self.flops = float(th * (10 * w.dk * w.dv + 8 * 32 * (w.dk + w.dv)))
+        self.delta = w.mode in (2, 3)
+        if not self.delta:
+            # read q, k, v, dO and the gates; write dq, dk, dv and the gate gradient
+            self.bytes = float(th * (e * (3 * w.dk + 4 * w.dv) + 8))
+            # forward recompute of the states and four d_k x d_v products per token-head,
+            # plus the chunk's score products (C = 32)
+            self.flops = float(th * (10 * w.dk * w.dv + 8 * 32 * (w.dk + w.dv)))
+        else:
+            gw = 4 * (w.dk if w.mode == 3 else 1)
+            # read q, k, v, dO, gates, b; write dq, dk, dv, the gate and rate gradients
+            self.bytes = float(th * (e * (4 * w.dk + 3 * w.dv) + 2 * gw + 8))
+            # per token-head: nine d_k x d_v products (forward states: E and the state update;
+            # reverse: E, dE, dW, E H^T, the carried cotangent (2), dq) and the chunk's
+            # C-wide products (C = 32: Gram, WY factors, dT, T^T dW, dq/dk score terms)
+            self.flops = float(th * (2 * 9 * w.dk * w.dv + 2 * 32 * (12 * w.dk + 7 * w.dv)))
         self.kind = "backward"
 
-    def step(self):
+    def _call(self):
         i = self.inp
-        self.la.prefill_backward(i["q"], i["k"], i["v"], self.dO, mode=self.w.mode, gate=i["gate"])
+        if self.delta:
+            return self.la.prefill_backward_delta(i["q"], i["k"], i["v"], self.dO, mode=self.w.mode,
+                                                  beta=i["beta"], gate=i["gate"])[:3]
+        return self.la.prefill_backward(i["q"], i["k"], i["v"], self.dO, mode=self.w.mode,
+                                        gate=i["gate"])[:3]
+
+    def step(self):
+        self._call()
 
     def e2e_setup(self):
         pin = lambda t: t.to("cpu").pin_memory()
-        self.h_in = {k: pin(self.inp[k]) for k in ("q", "k", "v", "gate")}
+        self.h_in = {k: pin(self.inp[k]) for k in ("q", "k", "v", "gate") + (("beta",) if self.delta else ())}
         self.h_do = pin(self.dO)
         self.h_out = [torch.empty(self.inp["q"].shape, dtype=self.w.dtype).pin_memory() for _ in range(3)]
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values()) + \
@@ -424,9 +442,7 @@ class BackwardCase:
         for k, v in self.h_in.items():
             self.inp[k].copy_(v, non_blocking=True)
         self.dO.copy_(self.h_do, non_blocking=True)
-        i = self.inp
-        dq, dk, dv, _, _ = self.la.prefill_backward(i["q"], i["k"], i["v"], self.dO, mode=self.w.mode,
-                                                    gate=i["gate"])
+        dq, dk, dv = self._call()
         for h, d in zip(self.h_out, (dq, dk, dv)):
             h.copy_(d, non_blocking=True)
 
@@ -551,8 +567,9 @@ def roofline(case, kernel_ms, step_ms, peaks, peak_src, prof):
     n = len(kernel_ms)
     names = ([k["name"] for k in prof["kernels"]] if prof and len(prof["kernels"]) == n
              else [f"launch {i}" for i in range(n)])
-    t_k = (kernel_ms[-1] if n else step_ms) * 1e-3
     t_call = (sum(kernel_ms) if n else step_ms) * 1e-3
+    # a backward call splits its work over sweeps that each do a share of it: the whole call
+    t_k = t_call if case.kind == "backward" else (kernel_ms[-1] if n else step_ms) * 1e-3
     if hbm_bound:
         unit, peak, work, scale = "GB/s", peaks["hbm_gbs"], case.bytes, 1e9
     else:
@@ -565,9 +582,9 @@ def roofline(case, kernel_ms, step_ms, peaks, peak_src, prof):
     return {
         "bound": "hbm" if hbm_bound else "tensor",
         "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak, "traffic": traffic,
-        "kernel": names[-1] if n else "call",
-        "kernel_ms": kernel_ms[-1] if n else step_ms,
-        "kernel_share": (kernel_ms[-1] / sum(kernel_ms)) if n else 1.0,
+        "kernel": (names[-1] if n and case.kind != "backward" else "call"),
+        "kernel_ms": t_k * 1e3,
+        "kernel_share": (t_k / t_call) if n else 1.0,
         "algorithmic_bytes": case.bytes, "algorithmic_flops": case.flops,
         "tensor_frac": case.flops / t_k / 1e12 / peaks["bf16_tflops"],
         "call": {"launches": n, "kernels": names, "kernel_ms": kernel_ms,
@@ -697,11 +714,15 @@ def oracle_sample_other(name, budget_s):
         from oracle import backward as ob
         w = W.BACKWARD_CONFIGS[name]
         inp = W.prefill_inputs(W.variant(w, B=1, H=min(w.H, 4), T=256), device="cpu")
-        a = {k: f(inp[k]) for k in ("q", "k", "v", "gate")}
+        a = {k: f(inp[k]) for k in ("q", "k", "v", "gate") + (("beta",) if w.mode in (2, 3) else ())}
         do = np.random.default_rng(0).standard_normal(a["v"].shape)
-        T, el = _timed_growing(lambda n: ob.prefill_backward(w.mode, a["q"][:, :, :n], a["k"][:, :, :n],
-                                                            a["v"][:, :, :n], a["gate"][:, :, :n],
-                                                            do[:, :, :n]), 32, 256, budget_s)
+        if w.mode in (2, 3):
+            run = lambda n: ob.delta_backward(w.mode, a["q"][:, :, :n], a["k"][:, :, :n], a["v"][:, :, :n],
+                                              a["gate"][:, :, :n], a["beta"][:, :, :n], do[:, :, :n])
+        else:
+            run = lambda n: ob.prefill_backward(w.mode, a["q"][:, :, :n], a["k"][:, :, :n], a["v"][:, :, :n],
+                                                a["gate"][:, :, :n], do[:, :, :n])
+        T, el = _timed_growing(run, 32, 256, budget_s)
         hs = a["q"].shape[1]
         return {"value": hs * T / el / w.H, "unit": "tokens/s", "cores": torch.get_num_threads(),
                 "kind": "oracle", "sample": f"{hs} heads x {T} tokens (fp64 PyTorch autograd on the CPU)"}
@@ -859,7 +880,7 @@ def main():
         for name in ("elu1_f32_small", "elu1_bf16_b4h16t4096", "gated_bf16_b8h16t8192",
                      "gdn_bf16_b2h16t32768", "gdn_decode_n256h32", "kda_bf16_b2h16t32768",
                      "kda_decode_n256h32", "conv_bf16_b2h16t32768", "gdn_varlen_bf16_n64h16",
-                     "retnet_bf16_b8h16t8192", "gated_bwd_bf16_b4h16t4096"):
+                     "retnet_bf16_b8h16t8192", "gated_bwd_bf16_b4h16t4096", "gdn_bwd_bf16_b2h16t32768"):
             if name == args.workload:
                 continue
             r = measure(la, name, args, dist, device, rank, world, flush, True)

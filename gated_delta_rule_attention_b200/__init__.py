@@ -25,7 +25,7 @@ import os
 import torch
 
 __all__ = ["MODE_ELU1_NORM", "MODE_GATED", "MODE_GATED_DELTA", "MODE_KDA", "MODE_RETNET", "FLAG_INIT_STATE", "LaError",
-           "prefill", "prefill_varlen", "prefill_backward", "decode_step", "short_conv", "short_conv_varlen", "short_conv_step", "check_status", "library",
+           "prefill", "prefill_varlen", "prefill_backward", "prefill_backward_delta", "decode_step", "short_conv", "short_conv_varlen", "short_conv_step", "check_status", "library",
            "library_path", "version", "kernel_launches", "workspace_size"]
 
 MODE_ELU1_NORM = 0
@@ -94,6 +94,9 @@ def library():
     lib.la_prefill_backward.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, fp, fp, vp, fp, vp, vp, vp,
                                         fp, fp, vp, ctypes.c_size_t, vp]
     lib.la_prefill_backward.restype = i
+    lib.la_prefill_backward_delta.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, fp, fp, fp, vp, fp, vp,
+                                              vp, vp, fp, fp, fp, vp, ctypes.c_size_t, vp]
+    lib.la_prefill_backward_delta.restype = i
     lib.la_short_conv.argtypes = [i, i, i, i, i, i, vp, fp, vp, vp, vp, u, vp]
     lib.la_short_conv.restype = i
     lib.la_short_conv_varlen.argtypes = [i, i, i, i, i, i, vp, vp, fp, vp, vp, vp, u, vp]
@@ -356,6 +359,50 @@ def prefill_backward(q, k, v, dO, *, mode: int, gate=None, state0=None, dstate=N
                                        ws.numel(), _stream_handle(q.device, stream))
     _check(st, "la_prefill_backward")
     return dq, dk, dv, dgate, dstate0
+
+
+def prefill_backward_delta(q, k, v, dO, *, mode: int, beta, gate=None, state0=None, dstate=None,
+                           need_dgate: bool = True, need_dstate0: bool | None = None, stream=None):
+    """Gradients of the delta-rule prefill (``la_prefill_backward_delta``, modes 2 and 3).
+
+    q, k: [B,H,T,d_k]; v, dO: [B,H,T,d_v]; beta: [B,H,T] fp32; gate: [B,H,T] (mode 2) or
+    [B,H,T,d_k] (mode 3) fp32, or None (a = 1); state0, dstate: [B,H,d_v,d_k] fp32 or None.
+    Returns (dq, dk, dv, dgate, dbeta, dstate0): dgate shaped like gate (None without a
+    gate), dbeta [B,H,T] fp32, dstate0 when ``need_dstate0`` (default: when state0 is given).
+    """
+    B, H, T, dk_ = q.shape
+    dv_ = v.shape[-1]
+    dt = q.dtype
+    dtype = _io_dtype(q)
+    _need(q, (B, H, T, dk_), dt, "q")
+    _need(k, (B, H, T, dk_), dt, "k")
+    _need(v, (B, H, T, dv_), dt, "v")
+    _need(dO, (B, H, T, dv_), dt, "dO")
+    _need(beta, (B, H, T), torch.float32, "beta")
+    if gate is not None:
+        _need(gate, _gate_shape(mode, (B, H, T), dk_, H), torch.float32, "gate")
+    for name, t in (("state0", state0), ("dstate", dstate)):
+        if t is not None:
+            _need(t, (B, H, dv_, dk_), torch.float32, name)
+    if need_dstate0 is None:
+        need_dstate0 = state0 is not None
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    dgate = torch.empty_like(gate) if (need_dgate and gate is not None) else None
+    dbeta = torch.empty_like(beta)
+    dstate0 = (torch.empty(B, H, dv_, dk_, device=q.device, dtype=torch.float32)
+               if need_dstate0 else None)
+    nbytes = int(library().la_backward_workspace_size(int(mode), B, H, T, dk_, dv_))
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    if stream is not None:
+        ws.record_stream(stream)   # freed on return: not reused before `stream`'s work is done
+    st = library().la_prefill_backward_delta(
+        int(mode), dtype, B, H, T, dk_, dv_, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(beta),
+        _ptr(state0), _ptr(dO), _ptr(dstate), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate), _ptr(dbeta),
+        _ptr(dstate0), _ptr(ws), ws.numel(), _stream_handle(q.device, stream))
+    _check(st, "la_prefill_backward_delta")
+    return dq, dk, dv, dgate, dbeta, dstate0
 
 
 def decode_step(q, k, v, *, mode: int, state, gate=None, beta=None, z=None, o=None,

@@ -66,27 +66,6 @@ int internal_mode(int mode) { return mode == LA_MODE_RETNET ? (int)LA_MODE_GATED
 
 bool dims_ok(int dk, int dv) { return (dk == 64 || dk == 128) && (dv == 64 || dv == 128); }
 
-// True if the byte ranges [p, p + n) and [q, q + m) share a byte.
-bool overlap(const void *p, size_t n, const void *q, size_t m) {
-    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
-    return p && q && n && m && a < b + m && b < a + n;
-}
-
-using Span = std::pair<const void *, size_t>;
-
-// True if the buffers a call writes (o, the state, z) share no byte with one another or with
-// any buffer it only reads (null spans are skipped).  The kernels read inputs while they
-// write outputs, so an overlap would be a race, not an in-place update.
-bool writes_disjoint(std::initializer_list<Span> writes, std::initializer_list<Span> reads) {
-    for (auto w = writes.begin(); w != writes.end(); ++w) {
-        for (auto u = w + 1; u != writes.end(); ++u)
-            if (overlap(w->first, w->second, u->first, u->second)) return false;
-        for (const Span &r : reads)
-            if (overlap(w->first, w->second, r.first, r.second)) return false;
-    }
-    return true;
-}
-
 // Bytes of a call's gate tensor: per token (a scalar, or d_k values in the per-channel mode)
 // or one value per head (the constant-decay mode).
 size_t gate_bytes(int mode, long long tokens_x_heads, int H, int d_k) {

@@ -24,6 +24,7 @@
 // a small kernel finishes dV and the gate gradient.  Tiles live in shared memory with one
 // float of row padding; the products are register-tiled (a thread holds up to 16 x 4
 // outputs), so that each shared load feeds several FMAs.
+#include "bwd_util.cuh"
 #include "la_internal.cuh"
 
 #include <cfloat>
@@ -61,26 +62,6 @@ __device__ __forceinline__ float block_sum(float x, float *red) {
     float s = 0.f;
     for (int i = 0; i < kBwdThreads / 32; ++i) s += red[i];
     return s;
-}
-
-// Register-tiled products on shared-memory operands.  A thread computes RM rows x RN
-// columns of an M x N output: rows r0 + i (i < RM) and columns lane + 32 n (n < RN), so
-// that the B operand's loads are consecutive across the warp and the A operand's are
-// broadcasts.  acc[i][n] += sum_k A(row, k) B(k, col).
-template <int RM, int RN, int K, typename FA, typename FB>
-__device__ __forceinline__ void tile_mma(float (&acc)[RM][RN], int r0, int lane, FA a, FB b) {
-#pragma unroll 4
-    for (int kk = 0; kk < K; ++kk) {
-        float av[RM], bv[RN];
-#pragma unroll
-        for (int i = 0; i < RM; ++i) av[i] = a(r0 + i, kk);
-#pragma unroll
-        for (int n = 0; n < RN; ++n) bv[n] = b(kk, lane + 32 * n);
-#pragma unroll
-        for (int i = 0; i < RM; ++i)
-#pragma unroll
-            for (int n = 0; n < RN; ++n) acc[i][n] = fmaf(av[i], bv[n], acc[i][n]);
-    }
 }
 
 template <int DK, int DV, int SPLIT, typename IO>
@@ -407,6 +388,8 @@ bool on_device(const void *p) {
 using namespace la;
 
 extern "C" size_t la_backward_workspace_size(la_mode_t mode, int B, int H, int T, int d_k, int d_v) {
+    if (mode == LA_MODE_GATED_DELTA || mode == LA_MODE_KDA)
+        return delta_backward_workspace_bytes(mode, B, H, T, d_k, d_v);
     if ((mode != LA_MODE_GATED && mode != LA_MODE_RETNET) || B < 1 || H < 1 || T < 1) return 0;
     const size_t nch = ((size_t)T + kBwdC - 1) / kBwdC;
     // every chunk-start state, then the fp32 accumulators of dv and dlam

@@ -3,6 +3,8 @@
 #pragma once
 
 #include <cstdint>
+#include <initializer_list>
+#include <utility>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -88,8 +90,31 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t work
 bool prefill_gdn_selected(int mode, int BH, bool packed);
 cudaError_t launch_prefill_gdn(const PrefillArgs &a);
 cudaError_t launch_short_conv(const ConvArgs &a);
+// Workspace of la_prefill_backward_delta (0 for other modes).
+size_t delta_backward_workspace_bytes(int mode, int B, int H, int T, int d_k, int d_v);
 // Zero the state (and z) of every packed sequence with no tokens (cu[s+1] <= cu[s]).
 cudaError_t launch_zero_empty_sequences(const PrefillArgs &a);
+
+// True if the byte ranges [p, p + n) and [q, q + m) share a byte.
+inline bool overlap(const void *p, size_t n, const void *q, size_t m) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+    return p && q && n && m && a < b + m && b < a + n;
+}
+
+using Span = std::pair<const void *, size_t>;
+
+// True if the buffers a call writes share no byte with one another or with any buffer it
+// only reads (null spans are skipped).  The kernels read inputs while they write outputs,
+// so an overlap would be a race, not an in-place update.
+inline bool writes_disjoint(std::initializer_list<Span> writes, std::initializer_list<Span> reads) {
+    for (auto w = writes.begin(); w != writes.end(); ++w) {
+        for (auto u = w + 1; u != writes.end(); ++u)
+            if (overlap(w->first, w->second, u->first, u->second)) return false;
+        for (const Span &r : reads)
+            if (overlap(w->first, w->second, r.first, r.second)) return false;
+    }
+    return true;
+}
 
 // fp32 <-> I/O element helpers used by the CUDA-core kernels.
 __device__ __forceinline__ float to_f32(float x) { return x; }

@@ -278,6 +278,7 @@ la_status_t la_short_conv_step(la_dtype_t dtype, int N, int H, int d, int width,
  *   dstate0       out [B, H, d_v, d_k] fp32 (the gradient of state0), or NULL
  *   workspace     device scratch of at least la_backward_workspace_size() bytes
  *                 (required: every chunk-start state is kept there)
+ * la_backward_workspace_size also sizes la_prefill_backward_delta's workspace (modes 2, 3).
  */
 size_t la_backward_workspace_size(la_mode_t mode, int B, int H, int T, int d_k, int d_v);
 la_status_t la_prefill_backward(la_mode_t mode, la_dtype_t dtype, int B, int H, int T, int d_k,
@@ -286,6 +287,45 @@ la_status_t la_prefill_backward(la_mode_t mode, la_dtype_t dtype, int B, int H, 
                                 const float *dstate, void *dq, void *dk, void *dv, float *dgate,
                                 float *dstate0, void *workspace, size_t workspace_bytes,
                                 void *stream);
+
+/*
+ * la_prefill_backward_delta -- gradients of the prefill for the delta-rule modes (2 and 3):
+ * the derivatives of L = sum_t do_t . o_t + <dS_T, S_T> for the update of [delta rule],
+ * S_t = S_{t-1} A_t (I - b_t k_t k_t^T) + b_t v_t k_t^T with A_t = a_t I (Gated DeltaNet) or
+ * Diag(a_t) (Kimi Delta Attention), o_t = S_t q_t, with respect to q, k, v, the gates, the
+ * rates b and the initial state.  The pages give no backward formulas; these are the plain
+ * derivatives, taken through the chunked form ([three forms]) with its WY factors
+ * T = (I + diag(b) Kgr)^-1, W = T diag(b) Kg, U = T diag(b) V, E = U - W S^T per chunk
+ * of 32 tokens; the gate gradient is d log a_t = (suffix sum within the chunk of
+ * dL/dlam), da_t = d log a_t / a_t.  CUDA cores, fp32 arithmetic; d_v is split over CTAs of
+ * 32 state rows each.
+ *
+ *   mode          LA_MODE_GATED_DELTA or LA_MODE_KDA (others: LA_ERR_UNSUPPORTED)
+ *   q, k          [B, H, T, d_k] I/O dtype      v, dO [B, H, T, d_v] I/O dtype
+ *   gate          [B, H, T] fp32 (mode 3: [B, H, T, d_k]) or NULL (a = 1); the gate gradient
+ *                 divides by a_t, so a gate of exactly 0 gives no finite dgate there
+ *   beta          [B, H, T] fp32, required
+ *   state0        [B, H, d_v, d_k] fp32 or NULL (zero)
+ *   dstate        [B, H, d_v, d_k] fp32 cotangent of S_T, or NULL (zero)
+ *   dq, dk        out [B, H, T, d_k] I/O dtype   dv out [B, H, T, d_v] I/O dtype
+ *   dgate         out, shaped like gate, or NULL (then not computed); needs gate
+ *   dbeta         out [B, H, T] fp32, or NULL
+ *   dstate0       out [B, H, d_v, d_k] fp32, or NULL
+ *   workspace     device scratch of at least la_backward_workspace_size() bytes (every
+ *                 chunk-start state and fp32 accumulators of dq, dk, db and the gate terms)
+ * d_k, d_v in {64, 128} (else LA_ERR_UNSUPPORTED); T >= 1.  Every pointer is device memory
+ * of the current device (16-byte aligned for the tensors of the I/O dtype and the
+ * workspace).  The buffers the call writes (dq, dk, dv, dgate, dbeta, dstate0, workspace)
+ * must not overlap one another or any input (LA_ERR_INVALID_ARG).  Asynchronous on
+ * `stream`; the caller keeps every buffer alive until the stream has passed the call.
+ */
+la_status_t la_prefill_backward_delta(la_mode_t mode, la_dtype_t dtype, int B, int H, int T,
+                                      int d_k, int d_v, const void *q, const void *k,
+                                      const void *v, const float *gate, const float *beta,
+                                      const float *state0, const void *dO, const float *dstate,
+                                      void *dq, void *dk, void *dv, float *dgate, float *dbeta,
+                                      float *dstate0, void *workspace, size_t workspace_bytes,
+                                      void *stream);
 
 /*
  * la_check_status -- synchronise `stream`, then report the first device-side failure
@@ -318,7 +358,8 @@ unsigned long long la_kernel_launches(void);
 
 /* Per-launch device timing, a measurement aid with no counterpart in the pages.
  * la_launch_timing(1) makes every later call of la_prefill, la_prefill_noalloc,
- * la_prefill_varlen, la_prefill_backward, la_decode_step and the la_short_conv* entry
+ * la_prefill_varlen, la_prefill_backward, la_prefill_backward_delta, la_decode_step and
+ * the la_short_conv* entry
  * points bracket each
  * kernel it enqueues
  * with two CUDA events recorded on the call's stream (at most 16 launches per call are

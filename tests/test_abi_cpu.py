@@ -197,11 +197,33 @@ def test_prefill_backward_argument_checks(lib):
     def call(mode=1, dtype=1, B=1, H=2, T=64, dk=128, dv=128):
         return lib.la_prefill_backward(mode, dtype, B, H, T, dk, dv, *([None] * 13), 0, None)
 
-    assert call(mode=2) == UNSUPPORTED     # the delta rule's backward is not built
+    assert call(mode=2) == UNSUPPORTED     # the delta rule has its own entry point
     assert call(mode=7) == INVALID
     assert call(T=0) == INVALID
     assert call(dk=32) == UNSUPPORTED
     assert call() == INVALID               # NULL tensors, before any launch
     assert call(mode=4) == INVALID         # mode 4 needs its gate
     assert lib.la_backward_workspace_size(1, 2, 3, 100, 64, 64) == 4 * 2 * 3 * (5 * 64 * 64 + 100 * 65)
-    assert lib.la_backward_workspace_size(2, 2, 3, 100, 64, 64) == 0
+    # delta rule: chunk-start states (4 chunks of 32), fp32 dq, dk, dL/dlam and db
+    BH, T, nch = 6, 100, 4
+    assert lib.la_backward_workspace_size(2, 2, 3, T, 64, 64) == 4 * (BH * nch * 64 * 64 + 2 * BH * T * 64
+                                                                      + BH * T + BH * T)
+    assert lib.la_backward_workspace_size(3, 2, 3, T, 64, 64) == 4 * (BH * nch * 64 * 64 + 3 * BH * T * 64
+                                                                      + BH * T)
+    assert lib.la_backward_workspace_size(0, 2, 3, T, 64, 64) == 0
+
+
+def test_prefill_backward_delta_argument_checks(lib):
+    INVALID, UNSUPPORTED = 1, 2
+
+    def call(mode=2, dtype=1, B=1, H=2, T=64, dk=128, dv=128):
+        return lib.la_prefill_backward_delta(mode, dtype, B, H, T, dk, dv, *([None] * 15), 0, None)
+
+    assert call(mode=1) == UNSUPPORTED     # scalar-gate modes: la_prefill_backward
+    assert call(mode=4) == UNSUPPORTED
+    assert call(mode=9) == INVALID
+    assert call(T=0) == INVALID
+    assert call(dk=96) == UNSUPPORTED
+    assert call(dtype=5) == INVALID
+    assert call() == INVALID               # NULL tensors, before any launch
+    assert call(mode=3) == INVALID

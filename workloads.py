@@ -166,10 +166,15 @@ def variant(w: Workload, **changes) -> Workload:
 
 # The backward pass of the scalar-gated prefill (mode 1): the default prefill's shape
 # (B4 H16 T4096, d = 128, bf16) with the gated recipe; output cotangents dO ~ N(0, 1).
+# The delta rule's backward (mode 2) on the long-context Gated DeltaNet prefill's shape and
+# recipe (B2 H16 T32768, d = 128, bf16, L2-normalised q and k, b = sigmoid(N(0, 1))).
 BACKWARD_CONFIGS = {
     "gated_bwd_bf16_b4h16t4096": Workload("gated_bwd_bf16_b4h16t4096", MODE_GATED, torch.bfloat16,
                                           B=4, H=16, T=4096, dk=128, dv=128, seed=11,
                                           qk_scale=1 / math.sqrt(128), gate="softplus"),
+    "gdn_bwd_bf16_b2h16t32768": Workload("gdn_bwd_bf16_b2h16t32768", MODE_GATED_DELTA, torch.bfloat16,
+                                         B=2, H=16, T=32768, dk=128, dv=128, seed=12,
+                                         qk_l2norm=True, gate="softplus", gate_shift=-3.0, beta=True),
 }
 
 
