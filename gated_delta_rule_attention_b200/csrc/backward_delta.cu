@@ -32,19 +32,25 @@
 // chunk (the state carries the rest), so d log a_t is the suffix sum of dL/dlam within the
 // chunk, and da_t = d log a_t / a_t.
 //
-// fp32 arithmetic on CUDA cores.  The rows of S (the d_v axis) evolve independently, so a
-// head's d_v is split into slices of 32 rows, one CTA each: a forward sweep stores every
-// chunk-start state slice in the workspace, then a reverse sweep carries H back through the
-// chunks.  Each CTA recomputes the chunk's d_v-independent factors (Kgr, T, W) and adds its
-// slice's share of dq, dk, db and dL/dlam (sums over d_v) into fp32 accumulators; dv and the
-// slice of dL/dS_0 are its own.  A finishing kernel converts dq and dk and takes the gate
-// suffix sums.  Gated DeltaNet's Gam is one C x C table per chunk; Kimi's per-channel Gam is
-// evaluated per product term (exp2 of the log-gate difference, no factor outside [0, 1]),
-// exact for any gate and slower.
+// The rows of S (the d_v axis) evolve independently, so a head's d_v is split into slices
+// of 32 rows, one CTA each: a forward sweep stores every chunk-start state slice in the
+// workspace, then a reverse sweep carries H back through the chunks.  Each CTA recomputes
+// the chunk's d_v-independent factors (Kgr, T, W) and adds its slice's share of dq, dk, db
+// and dL/dlam (sums over d_v) into fp32 accumulators; dv and the slice of dL/dS_0 are its
+// own.  A finishing kernel converts dq and dk and takes the gate suffix sums.
+//
+// The products run on the tensor cores as warp-level mma (m16n8k8, tf32 operands, fp32
+// accumulate): the tiles are 32 x 32 and 32 x d_k, too small and too many for tcgen05's
+// 128-row tiles, and each is followed by an element-wise step.  For fp32 I/O each operand
+// is split into a tf32 part and a tf32 remainder (three products, fp32 accuracy); for
+// bf16 I/O one tf32 product.  Gated DeltaNet's Gam is one C x C table per chunk folded into
+// the coefficient matrices; Kimi's per-channel Gam is evaluated per term on the CUDA cores
+// (exp2 of the log-gate difference, no factor outside [0, 1]), exact for any gate.
 #include "bwd_util.cuh"
 #include "la_internal.cuh"
 
 #include <cfloat>
+#include <type_traits>
 
 namespace la {
 namespace {
@@ -52,12 +58,15 @@ namespace {
 constexpr int kDT = 256;            // threads per CTA (8 warps)
 constexpr int kDC = 32;             // chunk length
 constexpr int kDVS = 32;            // d_v rows per CTA
-constexpr int kPC = kDC + 1;        // row pitch of C x C tiles
-constexpr int kPV = kDVS + 1;       // row pitch of C x d_v-slice tiles
+// Row pitches are 4 (mod 32) floats: the mma operand loads of a row-major tile
+// (row g, column t4 of a fragment) then fall in 32 distinct banks.
+constexpr int kPC = kDC + 4;        // C x C tiles
+constexpr int kPV = kDVS + 4;       // C x d_v-slice tiles
+template <int DK> __host__ __device__ constexpr int pitch_k() { return DK + 4; }
 
 template <int MODE, int DK>
 struct DeltaBwdSmem {
-    static constexpr int PK = DK + 1;
+    static constexpr int PK = pitch_k<DK>();
     static constexpr int CK = kDC * PK;     // C x d_k tile
     static constexpr int SK = kDVS * PK;    // d_v slice x d_k tile
     static constexpr int CC = kDC * kPC;
@@ -68,9 +77,14 @@ struct DeltaBwdSmem {
     static constexpr int nCC = 8;
     // C x d_v slice: Vs dOs Es dEs TdE
     static constexpr int nCV = 5;
-    // bet lam g dec dbl | gl col1 col2
-    static constexpr int kSmall = 5 * kDC + 3 * DK;
-    static constexpr int kFloats = nCK * CK + 2 * SK + nCC * CC + nCV * CV + kSmall;
+    // bet lam g dec dbl dbs dls | gl col1 col2
+    static constexpr int kSmall = 7 * kDC + 3 * DK;
+    // Gated DeltaNet stages the next chunk's raw inputs with cp.async while the current one
+    // is processed (Kimi's per-channel tiles leave no room): q, k [C][d_k], v, dO [C][32]
+    // in the I/O dtype (sized for 4-byte elements), the state slice [32][d_k], gate and b.
+    static constexpr bool kStage = MODE != 3;
+    static constexpr int kStageFloats = kStage ? 2 * kDC * DK + 2 * kDC * kDVS + kDVS * DK + 2 * kDC : 0;
+    static constexpr int kFloats = nCK * CK + 2 * SK + nCC * CC + nCV * CV + kSmall + kStageFloats;
     static constexpr size_t kBytes = sizeof(float) * kFloats;
     static_assert(kBytes <= 227 * 1024, "shared memory");
 };
@@ -84,7 +98,8 @@ struct ChunkTiles {
     float *Ss, *Hs;
     float *Am, *Km, *Tm, *Xm, *dAm, *dTm, *Gm, *BL;
     float *Vs, *dOs, *Es, *dEs, *TdE;
-    float *bet, *lam, *g, *dec, *dbl, *gl, *col1, *col2;
+    float *bet, *lam, *g, *dec, *dbl, *dbs, *dls, *gl, *col1, *col2;
+    float *sq, *sk, *sv, *sdo, *sS, *sg, *sb;   // staging (raw I/O elements in sq .. sdo)
 
     __device__ explicit ChunkTiles(float *sm) {
         float *p = sm;
@@ -100,7 +115,14 @@ struct ChunkTiles {
         dAm = take(L::CC); dTm = take(L::CC); Gm = take(L::CC); BL = take(L::CC);
         Vs = take(L::CV); dOs = take(L::CV); Es = take(L::CV); dEs = take(L::CV); TdE = take(L::CV);
         bet = take(kDC); lam = take(kDC); g = take(kDC); dec = take(kDC); dbl = take(kDC);
+        dbs = take(kDC); dls = take(kDC);
         gl = take(DK); col1 = take(DK); col2 = take(DK);
+        if constexpr (L::kStage) {
+            sq = take(kDC * DK); sk = take(kDC * DK); sv = take(kDC * kDVS); sdo = take(kDC * kDVS);
+            sS = take(kDVS * DK); sg = take(kDC); sb = take(kDC);
+        } else {
+            sq = sk = sv = sdo = sS = sg = sb = nullptr;
+        }
     }
     // Kg, Kl, Qg entries: per channel (mode 3) or the token's scalar factor (mode 2).
     __device__ __forceinline__ float kg(int t, int c) const {
@@ -125,6 +147,27 @@ struct ChunkTiles {
     }
 };
 
+// Fragment ownership of the warp products (bwd_util.cuh's warp_mma): a 32 x 32 output
+// gives warp w rows 16 (w & 1) .. +15 and columns 8 (w >> 1) .. +7 (one n-tile); a
+// 32 x d_k output gives it rows 16 (w & 1) .. +15 and d_k / 4 columns from
+// (d_k / 4)(w >> 1) (d_k / 32 n-tiles).  frag_each visits a thread's elements.
+struct Own {
+    int m0, n32, nk;
+};
+template <int DK>
+__device__ __forceinline__ Own ownership() {
+    const int w = threadIdx.x >> 5;
+    return {16 * (w & 1), 8 * (w >> 1), (DK / 4) * (w >> 1)};
+}
+template <int NT, typename F>
+__device__ __forceinline__ void frag_each(float (&d)[NT][4], int m0, int n0, F f) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) f(d[nt][r], m0 + g + 8 * (r >> 1), n0 + 8 * nt + 2 * t4 + (r & 1));
+}
+
 // Rows [t0, t0 + n) of a [rows, d] tensor into a C x d tile (pitch `pitch`), columns
 // [c0, c0 + w) of the source; rows n .. C-1 are zero.
 template <typename IO>
@@ -136,18 +179,84 @@ __device__ __forceinline__ void load_tile(const IO *__restrict__ src, size_t row
     }
 }
 
+// ---- cp.async staging of a chunk's raw inputs (Gated DeltaNet)
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Rows [0, n) of `w` elements (a multiple of 16 bytes) from src (row stride ld elements)
+// into dst (row stride w), 16 bytes per copy.
+template <typename IO>
+__device__ __forceinline__ void stage_rows(void *dst, const IO *src, int ld, int w, int n) {
+    constexpr int E = 16 / sizeof(IO);   // elements per copy
+    const int per = w / E;
+    for (int p = threadIdx.x; p < n * per; p += kDT) {
+        const int t = p / per, x = (p % per) * E;
+        cp_async16(static_cast<IO *>(dst) + t * w + x, src + (size_t)t * ld + x);
+    }
+}
+// One chunk's raw inputs into the staging buffers: k, v (columns j0 ..), gate, b, and for
+// the reverse sweep q, dO and the chunk-start state slice; rows [0, n).
+template <int MODE, int DK, typename IO>
+__device__ __forceinline__ void stage_chunk(const ChunkTiles<MODE, DK> &c, const IO *q, const IO *k,
+                                            const IO *v, const IO *dO, const float *gate,
+                                            const float *beta, const float *state, size_t r, int n,
+                                            int DV, int j0) {
+    stage_rows(c.sk, k + r * DK, DK, DK, n);
+    stage_rows(c.sv, v + r * DV + j0, DV, kDVS, n);
+    if (q) {
+        stage_rows(c.sq, q + r * DK, DK, DK, n);
+        stage_rows(c.sdo, dO + r * DV + j0, DV, kDVS, n);
+        stage_rows(c.sS, state, DK, DK, kDVS);
+    }
+    const int tid = threadIdx.x;
+    if (tid < n) cp_async4(c.sb + tid, beta + r + tid);
+    if (gate && tid >= 32 && tid - 32 < n) cp_async4(c.sg + tid - 32, gate + r + tid - 32);
+    cp_async_commit();
+}
+// Staged rows into a C x w fp32 tile (pitch `pitch`, a multiple of 4), zero past row n:
+// 16 bytes of staged elements per step, written as float4.
+template <typename IO>
+__device__ __forceinline__ void unstage(const void *src, int w, int n, float *dst, int pitch) {
+    constexpr int E = 16 / sizeof(IO);
+    for (int p = threadIdx.x; p < kDC * w / E; p += kDT) {
+        const int t = p * E / w, j = p * E % w;
+        float f[E];
+        if (t < n) {
+            const uint4 raw = *reinterpret_cast<const uint4 *>(static_cast<const IO *>(src) + t * w + j);
+            const IO *x = reinterpret_cast<const IO *>(&raw);
+#pragma unroll
+            for (int e = 0; e < E; ++e) f[e] = to_f32(x[e]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) f[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < E; e += 4)
+            *reinterpret_cast<float4 *>(dst + t * pitch + j + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+    }
+}
+
 // The chunk's gates: b (zero past the last token), the log2 gate prefix (held at its last
 // value past the last token) and the derived factors.  Mode 2: lam, g, dec, gl[all] = g_L
 // and the C x C table Gm = Gam; mode 3: Lg, gl, Kg, Kl (and Qg when `with_q`).
+// gate and beta point at the chunk's first token (global memory or the staging buffers).
 template <int MODE, int DK>
-__device__ void load_gates(const ChunkTiles<MODE, DK> &c, const float *__restrict__ gate,
-                           const float *__restrict__ beta, size_t row0, int n, bool with_q) {
-    constexpr int PK = DK + 1;
+__device__ void load_gates(const ChunkTiles<MODE, DK> &c, const float *gate, const float *beta, int n,
+                           bool with_q) {
+    constexpr int PK = pitch_k<DK>();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (warp == 0) {
-        c.bet[lane] = lane < n ? beta[row0 + lane] : 0.f;
+        c.bet[lane] = lane < n ? beta[lane] : 0.f;
         if constexpr (MODE != 3) {
-            float x = (gate && lane < n) ? log2f(fmaxf(gate[row0 + lane], FLT_MIN)) : 0.f;
+            float x = (gate && lane < n) ? log2f(fmaxf(gate[lane], FLT_MIN)) : 0.f;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, x, off);
@@ -165,7 +274,7 @@ __device__ void load_gates(const ChunkTiles<MODE, DK> &c, const float *__restric
         if (tid < DK) {
             float acc = 0.f;
             for (int t = 0; t < kDC; ++t) {
-                if (gate && t < n) acc += log2f(fmaxf(gate[(row0 + t) * DK + tid], FLT_MIN));
+                if (gate && t < n) acc += log2f(fmaxf(gate[t * DK + tid], FLT_MIN));
                 c.Lg[t * PK + tid] = acc;
             }
             c.gl[tid] = exp2f(c.Lg[(n - 1) * PK + tid]);
@@ -191,13 +300,16 @@ __device__ void load_gates(const ChunkTiles<MODE, DK> &c, const float *__restric
 }
 
 // Gam-weighted Gram products of the chunk: A (Q K^T, j <= t; only when `with_a`) into Am
-// and Kgr (K K^T, j < t) into Km, Lm = diag(b) Kgr into Xm.  Rows 4 w + i, column = lane.
-template <int MODE, int DK>
+// and Kgr (K K^T, j < t) into Km, Lm = diag(b) Kgr into Xm.  Mode 2: tensor-core products
+// scaled by the Gam table; mode 3: one exponential per term on the CUDA cores (rows
+// 4 w + i, column = lane).
+template <int MODE, int DK, bool SP>
 __device__ void grams(const ChunkTiles<MODE, DK> &c, bool with_a) {
-    constexpr int PK = DK + 1;
-    const int lane = threadIdx.x & 31, r0 = 4 * (threadIdx.x >> 5);
-    float aA[4][1] = {}, aK[4][1] = {};
+    constexpr int PK = pitch_k<DK>();
+    const int lane = threadIdx.x & 31;
     if constexpr (MODE == 3) {
+        const int r0 = 4 * (threadIdx.x >> 5);
+        float aA[4] = {}, aK[4] = {};
         for (int cc = 0; cc < DK; ++cc) {
             const float kj = c.Ks[lane * PK + cc], lj = c.Lg[lane * PK + cc];
 #pragma unroll
@@ -205,25 +317,35 @@ __device__ void grams(const ChunkTiles<MODE, DK> &c, bool with_a) {
                 const int t = r0 + i;
                 const float e = lane <= t ? exp2f(c.Lg[t * PK + cc] - lj) : 0.f;
                 const float ke = kj * e;
-                if (with_a) aA[i][0] = fmaf(c.Qs[t * PK + cc], ke, aA[i][0]);
-                aK[i][0] = fmaf(c.Ks[t * PK + cc], ke, aK[i][0]);
+                if (with_a) aA[i] = fmaf(c.Qs[t * PK + cc], ke, aA[i]);
+                aK[i] = fmaf(c.Ks[t * PK + cc], ke, aK[i]);
             }
         }
-    } else {
-        if (with_a)
-            tile_mma<4, 1, DK>(aA, r0, lane, [&](int t, int cc) { return c.Qs[t * PK + cc]; },
-                               [&](int cc, int j) { return c.Ks[j * PK + cc]; });
-        tile_mma<4, 1, DK>(aK, r0, lane, [&](int t, int cc) { return c.Ks[t * PK + cc]; },
-                           [&](int cc, int j) { return c.Ks[j * PK + cc]; });
-    }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int t = r0 + i, j = lane;
-        const float gm = MODE == 3 ? 1.f : c.Gm[t * kPC + j];
-        if (with_a) c.Am[t * kPC + j] = j <= t ? aA[i][0] * gm : 0.f;
-        const float kgr = j < t ? aK[i][0] * gm : 0.f;
-        c.Km[t * kPC + j] = kgr;
-        c.Xm[t * kPC + j] = c.bet[t] * kgr;
+        for (int i = 0; i < 4; ++i) {
+            const int t = r0 + i, j = lane;
+            if (with_a) c.Am[t * kPC + j] = j <= t ? aA[i] : 0.f;
+            const float kgr = j < t ? aK[i] : 0.f;
+            c.Km[t * kPC + j] = kgr;
+            c.Xm[t * kPC + j] = c.bet[t] * kgr;
+        }
+    } else {
+        const Own o = ownership<DK>();
+        float ak[1][4] = {};
+        warp_mma<1, DK, SP>(ak, o.m0, o.n32, [&](int t, int cc) { return c.Ks[t * PK + cc]; },
+                            [&](int cc, int j) { return c.Ks[j * PK + cc]; });
+        frag_each(ak, o.m0, o.n32, [&](float &v, int t, int j) {
+            const float kgr = j < t ? v * c.Gm[t * kPC + j] : 0.f;
+            c.Km[t * kPC + j] = kgr;
+            c.Xm[t * kPC + j] = c.bet[t] * kgr;
+        });
+        if (with_a) {
+            float aa[1][4] = {};
+            warp_mma<1, DK, SP>(aa, o.m0, o.n32, [&](int t, int cc) { return c.Qs[t * PK + cc]; },
+                                [&](int cc, int j) { return c.Ks[j * PK + cc]; });
+            frag_each(aa, o.m0, o.n32,
+                      [&](float &v, int t, int j) { c.Am[t * kPC + j] = v * c.Gm[t * kPC + j]; });
+        }
     }
 }
 
@@ -249,34 +371,38 @@ __device__ __forceinline__ void invert_unit_lower_32(const float *Lm, float *Tm)
     for (int i = 0; i < kDC; ++i) Tm[i * kPC + lane] = x[i];
 }
 
-// W = T diag(b) Kg into Wm and U = T diag(b) V into Es (the chunk's WY factors).
-template <int MODE, int DK>
-__device__ __forceinline__ void wy_factors(const ChunkTiles<MODE, DK> &c) {
-    constexpr int PK = DK + 1, NK = DK / 32;
-    const int lane = threadIdx.x & 31, r0 = 4 * (threadIdx.x >> 5);
+// W = T diag(b) Kg into Wm, U = T diag(b) V into Es and, with `with_de`,
+// dE = A^T dO + Kl H into dEs.
+template <int MODE, int DK, bool SP>
+__device__ __forceinline__ void wy_factors(const ChunkTiles<MODE, DK> &c, bool with_de) {
+    constexpr int PK = pitch_k<DK>(), NK = DK / 32;
+    const Own o = ownership<DK>();
     auto tb = [&](int t, int u) { return c.Tm[t * kPC + u] * c.bet[u]; };
-    float w[4][NK] = {};
-    tile_mma<4, NK, kDC>(w, r0, lane, tb, [&](int u, int cc) { return c.kg(u, cc); });
-    float uu[4][1] = {};
-    tile_mma<4, 1, kDC>(uu, r0, lane, tb, [&](int u, int j) { return c.Vs[u * kPV + j]; });
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-        for (int n = 0; n < NK; ++n) c.Wm[(r0 + i) * PK + lane + 32 * n] = w[i][n];
-        c.Es[(r0 + i) * kPV + lane] = uu[i][0];
+    float w[NK][4] = {};
+    warp_mma<NK, kDC, SP>(w, o.m0, o.nk, tb, [&](int u, int cc) { return c.kg(u, cc); });
+    frag_each(w, o.m0, o.nk, [&](float &v, int t, int cc) { c.Wm[t * PK + cc] = v; });
+    float uu[1][4] = {};
+    warp_mma<1, kDC, SP>(uu, o.m0, o.n32, tb, [&](int u, int j) { return c.Vs[u * kPV + j]; });
+    frag_each(uu, o.m0, o.n32, [&](float &v, int t, int j) { c.Es[t * kPV + j] = v; });
+    if (with_de) {
+        float de[1][4] = {};
+        warp_mma<1, kDC, SP>(de, o.m0, o.n32, [&](int t, int u) { return c.Am[u * kPC + t]; },
+                             [&](int u, int j) { return c.dOs[u * kPV + j]; });
+        warp_mma<1, DK, SP>(de, o.m0, o.n32, [&](int t, int cc) { return c.kl(t, cc); },
+                            [&](int cc, int j) { return c.Hs[j * PK + cc]; });
+        frag_each(de, o.m0, o.n32, [&](float &v, int t, int j) { c.dEs[t * kPV + j] = v; });
     }
 }
 
 // E = U - W S^T, in place in Es (each thread updates the entries it wrote as U).
-template <int MODE, int DK>
+template <int MODE, int DK, bool SP>
 __device__ __forceinline__ void new_values(const ChunkTiles<MODE, DK> &c) {
-    constexpr int PK = DK + 1;
-    const int lane = threadIdx.x & 31, r0 = 4 * (threadIdx.x >> 5);
-    float e[4][1] = {};
-    tile_mma<4, 1, DK>(e, r0, lane, [&](int t, int cc) { return c.Wm[t * PK + cc]; },
-                       [&](int cc, int j) { return c.Ss[j * PK + cc]; });
-#pragma unroll
-    for (int i = 0; i < 4; ++i) c.Es[(r0 + i) * kPV + lane] -= e[i][0];
+    constexpr int PK = pitch_k<DK>();
+    const Own o = ownership<DK>();
+    float e[1][4] = {};
+    warp_mma<1, DK, SP>(e, o.m0, o.n32, [&](int t, int cc) { return c.Wm[t * PK + cc]; },
+                        [&](int cc, int j) { return c.Ss[j * PK + cc]; });
+    frag_each(e, o.m0, o.n32, [&](float &v, int t, int j) { c.Es[t * kPV + j] -= v; });
 }
 
 // ---------------------------------------------------------------------------------------
@@ -287,10 +413,12 @@ delta_states_kernel(int T, int DV, const IO *__restrict__ k, const IO *__restric
                     const float *__restrict__ gate, const float *__restrict__ beta,
                     const float *__restrict__ S0, float *__restrict__ states) {
     using L = DeltaBwdSmem<MODE, DK>;
+    constexpr bool SP = std::is_same<IO, float>::value;
     constexpr int PK = L::PK, NK = DK / 32;
     extern __shared__ float smem[];
     const ChunkTiles<MODE, DK> c(smem);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, r0 = 4 * warp;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const Own o = ownership<DK>();
     const int NS = DV / kDVS;
     const size_t bh = blockIdx.x / NS;
     const int j0 = (blockIdx.x % NS) * kDVS;
@@ -300,80 +428,107 @@ delta_states_kernel(int T, int DV, const IO *__restrict__ k, const IO *__restric
     for (int p = tid; p < kDVS * DK; p += kDT)
         c.Ss[(p / DK) * PK + p % DK] = S0 ? S0[(bh * DV + j0) * DK + p] : 0.f;
     __syncthreads();
+    constexpr bool kStage = L::kStage;
+    constexpr int GW = MODE == 3 ? DK : 1;   // gate floats per token
+    auto stage = [&](int chs) {
+        const int ts = chs * kDC;
+        stage_chunk(c, static_cast<const IO *>(nullptr), k, v, static_cast<const IO *>(nullptr), gate, beta,
+                    nullptr, row0 + ts, min(kDC, T - ts), DV, j0);
+    };
+    if constexpr (kStage) stage(0);
     for (int ch = 0; ch < nch; ++ch) {
         const int t0 = ch * kDC, n = min(kDC, T - t0);
         float *dst = states + ((bh * nch + ch) * DV + j0) * (size_t)DK;
         for (int p = tid; p < kDVS * DK; p += kDT) dst[p] = c.Ss[(p / DK) * PK + p % DK];
-        load_tile(k, row0 + t0, DK, 0, DK, n, c.Ks, PK);
-        load_tile(v, row0 + t0, DV, j0, kDVS, n, c.Vs, kPV);
+        if constexpr (kStage) {
+            cp_async_wait_all();
+            __syncthreads();
+            unstage<IO>(c.sk, DK, n, c.Ks, PK);
+            unstage<IO>(c.sv, kDVS, n, c.Vs, kPV);
+        } else {
+            load_tile(k, row0 + t0, DK, 0, DK, n, c.Ks, PK);
+            load_tile(v, row0 + t0, DV, j0, kDVS, n, c.Vs, kPV);
+        }
         __syncthreads();
-        load_gates(c, gate, beta, row0 + t0, n, false);
-        grams(c, false);
+        if constexpr (kStage) {
+            load_gates(c, gate ? c.sg : nullptr, c.sb, n, false);
+            if (ch + 1 < nch) stage(ch + 1);   // the staging buffers have been read
+        } else {
+            load_gates(c, gate ? gate + (row0 + t0) * GW : nullptr, beta + row0 + t0, n, false);
+        }
+        grams<MODE, DK, SP>(c, false);
         __syncthreads();
         if (warp == 0) invert_unit_lower_32(c.Xm, c.Tm);
         __syncthreads();
-        wy_factors(c);
+        wy_factors<MODE, DK, SP>(c, false);
         __syncthreads();
-        new_values(c);
+        new_values<MODE, DK, SP>(c);
         __syncthreads();
-        // S <- diag(g_L) S + E^T Kl  (rows j of this slice: warp-owned rows r0 + i)
-        float s[4][NK] = {};
-        tile_mma<4, NK, kDC>(s, r0, lane, [&](int j, int t) { return c.Es[t * kPV + j]; },
-                             [&](int t, int cc) { return c.kl(t, cc); });
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int nn = 0; nn < NK; ++nn) {
-                const int cc = lane + 32 * nn;
-                float &x = c.Ss[(r0 + i) * PK + cc];
-                x = fmaf(c.gl[cc], x, s[i][nn]);
-            }
+        // S <- diag(g_L) S + E^T Kl  (this slice's rows j; Ss is not read in this step)
+        float s[NK][4] = {};
+        warp_mma<NK, kDC, SP>(s, o.m0, o.nk, [&](int j, int t) { return c.Es[t * kPV + j]; },
+                              [&](int t, int cc) { return c.kl(t, cc); });
+        frag_each(s, o.m0, o.nk, [&](float &val, int j, int cc) {
+            float &x = c.Ss[j * PK + cc];
+            x = fmaf(c.gl[cc], x, val);
+        });
         __syncthreads();
     }
 }
 
 // ---------------------------------------------------------------------------------------
-// Mode 3's Gam-weighted products, one term at a time (no factor outside [0, 1]).
-// Row side: acc[i][n] += sum_{j <= t} M(t, j) X[j][c] 2^(Lg[t][c] - Lg[j][c]);
-// column side: acc[i][n] += sum_{u >= t} M(u, t) X[u][c] 2^(Lg[u][c] - Lg[t][c]),
-// for t = r0 + i and c = lane + 32 n.
-template <int DK, typename FM>
-__device__ __forceinline__ void gam_rows(float (&acc)[4][DK / 32], int r0, int lane, const float *Lg,
+// Mode 3's Gam-weighted products, one term at a time (no factor outside [0, 1]), over a
+// thread's fragment elements (t, c):
+// row side     acc += sum_{j <= t} M(t, j) X[j][c] 2^(Lg[t][c] - Lg[j][c]),
+// column side  acc += sum_{u >= t} M(u, t) X[u][c] 2^(Lg[u][c] - Lg[t][c]).
+template <int NT, int DK, typename FM>
+__device__ __forceinline__ void gam_rows(float (&acc)[NT][4], int m0, int n0, const float *Lg,
                                          const float *X, FM m) {
-    constexpr int PK = DK + 1, NK = DK / 32;
-    float lt[4][NK];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int n = 0; n < NK; ++n) lt[i][n] = Lg[(r0 + i) * PK + lane + 32 * n];
-    for (int j = 0; j <= r0 + 3; ++j) {
-#pragma unroll
-        for (int n = 0; n < NK; ++n) {
-            const float x = X[j * PK + lane + 32 * n], lj = Lg[j * PK + lane + 32 * n];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                if (j <= r0 + i) acc[i][n] = fmaf(m(r0 + i, j) * x, exp2f(lt[i][n] - lj), acc[i][n]);
-        }
-    }
+    constexpr int PK = pitch_k<DK>();
+    frag_each(acc, m0, n0, [&](float &a, int t, int cc) {
+        const float lt = Lg[t * PK + cc];
+        float s = 0.f;
+        for (int j = 0; j <= t; ++j) s = fmaf(m(t, j) * X[j * PK + cc], exp2f(lt - Lg[j * PK + cc]), s);
+        a += s;
+    });
 }
-template <int DK, typename FM>
-__device__ __forceinline__ void gam_cols(float (&acc)[4][DK / 32], int r0, int lane, const float *Lg,
+template <int NT, int DK, typename FM>
+__device__ __forceinline__ void gam_cols(float (&acc)[NT][4], int m0, int n0, const float *Lg,
                                          const float *X, FM m) {
-    constexpr int PK = DK + 1, NK = DK / 32;
-    float lt[4][NK];
+    constexpr int PK = pitch_k<DK>();
+    frag_each(acc, m0, n0, [&](float &a, int t, int cc) {
+        const float lt = Lg[t * PK + cc];
+        float s = 0.f;
+        for (int u = t; u < kDC; ++u) s = fmaf(m(u, t) * X[u * PK + cc], exp2f(Lg[u * PK + cc] - lt), s);
+        a += s;
+    });
+}
+
+// p[0] += a, p[1] += b in global memory (one vector reduction; p 8-byte aligned).
+__device__ __forceinline__ void red_add2(float *p, float a, float b) {
+    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+}
+
+// Two fragment arrays of the same ownership, element by element.
+template <int NT, typename F>
+__device__ __forceinline__ void frag_each2(float (&d1)[NT][4], float (&d2)[NT][4], int m0, int n0, F f) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int n = 0; n < NK; ++n) lt[i][n] = Lg[(r0 + i) * PK + lane + 32 * n];
-    for (int u = r0; u < kDC; ++u) {
+        for (int r = 0; r < 4; ++r) f(d1[nt][r], d2[nt][r], m0 + g + 8 * (r >> 1), n0 + 8 * nt + 2 * t4 + (r & 1));
+}
+
+// part[h] holds a thread's share of row m0 + g + 8 h (summed over its columns): add the
+// warp's row sums into buf (shared memory, several warps share a row).
+__device__ __forceinline__ void rows_add(float (&part)[2], float *buf, int m0) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
-        for (int n = 0; n < NK; ++n) {
-            const float x = X[u * PK + lane + 32 * n], lu = Lg[u * PK + lane + 32 * n];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                if (u >= r0 + i) acc[i][n] = fmaf(m(u, r0 + i) * x, exp2f(lu - lt[i][n]), acc[i][n]);
-        }
+    for (int h = 0; h < 2; ++h) {
+        float s = part[h];
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        if ((lane & 3) == 0) atomicAdd(&buf[m0 + (lane >> 2) + 8 * h], s);
     }
 }
 
@@ -389,215 +544,212 @@ delta_backward_kernel(int T, int DV, const IO *__restrict__ q, const IO *__restr
                       float *__restrict__ dk_acc, float *__restrict__ dl_acc,
                       float *__restrict__ db_acc) {
     using L = DeltaBwdSmem<MODE, DK>;
+    constexpr bool SP = std::is_same<IO, float>::value;
     constexpr int PK = L::PK, NK = DK / 32;
     constexpr int DL = MODE == 3 ? DK : 1;   // entries of dL/dlam per token
     extern __shared__ float smem[];
     const ChunkTiles<MODE, DK> c(smem);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, r0 = 4 * warp;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g8 = lane >> 2, t4 = lane & 3;
+    const Own o = ownership<DK>();
     const int NS = DV / kDVS;
     const size_t bh = blockIdx.x / NS;
     const int j0 = (blockIdx.x % NS) * kDVS;
     const int nch = (T + kDC - 1) / kDC;
     const size_t row0 = bh * (size_t)T;
 
+    constexpr bool kStage = L::kStage;
+    constexpr int GW = MODE == 3 ? DK : 1;   // gate floats per token
+    auto stage = [&](int chs) {
+        const int ts = chs * kDC;
+        stage_chunk(c, q, k, v, dO, gate, beta, states + ((bh * nch + chs) * DV + j0) * (size_t)DK, row0 + ts,
+                    min(kDC, T - ts), DV, j0);
+    };
     for (int p = tid; p < kDVS * DK; p += kDT)
         c.Hs[(p / DK) * PK + p % DK] = dST ? dST[(bh * DV + j0) * DK + p] : 0.f;
+    if constexpr (kStage) stage(nch - 1);
     for (int ch = nch - 1; ch >= 0; --ch) {
         const int t0 = ch * kDC, n = min(kDC, T - t0), last = n - 1;
-        const size_t r = row0 + t0;
-        const float *src = states + ((bh * nch + ch) * DV + j0) * (size_t)DK;
-        for (int p = tid; p < kDVS * DK; p += kDT) c.Ss[(p / DK) * PK + p % DK] = src[p];
-        load_tile(q, r, DK, 0, DK, n, c.Qs, PK);
-        load_tile(k, r, DK, 0, DK, n, c.Ks, PK);
-        load_tile(v, r, DV, j0, kDVS, n, c.Vs, kPV);
-        load_tile(dO, r, DV, j0, kDVS, n, c.dOs, kPV);
-        if (tid < DK) c.col1[tid] = 0.f;
-        __syncthreads();
-        load_gates(c, gate, beta, r, n, true);
-        grams(c, true);
-        __syncthreads();
-
-        // T (warp 0); the other warps meanwhile form dE = A^T dO + Kl H
-        if (warp == 0) {
-            invert_unit_lower_32(c.Xm, c.Tm);
+        const size_t rr = row0 + t0;
+        if constexpr (kStage) {
+            cp_async_wait_all();
+            __syncthreads();
+            unstage<IO>(c.sq, DK, n, c.Qs, PK);
+            unstage<IO>(c.sk, DK, n, c.Ks, PK);
+            unstage<IO>(c.sv, kDVS, n, c.Vs, kPV);
+            unstage<IO>(c.sdo, kDVS, n, c.dOs, kPV);
+            unstage<float>(c.sS, DK, kDVS, c.Ss, PK);
         } else {
-            for (int p = tid - 32; p < kDC * kDVS; p += kDT - 32) {
-                const int t = p / kDVS, j = p % kDVS;
-                float a0 = 0.f, a1 = 0.f;
-                for (int u = t; u < kDC; ++u) a0 = fmaf(c.Am[u * kPC + t], c.dOs[u * kPV + j], a0);
-                for (int cc = 0; cc < DK; ++cc) a1 = fmaf(c.kl(t, cc), c.Hs[j * PK + cc], a1);
-                c.dEs[t * kPV + j] = a0 + a1;
-            }
+            const float *src = states + ((bh * nch + ch) * DV + j0) * (size_t)DK;
+            for (int p = tid; p < kDVS * DK; p += kDT) c.Ss[(p / DK) * PK + p % DK] = src[p];
+            load_tile(q, rr, DK, 0, DK, n, c.Qs, PK);
+            load_tile(k, rr, DK, 0, DK, n, c.Ks, PK);
+            load_tile(v, rr, DV, j0, kDVS, n, c.Vs, kPV);
+            load_tile(dO, rr, DV, j0, kDVS, n, c.dOs, kPV);
         }
+        if (tid < DK) c.col1[tid] = 0.f;
+        if (tid < kDC) c.dbl[tid] = c.dbs[tid] = c.dls[tid] = 0.f;
         __syncthreads();
-        wy_factors(c);
+        if (tid >= 32 && tid < 32 + DK) {   // colsum(S o H^T), while warp 0 scans the gates
+            const int cc = tid - 32;
+            float s = 0.f;
+            for (int j = 0; j < kDVS; ++j) s = fmaf(c.Ss[j * PK + cc], c.Hs[j * PK + cc], s);
+            c.col2[cc] = s;
+        }
+        if constexpr (kStage) {
+            load_gates(c, gate ? c.sg : nullptr, c.sb, n, true);
+            if (ch > 0) stage(ch - 1);   // the staging buffers have been read
+        } else {
+            load_gates(c, gate ? gate + rr * GW : nullptr, beta + rr, n, true);
+        }
+        grams<MODE, DK, SP>(c, true);
         __syncthreads();
-        new_values(c);
+        if (warp == 0) invert_unit_lower_32(c.Xm, c.Tm);
+        __syncthreads();
+        wy_factors<MODE, DK, SP>(c, true);   // W, U, dE = A^T dO + Kl H
+        __syncthreads();
+        new_values<MODE, DK, SP>(c);         // E = U - W S^T
         __syncthreads();
 
         {   // T^T dE (-> dv), dA = tril(dO E^T), dW = -dE S
-            float td[4][1] = {}, da[4][1] = {}, dw[4][NK] = {};
-            tile_mma<4, 1, kDC>(td, r0, lane, [&](int t, int u) { return c.Tm[u * kPC + t]; },
-                                [&](int u, int j) { return c.dEs[u * kPV + j]; });
-            tile_mma<4, 1, kDVS>(da, r0, lane, [&](int t, int i) { return c.dOs[t * kPV + i]; },
-                                 [&](int i, int j) { return c.Es[j * kPV + i]; });
-            tile_mma<4, NK, kDVS>(dw, r0, lane, [&](int t, int j) { return c.dEs[t * kPV + j]; },
-                                  [&](int j, int cc) { return c.Ss[j * PK + cc]; });
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int t = r0 + i;
-                c.TdE[t * kPV + lane] = td[i][0];
-                if (t < n) dv[(r + t) * DV + j0 + lane] = from_f32<IO>(c.bet[t] * td[i][0]);
-                c.dAm[t * kPC + lane] = lane <= t ? da[i][0] : 0.f;
-#pragma unroll
-                for (int nn = 0; nn < NK; ++nn) c.dWm[t * PK + lane + 32 * nn] = -dw[i][nn];
-            }
+            float td[1][4] = {}, da[1][4] = {}, dw[NK][4] = {};
+            warp_mma<1, kDC, SP>(td, o.m0, o.n32, [&](int t, int u) { return c.Tm[u * kPC + t]; },
+                                 [&](int u, int j) { return c.dEs[u * kPV + j]; });
+            frag_each(td, o.m0, o.n32, [&](float &x, int t, int j) {
+                c.TdE[t * kPV + j] = x;
+                if (t < n) dv[(rr + t) * DV + j0 + j] = from_f32<IO>(c.bet[t] * x);
+            });
+            warp_mma<1, kDVS, SP>(da, o.m0, o.n32, [&](int t, int i) { return c.dOs[t * kPV + i]; },
+                                  [&](int i, int j) { return c.Es[j * kPV + i]; });
+            frag_each(da, o.m0, o.n32, [&](float &x, int t, int j) { c.dAm[t * kPC + j] = j <= t ? x : 0.f; });
+            warp_mma<NK, kDVS, SP>(dw, o.m0, o.nk, [&](int t, int j) { return c.dEs[t * kPV + j]; },
+                                   [&](int j, int cc) { return c.Ss[j * PK + cc]; });
+            frag_each(dw, o.m0, o.nk, [&](float &x, int t, int cc) { c.dWm[t * PK + cc] = -x; });
         }
         __syncthreads();
-        float tdw[4][NK] = {};
-        {   // dT = (dW (diag(b)Kg)^T + dE (diag(b)V)^T), strictly lower; T^T dW (held)
-            float dt[4][1] = {};
-            tile_mma<4, 1, DK>(dt, r0, lane, [&](int t, int cc) { return c.dWm[t * PK + cc]; },
-                               [&](int cc, int u) { return c.kg(u, cc); });
-            tile_mma<4, 1, kDVS>(dt, r0, lane, [&](int t, int j) { return c.dEs[t * kPV + j]; },
-                                 [&](int j, int u) { return c.Vs[u * kPV + j]; });
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int t = r0 + i;
-                c.dTm[t * kPC + lane] = lane < t ? c.bet[lane] * dt[i][0] : 0.f;
-            }
-            tile_mma<4, NK, kDC>(tdw, r0, lane, [&](int t, int u) { return c.Tm[u * kPC + t]; },
-                                 [&](int u, int cc) { return c.dWm[u * PK + cc]; });
+        float tdw[NK][4] = {};
+        {   // dT = dW (diag(b)Kg)^T + dE (diag(b)V)^T, strictly lower; T^T dW (held)
+            float dt[1][4] = {};
+            warp_mma<1, DK, SP>(dt, o.m0, o.n32, [&](int t, int cc) { return c.dWm[t * PK + cc]; },
+                                [&](int cc, int u) { return c.kg(u, cc); });
+            warp_mma<1, kDVS, SP>(dt, o.m0, o.n32, [&](int t, int j) { return c.dEs[t * kPV + j]; },
+                                  [&](int j, int u) { return c.Vs[u * kPV + j]; });
+            frag_each(dt, o.m0, o.n32,
+                      [&](float &x, int t, int u) { c.dTm[t * kPC + u] = u < t ? c.bet[u] * x : 0.f; });
+            warp_mma<NK, kDC, SP>(tdw, o.m0, o.nk, [&](int t, int u) { return c.Tm[u * kPC + t]; },
+                                  [&](int u, int cc) { return c.dWm[u * PK + cc]; });
         }
         __syncthreads();
         {   // X = dT T^T (over Lm, no longer needed); T^T dW over dW
-            float x[4][1] = {};
-            tile_mma<4, 1, kDC>(x, r0, lane, [&](int t, int u) { return c.dTm[t * kPC + u]; },
-                                [&](int u, int j) { return c.Tm[j * kPC + u]; });
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                c.Xm[(r0 + i) * kPC + lane] = x[i][0];
-#pragma unroll
-                for (int nn = 0; nn < NK; ++nn) c.dWm[(r0 + i) * PK + lane + 32 * nn] = tdw[i][nn];
-            }
+            float x[1][4] = {};
+            warp_mma<1, kDC, SP>(x, o.m0, o.n32, [&](int t, int u) { return c.dTm[t * kPC + u]; },
+                                 [&](int u, int j) { return c.Tm[j * kPC + u]; });
+            frag_each(x, o.m0, o.n32, [&](float &val, int t, int j) { c.Xm[t * kPC + j] = val; });
+            frag_each(tdw, o.m0, o.nk, [&](float &val, int t, int cc) { c.dWm[t * PK + cc] = val; });
         }
         __syncthreads();
         {   // dLm = -T^T X (strictly lower); BL = diag(b) dLm; mode 2 folds Gam into BL and dA
-            float y[4][1] = {};
-            tile_mma<4, 1, kDC>(y, r0, lane, [&](int t, int u) { return c.Tm[u * kPC + t]; },
-                                [&](int u, int j) { return c.Xm[u * kPC + j]; });
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int t = r0 + i;
-                const float dlm = lane < t ? -y[i][0] : 0.f;
-                float part = dlm * c.Km[t * kPC + lane];
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-                if (lane == 0) c.dbl[t] = part;
-                const float gm = MODE == 3 ? 1.f : c.Gm[t * kPC + lane];
-                c.BL[t * kPC + lane] = c.bet[t] * dlm * gm;
-                if (MODE != 3) c.dAm[t * kPC + lane] *= gm;
-            }
+            float y[1][4] = {};
+            warp_mma<1, kDC, SP>(y, o.m0, o.n32, [&](int t, int u) { return c.Tm[u * kPC + t]; },
+                                 [&](int u, int j) { return c.Xm[u * kPC + j]; });
+            float part[2] = {0.f, 0.f};
+            frag_each(y, o.m0, o.n32, [&](float &val, int t, int j) {
+                const float dlm = j < t ? -val : 0.f;
+                part[(t - o.m0) >> 3] += dlm * c.Km[t * kPC + j];
+                const float gm = MODE == 3 ? 1.f : c.Gm[t * kPC + j];
+                c.BL[t * kPC + j] = c.bet[t] * dlm * gm;
+                if (MODE != 3) c.dAm[t * kPC + j] *= gm;
+            });
+            rows_add(part, c.dbl, o.m0);
         }
         // (E H^T)-terms and the carried cotangent, both from H at the chunk's end
-        float dkn[4][NK] = {}, hn[4][NK] = {};
-        tile_mma<4, NK, kDVS>(dkn, r0, lane, [&](int t, int j) { return c.Es[t * kPV + j]; },
-                              [&](int j, int cc) { return c.Hs[j * PK + cc]; });
+        float dkn[NK][4] = {}, hn[NK][4] = {};
+        warp_mma<NK, kDVS, SP>(dkn, o.m0, o.nk, [&](int t, int j) { return c.Es[t * kPV + j]; },
+                               [&](int j, int cc) { return c.Hs[j * PK + cc]; });
+        frag_each(dkn, o.m0, o.nk, [&](float &x, int t, int cc) { x *= c.decf(t, cc, last); });
 #pragma unroll
-        for (int nn = 0; nn < NK; ++nn) {
-            const int cc = lane + 32 * nn;
-            float s = 0.f;
+        for (int nt = 0; nt < NK; ++nt)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                dkn[i][nn] *= c.decf(r0 + i, cc, last);
-                s = fmaf(c.Ks[(r0 + i) * PK + cc], dkn[i][nn], s);
+            for (int h = 0; h < 2; ++h) {   // column sums of k o (g_L / g)(E H^T)
+                const int cc = o.nk + 8 * nt + 2 * t4 + h;
+                float s = fmaf(c.Ks[(o.m0 + g8) * PK + cc], dkn[nt][h],
+                               c.Ks[(o.m0 + g8 + 8) * PK + cc] * dkn[nt][2 + h]);
+                s += __shfl_xor_sync(0xffffffffu, s, 4);
+                s += __shfl_xor_sync(0xffffffffu, s, 8);
+                s += __shfl_xor_sync(0xffffffffu, s, 16);
+                if (g8 == 0) atomicAdd(&c.col1[cc], s);
             }
-            atomicAdd(&c.col1[cc], s);
-        }
-        if (tid < DK) {
-            float s = 0.f;
-            for (int j = 0; j < kDVS; ++j) s = fmaf(c.Ss[j * PK + tid], c.Hs[j * PK + tid], s);
-            c.col2[tid] = s;
-        }
-        {
-            float h2[4][NK] = {};
-            tile_mma<4, NK, kDC>(hn, r0, lane, [&](int j, int t) { return c.dOs[t * kPV + j]; },
-                                 [&](int t, int cc) { return c.qg(t, cc); });
-            tile_mma<4, NK, kDC>(h2, r0, lane, [&](int j, int t) { return c.dEs[t * kPV + j]; },
-                                 [&](int t, int cc) { return c.Wm[t * PK + cc]; });
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int nn = 0; nn < NK; ++nn) {
-                    const int cc = lane + 32 * nn;
-                    hn[i][nn] = fmaf(c.gl[cc], c.Hs[(r0 + i) * PK + cc], hn[i][nn] - h2[i][nn]);
-                }
+        {   // dL/dS^T = Qg^T dO + diag(g_L) H - W^T dE  (rows j of this slice)
+            float h2[NK][4] = {};
+            warp_mma<NK, kDC, SP>(hn, o.m0, o.nk, [&](int j, int t) { return c.dOs[t * kPV + j]; },
+                                  [&](int t, int cc) { return c.qg(t, cc); });
+            warp_mma<NK, kDC, SP>(h2, o.m0, o.nk, [&](int j, int t) { return c.dEs[t * kPV + j]; },
+                                  [&](int t, int cc) { return c.Wm[t * PK + cc]; });
+            frag_each2(hn, h2, o.m0, o.nk, [&](float &x, float &y, int j, int cc) {
+                x = fmaf(c.gl[cc], c.Hs[j * PK + cc], x - y);
+            });
         }
         __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int nn = 0; nn < NK; ++nn) c.Hs[(r0 + i) * PK + lane + 32 * nn] = hn[i][nn];
+        frag_each(hn, o.m0, o.nk, [&](float &x, int j, int cc) { c.Hs[j * PK + cc] = x; });
 
         // dq, dk_plus, dk_minus
-        float dq[4][NK] = {}, dkp[4][NK] = {};
-        tile_mma<4, NK, kDVS>(dq, r0, lane, [&](int t, int j) { return c.dOs[t * kPV + j]; },
-                              [&](int j, int cc) { return c.Ss[j * PK + cc]; });
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int nn = 0; nn < NK; ++nn) {
-                const int t = r0 + i, cc = lane + 32 * nn;
-                const float gtc = c.gf(t, cc);
-                dq[i][nn] *= gtc;
-                dkp[i][nn] = c.bet[t] * gtc * c.dWm[t * PK + cc];
-            }
+        float dq[NK][4] = {}, dkp[NK][4] = {};
+        warp_mma<NK, kDVS, SP>(dq, o.m0, o.nk, [&](int t, int j) { return c.dOs[t * kPV + j]; },
+                               [&](int j, int cc) { return c.Ss[j * PK + cc]; });
+        frag_each2(dq, dkp, o.m0, o.nk, [&](float &x, float &y, int t, int cc) {
+            const float gtc = c.gf(t, cc);
+            x *= gtc;
+            y = c.bet[t] * gtc * c.dWm[t * PK + cc];
+        });
         if constexpr (MODE == 3) {
-            gam_rows<DK>(dq, r0, lane, c.Lg, c.Ks, [&](int t, int j) { return c.dAm[t * kPC + j]; });
-            gam_rows<DK>(dkp, r0, lane, c.Lg, c.Ks, [&](int t, int j) { return c.BL[t * kPC + j]; });
-            gam_cols<DK>(dkn, r0, lane, c.Lg, c.Qs, [&](int u, int t) { return c.dAm[u * kPC + t]; });
-            gam_cols<DK>(dkn, r0, lane, c.Lg, c.Ks, [&](int u, int t) { return c.BL[u * kPC + t]; });
+            gam_rows<NK, DK>(dq, o.m0, o.nk, c.Lg, c.Ks, [&](int t, int j) { return c.dAm[t * kPC + j]; });
+            gam_rows<NK, DK>(dkp, o.m0, o.nk, c.Lg, c.Ks, [&](int t, int j) { return c.BL[t * kPC + j]; });
+            gam_cols<NK, DK>(dkn, o.m0, o.nk, c.Lg, c.Qs, [&](int u, int t) { return c.dAm[u * kPC + t]; });
+            gam_cols<NK, DK>(dkn, o.m0, o.nk, c.Lg, c.Ks, [&](int u, int t) { return c.BL[u * kPC + t]; });
         } else {
-            tile_mma<4, NK, kDC>(dq, r0, lane, [&](int t, int j) { return c.dAm[t * kPC + j]; },
-                                 [&](int j, int cc) { return c.Ks[j * PK + cc]; });
-            tile_mma<4, NK, kDC>(dkp, r0, lane, [&](int t, int j) { return c.BL[t * kPC + j]; },
-                                 [&](int j, int cc) { return c.Ks[j * PK + cc]; });
-            tile_mma<4, NK, kDC>(dkn, r0, lane, [&](int t, int u) { return c.dAm[u * kPC + t]; },
-                                 [&](int u, int cc) { return c.Qs[u * PK + cc]; });
-            tile_mma<4, NK, kDC>(dkn, r0, lane, [&](int t, int u) { return c.BL[u * kPC + t]; },
-                                 [&](int u, int cc) { return c.Ks[u * PK + cc]; });
+            warp_mma<NK, kDC, SP>(dq, o.m0, o.nk, [&](int t, int j) { return c.dAm[t * kPC + j]; },
+                                  [&](int j, int cc) { return c.Ks[j * PK + cc]; });
+            warp_mma<NK, kDC, SP>(dkp, o.m0, o.nk, [&](int t, int j) { return c.BL[t * kPC + j]; },
+                                  [&](int j, int cc) { return c.Ks[j * PK + cc]; });
+            warp_mma<NK, kDC, SP>(dkn, o.m0, o.nk, [&](int t, int u) { return c.dAm[u * kPC + t]; },
+                                  [&](int u, int cc) { return c.Qs[u * PK + cc]; });
+            warp_mma<NK, kDC, SP>(dkn, o.m0, o.nk, [&](int t, int u) { return c.BL[u * kPC + t]; },
+                                  [&](int u, int cc) { return c.Ks[u * PK + cc]; });
         }
-        __syncthreads();   // col1 complete
+        __syncthreads();   // col1, col2 and dbl complete
 
-        // this slice's shares of dq, dk, dL/dlam and db, added into the fp32 accumulators
+        {   // this slice's shares of dq, dk, dL/dlam and db, into the fp32 accumulators
+            float pdb[2] = {0.f, 0.f}, pdl[2] = {0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = r0 + i;
-            float dbs = 0.f, dls = 0.f;
+            for (int nt = 0; nt < NK; ++nt)
 #pragma unroll
-            for (int nn = 0; nn < NK; ++nn) {
-                const int cc = lane + 32 * nn;
-                const float qv = c.Qs[t * PK + cc], kv = c.Ks[t * PK + cc];
-                float dl = fmaf(qv, dq[i][nn], kv * (dkp[i][nn] - dkn[i][nn]));
-                if (t == last) dl += c.col1[cc] + c.gl[cc] * c.col2[cc];
-                dbs = fmaf(c.kg(t, cc), c.dWm[t * PK + cc], dbs);
-                if (t < n) {
-                    atomicAdd(&dq_acc[(r + t) * DK + cc], dq[i][nn]);
-                    atomicAdd(&dk_acc[(r + t) * DK + cc], dkp[i][nn] + dkn[i][nn]);
-                    if constexpr (DL > 1) atomicAdd(&dl_acc[(r + t) * DL + cc], dl);
+                for (int h = 0; h < 2; ++h) {   // elements 2h, 2h+1: row t, columns cc, cc + 1
+                    const int t = o.m0 + g8 + 8 * h, cc = o.nk + 8 * nt + 2 * t4;
+                    float dl[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int r = 2 * h + e, ce = cc + e;
+                        dl[e] = fmaf(c.Qs[t * PK + ce], dq[nt][r], c.Ks[t * PK + ce] * (dkp[nt][r] - dkn[nt][r]));
+                        if (t == last) dl[e] += c.col1[ce] + c.gl[ce] * c.col2[ce];
+                        pdb[h] = fmaf(c.kg(t, ce), c.dWm[t * PK + ce], pdb[h]);
+                        pdl[h] += dl[e];
+                    }
+                    if (t < n) {
+                        const size_t e0 = (rr + t) * DK + cc;
+                        red_add2(dq_acc + e0, dq[nt][2 * h], dq[nt][2 * h + 1]);
+                        red_add2(dk_acc + e0, dkp[nt][2 * h] + dkn[nt][2 * h], dkp[nt][2 * h + 1] + dkn[nt][2 * h + 1]);
+                        if constexpr (DL > 1) red_add2(dl_acc + e0, dl[0], dl[1]);
+                    }
                 }
-                dls += dl;
-            }
-            dbs = fmaf(c.Vs[t * kPV + lane], c.TdE[t * kPV + lane], dbs);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                dbs += __shfl_xor_sync(0xffffffffu, dbs, off);
-                if constexpr (DL == 1) dls += __shfl_xor_sync(0xffffffffu, dls, off);
-            }
-            if (lane == 0 && t < n) {
-                atomicAdd(&db_acc[r + t], dbs + c.dbl[t]);
-                if constexpr (DL == 1) atomicAdd(&dl_acc[r + t], dls);
-            }
+            rows_add(pdb, c.dbs, o.m0);
+            if constexpr (DL == 1) rows_add(pdl, c.dls, o.m0);
+        }
+        __syncthreads();
+        if (tid < n) {
+            float p2 = 0.f;
+            for (int j = 0; j < kDVS; ++j) p2 = fmaf(c.Vs[tid * kPV + j], c.TdE[tid * kPV + j], p2);
+            atomicAdd(&db_acc[rr + tid], c.dbs[tid] + p2 + c.dbl[tid]);
+            if constexpr (DL == 1) atomicAdd(&dl_acc[rr + tid], c.dls[tid]);
         }
         __syncthreads();
     }
