@@ -18,16 +18,20 @@
 // The last identity follows from differentiating the decay mask exp(lam_s - lam_j): lam_u
 // enters with + where it is the reading position and with - where it is the written one.
 //
-// fp32 arithmetic on CUDA cores, 256 threads per CTA and one or two CTAs per (batch, head)
-// (the d_k columns of S and G split between them): a forward sweep stores every chunk-start
-// state in the caller's workspace, then a reverse sweep carries G back through the chunks;
-// a small kernel finishes dV and the gate gradient.  Tiles live in shared memory with one
-// float of row padding; the products are register-tiled (a thread holds up to 16 x 4
-// outputs), so that each shared load feeds several FMAs.
-#include "bwd_util.cuh"
+// One or two CTAs per (batch, head) (the d_k columns of S and G split between them): a
+// forward sweep stores every chunk-start state in the caller's workspace, then a reverse
+// sweep carries G back through the chunks; a small kernel finishes dV and the gate gradient.
+// The products run on the tensor cores as warp-level mma (m16n8k8, tf32 operands, fp32
+// accumulate; each operand is split into a tf32 part and a remainder, three products,
+// fp32 accuracy): the tiles are 32 x 32 to 128 x 64, too small for tcgen05's
+// 128-row tiles and each followed by an element-wise step.  With bf16 I/O the next chunk's
+// inputs (and, in the reverse sweep, its start state) arrive by cp.async while the current
+// chunk is processed.
 #include "la_internal.cuh"
+#include "bwd_util.cuh"
 
 #include <cfloat>
+#include <type_traits>
 
 namespace la {
 namespace {
@@ -39,15 +43,18 @@ constexpr int kBwdC = 32;
 // columns of S and G, the products that stay within columns (dQ, dK, the state and G
 // updates), and a share of those that sum over them (dV, dlam), which it adds into fp32
 // accumulators in the workspace; a finishing kernel converts dV and takes the suffix sums.
-template <int DK, int DV, int SPLIT>
+// Row pitches are 4 (mod 32) floats (conflict-free mma operand loads).
+template <int DK, int DV, int SPLIT, bool STAGE>
 struct BwdSmem {
     static constexpr int DKH = DK / SPLIT;
-    static constexpr int kS = DV * (DKH + 1);
-    static constexpr int kQ = kBwdC * (DK + 1);
-    static constexpr int kV = kBwdC * (DV + 1);
-    static constexpr int kP = kBwdC * (kBwdC + 1);
-    static constexpr int kFloats = 2 * kS + 2 * kQ + 2 * kV + 2 * kP + 4 * kBwdC + 8;
+    static constexpr int PQ = DK + 4, PV = DV + 4, PS = DKH + 4, PC = kBwdC + 4;
+    static constexpr int kQ = kBwdC * PQ, kV = kBwdC * PV, kS = DV * PS, kP = kBwdC * PC;
+    // staged raw bf16 rows of q, k, v, dO (2 bytes each: C (2 DK + 2 DV) / 2 floats)
+    static constexpr int kRaw = STAGE ? kBwdC * (DK + DV) : 0;
+    // Qs Ks | Vs dOs | S, S' (double buffer), G | P dP | raw | lam gv dec dl graw | red
+    static constexpr int kFloats = 2 * kQ + 2 * kV + 3 * kS + 2 * kP + kRaw + 5 * kBwdC + 8;
     static constexpr size_t kBytes = sizeof(float) * kFloats;
+    static_assert(kBytes <= 227 * 1024, "shared memory");
 };
 template <int DK>
 constexpr int bwd_split() { return DK == 128 ? 2 : 1; }
@@ -64,6 +71,10 @@ __device__ __forceinline__ float block_sum(float x, float *red) {
     return s;
 }
 
+// fragment coordinates of warp_mma's element r of n-tile nt (bwd_util.cuh)
+__device__ __forceinline__ int frow(int m0, int r) { return m0 + ((threadIdx.x & 31) >> 2) + 8 * (r >> 1); }
+__device__ __forceinline__ int fcol(int n0, int nt, int r) { return n0 + 8 * nt + 2 * (threadIdx.x & 3) + (r & 1); }
+
 template <int DK, int DV, int SPLIT, typename IO>
 __global__ void __launch_bounds__(kBwdThreads)
 backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__restrict__ k,
@@ -72,28 +83,41 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
                 const float *__restrict__ dST, IO *__restrict__ dq, IO *__restrict__ dk,
                 float *__restrict__ dS0, float *__restrict__ ws, float *__restrict__ dv_acc,
                 float *__restrict__ dl_acc) {
-    using L = BwdSmem<DK, DV, SPLIT>;
-    constexpr int C = kBwdC, DKH = L::DKH, SK = DK + 1, SV = DV + 1, SH = DKH + 1, SP = C + 1;
-    constexpr int NW = kBwdThreads / 32;       // 8 warps
-    constexpr int RC = C / NW;                 // chunk rows per warp (4)
-    constexpr int RS = DV / NW;                // state rows per warp (16 or 8)
-    constexpr int NK = DKH / 32, NV = DV / 32; // columns per lane
+    constexpr bool STAGE = std::is_same<IO, __nv_bfloat16>::value;
+    // Operand splitting (bwd_util.cuh): computed operands (S, G, P, dP, scaled rows) are
+    // always split -- the gate gradient is a suffix sum over the whole sequence, where one
+    // tf32 rounding per product adds up; the inputs q, k, v, dO are split only for fp32 I/O
+    // (bf16 values are exact in tf32).
+    constexpr bool SP = std::is_same<IO, float>::value;
+    using L = BwdSmem<DK, DV, SPLIT, STAGE>;
+    constexpr int C = kBwdC, DKH = L::DKH, PQ = L::PQ, PV = L::PV, PS = L::PS, PC = L::PC;
+    constexpr int NW = kBwdThreads / 32;
+    // DV x DKH state tiles: DV / 16 row blocks of 16, the warps left over split the columns
+    constexpr int RB = DV / 16, CG = NW / RB, NTS = DKH / 8 / CG;
+    constexpr int NTQ = DKH / 32;             // C x DKH: rows 16 (w & 1), columns (DKH / 4)(w >> 1)
+    constexpr int NTV = DV / 32;              // C x DV:  rows 16 (w & 1), columns (DV / 4)(w >> 1)
+    static_assert(NW % RB == 0 && DKH % (8 * CG) == 0, "state partition");
     extern __shared__ float smem[];
-    float *S = smem;             // [DV][DKH+1]  state (forward) / chunk-start state (reverse)
-    float *G = S + L::kS;        // [DV][DKH+1]  dL/dS at the chunk's end
-    float *Qs = G + L::kS;       // [C][DK+1]
-    float *Ks = Qs + L::kQ;      // [C][DK+1]
-    float *Vs = Ks + L::kQ;      // [C][DV+1]
-    float *dOs = Vs + L::kV;     // [C][DV+1]
-    float *P = dOs + L::kV;      // [C][C+1]
-    float *dP = P + L::kP;       // [C][C+1]
-    float *lam = dP + L::kP;     // [C]   in-chunk log-gate prefix
-    float *gv = lam + C;         // [C]   g_t = exp(lam_t)
-    float *dec = gv + C;         // [C]   g_L / g_t
-    float *dl = dec + C;         // [C]   this CTA's share of dlam
-    float *red = dl + C;         // [8]
+    float *Qs = smem;                // [C][PQ]
+    float *Ks = Qs + L::kQ;          // [C][PQ]
+    float *Vs = Ks + L::kQ;          // [C][PV]
+    float *dOs = Vs + L::kV;         // [C][PV]
+    float *Sb0 = dOs + L::kV;        // [DV][PS]  chunk-start state (two buffers, reverse)
+    float *Sb1 = Sb0 + L::kS;
+    float *G = Sb1 + L::kS;          // [DV][PS]  dL/dS at the chunk's end
+    float *P = G + L::kS;            // [C][PC]
+    float *dP = P + L::kP;           // [C][PC]
+    float *raw = dP + L::kP;         // staged q | k | v | dO rows (bf16)
+    float *lam = raw + L::kRaw;      // [C]   in-chunk log-gate prefix
+    float *gv = lam + C;             // [C]   g_t = exp(lam_t)
+    float *dec = gv + C;             // [C]   g_L / g_t
+    float *dl = dec + C;             // [C]   this CTA's share of dlam
+    float *graw = dl + C;            // [C]   staged gates
+    float *red = graw + C;           // [8]
+    __nv_bfloat16 *rq = reinterpret_cast<__nv_bfloat16 *>(raw);
+    __nv_bfloat16 *rk = rq + C * DK, *rv = rk + C * DK, *rdo = rv + C * DV;
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5;
     const size_t bh = blockIdx.x / SPLIT;
     const int kh = blockIdx.x % SPLIT, c0 = kh * DKH;   // this CTA's columns c0 .. c0 + DKH
     const int nch = (T + C - 1) / C;
@@ -101,186 +125,240 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
     const float *gh = gate ? (gate_heads ? gate + bh % gate_heads : gate + row0) : nullptr;
     const int gt = gate_heads ? 0 : 1;
     float *wsh = ws + (size_t)blockIdx.x * (nch + 1) * DV * DKH;
+    const int mq = 16 * (warp & 1), n32 = 8 * (warp >> 1), nq = (DKH / 4) * (warp >> 1),
+              nv = (DV / 4) * (warp >> 1);
+    const int ms = 16 * (warp % RB), ns = (DKH / CG) * (warp / RB);
 
-    auto load_gates = [&](int t0, int Lc) {
-        if (tid < C) lam[tid] = (gh && tid < Lc) ? logf(fmaxf(gh[(size_t)(t0 + tid) * gt], FLT_MIN)) : 0.f;
-        __syncthreads();
-        if (tid == 0)
-            for (int i = 1; i < C; ++i) lam[i] += lam[i - 1];
-        __syncthreads();
-        if (tid < C) {
-            gv[tid] = expf(lam[tid]);
-            dec[tid] = expf(lam[Lc - 1] - lam[tid]);
+    // gates of chunk t0 (Lc tokens): from the staged copy or global memory
+    auto load_gates = [&](int t0, int Lc, bool staged) {
+        if (warp == 0) {
+            const int lane = tid & 31;
+            float a = 1.f;
+            if (gh && lane < Lc) a = staged && gt ? graw[lane] : gh[(size_t)(t0 + lane) * gt];
+            float x = lane < Lc ? logf(fmaxf(a, FLT_MIN)) : 0.f;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += y;
+            }
+            const float xl = __shfl_sync(0xffffffffu, x, Lc - 1);
+            lam[lane] = x;
+            gv[lane] = expf(x);
+            dec[lane] = expf(xl - x);
         }
-        __syncthreads();
     };
-    auto load_rows = [&](const IO *src, float *dst, int t0, int Lc, int d, int stride) {
+    // stage chunk c's rows (k, v; with `rev` also q, dO) and gates
+    auto stage = [&](int c, bool rev) {
+        const int t0 = c * C, Lc = min(C, T - t0);
+        stage_rows<kBwdThreads>(rk, k + (row0 + t0) * DK, DK, DK, Lc);
+        stage_rows<kBwdThreads>(rv, v + (row0 + t0) * DV, DV, DV, Lc);
+        if (rev) {
+            stage_rows<kBwdThreads>(rq, q + (row0 + t0) * DK, DK, DK, Lc);
+            stage_rows<kBwdThreads>(rdo, dO + (row0 + t0) * DV, DV, DV, Lc);
+        }
+        if (gh && gt && tid >= 64 && tid - 64 < Lc) cp_async4(graw + tid - 64, gh + t0 + tid - 64);
+        cp_async_commit();
+    };
+    auto load_direct = [&](const IO *src, float *dst, int t0, int Lc, int d, int pitch) {
         for (int p = tid; p < C * d; p += kBwdThreads) {
             const int i = p / d, j = p % d;
-            dst[i * stride + j] = i < Lc ? to_f32(src[(row0 + t0 + i) * d + j]) : 0.f;
+            dst[i * pitch + j] = i < Lc ? to_f32(src[(row0 + t0 + i) * d + j]) : 0.f;
         }
     };
-    auto st_idx = [&](int p) { return (p / DKH) * SH + p % DKH; };       // p over DV x DKH
-    auto gl_idx = [&](int p) { return (p / DKH) * DK + c0 + p % DKH; };  // into [DV][DK]
 
     // ---- forward sweep: chunk-start states (this CTA's columns) into the workspace
-    for (int p = tid; p < DV * DKH; p += kBwdThreads) S[st_idx(p)] = S0 ? S0[bh * DV * DK + gl_idx(p)] : 0.f;
+    float *S = Sb0;
+    for (int p = tid; p < DV * DKH; p += kBwdThreads)
+        S[(p / DKH) * PS + p % DKH] = S0 ? S0[bh * DV * DK + (p / DKH) * DK + c0 + p % DKH] : 0.f;
+    if constexpr (STAGE) stage(0, false);
     __syncthreads();
     for (int c = 0; c <= nch; ++c) {
-        for (int p = tid; p < DV * DKH; p += kBwdThreads) wsh[(size_t)c * DV * DKH + p] = S[st_idx(p)];
+        for (int p = tid; p < DV * DKH / 4; p += kBwdThreads) {   // store S (float4)
+            const int i = p / (DKH / 4), j = 4 * (p % (DKH / 4));
+            *reinterpret_cast<float4 *>(wsh + (size_t)c * DV * DKH + i * DKH + j) =
+                *reinterpret_cast<const float4 *>(S + i * PS + j);
+        }
         if (c == nch) break;
         const int t0 = c * C, Lc = min(C, T - t0);
-        load_rows(k, Ks, t0, Lc, DK, SK);
-        load_rows(v, Vs, t0, Lc, DV, SV);
-        load_gates(t0, Lc);   // (synchronises: every thread has stored S)
-        // S <- g_L S + sum_j (dec_j v_j) k_j^T
+        if constexpr (STAGE) {
+            cp_async_wait_all();
+            __syncthreads();
+            unstage<kBwdThreads, IO>(rk, C, DK, Lc, Ks, PQ);
+            unstage<kBwdThreads, IO>(rv, C, DV, Lc, Vs, PV);
+        } else {
+            load_direct(k, Ks, t0, Lc, DK, PQ);
+            load_direct(v, Vs, t0, Lc, DV, PV);
+        }
+        load_gates(t0, Lc, STAGE);
+        __syncthreads();
+        if constexpr (STAGE) if (c + 1 < nch) stage(c + 1, false);
+        // S <- g_L S + (dec o V)^T K   (this CTA's columns; state partition)
         const float gL = gv[Lc - 1];
-        float acc[RS][NK] = {};
-        tile_mma<RS, NK, C>(acc, RS * warp, lane, [&](int i, int j) { return dec[j] * Vs[j * SV + i]; },
-                            [&](int j, int cc) { return Ks[j * SK + c0 + cc]; });
+        float acc[NTS][4] = {};
+        warp_mma<NTS, C, true, SP>(acc, ms, ns, [&](int i, int j) { return dec[j] * Vs[j * PV + i]; },
+                             [&](int j, int cc) { return Ks[j * PQ + c0 + cc]; });
 #pragma unroll
-        for (int i = 0; i < RS; ++i)
+        for (int nt = 0; nt < NTS; ++nt)
 #pragma unroll
-            for (int n = 0; n < NK; ++n) {
-                float &x = S[(RS * warp + i) * SH + lane + 32 * n];
-                x = fmaf(gL, x, acc[i][n]);
+            for (int r = 0; r < 4; ++r) {
+                float &x = S[frow(ms, r) * PS + fcol(ns, nt, r)];
+                x = fmaf(gL, x, acc[nt][r]);
             }
         __syncthreads();
     }
-    __syncthreads();
 
     // ---- reverse sweep
     // S holds this CTA's columns of S_T: its share of <dS_T, S_T> (dlam at the last token)
-    float part = 0.f;
+    float part0 = 0.f;
     for (int p = tid; p < DV * DKH; p += kBwdThreads) {
-        const float g0 = dST ? dST[bh * DV * DK + gl_idx(p)] : 0.f;
-        G[st_idx(p)] = g0;
-        part = fmaf(g0, S[st_idx(p)], part);
+        const int i = p / DKH, j = p % DKH;
+        const float g0 = dST ? dST[bh * DV * DK + i * DK + c0 + j] : 0.f;
+        G[i * PS + j] = g0;
+        part0 = fmaf(g0, S[i * PS + j], part0);
     }
-    const float final_dot = block_sum(part, red);
+    const float final_dot = block_sum(part0, red);
     if (tid == 0 && final_dot != 0.f) atomicAdd(&dl_acc[row0 + T - 1], final_dot);
+    float *Sc = (S == Sb0) ? Sb1 : Sb0;   // the chunk's start state
+    float *Sn = S;                        // the next (earlier) chunk's, staged meanwhile
+    auto stage_state = [&](int c, float *dst) {
+        const float *src = wsh + (size_t)c * DV * DKH;
+        for (int p = tid; p < DV * DKH / 4; p += kBwdThreads) {
+            const int i = p / (DKH / 4), j = 4 * (p % (DKH / 4));
+            cp_async16(dst + i * PS + j, src + i * DKH + j);
+        }
+    };
+    if constexpr (STAGE) {
+        __syncthreads();   // S_T read
+        stage_state(nch - 1, Sc);
+        stage(nch - 1, true);
+    }
     for (int c = nch - 1; c >= 0; --c) {
         const int t0 = c * C, Lc = min(C, T - t0);
-        load_rows(q, Qs, t0, Lc, DK, SK);
-        load_rows(k, Ks, t0, Lc, DK, SK);
-        load_rows(v, Vs, t0, Lc, DV, SV);
-        load_rows(dO, dOs, t0, Lc, DV, SV);
-        for (int p = tid; p < DV * DKH; p += kBwdThreads) S[st_idx(p)] = wsh[(size_t)c * DV * DKH + p];
+        if constexpr (STAGE) {
+            cp_async_wait_all();
+            __syncthreads();
+            unstage<kBwdThreads, IO>(rq, C, DK, Lc, Qs, PQ);
+            unstage<kBwdThreads, IO>(rk, C, DK, Lc, Ks, PQ);
+            unstage<kBwdThreads, IO>(rv, C, DV, Lc, Vs, PV);
+            unstage<kBwdThreads, IO>(rdo, C, DV, Lc, dOs, PV);
+        } else {
+            load_direct(q, Qs, t0, Lc, DK, PQ);
+            load_direct(k, Ks, t0, Lc, DK, PQ);
+            load_direct(v, Vs, t0, Lc, DV, PV);
+            load_direct(dO, dOs, t0, Lc, DV, PV);
+            const float *src = wsh + (size_t)c * DV * DKH;
+            for (int p = tid; p < DV * DKH; p += kBwdThreads) Sc[(p / DKH) * PS + p % DKH] = src[p];
+        }
         if (tid < C) dl[tid] = 0.f;
-        load_gates(t0, Lc);   // (synchronises)
-        const float gL = gv[Lc - 1];
-        // causal decayed score matrices P = (Q K^T) o D, dP = (dO V^T) o D (full rows)
-        for (int p = tid; p < C * C; p += kBwdThreads) {
-            const int t = p / C, j = p % C;
-            float pv = 0.f, dpv = 0.f;
-            if (t < Lc && j <= t) {
-                const float dd = expf(lam[t] - lam[j]);
-                float a1 = 0.f, a2 = 0.f;
-                for (int cc = 0; cc < DK; ++cc) a1 = fmaf(Qs[t * SK + cc], Ks[j * SK + cc], a1);
-                for (int i = 0; i < DV; ++i) a2 = fmaf(dOs[t * SV + i], Vs[j * SV + i], a2);
-                pv = a1 * dd;
-                dpv = a2 * dd;
+        load_gates(t0, Lc, STAGE);
+        __syncthreads();
+        if constexpr (STAGE) {
+            if (c > 0) {   // the staging buffers and Sn are free
+                stage_state(c - 1, Sn);
+                stage(c - 1, true);
             }
-            P[t * SP + j] = pv;
-            dP[t * SP + j] = dpv;
+        }
+        {   // causal decayed score matrices P = (Q K^T) o D, dP = (dO V^T) o D
+            float pp[1][4] = {}, dd[1][4] = {};
+            warp_mma<1, DK, SP>(pp, mq, n32, [&](int t, int cc) { return Qs[t * PQ + cc]; },
+                                [&](int cc, int j) { return Ks[j * PQ + cc]; });
+            warp_mma<1, DV, SP>(dd, mq, n32, [&](int t, int i) { return dOs[t * PV + i]; },
+                                [&](int i, int j) { return Vs[j * PV + i]; });
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int t = frow(mq, r), j = fcol(n32, 0, r);
+                const float w = (t < Lc && j <= t) ? expf(lam[t] - lam[j]) : 0.f;
+                P[t * PC + j] = pp[0][r] * w;
+                dP[t * PC + j] = dd[0][r] * w;
+            }
         }
         __syncthreads();
-        const int r0 = RC * warp;   // this warp's chunk rows
-        {   // dQ = diag(g) dO S_c + dP K   (this CTA's columns)
-            float acc[RC][NK] = {};
-            tile_mma<RC, NK, DV>(acc, r0, lane, [&](int t, int i) { return dOs[t * SV + i]; },
-                                 [&](int i, int cc) { return S[i * SH + cc]; });
+        {   // dQ = diag(g) dO S_c + dP K,  dK = dP^T Q + diag(g_L / g) V G  (this CTA's columns)
+            float aq[NTQ][4] = {}, ak[NTQ][4] = {};
+            warp_mma<NTQ, DV, SP, true>(aq, mq, nq, [&](int t, int i) { return dOs[t * PV + i]; },
+                                  [&](int i, int cc) { return Sc[i * PS + cc]; });
+            warp_mma<NTQ, DV, SP, true>(ak, mq, nq, [&](int t, int i) { return Vs[t * PV + i]; },
+                                  [&](int i, int cc) { return G[i * PS + cc]; });
 #pragma unroll
-            for (int i = 0; i < RC; ++i)
+            for (int nt = 0; nt < NTQ; ++nt)
 #pragma unroll
-                for (int n = 0; n < NK; ++n) acc[i][n] *= gv[r0 + i];
-            tile_mma<RC, NK, C>(acc, r0, lane, [&](int t, int j) { return dP[t * SP + j]; },
-                                [&](int j, int cc) { return Ks[j * SK + c0 + cc]; });
+                for (int r = 0; r < 4; ++r) {
+                    aq[nt][r] *= gv[frow(mq, r)];
+                    ak[nt][r] *= dec[frow(mq, r)];
+                }
+            warp_mma<NTQ, C, true, SP>(aq, mq, nq, [&](int t, int j) { return dP[t * PC + j]; },
+                                 [&](int j, int cc) { return Ks[j * PQ + c0 + cc]; });
+            warp_mma<NTQ, C, true, SP>(ak, mq, nq, [&](int t, int s2) { return dP[s2 * PC + t]; },
+                                 [&](int s2, int cc) { return Qs[s2 * PQ + c0 + cc]; });
+            float part[2] = {0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < RC; ++i) {
-                const int t = r0 + i;
-                float qd = 0.f;
+            for (int nt = 0; nt < NTQ; ++nt)
 #pragma unroll
-                for (int n = 0; n < NK; ++n) {
-                    const int cc = c0 + lane + 32 * n;
-                    qd = fmaf(Qs[t * SK + cc], acc[i][n], qd);
-                    if (t < Lc) dq[(row0 + t0 + t) * DK + cc] = from_f32<IO>(acc[i][n]);
+                for (int r = 0; r < 4; ++r) {
+                    const int t = frow(mq, r), cc = c0 + fcol(nq, nt, r);
+                    part[r >> 1] += Qs[t * PQ + cc] * aq[nt][r] - Ks[t * PQ + cc] * ak[nt][r];
+                    if (t < Lc) {
+                        dq[(row0 + t0 + t) * DK + cc] = from_f32<IO>(aq[nt][r]);
+                        dk[(row0 + t0 + t) * DK + cc] = from_f32<IO>(ak[nt][r]);
+                    }
                 }
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) qd += __shfl_xor_sync(0xffffffffu, qd, off);
-                if (lane == 0 && t < Lc) atomicAdd(&dl[t], qd);
-            }
-        }
-        {   // dK = dP^T Q + diag(g_L / g) V G   (this CTA's columns)
-            float acc[RC][NK] = {};
-            tile_mma<RC, NK, DV>(acc, r0, lane, [&](int t, int i) { return Vs[t * SV + i]; },
-                                 [&](int i, int cc) { return G[i * SH + cc]; });
-#pragma unroll
-            for (int i = 0; i < RC; ++i)
-#pragma unroll
-                for (int n = 0; n < NK; ++n) acc[i][n] *= dec[r0 + i];
-            tile_mma<RC, NK, C>(acc, r0, lane, [&](int t, int s) { return dP[s * SP + t]; },
-                                [&](int s, int cc) { return Qs[s * SK + c0 + cc]; });
-#pragma unroll
-            for (int i = 0; i < RC; ++i) {
-                const int t = r0 + i;
-                float kd = 0.f;
-#pragma unroll
-                for (int n = 0; n < NK; ++n) {
-                    const int cc = c0 + lane + 32 * n;
-                    kd = fmaf(Ks[t * SK + cc], acc[i][n], kd);
-                    if (t < Lc) dk[(row0 + t0 + t) * DK + cc] = from_f32<IO>(acc[i][n]);
-                }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) kd += __shfl_xor_sync(0xffffffffu, kd, off);
-                if (lane == 0 && t < Lc) atomicAdd(&dl[t], -kd);
+            for (int h = 0; h < 2; ++h) {   // row sums of the warp into dl
+                float s = part[h];
+                s += __shfl_xor_sync(0xffffffffu, s, 1);
+                s += __shfl_xor_sync(0xffffffffu, s, 2);
+                if ((tid & 3) == 0) atomicAdd(&dl[mq + ((tid & 31) >> 2) + 8 * h], s);
             }
         }
         {   // dV = P^T dO + diag(g_L / g) K G^T: this CTA's columns' share, added up in fp32
-            float acc[RC][NV] = {};
-            tile_mma<RC, NV, DKH>(acc, r0, lane, [&](int t, int cc) { return Ks[t * SK + c0 + cc]; },
-                                  [&](int cc, int i) { return G[i * SH + cc]; });
+            float av[NTV][4] = {};
+            warp_mma<NTV, DKH, SP, true>(av, mq, nv, [&](int t, int cc) { return Ks[t * PQ + c0 + cc]; },
+                                   [&](int cc, int i) { return G[i * PS + cc]; });
 #pragma unroll
-            for (int i = 0; i < RC; ++i)
+            for (int nt = 0; nt < NTV; ++nt)
 #pragma unroll
-                for (int n = 0; n < NV; ++n) acc[i][n] *= dec[r0 + i];
+                for (int r = 0; r < 4; ++r) av[nt][r] *= dec[frow(mq, r)];
             if (kh == 0)
-                tile_mma<RC, NV, C>(acc, r0, lane, [&](int t, int s) { return P[s * SP + t]; },
-                                    [&](int s, int i) { return dOs[s * SV + i]; });
+                warp_mma<NTV, C, true, SP>(av, mq, nv, [&](int t, int s2) { return P[s2 * PC + t]; },
+                                     [&](int s2, int i) { return dOs[s2 * PV + i]; });
 #pragma unroll
-            for (int i = 0; i < RC; ++i) {
-                const int t = r0 + i;
-                if (t < Lc)
+            for (int nt = 0; nt < NTV; ++nt)
 #pragma unroll
-                    for (int n = 0; n < NV; ++n) {
-                        float *dst = dv_acc + (row0 + t0 + t) * DV + lane + 32 * n;
-                        if (SPLIT == 1) *dst = acc[i][n];
-                        else atomicAdd(dst, acc[i][n]);
+                for (int h = 0; h < 2; ++h) {
+                    const int t = frow(mq, 2 * h), i = fcol(nv, nt, 2 * h);
+                    if (t < Lc) {
+                        float *dst = dv_acc + (row0 + t0 + t) * DV + i;
+                        if (SPLIT == 1) *reinterpret_cast<float2 *>(dst) = make_float2(av[nt][2 * h], av[nt][2 * h + 1]);
+                        else red_add2(dst, av[nt][2 * h], av[nt][2 * h + 1]);
                     }
-            }
+                }
         }
-        __syncthreads();
+        __syncthreads();   // dl complete; every read of G done
         if (tid < Lc) {
             if (SPLIT == 1) dl_acc[row0 + t0 + tid] += dl[tid];
             else atomicAdd(&dl_acc[row0 + t0 + tid], dl[tid]);
         }
-        // carry G to the chunk start: G <- g_L G + dO^T diag(g) Q   (this CTA's columns)
-        {
-            float acc[RS][NK] = {};
-            tile_mma<RS, NK, C>(acc, RS * warp, lane, [&](int i, int t) { return gv[t] * dOs[t * SV + i]; },
-                                [&](int t, int cc) { return Qs[t * SK + c0 + cc]; });
+        {   // carry G to the chunk start: G <- g_L G + dO^T diag(g) Q   (this CTA's columns)
+            const float gL = gv[Lc - 1];
+            float ag[NTS][4] = {};
+            warp_mma<NTS, C, true, SP>(ag, ms, ns, [&](int i, int t) { return gv[t] * dOs[t * PV + i]; },
+                                 [&](int t, int cc) { return Qs[t * PQ + c0 + cc]; });
 #pragma unroll
-            for (int i = 0; i < RS; ++i)
+            for (int nt = 0; nt < NTS; ++nt)
 #pragma unroll
-                for (int n = 0; n < NK; ++n) {
-                    float &x = G[(RS * warp + i) * SH + lane + 32 * n];
-                    x = fmaf(gL, x, acc[i][n]);
+                for (int r = 0; r < 4; ++r) {
+                    float &x = G[frow(ms, r) * PS + fcol(ns, nt, r)];
+                    x = fmaf(gL, x, ag[nt][r]);
                 }
         }
         __syncthreads();
+        float *tmp = Sc;
+        Sc = Sn;
+        Sn = tmp;
     }
     if (dS0)
-        for (int p = tid; p < DV * DKH; p += kBwdThreads) dS0[bh * DV * DK + gl_idx(p)] = G[st_idx(p)];
+        for (int p = tid; p < DV * DKH; p += kBwdThreads)
+            dS0[bh * DV * DK + (p / DKH) * DK + c0 + p % DKH] = G[(p / DKH) * PS + p % DKH];
 }
 
 // Per (batch, head): dV from its fp32 accumulator, and the gate gradient
@@ -324,7 +402,7 @@ cudaError_t launch_bwd(int BH, int T, int gate_heads, const void *q, const void 
                        void *dq, void *dk, void *dv, float *dgate, float *dS0, float *ws,
                        cudaStream_t st) {
     constexpr int SPLIT = bwd_split<DK>();
-    using L = BwdSmem<DK, DV, SPLIT>;
+    using L = BwdSmem<DK, DV, SPLIT, std::is_same<IO, __nv_bfloat16>::value>;
     const size_t nch = ((size_t)T + kBwdC - 1) / kBwdC;
     float *dv_acc = ws + (size_t)BH * (nch + 1) * DV * DK;
     float *dl_acc = dv_acc + (size_t)BH * T * DV;

@@ -46,8 +46,8 @@
 // bf16 I/O one tf32 product.  Gated DeltaNet's Gam is one C x C table per chunk folded into
 // the coefficient matrices; Kimi's per-channel Gam is evaluated per term on the CUDA cores
 // (exp2 of the log-gate difference, no factor outside [0, 1]), exact for any gate.
-#include "bwd_util.cuh"
 #include "la_internal.cuh"
+#include "bwd_util.cuh"
 
 #include <cfloat>
 #include <type_traits>
@@ -179,29 +179,6 @@ __device__ __forceinline__ void load_tile(const IO *__restrict__ src, size_t row
     }
 }
 
-// ---- cp.async staging of a chunk's raw inputs (Gated DeltaNet)
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
-    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// Rows [0, n) of `w` elements (a multiple of 16 bytes) from src (row stride ld elements)
-// into dst (row stride w), 16 bytes per copy.
-template <typename IO>
-__device__ __forceinline__ void stage_rows(void *dst, const IO *src, int ld, int w, int n) {
-    constexpr int E = 16 / sizeof(IO);   // elements per copy
-    const int per = w / E;
-    for (int p = threadIdx.x; p < n * per; p += kDT) {
-        const int t = p / per, x = (p % per) * E;
-        cp_async16(static_cast<IO *>(dst) + t * w + x, src + (size_t)t * ld + x);
-    }
-}
 // One chunk's raw inputs into the staging buffers: k, v (columns j0 ..), gate, b, and for
 // the reverse sweep q, dO and the chunk-start state slice; rows [0, n).
 template <int MODE, int DK, typename IO>
@@ -209,41 +186,18 @@ __device__ __forceinline__ void stage_chunk(const ChunkTiles<MODE, DK> &c, const
                                             const IO *v, const IO *dO, const float *gate,
                                             const float *beta, const float *state, size_t r, int n,
                                             int DV, int j0) {
-    stage_rows(c.sk, k + r * DK, DK, DK, n);
-    stage_rows(c.sv, v + r * DV + j0, DV, kDVS, n);
+    stage_rows<kDT>(c.sk, k + r * DK, DK, DK, n);
+    stage_rows<kDT>(c.sv, v + r * DV + j0, DV, kDVS, n);
     if (q) {
-        stage_rows(c.sq, q + r * DK, DK, DK, n);
-        stage_rows(c.sdo, dO + r * DV + j0, DV, kDVS, n);
-        stage_rows(c.sS, state, DK, DK, kDVS);
+        stage_rows<kDT>(c.sq, q + r * DK, DK, DK, n);
+        stage_rows<kDT>(c.sdo, dO + r * DV + j0, DV, kDVS, n);
+        stage_rows<kDT>(c.sS, state, DK, DK, kDVS);
     }
     const int tid = threadIdx.x;
     if (tid < n) cp_async4(c.sb + tid, beta + r + tid);
     if (gate && tid >= 32 && tid - 32 < n) cp_async4(c.sg + tid - 32, gate + r + tid - 32);
     cp_async_commit();
 }
-// Staged rows into a C x w fp32 tile (pitch `pitch`, a multiple of 4), zero past row n:
-// 16 bytes of staged elements per step, written as float4.
-template <typename IO>
-__device__ __forceinline__ void unstage(const void *src, int w, int n, float *dst, int pitch) {
-    constexpr int E = 16 / sizeof(IO);
-    for (int p = threadIdx.x; p < kDC * w / E; p += kDT) {
-        const int t = p * E / w, j = p * E % w;
-        float f[E];
-        if (t < n) {
-            const uint4 raw = *reinterpret_cast<const uint4 *>(static_cast<const IO *>(src) + t * w + j);
-            const IO *x = reinterpret_cast<const IO *>(&raw);
-#pragma unroll
-            for (int e = 0; e < E; ++e) f[e] = to_f32(x[e]);
-        } else {
-#pragma unroll
-            for (int e = 0; e < E; ++e) f[e] = 0.f;
-        }
-#pragma unroll
-        for (int e = 0; e < E; e += 4)
-            *reinterpret_cast<float4 *>(dst + t * pitch + j + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
-    }
-}
-
 // The chunk's gates: b (zero past the last token), the log2 gate prefix (held at its last
 // value past the last token) and the derived factors.  Mode 2: lam, g, dec, gl[all] = g_L
 // and the C x C table Gm = Gam; mode 3: Lg, gl, Kg, Kl (and Qg when `with_q`).
@@ -443,8 +397,8 @@ delta_states_kernel(int T, int DV, const IO *__restrict__ k, const IO *__restric
         if constexpr (kStage) {
             cp_async_wait_all();
             __syncthreads();
-            unstage<IO>(c.sk, DK, n, c.Ks, PK);
-            unstage<IO>(c.sv, kDVS, n, c.Vs, kPV);
+            unstage<kDT, IO>(c.sk, kDC, DK, n, c.Ks, PK);
+            unstage<kDT, IO>(c.sv, kDC, kDVS, n, c.Vs, kPV);
         } else {
             load_tile(k, row0 + t0, DK, 0, DK, n, c.Ks, PK);
             load_tile(v, row0 + t0, DV, j0, kDVS, n, c.Vs, kPV);
@@ -502,11 +456,6 @@ __device__ __forceinline__ void gam_cols(float (&acc)[NT][4], int m0, int n0, co
         for (int u = t; u < kDC; ++u) s = fmaf(m(u, t) * X[u * PK + cc], exp2f(Lg[u * PK + cc] - lt), s);
         a += s;
     });
-}
-
-// p[0] += a, p[1] += b in global memory (one vector reduction; p 8-byte aligned).
-__device__ __forceinline__ void red_add2(float *p, float a, float b) {
-    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
 }
 
 // Two fragment arrays of the same ownership, element by element.
@@ -574,11 +523,11 @@ delta_backward_kernel(int T, int DV, const IO *__restrict__ q, const IO *__restr
         if constexpr (kStage) {
             cp_async_wait_all();
             __syncthreads();
-            unstage<IO>(c.sq, DK, n, c.Qs, PK);
-            unstage<IO>(c.sk, DK, n, c.Ks, PK);
-            unstage<IO>(c.sv, kDVS, n, c.Vs, kPV);
-            unstage<IO>(c.sdo, kDVS, n, c.dOs, kPV);
-            unstage<float>(c.sS, DK, kDVS, c.Ss, PK);
+            unstage<kDT, IO>(c.sq, kDC, DK, n, c.Qs, PK);
+            unstage<kDT, IO>(c.sk, kDC, DK, n, c.Ks, PK);
+            unstage<kDT, IO>(c.sv, kDC, kDVS, n, c.Vs, kPV);
+            unstage<kDT, IO>(c.sdo, kDC, kDVS, n, c.dOs, kPV);
+            unstage<kDT, float>(c.sS, kDC, DK, kDVS, c.Ss, PK);
         } else {
             const float *src = states + ((bh * nch + ch) * DV + j0) * (size_t)DK;
             for (int p = tid; p < kDVS * DK; p += kDT) c.Ss[(p / DK) * PK + p % DK] = src[p];

@@ -1,5 +1,6 @@
-// bwd_util.cuh -- register-tiled products on shared-memory operands, shared by the
-// backward kernels.
+// bwd_util.cuh -- products on shared-memory operands (register-tiled CUDA-core and
+// warp-level tensor-core forms), cp.async staging and reductions shared by the backward
+// kernels.  Include after la_internal.cuh (to_f32).
 #pragma once
 
 #include <cstdint>
@@ -28,9 +29,10 @@ __device__ __forceinline__ void tile_mma(float (&acc)[RM][RN], int r0, int lane,
 
 // Warp-level products on the tensor cores (mma.sync m16n8k8, tf32 operands, fp32
 // accumulate): d[nt] += sum_{k<K} A(m, k) B(k, n) for the 16 x 8 NT block at rows m0..m0+15,
-// columns n0..n0+8 NT-1.  The accessors return fp32; with SPLIT each operand is split into
-// a tf32 high part and a tf32 remainder and three products keep fp32 accuracy
-// (hi*hi + hi*lo + lo*hi), else the operands are rounded to tf32 once.
+// columns n0..n0+8 NT-1.  The accessors return fp32.  An operand marked for splitting is
+// taken as a tf32 high part plus a tf32 remainder, and the products keep fp32 accuracy
+// (hi*hi + hi*lo + lo*hi); an unsplit operand is rounded to tf32 once, which is exact for
+// values that came from bf16.
 // Element r of d[nt] sits at row m0 + (lane >> 2) + 8 (r >> 1), column
 // n0 + 8 nt + 2 (lane & 3) + (r & 1).
 __device__ __forceinline__ uint32_t tf32_bits(float x) {
@@ -46,7 +48,7 @@ __device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-template <int NT, int K, bool SPLIT, typename FA, typename FB>
+template <int NT, int K, bool SPLIT, bool SPLIT_B = SPLIT, typename FA, typename FB>
 __device__ __forceinline__ void warp_mma(float (&d)[NT][4], int m0, int n0, FA a, FB b) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
 #pragma unroll 2
@@ -64,13 +66,62 @@ __device__ __forceinline__ void warp_mma(float (&d)[NT][4], int m0, int n0, FA a
             const float b0 = b(kk + t4, n0 + 8 * nt + g), b1 = b(kk + t4 + 4, n0 + 8 * nt + g);
             const uint32_t bh0 = tf32_bits(b0), bh1 = tf32_bits(b1);
             mma_16x8x8_tf32(d[nt], ah, bh0, bh1);
-            if (SPLIT) {
+            if (SPLIT_B)
                 mma_16x8x8_tf32(d[nt], ah, tf32_bits(b0 - __uint_as_float(bh0)),
                                 tf32_bits(b1 - __uint_as_float(bh1)));
-                mma_16x8x8_tf32(d[nt], al, bh0, bh1);
-            }
+            if (SPLIT) mma_16x8x8_tf32(d[nt], al, bh0, bh1);
         }
     }
+}
+
+// ---- cp.async staging of raw inputs (16-byte copies into shared memory)
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Rows [0, n) of `w` elements (w * sizeof(IO) a multiple of 16 bytes) from src (row stride
+// ld elements, 16-byte aligned rows) into dst (row stride w); NT threads take part.
+template <int NT, typename IO>
+__device__ __forceinline__ void stage_rows(void *dst, const IO *src, int ld, int w, int n) {
+    constexpr int E = 16 / sizeof(IO);   // elements per copy
+    const int per = w / E;
+    for (int p = threadIdx.x; p < n * per; p += NT) {
+        const int t = p / per, x = (p % per) * E;
+        cp_async16(static_cast<IO *>(dst) + t * w + x, src + (size_t)t * ld + x);
+    }
+}
+// `rows` staged rows of w elements into an fp32 tile (pitch a multiple of 4 floats), zero
+// past row n: 16 bytes of staged elements per step, written as float4.
+template <int NT, typename IO>
+__device__ __forceinline__ void unstage(const void *src, int rows, int w, int n, float *dst, int pitch) {
+    constexpr int E = 16 / sizeof(IO);
+    for (int p = threadIdx.x; p < rows * w / E; p += NT) {
+        const int t = p * E / w, j = p * E % w;
+        float f[E];
+        if (t < n) {
+            const uint4 raw = *reinterpret_cast<const uint4 *>(static_cast<const IO *>(src) + t * w + j);
+            const IO *x = reinterpret_cast<const IO *>(&raw);
+#pragma unroll
+            for (int e = 0; e < E; ++e) f[e] = to_f32(x[e]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) f[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < E; e += 4)
+            *reinterpret_cast<float4 *>(dst + t * pitch + j + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+    }
+}
+// p[0] += a, p[1] += b in global memory (one vector reduction; p 8-byte aligned).
+__device__ __forceinline__ void red_add2(float *p, float a, float b) {
+    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
 }
 
 }  // namespace la

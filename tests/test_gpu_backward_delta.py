@@ -159,3 +159,11 @@ def test_delta_backward_full_size_sampled(la):
         got_db = f(db)[T - 1]
         assert abs(got_db - want_db) <= tol * max(abs(want_db), np.abs(u).max() * np.abs(v[T - 1]).max()), \
             (b, h, got_db, want_db)
+
+
+@pytest.mark.parametrize("mode", [2, 3])
+def test_delta_backward_bf16_long(la, mode):
+    """bf16 I/O over 4096 tokens (128 chunks): the gate gradient is a suffix sum within each
+    chunk, but the carried cotangent and states cross all 128 chunks."""
+    inp, dO, dST = _case(mode, torch.bfloat16, 128, 128, 4096, -3.0, seed=60 + mode, H=1)
+    _compare(la, mode, torch.bfloat16, inp, dO, inp["state0"], dST)
