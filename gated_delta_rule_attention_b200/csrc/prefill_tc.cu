@@ -36,8 +36,9 @@
 //   K~, Q~ = K, Q times 2^(lam_t - lam_ref(t)), in place in the stage;
 // then K~ -> K o Gamma (W^T = (K o Gamma)^T (T diag b)^T), Q~ -> Q o Gamma (the O
 // product), Kb -> K o 2^(lam_L - lam) (dS = E^T Kb), and S <- S Diag(2^lam_L) + dS.
-// Every factor stays within 2^120 because each per-token log2 gate is clamped at -7.5
-// (a >= 0.0055); the CUDA-core kernel (chunk 32) takes gates below that as they are.
+// Every factor of G stays within 2^120 because G's per-token log2 gates are bounded below
+// at -7.5 (a >= 0.0055); the other products take the exact gates (see kda_exact below), and
+// the CUDA-core kernel (chunk 32) takes every gate as it is everywhere.
 // Kb is written only after the previous chunk's products are done (it is one buffer);
 // T diag(b g) is not needed, and its slot holds Kb0; outputs are staged in the chunk's V
 // slot, so that Kb takes the output staging slot.
@@ -81,8 +82,10 @@ constexpr uint32_t kColDS = 0, kColG = 128, kColU = 192, kColW = 256, kColY = 32
 // Kimi Delta Attention (mode 3): the first-half product G0 (N = 32) borrows the first 32
 // U columns, free until the U^T product of the same chunk.
 constexpr uint32_t kColG0 = kColU;
-// Mode 3 clamps each per-channel log2 gate at -kKdaLog2Clamp (a >= 2^-7.5 = 0.0055), so
-// that no operand factor 2^(lambda_t - lambda_ref) over half a half-chunk exceeds 2^120.
+// Mode 3 bounds each per-channel log2 gate at -kKdaLog2Clamp (a >= 2^-7.5 = 0.0055) inside
+// the Gram products G, so that no operand factor 2^(lambda_t - lambda_ref) over half a
+// half-chunk exceeds 2^120; the state-facing operands (K o Gamma, Q o Gamma,
+// K o 2^(lambda_L - lambda)) and the state's column decay take the exact gates (kda_exact).
 constexpr float kKdaLog2Clamp = 7.5f;
 
 // kLocalTrans (delta rule): one launch of both no-output passes, CTAs [0, split) local,
@@ -226,6 +229,7 @@ struct SmallKda {
     float edec[2][128];      // 2^(lambda_L - lambda_47): Kb -> K 2^(lambda_L - lambda)
     float egl[2][128];       // 2^lambda_L: the state's column decay over the chunk
     float tot0[128], tot1[128], x15b[128];   // half totals and the second half's prefix at 15
+    float tot0u[128], tot1u[128];            // half totals of the unbounded log2 gates
 };
 
 // Shared-memory layout (bytes from the 1024-aligned base).
@@ -496,9 +500,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
         // ---- mode 3: thread e owns channel kch for the token half khh of every chunk
         const int kch = e & 127, khh = e >> 7;
-        float kx[32];            // inclusive prefix of the clamped log2 gates within the half
+        float kx[32];            // inclusive prefix of the bounded log2 gates within the half
         float kx15 = 0.f;        // the prefix at the half's reference token (15 or 47)
         float kref = 0.f;        // exponent base of Kb: lambda_47 in this thread's prefix units
+        bool kcl = false;        // some log2 gate of the chunk was below -kKdaLog2Clamp
         // L2 prefetch of chunk c's gate rows (64 tokens x 512 B: one line per thread)
         auto kda_prefetch = [&](int c) {
             const int t0 = tb + kC * c, tok = e >> 2;
@@ -515,9 +520,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // prefixes, the exchange between the halves, and the chunk's decay vectors
         auto kda_prefix = [&](int c, const float (&g)[32]) {
             float acc = 0.f;
+            bool low = false;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                acc += fmaxf(lg2(fmaxf(g[i], FLT_MIN)), -kKdaLog2Clamp);
+                const float l = lg2(fmaxf(g[i], FLT_MIN));
+                low |= l < -kKdaLog2Clamp;
+                acc += fmaxf(l, -kKdaLog2Clamp);
                 kx[i] = acc;
             }
             kx15 = kx[15];
@@ -527,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 sk->tot1[kch] = acc;
                 sk->x15b[kch] = kx15;
             }
-            epi_sync();
+            kcl = named_sync_any(1, kEpi, low);   // (the epilogue barrier, with an OR)
             const float tot0 = sk->tot0[kch];
             kref = (khh == 0) ? tot0 + sk->x15b[kch] : kx15;
             if (khh == 0) {
@@ -567,7 +575,51 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             epi_sync();
             if (e == 0) mbar_arrive(&sm->prep_done);
         };
-        (void)kda_prefetch; (void)kda_load; (void)kda_prefix; (void)kda_scale;
+        // Chunk c's state-facing operands with the exact gates, in a chunk where some log2
+        // gate is below -kKdaLog2Clamp (kcl): the Gram products G keep the bounded gates
+        // (their factors around the reference tokens must stay finite), while K o Gamma,
+        // Q o Gamma, K o 2^(lambda_L - lambda) and the state's column decay 2^lambda_L need
+        // no reference and take every gate as it is.  Each thread rescales its own channel
+        // and token half by 2^(lambda_exact - lambda_bounded) <= 1 (and the corresponding
+        // ratio for Kb), after the per-channel conversion of the A-epilogue.
+        auto kda_exact = [&](int c, int b2) {
+            const int t0 = tb + kC * c;
+            const int L = min(kC, te - t0);
+            const float *gp = p.gate + ((size_t)bh * p.T + t0 + 32 * khh) * kD + kch;
+            float accu = 0.f;
+            for (int i = 0; i < 32; ++i)
+                accu += (p.gate && 32 * khh + i < L) ? lg2(fmaxf(gp[(size_t)i * kD], FLT_MIN)) : 0.f;
+            if (khh == 0) sk->tot0u[kch] = accu;
+            else sk->tot1u[kch] = accu;
+            epi_sync();
+            const float tot0 = sk->tot0[kch], tot0u = sk->tot0u[kch];
+            const float lL = tot0 + sk->tot1[kch], lLu = tot0u + sk->tot1u[kch];
+            const float base = khh ? tot0 : 0.f, baseu = khh ? tot0u : 0.f;
+            const uint32_t stg = (c % NST) * Y::kStage;
+            const uint32_t cb = (uint32_t)(kch >> 6), cc = (uint32_t)(kch & 63);
+            float x = 0.f, xu = 0.f;
+            for (int i = 0; i < 32; ++i) {
+                const float l = (p.gate && 32 * khh + i < L) ? lg2(fmaxf(gp[(size_t)i * kD], FLT_MIN)) : 0.f;
+                x += fmaxf(l, -kKdaLog2Clamp);
+                xu += l;
+                const float lam_b = base + x, lam_u = baseu + xu;
+                const float fk = ex2(lam_u - lam_b);                  // K o Gamma, Q o Gamma
+                const float fb = ex2((lLu - lam_u) - (lL - lam_b));   // K o 2^(lambda_L - lambda)
+                if (fk == 1.f && fb == 1.f) continue;
+                const uint32_t tt = 32 * khh + i;
+                const uint32_t o = sw128_off(tt, cc >> 3) + ((cc & 7) << 1);
+                __nv_bfloat16 *kp = reinterpret_cast<__nv_bfloat16 *>(smem_raw + stg + cb * 16384 + o);
+                *kp = __float2bfloat16_rn(__bfloat162float(*kp) * fk);
+                if (kOut) {
+                    __nv_bfloat16 *qp = kp + 4096;
+                    *qp = __float2bfloat16_rn(__bfloat162float(*qp) * fk);
+                }
+                __nv_bfloat16 *bp = reinterpret_cast<__nv_bfloat16 *>(smem_raw + Y::kKb + cb * 8192 + o);
+                *bp = __float2bfloat16_rn(__bfloat162float(*bp) * fb);
+            }
+            if (khh == 0) sk->egl[b2][kch] = ex2(lLu);
+        };
+        (void)kda_prefetch; (void)kda_load; (void)kda_prefix; (void)kda_scale; (void)kda_exact;
 
         // ---- chunk prologue: gates; releases G's inputs to the MMA (mode 3: kda_scale does)
         auto prep = [&](int c, GateRaw raw) -> bool {
@@ -685,6 +737,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     const float4 d1 = *reinterpret_cast<const float4 *>(ed + c0 + 4);
                     const uint32_t ba = sb + Y::kKb + half * 8192 + (n & 511) * 16;
                     sts128(ba, scale_bf16x8v(lds128(ba), d0, d1));
+                }
+                if (kcl) {   // uniform over the epilogue threads
+                    epi_sync();
+                    kda_exact(c, buf);
                 }
             } else if (kOut) {
                 // after G: Q <- diag(g) Q in place

@@ -231,11 +231,24 @@ def test_kda_cuda_core_path(la, T):
 
 
 @pytest.mark.parametrize("chunk", [0, 32])
-def test_kda_strong_decay(la, chunk):
-    """Gates near 0.0025 on every channel.  The tensor-core path clamps each per-token,
-    per-channel gate at 2^-7.5 = 0.0055 (its operands carry the decays as factors
-    2^(lambda_t - lambda_ref) that must stay finite); such a gate changes the state by
-    at most 0.55 % of what it forgets, inside the bf16 tolerance.  The CUDA-core path
-    (chunk 32) takes the gates as given."""
-    w = small(3, torch.bfloat16, 128, 200, gate_shift=6.0, seed=324)
+@pytest.mark.parametrize("shift", [6.0, 9.0])
+def test_kda_strong_decay(la, chunk, shift):
+    """Per-channel gates near 0.0025 (shift 6) and down to 1e-4 and below (shift 9), held to
+    the bf16 tolerance on both paths.  The tensor-core path bounds the log2 gates at -7.5 only
+    inside the Gram products G (their operand factors around reference tokens must stay
+    finite); every state-facing factor takes the gates as given.  The CUDA-core path
+    (chunk 32) takes them as given everywhere."""
+    w = small(3, torch.bfloat16, 128, 200, gate_shift=shift, seed=324)
+    if shift == 9.0:
+        assert float(W.prefill_inputs(w, device="cuda")["gate"].min()) < 1e-4
     run_and_compare(la, w, init_std=0.05, chunk=chunk)
+
+
+@pytest.mark.parametrize("shift", [4.0, 6.0, 9.0])
+def test_kda_large_initial_state_and_tiny_gates(la, shift):
+    """An initial state far larger than the per-token updates (std 10) with gates below 0.005
+    on the tensor-core path: the outputs must show the state forgotten.  A floor on the gates
+    of the state-facing factors would leave 2^-7.5 of it in every output (a 22 % error here);
+    the exact factors keep the outputs within the bf16 tolerance."""
+    w = small(3, torch.bfloat16, 128, 160, B=1, gate_shift=shift, seed=77)
+    run_and_compare(la, w, init_std=10.0)
