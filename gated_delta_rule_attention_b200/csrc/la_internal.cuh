@@ -88,7 +88,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t work
 // The single-pass gated-delta prefill (d_v split over four CTAs per head, no workspace):
 // whether it serves a call of BH head rows (dense or packed), and its launcher.
 bool prefill_gdn_selected(int mode, int BH, bool packed);
-cudaError_t launch_prefill_gdn(const PrefillArgs &a);
+cudaError_t launch_prefill_gdn(const PrefillArgs &a, void *workspace, size_t workspace_bytes);
+// Workspace with which it runs its two-pass variant (per-chunk factors formed in parallel).
+size_t prefill_gdn_workspace_bytes(int BH, int T);
 cudaError_t launch_short_conv(const ConvArgs &a);
 // Workspace of la_prefill_backward_delta (0 for other modes).
 size_t delta_backward_workspace_bytes(int mode, int B, int H, int T, int d_k, int d_v);

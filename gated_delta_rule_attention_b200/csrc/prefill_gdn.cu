@@ -46,6 +46,7 @@
 #include "ptx.cuh"
 #include "tc_util.cuh"
 #include "tmap.cuh"
+#include "bwd_util.cuh"
 
 #include <cfloat>
 #include <cstddef>
@@ -110,6 +111,7 @@ struct Small {
     uint64_t g_done, wu_done, w_free, u_free;
     uint64_t p_done, ds_done;
     uint64_t ae_done[2];
+    uint64_t a_full[2];   // two-pass variant: the A tile of each parity has arrived
     uint32_t tmem_base;
     int abort;
 };
@@ -117,6 +119,31 @@ static_assert(sizeof(Gates) % 16 == 0 && offsetof(Gates, cf) % 16 == 0, "float4 
 static_assert(kSmall % 16 == 0, "gate rows are read as float4");
 constexpr uint32_t kBytes = kSmall + sizeof(Small);
 static_assert(kBytes <= 227 * 1024, "shared memory per CTA");
+
+// Shared-memory layouts of the two variants.  The two-pass variant reads A, T diag(b) and
+// T diag(b g) from pass 1: the stage carries the two T tiles after V (each 128-row A
+// operand of W and U starts 8 KB before its tile, on the stage's own data), and the Lm, Tm
+// and Zs buffers of the inverse are not needed.
+template <bool TWO>
+struct GLay;
+template <>
+struct GLay<false> {
+    static constexpr uint32_t kStage = ::la::kStage, kA0 = ::la::kA0, kA1 = ::la::kA1, kTbg = ::la::kTbg,
+                              kTb = ::la::kTb, kLm = ::la::kLm, kTm = ::la::kTm, kZs = ::la::kZs,
+                              kS = ::la::kS, kE = ::la::kE, kEp = ::la::kEp, kSmall = ::la::kSmall,
+                              kBytes = ::la::kBytes;
+};
+template <>
+struct GLay<true> {
+    static constexpr uint32_t kStage = 57344;   // [Q0 | K0 | Q1 | K1 | V | T diag(b) | T diag(b g)]
+    static constexpr uint32_t kTbOff = 40960, kTbgOff = 49152;
+    static constexpr uint32_t kA0 = kStages * kStage, kA1 = kA0 + 8192;
+    static constexpr uint32_t kTbg = 0, kTb = 0, kLm = 0, kTm = 0, kZs = 0;   // (not used)
+    static constexpr uint32_t kS = kA1 + 8192, kE = kS + 16384, kEp = kE + 8192, kSmall = kEp + 8192;
+    static constexpr uint32_t kBytes = kSmall + sizeof(Small);
+};
+static_assert(GLay<true>::kS % 1024 == 0 && GLay<true>::kA0 % 1024 == 0, "1024-byte aligned tiles");
+static_assert(GLay<true>::kBytes <= 227 * 1024, "shared memory per CTA");
 
 struct GdnParams {
     CUtensorMap tq, tk, tv;     // [BH][T][128] bf16, 64 x 64 boxes, 128B swizzle
@@ -129,6 +156,10 @@ struct GdnParams {
     const int *cu;              // packed sequences (nullptr: dense)
     int T, BH;
     unsigned *err;
+    // two-pass variant: pass 1's per-chunk [A | T diag(b) | T diag(b g)] images,
+    // [BH][nchunks][3][64 x 64] bf16 (nullptr: single pass)
+    const __nv_bfloat16 *img;
+    int nchunks;
 };
 
 __device__ __forceinline__ void gdn_range(const GdnParams &p, int unit, int &bh, int &seq, int &tb,
@@ -180,7 +211,131 @@ __device__ __forceinline__ void st_row32_mn(uint32_t tile, uint32_t row, const f
     }
 }
 
+// ---------------------------------------------------------------------------------------
+// Two-pass variant, pass 1: the state-independent factors of every chunk at once, one CTA
+// per (head row, chunk).  Per chunk it writes three bf16 64 x 64 tiles, each the 8 KB
+// 128B-swizzled image the tensor cores read (rows of 128 bytes):
+//   A = (Q K^T) 2^(lam_t - lam_j) (j <= t),   T diag(b),   T diag(b g)   (j <= t),
+// T = (I + Lm)^-1, Lm = strictly-lower(diag(b) 2^(lam_t - lam_j) K K^T).  The Gram products
+// run as warp-level tensor-core mma (tf32 operands, which hold the bf16 inputs exactly; fp32
+// accumulate); every pair decay is one exponential (no factor outside [0, 1]).  The gate
+// prefix is formed exactly as pass 2's gate warp forms it.
+constexpr int kFacT = 256;
+constexpr int kFacPitch = kD + 8;                              // bf16 pitch of the Q, K rows
+constexpr uint32_t kFacQ = 0;                                  // Q [64][136] bf16
+constexpr uint32_t kFacK = kFacQ + kC * kFacPitch * 2;         // K
+constexpr uint32_t kFacLm = kFacK + kC * kFacPitch * 2;        // fp32 [64][kTStride]
+constexpr uint32_t kFacTm = kFacLm + kC * kTStride * 4;
+constexpr uint32_t kFacZs = kFacTm + kC * kTStride * 4;        // 4 x 272 floats
+constexpr uint32_t kFacImg = (kFacZs + 4 * 272 * 4 + 1023) & ~1023u;   // [A | T diag(b) | T diag(b g)]
+constexpr uint32_t kFacG = kFacImg + 3 * 8192;                 // lam, bet, bg [64] each
+constexpr uint32_t kFacBytes = kFacG + 3 * kC * 4;
+constexpr int kImgHalves = 3 * 4096;                           // bf16 elements per chunk record
+
+__global__ void __launch_bounds__(kFacT, 2)
+gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                         const float *__restrict__ gate, const float *__restrict__ beta, int T, int nch,
+                         __nv_bfloat16 *__restrict__ img) {
+    extern __shared__ __align__(1024) uint8_t fsm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x / nch, c = blockIdx.x % nch;
+    const int t0 = c * kC, L = min(kC, T - t0);
+    const size_t row0 = (size_t)bh * T + t0;
+    __nv_bfloat16 *Qs = reinterpret_cast<__nv_bfloat16 *>(fsm + kFacQ);
+    __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(fsm + kFacK);
+    float *Lm = reinterpret_cast<float *>(fsm + kFacLm);
+    float *Tm = reinterpret_cast<float *>(fsm + kFacTm);
+    float *Zs = reinterpret_cast<float *>(fsm + kFacZs);
+    uint8_t *im = fsm + kFacImg;
+    float *lam = reinterpret_cast<float *>(fsm + kFacG), *bet = lam + kC, *bg = bet + kC;
+
+    // rows of q and k in 16-byte pieces, zero past the sequence end
+    for (int p = tid; p < 2 * kC * 16; p += kFacT) {
+        const int which = p >> 10, r = (p >> 4) & 63, x = p & 15;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < L) v = *reinterpret_cast<const uint4 *>((which ? k : q) + (row0 + r) * kD + 8 * x);
+        *reinterpret_cast<uint4 *>((which ? Ks : Qs) + r * kFacPitch + 8 * x) = v;
+    }
+    if (warp == 0) {   // lane l takes tokens 2l, 2l + 1
+        float a0 = 1.f, a1 = 1.f, b0 = 0.f, b1 = 0.f;
+        const int i0 = 2 * lane, i1 = 2 * lane + 1;
+        if (i0 < L) {
+            if (gate) a0 = gate[row0 + i0];
+            b0 = beta[row0 + i0];
+        }
+        if (i1 < L) {
+            if (gate) a1 = gate[row0 + i1];
+            b1 = beta[row0 + i1];
+        }
+        const float g0 = (i0 < L) ? lg2(fmaxf(a0, FLT_MIN)) : 0.f;
+        const float g1 = (i1 < L) ? lg2(fmaxf(a1, FLT_MIN)) : 0.f;
+        float x = g0 + g1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float n = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += n;
+        }
+        const float l1 = x, l0 = x - g1;
+        lam[i0] = l0;
+        lam[i1] = l1;
+        bet[i0] = b0;
+        bet[i1] = b1;
+        bg[i0] = b0 * ex2(l0);
+        bg[i1] = b1 * ex2(l1);
+    }
+    __syncthreads();
+    {   // G = K K^T -> Lm (j < t), Q K^T -> A (j <= t): warp w rows 16 (w & 3), columns 32 (w >> 2)
+        const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
+        const int g = lane >> 2, t4 = lane & 3;
+        float gk[4][4] = {}, gq[4][4] = {};
+        warp_mma<4, kD, false>(gk, m0, n0, [&](int t, int cc) { return __bfloat162float(Ks[t * kFacPitch + cc]); },
+                               [&](int cc, int j) { return __bfloat162float(Ks[j * kFacPitch + cc]); });
+        warp_mma<4, kD, false>(gq, m0, n0, [&](int t, int cc) { return __bfloat162float(Qs[t * kFacPitch + cc]); },
+                               [&](int cc, int j) { return __bfloat162float(Ks[j * kFacPitch + cc]); });
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int t = m0 + g + 8 * h, j = n0 + 8 * nt + 2 * t4;
+                float a2[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int jj = j + e;
+                    const float dd = jj <= t ? ex2(lam[t] - lam[jj]) : 0.f;
+                    Lm[t * kTStride + jj] = jj < t ? bet[t] * gk[nt][2 * h + e] * dd : 0.f;
+                    a2[e] = gq[nt][2 * h + e] * dd;
+                }
+                *reinterpret_cast<uint32_t *>(im + sw128_off(t, j >> 3) + (j & 7) * 2) = pack_bf16x2(a2[0], a2[1]);
+            }
+    }
+    __syncthreads();
+    invert_unit_lower_rec<1, kFacT>(Lm, Tm, Zs, tid);
+    __syncthreads();
+    {   // T diag(b), T diag(b g) (lower triangle)
+        const int t = tid >> 2, j0 = 16 * (tid & 3);
+        float v1[16], v2[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+            const int j = j0 + jj;
+            const float tj = (j <= t) ? Tm[t * kTStride + j] : 0.f;
+            v1[jj] = tj * bet[j];
+            v2[jj] = tj * bg[j];
+        }
+        st_row_bf16x16(smem_u32(im + 8192), t, j0 >> 3, v1);
+        st_row_bf16x16(smem_u32(im + 16384), t, j0 >> 3, v2);
+    }
+    __syncthreads();
+    uint4 *dst = reinterpret_cast<uint4 *>(img + ((size_t)bh * nch + c) * kImgHalves);
+    for (int p = tid; p < 3 * 512; p += kFacT) dst[p] = reinterpret_cast<const uint4 *>(im)[p];
+}
+
+template <bool TWO>
 __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_constant__ GdnParams p) {
+    using GL = GLay<TWO>;
+    // the variant's layout (shadows the single-pass constants)
+    constexpr uint32_t kStage = GL::kStage, kA0 = GL::kA0, kA1 = GL::kA1, kTbg = GL::kTbg, kTb = GL::kTb,
+                       kLm = GL::kLm, kTm = GL::kTm, kZs = GL::kZs, kS = GL::kS, kE = GL::kE, kEp = GL::kEp,
+                       kSmall = GL::kSmall;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sb = smem_u32(smem_raw);
     if (sb & 1023u) {
@@ -209,6 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
         mbar_init(&sm->ds_done, 1);
         mbar_init(&sm->ae_done[0], 1);
         mbar_init(&sm->ae_done[1], 1);
+        mbar_init(&sm->a_full[0], 1);
+        mbar_init(&sm->a_full[1], 1);
         sm->abort = 0;
         fence_mbar_init();
     }
@@ -248,6 +405,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                 tma_load_3d(st + 16384, &p.tq, 64, t, bh, &sm->full[s]);
                 tma_load_3d(st + 24576, &p.tk, 64, t, bh, &sm->full[s]);
                 tma_load_3d(st + 32768, &p.tv, vx, t, bh, &sm->full[s]);
+                if constexpr (TWO) {   // T diag(b), T diag(b g) of chunk c (pass 1)
+                    const __nv_bfloat16 *rec = p.img + ((size_t)bh * p.nchunks + c) * kImgHalves;
+                    bulk_load(st + GL::kTbOff, rec + 4096, 8192, &sm->full[s]);
+                    bulk_load(st + GL::kTbgOff, rec + 8192, 8192, &sm->full[s]);
+                }
                 issued[s] = u + 1;
                 // the chunk three ahead of this one into L2 (the slices of a head share it)
                 const int tp = t + kStages * kC;
@@ -307,6 +469,40 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
         }
     } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------------------ prep warps 4-11
+        if constexpr (TWO) {
+            // two-pass: one thread copies each chunk's A tile and issues W and U from the
+            // stage's T tiles; the factors themselves came from pass 1
+            if (threadIdx.x == 128) {
+                int issued[2] = {0, 0};
+                for (int c = 0; c < nch; ++c) {
+                    const int s = c % kStages, b = c & 1;
+                    // A(c) into its parity buffer once A E(c - 2) has read it
+                    if (c >= 2 && !mbar_wait(&sm->ae_done[b], ((c >> 1) - 1) & 1, abort, p.err)) break;
+                    mbar_arrive_expect_tx(&sm->a_full[b], 8192);
+                    bulk_load(sb + (b ? kA1 : kA0), p.img + ((size_t)bh * p.nchunks + c) * kImgHalves, 8192,
+                              &sm->a_full[b]);
+                    issued[b] = (c >> 1) + 1;
+                    // W = T diag(b g) K, U = T diag(b) V (rows 64-127) once the stage is in and
+                    // the chain has read W(c - 1), U(c - 1)
+                    if (!mbar_wait(&sm->full[s], (c / kStages) & 1, abort, p.err)) break;
+                    if (c >= 1 && !(mbar_wait(&sm->w_free, (c - 1) & 1, abort, p.err) &&
+                                    mbar_wait(&sm->u_free, (c - 1) & 1, abort, p.err)))
+                        break;
+                    tc_fence_after();
+                    const uint32_t st = sb + s * kStage;
+                    mma_chain<4, true, false>(tm + kColW, dk(st + GL::kTbgOff - 8192), dmn(st + 8192, 16384), id_w,
+                                              false);
+                    mma_chain<4, true, false>(tm + kColU, dk(st + GL::kTbOff - 8192), dmn(st + 32768, 8192), id_u,
+                                              false);
+                    mma_commit(&sm->wu_done);
+                }
+                // nothing issued here may still write tensor or shared memory at exit
+                mma_commit(&sm->g_done);
+                drain_wait(&sm->g_done, 0);
+                for (int b = 0; b < 2; ++b)
+                    if (issued[b] > 0) drain_wait(&sm->a_full[b], (issued[b] - 1) & 1);
+            }
+        } else {
         const int pe = threadIdx.x - 128;           // 0..255
         const int pq = warp & 3;                    // tensor-memory lane quarter
         const int ph = (warp - 4) >> 2;             // column half of G
@@ -440,6 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
             mma_commit(&sm->g_done);   // completes phase nch (the G products took 0 .. nch-1)
             drain_wait(&sm->g_done, (uint32_t)nch & 1);
         }
+        }
     } else if (warp >= 12) {
         // ------------------------------------------------------------ chain warps 12-15
         const int ce = threadIdx.x - 384;           // 0..127
@@ -554,9 +751,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                         mma_commit(&sm->empty[s]);
                         // rows 0-63 of P += A E  (the 64 rows after the A tile multiply into
                         // rows 64-127, already read)
-                        mma_chain<4, true, false>(tm + kColP + kDV * par, dk(sb + (par ? kA1 : kA0)),
-                                                  dmn(sb + kE, 8192), id_ae, true);
-                        mma_commit(&sm->ae_done[par]);
+                        if (!TWO || mbar_wait(&sm->a_full[par], (c >> 1) & 1, abort, p.err)) {
+                            mma_chain<4, true, false>(tm + kColP + kDV * par, dk(sb + (par ? kA1 : kA0)),
+                                                      dmn(sb + kE, 8192), id_ae, true);
+                            mma_commit(&sm->ae_done[par]);
+                        }
                     }
                 }
             } else if (c >= 1) {
@@ -638,7 +837,14 @@ bool prefill_gdn_selected(int mode, int BH, bool packed) {
     return mode == LA_MODE_GATED_DELTA && !packed && BH * kNS >= 64 && BH * kNS <= 148;
 }
 
-cudaError_t launch_prefill_gdn(const PrefillArgs &a) {
+size_t prefill_gdn_workspace_bytes(int BH, int T) {
+    return sizeof(__nv_bfloat16) * (size_t)kImgHalves * (size_t)BH * (size_t)((T + kC - 1) / kC);
+}
+
+// With a workspace of at least prefill_gdn_workspace_bytes (dense calls), pass 1 forms every
+// chunk's A, T diag(b), T diag(b g) at once and the chain kernel reads them (two-pass);
+// otherwise the single pass forms them itself.
+cudaError_t launch_prefill_gdn(const PrefillArgs &a, void *workspace, size_t workspace_bytes) {
     const int BH = a.cu ? a.H : a.B * a.H;
     GdnParams p;
     memset(&p, 0, sizeof(p));
@@ -661,11 +867,30 @@ cudaError_t launch_prefill_gdn(const PrefillArgs &a) {
     p.BH = BH;
     p.err = device_error_word();
     const int units = a.cu ? a.nseq * a.H : BH;
-    cudaError_t e = cudaFuncSetAttribute(gdn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kBytes);
+    const bool two = !a.cu && workspace && (reinterpret_cast<uintptr_t>(workspace) & 15u) == 0 &&
+                     workspace_bytes >= prefill_gdn_workspace_bytes(BH, a.T);
+    cudaError_t e;
+    if (two) {
+        const int nch = (a.T + kC - 1) / kC;
+        p.img = static_cast<const __nv_bfloat16 *>(workspace);
+        p.nchunks = nch;
+        e = cudaFuncSetAttribute(gdn_chunk_factors_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kFacBytes);
+        if (e != cudaSuccess) return e;
+        timer_begin(a.stream);
+        gdn_chunk_factors_kernel<<<(unsigned)BH * nch, kFacT, kFacBytes, a.stream>>>(
+            static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k), a.gate, a.beta, a.T,
+            nch, static_cast<__nv_bfloat16 *>(workspace));
+        timer_end(a.stream);
+        note_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    auto kern = two ? gdn_prefill_kernel<true> : gdn_prefill_kernel<false>;
+    const uint32_t bytes = two ? GLay<true>::kBytes : GLay<false>::kBytes;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     timer_begin(a.stream);
-    gdn_prefill_kernel<<<units * kNS, kThreads, kBytes, a.stream>>>(p);
+    kern<<<units * kNS, kThreads, bytes, a.stream>>>(p);
     timer_end(a.stream);
     note_launches(1);
     return cudaGetLastError();

@@ -2132,7 +2132,7 @@ bool prefill_tc_supports(int mode, int dtype, int dk, int dv, int chunk) {
 
 size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T, bool minimal) {
     const int BH = B * H;
-    if (prefill_gdn_selected(mode, BH, false)) return 0;
+    if (prefill_gdn_selected(mode, BH, false)) return minimal ? 0 : prefill_gdn_workspace_bytes(BH, T);
     Plan pl = plan_for(mode, BH, T);
     if (minimal && mode >= 2) pl.sub = 1;   // the smallest segmented plan
     return sizeof(float) * workspace_floats(mode, BH, pl);
@@ -2160,7 +2160,7 @@ cudaError_t run_packed(const PrefillArgs &a, const TcParams &base) {
 
 cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes) {
     const int BH = a.B * a.H;
-    if (prefill_gdn_selected(a.mode, BH, a.cu != nullptr)) return launch_prefill_gdn(a);
+    if (prefill_gdn_selected(a.mode, BH, a.cu != nullptr)) return launch_prefill_gdn(a, workspace, workspace_bytes);
     const Plan pl = plan_for(a.mode, BH, a.T, workspace ? workspace_bytes : 0);
     TcParams p;
     memset(&p, 0, sizeof(p));

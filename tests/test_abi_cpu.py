@@ -93,9 +93,10 @@ def test_workspace_size_query(lib):
     # bf16, d = 128: the tensor-core kernels; few heads and a long sequence -> segments
     assert lib.la_prefill_workspace_size(2, 1, 1, 8, 32768, 128, 128, 0) > 0
     assert lib.la_prefill_workspace_size(3, 1, 2, 16, 32768, 128, 128, 0) > 0
-    # the gated delta rule with 16-37 head rows: the single-pass kernel, no workspace
-    assert lib.la_prefill_workspace_size(2, 1, 2, 16, 32768, 128, 128, 0) == 0
-    assert lib.la_prefill_workspace_size(2, 1, 1, 37, 32768, 128, 128, 0) == 0
+    # the gated delta rule with 16-37 head rows: the single-pass kernel, whose two-pass
+    # variant keeps each chunk's A, T diag(b), T diag(b g) (3 x 8 KB) in the workspace
+    assert lib.la_prefill_workspace_size(2, 1, 2, 16, 32768, 128, 128, 0) == 32 * 512 * 24576
+    assert lib.la_prefill_workspace_size(2, 1, 1, 37, 32768, 128, 128, 0) == 37 * 512 * 24576
     assert lib.la_prefill_workspace_size(2, 1, 1, 38, 32768, 128, 128, 0) > 0
     assert lib.la_prefill_workspace_size(1, 1, 8, 16, 8192, 128, 128, 0) == 0   # 128 heads
     assert lib.la_prefill_workspace_size(0, 0, 1, 2, 256, 64, 64, 0) == 0       # fp32 path

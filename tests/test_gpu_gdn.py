@@ -34,15 +34,19 @@ def gdn(T, B=1, H=16, gate="softplus", shift=0.0, seed=500):
 
 
 def check(la, w, inp, init=False, heads=None):
-    state = inp["state0"].clone()
-    o, S, _ = la.prefill(inp["q"], inp["k"], inp["v"], mode=2, gate=inp["gate"],
-                         beta=inp["beta"], state=state, init_state=init, workspace=None)
-    la.check_status()
+    """Both variants: the single pass (no workspace) and the two-pass variant (pass 1 forms
+    every chunk's A, T diag(b), T diag(b g) into the workspace)."""
     if heads is None:
         heads = list(itertools.product(range(w.B), range(w.H)))
     ro, rS, _ = oracle_prefill_slices(2, inp, heads, init_state=init)
-    eo = slice_rel_err(pick(o, heads), ro, lead=1)
-    eS = slice_rel_err(pick(S, heads), rS, lead=1)
+    for ws in (None, "auto"):
+        state = inp["state0"].clone()
+        o, S, _ = la.prefill(inp["q"], inp["k"], inp["v"], mode=2, gate=inp["gate"],
+                             beta=inp["beta"], state=state, init_state=init, workspace=ws)
+        la.check_status()
+        eo = slice_rel_err(pick(o, heads), ro, lead=1)
+        eS = slice_rel_err(pick(S, heads), rS, lead=1)
+        assert eo <= TOL[torch.bfloat16] and eS <= TOL[torch.bfloat16], (ws, eo, eS)
     tol = TOL[torch.bfloat16]
     assert eo <= tol, f"output rel err {eo:.3e} > {tol}"
     assert eS <= tol, f"state rel err {eS:.3e} > {tol}"
@@ -114,7 +118,8 @@ def test_single_pass_matches_segmented_path(la):
     head rows, which take the segmented kernels (local, transition, combine, outputs)."""
     w = gdn(1500, B=1, H=16, shift=-1.0, seed=506)
     inp = W.prefill_inputs(w, device="cuda")
-    assert la.workspace_size(2, torch.bfloat16, 1, 16, w.T, 128, 128) == 0
+    # 16 head rows: the two-pass variant's per-chunk factors (24 KB a chunk); 8: segments
+    assert la.workspace_size(2, torch.bfloat16, 1, 16, w.T, 128, 128) == 16 * ((w.T + 63) // 64) * 24576
     assert la.workspace_size(2, torch.bfloat16, 1, 8, w.T, 128, 128) > 0
     o, S, _ = la.prefill(inp["q"], inp["k"], inp["v"], mode=2, gate=inp["gate"], beta=inp["beta"])
     for h in (0, 8):
