@@ -79,6 +79,7 @@ constexpr uint32_t kColU = 192;    // 64   U (the V half) in lanes 64-127
 constexpr uint32_t kColQW = 256;   // 2 x 64: [diag(g) Q; W] as bf16 pairs, per chunk parity
 constexpr uint32_t kColP = 384;    // 2 x 32: P (+ A E) per chunk parity
 constexpr uint32_t kColDS = 448;   // 32   dS^T
+constexpr uint32_t kColU2 = 0;     // 64   two-pass variant: U of odd chunks (G is not formed)
 constexpr uint32_t kTmemCols = 512;
 
 // shared memory (bytes from the 1024-aligned base)
@@ -112,6 +113,9 @@ struct Small {
     uint64_t p_done, ds_done;
     uint64_t ae_done[2];
     uint64_t a_full[2];   // two-pass variant: the A tile of each parity has arrived
+    uint64_t u_free2[2];  // two-pass variant: U buffer of each parity read by the chain
+    uint64_t qw_ready[2]; // two-pass variant: [diag(g) Q; W] of each parity in tensor memory
+    uint64_t p_done2[2];  // two-pass variant: P of each parity done (its A operand is free)
     uint32_t tmem_base;
     int abort;
 };
@@ -217,8 +221,8 @@ __device__ __forceinline__ void st_row32_mn(uint32_t tile, uint32_t row, const f
 // 128B-swizzled image the tensor cores read (rows of 128 bytes):
 //   A = (Q K^T) 2^(lam_t - lam_j) (j <= t),   T diag(b),   T diag(b g)   (j <= t),
 // T = (I + Lm)^-1, Lm = strictly-lower(diag(b) 2^(lam_t - lam_j) K K^T).  The Gram products
-// run as warp-level tensor-core mma (tf32 operands, which hold the bf16 inputs exactly; fp32
-// accumulate); every pair decay is one exponential (no factor outside [0, 1]).  The gate
+// run as warp-level tensor-core mma on the bf16 rows (m16n8k16, fp32 accumulate); every pair
+// decay is one exponential (no factor outside [0, 1]).  The gate
 // prefix is formed exactly as pass 2's gate warp forms it.
 constexpr int kFacT = 256;
 constexpr int kFacPitch = kD + 8;                              // bf16 pitch of the Q, K rows
@@ -288,10 +292,8 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
         const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
         const int g = lane >> 2, t4 = lane & 3;
         float gk[4][4] = {}, gq[4][4] = {};
-        warp_mma<4, kD, false>(gk, m0, n0, [&](int t, int cc) { return __bfloat162float(Ks[t * kFacPitch + cc]); },
-                               [&](int cc, int j) { return __bfloat162float(Ks[j * kFacPitch + cc]); });
-        warp_mma<4, kD, false>(gq, m0, n0, [&](int t, int cc) { return __bfloat162float(Qs[t * kFacPitch + cc]); },
-                               [&](int cc, int j) { return __bfloat162float(Ks[j * kFacPitch + cc]); });
+        warp_mma_bf16<4, kD>(gk, m0, n0, Ks, kFacPitch, Ks, kFacPitch);
+        warp_mma_bf16<4, kD>(gq, m0, n0, Qs, kFacPitch, Ks, kFacPitch);
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -366,6 +368,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
         mbar_init(&sm->ae_done[1], 1);
         mbar_init(&sm->a_full[0], 1);
         mbar_init(&sm->a_full[1], 1);
+        mbar_init(&sm->u_free2[0], 1);
+        mbar_init(&sm->u_free2[1], 1);
+        mbar_init(&sm->qw_ready[0], 1);
+        mbar_init(&sm->qw_ready[1], 1);
+        mbar_init(&sm->p_done2[0], 1);
+        mbar_init(&sm->p_done2[1], 1);
         sm->abort = 0;
         fence_mbar_init();
     }
@@ -470,37 +478,90 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
     } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------------------ prep warps 4-11
         if constexpr (TWO) {
-            // two-pass: one thread copies each chunk's A tile and issues W and U from the
-            // stage's T tiles; the factors themselves came from pass 1
-            if (threadIdx.x == 128) {
-                int issued[2] = {0, 0};
-                for (int c = 0; c < nch; ++c) {
-                    const int s = c % kStages, b = c & 1;
+            // Two-pass: thread 128 copies each chunk's A tile and issues W and U from the
+            // stage's T tiles (the factors themselves came from pass 1); the eight warps then
+            // write [diag(g) Q; W] of the chunk into tensor memory as the A operand of P, a
+            // chunk or two ahead of the chain, which only waits for it (qw_ready).
+            const int pq = warp & 3, ph = (warp - 4) >> 2;   // lane quarter; which half of the work
+            const uint32_t tl = tm + ((uint32_t)(32 * pq) << 16);
+            const int prow = 32 * pq + lane;
+            const bool lead = threadIdx.x == 128;
+            int issued[2] = {0, 0};
+            for (int c = 0; c < nch; ++c) {
+                const int s = c % kStages, b = c & 1;
+                bool ok = true;
+                if (lead) {
                     // A(c) into its parity buffer once A E(c - 2) has read it
-                    if (c >= 2 && !mbar_wait(&sm->ae_done[b], ((c >> 1) - 1) & 1, abort, p.err)) break;
-                    mbar_arrive_expect_tx(&sm->a_full[b], 8192);
-                    bulk_load(sb + (b ? kA1 : kA0), p.img + ((size_t)bh * p.nchunks + c) * kImgHalves, 8192,
-                              &sm->a_full[b]);
-                    issued[b] = (c >> 1) + 1;
-                    // W = T diag(b g) K, U = T diag(b) V (rows 64-127) once the stage is in and
-                    // the chain has read W(c - 1), U(c - 1)
-                    if (!mbar_wait(&sm->full[s], (c / kStages) & 1, abort, p.err)) break;
-                    if (c >= 1 && !(mbar_wait(&sm->w_free, (c - 1) & 1, abort, p.err) &&
-                                    mbar_wait(&sm->u_free, (c - 1) & 1, abort, p.err)))
-                        break;
-                    tc_fence_after();
-                    const uint32_t st = sb + s * kStage;
-                    mma_chain<4, true, false>(tm + kColW, dk(st + GL::kTbgOff - 8192), dmn(st + 8192, 16384), id_w,
-                                              false);
-                    mma_chain<4, true, false>(tm + kColU, dk(st + GL::kTbOff - 8192), dmn(st + 32768, 8192), id_u,
-                                              false);
-                    mma_commit(&sm->wu_done);
+                    ok = c < 2 || mbar_wait(&sm->ae_done[b], ((c >> 1) - 1) & 1, abort, p.err);
+                    if (ok) {
+                        mbar_arrive_expect_tx(&sm->a_full[b], 8192);
+                        bulk_load(sb + (b ? kA1 : kA0), p.img + ((size_t)bh * p.nchunks + c) * kImgHalves, 8192,
+                                  &sm->a_full[b]);
+                        issued[b] = (c >> 1) + 1;
+                    }
+                    // W = T diag(b g) K, U = T diag(b) V (rows 64-127) once the stage is in, W(c - 1)
+                    // was read (the group's own step below) and U(c - 2) was read by the chain
+                    // (U has a buffer per chunk parity)
+                    ok = ok && mbar_wait(&sm->full[s], (c / kStages) & 1, abort, p.err) &&
+                         (c < 2 || mbar_wait(&sm->u_free2[b], ((c >> 1) - 1) & 1, abort, p.err));
+                    if (ok) {
+                        tc_fence_after();
+                        const uint32_t st = sb + s * kStage;
+                        mma_chain<4, true, false>(tm + kColW, dk(st + GL::kTbgOff - 8192), dmn(st + 8192, 16384),
+                                                  id_w, false);
+                        mma_chain<4, true, false>(tm + (b ? kColU2 : kColU), dk(st + GL::kTbOff - 8192),
+                                                  dmn(st + 32768, 8192), id_u, false);
+                        mma_commit(&sm->wu_done);
+                        // W(c) formed, and P(c - 2) done with this parity's A operand buffer
+                        ok = mbar_wait(&sm->wu_done, c & 1, abort, p.err) &&
+                             (c < 2 || mbar_wait(&sm->p_done2[b], ((c >> 1) - 1) & 1, abort, p.err));
+                    }
                 }
-                // nothing issued here may still write tensor or shared memory at exit
+                // every thread reads the stage's Q tile and gates
+                mbar_wait(&sm->full[s], (c / kStages) & 1, abort, p.err);
+                if (named_sync_any(kBarPrep, kPrepT, !ok || *abort != 0)) break;
+                tc_fence_after();
+                const uint32_t dst = tl + kColQW + 64 * b;
+                if (pq < 2) {   // rows 0-63: diag(g) Q, column half ph
+                    const int t = prow;
+                    const float gt = ex2(sm->gt[s].lam[t]);
+                    const uint32_t st = sb + s * kStage;
+                    uint32_t w[32];
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint4 x = scale_bf16x8(lds128(st + 16384 * ph + sw128_off(t, ch)), gt);
+                        w[4 * ch + 0] = x.x;
+                        w[4 * ch + 1] = x.y;
+                        w[4 * ch + 2] = x.z;
+                        w[4 * ch + 3] = x.w;
+                    }
+                    tmem_st32(dst + 32 * ph, w);
+                } else {        // rows 64-127: W as bf16, column quarters 2 ph, 2 ph + 1
+#pragma unroll 1
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int h = 2 * ph + hh;
+                        float f[32];
+                        tmem_ld32(tl + kColW + 32 * h, f);
+                        uint32_t w[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(f[2 * j], f[2 * j + 1]);
+                        tmem_st16u(dst + 16 * h, w);
+                    }
+                }
+                tc_fence_before();
+                named_sync(kBarPrep, kPrepT);
+                if (lead) {
+                    mbar_arrive(&sm->w_free);
+                    // A(c) has arrived too: the chain's A E(c) needs no wait of its own
+                    if (!mbar_wait(&sm->a_full[b], (c >> 1) & 1, abort, p.err)) break;
+                    mbar_arrive(&sm->qw_ready[b]);
+                }
+            }
+            if (lead) {   // nothing issued here may still write tensor or shared memory at exit
                 mma_commit(&sm->g_done);
                 drain_wait(&sm->g_done, 0);
-                for (int b = 0; b < 2; ++b)
-                    if (issued[b] > 0) drain_wait(&sm->a_full[b], (issued[b] - 1) & 1);
+                for (int bb = 0; bb < 2; ++bb)
+                    if (issued[bb] > 0) drain_wait(&sm->a_full[bb], (issued[bb] - 1) & 1);
             }
         } else {
         const int pe = threadIdx.x - 128;           // 0..255
@@ -658,6 +719,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
             mma_chain_ts<8>(tm + kColP + kDV * (c & 1), tm + kColQW + 64 * (c & 1), dmn(sb + kS, 8192),
                             id_p, false);
             mma_commit(&sm->p_done);
+            if (TWO) mma_commit(&sm->p_done2[c & 1]);
+        };
+        // two-pass: the prep warps wrote [diag(g) Q; W] of chunk c; the chain meets after the
+        // elected thread saw it (which also orders the stage's gates before their reads)
+        auto qw_wait = [&](int c) -> bool {
+            return group_wait(&sm->qw_ready[c & 1], (c >> 1) & 1, ce == 0, kBarChain, kChainT, abort, p.err);
         };
         // [diag(g) Q; W] of chunk c into tensor memory as the A operand of P
         auto qw_step = [&](int c) -> bool {
@@ -700,7 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
             if (ce == 0) mbar_arrive(&sm->w_free);
             return true;
         };
-        bool ok = qw_step(0);
+        bool ok = TWO ? qw_wait(0) : qw_step(0);
         if (ok && ce == 0) issue_p(0);
         // Iteration c: E of chunk c (lanes 64-127) and the outputs of chunk c - 1 (lanes 0-63);
         // the A operand of chunk c + 1 while dS(c) is formed; the state update and P(c + 1).
@@ -727,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                     const float *lam = sm->gt[s].lam;
                     float y[32], uu[32];
                     tmem_ld32(tl + kColP + kDV * par, y);
-                    tmem_ld32(tl + kColU + kDV * (vs & 1), uu);
+                    tmem_ld32(tl + ((TWO && par) ? kColU2 : kColU) + kDV * (vs & 1), uu);
                     const float dec = (t < L) ? ex2(lam[kC - 1] - lam[t]) : 0.f;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
@@ -741,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                     tc_fence_before();
                     named_sync(kBarChainE, 64);
                     if (row == 64) {
-                        mbar_arrive(&sm->u_free);
+                        mbar_arrive(TWO ? &sm->u_free2[par] : &sm->u_free);
                         tc_fence_after();
                         const uint32_t st = sb + s * kStage;
                         // dS^T = K^T E'   (E' = diag(dec) E)
@@ -751,11 +818,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                         mma_commit(&sm->empty[s]);
                         // rows 0-63 of P += A E  (the 64 rows after the A tile multiply into
                         // rows 64-127, already read)
-                        if (!TWO || mbar_wait(&sm->a_full[par], (c >> 1) & 1, abort, p.err)) {
-                            mma_chain<4, true, false>(tm + kColP + kDV * par, dk(sb + (par ? kA1 : kA0)),
-                                                      dmn(sb + kE, 8192), id_ae, true);
-                            mma_commit(&sm->ae_done[par]);
-                        }
+                        // (two-pass: A(c) arrived before the chain saw qw_ready(c))
+                        mma_chain<4, true, false>(tm + kColP + kDV * par, dk(sb + (par ? kA1 : kA0)),
+                                                  dmn(sb + kE, 8192), id_ae, true);
+                        mma_commit(&sm->ae_done[par]);
                     }
                 }
             } else if (c >= 1) {
@@ -782,10 +848,19 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                     }
                 }
             }
-            if (c + 1 < nch && !qw_step(c + 1)) break;
+            if (!TWO && c + 1 < nch && !qw_step(c + 1)) break;
             if (!cur) continue;
-            // ---- state: S^T <- g_{L-1} S^T + dS^T; bf16 copy for the next chunk
-            if (!group_wait(&sm->ds_done, par, ce == 0, kBarChain, kChainT, abort, p.err)) break;
+            // ---- state: S^T <- g_{L-1} S^T + dS^T; bf16 copy for the next chunk (two-pass: one
+            // meeting also covers the next chunk's A operand of P)
+            if constexpr (TWO) {
+                if (ce == 0) {
+                    if (c + 1 < nch) mbar_wait(&sm->qw_ready[(c + 1) & 1], ((c + 1) >> 1) & 1, abort, p.err);
+                    mbar_wait(&sm->ds_done, par, abort, p.err);
+                }
+                if (named_sync_any(kBarChain, kChainT, *abort != 0)) break;
+            } else {
+                if (!group_wait(&sm->ds_done, par, ce == 0, kBarChain, kChainT, abort, p.err)) break;
+            }
             tc_fence_after();
             const bool last = (c + 1 == nch);
             {
