@@ -216,8 +216,8 @@ __device__ __forceinline__ void st_row32_mn(uint32_t tile, uint32_t row, const f
 }
 
 // ---------------------------------------------------------------------------------------
-// Two-pass variant, pass 1: the state-independent factors of every chunk at once, one CTA
-// per (head row, chunk).  Per chunk it writes three bf16 64 x 64 tiles, each the 8 KB
+// Two-pass variant, pass 1: the state-independent factors of every chunk at once, two CTAs
+// per SM over all (head row, chunk) pairs.  Per chunk it writes three bf16 64 x 64 tiles, each the 8 KB
 // 128B-swizzled image the tensor cores read (rows of 128 bytes):
 //   A = (Q K^T) 2^(lam_t - lam_j) (j <= t),   T diag(b),   T diag(b g)   (j <= t),
 // T = (I + Lm)^-1, Lm = strictly-lower(diag(b) 2^(lam_t - lam_j) K K^T).  The Gram products
@@ -226,74 +226,98 @@ __device__ __forceinline__ void st_row32_mn(uint32_t tile, uint32_t row, const f
 // prefix is formed exactly as pass 2's gate warp forms it.
 constexpr int kFacT = 256;
 constexpr int kFacPitch = kD + 8;                              // bf16 pitch of the Q, K rows
-constexpr uint32_t kFacQ = 0;                                  // Q [64][136] bf16
-constexpr uint32_t kFacK = kFacQ + kC * kFacPitch * 2;         // K
-constexpr uint32_t kFacLm = kFacK + kC * kFacPitch * 2;        // fp32 [64][kTStride]
-constexpr uint32_t kFacTm = kFacLm + kC * kTStride * 4;
-constexpr uint32_t kFacZs = kFacTm + kC * kTStride * 4;        // 4 x 272 floats
+constexpr uint32_t kFacTile = kC * kFacPitch * 2;              // 17408 B: a Q or K tile
+static_assert(kFacTile == kC * kTStride * 4, "Lm / Tm reuse the Q / K tiles");
+constexpr uint32_t kFacBuf = 2 * kFacTile;                     // [Q | K] of one chunk
+constexpr uint32_t kFacZs = 2 * kFacBuf;                       // two chunk buffers, then Zs
 constexpr uint32_t kFacImg = (kFacZs + 4 * 272 * 4 + 1023) & ~1023u;   // [A | T diag(b) | T diag(b g)]
-constexpr uint32_t kFacG = kFacImg + 3 * 8192;                 // lam, bet, bg [64] each
-constexpr uint32_t kFacBytes = kFacG + 3 * kC * 4;
+constexpr uint32_t kFacG = kFacImg + 3 * 8192;                 // raw gate, beta [2][64] each
+constexpr uint32_t kFacL = kFacG + 4 * kC * 4;                 // lam, bet, bg [64] each
+constexpr uint32_t kFacBytes = kFacL + 3 * kC * 4;
 constexpr int kImgHalves = 3 * 4096;                           // bf16 elements per chunk record
 
+// Each CTA takes chunks blockIdx.x, blockIdx.x + gridDim.x, ... (chunk i = head row i / nch,
+// chunk i % nch); the next chunk's rows, gates and rates arrive by cp.async while the
+// current one is processed.  Lm and Tm of the inverse take the places of the chunk's Q and
+// K tiles once the Gram products have read them.
 __global__ void __launch_bounds__(kFacT, 2)
 gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                          const float *__restrict__ gate, const float *__restrict__ beta, int T, int nch,
-                         __nv_bfloat16 *__restrict__ img) {
+                         int total, __nv_bfloat16 *__restrict__ img) {
     extern __shared__ __align__(1024) uint8_t fsm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x / nch, c = blockIdx.x % nch;
-    const int t0 = c * kC, L = min(kC, T - t0);
-    const size_t row0 = (size_t)bh * T + t0;
-    __nv_bfloat16 *Qs = reinterpret_cast<__nv_bfloat16 *>(fsm + kFacQ);
-    __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(fsm + kFacK);
-    float *Lm = reinterpret_cast<float *>(fsm + kFacLm);
-    float *Tm = reinterpret_cast<float *>(fsm + kFacTm);
     float *Zs = reinterpret_cast<float *>(fsm + kFacZs);
     uint8_t *im = fsm + kFacImg;
-    float *lam = reinterpret_cast<float *>(fsm + kFacG), *bet = lam + kC, *bg = bet + kC;
-
-    // rows of q and k in 16-byte pieces, zero past the sequence end
-    for (int p = tid; p < 2 * kC * 16; p += kFacT) {
-        const int which = p >> 10, r = (p >> 4) & 63, x = p & 15;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r < L) v = *reinterpret_cast<const uint4 *>((which ? k : q) + (row0 + r) * kD + 8 * x);
-        *reinterpret_cast<uint4 *>((which ? Ks : Qs) + r * kFacPitch + 8 * x) = v;
-    }
-    if (warp == 0) {   // lane l takes tokens 2l, 2l + 1
-        float a0 = 1.f, a1 = 1.f, b0 = 0.f, b1 = 0.f;
-        const int i0 = 2 * lane, i1 = 2 * lane + 1;
-        if (i0 < L) {
-            if (gate) a0 = gate[row0 + i0];
-            b0 = beta[row0 + i0];
+    float *graw = reinterpret_cast<float *>(fsm + kFacG), *braw = graw + 2 * kC;
+    float *lam = reinterpret_cast<float *>(fsm + kFacL), *bet = lam + kC, *bg = bet + kC;
+    auto chunk_of = [&](int item, size_t &row0, int &L) {
+        const int bh = item / nch, c = item % nch;
+        row0 = (size_t)bh * T + (size_t)c * kC;
+        L = min(kC, T - c * kC);
+    };
+    // rows [0, L) of q and k (16-byte copies; rows past L zeroed), gates and rates
+    auto stage = [&](int item, int buf) {
+        size_t row0;
+        int L;
+        chunk_of(item, row0, L);
+        uint8_t *base = fsm + buf * kFacBuf;
+        for (int p = tid; p < 2 * kC * 16; p += kFacT) {
+            const int which = p >> 10, r = (p >> 4) & 63, x = p & 15;
+            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(base + which * kFacTile) + r * kFacPitch + 8 * x;
+            if (r < L) cp_async16(dst, (which ? k : q) + (row0 + r) * kD + 8 * x);
+            else *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
         }
-        if (i1 < L) {
-            if (gate) a1 = gate[row0 + i1];
-            b1 = beta[row0 + i1];
-        }
-        const float g0 = (i0 < L) ? lg2(fmaxf(a0, FLT_MIN)) : 0.f;
-        const float g1 = (i1 < L) ? lg2(fmaxf(a1, FLT_MIN)) : 0.f;
-        float x = g0 + g1;
+        if (tid < L) cp_async4(braw + buf * kC + tid, beta + row0 + tid);
+        if (gate && tid >= 64 && tid - 64 < L) cp_async4(graw + buf * kC + tid - 64, gate + row0 + tid - 64);
+        cp_async_commit();
+    };
+    if ((int)blockIdx.x < total) stage(blockIdx.x, 0);
+    for (int item = blockIdx.x, it = 0; item < total; item += gridDim.x, ++it) {
+        const int cur = it & 1;
+        size_t row0;
+        int L;
+        chunk_of(item, row0, L);
+        __nv_bfloat16 *Qs = reinterpret_cast<__nv_bfloat16 *>(fsm + cur * kFacBuf);
+        __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(fsm + cur * kFacBuf + kFacTile);
+        float *Lm = reinterpret_cast<float *>(fsm + cur * kFacBuf);            // over Q
+        float *Tm = reinterpret_cast<float *>(fsm + cur * kFacBuf + kFacTile); // over K
+        cp_async_wait_all();
+        __syncthreads();   // this chunk's rows are in; the other buffer and the images are free
+        if (item + (int)gridDim.x < total) stage(item + gridDim.x, cur ^ 1);
+        if (warp == 0) {   // lane l takes tokens 2l, 2l + 1, as pass 2's gate warp
+            float a0 = 1.f, a1 = 1.f, b0 = 0.f, b1 = 0.f;
+            const int i0 = 2 * lane, i1 = 2 * lane + 1;
+            if (i0 < L) {
+                if (gate) a0 = graw[cur * kC + i0];
+                b0 = braw[cur * kC + i0];
+            }
+            if (i1 < L) {
+                if (gate) a1 = graw[cur * kC + i1];
+                b1 = braw[cur * kC + i1];
+            }
+            const float g0 = (i0 < L) ? lg2(fmaxf(a0, FLT_MIN)) : 0.f;
+            const float g1 = (i1 < L) ? lg2(fmaxf(a1, FLT_MIN)) : 0.f;
+            float x = g0 + g1;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const float n = __shfl_up_sync(0xffffffffu, x, off);
-            if (lane >= off) x += n;
+            for (int off = 1; off < 32; off <<= 1) {
+                const float n = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += n;
+            }
+            const float l1 = x, l0 = x - g1;
+            lam[i0] = l0;
+            lam[i1] = l1;
+            bet[i0] = b0;
+            bet[i1] = b1;
+            bg[i0] = b0 * ex2(l0);
+            bg[i1] = b1 * ex2(l1);
         }
-        const float l1 = x, l0 = x - g1;
-        lam[i0] = l0;
-        lam[i1] = l1;
-        bet[i0] = b0;
-        bet[i1] = b1;
-        bg[i0] = b0 * ex2(l0);
-        bg[i1] = b1 * ex2(l1);
-    }
-    __syncthreads();
-    {   // G = K K^T -> Lm (j < t), Q K^T -> A (j <= t): warp w rows 16 (w & 3), columns 32 (w >> 2)
+        // G = K K^T -> Lm (j < t), Q K^T -> A (j <= t): warp w rows 16 (w & 3), columns 32 (w >> 2)
         const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
         const int g = lane >> 2, t4 = lane & 3;
         float gk[4][4] = {}, gq[4][4] = {};
         warp_mma_bf16<4, kD>(gk, m0, n0, Ks, kFacPitch, Ks, kFacPitch);
         warp_mma_bf16<4, kD>(gq, m0, n0, Qs, kFacPitch, Ks, kFacPitch);
+        __syncthreads();   // Q and K read (Lm, Tm take their places); the gates are in
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -309,26 +333,27 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
                 }
                 *reinterpret_cast<uint32_t *>(im + sw128_off(t, j >> 3) + (j & 7) * 2) = pack_bf16x2(a2[0], a2[1]);
             }
-    }
-    __syncthreads();
-    invert_unit_lower_rec<1, kFacT>(Lm, Tm, Zs, tid);
-    __syncthreads();
-    {   // T diag(b), T diag(b g) (lower triangle)
-        const int t = tid >> 2, j0 = 16 * (tid & 3);
-        float v1[16], v2[16];
+        __syncthreads();
+        invert_unit_lower_rec<1, kFacT>(Lm, Tm, Zs, tid);
+        __syncthreads();
+        {   // T diag(b), T diag(b g) (lower triangle)
+            const int t = tid >> 2, j0 = 16 * (tid & 3);
+            float v1[16], v2[16];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-            const int j = j0 + jj;
-            const float tj = (j <= t) ? Tm[t * kTStride + j] : 0.f;
-            v1[jj] = tj * bet[j];
-            v2[jj] = tj * bg[j];
+            for (int jj = 0; jj < 16; ++jj) {
+                const int j = j0 + jj;
+                const float tj = (j <= t) ? Tm[t * kTStride + j] : 0.f;
+                v1[jj] = tj * bet[j];
+                v2[jj] = tj * bg[j];
+            }
+            st_row_bf16x16(smem_u32(im + 8192), t, j0 >> 3, v1);
+            st_row_bf16x16(smem_u32(im + 16384), t, j0 >> 3, v2);
         }
-        st_row_bf16x16(smem_u32(im + 8192), t, j0 >> 3, v1);
-        st_row_bf16x16(smem_u32(im + 16384), t, j0 >> 3, v2);
+        __syncthreads();
+        uint4 *dst = reinterpret_cast<uint4 *>(img + (size_t)item * kImgHalves);
+        for (int p = tid; p < 3 * 512; p += kFacT) dst[p] = reinterpret_cast<const uint4 *>(im)[p];
     }
-    __syncthreads();
-    uint4 *dst = reinterpret_cast<uint4 *>(img + ((size_t)bh * nch + c) * kImgHalves);
-    for (int p = tid; p < 3 * 512; p += kFacT) dst[p] = reinterpret_cast<const uint4 *>(im)[p];
+    cp_async_wait_all();
 }
 
 template <bool TWO>
@@ -952,10 +977,16 @@ cudaError_t launch_prefill_gdn(const PrefillArgs &a, void *workspace, size_t wor
         e = cudaFuncSetAttribute(gdn_chunk_factors_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kFacBytes);
         if (e != cudaSuccess) return e;
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return cudaErrorUnknown;
+        const int total = BH * nch;
+        const int grid = total < 2 * sms ? total : 2 * sms;
         timer_begin(a.stream);
-        gdn_chunk_factors_kernel<<<(unsigned)BH * nch, kFacT, kFacBytes, a.stream>>>(
+        gdn_chunk_factors_kernel<<<(unsigned)grid, kFacT, kFacBytes, a.stream>>>(
             static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k), a.gate, a.beta, a.T,
-            nch, static_cast<__nv_bfloat16 *>(workspace));
+            nch, total, static_cast<__nv_bfloat16 *>(workspace));
         timer_end(a.stream);
         note_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
