@@ -175,6 +175,10 @@ BACKWARD_CONFIGS = {
     "gdn_bwd_bf16_b2h16t32768": Workload("gdn_bwd_bf16_b2h16t32768", MODE_GATED_DELTA, torch.bfloat16,
                                          B=2, H=16, T=32768, dk=128, dv=128, seed=12,
                                          qk_l2norm=True, gate="softplus", gate_shift=-3.0, beta=True),
+    # profiling case: the same recipe at an eighth of the length (counter captures)
+    "gdn_bwd_bf16_b2h16t4096": Workload("gdn_bwd_bf16_b2h16t4096", MODE_GATED_DELTA, torch.bfloat16,
+                                        B=2, H=16, T=4096, dk=128, dv=128, seed=12,
+                                        qk_l2norm=True, gate="softplus", gate_shift=-3.0, beta=True),
 }
 
 
