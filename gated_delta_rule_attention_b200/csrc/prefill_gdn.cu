@@ -67,7 +67,7 @@ constexpr int kThreads = 512;
 constexpr int kPrepT = 256;      // warps 4-11
 constexpr int kChainT = 128;     // warps 12-15
 // named barriers
-constexpr uint32_t kBarPrep = 1, kBarChain = 3, kBarChainE = 4, kBarChainO = 5;
+constexpr uint32_t kBarPrep = 1, kBarChain = 3, kBarChainE = 4;
 // A chunk whose column decay factor 2^(lam_{16b} - lam_j) inside a 16-token block exceeds
 // 2^kFastSpan takes the exact per-element exponentials (no overflow in the fast factors).
 constexpr float kFastSpan = 100.f;
@@ -804,16 +804,19 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
             // the stage's gates were observed in qw_step(c); read before the barrier below,
             // which precedes the stage's release (dS(c) is issued after it)
             const float gL = cur ? ex2(sm->gt[s].lam[kC - 1]) : 1.f;
-            if (cur) {
-                if (!group_wait(&sm->p_done, par, ce == 0, kBarChain, kChainT, abort, p.err)) break;
+            // P(c) done, and A E(c - 1) (which frees the E tiles and completes the outputs of
+            // chunk c - 1; the tensor core ran it before P(c)): one meeting of the chain
+            {
+                if (ce == 0) {
+                    if (cur) mbar_wait(&sm->p_done, par, abort, p.err);
+                    if (c >= 1) mbar_wait(&sm->ae_done[(c - 1) & 1], ((c - 1) >> 1) & 1, abort, p.err);
+                }
+                if (named_sync_any(kBarChain, kChainT, *abort != 0)) break;
                 tc_fence_after();
             }
             if (cq >= 2) {
                 if (cur) {
-                    // E = U - W S^T; the E tiles are free once A E(c - 1) is done
-                    if (c >= 1 && !group_wait(&sm->ae_done[(c - 1) & 1], ((c - 1) >> 1) & 1, row == 64,
-                                              kBarChainE, 64, abort, p.err))
-                        break;
+                    // E = U - W S^T
                     const int t = row - 64;
                     const int L = sm->gt[s].len;
                     const float *lam = sm->gt[s].lam;
@@ -851,10 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                 }
             } else if (c >= 1) {
                 // outputs of chunk c - 1: rows 0-63 of P (lanes 0-63), the slice's 32 columns
-                if (!group_wait(&sm->ae_done[(c - 1) & 1], ((c - 1) >> 1) & 1, row == 0, kBarChainO, 64,
-                                abort, p.err))
-                    break;
-                tc_fence_after();
+
                 const int t = row;
                 const int t0 = tb + kC * (c - 1);
                 const int L = min(kC, te - t0);
