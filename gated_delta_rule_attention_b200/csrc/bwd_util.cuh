@@ -104,6 +104,95 @@ __device__ __forceinline__ void warp_mma_bf16(float (&d)[NT][4], int m0, int n0,
     }
 }
 
+// ---- bf16 fragments by ldmatrix for mma.sync m16n8k16 (tiles row-major in shared memory,
+// pitch in bf16 elements; 16-byte aligned rows; a pitch of 2P bytes = 16 (mod 32) avoids
+// bank conflicts)
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_addr(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_addr(p)));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1]) : "r"(smem_addr(p)));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1]) : "r"(smem_addr(p)));
+}
+// The A fragment (rows m0..m0+15, k0..k0+15) of A = X (X row-major [m][k]) or, with TRANS,
+// of A = X^T (X row-major [k][m]).
+template <bool TRANS>
+__device__ __forceinline__ void frag_a(uint32_t (&a)[4], const __nv_bfloat16 *X, int pitch, int m0, int k0) {
+    const int l = threadIdx.x & 31;
+    if (!TRANS) ldsm_x4(a, X + (m0 + (l & 15)) * pitch + k0 + 8 * (l >> 4));
+    else ldsm_x4_t(a, X + (k0 + (l & 7) + 8 * (l >> 4)) * pitch + m0 + 8 * ((l >> 3) & 1));
+}
+// The B fragment (k0..k0+15, n0..n0+7) of B = X^T (X row-major [n][k]) or, with TRANS, of
+// B = X (X row-major [k][n]).
+template <bool TRANS>
+__device__ __forceinline__ void frag_b(uint32_t (&b)[2], const __nv_bfloat16 *X, int pitch, int k0, int n0) {
+    const int l = threadIdx.x & 15;
+    if (!TRANS) ldsm_x2(b, X + (n0 + (l & 7)) * pitch + k0 + 8 * (l >> 3));
+    else ldsm_x2_t(b, X + (k0 + l) * pitch + n0);
+}
+// frag_b on an unpadded tile of rows of `w` elements (w >= 64) whose 16-byte chunks are
+// XOR-swizzled by the row: chunk j of row r sits at chunk j ^ (r & 7).  Eight consecutive
+// rows at one logical chunk then fall in eight different bank groups.
+template <bool TRANS>
+__device__ __forceinline__ void frag_b_sw(uint32_t (&b)[2], const __nv_bfloat16 *X, int w, int k0, int n0) {
+    const int l = threadIdx.x & 15;
+    if (!TRANS) {
+        const int r = n0 + (l & 7), j = (k0 >> 3) + (l >> 3);
+        ldsm_x2(b, X + r * w + 8 * (j ^ (r & 7)));
+    } else {
+        const int r = k0 + l;
+        ldsm_x2_t(b, X + r * w + 8 * ((n0 >> 3) ^ (r & 7)));
+    }
+}
+// d[nt] += A B over K for the 16 x 8 NT block at (m0, n0), A and B bf16 tiles; an operand
+// given with a second (remainder) tile is taken as high + low parts: products
+// hi*hi + hi*lo + lo*hi (a computed fp32 value v = bf16(v) + bf16(v - bf16(v)) to 2^-17).
+// With SWB, B is a swizzled tile (frag_b_sw) and pb its row length.
+template <int NT, int K, bool TA, bool TB, bool SWB = false>
+__device__ __forceinline__ void mma_bf16_tiles(float (&d)[NT][4], int m0, int n0,
+                                               const __nv_bfloat16 *A, const __nv_bfloat16 *Alo, int pa,
+                                               const __nv_bfloat16 *B, const __nv_bfloat16 *Blo, int pb) {
+    auto fb = [&](uint32_t (&b)[2], const __nv_bfloat16 *X, int kk, int n) {
+        if constexpr (SWB) frag_b_sw<TB>(b, X, pb, kk, n);
+        else frag_b<TB>(b, X, pb, kk, n);
+    };
+#pragma unroll
+    for (int kk = 0; kk < K; kk += 16) {
+        uint32_t a[4], al[4];
+        frag_a<TA>(a, A, pa, m0, kk);
+        if (Alo) frag_a<TA>(al, Alo, pa, m0, kk);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            uint32_t b[2];
+            fb(b, B, kk, n0 + 8 * nt);
+            mma_16x8x16_bf16(d[nt], a, b[0], b[1]);
+            if (Blo) {
+                uint32_t bl[2];
+                fb(bl, Blo, kk, n0 + 8 * nt);
+                mma_16x8x16_bf16(d[nt], a, bl[0], bl[1]);
+            }
+            if (Alo) mma_16x8x16_bf16(d[nt], al, b[0], b[1]);
+        }
+    }
+}
+// v as bf16 high and low parts
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16 &hi, __nv_bfloat16 &lo) {
+    hi = __float2bfloat16_rn(v);
+    lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+
 // ---- cp.async staging of raw inputs (16-byte copies into shared memory)
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     const unsigned d = (unsigned)__cvta_generic_to_shared(dst);

@@ -204,7 +204,8 @@ def test_prefill_backward_argument_checks(lib):
     assert call(dk=32) == UNSUPPORTED
     assert call() == INVALID               # NULL tensors, before any launch
     assert call(mode=4) == INVALID         # mode 4 needs its gate
-    assert lib.la_backward_workspace_size(1, 2, 3, 100, 64, 64) == 4 * 2 * 3 * (5 * 64 * 64 + 100 * 65)
+    # 4 chunks: 9 [d_v, d_k] fp32-sized slots (states and cotangents) and dlam per (b, h)
+    assert lib.la_backward_workspace_size(1, 2, 3, 100, 64, 64) == 4 * 2 * 3 * (9 * 64 * 64 + 100)
     # delta rule: chunk-start states (4 chunks of 32), fp32 dq, dk, dL/dlam and db
     BH, T, nch = 6, 100, 4
     assert lib.la_backward_workspace_size(2, 2, 3, T, 64, 64) == 4 * (BH * nch * 64 * 64 + 2 * BH * T * 64
