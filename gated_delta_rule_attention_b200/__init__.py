@@ -25,7 +25,7 @@ import os
 import torch
 
 __all__ = ["MODE_ELU1_NORM", "MODE_GATED", "MODE_GATED_DELTA", "MODE_KDA", "MODE_RETNET", "FLAG_INIT_STATE", "LaError",
-           "prefill", "prefill_varlen", "prefill_backward", "prefill_backward_delta", "decode_step", "short_conv", "short_conv_varlen", "short_conv_step", "check_status", "library",
+           "prefill", "prefill_varlen", "prefill_backward", "prefill_backward_delta", "decode_step", "short_conv", "short_conv_varlen", "short_conv_step", "prefill_conv", "check_status", "library",
            "library_path", "version", "kernel_launches", "workspace_size"]
 
 MODE_ELU1_NORM = 0
@@ -103,6 +103,11 @@ def library():
     lib.la_short_conv_varlen.restype = i
     lib.la_short_conv_step.argtypes = [i, i, i, i, i, vp, fp, vp, vp, u, vp]
     lib.la_short_conv_step.restype = i
+    lib.la_prefill_conv_workspace_size.argtypes = [i, i, i]
+    lib.la_prefill_conv_workspace_size.restype = ctypes.c_size_t
+    lib.la_prefill_conv.argtypes = [i, i, i, i, i, i, vp, vp, vp, fp, fp, fp, vp, vp, u, u, vp, fp, fp,
+                                    fp, vp, u, vp, ctypes.c_size_t, vp]
+    lib.la_prefill_conv.restype = i
     lib.la_selftest_wait_timeout.argtypes = [vp]
     lib.la_selftest_wait_timeout.restype = i
     if hasattr(lib, "la_launch_timing"):   # diagnostic hook, absent from older builds
@@ -544,6 +549,60 @@ def short_conv_step(x, w, window, *, heads: int, silu: bool = False, l2norm: boo
                                       _conv_flags(silu, l2norm), _stream_handle(x.device, stream))
     _check(st, "la_short_conv_step")
     return y
+
+
+def prefill_conv(xq, xk, xv, wq, wk, wv, *, heads: int, beta, gate=None, window=None,
+                 window_out=None, qk_silu: bool = True, qk_l2norm: bool = True, v_silu: bool = True,
+                 state=None, init_state: bool | None = None, y=None, o=None, stream=None):
+    """A Gated DeltaNet layer's attention path from its projections (``la_prefill_conv``):
+    the short convolution of xq, xk, xv fused into the gated-delta prefill's loads.
+
+    xq, xk, xv: [B, T, H*128] bf16 token-major; wq, wk, wv: [H*128, width] fp32 taps;
+    window: [3, B, width-1, H*128] bf16 (the q, k, v windows; None: zeros); gate, beta:
+    [B, H, T] fp32; state: [B, H, 128, 128] fp32 (S_0 when ``init_state``, default: when
+    given).  SiLU and the head-row L2 norm apply to q and k per ``qk_silu`` /
+    ``qk_l2norm``, SiLU to v per ``v_silu``.  Returns (o [B, H, T, 128], state,
+    y [3, B, H, T, 128] the convolved q, k, v, window_out [3, B, width-1, H*128]).
+    """
+    B, T, C = xq.shape
+    width = wq.shape[1]
+    if C % heads:
+        raise ValueError("the projections' last dimension must be heads * d")
+    d = C // heads
+    dt = torch.bfloat16
+    for name, t in (("xq", xq), ("xk", xk), ("xv", xv)):
+        _need(t, (B, T, C), dt, name)
+    for name, t in (("wq", wq), ("wk", wk), ("wv", wv)):
+        _need(t, (C, width), torch.float32, name)
+    _need(beta, (B, heads, T), torch.float32, "beta")
+    if gate is not None:
+        _need(gate, (B, heads, T), torch.float32, "gate")
+    if window is not None:
+        _need(window, (3, B, width - 1, C), dt, "window")
+    if window_out is None:
+        window_out = torch.empty(3, B, width - 1, C, device=xq.device, dtype=dt)
+    _need(window_out, (3, B, width - 1, C), dt, "window_out")
+    if init_state is None:
+        init_state = state is not None
+    if state is None:
+        state = torch.empty(B, heads, d, d, device=xq.device, dtype=torch.float32)
+    _need(state, (B, heads, d, d), torch.float32, "state")
+    if y is None:
+        y = torch.empty(3, B, heads, T, d, device=xq.device, dtype=dt)
+    _need(y, (3, B, heads, T, d), dt, "y")
+    if o is None:
+        o = torch.empty(B, heads, T, d, device=xq.device, dtype=dt)
+    _need(o, (B, heads, T, d), dt, "o")
+    ws = _workspace(xq.device, int(library().la_prefill_conv_workspace_size(B, heads, T)), stream)
+    ws_bytes = 0 if ws is None else ws.numel()
+    st = library().la_prefill_conv(LA_BF16, B, heads, T, d, width, _ptr(xq), _ptr(xk), _ptr(xv),
+                                   _ptr(wq), _ptr(wk), _ptr(wv), _ptr(window), _ptr(window_out),
+                                   _conv_flags(qk_silu, qk_l2norm), _conv_flags(v_silu, False), _ptr(y),
+                                   _ptr(gate), _ptr(beta), _ptr(state), _ptr(o),
+                                   FLAG_INIT_STATE if init_state else 0, _ptr(ws), ws_bytes,
+                                   _stream_handle(xq.device, stream))
+    _check(st, "la_prefill_conv")
+    return o, state, y, window_out
 
 
 def selftest_wait_timeout(stream=None):

@@ -408,3 +408,71 @@ extern "C" int la_version(void) { return 100; }
 extern "C" unsigned long long la_kernel_launches(void) {
     return g_launches.load(std::memory_order_relaxed);
 }
+
+extern "C" size_t la_prefill_conv_workspace_size(int B, int H, int T) {
+    if (B < 1 || H < 1 || T < 1 || (long long)B * H > INT32_MAX) return 0;
+    return prefill_gdn_workspace_bytes(B * H, T);
+}
+
+extern "C" la_status_t la_prefill_conv(la_dtype_t dtype, int B, int H, int T, int d, int width,
+                                       const void *xq, const void *xk, const void *xv, const float *wq,
+                                       const float *wk, const float *wv, const void *window_in,
+                                       void *window_out, unsigned flags_qk, unsigned flags_v, void *y,
+                                       const float *gate, const float *beta, float *state, void *o,
+                                       unsigned flags, void *workspace, size_t workspace_bytes,
+                                       void *stream) {
+    timer_reset();
+    if (dtype != LA_BF16) return dtype == LA_F32 ? LA_ERR_UNSUPPORTED : LA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || T < 1 || width < 1 || width > 4) return LA_ERR_INVALID_ARG;
+    if (d != 128) return d == 64 ? LA_ERR_UNSUPPORTED : LA_ERR_INVALID_ARG;
+    if ((flags & ~LA_FLAG_INIT_STATE) || ((flags_qk | flags_v) & ~(LA_CONV_SILU | LA_CONV_L2NORM)))
+        return LA_ERR_INVALID_ARG;
+    const long long BH = (long long)B * H;
+    if (BH > INT32_MAX || BH * T * d > kMaxElems) return LA_ERR_INVALID_ARG;
+    const void *need16[] = {xq, xk, xv, y, o, state, workspace};
+    for (const void *p : need16)
+        if (!tensor_ok(p, 16)) return LA_ERR_INVALID_ARG;
+    const float *need4[] = {wq, wk, wv, beta};
+    for (const float *p : need4)
+        if (!tensor_ok(p, 4)) return LA_ERR_INVALID_ARG;
+    if (gate && !tensor_ok(gate, 4)) return LA_ERR_INVALID_ARG;
+    if (width > 1) {
+        if (window_in && !tensor_ok(window_in, 16)) return LA_ERR_INVALID_ARG;
+        if (window_out && !tensor_ok(window_out, 16)) return LA_ERR_INVALID_ARG;
+    }
+    if (workspace_bytes < la_prefill_conv_workspace_size(B, H, T)) return LA_ERR_INVALID_ARG;
+    const size_t th = (size_t)BH * T, xb = th * d * 2, win = (size_t)3 * B * (width - 1) * H * d * 2;
+    const size_t wb = sizeof(float) * (size_t)H * d * width;
+    if (!writes_disjoint({{y, 3 * xb}, {o, xb}, {state, sizeof(float) * BH * d * d},
+                          {width > 1 ? window_out : nullptr, win}, {workspace, workspace_bytes}},
+                         {{xq, xb}, {xk, xb}, {xv, xb}, {wq, wb}, {wk, wb}, {wv, wb},
+                          {width > 1 ? window_in : nullptr, win}, {gate, sizeof(float) * th},
+                          {beta, sizeof(float) * th}}))
+        return LA_ERR_INVALID_ARG;
+    PrefillArgs a;
+    a.mode = LA_MODE_GATED_DELTA;
+    a.dtype = LA_BF16;
+    a.B = B; a.H = H; a.T = T; a.dk = d; a.dv = d;
+    const __nv_bfloat16 *yb = static_cast<const __nv_bfloat16 *>(y);
+    a.q = yb;
+    a.k = yb + th * d;
+    a.v = yb + 2 * th * d;
+    a.gate = gate;
+    a.beta = beta;
+    a.state = state;
+    a.z = nullptr;
+    a.o = o;
+    a.chunk = 64;
+    a.init_state = (flags & LA_FLAG_INIT_STATE) != 0;
+    a.stream = static_cast<cudaStream_t>(stream);
+    ConvSpec cs;
+    cs.x[0] = xq; cs.x[1] = xk; cs.x[2] = xv;
+    cs.w[0] = wq; cs.w[1] = wk; cs.w[2] = wv;
+    cs.win_in = width > 1 ? window_in : nullptr;
+    cs.win_out = width > 1 ? window_out : nullptr;
+    cs.y = y;
+    cs.width = width;
+    cs.fqk = flags_qk;
+    cs.fv = flags_v;
+    return from_cuda(launch_prefill_gdn_conv(a, cs, workspace, workspace_bytes));
+}

@@ -18,15 +18,17 @@
 // The last identity follows from differentiating the decay mask exp(lam_s - lam_j): lam_u
 // enters with + where it is the reading position and with - where it is the written one.
 //
-// One or two CTAs per (batch, head) (the d_k columns of S and G split between them): a
-// forward sweep stores every chunk-start state in the caller's workspace, then a reverse
-// sweep carries G back through the chunks; a small kernel finishes dV and the gate gradient.
-// The products run on the tensor cores as warp-level mma (m16n8k8, tf32 operands, fp32
-// accumulate; each operand is split into a tf32 part and a remainder, three products,
-// fp32 accuracy): the tiles are 32 x 32 to 128 x 64, too small for tcgen05's
-// 128-row tiles and each followed by an element-wise step.  With bf16 I/O the next chunk's
-// inputs (and, in the reverse sweep, its start state) arrive by cp.async while the current
-// chunk is processed.
+// The products are 32 x 32 to 128 x 128 tiles, each followed by an element-wise step: they
+// run on the tensor cores as warp-level mma (bwd_util.cuh), with every computed operand
+// split into high and low parts so that the products keep fp32 accuracy.
+//
+// fp32 I/O: one or two CTAs per (batch, head) (the d_k columns of S and G split between
+// them): a forward sweep stores every chunk-start state in the caller's workspace, then a
+// reverse sweep carries G back through the chunks and forms each chunk's gradients; a
+// small kernel finishes dV and the gate gradient (m16n8k8 tf32 products).
+//
+// bf16 I/O: the two carries first (every S_c and G, one scan launch), then every chunk's
+// gradients at once, then the gate gradient (m16n8k16 bf16 products; see below).
 #include "la_internal.cuh"
 #include "bwd_util.cuh"
 
@@ -44,15 +46,13 @@ constexpr int kBwdC = 32;
 // updates), and a share of those that sum over them (dV, dlam), which it adds into fp32
 // accumulators in the workspace; a finishing kernel converts dV and takes the suffix sums.
 // Row pitches are 4 (mod 32) floats (conflict-free mma operand loads).
-template <int DK, int DV, int SPLIT, bool STAGE>
+template <int DK, int DV, int SPLIT>
 struct BwdSmem {
     static constexpr int DKH = DK / SPLIT;
     static constexpr int PQ = DK + 4, PV = DV + 4, PS = DKH + 4, PC = kBwdC + 4;
     static constexpr int kQ = kBwdC * PQ, kV = kBwdC * PV, kS = DV * PS, kP = kBwdC * PC;
-    // staged raw bf16 rows of q, k, v, dO (2 bytes each: C (2 DK + 2 DV) / 2 floats)
-    static constexpr int kRaw = STAGE ? kBwdC * (DK + DV) : 0;
-    // Qs Ks | Vs dOs | S, S' (double buffer), G | P dP | raw | lam gv dec dl graw | red
-    static constexpr int kFloats = 2 * kQ + 2 * kV + 3 * kS + 2 * kP + kRaw + 5 * kBwdC + 8;
+    // Qs Ks | Vs dOs | S, S_c, G | P dP | lam gv dec dl | red
+    static constexpr int kFloats = 2 * kQ + 2 * kV + 3 * kS + 2 * kP + 4 * kBwdC + 8;
     static constexpr size_t kBytes = sizeof(float) * kFloats;
     static_assert(kBytes <= 227 * 1024, "shared memory");
 };
@@ -75,21 +75,19 @@ __device__ __forceinline__ float block_sum(float x, float *red) {
 __device__ __forceinline__ int frow(int m0, int r) { return m0 + ((threadIdx.x & 31) >> 2) + 8 * (r >> 1); }
 __device__ __forceinline__ int fcol(int n0, int nt, int r) { return n0 + 8 * nt + 2 * (threadIdx.x & 3) + (r & 1); }
 
-template <int DK, int DV, int SPLIT, typename IO>
+template <int DK, int DV, int SPLIT>
 __global__ void __launch_bounds__(kBwdThreads)
-backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__restrict__ k,
-                const IO *__restrict__ v, const float *__restrict__ gate,
-                const float *__restrict__ S0, const IO *__restrict__ dO,
-                const float *__restrict__ dST, IO *__restrict__ dq, IO *__restrict__ dk,
+backward_kernel(int T, int gate_heads, const float *__restrict__ q, const float *__restrict__ k,
+                const float *__restrict__ v, const float *__restrict__ gate,
+                const float *__restrict__ S0, const float *__restrict__ dO,
+                const float *__restrict__ dST, float *__restrict__ dq, float *__restrict__ dk,
                 float *__restrict__ dS0, float *__restrict__ ws, float *__restrict__ dv_acc,
                 float *__restrict__ dl_acc) {
-    constexpr bool STAGE = std::is_same<IO, __nv_bfloat16>::value;
-    // Operand splitting (bwd_util.cuh): computed operands (S, G, P, dP, scaled rows) are
-    // always split -- the gate gradient is a suffix sum over the whole sequence, where one
-    // tf32 rounding per product adds up; the inputs q, k, v, dO are split only for fp32 I/O
-    // (bf16 values are exact in tf32).
-    constexpr bool SP = std::is_same<IO, float>::value;
-    using L = BwdSmem<DK, DV, SPLIT, STAGE>;
+    // Operand splitting (bwd_util.cuh): every operand is split -- fp32 inputs have more
+    // mantissa than tf32, and the gate gradient is a suffix sum over the whole sequence,
+    // where one tf32 rounding per product adds up.
+    constexpr bool SP = true;
+    using L = BwdSmem<DK, DV, SPLIT>;
     constexpr int C = kBwdC, DKH = L::DKH, PQ = L::PQ, PV = L::PV, PS = L::PS, PC = L::PC;
     constexpr int NW = kBwdThreads / 32;
     // DV x DKH state tiles: DV / 16 row blocks of 16, the warps left over split the columns
@@ -107,15 +105,11 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
     float *G = Sb1 + L::kS;          // [DV][PS]  dL/dS at the chunk's end
     float *P = G + L::kS;            // [C][PC]
     float *dP = P + L::kP;           // [C][PC]
-    float *raw = dP + L::kP;         // staged q | k | v | dO rows (bf16)
-    float *lam = raw + L::kRaw;      // [C]   in-chunk log-gate prefix
+    float *lam = dP + L::kP;         // [C]   in-chunk log-gate prefix
     float *gv = lam + C;             // [C]   g_t = exp(lam_t)
     float *dec = gv + C;             // [C]   g_L / g_t
     float *dl = dec + C;             // [C]   this CTA's share of dlam
-    float *graw = dl + C;            // [C]   staged gates
-    float *red = graw + C;           // [8]
-    __nv_bfloat16 *rq = reinterpret_cast<__nv_bfloat16 *>(raw);
-    __nv_bfloat16 *rk = rq + C * DK, *rv = rk + C * DK, *rdo = rv + C * DV;
+    float *red = dl + C;             // [8]
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const size_t bh = blockIdx.x / SPLIT;
@@ -129,12 +123,12 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
               nv = (DV / 4) * (warp >> 1);
     const int ms = 16 * (warp % RB), ns = (DKH / CG) * (warp / RB);
 
-    // gates of chunk t0 (Lc tokens): from the staged copy or global memory
-    auto load_gates = [&](int t0, int Lc, bool staged) {
+    // gates of chunk t0 (Lc tokens)
+    auto load_gates = [&](int t0, int Lc) {
         if (warp == 0) {
             const int lane = tid & 31;
             float a = 1.f;
-            if (gh && lane < Lc) a = staged && gt ? graw[lane] : gh[(size_t)(t0 + lane) * gt];
+            if (gh && lane < Lc) a = gh[(size_t)(t0 + lane) * gt];
             float x = lane < Lc ? logf(fmaxf(a, FLT_MIN)) : 0.f;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -147,22 +141,10 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
             dec[lane] = expf(xl - x);
         }
     };
-    // stage chunk c's rows (k, v; with `rev` also q, dO) and gates
-    auto stage = [&](int c, bool rev) {
-        const int t0 = c * C, Lc = min(C, T - t0);
-        stage_rows<kBwdThreads>(rk, k + (row0 + t0) * DK, DK, DK, Lc);
-        stage_rows<kBwdThreads>(rv, v + (row0 + t0) * DV, DV, DV, Lc);
-        if (rev) {
-            stage_rows<kBwdThreads>(rq, q + (row0 + t0) * DK, DK, DK, Lc);
-            stage_rows<kBwdThreads>(rdo, dO + (row0 + t0) * DV, DV, DV, Lc);
-        }
-        if (gh && gt && tid >= 64 && tid - 64 < Lc) cp_async4(graw + tid - 64, gh + t0 + tid - 64);
-        cp_async_commit();
-    };
-    auto load_direct = [&](const IO *src, float *dst, int t0, int Lc, int d, int pitch) {
+    auto load_direct = [&](const float *src, float *dst, int t0, int Lc, int d, int pitch) {
         for (int p = tid; p < C * d; p += kBwdThreads) {
             const int i = p / d, j = p % d;
-            dst[i * pitch + j] = i < Lc ? to_f32(src[(row0 + t0 + i) * d + j]) : 0.f;
+            dst[i * pitch + j] = i < Lc ? src[(row0 + t0 + i) * d + j] : 0.f;
         }
     };
 
@@ -170,7 +152,6 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
     float *S = Sb0;
     for (int p = tid; p < DV * DKH; p += kBwdThreads)
         S[(p / DKH) * PS + p % DKH] = S0 ? S0[bh * DV * DK + (p / DKH) * DK + c0 + p % DKH] : 0.f;
-    if constexpr (STAGE) stage(0, false);
     __syncthreads();
     for (int c = 0; c <= nch; ++c) {
         for (int p = tid; p < DV * DKH / 4; p += kBwdThreads) {   // store S (float4)
@@ -180,18 +161,10 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
         }
         if (c == nch) break;
         const int t0 = c * C, Lc = min(C, T - t0);
-        if constexpr (STAGE) {
-            cp_async_wait_all();
-            __syncthreads();
-            unstage<kBwdThreads, IO>(rk, C, DK, Lc, Ks, PQ);
-            unstage<kBwdThreads, IO>(rv, C, DV, Lc, Vs, PV);
-        } else {
-            load_direct(k, Ks, t0, Lc, DK, PQ);
-            load_direct(v, Vs, t0, Lc, DV, PV);
-        }
-        load_gates(t0, Lc, STAGE);
+        load_direct(k, Ks, t0, Lc, DK, PQ);
+        load_direct(v, Vs, t0, Lc, DV, PV);
+        load_gates(t0, Lc);
         __syncthreads();
-        if constexpr (STAGE) if (c + 1 < nch) stage(c + 1, false);
         // S <- g_L S + (dec o V)^T K   (this CTA's columns; state partition)
         const float gL = gv[Lc - 1];
         float acc[NTS][4] = {};
@@ -219,45 +192,17 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
     const float final_dot = block_sum(part0, red);
     if (tid == 0 && final_dot != 0.f) atomicAdd(&dl_acc[row0 + T - 1], final_dot);
     float *Sc = (S == Sb0) ? Sb1 : Sb0;   // the chunk's start state
-    float *Sn = S;                        // the next (earlier) chunk's, staged meanwhile
-    auto stage_state = [&](int c, float *dst) {
-        const float *src = wsh + (size_t)c * DV * DKH;
-        for (int p = tid; p < DV * DKH / 4; p += kBwdThreads) {
-            const int i = p / (DKH / 4), j = 4 * (p % (DKH / 4));
-            cp_async16(dst + i * PS + j, src + i * DKH + j);
-        }
-    };
-    if constexpr (STAGE) {
-        __syncthreads();   // S_T read
-        stage_state(nch - 1, Sc);
-        stage(nch - 1, true);
-    }
     for (int c = nch - 1; c >= 0; --c) {
         const int t0 = c * C, Lc = min(C, T - t0);
-        if constexpr (STAGE) {
-            cp_async_wait_all();
-            __syncthreads();
-            unstage<kBwdThreads, IO>(rq, C, DK, Lc, Qs, PQ);
-            unstage<kBwdThreads, IO>(rk, C, DK, Lc, Ks, PQ);
-            unstage<kBwdThreads, IO>(rv, C, DV, Lc, Vs, PV);
-            unstage<kBwdThreads, IO>(rdo, C, DV, Lc, dOs, PV);
-        } else {
-            load_direct(q, Qs, t0, Lc, DK, PQ);
-            load_direct(k, Ks, t0, Lc, DK, PQ);
-            load_direct(v, Vs, t0, Lc, DV, PV);
-            load_direct(dO, dOs, t0, Lc, DV, PV);
-            const float *src = wsh + (size_t)c * DV * DKH;
-            for (int p = tid; p < DV * DKH; p += kBwdThreads) Sc[(p / DKH) * PS + p % DKH] = src[p];
-        }
+        load_direct(q, Qs, t0, Lc, DK, PQ);
+        load_direct(k, Ks, t0, Lc, DK, PQ);
+        load_direct(v, Vs, t0, Lc, DV, PV);
+        load_direct(dO, dOs, t0, Lc, DV, PV);
+        const float *src = wsh + (size_t)c * DV * DKH;
+        for (int p = tid; p < DV * DKH; p += kBwdThreads) Sc[(p / DKH) * PS + p % DKH] = src[p];
         if (tid < C) dl[tid] = 0.f;
-        load_gates(t0, Lc, STAGE);
+        load_gates(t0, Lc);
         __syncthreads();
-        if constexpr (STAGE) {
-            if (c > 0) {   // the staging buffers and Sn are free
-                stage_state(c - 1, Sn);
-                stage(c - 1, true);
-            }
-        }
         {   // causal decayed score matrices P = (Q K^T) o D, dP = (dO V^T) o D
             float pp[1][4] = {}, dd[1][4] = {};
             warp_mma<1, DK, SP>(pp, mq, n32, [&](int t, int cc) { return Qs[t * PQ + cc]; },
@@ -298,8 +243,8 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
                     const int t = frow(mq, r), cc = c0 + fcol(nq, nt, r);
                     part[r >> 1] += Qs[t * PQ + cc] * aq[nt][r] - Ks[t * PQ + cc] * ak[nt][r];
                     if (t < Lc) {
-                        dq[(row0 + t0 + t) * DK + cc] = from_f32<IO>(aq[nt][r]);
-                        dk[(row0 + t0 + t) * DK + cc] = from_f32<IO>(ak[nt][r]);
+                        dq[(row0 + t0 + t) * DK + cc] = aq[nt][r];
+                        dk[(row0 + t0 + t) * DK + cc] = ak[nt][r];
                     }
                 }
 #pragma unroll
@@ -352,9 +297,6 @@ backward_kernel(int T, int gate_heads, const IO *__restrict__ q, const IO *__res
                 }
         }
         __syncthreads();
-        float *tmp = Sc;
-        Sc = Sn;
-        Sn = tmp;
     }
     if (dS0)
         for (int p = tid; p < DV * DKH; p += kBwdThreads)
@@ -808,18 +750,18 @@ cudaError_t launch_bwd(int BH, int T, int gate_heads, const void *q, const void 
         return cudaGetLastError();
     } else {
         constexpr int SPLIT = bwd_split<DK>();
-        using L = BwdSmem<DK, DV, SPLIT, false>;
+        using L = BwdSmem<DK, DV, SPLIT>;
         float *dv_acc = ws + (size_t)BH * (nch + 1) * DV * DK;
         float *dl_acc = dv_acc + (size_t)BH * T * DV;
         e = cudaMemsetAsync(dv_acc, 0, sizeof(float) * (size_t)BH * T * (DV + 1), st);
         if (e != cudaSuccess) return e;
-        auto kern = backward_kernel<DK, DV, SPLIT, IO>;
+        auto kern = backward_kernel<DK, DV, SPLIT>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
         if (e != cudaSuccess) return e;
         timer_begin(st);
         kern<<<(unsigned)(BH * SPLIT), kBwdThreads, L::kBytes, st>>>(
-            T, gate_heads, static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v),
-            gate, S0, static_cast<const IO *>(dO), dST, static_cast<IO *>(dq), static_cast<IO *>(dk), dS0,
+            T, gate_heads, static_cast<const float *>(q), static_cast<const float *>(k), static_cast<const float *>(v),
+            gate, S0, static_cast<const float *>(dO), dST, static_cast<float *>(dq), static_cast<float *>(dk), dS0,
             ws, dv_acc, dl_acc);
         timer_end(st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -89,6 +89,19 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t work
 // whether it serves a call of BH head rows (dense or packed), and its launcher.
 bool prefill_gdn_selected(int mode, int BH, bool packed);
 cudaError_t launch_prefill_gdn(const PrefillArgs &a, void *workspace, size_t workspace_bytes);
+// la_prefill_conv: the short convolution of q, k, v fused into the gated-delta prefill's
+// first pass (dense, bf16, d = 128; the workspace of the two-pass variant is required).
+struct ConvSpec {
+    const void *x[3];      // [B, T, H*128] token-major q, k, v projections
+    const float *w[3];     // [H*128, width] taps
+    const void *win_in;    // [3, B, width-1, H*128] or nullptr
+    void *win_out;         // [3, B, width-1, H*128] or nullptr; never overlaps win_in
+    void *y;               // [3, B, H, T, 128] out: the convolved q, k, v
+    int width;
+    unsigned fqk, fv;      // LA_CONV_* flags for q and k, for v
+};
+cudaError_t launch_prefill_gdn_conv(const PrefillArgs &a, const ConvSpec &cs, void *workspace,
+                                    size_t workspace_bytes);
 // Workspace with which it runs its two-pass variant (per-chunk factors formed in parallel).
 size_t prefill_gdn_workspace_bytes(int BH, int T);
 cudaError_t launch_short_conv(const ConvArgs &a);

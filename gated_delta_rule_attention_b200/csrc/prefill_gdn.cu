@@ -236,36 +236,155 @@ constexpr uint32_t kFacL = kFacG + 4 * kC * 4;                 // lam, bet, bg [
 constexpr uint32_t kFacBytes = kFacL + 3 * kC * 4;
 constexpr int kImgHalves = 3 * 4096;                           // bf16 elements per chunk record
 
+// Fused variant: q, k, v come from the token-major projections x through the short causal
+// convolution (with the SiLU and the head-row L2 norm per flags) of the lesson page's
+// section "Hybrids of 2025: Qwen3-Next and Kimi Linear", computed here as the rows arrive;
+// the convolved q, k, v go out for pass 2 (and the caller).  The arithmetic is that of the
+// stand-alone convolution kernel, operation for operation, so the two give the same bits.
+struct FacConv {
+    const __nv_bfloat16 *x[3];     // [B, T, H*128] token-major q, k, v projections
+    const float *w[3];             // [H*128, width] taps
+    const __nv_bfloat16 *win_in;   // [3, B, width-1, H*128] or nullptr (zeros)
+    __nv_bfloat16 *win_out;        // [3, B, width-1, H*128] or nullptr (never overlaps win_in)
+    __nv_bfloat16 *y;              // [3, B, H, T, 128] out
+    int B, H, width;
+    unsigned fqk, fv;              // LA_CONV_SILU | LA_CONV_L2NORM for q and k, for v
+};
+template <bool CONV>
+struct FacLay {   // the raw rows of the fused variant carry the 3 tokens before the chunk
+    static constexpr uint32_t kHalo = CONV ? 3 * kFacPitch * 2 : 0;
+    static constexpr uint32_t kTile = kHalo + kFacTile;                   // one Q or K buffer
+    static constexpr uint32_t kBuf = 2 * kTile;
+    static constexpr uint32_t kZs = 2 * kBuf;
+    static constexpr uint32_t kImg = (kZs + 4 * 272 * 4 + 1023) & ~1023u;  // also the raw v rows
+    static constexpr uint32_t kG = kImg + 3 * 8192;
+    static constexpr uint32_t kL = kG + 4 * kC * 4;
+    static constexpr uint32_t kBytes = kL + 3 * kC * 4;
+    static_assert(kHalo % 16 == 0 && kTile % 16 == 0, "16-byte rows");
+    static_assert(67 * 256 <= 3 * 8192, "raw v rows fit the image area");
+};
+static_assert(FacLay<false>::kBytes == kFacBytes, "plain layout");
+
+__device__ __forceinline__ float silu_tanh(float u) {   // u sigmoid(u), sigmoid = (1 + tanh(u/2)) / 2
+    float t;
+    const float h = 0.5f * u;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
+}
+__device__ __forceinline__ void unpack8(const uint4 &r, float (&f)[8]) {   // bf16 -> fp32 is exact
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        f[2 * j] = __uint_as_float(w[j] << 16);
+        f[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+}
+// Taps of 8 channels c0 .. c0 + 7 aligned to the window: e[3] multiplies the current token,
+// e[k] (k < 3) the token 3 - k before it (zero where the width has no tap).
+__device__ __forceinline__ void load_taps_aligned(const float *w, int width, size_t c0, float (&e)[4][8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float *wc = w + (c0 + j) * width;
+        e[3][j] = wc[width - 1];
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int i = k - (4 - width);   // tap index of the token 3 - k back
+            e[k][j] = i >= 0 ? wc[i] : 0.f;
+        }
+    }
+}
+// One token's 8 channels: u = w[W-1] x_t + sum_{i < W-1} w[i] x_{t-(W-1)+i} (in that order),
+// then SiLU and the head-row L2 norm per `fl` (the row's 16 chunks are the 16 lanes of a
+// half-warp: every lane of the warp calls this together).  win[k] is the token 3 - k back.
+__device__ __forceinline__ uint4 conv_token(const float (&e)[4][8], int width, const uint4 (&win)[3],
+                                            const uint4 &xr, unsigned fl) {
+    float x[8], u[8];
+    unpack8(xr, x);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) u[j] = e[3][j] * x[j];
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+        if (k >= 4 - width) {
+            float p[8];
+            unpack8(win[k], p);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) u[j] = fmaf(e[k][j], p[j], u[j]);
+        }
+    if (fl & LA_CONV_SILU)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) u[j] = silu_tanh(u[j]);
+    if (fl & LA_CONV_L2NORM) {
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s = fmaf(u[j], u[j], s);
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        const float r = rsqrtf(s + 1e-6f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) u[j] *= r;
+    }
+    return make_uint4(pack_bf16x2(u[0], u[1]), pack_bf16x2(u[2], u[3]), pack_bf16x2(u[4], u[5]),
+                      pack_bf16x2(u[6], u[7]));
+}
+
 // Each CTA takes chunks blockIdx.x, blockIdx.x + gridDim.x, ... (chunk i = head row i / nch,
 // chunk i % nch); the next chunk's rows, gates and rates arrive by cp.async while the
 // current one is processed.  Lm and Tm of the inverse take the places of the chunk's Q and
-// K tiles once the Gram products have read them.
+// K tiles once the Gram products have read them.  With CONV the staged rows are raw
+// projections (3 tokens in front of the chunk included), convolved in place; the raw v
+// rows arrive in the image area and are convolved straight out after the Gram products.
+template <bool CONV>
 __global__ void __launch_bounds__(kFacT, 2)
 gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                          const float *__restrict__ gate, const float *__restrict__ beta, int T, int nch,
-                         int total, __nv_bfloat16 *__restrict__ img) {
+                         int total, __nv_bfloat16 *__restrict__ img, const FacConv cv) {
+    using FL = FacLay<CONV>;
     extern __shared__ __align__(1024) uint8_t fsm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    float *Zs = reinterpret_cast<float *>(fsm + kFacZs);
-    uint8_t *im = fsm + kFacImg;
-    float *graw = reinterpret_cast<float *>(fsm + kFacG), *braw = graw + 2 * kC;
-    float *lam = reinterpret_cast<float *>(fsm + kFacL), *bet = lam + kC, *bg = bet + kC;
+    float *Zs = reinterpret_cast<float *>(fsm + FL::kZs);
+    uint8_t *im = fsm + FL::kImg;
+    float *graw = reinterpret_cast<float *>(fsm + FL::kG), *braw = graw + 2 * kC;
+    float *lam = reinterpret_cast<float *>(fsm + FL::kL), *bet = lam + kC, *bg = bet + kC;
     auto chunk_of = [&](int item, size_t &row0, int &L) {
         const int bh = item / nch, c = item % nch;
         row0 = (size_t)bh * T + (size_t)c * kC;
         L = min(kC, T - c * kC);
+    };
+    const int W1 = CONV ? cv.width - 1 : 0;
+    const size_t Cx = CONV ? (size_t)cv.H * kD : 0;   // channels of a projection row
+    // (fused) the 16-byte piece x8 .. x8 + 7 of head h's channels of projection z at token t
+    // of batch row b: the projection, else the carried window, else nothing (zeros)
+    auto raw_src = [&](int z, int b, int h, int t, int x8) -> const __nv_bfloat16 * {
+        if (t >= T) return nullptr;
+        // (selects, not an indexed parameter array: that would go through local memory)
+        const __nv_bfloat16 *xz = z == 0 ? cv.x[0] : (z == 1 ? cv.x[1] : cv.x[2]);
+        if (t >= 0) return xz + ((size_t)b * T + t) * Cx + (size_t)h * kD + x8;
+        const int j = W1 + t;
+        if (j < 0 || !cv.win_in) return nullptr;
+        return cv.win_in + (((size_t)z * cv.B + b) * W1 + j) * Cx + (size_t)h * kD + x8;
     };
     // rows [0, L) of q and k (16-byte copies; rows past L zeroed), gates and rates
     auto stage = [&](int item, int buf) {
         size_t row0;
         int L;
         chunk_of(item, row0, L);
-        uint8_t *base = fsm + buf * kFacBuf;
-        for (int p = tid; p < 2 * kC * 16; p += kFacT) {
-            const int which = p >> 10, r = (p >> 4) & 63, x = p & 15;
-            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(base + which * kFacTile) + r * kFacPitch + 8 * x;
-            if (r < L) cp_async16(dst, (which ? k : q) + (row0 + r) * kD + 8 * x);
-            else *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        uint8_t *base = fsm + buf * FL::kBuf;
+        if constexpr (CONV) {   // 67 raw rows: tokens c*64 - 3 .. c*64 + 63
+            const int bh = item / nch, c = item % nch, b = bh / cv.H, h = bh % cv.H;
+            for (int p = tid; p < 2 * 67 * 16; p += kFacT) {
+                const int which = p / (67 * 16), r = (p >> 4) % 67, x = p & 15;
+                __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(base + which * FL::kTile) + r * kFacPitch + 8 * x;
+                const __nv_bfloat16 *s = raw_src(which, b, h, c * kC - 3 + r, 8 * x);
+                if (s) cp_async16(dst, s);
+                else *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+            }
+        } else {
+            for (int p = tid; p < 2 * kC * 16; p += kFacT) {
+                const int which = p >> 10, r = (p >> 4) & 63, x = p & 15;
+                __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(base + which * FL::kTile) + r * kFacPitch + 8 * x;
+                if (r < L) cp_async16(dst, (which ? k : q) + (row0 + r) * kD + 8 * x);
+                else *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+            }
         }
         if (tid < L) cp_async4(braw + buf * kC + tid, beta + row0 + tid);
         if (gate && tid >= 64 && tid - 64 < L) cp_async4(graw + buf * kC + tid - 64, gate + row0 + tid - 64);
@@ -277,13 +396,57 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
         size_t row0;
         int L;
         chunk_of(item, row0, L);
-        __nv_bfloat16 *Qs = reinterpret_cast<__nv_bfloat16 *>(fsm + cur * kFacBuf);
-        __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(fsm + cur * kFacBuf + kFacTile);
-        float *Lm = reinterpret_cast<float *>(fsm + cur * kFacBuf);            // over Q
-        float *Tm = reinterpret_cast<float *>(fsm + cur * kFacBuf + kFacTile); // over K
+        __nv_bfloat16 *Qs = reinterpret_cast<__nv_bfloat16 *>(fsm + cur * FL::kBuf + FL::kHalo);
+        __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(fsm + cur * FL::kBuf + FL::kTile + FL::kHalo);
+        float *Lm = reinterpret_cast<float *>(Qs);   // over Q
+        float *Tm = reinterpret_cast<float *>(Ks);   // over K
         cp_async_wait_all();
         __syncthreads();   // this chunk's rows are in; the other buffer and the images are free
-        if (item + (int)gridDim.x < total) stage(item + gridDim.x, cur ^ 1);
+        const bool pref = item + (int)gridDim.x < total;
+        if constexpr (CONV) {
+            const int bh = item / nch, c = item % nch, b = bh / cv.H, h = bh % cv.H;
+            // the raw v rows into the image area (their own commit group, ahead of the prefetch)
+            for (int p = tid; p < 67 * 16; p += kFacT) {
+                const int r = p >> 4, x = p & 15;
+                const __nv_bfloat16 *s = raw_src(2, b, h, c * kC - 3 + r, 8 * x);
+                if (s) cp_async16(im + r * 256 + 16 * x, s);
+                else *reinterpret_cast<uint4 *>(im + r * 256 + 16 * x) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            cp_async_commit();
+            if (c == nch - 1 && cv.win_out) {   // the carried windows after the sequence
+                for (int p = tid; p < 3 * W1 * 16; p += kFacT) {
+                    const int z = p / (W1 * 16), j = (p >> 4) % W1, x = p & 15;
+                    const __nv_bfloat16 *s = raw_src(z, b, h, T - W1 + j, 8 * x);
+                    *reinterpret_cast<uint4 *>(cv.win_out + (((size_t)z * cv.B + b) * W1 + j) * Cx + (size_t)h * kD + 8 * x) =
+                        s ? *reinterpret_cast<const uint4 *>(s) : make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+        }
+        if (pref) stage(item + gridDim.x, cur ^ 1);
+        if constexpr (CONV) {
+            // q (threads 0-127) and k (128-255) in place: a thread takes the 8 channels cc of
+            // tokens 8 rr .. 8 rr + 7, the 16 chunks of a token row in one half-warp
+            const int z = tid >> 7, rr = (tid >> 4) & 7, cc = tid & 15;
+            const int bh = item / nch, h = bh % cv.H;
+            const uint32_t rows = smem_u32(fsm + cur * FL::kBuf + z * FL::kTile) + 16 * cc;
+            float wr[4][8];
+            load_taps_aligned(z ? cv.w[1] : cv.w[0], cv.width, (size_t)h * kD + 8 * cc, wr);
+            // the run's 8 raw rows and the 3 in front of it, all loaded before any is replaced
+            uint4 xr[11];
+#pragma unroll
+            for (int i = 0; i < 11; ++i) xr[i] = lds128(rows + (8 * rr + i) * (kFacPitch * 2));
+            __syncthreads();   // every thread holds the raw rows it reads
+            __nv_bfloat16 *yz = cv.y + (size_t)z * cv.B * cv.H * T * kD + row0 * kD + 8 * cc;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int t = 8 * rr + i;
+                const uint4 win[3] = {xr[i], xr[i + 1], xr[i + 2]};
+                const uint4 o = conv_token(wr, cv.width, win, xr[i + 3], cv.fqk);
+                sts128(rows + (t + 3) * (kFacPitch * 2), t < L ? o : make_uint4(0u, 0u, 0u, 0u));
+                if (t < L) *reinterpret_cast<uint4 *>(yz + (size_t)t * kD) = o;
+            }
+            __syncthreads();   // the chunk's q and k rows are convolved
+        }
         if (warp == 0) {   // lane l takes tokens 2l, 2l + 1, as pass 2's gate warp
             float a0 = 1.f, a1 = 1.f, b0 = 0.f, b1 = 0.f;
             const int i0 = 2 * lane, i1 = 2 * lane + 1;
@@ -317,7 +480,30 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
         float gk[4][4] = {}, gq[4][4] = {};
         warp_mma_bf16<4, kD>(gk, m0, n0, Ks, kFacPitch, Ks, kFacPitch);
         warp_mma_bf16<4, kD>(gq, m0, n0, Qs, kFacPitch, Ks, kFacPitch);
+        if constexpr (CONV) {
+            if (pref) asm volatile("cp.async.wait_group 1;" ::: "memory");   // the raw v rows
+            else asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
         __syncthreads();   // Q and K read (Lm, Tm take their places); the gates are in
+        if constexpr (CONV) {   // v: 16 runs of 4 tokens, straight out (no head norm unless asked)
+            const int rr = tid >> 4, cc = tid & 15;
+            const int bh = item / nch, h = bh % cv.H;
+            const uint32_t rows = smem_u32(im) + 16 * cc;
+            float wr[4][8];
+            load_taps_aligned(cv.w[2], cv.width, (size_t)h * kD + 8 * cc, wr);
+            uint4 xr[7];
+#pragma unroll
+            for (int i = 0; i < 7; ++i) xr[i] = lds128(rows + (4 * rr + i) * 256);
+            __nv_bfloat16 *yv = cv.y + (size_t)2 * cv.B * cv.H * T * kD + row0 * kD + 8 * cc;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = 4 * rr + i;
+                const uint4 win[3] = {xr[i], xr[i + 1], xr[i + 2]};
+                const uint4 o = conv_token(wr, cv.width, win, xr[i + 3], cv.fv);
+                if (t < L) *reinterpret_cast<uint4 *>(yv + (size_t)t * kD) = o;
+            }
+            __syncthreads();   // the raw v rows are read: the image area is free
+        }
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -944,7 +1130,8 @@ size_t prefill_gdn_workspace_bytes(int BH, int T) {
 // With a workspace of at least prefill_gdn_workspace_bytes (dense calls), pass 1 forms every
 // chunk's A, T diag(b), T diag(b g) at once and the chain kernel reads them (two-pass);
 // otherwise the single pass forms them itself.
-cudaError_t launch_prefill_gdn(const PrefillArgs &a, void *workspace, size_t workspace_bytes) {
+namespace {
+cudaError_t launch_gdn(const PrefillArgs &a, void *workspace, size_t workspace_bytes, const ConvSpec *cs) {
     const int BH = a.cu ? a.H : a.B * a.H;
     GdnParams p;
     memset(&p, 0, sizeof(p));
@@ -969,13 +1156,31 @@ cudaError_t launch_prefill_gdn(const PrefillArgs &a, void *workspace, size_t wor
     const int units = a.cu ? a.nseq * a.H : BH;
     const bool two = !a.cu && workspace && (reinterpret_cast<uintptr_t>(workspace) & 15u) == 0 &&
                      workspace_bytes >= prefill_gdn_workspace_bytes(BH, a.T);
+    if (cs && !two) return cudaErrorInvalidValue;   // the fused convolution lives in pass 1
     cudaError_t e;
     if (two) {
         const int nch = (a.T + kC - 1) / kC;
         p.img = static_cast<const __nv_bfloat16 *>(workspace);
         p.nchunks = nch;
-        e = cudaFuncSetAttribute(gdn_chunk_factors_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kFacBytes);
+        FacConv fc;
+        memset(&fc, 0, sizeof(fc));
+        if (cs) {
+            for (int z = 0; z < 3; ++z) {
+                fc.x[z] = static_cast<const __nv_bfloat16 *>(cs->x[z]);
+                fc.w[z] = cs->w[z];
+            }
+            fc.win_in = static_cast<const __nv_bfloat16 *>(cs->win_in);
+            fc.win_out = static_cast<__nv_bfloat16 *>(cs->win_out);
+            fc.y = static_cast<__nv_bfloat16 *>(cs->y);
+            fc.B = a.B;
+            fc.H = a.H;
+            fc.width = cs->width;
+            fc.fqk = cs->fqk;
+            fc.fv = cs->fv;
+        }
+        auto fac = cs ? gdn_chunk_factors_kernel<true> : gdn_chunk_factors_kernel<false>;
+        const uint32_t fbytes = cs ? FacLay<true>::kBytes : FacLay<false>::kBytes;
+        e = cudaFuncSetAttribute(fac, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fbytes);
         if (e != cudaSuccess) return e;
         int dev = 0, sms = 148;
         if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -984,9 +1189,9 @@ cudaError_t launch_prefill_gdn(const PrefillArgs &a, void *workspace, size_t wor
         const int total = BH * nch;
         const int grid = total < 2 * sms ? total : 2 * sms;
         timer_begin(a.stream);
-        gdn_chunk_factors_kernel<<<(unsigned)grid, kFacT, kFacBytes, a.stream>>>(
+        fac<<<(unsigned)grid, kFacT, fbytes, a.stream>>>(
             static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k), a.gate, a.beta, a.T,
-            nch, total, static_cast<__nv_bfloat16 *>(workspace));
+            nch, total, static_cast<__nv_bfloat16 *>(workspace), fc);
         timer_end(a.stream);
         note_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1000,6 +1205,18 @@ cudaError_t launch_prefill_gdn(const PrefillArgs &a, void *workspace, size_t wor
     timer_end(a.stream);
     note_launches(1);
     return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_prefill_gdn(const PrefillArgs &a, void *workspace, size_t workspace_bytes) {
+    return launch_gdn(a, workspace, workspace_bytes, nullptr);
+}
+
+// Pass 1 convolves the projections as it loads them and writes the convolved q, k, v
+// (a.q, a.k, a.v point into cs.y); pass 2 reads those.
+cudaError_t launch_prefill_gdn_conv(const PrefillArgs &a, const ConvSpec &cs, void *workspace,
+                                    size_t workspace_bytes) {
+    return launch_gdn(a, workspace, workspace_bytes, &cs);
 }
 
 }  // namespace la

@@ -261,6 +261,36 @@ la_status_t la_short_conv_step(la_dtype_t dtype, int N, int H, int d, int width,
                                unsigned flags, void *stream);
 
 /*
+ * la_prefill_conv -- a Gated DeltaNet layer's attention path from its projections: the
+ * short convolution of section "Hybrids of 2025: Qwen3-Next and Kimi Linear" (as
+ * la_short_conv) fused into the loads of the gated-delta prefill ([delta rule], mode 2, as
+ * la_prefill with a workspace).  The prefill's first pass
+ * reads the token-major projections with the three tokens in front of each chunk,
+ * convolves them as they arrive and writes the convolved q, k, v once; the second pass
+ * reads those.  The results equal three la_short_conv calls followed by la_prefill (mode
+ * 2) on the same two-pass kernels, bit for bit.
+ *
+ *   dtype        LA_BF16 (LA_F32: LA_ERR_UNSUPPORTED)
+ *   d            128 (= d_k = d_v; 64: LA_ERR_UNSUPPORTED); width 1..4
+ *   xq, xk, xv   [B, T, H*d] token-major projections
+ *   wq, wk, wv   [H*d, width] fp32 taps
+ *   window_in    [3, B, width-1, H*d] the q, k, v windows in front of x_0, or NULL (zeros)
+ *   window_out   [3, B, width-1, H*d] out, or NULL; must not overlap window_in
+ *   flags_qk, flags_v   LA_CONV_SILU | LA_CONV_L2NORM for q and k, for v
+ *   y            [3, B, H, T, d] out: the convolved q, k, v (the backward pass takes them)
+ *   gate, beta, state, o, flags   as la_prefill in mode 2 (gate [B, H, T] or NULL)
+ *   workspace    at least la_prefill_conv_workspace_size() bytes (required), 16-byte aligned
+ * T >= 1.  No output may overlap an input; LA_ERR_INVALID_ARG otherwise.  Two launches.
+ */
+size_t la_prefill_conv_workspace_size(int B, int H, int T);
+la_status_t la_prefill_conv(la_dtype_t dtype, int B, int H, int T, int d, int width, const void *xq,
+                            const void *xk, const void *xv, const float *wq, const float *wk,
+                            const float *wv, const void *window_in, void *window_out,
+                            unsigned flags_qk, unsigned flags_v, void *y, const float *gate,
+                            const float *beta, float *state, void *o, unsigned flags,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * la_prefill_backward -- gradients of the prefill for the scalar-gate modes (1 and 4):
  * the derivatives of L = sum_t do_t . o_t + <dS_T, S_T> for the recurrence of
  * [decay/gates], S_t = a_t S_{t-1} + v_t k_t^T, o_t = S_t q_t, with respect to q, k, v, the
@@ -269,7 +299,10 @@ la_status_t la_short_conv_step(la_dtype_t dtype, int N, int H, int d, int width,
  *   dQ = diag(g) dO S_c + dP K,  dK = dP^T Q + diag(g_L/g) V G,  dV = P^T dO + diag(g_L/g) K G^T
  * per chunk (P = (Q K^T) o D, dP = (dO V^T) o D, S_c the chunk-start state, G = dL/dS at
  * the chunk's end), and d log a_t = sum_{u >= t} (q_u . dq_u - k_u . dk_u) (plus
- * <dS_T, S_T> at the last token).  CUDA cores, fp32 arithmetic, one CTA per (b, h).
+ * <dS_T, S_T> at the last token).  Warp-level tensor-core products with fp32 accuracy
+ * (computed operands split into high and low parts), fp32 accumulation.  bf16 I/O: three
+ * launches (the chunk-start states and chunk-end cotangents, every chunk's gradients, the
+ * gate gradient); fp32 I/O: two (forward and reverse sweeps, then dv and the gate gradient).
  *
  *   mode          LA_MODE_GATED or LA_MODE_RETNET (others: LA_ERR_UNSUPPORTED)
  *   q, k          [B, H, T, d_k] I/O dtype      v, dO [B, H, T, d_v] I/O dtype
@@ -281,7 +314,8 @@ la_status_t la_short_conv_step(la_dtype_t dtype, int N, int H, int d, int width,
  *                 gates as fixed and requires NULL.  Gates must be > 0: d a = d log a / a.
  *   dstate0       out [B, H, d_v, d_k] fp32 (the gradient of state0), or NULL
  *   workspace     device scratch of at least la_backward_workspace_size() bytes
- *                 (required: every chunk-start state is kept there)
+ *                 (required: every chunk-start state, and with bf16 I/O every chunk-end
+ *                 cotangent, is kept there)
  * la_backward_workspace_size also sizes la_prefill_backward_delta's workspace (modes 2, 3).
  */
 size_t la_backward_workspace_size(la_mode_t mode, int B, int H, int T, int d_k, int d_v);

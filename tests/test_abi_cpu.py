@@ -229,3 +229,27 @@ def test_prefill_backward_delta_argument_checks(lib):
     assert call(dtype=5) == INVALID
     assert call() == INVALID               # NULL tensors, before any launch
     assert call(mode=3) == INVALID
+
+
+def test_prefill_conv_argument_checks(lib):
+    """la_prefill_conv refuses what it has no kernel for and malformed calls before any
+    launch (no GPU needed: every check below fails before a pointer is used)."""
+    INVALID, UNSUPPORTED = 1, 2
+
+    def call(dtype=1, B=1, H=2, T=64, d=128, width=4, flags=0, fqk=6, fv=2):
+        return lib.la_prefill_conv(dtype, B, H, T, d, width, *([None] * 8), fqk, fv, *([None] * 5),
+                                   flags, None, 0, None)
+    assert call(dtype=0) == UNSUPPORTED      # fp32: the fused path is bf16 only
+    assert call(dtype=7) == INVALID
+    assert call(d=64) == UNSUPPORTED
+    assert call(d=96) == INVALID
+    assert call(width=0) == INVALID
+    assert call(width=5) == INVALID
+    assert call(T=0) == INVALID
+    assert call(flags=2) == INVALID
+    assert call(fqk=8) == INVALID
+    assert call() == INVALID                 # NULL tensors
+    # the two-pass images: 3 x 8 KB per chunk of 64 tokens
+    assert lib.la_prefill_conv_workspace_size(2, 16, 32768) == 32 * 512 * 24576
+    assert lib.la_prefill_conv_workspace_size(1, 1, 65) == 2 * 24576
+    assert lib.la_prefill_conv_workspace_size(0, 1, 64) == 0
