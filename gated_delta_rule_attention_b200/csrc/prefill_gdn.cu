@@ -431,21 +431,30 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
             const uint32_t rows = smem_u32(fsm + cur * FL::kBuf + z * FL::kTile) + 16 * cc;
             float wr[4][8];
             load_taps_aligned(z ? cv.w[1] : cv.w[0], cv.width, (size_t)h * kD + 8 * cc, wr);
-            // the run's 8 raw rows and the 3 in front of it, all loaded before any is replaced
-            uint4 xr[11];
+            // the 3 raw rows in front of the run are read before any thread replaces them
+            uint4 win[3];
 #pragma unroll
-            for (int i = 0; i < 11; ++i) xr[i] = lds128(rows + (8 * rr + i) * (kFacPitch * 2));
-            __syncthreads();   // every thread holds the raw rows it reads
-            __nv_bfloat16 *yz = cv.y + (size_t)z * cv.B * cv.H * T * kD + row0 * kD + 8 * cc;
-#pragma unroll
+            for (int i = 0; i < 3; ++i) win[i] = lds128(rows + (8 * rr + i) * (kFacPitch * 2));
+            __syncthreads();
+#pragma unroll 2
             for (int i = 0; i < 8; ++i) {
                 const int t = 8 * rr + i;
-                const uint4 win[3] = {xr[i], xr[i + 1], xr[i + 2]};
-                const uint4 o = conv_token(wr, cv.width, win, xr[i + 3], cv.fqk);
-                sts128(rows + (t + 3) * (kFacPitch * 2), t < L ? o : make_uint4(0u, 0u, 0u, 0u));
-                if (t < L) *reinterpret_cast<uint4 *>(yz + (size_t)t * kD) = o;
+                const uint32_t a = rows + (t + 3) * (kFacPitch * 2);
+                const uint4 xr = lds128(a);
+                const uint4 o = conv_token(wr, cv.width, win, xr, cv.fqk);
+                sts128(a, t < L ? o : make_uint4(0u, 0u, 0u, 0u));
+                win[0] = win[1];
+                win[1] = win[2];
+                win[2] = xr;
             }
+            fence_async_smem();   // the rows leave by bulk copies below
             __syncthreads();   // the chunk's q and k rows are convolved
+            if (tid < 2 * kC && (tid & 63) < L) {   // row tid & 63 of q (threads 0-63) or k
+                const int zz = tid >> 6, t = tid & 63;
+                bulk_store(cv.y + (size_t)zz * cv.B * cv.H * T * kD + (row0 + t) * kD,
+                           smem_u32(fsm + cur * FL::kBuf + zz * FL::kTile) + (t + 3) * (kFacPitch * 2), 2 * kD);
+                tma_store_commit();
+            }
         }
         if (warp == 0) {   // lane l takes tokens 2l, 2l + 1, as pass 2's gate warp
             float a0 = 1.f, a1 = 1.f, b0 = 0.f, b1 = 0.f;
@@ -483,6 +492,7 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
         if constexpr (CONV) {
             if (pref) asm volatile("cp.async.wait_group 1;" ::: "memory");   // the raw v rows
             else asm volatile("cp.async.wait_group 0;" ::: "memory");
+            tma_store_wait_read<0>();   // the q, k rows have left the tiles
         }
         __syncthreads();   // Q and K read (Lm, Tm take their places); the gates are in
         if constexpr (CONV) {   // v: 16 runs of 4 tokens, straight out (no head norm unless asked)
@@ -491,18 +501,28 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
             const uint32_t rows = smem_u32(im) + 16 * cc;
             float wr[4][8];
             load_taps_aligned(cv.w[2], cv.width, (size_t)h * kD + 8 * cc, wr);
-            uint4 xr[7];
+            uint4 win[3];
 #pragma unroll
-            for (int i = 0; i < 7; ++i) xr[i] = lds128(rows + (4 * rr + i) * 256);
-            __nv_bfloat16 *yv = cv.y + (size_t)2 * cv.B * cv.H * T * kD + row0 * kD + 8 * cc;
-#pragma unroll
+            for (int i = 0; i < 3; ++i) win[i] = lds128(rows + (4 * rr + i) * 256);
+            __syncthreads();   // the rows in front of every run are read: convolve in place
+#pragma unroll 2
             for (int i = 0; i < 4; ++i) {
                 const int t = 4 * rr + i;
-                const uint4 win[3] = {xr[i], xr[i + 1], xr[i + 2]};
-                const uint4 o = conv_token(wr, cv.width, win, xr[i + 3], cv.fv);
-                if (t < L) *reinterpret_cast<uint4 *>(yv + (size_t)t * kD) = o;
+                const uint32_t a = rows + (t + 3) * 256;
+                const uint4 xr = lds128(a);
+                sts128(a, conv_token(wr, cv.width, win, xr, cv.fv));
+                win[0] = win[1];
+                win[1] = win[2];
+                win[2] = xr;
             }
-            __syncthreads();   // the raw v rows are read: the image area is free
+            fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {   // the chunk's v rows are contiguous in shared and global memory
+                bulk_store(cv.y + (size_t)2 * cv.B * cv.H * T * kD + row0 * kD, smem_u32(im) + 3 * 256, L * 2 * kD);
+                tma_store_commit();
+                tma_store_wait_read<0>();
+            }
+            __syncthreads();   // the v rows have left: the image area is free
         }
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
@@ -540,6 +560,7 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
         for (int p = tid; p < 3 * 512; p += kFacT) dst[p] = reinterpret_cast<const uint4 *>(im)[p];
     }
     cp_async_wait_all();
+    if constexpr (CONV) tma_store_wait_all<0>();
 }
 
 template <bool TWO>

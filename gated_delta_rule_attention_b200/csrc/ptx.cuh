@@ -107,6 +107,12 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+// Untiled bulk copy of `bytes` (a multiple of 16) from shared `src` to global `dst` (both
+// 16-byte aligned), in the thread's bulk group (tma_store_commit / tma_store_wait_*).
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
 // Prefetch the 3-D box at (x, y, z) into L2 (no shared memory, no completion).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int x, int y, int z) {
     asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
