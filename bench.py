@@ -617,8 +617,85 @@ def compact(res, roof, cpu):
             "e2e": _sig(res["e2e"]["value"]) if res.get("e2e") else None}
 
 
+class LayerCase:
+    """One step = a Gated DeltaNet layer's attention path from its projections: the short
+    convolution of q, k, v (SiLU, q/k L2 norm) and the gated-delta prefill, either fused
+    (la_prefill_conv) or as three la_short_conv calls and la_prefill."""
+
+    def __init__(self, la, lw: W.LayerWorkload, device, rank):
+        self.la, self.lw, self.device = la, lw, device
+        cw, pw = lw.conv, lw.prefill
+        self.x, self.wt = [], []
+        for i in range(3):
+            x, w, _ = W.conv_inputs(cw.B, cw.T, cw.H * 128, cw.width, cw.dtype,
+                                    seed=cw.seed + 10 * i + 1000 * rank, device=device, window=False)
+            self.x.append(x)
+            self.wt.append(w)
+        inp = W.prefill_inputs(W.variant(pw, seed=pw.seed + 1000 * rank), device=device)
+        self.gate, self.beta = inp["gate"], inp["beta"]
+        del inp
+        B, H, T = cw.B, cw.H, cw.T
+        self.y = torch.empty(3, B, H, T, 128, device=device, dtype=cw.dtype)
+        self.win = torch.empty(3, B, cw.width - 1, H * 128, device=device, dtype=cw.dtype)
+        self.o = torch.empty(B, H, T, 128, device=device, dtype=cw.dtype)
+        self.state = torch.empty(B, H, 128, 128, device=device)
+        self.tokens = lw.tokens
+        pb, pf = prefill_algorithmic(pw)
+        e = io_bytes(cw.dtype)
+        th = B * H * T * 128
+        # projections in, convolved q, k, v out (the layer's backward takes them), then the
+        # prefill's bytes without its q, k, v reads (they are the rows just written)
+        self.bytes = float(3 * th * e + 3 * th * e + pb - 3 * th * e
+                           + 3 * (H * 128 * cw.width * 4 + B * (cw.width - 1) * H * 128 * e))
+        self.flops = float(3 * 2 * cw.width * th + pf)
+        self.kind = "layer"
+
+    def _call(self, x, collect=None):
+        la, cw = self.la, self.lw.conv
+        if self.lw.fused:
+            la.prefill_conv(*x, *self.wt, heads=cw.H, gate=self.gate, beta=self.beta, window_out=self.win,
+                            y=self.y, o=self.o, state=self.state, init_state=False)
+            if collect is not None:
+                collect.extend(la.launch_times())
+            return
+        for i in range(3):
+            la.short_conv(x[i], self.wt[i], heads=cw.H, window_out=self.win[i], silu=cw.silu,
+                          l2norm=cw.l2norm_qk and i < 2, y=self.y[i])
+            if collect is not None:
+                collect.extend(la.launch_times())
+        la.prefill(self.y[0], self.y[1], self.y[2], mode=2, gate=self.gate, beta=self.beta,
+                   state=self.state, o=self.o, init_state=False, workspace="auto")
+        if collect is not None:
+            collect.extend(la.launch_times())
+
+    def step(self):
+        self._call(self.x)
+
+    def step_collect(self):
+        out = []
+        self._call(self.x, out)
+        return out
+
+    def e2e_setup(self):
+        self.h_x = [x.to("cpu").pin_memory() for x in self.x]
+        self.h_g = [t.to("cpu").pin_memory() for t in (self.gate, self.beta)]
+        self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_x + self.h_g)
+        self.d2h = self.h_o.numel() * self.h_o.element_size()
+
+    def e2e_step(self):
+        for hx, x in zip(self.h_x, self.x):
+            x.copy_(hx, non_blocking=True)
+        self.gate.copy_(self.h_g[0], non_blocking=True)
+        self.beta.copy_(self.h_g[1], non_blocking=True)
+        self._call(self.x)
+        self.h_o.copy_(self.o, non_blocking=True)
+
+
 def measure(la, name, args, dist, device, rank, world, flush, with_e2e, sampler=None):
-    if name in W.CONV_CONFIGS:
+    if name in W.LAYER_CONFIGS:
+        case = LayerCase(la, W.LAYER_CONFIGS[name], device, rank)
+    elif name in W.CONV_CONFIGS:
         case = ConvCase(la, W.CONV_CONFIGS[name], device, rank)
     elif name in W.VARLEN_CONFIGS:
         case = VarlenCase(la, W.VARLEN_CONFIGS[name], device, rank)
@@ -698,6 +775,21 @@ def oracle_sample_other(name, budget_s):
         # one token = the three projections q, k, v
         return {"value": T / el / 3, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                 "sample": f"1 x {T} tokens of one {cw.H}x{cw.dk} projection (fp64 numpy), /3"}
+    if name in W.LAYER_CONFIGS:
+        from oracle import conv as oc
+        lw = W.LAYER_CONFIGS[name]
+        cw = lw.conv
+        xs = [f(W.conv_inputs(1, 512, 128, cw.width, cw.dtype, seed=cw.seed + i, window=False)[0]) for i in range(3)]
+        ws_ = [f(W.conv_inputs(1, 1, 128, cw.width, cw.dtype, seed=cw.seed + i, window=False)[1]) for i in range(3)]
+        inp = W.prefill_inputs(W.variant(lw.prefill, B=1, H=1, T=512), device="cpu")
+
+        def run(n):
+            ys = [oc.short_conv(xs[i][:, :n], ws_[i], H=1, silu=cw.silu, l2norm=cw.l2norm_qk and i < 2)[0]
+                  for i in range(3)]
+            oracle.prefill(2, ys[0], ys[1], ys[2], f(inp["gate"])[:, :, :n], f(inp["beta"])[:, :, :n])
+        T, el = _timed_growing(run, 64, 512, budget_s)
+        return {"value": T / el / cw.H, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+                "sample": f"1 head x {T} tokens: fp64 convolution (numpy) then the fp64 C recurrence, /{cw.H} heads"}
     if name in W.VARLEN_CONFIGS:
         vw = W.VARLEN_CONFIGS[name]
         L = sorted(vw.lengths())[: max(2, vw.N // 8)]
@@ -825,6 +917,14 @@ def workload_config(name, world):
                           "H": cw.H, "T": cw.T, "d_k": cw.dk, "d_v": cw.dv, "width": cw.width,
                           "silu": cw.silu, "l2norm_qk": cw.l2norm_qk, "global_batch": cw.B * world,
                           "seq_len": cw.T, **common}
+    if name in W.LAYER_CONFIGS:
+        lw = W.LAYER_CONFIGS[name]
+        cw = lw.conv
+        return cw.dtype, {"workload": name, "kind": "short convolution + gated-delta prefill ("
+                          + ("fused" if lw.fused else "separate calls") + ")", "mode": 2, "B": cw.B,
+                          "H": cw.H, "T": cw.T, "d_k": 128, "d_v": 128, "width": cw.width,
+                          "global_batch": cw.B * world, "seq_len": cw.T, "state_dtype": "f32",
+                          "accum": "f32", **common}
     if name in W.VARLEN_CONFIGS:
         vw = W.VARLEN_CONFIGS[name]
         L = vw.lengths()
@@ -847,7 +947,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=sorted(list(W.CONFIGS) + list(W.CONV_CONFIGS) + list(W.VARLEN_CONFIGS) +
-                                   list(W.BACKWARD_CONFIGS)))
+                                   list(W.BACKWARD_CONFIGS) + list(W.LAYER_CONFIGS)))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--extras", type=int, default=-1,
                     help="1: also measure the other workloads (default: on at N=1)")
@@ -880,7 +980,8 @@ def main():
         for name in ("elu1_f32_small", "elu1_bf16_b4h16t4096", "gated_bf16_b8h16t8192",
                      "gdn_bf16_b2h16t32768", "gdn_decode_n256h32", "kda_bf16_b2h16t32768",
                      "kda_decode_n256h32", "conv_bf16_b2h16t32768", "gdn_varlen_bf16_n64h16",
-                     "retnet_bf16_b8h16t8192", "gated_bwd_bf16_b4h16t4096", "gdn_bwd_bf16_b2h16t32768"):
+                     "retnet_bf16_b8h16t8192", "gated_bwd_bf16_b4h16t4096", "gdn_bwd_bf16_b2h16t32768",
+                     "gdn_layer_fused_bf16_b2h16t32768", "gdn_layer_split_bf16_b2h16t32768"):
             if name == args.workload:
                 continue
             r = measure(la, name, args, dist, device, rank, world, flush, True)

@@ -14,7 +14,8 @@ if ROOT not in sys.path:
 import bench  # noqa: E402
 import workloads as W  # noqa: E402
 
-ALL = (list(W.CONFIGS) + list(W.CONV_CONFIGS) + list(W.VARLEN_CONFIGS) + list(W.BACKWARD_CONFIGS))
+ALL = (list(W.CONFIGS) + list(W.CONV_CONFIGS) + list(W.VARLEN_CONFIGS) + list(W.BACKWARD_CONFIGS)
+       + list(W.LAYER_CONFIGS))
 
 
 @pytest.mark.parametrize("name", ALL)

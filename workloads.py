@@ -210,6 +210,27 @@ CONV_CONFIGS = {
 }
 
 
+# A Gated DeltaNet layer's attention path from its projections: the convolution above, then
+# the gated-delta prefill workload (its gate and beta recipe), fused in one call
+# (la_prefill_conv) or as the separate calls (three la_short_conv, la_prefill).
+@dataclasses.dataclass(frozen=True)
+class LayerWorkload:
+    name: str
+    conv: "ConvWorkload"
+    prefill: "Workload"
+    fused: bool
+
+    @property
+    def tokens(self) -> int:
+        return self.conv.B * self.conv.T
+
+
+LAYER_CONFIGS = {
+    n: LayerWorkload(n, CONV_CONFIGS["conv_bf16_b2h16t32768"], CONFIGS["gdn_bf16_b2h16t32768"], fused)
+    for n, fused in (("gdn_layer_fused_bf16_b2h16t32768", True), ("gdn_layer_split_bf16_b2h16t32768", False))
+}
+
+
 def conv_inputs(B, T, C, width, dtype, seed, device="cpu", window=True):
     """Projection output x [B,T,C] ~ N(0,1), taps w [C,width] ~ N(0,1)/sqrt(width) (fp32),
     carried window [B,width-1,C] ~ N(0,1) (or None).  Draw order: x, w, window."""
