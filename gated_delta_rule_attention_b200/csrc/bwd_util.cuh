@@ -74,11 +74,8 @@ __device__ __forceinline__ void warp_mma(float (&d)[NT][4], int m0, int n0, FA a
     }
 }
 
-// Warp-level bf16 products (mma.sync m16n8k16, fp32 accumulate) on bf16 tiles in shared
-// memory: d[nt] += sum_{k<K} A[m][k] B[n][k] for the 16 x 8 NT block at rows m0.., columns
-// n0..; A and B are row-major bf16 with row pitches lda, ldb (elements, even), so that each
-// fragment register is one 32-bit load of two consecutive k.  Element r of d[nt] sits as in
-// warp_mma.
+// Warp-level bf16 products (mma.sync m16n8k16, fp32 accumulate): d += A B for one 16 x 8
+// block; element r of d sits as in warp_mma.  The fragments come from ldmatrix below.
 __device__ __forceinline__ void mma_16x8x16_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                                  uint32_t b1) {
     asm volatile(
@@ -87,23 +84,6 @@ __device__ __forceinline__ void mma_16x8x16_bf16(float (&d)[4], const uint32_t (
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-template <int NT, int K>
-__device__ __forceinline__ void warp_mma_bf16(float (&d)[NT][4], int m0, int n0, const __nv_bfloat16 *A,
-                                              int lda, const __nv_bfloat16 *B, int ldb) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
-    auto w32 = [](const __nv_bfloat16 *p) { return *reinterpret_cast<const uint32_t *>(p); };
-#pragma unroll 4
-    for (int kk = 0; kk < K; kk += 16) {
-        const __nv_bfloat16 *a0 = A + (m0 + g) * lda + kk + 2 * t4, *a1 = a0 + 8 * lda;
-        const uint32_t af[4] = {w32(a0), w32(a1), w32(a0 + 8), w32(a1 + 8)};
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const __nv_bfloat16 *b = B + (n0 + 8 * nt + g) * ldb + kk + 2 * t4;
-            mma_16x8x16_bf16(d[nt], af, w32(b), w32(b + 8));
-        }
-    }
-}
-
 // ---- bf16 fragments by ldmatrix for mma.sync m16n8k16 (tiles row-major in shared memory,
 // pitch in bf16 elements; 16-byte aligned rows; a pitch of 2P bytes = 16 (mod 32) avoids
 // bank conflicts)

@@ -487,8 +487,19 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
         const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
         const int g = lane >> 2, t4 = lane & 3;
         float gk[4][4] = {}, gq[4][4] = {};
-        warp_mma_bf16<4, kD>(gk, m0, n0, Ks, kFacPitch, Ks, kFacPitch);
-        warp_mma_bf16<4, kD>(gq, m0, n0, Qs, kFacPitch, Ks, kFacPitch);
+#pragma unroll 4
+        for (int kk = 0; kk < kD; kk += 16) {   // both products share the K fragments (ldmatrix)
+            uint32_t ak[4], aq[4];
+            frag_a<false>(ak, Ks, kFacPitch, m0, kk);
+            frag_a<false>(aq, Qs, kFacPitch, m0, kk);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                uint32_t b[2];
+                frag_b<false>(b, Ks, kFacPitch, kk, n0 + 8 * nt);
+                mma_16x8x16_bf16(gk[nt], ak, b[0], b[1]);
+                mma_16x8x16_bf16(gq[nt], aq, b[0], b[1]);
+            }
+        }
         if constexpr (CONV) {
             if (pref) asm volatile("cp.async.wait_group 1;" ::: "memory");   // the raw v rows
             else asm volatile("cp.async.wait_group 0;" ::: "memory");
