@@ -159,3 +159,39 @@ def test_fused_refuses_bad_arguments(la):
     xq.copy_(x3[0])
     with pytest.raises(la.LaError):   # y over an input
         la.prefill_conv(xq, *x3[1:], *w3, heads=H, gate=gate, beta=beta, y=buf[:3 * n].view(3, B, H, T, 128))
+
+
+def test_fused_full_size_sampled(la):
+    """The benchmark's layer workload in its launch configuration (B2 H16 T32768): the fused
+    call equals the separate calls bit for bit, the convolution outputs match the oracle on
+    sampled token ranges, and sampled heads' outputs and final states match the oracle's
+    recurrence on the convolved q, k, v."""
+    lw = W.LAYER_CONFIGS["gdn_layer_fused_bf16_b2h16t32768"]
+    cw, pw = lw.conv, lw.prefill
+    B, H, T = cw.B, cw.H, cw.T
+    xs = [W.conv_inputs(B, T, H * 128, cw.width, cw.dtype, seed=cw.seed + 10 * i, device="cuda", window=False)
+          for i in range(3)]
+    inp = W.prefill_inputs(pw, device="cuda")
+    gate, beta = inp["gate"], inp["beta"]
+    del inp
+    x3, w3 = [x for x, _, _ in xs], [w for _, w, _ in xs]
+    o, S, y, wout = la.prefill_conv(*x3, *w3, heads=H, gate=gate, beta=beta)
+    ys = [la.short_conv(x3[i], w3[i], heads=H, silu=True, l2norm=(i < 2))[0] for i in range(3)]
+    o2, S2, _ = la.prefill(*ys, mode=la.MODE_GATED_DELTA, gate=gate, beta=beta)
+    la.check_status()
+    for i in range(3):
+        assert torch.equal(y[i], ys[i]), f"y[{i}]"
+    assert torch.equal(o, o2) and torch.equal(S, S2)
+    for i in range(3):
+        np.testing.assert_array_equal(f64(wout[i]), f64(x3[i][:, -3:]))
+    for b, t0, n in [(0, 0, 40), (1, 17000, 33), (1, T - 50, 50)]:
+        for i in range(3):
+            win = x3[i][b:b + 1, t0 - 3:t0] if t0 >= 3 else None
+            ref, _ = oconv.short_conv(f64(x3[i][b:b + 1, t0:t0 + n]), f64(w3[i]), None if win is None else f64(win),
+                                      H=H, silu=True, l2norm=(i < 2))
+            close(y[i][b:b + 1, :, t0:t0 + n], ref, True)
+    for b, h in [(0, 3), (1, 12)]:
+        sl = lambda t: f64(t[b:b + 1, h:h + 1])
+        ro, rS, _ = oracle.prefill(2, sl(y[0]), sl(y[1]), sl(y[2]), sl(gate), sl(beta))
+        assert slice_rel_err(sl(o), ro) < TOL[BF], f"o head ({b},{h})"
+        assert slice_rel_err(sl(S), rS) < TOL[BF], f"S head ({b},{h})"
