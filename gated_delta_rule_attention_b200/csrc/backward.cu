@@ -837,6 +837,7 @@ extern "C" la_status_t la_prefill_backward(la_mode_t mode, la_dtype_t dtype, int
     if (!((d_k == 64 || d_k == 128) && (d_v == 64 || d_v == 128))) return LA_ERR_UNSUPPORTED;
     const long long BH = (long long)B * H;
     if (BH > INT32_MAX || BH * T * (long long)(d_k > d_v ? d_k : d_v) > (1ll << 40)) return LA_ERR_INVALID_ARG;
+    if (BH * 2 * (d_v / kScanRows) > INT32_MAX) return LA_ERR_INVALID_ARG;   // the scan's grid
     if (mode == LA_MODE_RETNET && (!gate || dgate)) return LA_ERR_INVALID_ARG;   // gamma is fixed
     if (mode == LA_MODE_GATED && dgate && !gate) return LA_ERR_INVALID_ARG;
     const void *need[] = {q, k, v, dO, dq, dk, dv};
