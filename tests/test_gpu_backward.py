@@ -96,3 +96,33 @@ def test_backward_full_size_sampled(la):
         for name, x, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv), ("dgate", dg, rg)):
             e = slice_rel_err(sl(x), r)
             assert e < TOL[w.dtype], f"{name} head ({b},{h}): {e:.3e}"
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+@pytest.mark.parametrize("T", [1, 33, 300])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_backward_bf16_head_sizes(la, dk, dv, T, with_state):
+    """bf16 I/O runs the state scans and the per-chunk kernel: every head-size pair they are
+    built for, ragged tails, one and many chunks."""
+    B, H = 2, 2
+    w = W.Workload("bwd", 1, torch.bfloat16, B=B, H=H, T=T, dk=dk, dv=dv, seed=7 * T + dk + dv,
+                   qk_scale=1 / np.sqrt(dk), gate="softplus", gate_shift=-2.0)
+    inp = W.prefill_inputs(w, device="cuda", init_state_std=0.1)
+    g = torch.Generator(device="cuda").manual_seed(T + 3)
+    dO = torch.randn(B, H, T, dv, generator=g, device="cuda").to(torch.bfloat16)
+    dST = torch.randn(B, H, dv, dk, generator=g, device="cuda") * 0.1
+    S0 = inp["state0"] if with_state else None
+    dS = dST if with_state else None
+    dq, dk_, dv_, dg, dS0 = la.prefill_backward(inp["q"], inp["k"], inp["v"], dO, mode=1, gate=inp["gate"],
+                                                state0=S0, dstate=dS, need_dstate0=with_state)
+    la.check_status()
+    f = lambda t: None if t is None else f64(t)
+    rq, rk, rv, rg, rS0 = ob.prefill_backward(1, f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["gate"]),
+                                              f(dO), f(S0), f(dS))
+    tol = TOL[torch.bfloat16]
+    for name, x, r in (("dq", dq, rq), ("dk", dk_, rk), ("dv", dv_, rv), ("dgate", dg, rg)):
+        e = slice_rel_err(f64(x), r)
+        assert e < tol, f"{name}: {e:.3e}"
+    if with_state:
+        e = slice_rel_err(f64(dS0), rS0)
+        assert e < tol, f"dS0: {e:.3e}"
