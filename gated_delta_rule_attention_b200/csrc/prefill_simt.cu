@@ -30,10 +30,16 @@
 //   O = (Q o G) S^T + A E,   S <- S Diag(G_L) + E^T (K o exp(lam_L - lam)).
 //
 // One CTA (256 threads) per (batch, head) -- or per (sequence, head) of packed
-// variable-length sequences -- walks the chunks in order; all tiles are fp32
-// in shared memory with one float of row padding so that row-strided reads are
-// bank-conflict free.
+// variable-length sequences -- walks the chunks in order; all tiles are fp32 in shared
+// memory.  The chunk's products (Q K^T, K K^T, W S^T, Q S^T, A X and the state update)
+// run on the tensor cores as warp-level mma (tf32 m16n8k8, each operand split into a tf32
+// part and its remainder: three products per tile, fp32 accuracy), in 16 x 32 tiles dealt
+// round-robin to the eight warps; row pitches are 4 (mod 32) floats so that the fragment
+// loads are conflict free.  Mode 3's A and Lm keep a per-term exponential inside the dot
+// product and stay on the CUDA cores (there the pitch is d + 1, conflict free for its
+// row-strided reads); the forward substitution is a CUDA-core recurrence in every mode.
 #include "la_internal.cuh"
+#include "bwd_util.cuh"
 
 #include <cfloat>
 
@@ -44,10 +50,11 @@ constexpr int kSimtThreads = 256;
 
 template <int MODE, int DK, int DV, int C>
 struct SimtSmem {
-    static constexpr int kS = DV * (DK + 1);
-    static constexpr int kQ = C * (DK + 1);
-    static constexpr int kV = C * (DV + 1);
-    static constexpr int kA = C * (C + 1);
+    static constexpr int SK = DK + (MODE == 3 ? 1 : 4), SV = DV + 4, SA = C + 4;   // row pitches
+    static constexpr int kS = DV * SK;
+    static constexpr int kQ = C * SK;
+    static constexpr int kV = C * SV;
+    static constexpr int kA = C * SA;
     static constexpr int kLamC = (MODE == 3) ? kQ : 0;   // per-channel log-gate prefix
     static constexpr int kFloats = kS + 3 * kQ + kV + 2 * kA + 4 * C + DK + kLamC;
     static constexpr size_t kBytes = sizeof(float) * kFloats;
@@ -77,8 +84,16 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
     float *zs = dec + C;             // [DK]
     float *lamC = zs + DK;           // [C][DK+1]  mode 3
 
-    constexpr int SK = DK + 1, SV = DV + 1, SA = C + 1;
-    const int tid = threadIdx.x;
+    constexpr int SK = L::SK, SV = L::SV, SA = L::SA;
+    const int tid = threadIdx.x, lane = tid & 31;
+    // the warp's 16 x 32 tiles of an M x N product (four 8-column n-tiles), round-robin
+    auto for_tiles = [&](int M, int N, auto f) {
+        const int per = N / 32, ntile = (M / 16) * per;
+        for (int mt = tid >> 5; mt < ntile; mt += kSimtThreads / 32) f(16 * (mt / per), 32 * (mt % per));
+    };
+    // fragment element r of n-tile nt at (m0, n0): row, column
+    auto frow = [&](int m0, int r) { return m0 + (lane >> 2) + 8 * (r >> 1); };
+    auto fcol = [&](int n0, int nt, int r) { return n0 + 8 * nt + 2 * (lane & 3) + (r & 1); };
     // The state slot is blockIdx.x: (batch, head) for dense tensors, (sequence, head) for
     // packed ones.  row0 is the first token row of the CTA in the [rows][d] view of
     // q, k, v and o, n its token count.
@@ -113,16 +128,20 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
     for (int t0 = 0; t0 < n; t0 += C) {
         const int Lc = min(C, n - t0);
         // ---- load the chunk (phi applied in mode 0) and the gates
-        for (int p = tid; p < Lc * DK; p += kSimtThreads) {
+        for (int p = tid; p < C * DK; p += kSimtThreads) {   // rows past the chunk's end: zero
             const int i = p / DK, j = p % DK;
-            float qv = to_f32(qh[(size_t)(t0 + i) * DK + j]);
-            float kv = to_f32(kh[(size_t)(t0 + i) * DK + j]);
-            if (MODE == 0) { qv = feature_phi(qv); kv = feature_phi(kv); }
+            float qv = 0.f, kv = 0.f;
+            if (i < Lc) {
+                qv = to_f32(qh[(size_t)(t0 + i) * DK + j]);
+                kv = to_f32(kh[(size_t)(t0 + i) * DK + j]);
+                if (MODE == 0) { qv = feature_phi(qv); kv = feature_phi(kv); }
+            }
             Qs[i * SK + j] = qv;
             Ks[i * SK + j] = kv;
+            if (kDelta) Ws[i * SK + j] = 0.f;
         }
-        for (int p = tid; p < Lc * DV; p += kSimtThreads)
-            Vs[(p / DV) * SV + p % DV] = to_f32(vh[(size_t)(t0 + p / DV) * DV + p % DV]);
+        for (int p = tid; p < C * DV; p += kSimtThreads)
+            Vs[(p / DV) * SV + p % DV] = p / DV < Lc ? to_f32(vh[(size_t)(t0 + p / DV) * DV + p % DV]) : 0.f;
         if (tid < Lc) {
             lam[tid] = (MODE != 0 && MODE != 3 && gh) ? logf(fmaxf(gh[(t0 + tid) * gt], FLT_MIN)) : 0.f;
             bet[tid] = kDelta ? bh_beta[t0 + tid] : 0.f;
@@ -143,24 +162,43 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
         if (tid < Lc) dec[tid] = expf(lam[Lc - 1] - lam[tid]);
 
         // ---- intra-chunk scores A (and the delta-rule matrix Lm)
-        for (int p = tid; p < C * C; p += kSimtThreads) {
-            const int i = p / C, j = p % C;
-            float aij = 0.f, lij = 0.f;
-            if (i < Lc && j <= i) {
-                float qk = 0.f, kk = 0.f;
+        if constexpr (MODE == 3) {   // a decay per channel inside the dot products
+            for (int p = tid; p < C * C; p += kSimtThreads) {
+                const int i = p / C, j = p % C;
+                float aij = 0.f, lij = 0.f;
+                if (i < Lc && j <= i) {
+                    float qk = 0.f, kk = 0.f;
 #pragma unroll 8
-                for (int c = 0; c < DK; ++c) {
-                    const float kj = (MODE == 3) ? Ks[j * SK + c] * expf(lamC[i * SK + c] - lamC[j * SK + c])
-                                                 : Ks[j * SK + c];
-                    qk = fmaf(Qs[i * SK + c], kj, qk);
-                    if (kDelta) kk = fmaf(Ks[i * SK + c], kj, kk);
+                    for (int c = 0; c < DK; ++c) {
+                        const float kj = Ks[j * SK + c] * expf(lamC[i * SK + c] - lamC[j * SK + c]);
+                        qk = fmaf(Qs[i * SK + c], kj, qk);
+                        kk = fmaf(Ks[i * SK + c], kj, kk);
+                    }
+                    aij = qk;
+                    if (j < i) lij = bet[i] * kk;
                 }
-                const float d = (MODE == 0 || MODE == 3) ? 1.f : expf(lam[i] - lam[j]);
-                aij = qk * d;
-                if (kDelta && j < i) lij = bet[i] * d * kk;
+                A[i * SA + j] = aij;
+                Lm[i * SA + j] = lij;
             }
-            A[i * SA + j] = aij;
-            if (kDelta) Lm[i * SA + j] = lij;
+        } else {
+            for_tiles(C, C, [&](int m0, int n0) {
+                float qk[4][4] = {}, kk[4][4] = {};
+                warp_mma<4, DK, true>(qk, m0, n0, [&](int i, int c) { return Qs[i * SK + c]; },
+                                      [&](int c, int j) { return Ks[j * SK + c]; });
+                if (kDelta)
+                    warp_mma<4, DK, true>(kk, m0, n0, [&](int i, int c) { return Ks[i * SK + c]; },
+                                          [&](int c, int j) { return Ks[j * SK + c]; });
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int i = frow(m0, r), j = fcol(n0, nt, r);
+                        const bool in = i < Lc && j <= i;
+                        const float d = (MODE == 0 || !in) ? 1.f : expf(lam[i] - lam[j]);
+                        A[i * SA + j] = in ? qk[nt][r] * d : 0.f;
+                        if (kDelta) Lm[i * SA + j] = (in && j < i) ? bet[i] * d * kk[nt][r] : 0.f;
+                    }
+            });
         }
         __syncthreads();
 
@@ -191,14 +229,19 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
                 }
                 __syncthreads();
             }
-            // E = U - W S^T, in place over U
-            for (int p = tid; p < Lc * DV; p += kSimtThreads) {
-                const int t = p / DV, i = p % DV;
-                float acc = Vs[t * SV + i];
-#pragma unroll 8
-                for (int c = 0; c < DK; ++c) acc = fmaf(-Ws[t * SK + c], S[i * SK + c], acc);
-                Vs[t * SV + i] = acc;
-            }
+            // E = U - W S^T, in place over U (rows past the chunk's end stay zero)
+            for_tiles(C, DV, [&](int m0, int n0) {
+                float ws[4][4] = {};
+                warp_mma<4, DK, true>(ws, m0, n0, [&](int t, int c) { return Ws[t * SK + c]; },
+                                      [&](int c, int i) { return S[i * SK + c]; });
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int t = frow(m0, r), i = fcol(n0, nt, r);
+                        Vs[t * SV + i] = t < Lc ? Vs[t * SV + i] - ws[nt][r] : 0.f;
+                    }
+            });
         }
         __syncthreads();
         if (MODE == 3) {
@@ -213,31 +256,43 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
         }
 
         // ---- output: O = diag(g) Q S^T + A X   (mode 0: / den)
-        for (int p = tid; p < Lc * DV; p += kSimtThreads) {
-            const int t = p / DV, i = p % DV;
-            float inter = 0.f;
-#pragma unroll 8
-            for (int c = 0; c < DK; ++c) inter = fmaf(Qs[t * SK + c], S[i * SK + c], inter);
-            float intra = 0.f;
-            for (int j = 0; j <= t; ++j) intra = fmaf(A[t * SA + j], Vs[j * SV + i], intra);
-            float out;
-            if (MODE == 0) out = (inter + intra) / den[t];
-            else if (MODE == 3) out = inter + intra;
-            else out = fmaf(expf(lam[t]), inter, intra);
-            oh[(size_t)(t0 + t) * DV + i] = from_f32<IO>(out);
-        }
+        for_tiles(C, DV, [&](int m0, int n0) {
+            float inter[4][4] = {}, intra[4][4] = {};
+            warp_mma<4, DK, true>(inter, m0, n0, [&](int t, int c) { return Qs[t * SK + c]; },
+                                  [&](int c, int i) { return S[i * SK + c]; });
+            warp_mma<4, C, true>(intra, m0, n0, [&](int t, int j) { return A[t * SA + j]; },
+                                 [&](int j, int i) { return Vs[j * SV + i]; });
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int t = frow(m0, r), i = fcol(n0, nt, r);
+                    if (t >= Lc) continue;
+                    float out;
+                    if (MODE == 0) out = (inter[nt][r] + intra[nt][r]) / den[t];
+                    else if (MODE == 3) out = inter[nt][r] + intra[nt][r];
+                    else out = fmaf(expf(lam[t]), inter[nt][r], intra[nt][r]);
+                    oh[(size_t)(t0 + t) * DV + i] = from_f32<IO>(out);
+                }
+        });
         __syncthreads();
 
         // ---- state update: S <- g_L S + sum_j exp(lam_L - lam_j) x_j k_j^T
         const float gL = (MODE == 0 || MODE == 3) ? 1.f : expf(lam[Lc - 1]);
-        for (int p = tid; p < DV * DK; p += kSimtThreads) {
-            const int i = p / DK, c = p % DK;
-            float acc = 0.f;
-            for (int j = 0; j < Lc; ++j)
-                acc = fmaf((MODE == 3 ? 1.f : dec[j]) * Vs[j * SV + i], Ks[j * SK + c], acc);
-            const float g = (MODE == 3) ? expf(lamC[(Lc - 1) * SK + c]) : gL;
-            S[i * SK + c] = fmaf(g, S[i * SK + c], acc);
-        }
+        for_tiles(DV, DK, [&](int m0, int n0) {
+            float acc[4][4] = {};
+            warp_mma<4, C, true>(acc, m0, n0,
+                                 [&](int i, int j) { return j < Lc ? (MODE == 3 ? 1.f : dec[j]) * Vs[j * SV + i] : 0.f; },
+                                 [&](int j, int c) { return Ks[j * SK + c]; });
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int i = frow(m0, r), c = fcol(n0, nt, r);
+                    const float g = (MODE == 3) ? expf(lamC[(Lc - 1) * SK + c]) : gL;
+                    S[i * SK + c] = fmaf(g, S[i * SK + c], acc[nt][r]);
+                }
+        });
         if (MODE == 0) {
             for (int c = tid; c < DK; c += kSimtThreads) {
                 float acc = 0.f;
