@@ -122,6 +122,13 @@ __device__ __forceinline__ void frag_b(uint32_t (&b)[2], const __nv_bfloat16 *X,
     if (!TRANS) ldsm_x2(b, X + (n0 + (l & 7)) * pitch + k0 + 8 * (l >> 3));
     else ldsm_x2_t(b, X + (k0 + l) * pitch + n0);
 }
+// frag_a<false> on a 128B-swizzled tile of 64-element rows (chunk j of row r at chunk
+// j ^ (r & 7), no padding): the A fragment (rows m0..m0+15, k0..k0+15).
+__device__ __forceinline__ void frag_a_sw64(uint32_t (&a)[4], const __nv_bfloat16 *X, int m0, int k0) {
+    const int l = threadIdx.x & 31;
+    const int r = m0 + (l & 15), j = (k0 >> 3) + (l >> 4);
+    ldsm_x4(a, X + r * 64 + 8 * (j ^ (r & 7)));
+}
 // frag_b on an unpadded tile of rows of `w` elements (w >= 64) whose 16-byte chunks are
 // XOR-swizzled by the row: chunk j of row r sits at chunk j ^ (r & 7).  Eight consecutive
 // rows at one logical chunk then fall in eight different bank groups.

@@ -104,6 +104,12 @@ cudaError_t launch_prefill_gdn_conv(const PrefillArgs &a, const ConvSpec &cs, vo
                                     size_t workspace_bytes);
 // Workspace with which it runs its two-pass variant (per-chunk factors formed in parallel).
 size_t prefill_gdn_workspace_bytes(int BH, int T);
+// KDA (mode 3) on the same chain kernel, two-pass only: whether a call of BH head rows
+// qualifies, the workspace it needs (its per-chunk records), and its launcher (which also
+// needs a 16-byte aligned gate tensor).
+bool prefill_kda2_selected(int mode, int BH, bool packed);
+size_t prefill_kda2_workspace_bytes(int BH, int T);
+cudaError_t launch_prefill_kda2(const PrefillArgs &a, void *workspace, size_t workspace_bytes);
 cudaError_t launch_short_conv(const ConvArgs &a);
 // Workspace of la_prefill_backward_delta (0 for other modes).
 size_t delta_backward_workspace_bytes(int mode, int B, int H, int T, int d_k, int d_v);

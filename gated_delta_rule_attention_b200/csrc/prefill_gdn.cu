@@ -124,30 +124,47 @@ static_assert(kSmall % 16 == 0, "gate rows are read as float4");
 constexpr uint32_t kBytes = kSmall + sizeof(Small);
 static_assert(kBytes <= 227 * 1024, "shared memory per CTA");
 
-// Shared-memory layouts of the two variants.  The two-pass variant reads A, T diag(b) and
-// T diag(b g) from pass 1: the stage carries the two T tiles after V (each 128-row A
-// operand of W and U starts 8 KB before its tile, on the stage's own data), and the Lm, Tm
-// and Zs buffers of the inverse are not needed.
-template <bool TWO>
+// Shared-memory layouts of the variants (kSingle, kTwoGdn, kTwoKda).  The two-pass variant
+// reads A, T diag(b) and T diag(b g) from pass 1: the stage carries the two T tiles after V
+// (each 128-row A operand of W and U starts 8 KB before its tile, on the stage's own data),
+// and the Lm, Tm and Zs buffers of the inverse are not needed.  The KDA variant's stage is
+// [V | T diag(b) | K o 2^(lam_L - lam) | Gam_L]: Q o Gam and W go from pass 1's record
+// straight into tensor memory, so no Q or K tile is staged.
+constexpr int kSingle = 0, kTwoGdn = 1, kTwoKda = 2;
+template <int VAR>
 struct GLay;
 template <>
-struct GLay<false> {
+struct GLay<kSingle> {
     static constexpr uint32_t kStage = ::la::kStage, kA0 = ::la::kA0, kA1 = ::la::kA1, kTbg = ::la::kTbg,
                               kTb = ::la::kTb, kLm = ::la::kLm, kTm = ::la::kTm, kZs = ::la::kZs,
                               kS = ::la::kS, kE = ::la::kE, kEp = ::la::kEp, kSmall = ::la::kSmall,
                               kBytes = ::la::kBytes;
+    static constexpr uint32_t kVOff = 32768, kTbOff = 0, kTbgOff = 0, kKlOff = 8192, kKlHalf = 16384, kGlOff = 0;
 };
 template <>
-struct GLay<true> {
+struct GLay<kTwoGdn> {
     static constexpr uint32_t kStage = 57344;   // [Q0 | K0 | Q1 | K1 | V | T diag(b) | T diag(b g)]
-    static constexpr uint32_t kTbOff = 40960, kTbgOff = 49152;
+    static constexpr uint32_t kVOff = 32768, kTbOff = 40960, kTbgOff = 49152, kKlOff = 8192, kKlHalf = 16384,
+                              kGlOff = 0;
     static constexpr uint32_t kA0 = kStages * kStage, kA1 = kA0 + 8192;
     static constexpr uint32_t kTbg = 0, kTb = 0, kLm = 0, kTm = 0, kZs = 0;   // (not used)
     static constexpr uint32_t kS = kA1 + 8192, kE = kS + 16384, kEp = kE + 8192, kSmall = kEp + 8192;
     static constexpr uint32_t kBytes = kSmall + sizeof(Small);
 };
-static_assert(GLay<true>::kS % 1024 == 0 && GLay<true>::kA0 % 1024 == 0, "1024-byte aligned tiles");
-static_assert(GLay<true>::kBytes <= 227 * 1024, "shared memory per CTA");
+template <>
+struct GLay<kTwoKda> {
+    static constexpr uint32_t kStage = 33792;   // [V | T diag(b) | K o 2^(lam_L - lam) (two halves) | Gam_L]
+    static constexpr uint32_t kVOff = 0, kTbOff = 8192, kTbgOff = 0, kKlOff = 16384, kKlHalf = 8192,
+                              kGlOff = 32768;
+    static constexpr uint32_t kA0 = kStages * kStage, kA1 = kA0 + 8192;
+    static constexpr uint32_t kTbg = 0, kTb = 0, kLm = 0, kTm = 0, kZs = 0;   // (not used)
+    static constexpr uint32_t kS = kA1 + 8192, kE = kS + 16384, kEp = kE + 8192, kSmall = kEp + 8192;
+    static constexpr uint32_t kBytes = kSmall + sizeof(Small);
+};
+static_assert(GLay<kTwoGdn>::kS % 1024 == 0 && GLay<kTwoGdn>::kA0 % 1024 == 0, "1024-byte aligned tiles");
+static_assert(GLay<kTwoKda>::kS % 1024 == 0 && GLay<kTwoKda>::kA0 % 1024 == 0 && GLay<kTwoKda>::kStage % 1024 == 0,
+              "1024-byte aligned tiles");
+static_assert(GLay<kTwoGdn>::kBytes <= 227 * 1024 && GLay<kTwoKda>::kBytes <= 227 * 1024, "shared memory per CTA");
 
 struct GdnParams {
     CUtensorMap tq, tk, tv;     // [BH][T][128] bf16, 64 x 64 boxes, 128B swizzle
@@ -574,9 +591,273 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
     if constexpr (CONV) tma_store_wait_all<0>();
 }
 
-template <bool TWO>
+// ---------------------------------------------------------------------------------------
+// Kimi Delta Attention (mode 3: Diag(a_t) with one decay per channel c of d_k, section
+// "The delta rule and Gated DeltaNet"), two-pass variant.  With the in-chunk log2 prefix
+// lam_tc per channel, Gam_tc = 2^lam_tc and L the chunk's last token, the chunked form is
+//   A_tj = sum_c q_tc k_jc 2^(lam_tc - lam_jc) (j <= t),
+//   Lm_tj = b_t sum_c k_tc k_jc 2^(lam_tc - lam_jc) (j < t),   T = (I + Lm)^-1,
+//   W = T diag(b) (K o Gam),   U = T diag(b) V,   E = U - W S^T,
+//   O = (Q o Gam) S^T + A E,   S^T <- Diag(Gam_L) S^T + (K o 2^(lam_L - lam))^T E,
+// so the chain of pass 2 is the gated-delta one with the decays moved into the operands.
+// Pass 1 writes per chunk a record of bf16 128B-swizzled images (rows of 128 bytes):
+constexpr uint32_t kKrA = 0;         // A                       64 x 64
+constexpr uint32_t kKrTb = 8192;     // T diag(b)               64 x 64
+constexpr uint32_t kKrQg = 16384;    // Q o Gam                 64 x 128 (two 64-column images)
+constexpr uint32_t kKrW = 32768;     // W                       64 x 128
+constexpr uint32_t kKrKl = 49152;    // K o 2^(lam_L - lam)     64 x 128
+constexpr uint32_t kKrGl = 65536;    // Gam_L                   128 fp32
+constexpr uint32_t kKdaRec = 66048;
+// Inside the Gram products A and Lm the pair decay is split between the two operands around
+// a reference token r: q_t 2^(lam_t - lam_r) times k_j 2^(lam_r - lam_j).  Off the diagonal
+// 16-token blocks r is the last token of j's block and both factors are <= 1 (exact up to
+// rounding: a factor that underflows belongs to a product below 2^-126); on a diagonal block
+// r is its first token and the key factor can grow over up to 15 tokens of decay, so there
+// the log2 gates are bounded below at kGramLog2Floor (a >= 0.0055), which keeps every factor
+// below 2^113.  Only pair weights across such a gate, already below 0.0055, move; every
+// state-facing factor (Gam, 2^(lam_L - lam), Gam_L) takes the gates exactly.
+constexpr float kGramLog2Floor = -7.5f;
+constexpr int kKP = kD + 8;                               // bf16 pitch of the Q, K, K-hat, K o Gam rows
+constexpr int kLP = kD + 8;                               // fp32 pitch of the gate / prefix rows
+constexpr uint32_t kKT = kC * kKP * 2;                    // 17408 B
+static_assert(kKT == kC * kTStride * 4, "Lm / Tm take the places of the Q / K rows");
+constexpr uint32_t kkQ = 0;                               // Q rows; then Lm
+constexpr uint32_t kkK = kkQ + kKT;                       // K rows; then Tm; then the W images
+constexpr uint32_t kkL = kkK + kKT;                       // gates -> bounded prefix; then A, T diag(b) images
+constexpr uint32_t kkH = kkL + kC * kLP * 4;              // K-hat: k_j 2^(lam_r - lam_j), r its block's first token
+constexpr uint32_t kkG = kkH + kKT;                       // K o Gam (the B operand of W)
+constexpr uint32_t kkZ = kkG + kKT;                       // Zs of the inverse (4 x 272 floats)
+constexpr uint32_t kkB = kkZ + 4 * 272 * 4;               // beta [64]
+constexpr uint32_t kkS = kkB + kC * 4;                    // sums over tokens 0-31 (exact, bounded), 32-63 (exact)
+constexpr uint32_t kkC = kkS + 3 * kD * 4;                // 2^(lam_{16J+15} - lam_{16J}) of blocks J = 0..2
+constexpr uint32_t kkBytes = kkC + 3 * kD * 4;
+static_assert(2 * (kkBytes + 1024) <= 228 * 1024, "two CTAs per SM");
+
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t w, float f0, float f1) {
+    const float2 v = unpack_bf16x2(w);
+    return pack_bf16x2(v.x * f0, v.y * f1);
+}
+// byte offset of element (t, c) in a pair of 64-column 128B-swizzled images
+__device__ __forceinline__ uint32_t img2_off(int t, int c) {
+    return (uint32_t)(c >> 6) * 8192u + sw128_off(t, (c & 63) >> 3) + (uint32_t)(c & 7) * 2u;
+}
+
+// Two CTAs per SM over all (head row, chunk) pairs, one chunk at a time; the next chunk's
+// rows are prefetched into L2 while the current one is processed.
+__global__ void __launch_bounds__(kFacT, 2)
+kda_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                         const float *__restrict__ gate, const float *__restrict__ beta, int T, int nch,
+                         int total, uint8_t *__restrict__ rec) {
+    extern __shared__ __align__(1024) uint8_t ksm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    __nv_bfloat16 *Qs = reinterpret_cast<__nv_bfloat16 *>(ksm + kkQ);
+    __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(ksm + kkK);
+    __nv_bfloat16 *Kh = reinterpret_cast<__nv_bfloat16 *>(ksm + kkH);
+    __nv_bfloat16 *Kg = reinterpret_cast<__nv_bfloat16 *>(ksm + kkG);
+    float *Lh = reinterpret_cast<float *>(ksm + kkL);
+    float *Lm = reinterpret_cast<float *>(ksm + kkQ), *Tm = reinterpret_cast<float *>(ksm + kkK);
+    float *Zs = reinterpret_cast<float *>(ksm + kkZ), *bet = reinterpret_cast<float *>(ksm + kkB);
+    float *sums = reinterpret_cast<float *>(ksm + kkS), *cJ = reinterpret_cast<float *>(ksm + kkC);
+    uint8_t *imA = ksm + kkL, *imW = ksm + kkK;
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const int c0 = item % nch;
+        const size_t row0 = (size_t)(item / nch) * T + (size_t)c0 * kC;
+        const int L = min(kC, T - c0 * kC);
+        uint8_t *rc = rec + (size_t)item * kKdaRec;
+        // ---- rows [0, L) of q, k and the gates (rows past L: zero, gate 1), beta
+        for (int p = tid; p < 2 * kC * 16; p += kFacT) {
+            const int which = p >> 10, r = (p >> 4) & 63, x = p & 15;
+            __nv_bfloat16 *dst = (which ? Ks : Qs) + r * kKP + 8 * x;
+            if (r < L) cp_async16(dst, (which ? k : q) + (row0 + r) * kD + 8 * x);
+            else *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (gate)
+            for (int p = tid; p < kC * 32; p += kFacT) {
+                const int r = p >> 5, x = p & 31;
+                if (r < L) cp_async16(Lh + r * kLP + 4 * x, gate + (row0 + r) * kD + 4 * x);
+            }
+        cp_async_commit();
+        if (tid < kC) bet[tid] = tid < L ? beta[row0 + tid] : 0.f;
+        cp_async_wait_all();
+        __syncthreads();
+        // ---- per-channel prefixes: thread (c, half) scans 32 tokens; Q o Gam and
+        // K o 2^(lam_L - lam) leave for the record, K o Gam stays for W
+        {
+            const int ch = tid & 127, hf = tid >> 7;
+            float lx[32];
+            float sx = 0.f, sb = 0.f;
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                const int t = 32 * hf + m;
+                const float g = (gate && t < L) ? lg2(fmaxf(Lh[t * kLP + ch], FLT_MIN)) : 0.f;
+                sx += g;
+                sb += fmaxf(g, kGramLog2Floor);
+                lx[m] = sx;
+                Lh[t * kLP + ch] = sb;
+            }
+            sums[hf * 2 * kD + ch] = sx;   // [0]: exact 0-31, [2]: exact 32-63
+            if (hf == 0) sums[kD + ch] = sb;
+            __syncthreads();
+            const float off = hf ? sums[ch] : 0.f, lL = sums[ch] + sums[2 * kD + ch];
+            if (hf) {
+                const float offb = sums[kD + ch];
+#pragma unroll
+                for (int m = 0; m < 32; ++m) Lh[(32 + m) * kLP + ch] += offb;
+            }
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                const int t = 32 * hf + m;
+                const float lt = lx[m] + off;
+                const float gm = ex2(lt), kv = __bfloat162float(Ks[t * kKP + ch]);
+                Kg[t * kKP + ch] = __float2bfloat16_rn(kv * gm);
+                const uint32_t o = img2_off(t, ch);
+                *reinterpret_cast<__nv_bfloat16 *>(rc + kKrQg + o) =
+                    __float2bfloat16_rn(__bfloat162float(Qs[t * kKP + ch]) * gm);
+                *reinterpret_cast<__nv_bfloat16 *>(rc + kKrKl + o) = __float2bfloat16_rn(kv * ex2(lL - lt));
+            }
+            if (hf == 0) reinterpret_cast<float *>(rc + kKrGl)[ch] = ex2(lL);
+        }
+        __syncthreads();   // the bounded prefix is complete
+        // ---- K-hat (reference: the first token of the key's block) and the block factors
+        {
+            const int ch = tid & 127, hf = tid >> 7;
+#pragma unroll 8
+            for (int m = 0; m < 32; ++m) {
+                const int j = 32 * hf + m, r = j & ~15;
+                const float f = ex2(Lh[r * kLP + ch] - Lh[j * kLP + ch]);
+                Kh[j * kKP + ch] = __float2bfloat16_rn(__bfloat162float(Ks[j * kKP + ch]) * f);
+            }
+            if (hf == 0)
+#pragma unroll
+                for (int J = 0; J < 3; ++J)
+                    cJ[J * kD + ch] = ex2(Lh[(16 * J + 15) * kLP + ch] - Lh[16 * J * kLP + ch]);
+        }
+        __syncthreads();
+        // ---- Gram products: warp w rows 16 (w & 3) (block I), columns 32 (w >> 2) (blocks J)
+        const int I = warp & 3, Jp = warp >> 2, m0 = 16 * I;
+        const int g = lane >> 2, t4 = lane & 3;
+        float gq[2][2][4] = {}, gk[2][2][4] = {};
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            const int J = 2 * Jp + jj;
+            if (J > I) continue;   // (warp-uniform)
+            const int r = (J == I) ? 16 * I : 16 * J + 15;
+#pragma unroll 2
+            for (int kk = 0; kk < kD; kk += 16) {
+                uint32_t aq[4], ak[4];
+                frag_a<false>(aq, Qs, kKP, m0, kk);
+                frag_a<false>(ak, Ks, kKP, m0, kk);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {   // a[i]: row m0 + g + 8 (i & 1), channels cc, cc + 1
+                    const int t = m0 + g + 8 * (i & 1), cc = kk + 2 * t4 + 8 * (i >> 1);
+                    const float2 lt = *reinterpret_cast<const float2 *>(Lh + t * kLP + cc);
+                    const float2 lr = *reinterpret_cast<const float2 *>(Lh + r * kLP + cc);
+                    const float f0 = ex2(lt.x - lr.x), f1 = ex2(lt.y - lr.y);
+                    aq[i] = scale_bf16x2(aq[i], f0, f1);
+                    ak[i] = scale_bf16x2(ak[i], f0, f1);
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    uint32_t b[2];
+                    frag_b<false>(b, Kh, kKP, kk, 16 * J + 8 * nt);
+                    if (J < I)   // to the end of block J: b[i] holds channels kk + 2 t4 + 8 i, + 1
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const float2 f = *reinterpret_cast<const float2 *>(cJ + J * kD + kk + 2 * t4 + 8 * i);
+                            b[i] = scale_bf16x2(b[i], f.x, f.y);
+                        }
+                    mma_16x8x16_bf16(gq[jj][nt], aq, b[0], b[1]);
+                    mma_16x8x16_bf16(gk[jj][nt], ak, b[0], b[1]);
+                }
+            }
+        }
+        // the next chunk's rows into L2
+        if (item + (int)gridDim.x < total) {
+            const int nx = item + gridDim.x, nc = nx % nch;
+            const size_t nrow = (size_t)(nx / nch) * T + (size_t)nc * kC;
+            const int nL = min(kC, T - nc * kC);
+            for (int p = tid; p < 8 * kC; p += kFacT) {   // per row: 2 lines of q, 2 of k, 4 of gates
+                const int r = p >> 3, z = p & 7;
+                if (r >= nL) continue;
+                if (z < 2) prefetch_l2(q + (nrow + r) * kD + 64 * z);
+                else if (z < 4) prefetch_l2(k + (nrow + r) * kD + 64 * (z - 2));
+                else if (gate) prefetch_l2(gate + (nrow + r) * kD + 32 * (z - 4));
+            }
+        }
+        __syncthreads();   // Q, K, K-hat and the prefix are read: Lm over Q, the images over the prefix
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int t = m0 + g + 8 * h, j = 32 * Jp + 16 * jj + 8 * nt + 2 * t4;
+                    float a2[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int je = j + e;
+                        Lm[t * kTStride + je] = je < t ? bet[t] * gk[jj][nt][2 * h + e] : 0.f;
+                        a2[e] = je <= t ? gq[jj][nt][2 * h + e] : 0.f;
+                    }
+                    *reinterpret_cast<uint32_t *>(imA + sw128_off(t, j >> 3) + (j & 7) * 2) = pack_bf16x2(a2[0], a2[1]);
+                }
+        __syncthreads();
+        invert_unit_lower_rec<1, kFacT>(Lm, Tm, Zs, tid);
+        __syncthreads();
+        {   // T diag(b) (lower triangle)
+            const int t = tid >> 2, j0 = 16 * (tid & 3);
+            float v1[16];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+                const int j = j0 + jj;
+                v1[jj] = (j <= t) ? Tm[t * kTStride + j] * bet[j] : 0.f;
+            }
+            st_row_bf16x16(smem_u32(imA + 8192), t, j0 >> 3, v1);
+        }
+        __syncthreads();
+        {   // W = T diag(b) (K o Gam): warp w rows 16 (w & 3), channels 64 (w >> 2); images over Tm
+            const int n0 = 64 * Jp;
+            const __nv_bfloat16 *Tb = reinterpret_cast<const __nv_bfloat16 *>(imA + 8192);
+            float acc[8][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < kC; kk += 16) {
+                uint32_t a[4];
+                frag_a_sw64(a, Tb, m0, kk);
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) {
+                    uint32_t b[2];
+                    frag_b<true>(b, Kg, kKP, kk, n0 + 8 * nt);
+                    mma_16x8x16_bf16(acc[nt], a, b[0], b[1]);
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int t = m0 + g + 8 * h, cc = n0 + 8 * nt + 2 * t4;
+                    *reinterpret_cast<uint32_t *>(imW + img2_off(t, cc)) = pack_bf16x2(acc[nt][2 * h], acc[nt][2 * h + 1]);
+                }
+        }
+        __syncthreads();
+        {   // the record's A, T diag(b) and W images
+            uint4 *d = reinterpret_cast<uint4 *>(rc);
+            const uint4 *sa = reinterpret_cast<const uint4 *>(imA), *sw = reinterpret_cast<const uint4 *>(imW);
+            for (int p = tid; p < 1024; p += kFacT) d[p] = sa[p];
+            for (int p = tid; p < 1024; p += kFacT) d[kKrW / 16 + p] = sw[p];
+        }
+        __syncthreads();   // the tiles are free for the next chunk's rows
+    }
+}
+
+template <int VAR>
 __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_constant__ GdnParams p) {
-    using GL = GLay<TWO>;
+    constexpr bool TWO = VAR != kSingle, KDA = VAR == kTwoKda;
+    using GL = GLay<VAR>;
+    // pass 1's record of chunk c of this head row (two-pass variants)
+    auto record = [&](int bh_, int c_) -> const uint8_t * {
+        return reinterpret_cast<const uint8_t *>(p.img) +
+               ((size_t)bh_ * p.nchunks + c_) * (size_t)(KDA ? kKdaRec : 2 * kImgHalves);
+    };
     // the variant's layout (shadows the single-pass constants)
     constexpr uint32_t kStage = GL::kStage, kA0 = GL::kA0, kA1 = GL::kA1, kTbg = GL::kTbg, kTb = GL::kTb,
                        kLm = GL::kLm, kTm = GL::kTm, kZs = GL::kZs, kS = GL::kS, kE = GL::kE, kEp = GL::kEp,
@@ -640,8 +921,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            tma_prefetch_desc(&p.tq);
-            tma_prefetch_desc(&p.tk);
+            if (!KDA) {
+                tma_prefetch_desc(&p.tq);
+                tma_prefetch_desc(&p.tk);
+            }
             tma_prefetch_desc(&p.tv);
             const int vx = 64 * (vs >> 1);
             int issued[kStages] = {0, 0, 0};
@@ -650,25 +933,38 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                 if (u >= 1 && !mbar_wait(&sm->empty[s], (u - 1) & 1, abort, p.err)) break;
                 const uint32_t st = sb + s * kStage;
                 const int t = tb + kC * c;
-                mbar_arrive_expect_tx(&sm->full[s], kStage);
-                tma_load_3d(st + 0, &p.tq, 0, t, bh, &sm->full[s]);
-                tma_load_3d(st + 8192, &p.tk, 0, t, bh, &sm->full[s]);
-                tma_load_3d(st + 16384, &p.tq, 64, t, bh, &sm->full[s]);
-                tma_load_3d(st + 24576, &p.tk, 64, t, bh, &sm->full[s]);
-                tma_load_3d(st + 32768, &p.tv, vx, t, bh, &sm->full[s]);
-                if constexpr (TWO) {   // T diag(b), T diag(b g) of chunk c (pass 1)
-                    const __nv_bfloat16 *rec = p.img + ((size_t)bh * p.nchunks + c) * kImgHalves;
-                    bulk_load(st + GL::kTbOff, rec + 4096, 8192, &sm->full[s]);
-                    bulk_load(st + GL::kTbgOff, rec + 8192, 8192, &sm->full[s]);
+                if constexpr (KDA) {   // V, then T diag(b), K o 2^(lam_L - lam) and Gam_L (pass 1)
+                    const uint8_t *rec = record(bh, c);
+                    mbar_arrive_expect_tx(&sm->full[s], 8192 + 8192 + 16384 + 512);
+                    tma_load_3d(st + GL::kVOff, &p.tv, vx, t, bh, &sm->full[s]);
+                    bulk_load(st + GL::kTbOff, rec + kKrTb, 8192, &sm->full[s]);
+                    bulk_load(st + GL::kKlOff, rec + kKrKl, 16384, &sm->full[s]);
+                    bulk_load(st + GL::kGlOff, rec + kKrGl, 512, &sm->full[s]);
+                } else {
+                    mbar_arrive_expect_tx(&sm->full[s], kStage);
+                    tma_load_3d(st + 0, &p.tq, 0, t, bh, &sm->full[s]);
+                    tma_load_3d(st + 8192, &p.tk, 0, t, bh, &sm->full[s]);
+                    tma_load_3d(st + 16384, &p.tq, 64, t, bh, &sm->full[s]);
+                    tma_load_3d(st + 24576, &p.tk, 64, t, bh, &sm->full[s]);
+                    tma_load_3d(st + 32768, &p.tv, vx, t, bh, &sm->full[s]);
+                    if constexpr (TWO) {   // T diag(b), T diag(b g) of chunk c (pass 1)
+                        const uint8_t *rec = record(bh, c);
+                        bulk_load(st + GL::kTbOff, rec + 8192, 8192, &sm->full[s]);
+                        bulk_load(st + GL::kTbgOff, rec + 16384, 8192, &sm->full[s]);
+                    }
                 }
                 issued[s] = u + 1;
                 // the chunk three ahead of this one into L2 (the slices of a head share it)
                 const int tp = t + kStages * kC;
                 if (tp < te) {
-                    tma_prefetch_l2_3d(&p.tq, 0, tp, bh);
-                    tma_prefetch_l2_3d(&p.tq, 64, tp, bh);
-                    tma_prefetch_l2_3d(&p.tk, 0, tp, bh);
-                    tma_prefetch_l2_3d(&p.tk, 64, tp, bh);
+                    if constexpr (KDA) {
+                        bulk_prefetch_l2(record(bh, c + kStages), kKdaRec);
+                    } else {
+                        tma_prefetch_l2_3d(&p.tq, 0, tp, bh);
+                        tma_prefetch_l2_3d(&p.tq, 64, tp, bh);
+                        tma_prefetch_l2_3d(&p.tk, 0, tp, bh);
+                        tma_prefetch_l2_3d(&p.tk, 64, tp, bh);
+                    }
                     tma_prefetch_l2_3d(&p.tv, vx, tp, bh);
                 }
             }
@@ -733,13 +1029,21 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
             for (int c = 0; c < nch; ++c) {
                 const int s = c % kStages, b = c & 1;
                 bool ok = true;
+                // KDA: this thread's half row of Q o Gam (rows 0-63) or W (rows 64-127), read
+                // from the record before the waits below
+                uint4 pre[8];
+                if constexpr (KDA) {
+                    const uint8_t *src = record(bh, c) + (pq < 2 ? kKrQg : kKrW) + 8192 * ph;
+                    const int t = prow & 63;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) pre[ch] = *reinterpret_cast<const uint4 *>(src + sw128_off(t, ch));
+                }
                 if (lead) {
                     // A(c) into its parity buffer once A E(c - 2) has read it
                     ok = c < 2 || mbar_wait(&sm->ae_done[b], ((c >> 1) - 1) & 1, abort, p.err);
                     if (ok) {
                         mbar_arrive_expect_tx(&sm->a_full[b], 8192);
-                        bulk_load(sb + (b ? kA1 : kA0), p.img + ((size_t)bh * p.nchunks + c) * kImgHalves, 8192,
-                                  &sm->a_full[b]);
+                        bulk_load(sb + (b ? kA1 : kA0), record(bh, c), 8192, &sm->a_full[b]);
                         issued[b] = (c >> 1) + 1;
                     }
                     // W = T diag(b g) K, U = T diag(b) V (rows 64-127) once the stage is in, W(c - 1)
@@ -750,10 +1054,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                     if (ok) {
                         tc_fence_after();
                         const uint32_t st = sb + s * kStage;
-                        mma_chain<4, true, false>(tm + kColW, dk(st + GL::kTbgOff - 8192), dmn(st + 8192, 16384),
-                                                  id_w, false);
+                        if (!KDA)   // (KDA: W comes from pass 1)
+                            mma_chain<4, true, false>(tm + kColW, dk(st + GL::kTbgOff - 8192),
+                                                      dmn(st + 8192, 16384), id_w, false);
                         mma_chain<4, true, false>(tm + (b ? kColU2 : kColU), dk(st + GL::kTbOff - 8192),
-                                                  dmn(st + 32768, 8192), id_u, false);
+                                                  dmn(st + GL::kVOff, 8192), id_u, false);
                         mma_commit(&sm->wu_done);
                         // W(c) formed, and P(c - 2) done with this parity's A operand buffer
                         ok = mbar_wait(&sm->wu_done, c & 1, abort, p.err) &&
@@ -765,7 +1070,17 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                 if (named_sync_any(kBarPrep, kPrepT, !ok || *abort != 0)) break;
                 tc_fence_after();
                 const uint32_t dst = tl + kColQW + 64 * b;
-                if (pq < 2) {   // rows 0-63: diag(g) Q, column half ph
+                if constexpr (KDA) {   // rows 0-63: Q o Gam, rows 64-127: W, column half ph
+                    uint32_t w[32];
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        w[4 * ch + 0] = pre[ch].x;
+                        w[4 * ch + 1] = pre[ch].y;
+                        w[4 * ch + 2] = pre[ch].z;
+                        w[4 * ch + 3] = pre[ch].w;
+                    }
+                    tmem_st32(dst + 32 * ph, w);
+                } else if (pq < 2) {   // rows 0-63: diag(g) Q, column half ph
                     const int t = prow;
                     const float gt = ex2(sm->gt[s].lam[t]);
                     const uint32_t st = sb + s * kStage;
@@ -1021,7 +1336,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
             const bool cur = c < nch;
             // the stage's gates were observed in qw_step(c); read before the barrier below,
             // which precedes the stage's release (dS(c) is issued after it)
-            const float gL = cur ? ex2(sm->gt[s].lam[kC - 1]) : 1.f;
+            // (KDA: the stage's per-row decay Gam_L of the chunk, d_k row `row`)
+            float gL = 1.f;
+            if (cur) {
+                if constexpr (KDA) {
+                    mbar_wait(&sm->full[s], (c / kStages) & 1, abort, p.err);
+                    gL = reinterpret_cast<const float *>(smem_raw + s * kStage + GL::kGlOff)[row];
+                } else {
+                    gL = ex2(sm->gt[s].lam[kC - 1]);
+                }
+            }
             // P(c) done, and A E(c - 1) (which frees the E tiles and completes the outputs of
             // chunk c - 1; the tensor core ran it before P(c)): one meeting of the chain
             {
@@ -1058,8 +1382,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                         tc_fence_after();
                         const uint32_t st = sb + s * kStage;
                         // dS^T = K^T E'   (E' = diag(dec) E)
-                        mma_chain<4, false, false>(tm + kColDS, dmn(st + 8192, 16384), dmn(sb + kEp, 8192),
-                                                   id_ds, false);
+                        // (KDA: K o 2^(lam_L - lam) in place of K, and E' = E)
+                        mma_chain<4, false, false>(tm + kColDS, dmn(st + GL::kKlOff, GL::kKlHalf),
+                                                   dmn(sb + kEp, 8192), id_ds, false);
                         mma_commit(&sm->ds_done);
                         mma_commit(&sm->empty[s]);
                         // rows 0-63 of P += A E  (the 64 rows after the A tile multiply into
@@ -1159,12 +1484,23 @@ size_t prefill_gdn_workspace_bytes(int BH, int T) {
     return sizeof(__nv_bfloat16) * (size_t)kImgHalves * (size_t)BH * (size_t)((T + kC - 1) / kC);
 }
 
+bool prefill_kda2_selected(int mode, int BH, bool packed) {
+    // The same head-row range as the gated delta rule; KDA runs here only in the two-pass
+    // variant (with a workspace of prefill_kda2_workspace_bytes), else on the segmented kernels.
+    return mode == LA_MODE_KDA && !packed && BH * kNS >= 64 && BH * kNS <= 148;
+}
+
+size_t prefill_kda2_workspace_bytes(int BH, int T) {
+    return (size_t)kKdaRec * (size_t)BH * (size_t)((T + kC - 1) / kC);
+}
+
 // With a workspace of at least prefill_gdn_workspace_bytes (dense calls), pass 1 forms every
 // chunk's A, T diag(b), T diag(b g) at once and the chain kernel reads them (two-pass);
 // otherwise the single pass forms them itself.
 namespace {
 cudaError_t launch_gdn(const PrefillArgs &a, void *workspace, size_t workspace_bytes, const ConvSpec *cs) {
     const int BH = a.cu ? a.H : a.B * a.H;
+    const bool kda = a.mode == LA_MODE_KDA;   // (two-pass only; its gates go to pass 1)
     GdnParams p;
     memset(&p, 0, sizeof(p));
     const uint64_t row_pitch = kD * 2, head_pitch = (uint64_t)a.T * kD * 2;
@@ -1175,7 +1511,7 @@ cudaError_t launch_gdn(const PrefillArgs &a, void *workspace, size_t workspace_b
         !make_tmap_3d(&p.tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, a.T, BH, row_pitch,
                       head_pitch, 64, kC, true))
         return cudaErrorInvalidValue;
-    p.gate = a.gate;
+    p.gate = kda ? nullptr : a.gate;
     p.beta = a.beta;
     p.o = static_cast<__nv_bfloat16 *>(a.o);
     p.s_in = a.init_state ? a.state : nullptr;
@@ -1187,8 +1523,10 @@ cudaError_t launch_gdn(const PrefillArgs &a, void *workspace, size_t workspace_b
     p.err = device_error_word();
     const int units = a.cu ? a.nseq * a.H : BH;
     const bool two = !a.cu && workspace && (reinterpret_cast<uintptr_t>(workspace) & 15u) == 0 &&
-                     workspace_bytes >= prefill_gdn_workspace_bytes(BH, a.T);
+                     workspace_bytes >= (kda ? prefill_kda2_workspace_bytes(BH, a.T)
+                                             : prefill_gdn_workspace_bytes(BH, a.T));
     if (cs && !two) return cudaErrorInvalidValue;   // the fused convolution lives in pass 1
+    if (kda && (!two || cs || (reinterpret_cast<uintptr_t>(a.gate) & 15u) != 0)) return cudaErrorInvalidValue;
     cudaError_t e;
     if (two) {
         const int nch = (a.T + kC - 1) / kC;
@@ -1211,8 +1549,10 @@ cudaError_t launch_gdn(const PrefillArgs &a, void *workspace, size_t workspace_b
             fc.fv = cs->fv;
         }
         auto fac = cs ? gdn_chunk_factors_kernel<true> : gdn_chunk_factors_kernel<false>;
-        const uint32_t fbytes = cs ? FacLay<true>::kBytes : FacLay<false>::kBytes;
-        e = cudaFuncSetAttribute(fac, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fbytes);
+        const uint32_t fbytes = kda ? kkBytes : cs ? FacLay<true>::kBytes : FacLay<false>::kBytes;
+        e = kda ? cudaFuncSetAttribute(kda_chunk_factors_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)fbytes)
+                : cudaFuncSetAttribute(fac, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fbytes);
         if (e != cudaSuccess) return e;
         int dev = 0, sms = 148;
         if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -1221,15 +1561,20 @@ cudaError_t launch_gdn(const PrefillArgs &a, void *workspace, size_t workspace_b
         const int total = BH * nch;
         const int grid = total < 2 * sms ? total : 2 * sms;
         timer_begin(a.stream);
-        fac<<<(unsigned)grid, kFacT, fbytes, a.stream>>>(
-            static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k), a.gate, a.beta, a.T,
-            nch, total, static_cast<__nv_bfloat16 *>(workspace), fc);
+        if (kda)
+            kda_chunk_factors_kernel<<<(unsigned)grid, kFacT, fbytes, a.stream>>>(
+                static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k), a.gate, a.beta,
+                a.T, nch, total, static_cast<uint8_t *>(workspace));
+        else
+            fac<<<(unsigned)grid, kFacT, fbytes, a.stream>>>(
+                static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k), a.gate, a.beta,
+                a.T, nch, total, static_cast<__nv_bfloat16 *>(workspace), fc);
         timer_end(a.stream);
         note_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    auto kern = two ? gdn_prefill_kernel<true> : gdn_prefill_kernel<false>;
-    const uint32_t bytes = two ? GLay<true>::kBytes : GLay<false>::kBytes;
+    auto kern = kda ? gdn_prefill_kernel<kTwoKda> : two ? gdn_prefill_kernel<kTwoGdn> : gdn_prefill_kernel<kSingle>;
+    const uint32_t bytes = kda ? GLay<kTwoKda>::kBytes : two ? GLay<kTwoGdn>::kBytes : GLay<kSingle>::kBytes;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     timer_begin(a.stream);
@@ -1241,6 +1586,12 @@ cudaError_t launch_gdn(const PrefillArgs &a, void *workspace, size_t workspace_b
 }  // namespace
 
 cudaError_t launch_prefill_gdn(const PrefillArgs &a, void *workspace, size_t workspace_bytes) {
+    return launch_gdn(a, workspace, workspace_bytes, nullptr);
+}
+
+// KDA (mode 3) in the two-pass variant: the caller checked prefill_kda2_selected, the
+// workspace size and a 16-byte aligned gate tensor.
+cudaError_t launch_prefill_kda2(const PrefillArgs &a, void *workspace, size_t workspace_bytes) {
     return launch_gdn(a, workspace, workspace_bytes, nullptr);
 }
 

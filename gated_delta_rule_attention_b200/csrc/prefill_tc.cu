@@ -2133,6 +2133,7 @@ bool prefill_tc_supports(int mode, int dtype, int dk, int dv, int chunk) {
 size_t prefill_tc_workspace_bytes(int mode, int B, int H, int T, bool minimal) {
     const int BH = B * H;
     if (prefill_gdn_selected(mode, BH, false)) return minimal ? 0 : prefill_gdn_workspace_bytes(BH, T);
+    if (!minimal && prefill_kda2_selected(mode, BH, false)) return prefill_kda2_workspace_bytes(BH, T);
     Plan pl = plan_for(mode, BH, T);
     if (minimal && mode >= 2) pl.sub = 1;   // the smallest segmented plan
     return sizeof(float) * workspace_floats(mode, BH, pl);
@@ -2161,6 +2162,12 @@ cudaError_t run_packed(const PrefillArgs &a, const TcParams &base) {
 cudaError_t launch_prefill_tc(const PrefillArgs &a, void *workspace, size_t workspace_bytes) {
     const int BH = a.B * a.H;
     if (prefill_gdn_selected(a.mode, BH, a.cu != nullptr)) return launch_prefill_gdn(a, workspace, workspace_bytes);
+    // KDA with room for the per-chunk records (and gates the bulk copies can read): the
+    // two-pass chain kernel; otherwise the segmented kernels with what the workspace allows
+    if (prefill_kda2_selected(a.mode, BH, a.cu != nullptr) && workspace &&
+        workspace_bytes >= prefill_kda2_workspace_bytes(BH, a.T) &&
+        (reinterpret_cast<uintptr_t>(workspace) & 15u) == 0 && (reinterpret_cast<uintptr_t>(a.gate) & 15u) == 0)
+        return launch_prefill_kda2(a, workspace, workspace_bytes);
     const Plan pl = plan_for(a.mode, BH, a.T, workspace ? workspace_bytes : 0);
     TcParams p;
     memset(&p, 0, sizeof(p));

@@ -98,6 +98,10 @@ def test_workspace_size_query(lib):
     assert lib.la_prefill_workspace_size(2, 1, 2, 16, 32768, 128, 128, 0) == 32 * 512 * 24576
     assert lib.la_prefill_workspace_size(2, 1, 1, 37, 32768, 128, 128, 0) == 37 * 512 * 24576
     assert lib.la_prefill_workspace_size(2, 1, 1, 38, 32768, 128, 128, 0) > 0
+    # KDA with 16-37 head rows: the two-pass chain kernel's per-chunk records (A, T diag(b)
+    # 8 KB each, Q o Gam, W, K o 2^(lam_L - lam) 16 KB each, Gam_L 512 B)
+    assert lib.la_prefill_workspace_size(3, 1, 2, 16, 32768, 128, 128, 0) == 32 * 512 * 66048
+    assert lib.la_prefill_workspace_size(3, 1, 1, 16, 65, 128, 128, 0) == 16 * 2 * 66048
     assert lib.la_prefill_workspace_size(1, 1, 8, 16, 8192, 128, 128, 0) == 0   # 128 heads
     assert lib.la_prefill_workspace_size(0, 0, 1, 2, 256, 64, 64, 0) == 0       # fp32 path
     assert lib.la_prefill_workspace_size(3, 1, 1, 1, 64, 128, 128, 0) == 0
