@@ -608,38 +608,42 @@ constexpr uint32_t kKrW = 32768;     // W                       64 x 128
 constexpr uint32_t kKrKl = 49152;    // K o 2^(lam_L - lam)     64 x 128
 constexpr uint32_t kKrGl = 65536;    // Gam_L                   128 fp32
 constexpr uint32_t kKdaRec = 66048;
-// Inside the Gram products A and Lm the pair decay is split between the two operands around
-// a reference token r: q_t 2^(lam_t - lam_r) times k_j 2^(lam_r - lam_j).  Off the diagonal
-// 16-token blocks r is the last token of j's block and both factors are <= 1 (exact up to
-// rounding: a factor that underflows belongs to a product below 2^-126); on a diagonal block
-// r is its first token and the key factor can grow over up to 15 tokens of decay, so there
-// the log2 gates are bounded below at kGramLog2Floor (a >= 0.0055), which keeps every factor
-// below 2^113.  Only pair weights across such a gate, already below 0.0055, move; every
-// state-facing factor (Gam, 2^(lam_L - lam), Gam_L) takes the gates exactly.
+// The Gram products A and Lm take the pair decay of 16-token blocks I (rows) and J <= I
+// (columns) in three factors, with s_I the first token of block I and e_J the last of J:
+//   2^(lam_t - lam_j) = 2^(lam_t - lam_{s_I})  [rows: F_t, in [2^-113, 1]]
+//                     x 2^(lam_{s_I} - lam_{e_J}) [per channel, off the diagonal: D_IJ <= 1]
+//                     x 2^(lam_{e_J} - lam_{s_J}) [per channel, off the diagonal: c_J <= 1]
+//                     x 2^(lam_{s_J} - lam_j)  [columns: Fi_j, in [1, 2^113]].
+// On a diagonal block (I = J) the middle factors are 1.  Off it, q_t F_t D_IJ <= 1 and
+// k_j Fi_j c_J = k_j 2^(lam_{e_J} - lam_j) <= 1, so a factor that underflows belongs to a
+// pair weight below 2^-126.  F and Fi span at most 15 tokens of decay, which stays inside
+// the exponent range because the Gram products bound each log2 gate below at
+// kGramLog2Floor (a >= 0.0055): only pair weights across such a gate, already below 0.0055,
+// move.  Every state-facing factor (Gam, 2^(lam_L - lam), Gam_L) takes the gates exactly.
 constexpr float kGramLog2Floor = -7.5f;
 constexpr int kKP = kD + 8;                               // bf16 pitch of the Q, K, K-hat, K o Gam rows
-constexpr int kLP = kD + 8;                               // fp32 pitch of the gate / prefix rows
 constexpr uint32_t kKT = kC * kKP * 2;                    // 17408 B
 static_assert(kKT == kC * kTStride * 4, "Lm / Tm take the places of the Q / K rows");
-constexpr uint32_t kkQ = 0;                               // Q rows; then Lm
-constexpr uint32_t kkK = kkQ + kKT;                       // K rows; then Tm; then the W images
-constexpr uint32_t kkL = kkK + kKT;                       // gates -> bounded prefix; then A, T diag(b) images
-constexpr uint32_t kkH = kkL + kC * kLP * 4;              // K-hat: k_j 2^(lam_r - lam_j), r its block's first token
+constexpr uint32_t kkQ = 0;                               // Q rows, scaled by F in place; then Lm
+constexpr uint32_t kkK = kkQ + kKT;                       // K rows, scaled by F in place; then Tm; then W
+constexpr uint32_t kkR = kkK + kKT;                       // raw gates [64][128]; then the Q o Gam, K o 2^(lam_L - lam) images
+constexpr uint32_t kkH = kkR + kC * kD * 4;               // K-hat = K o Fi; then the A, T diag(b) images
 constexpr uint32_t kkG = kkH + kKT;                       // K o Gam (the B operand of W)
-constexpr uint32_t kkZ = kkG + kKT;                       // Zs of the inverse (4 x 272 floats)
+constexpr uint32_t kkZ = kkG + kKT;                       // Zs of the inverse; first the block-edge prefixes
 constexpr uint32_t kkB = kkZ + 4 * 272 * 4;               // beta [64]
-constexpr uint32_t kkS = kkB + kC * 4;                    // sums over tokens 0-31 (exact, bounded), 32-63 (exact)
-constexpr uint32_t kkC = kkS + 3 * kD * 4;                // 2^(lam_{16J+15} - lam_{16J}) of blocks J = 0..2
-constexpr uint32_t kkBytes = kkC + 3 * kD * 4;
+constexpr uint32_t kkF = kkB + kC * 4;                    // D_IJ [6][64], c_J [3][64] bf16 pairs; first the half sums
+constexpr uint32_t kkBytes = kkF + 9 * 64 * 4;
 static_assert(2 * (kkBytes + 1024) <= 228 * 1024, "two CTAs per SM");
+static_assert(8 * kD * 4 <= 4 * 272 * 4 && 3 * kD * 4 <= 9 * 64 * 4, "scratch overlays");
 
-__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t w, float f0, float f1) {
-    const float2 v = unpack_bf16x2(w);
-    return pack_bf16x2(v.x * f0, v.y * f1);
-}
 // byte offset of element (t, c) in a pair of 64-column 128B-swizzled images
 __device__ __forceinline__ uint32_t img2_off(int t, int c) {
     return (uint32_t)(c >> 6) * 8192u + sw128_off(t, (c & 63) >> 3) + (uint32_t)(c & 7) * 2u;
+}
+__device__ __forceinline__ uint32_t hmul_bf16x2(uint32_t a, uint32_t b) {
+    const __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&a),
+                                     *reinterpret_cast<const __nv_bfloat162 *>(&b));
+    return *reinterpret_cast<const uint32_t *>(&r);
 }
 
 // Two CTAs per SM over all (head row, chunk) pairs, one chunk at a time; the next chunk's
@@ -654,17 +658,19 @@ kda_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
     __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(ksm + kkK);
     __nv_bfloat16 *Kh = reinterpret_cast<__nv_bfloat16 *>(ksm + kkH);
     __nv_bfloat16 *Kg = reinterpret_cast<__nv_bfloat16 *>(ksm + kkG);
-    float *Lh = reinterpret_cast<float *>(ksm + kkL);
+    float *Gr = reinterpret_cast<float *>(ksm + kkR);
     float *Lm = reinterpret_cast<float *>(ksm + kkQ), *Tm = reinterpret_cast<float *>(ksm + kkK);
     float *Zs = reinterpret_cast<float *>(ksm + kkZ), *bet = reinterpret_cast<float *>(ksm + kkB);
-    float *sums = reinterpret_cast<float *>(ksm + kkS), *cJ = reinterpret_cast<float *>(ksm + kkC);
-    uint8_t *imA = ksm + kkL, *imW = ksm + kkK;
+    float *edge = Zs;                                           // [s_0..s_3, e_0..e_3][128]
+    float *sums = reinterpret_cast<float *>(ksm + kkF);         // [3][128]
+    const uint32_t *Dp = reinterpret_cast<const uint32_t *>(ksm + kkF);   // [9][64] bf16 pairs
+    uint8_t *imR = ksm + kkR, *imA = ksm + kkH, *imW = ksm + kkK;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
         const int c0 = item % nch;
         const size_t row0 = (size_t)(item / nch) * T + (size_t)c0 * kC;
         const int L = min(kC, T - c0 * kC);
         uint8_t *rc = rec + (size_t)item * kKdaRec;
-        // ---- rows [0, L) of q, k and the gates (rows past L: zero, gate 1), beta
+        // ---- rows [0, L) of q, k and the gates (rows past L: zero; their gates are not read), beta
         for (int p = tid; p < 2 * kC * 16; p += kFacT) {
             const int which = p >> 10, r = (p >> 4) & 63, x = p & 15;
             __nv_bfloat16 *dst = (which ? Ks : Qs) + r * kKP + 8 * x;
@@ -672,65 +678,84 @@ kda_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
             else *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
         }
         if (gate)
-            for (int p = tid; p < kC * 32; p += kFacT) {
-                const int r = p >> 5, x = p & 31;
-                if (r < L) cp_async16(Lh + r * kLP + 4 * x, gate + (row0 + r) * kD + 4 * x);
-            }
+            for (int p = tid; p < L * 32; p += kFacT) cp_async16(Gr + 4 * p, gate + row0 * kD + 4 * p);
         cp_async_commit();
         if (tid < kC) bet[tid] = tid < L ? beta[row0 + tid] : 0.f;
         cp_async_wait_all();
         __syncthreads();
-        // ---- per-channel prefixes: thread (c, half) scans 32 tokens; Q o Gam and
-        // K o 2^(lam_L - lam) leave for the record, K o Gam stays for W
+        // ---- thread (c, half): the prefixes of channel c over tokens 32 half .. + 31, exact
+        // (lx) and with the Gram products' bound (lb)
+        const int ch = tid & 127, hf = tid >> 7;
+        float lx[32], lb[32];
         {
-            const int ch = tid & 127, hf = tid >> 7;
-            float lx[32];
             float sx = 0.f, sb = 0.f;
 #pragma unroll
             for (int m = 0; m < 32; ++m) {
                 const int t = 32 * hf + m;
-                const float g = (gate && t < L) ? lg2(fmaxf(Lh[t * kLP + ch], FLT_MIN)) : 0.f;
+                const float g = (gate && t < L) ? lg2(fmaxf(Gr[t * kD + ch], FLT_MIN)) : 0.f;
                 sx += g;
                 sb += fmaxf(g, kGramLog2Floor);
                 lx[m] = sx;
-                Lh[t * kLP + ch] = sb;
+                lb[m] = sb;
             }
-            sums[hf * 2 * kD + ch] = sx;   // [0]: exact 0-31, [2]: exact 32-63
-            if (hf == 0) sums[kD + ch] = sb;
-            __syncthreads();
-            const float off = hf ? sums[ch] : 0.f, lL = sums[ch] + sums[2 * kD + ch];
-            if (hf) {
-                const float offb = sums[kD + ch];
-#pragma unroll
-                for (int m = 0; m < 32; ++m) Lh[(32 + m) * kLP + ch] += offb;
+            if (hf == 0) {
+                sums[ch] = sx;
+                sums[kD + ch] = sb;
+            } else {
+                sums[2 * kD + ch] = sx;
             }
-#pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                const int t = 32 * hf + m;
-                const float lt = lx[m] + off;
-                const float gm = ex2(lt), kv = __bfloat162float(Ks[t * kKP + ch]);
-                Kg[t * kKP + ch] = __float2bfloat16_rn(kv * gm);
-                const uint32_t o = img2_off(t, ch);
-                *reinterpret_cast<__nv_bfloat16 *>(rc + kKrQg + o) =
-                    __float2bfloat16_rn(__bfloat162float(Qs[t * kKP + ch]) * gm);
-                *reinterpret_cast<__nv_bfloat16 *>(rc + kKrKl + o) = __float2bfloat16_rn(kv * ex2(lL - lt));
-            }
-            if (hf == 0) reinterpret_cast<float *>(rc + kKrGl)[ch] = ex2(lL);
         }
-        __syncthreads();   // the bounded prefix is complete
-        // ---- K-hat (reference: the first token of the key's block) and the block factors
-        {
-            const int ch = tid & 127, hf = tid >> 7;
-#pragma unroll 8
-            for (int m = 0; m < 32; ++m) {
-                const int j = 32 * hf + m, r = j & ~15;
-                const float f = ex2(Lh[r * kLP + ch] - Lh[j * kLP + ch]);
-                Kh[j * kKP + ch] = __float2bfloat16_rn(__bfloat162float(Ks[j * kKP + ch]) * f);
-            }
-            if (hf == 0)
+        __syncthreads();   // the half sums are in; the raw gates are read
+        const float lL = sums[ch] + sums[2 * kD + ch];   // exact prefix at the chunk's last token
+        if (hf) {
+            const float ox = sums[ch], ob = sums[kD + ch];
 #pragma unroll
-                for (int J = 0; J < 3; ++J)
-                    cJ[J * kD + ch] = ex2(Lh[(16 * J + 15) * kLP + ch] - Lh[16 * J * kLP + ch]);
+            for (int m = 0; m < 32; ++m) {
+                lx[m] += ox;
+                lb[m] += ob;
+            }
+        }
+        if (hf == 0) reinterpret_cast<float *>(rc + kKrGl)[ch] = ex2(lL);
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {   // this half's blocks: bounded prefix at their first and last tokens
+            edge[(2 * hf + b) * kD + ch] = lb[16 * b];
+            edge[(4 + 2 * hf + b) * kD + ch] = lb[16 * b + 15];
+        }
+        // ---- per element: Q o Gam and K o 2^(lam_L - lam) (images, for the record), K o Gam
+        // (for W), and the Gram operands Q F, K F (in place) and K Fi
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {
+            const int t = 32 * hf + m;
+            const float qv = __bfloat162float(Qs[t * kKP + ch]), kv = __bfloat162float(Ks[t * kKP + ch]);
+            const float gm = ex2(lx[m]);
+            const float d = lb[m] - lb[16 * (m >> 4)];   // <= 0, >= 15 kGramLog2Floor
+            const float f = ex2(d), fi = ex2(-d);
+            const uint32_t o = img2_off(t, ch);
+            *reinterpret_cast<__nv_bfloat16 *>(imR + o) = __float2bfloat16_rn(qv * gm);
+            *reinterpret_cast<__nv_bfloat16 *>(imR + 16384 + o) = __float2bfloat16_rn(kv * ex2(lL - lx[m]));
+            Kg[t * kKP + ch] = __float2bfloat16_rn(kv * gm);
+            Qs[t * kKP + ch] = __float2bfloat16_rn(qv * f);
+            Ks[t * kKP + ch] = __float2bfloat16_rn(kv * f);
+            Kh[t * kKP + ch] = __float2bfloat16_rn(kv * fi);
+        }
+        __syncthreads();   // the block edges are in (and the half sums read)
+        if (tid < 64) {    // D_IJ = 2^(lam_{s_I} - lam_{e_J}) (I > J), c_J = 2^(lam_{e_J} - lam_{s_J}) (J < 3), channel pairs
+            const int c2 = 2 * tid;
+            auto pair = [&](float a0, float a1) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(ex2(a0), ex2(a1));
+                return *reinterpret_cast<const uint32_t *>(&h);
+            };
+            uint32_t *D = reinterpret_cast<uint32_t *>(ksm + kkF);
+#pragma unroll
+            for (int I = 1; I < 4; ++I)
+#pragma unroll
+                for (int J = 0; J < I; ++J)
+                    D[(I * (I - 1) / 2 + J) * 64 + tid] = pair(edge[I * kD + c2] - edge[(4 + J) * kD + c2],
+                                                               edge[I * kD + c2 + 1] - edge[(4 + J) * kD + c2 + 1]);
+#pragma unroll
+            for (int J = 0; J < 3; ++J)
+                D[(6 + J) * 64 + tid] = pair(edge[(4 + J) * kD + c2] - edge[J * kD + c2],
+                                             edge[(4 + J) * kD + c2 + 1] - edge[J * kD + c2 + 1]);
         }
         __syncthreads();
         // ---- Gram products: warp w rows 16 (w & 3) (block I), columns 32 (w >> 2) (blocks J)
@@ -741,31 +766,33 @@ kda_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
         for (int jj = 0; jj < 2; ++jj) {
             const int J = 2 * Jp + jj;
             if (J > I) continue;   // (warp-uniform)
-            const int r = (J == I) ? 16 * I : 16 * J + 15;
-#pragma unroll 2
+            const uint32_t *DI = Dp + (I * (I - 1) / 2 + J) * 64, *CJ = Dp + (6 + J) * 64;
+#pragma unroll 4
             for (int kk = 0; kk < kD; kk += 16) {
                 uint32_t aq[4], ak[4];
                 frag_a<false>(aq, Qs, kKP, m0, kk);
                 frag_a<false>(ak, Ks, kKP, m0, kk);
+                uint32_t dd[2] = {0u, 0u}, cc[2] = {0u, 0u};
+                if (J < I) {   // fragment registers i hold channel pairs kk/2 + t4 + 4 (i >> 1)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {   // a[i]: row m0 + g + 8 (i & 1), channels cc, cc + 1
-                    const int t = m0 + g + 8 * (i & 1), cc = kk + 2 * t4 + 8 * (i >> 1);
-                    const float2 lt = *reinterpret_cast<const float2 *>(Lh + t * kLP + cc);
-                    const float2 lr = *reinterpret_cast<const float2 *>(Lh + r * kLP + cc);
-                    const float f0 = ex2(lt.x - lr.x), f1 = ex2(lt.y - lr.y);
-                    aq[i] = scale_bf16x2(aq[i], f0, f1);
-                    ak[i] = scale_bf16x2(ak[i], f0, f1);
+                    for (int i = 0; i < 2; ++i) {
+                        dd[i] = DI[kk / 2 + t4 + 4 * i];
+                        cc[i] = CJ[kk / 2 + t4 + 4 * i];
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        aq[i] = hmul_bf16x2(aq[i], dd[i >> 1]);
+                        ak[i] = hmul_bf16x2(ak[i], dd[i >> 1]);
+                    }
                 }
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     uint32_t b[2];
                     frag_b<false>(b, Kh, kKP, kk, 16 * J + 8 * nt);
-                    if (J < I)   // to the end of block J: b[i] holds channels kk + 2 t4 + 8 i, + 1
-#pragma unroll
-                        for (int i = 0; i < 2; ++i) {
-                            const float2 f = *reinterpret_cast<const float2 *>(cJ + J * kD + kk + 2 * t4 + 8 * i);
-                            b[i] = scale_bf16x2(b[i], f.x, f.y);
-                        }
+                    if (J < I) {
+                        b[0] = hmul_bf16x2(b[0], cc[0]);
+                        b[1] = hmul_bf16x2(b[1], cc[1]);
+                    }
                     mma_16x8x16_bf16(gq[jj][nt], aq, b[0], b[1]);
                     mma_16x8x16_bf16(gk[jj][nt], ak, b[0], b[1]);
                 }
@@ -784,7 +811,7 @@ kda_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
                 else if (gate) prefetch_l2(gate + (nrow + r) * kD + 32 * (z - 4));
             }
         }
-        __syncthreads();   // Q, K, K-hat and the prefix are read: Lm over Q, the images over the prefix
+        __syncthreads();   // the operands are read: Lm over Q, the A image over K-hat
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
@@ -834,16 +861,23 @@ kda_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
             for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int t = m0 + g + 8 * h, cc = n0 + 8 * nt + 2 * t4;
-                    *reinterpret_cast<uint32_t *>(imW + img2_off(t, cc)) = pack_bf16x2(acc[nt][2 * h], acc[nt][2 * h + 1]);
+                    const int t = m0 + g + 8 * h, c = n0 + 8 * nt + 2 * t4;
+                    *reinterpret_cast<uint32_t *>(imW + img2_off(t, c)) = pack_bf16x2(acc[nt][2 * h], acc[nt][2 * h + 1]);
                 }
         }
         __syncthreads();
-        {   // the record's A, T diag(b) and W images
+        {   // the record: A and T diag(b), Q o Gam, W, K o 2^(lam_L - lam)
             uint4 *d = reinterpret_cast<uint4 *>(rc);
-            const uint4 *sa = reinterpret_cast<const uint4 *>(imA), *sw = reinterpret_cast<const uint4 *>(imW);
-            for (int p = tid; p < 1024; p += kFacT) d[p] = sa[p];
-            for (int p = tid; p < 1024; p += kFacT) d[kKrW / 16 + p] = sw[p];
+            const uint4 *sa = reinterpret_cast<const uint4 *>(imA), *sr = reinterpret_cast<const uint4 *>(imR),
+                        *sw = reinterpret_cast<const uint4 *>(imW);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int p = tid + kFacT * i;
+                d[kKrA / 16 + p] = sa[p];
+                d[kKrQg / 16 + p] = sr[p];
+                d[kKrW / 16 + p] = sw[p];
+                d[kKrKl / 16 + p] = sr[1024 + p];
+            }
         }
         __syncthreads();   // the tiles are free for the next chunk's rows
     }

@@ -79,14 +79,18 @@ CONFIGS = {
     "retnet_bf16_b8h16t8192": Workload("retnet_bf16_b8h16t8192", MODE_RETNET, torch.bfloat16, B=8,
                                        H=16, T=8192, dk=128, dv=128, seed=10,
                                        qk_scale=1 / math.sqrt(128), gate="retnet"),
-    # Profiling cases of the gated delta rule (counter captures need a few GB on the device
-    # at most): the B2 H16 recipe at a quarter of its length (200 MB of inputs, more than
+    # Profiling cases of the gated delta rule and KDA (counter captures need a few GB on the
+    # device at most): the B2 H16 recipe at a quarter of its length (200 MB of inputs, more than
     # L2), and 8 heads, which take the segmented kernels.
     "gdn_bf16_b2h16t8192": Workload("gdn_bf16_b2h16t8192", MODE_GATED_DELTA, torch.bfloat16, B=2,
                                     H=16, T=8192, dk=128, dv=128, seed=4, qk_l2norm=True,
                                     gate="softplus", beta=True),
     "gdn_bf16_b1h8t16384": Workload("gdn_bf16_b1h8t16384", MODE_GATED_DELTA, torch.bfloat16, B=1,
                                     H=8, T=16384, dk=128, dv=128, seed=4, qk_l2norm=True,
+                                    gate="softplus", beta=True),
+    # the KDA recipe at a quarter of its length (600 MB of inputs with the per-channel gates)
+    "kda_bf16_b2h16t8192": Workload("kda_bf16_b2h16t8192", MODE_KDA, torch.bfloat16, B=2, H=16,
+                                    T=8192, dk=128, dv=128, seed=6, qk_l2norm=True,
                                     gate="softplus", beta=True),
 }
 
