@@ -116,6 +116,7 @@ struct Small {
     uint64_t u_free2[2];  // two-pass variant: U buffer of each parity read by the chain
     uint64_t qw_ready[2]; // two-pass variant: [diag(g) Q; W] of each parity in tensor memory
     uint64_t p_done2[2];  // two-pass variant: P of each parity done (its A operand is free)
+    uint64_t p_issued;    // KDA variant: the chain has issued P of the next chunk
     uint32_t tmem_base;
     int abort;
 };
@@ -932,6 +933,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
         mbar_init(&sm->qw_ready[1], 1);
         mbar_init(&sm->p_done2[0], 1);
         mbar_init(&sm->p_done2[1], 1);
+        mbar_init(&sm->p_issued, 1);
         sm->abort = 0;
         fence_mbar_init();
     }
@@ -1083,8 +1085,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                     // W = T diag(b g) K, U = T diag(b) V (rows 64-127) once the stage is in, W(c - 1)
                     // was read (the group's own step below) and U(c - 2) was read by the chain
                     // (U has a buffer per chunk parity)
+                    // ... and (KDA: U alone, W comes from pass 1), so that it queues behind the
+                    // chain's P(c - 1) instead of in front of it (the tensor pipe runs in issue
+                    // order), once P(c - 1) has been issued: it then runs while the chain forms
+                    // E(c - 1).  (The gated delta rule issues W and U as early as it can: W(c)
+                    // has to be converted into the operand of P(c) in time.)
                     ok = ok && mbar_wait(&sm->full[s], (c / kStages) & 1, abort, p.err) &&
-                         (c < 2 || mbar_wait(&sm->u_free2[b], ((c >> 1) - 1) & 1, abort, p.err));
+                         (c < 2 || mbar_wait(&sm->u_free2[b], ((c >> 1) - 1) & 1, abort, p.err)) &&
+                         (!KDA || c < 1 || mbar_wait(&sm->p_issued, (c - 1) & 1, abort, p.err));
                     if (ok) {
                         tc_fence_after();
                         const uint32_t st = sb + s * kStage;
@@ -1312,6 +1320,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_prefill_kernel(const __grid_c
                             id_p, false);
             mma_commit(&sm->p_done);
             if (TWO) mma_commit(&sm->p_done2[c & 1]);
+            if (KDA) mbar_arrive(&sm->p_issued);
         };
         // two-pass: the prep warps wrote [diag(g) Q; W] of chunk c; the chain meets after the
         // elected thread saw it (which also orders the stage's gates before their reads)
