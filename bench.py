@@ -168,18 +168,20 @@ def source_file_shas():
 
 def ncu_traffic(workload: str):
     """The committed ncu launch summary of `workload` (kernels in launch order, each with
-    its DRAM bytes per launch and time share), or None when any source file that existed
-    when it was taken has changed since (a file added later cannot change those kernels:
-    every translation unit and header they were built from is among the recorded ones)."""
+    its DRAM bytes per launch and time share), or None when a source file it was taken on
+    has changed since.  An entry lists the files its kernels were built from (their
+    translation units, every header, the C ABI); an entry without its own list is checked
+    against every file recorded for the whole summary."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
         now = source_file_shas()
-        rec = t.get("sources")
+        entry = t["workloads"][workload]
+        rec = entry.get("sources") or t.get("sources")
         if not rec or any(now.get(fn) != sha for fn, sha in rec.items()):
             return None
-        return t["workloads"][workload]
+        return entry
     except Exception:
         return None
 

@@ -112,11 +112,15 @@ typedef enum {
  *   flags  0 or LA_FLAG_INIT_STATE.
  *   workspace, workspace_bytes
  *          optional device scratch owned by the caller (NULL / 0 allowed).  With at least
- *          la_prefill_workspace_size() bytes the tensor-core kernel splits each sequence
- *          into segments processed in parallel and chains their states exactly; with
- *          less it takes the fastest segment plan that fits, or runs each sequence in
- *          one pass (same result up to rounding, less parallelism when B*H is small).  Calls that share a workspace must not
- *          overlap on the device.
+ *          la_prefill_workspace_size() bytes the tensor-core kernels take their fastest
+ *          form: modes 2 and 3 with 16 to 37 head rows (B*H) first form every chunk's
+ *          state-independent factors into the workspace (mode 2: 24 KB per chunk and head
+ *          row; mode 3: 66 048 bytes, and the gate tensor 16-byte aligned), then carry the
+ *          state through the chunks; other calls split each sequence into segments
+ *          processed in parallel and chain their states exactly.  With less they take the
+ *          fastest plan that fits (mode 2 with 16 to 37 head rows: its single pass; other
+ *          calls: a smaller segment plan, or one pass per sequence), with the same result
+ *          up to rounding.  Calls that share a workspace must not overlap on the device.
  * T = 0 is allowed: nothing is read from q, k, v, o; the state is left as given (with
  * LA_FLAG_INIT_STATE) or zeroed.  q, k, v, o may then be NULL.
  * o must not overlap q, k, v or the state.

@@ -51,14 +51,21 @@ def test_decode_algorithmic_counts():
 
 
 def test_committed_traffic_is_keyed_to_sources():
-    """traffic.json records every kernel source's hash; bench.py uses it only while all of
-    them are unchanged (otherwise roofline.traffic is null)."""
+    """Each traffic.json entry records the hashes of the sources its kernels were built from
+    (their translation units, every header, the C ABI); bench.py uses an entry only while
+    all of them are unchanged (otherwise roofline.traffic is null)."""
     import json
     with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
         t = json.load(f)
-    assert t["sources"] and bench.DEFAULT_WORKLOAD in t["workloads"]
-    same = all(bench.source_file_shas().get(fn) == sha for fn, sha in t["sources"].items())
-    got = bench.ncu_traffic(bench.DEFAULT_WORKLOAD)
-    assert (got is not None) == same
-    if got is not None:
-        assert got["kernels"][-1]["dram_bytes_per_launch"] > 0
+    assert bench.DEFAULT_WORKLOAD in t["workloads"]
+    now = bench.source_file_shas()
+    for name, entry in t["workloads"].items():
+        rec = entry.get("sources") or t.get("sources")
+        assert rec, name
+        if "sources" in entry:   # its kernels' own files, every header and the C ABI
+            assert "abi.cu" in rec and all(fn in rec for fn in now if fn.endswith(".cuh")), name
+        same = all(now.get(fn) == sha for fn, sha in rec.items())
+        got = bench.ncu_traffic(name)
+        assert (got is not None) == same, name
+        if got is not None:
+            assert got["kernels"][-1]["dram_bytes_per_launch"] > 0
