@@ -630,12 +630,12 @@ constexpr uint32_t kkK = kkQ + kKT;                       // K rows, scaled by F
 constexpr uint32_t kkR = kkK + kKT;                       // raw gates [64][128]; then the Q o Gam, K o 2^(lam_L - lam) images
 constexpr uint32_t kkH = kkR + kC * kD * 4;               // K-hat = K o Fi; then the A, T diag(b) images
 constexpr uint32_t kkG = kkH + kKT;                       // K o Gam (the B operand of W)
-constexpr uint32_t kkZ = kkG + kKT;                       // Zs of the inverse; first the block-edge prefixes
-constexpr uint32_t kkB = kkZ + 4 * 272 * 4;               // beta [64]
-constexpr uint32_t kkF = kkB + kC * 4;                    // D_IJ [6][64], c_J [3][64] bf16 pairs; first the half sums
+constexpr uint32_t kkZ = kkG + kKT;                       // Zs of the inverse
+constexpr uint32_t kkS = kkZ + 4 * 272 * 4;               // per 16-token block and channel pair: sums, first steps
+constexpr uint32_t kkB = kkS + 4 * 64 * 16 + 4 * 64 * 8;  // beta [64]
+constexpr uint32_t kkF = kkB + kC * 4;                    // D_IJ [6][64], c_J [3][64] bf16 pairs
 constexpr uint32_t kkBytes = kkF + 9 * 64 * 4;
 static_assert(2 * (kkBytes + 1024) <= 228 * 1024, "two CTAs per SM");
-static_assert(8 * kD * 4 <= 4 * 272 * 4 && 3 * kD * 4 <= 9 * 64 * 4, "scratch overlays");
 
 // byte offset of element (t, c) in a pair of 64-column 128B-swizzled images
 __device__ __forceinline__ uint32_t img2_off(int t, int c) {
@@ -662,8 +662,8 @@ kda_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
     float *Gr = reinterpret_cast<float *>(ksm + kkR);
     float *Lm = reinterpret_cast<float *>(ksm + kkQ), *Tm = reinterpret_cast<float *>(ksm + kkK);
     float *Zs = reinterpret_cast<float *>(ksm + kkZ), *bet = reinterpret_cast<float *>(ksm + kkB);
-    float *edge = Zs;                                           // [s_0..s_3, e_0..e_3][128]
-    float *sums = reinterpret_cast<float *>(ksm + kkF);         // [3][128]
+    float4 *bsum = reinterpret_cast<float4 *>(ksm + kkS);      // [block][pair]: exact sums (2), bounded sums (2)
+    float2 *bfirst = reinterpret_cast<float2 *>(ksm + kkS + 4 * 64 * 16);   // [block][pair]: bounded first steps
     const uint32_t *Dp = reinterpret_cast<const uint32_t *>(ksm + kkF);   // [9][64] bf16 pairs
     uint8_t *imR = ksm + kkR, *imA = ksm + kkH, *imW = ksm + kkK;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
@@ -684,64 +684,63 @@ kda_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
         if (tid < kC) bet[tid] = tid < L ? beta[row0 + tid] : 0.f;
         cp_async_wait_all();
         __syncthreads();
-        // ---- thread (c, half): the prefixes of channel c over tokens 32 half .. + 31, exact
-        // (lx) and with the Gram products' bound (lb)
-        const int ch = tid & 127, hf = tid >> 7;
-        float lx[32], lb[32];
+        // ---- thread (channel pair cp, 16-token block J0): the prefixes of channels 2 cp, 2 cp + 1
+        // inside the block, exact (lx) and with the Gram products' bound (lb)
+        const int cp = tid & 63, J0 = tid >> 6, c2 = 2 * cp;
+        float lx[16][2], lb[16][2];
         {
-            float sx = 0.f, sb = 0.f;
+            float sx0 = 0.f, sx1 = 0.f, sb0 = 0.f, sb1 = 0.f, f0 = 0.f, f1 = 0.f;
 #pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                const int t = 32 * hf + m;
-                const float g = (gate && t < L) ? lg2(fmaxf(Gr[t * kD + ch], FLT_MIN)) : 0.f;
-                sx += g;
-                sb += fmaxf(g, kGramLog2Floor);
-                lx[m] = sx;
-                lb[m] = sb;
+            for (int m = 0; m < 16; ++m) {
+                const int t = 16 * J0 + m;
+                float g0 = 0.f, g1 = 0.f;
+                if (gate && t < L) {
+                    const float2 a = *reinterpret_cast<const float2 *>(Gr + t * kD + c2);
+                    g0 = lg2(fmaxf(a.x, FLT_MIN));
+                    g1 = lg2(fmaxf(a.y, FLT_MIN));
+                }
+                const float h0 = fmaxf(g0, kGramLog2Floor), h1 = fmaxf(g1, kGramLog2Floor);
+                if (m == 0) {
+                    f0 = h0;
+                    f1 = h1;
+                }
+                sx0 += g0;
+                sx1 += g1;
+                sb0 += h0;
+                sb1 += h1;
+                lx[m][0] = sx0;
+                lx[m][1] = sx1;
+                lb[m][0] = sb0;
+                lb[m][1] = sb1;
             }
-            if (hf == 0) {
-                sums[ch] = sx;
-                sums[kD + ch] = sb;
-            } else {
-                sums[2 * kD + ch] = sx;
+            bsum[J0 * 64 + cp] = make_float4(sx0, sx1, sb0, sb1);
+            bfirst[J0 * 64 + cp] = make_float2(f0, f1);
+        }
+        __syncthreads();   // the block sums are in; the raw gates are read
+        // exact prefix before the block and at the chunk's last token
+        float ox0 = 0.f, ox1 = 0.f, lL0 = 0.f, lL1 = 0.f;
+#pragma unroll
+        for (int J = 0; J < 4; ++J) {
+            const float4 v = bsum[J * 64 + cp];
+            if (J < J0) {
+                ox0 += v.x;
+                ox1 += v.y;
             }
+            lL0 += v.x;
+            lL1 += v.y;
         }
-        __syncthreads();   // the half sums are in; the raw gates are read
-        const float lL = sums[ch] + sums[2 * kD + ch];   // exact prefix at the chunk's last token
-        if (hf) {
-            const float ox = sums[ch], ob = sums[kD + ch];
+        if (J0 == 0) *reinterpret_cast<float2 *>(rc + kKrGl + 4 * c2) = make_float2(ex2(lL0), ex2(lL1));
+        if (tid < 64) {    // D_IJ = 2^(lam_{s_I} - lam_{e_J}) (I > J), c_J = 2^(lam_{e_J} - lam_{s_J}) (J < 3)
+            float tb[4][2], fb[4][2];
 #pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                lx[m] += ox;
-                lb[m] += ob;
+            for (int J = 0; J < 4; ++J) {
+                const float4 v = bsum[J * 64 + cp];
+                const float2 f = bfirst[J * 64 + cp];
+                tb[J][0] = v.z;
+                tb[J][1] = v.w;
+                fb[J][0] = f.x;
+                fb[J][1] = f.y;
             }
-        }
-        if (hf == 0) reinterpret_cast<float *>(rc + kKrGl)[ch] = ex2(lL);
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {   // this half's blocks: bounded prefix at their first and last tokens
-            edge[(2 * hf + b) * kD + ch] = lb[16 * b];
-            edge[(4 + 2 * hf + b) * kD + ch] = lb[16 * b + 15];
-        }
-        // ---- per element: Q o Gam and K o 2^(lam_L - lam) (images, for the record), K o Gam
-        // (for W), and the Gram operands Q F, K F (in place) and K Fi
-#pragma unroll
-        for (int m = 0; m < 32; ++m) {
-            const int t = 32 * hf + m;
-            const float qv = __bfloat162float(Qs[t * kKP + ch]), kv = __bfloat162float(Ks[t * kKP + ch]);
-            const float gm = ex2(lx[m]);
-            const float d = lb[m] - lb[16 * (m >> 4)];   // <= 0, >= 15 kGramLog2Floor
-            const float f = ex2(d), fi = ex2(-d);
-            const uint32_t o = img2_off(t, ch);
-            *reinterpret_cast<__nv_bfloat16 *>(imR + o) = __float2bfloat16_rn(qv * gm);
-            *reinterpret_cast<__nv_bfloat16 *>(imR + 16384 + o) = __float2bfloat16_rn(kv * ex2(lL - lx[m]));
-            Kg[t * kKP + ch] = __float2bfloat16_rn(kv * gm);
-            Qs[t * kKP + ch] = __float2bfloat16_rn(qv * f);
-            Ks[t * kKP + ch] = __float2bfloat16_rn(kv * f);
-            Kh[t * kKP + ch] = __float2bfloat16_rn(kv * fi);
-        }
-        __syncthreads();   // the block edges are in (and the half sums read)
-        if (tid < 64) {    // D_IJ = 2^(lam_{s_I} - lam_{e_J}) (I > J), c_J = 2^(lam_{e_J} - lam_{s_J}) (J < 3), channel pairs
-            const int c2 = 2 * tid;
             auto pair = [&](float a0, float a1) {
                 const __nv_bfloat162 h = __floats2bfloat162_rn(ex2(a0), ex2(a1));
                 return *reinterpret_cast<const uint32_t *>(&h);
@@ -750,15 +749,40 @@ kda_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
 #pragma unroll
             for (int I = 1; I < 4; ++I)
 #pragma unroll
-                for (int J = 0; J < I; ++J)
-                    D[(I * (I - 1) / 2 + J) * 64 + tid] = pair(edge[I * kD + c2] - edge[(4 + J) * kD + c2],
-                                                               edge[I * kD + c2 + 1] - edge[(4 + J) * kD + c2 + 1]);
+                for (int J = 0; J < I; ++J) {   // lam_{s_I} - lam_{e_J}: I's first step and the blocks between
+                    float e0 = fb[I][0], e1 = fb[I][1];
 #pragma unroll
-            for (int J = 0; J < 3; ++J)
-                D[(6 + J) * 64 + tid] = pair(edge[(4 + J) * kD + c2] - edge[J * kD + c2],
-                                             edge[(4 + J) * kD + c2 + 1] - edge[J * kD + c2 + 1]);
+                    for (int K = J + 1; K < I; ++K) {
+                        e0 += tb[K][0];
+                        e1 += tb[K][1];
+                    }
+                    D[(I * (I - 1) / 2 + J) * 64 + cp] = pair(e0, e1);
+                }
+#pragma unroll
+            for (int J = 0; J < 3; ++J) D[(6 + J) * 64 + cp] = pair(tb[J][0] - fb[J][0], tb[J][1] - fb[J][1]);
         }
-        __syncthreads();
+        // ---- per element pair: Q o Gam and K o 2^(lam_L - lam) (images, for the record), K o Gam
+        // (for W), and the Gram operands Q F, K F (in place) and K Fi, F = 2^(lb - lb_{s_J0})
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const int t = 16 * J0 + m;
+            const float2 qv = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(Qs + t * kKP + c2));
+            const float2 kv = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(Ks + t * kKP + c2));
+            const float l0 = lx[m][0] + ox0, l1 = lx[m][1] + ox1;
+            const float gm0 = ex2(l0), gm1 = ex2(l1);
+            const float d0 = lb[m][0] - lb[0][0], d1 = lb[m][1] - lb[0][1];   // <= 0, >= 15 kGramLog2Floor
+            const float fa0 = ex2(d0), fa1 = ex2(d1);
+            const float fi0 = ex2(-d0), fi1 = ex2(-d1);
+            const uint32_t o = img2_off(t, c2);
+            *reinterpret_cast<uint32_t *>(imR + o) = pack_bf16x2(qv.x * gm0, qv.y * gm1);
+            *reinterpret_cast<uint32_t *>(imR + 16384 + o) =
+                pack_bf16x2(kv.x * ex2(lL0 - l0), kv.y * ex2(lL1 - l1));
+            *reinterpret_cast<uint32_t *>(Kg + t * kKP + c2) = pack_bf16x2(kv.x * gm0, kv.y * gm1);
+            *reinterpret_cast<uint32_t *>(Qs + t * kKP + c2) = pack_bf16x2(qv.x * fa0, qv.y * fa1);
+            *reinterpret_cast<uint32_t *>(Ks + t * kKP + c2) = pack_bf16x2(kv.x * fa0, kv.y * fa1);
+            *reinterpret_cast<uint32_t *>(Kh + t * kKP + c2) = pack_bf16x2(kv.x * fi0, kv.y * fi1);
+        }
+        __syncthreads();   // the operands and the block factors are in
         // ---- Gram products: warp w rows 16 (w & 3) (block I), columns 32 (w >> 2) (blocks J)
         const int I = warp & 3, Jp = warp >> 2, m0 = 16 * I;
         const int g = lane >> 2, t4 = lane & 3;
@@ -867,21 +891,19 @@ kda_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
                 }
         }
         __syncthreads();
-        {   // the record: A and T diag(b), Q o Gam, W, K o 2^(lam_L - lam)
-            uint4 *d = reinterpret_cast<uint4 *>(rc);
-            const uint4 *sa = reinterpret_cast<const uint4 *>(imA), *sr = reinterpret_cast<const uint4 *>(imR),
-                        *sw = reinterpret_cast<const uint4 *>(imW);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int p = tid + kFacT * i;
-                d[kKrA / 16 + p] = sa[p];
-                d[kKrQg / 16 + p] = sr[p];
-                d[kKrW / 16 + p] = sw[p];
-                d[kKrKl / 16 + p] = sr[1024 + p];
-            }
+        fence_async_smem();   // the images leave by bulk copies
+        __syncthreads();
+        if (tid == 0) {   // the record: A and T diag(b), Q o Gam, W, K o 2^(lam_L - lam)
+            bulk_store(rc + kKrA, smem_u32(imA), 16384);
+            bulk_store(rc + kKrQg, smem_u32(imR), 16384);
+            bulk_store(rc + kKrW, smem_u32(imW), 16384);
+            bulk_store(rc + kKrKl, smem_u32(imR + 16384), 16384);
+            tma_store_commit();
+            tma_store_wait_read<0>();   // (before the next chunk's rows land on the images)
         }
-        __syncthreads();   // the tiles are free for the next chunk's rows
+        __syncthreads();
     }
+    if (tid == 0) tma_store_wait_all<0>();
 }
 
 template <int VAR>
