@@ -419,6 +419,7 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
         float *Lm = reinterpret_cast<float *>(Qs);   // over Q
         float *Tm = reinterpret_cast<float *>(Ks);   // over K
         cp_async_wait_all();
+        if (tid == 0) tma_store_wait_read<0>();   // the previous chunk's images have been read out
         __syncthreads();   // this chunk's rows are in; the other buffer and the images are free
         const bool pref = item + (int)gridDim.x < total;
         if constexpr (CONV) {
@@ -584,12 +585,15 @@ gdn_chunk_factors_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat1
             st_row_bf16x16(smem_u32(im + 8192), t, j0 >> 3, v1);
             st_row_bf16x16(smem_u32(im + 16384), t, j0 >> 3, v2);
         }
+        fence_async_smem();   // the images leave by a bulk copy
         __syncthreads();
-        uint4 *dst = reinterpret_cast<uint4 *>(img + (size_t)item * kImgHalves);
-        for (int p = tid; p < 3 * 512; p += kFacT) dst[p] = reinterpret_cast<const uint4 *>(im)[p];
+        if (tid == 0) {
+            bulk_store(img + (size_t)item * kImgHalves, smem_u32(im), 3 * 8192);
+            tma_store_commit();
+        }
     }
     cp_async_wait_all();
-    if constexpr (CONV) tma_store_wait_all<0>();
+    tma_store_wait_all<0>();
 }
 
 // ---------------------------------------------------------------------------------------
