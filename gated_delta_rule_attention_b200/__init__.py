@@ -222,6 +222,12 @@ def prefill(q, k, v, *, mode: int, gate=None, beta=None, state=None, z=None, o=N
     CUDA tensors run in place on the current stream.  If the inputs are CPU tensors they
     are copied to the current CUDA device, the call runs there, and the outputs are
     copied back to the CPU (the end-to-end path); the computation is still the kernel's.
+
+    ``workspace``: "auto" (a per-stream scratch buffer of ``workspace_size`` bytes, kept for
+    later calls), None (no scratch: the kernels' single-pass or smallest forms), or a uint8
+    CUDA tensor.  The fastest forms can need a large one: the gated delta rule and KDA with
+    16 to 37 head rows keep per-chunk factors (24 KB, KDA 66 048 bytes, per chunk and head
+    row: 0.4 and 1.08 GB at B2 H16 T32768).
     """
     host = q.device.type == "cpu"
     if host:
