@@ -57,7 +57,9 @@ struct SimtSmem {
     static constexpr int kA = C * SA;
     static constexpr int kLamC = (MODE == 3) ? kQ : 0;   // per-channel log-gate prefix
     static constexpr int kFloats = kS + 3 * kQ + kV + 2 * kA + 4 * C + DK + kLamC;
-    static constexpr size_t kBytes = sizeof(float) * kFloats;
+    static constexpr int kRawOff = (kFloats + 3) & ~3;   // 16-byte aligned: the next chunk's raw rows
+    template <typename IO>
+    static constexpr size_t bytes() { return sizeof(float) * kRawOff + sizeof(IO) * (2 * C * DK + C * DV); }
 };
 
 template <int MODE, int DK, int DV, int C, typename IO>
@@ -83,6 +85,9 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
     float *dec = den + C;            // [C]
     float *zs = dec + C;             // [DK]
     float *lamC = zs + DK;           // [C][DK+1]  mode 3
+    IO *Rq = reinterpret_cast<IO *>(smem + L::kRawOff);   // raw q, k, v rows of the next chunk
+    IO *Rk = Rq + C * DK;
+    IO *Rv = Rk + C * DK;
 
     constexpr int SK = L::SK, SV = L::SV, SA = L::SA;
     const int tid = threadIdx.x, lane = tid & 31;
@@ -119,21 +124,42 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
     const float *bh_beta = beta ? beta + row0 : nullptr;
     float *Sg = state + bh * (size_t)DV * DK;
 
+    // the raw q, k, v rows [t0, t0 + C) of the CTA's tokens into Rq, Rk, Rv (16-byte copies,
+    // in flight while the previous chunk is processed; rows past the end are not copied)
+    auto issue_raw = [&](int t0) {
+        const int Lc = min(C, n - t0);
+        constexpr int QK16 = DK * (int)sizeof(IO) / 16, V16 = DV * (int)sizeof(IO) / 16;
+        for (int p = tid; p < Lc * QK16; p += kSimtThreads) {
+            const int i = p / QK16, x = p % QK16;
+            cp_async16(reinterpret_cast<uint8_t *>(Rq + i * DK) + 16 * x,
+                       reinterpret_cast<const uint8_t *>(qh + (size_t)(t0 + i) * DK) + 16 * x);
+            cp_async16(reinterpret_cast<uint8_t *>(Rk + i * DK) + 16 * x,
+                       reinterpret_cast<const uint8_t *>(kh + (size_t)(t0 + i) * DK) + 16 * x);
+        }
+        for (int p = tid; p < Lc * V16; p += kSimtThreads) {
+            const int i = p / V16, x = p % V16;
+            cp_async16(reinterpret_cast<uint8_t *>(Rv + i * DV) + 16 * x,
+                       reinterpret_cast<const uint8_t *>(vh + (size_t)(t0 + i) * DV) + 16 * x);
+        }
+        cp_async_commit();
+    };
+    if (n > 0) issue_raw(0);
     for (int p = tid; p < DV * DK; p += kSimtThreads)
         S[(p / DK) * SK + p % DK] = init_state ? Sg[p] : 0.f;
     if (MODE == 0)
         for (int p = tid; p < DK; p += kSimtThreads) zs[p] = init_state ? zg[bh * DK + p] : 0.f;
-    __syncthreads();
 
     for (int t0 = 0; t0 < n; t0 += C) {
         const int Lc = min(C, n - t0);
-        // ---- load the chunk (phi applied in mode 0) and the gates
+        cp_async_wait_all();
+        __syncthreads();   // the chunk's raw rows are in (and the previous chunk is done)
+        // ---- the chunk's tiles from the raw rows (phi applied in mode 0) and the gates
         for (int p = tid; p < C * DK; p += kSimtThreads) {   // rows past the chunk's end: zero
             const int i = p / DK, j = p % DK;
             float qv = 0.f, kv = 0.f;
             if (i < Lc) {
-                qv = to_f32(qh[(size_t)(t0 + i) * DK + j]);
-                kv = to_f32(kh[(size_t)(t0 + i) * DK + j]);
+                qv = to_f32(Rq[i * DK + j]);
+                kv = to_f32(Rk[i * DK + j]);
                 if (MODE == 0) { qv = feature_phi(qv); kv = feature_phi(kv); }
             }
             Qs[i * SK + j] = qv;
@@ -141,7 +167,7 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
             if (kDelta) Ws[i * SK + j] = 0.f;
         }
         for (int p = tid; p < C * DV; p += kSimtThreads)
-            Vs[(p / DV) * SV + p % DV] = p / DV < Lc ? to_f32(vh[(size_t)(t0 + p / DV) * DV + p % DV]) : 0.f;
+            Vs[(p / DV) * SV + p % DV] = p / DV < Lc ? to_f32(Rv[(p / DV) * DV + p % DV]) : 0.f;
         if (tid < Lc) {
             lam[tid] = (MODE != 0 && MODE != 3 && gh) ? logf(fmaxf(gh[(t0 + tid) * gt], FLT_MIN)) : 0.f;
             bet[tid] = kDelta ? bh_beta[t0 + tid] : 0.f;
@@ -155,7 +181,8 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
                 }
             }
         }
-        __syncthreads();
+        __syncthreads();   // the raw rows are read: the next chunk's may land
+        if (t0 + C < n) issue_raw(t0 + C);
         if (tid == 0)
             for (int i = 1; i < Lc; ++i) lam[i] += lam[i - 1];
         __syncthreads();
@@ -311,13 +338,14 @@ prefill_simt_kernel(int T, int H, const int *__restrict__ cu, const IO *__restri
 template <int MODE, int DK, int DV, int C, typename IO>
 cudaError_t launch_one(const PrefillArgs &a) {
     using L = SimtSmem<MODE, DK, DV, C>;
+    constexpr size_t kBytes = L::template bytes<IO>();
+    static_assert(kBytes <= 227 * 1024, "shared memory per CTA");
     auto kern = prefill_simt_kernel<MODE, DK, DV, C, IO>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)L::kBytes);
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBytes);
     if (err != cudaSuccess) return err;
     timer_begin(a.stream);
     const unsigned grid = (unsigned)(a.cu ? (size_t)a.nseq * a.H : (size_t)a.B * a.H);
-    kern<<<grid, kSimtThreads, L::kBytes, a.stream>>>(
+    kern<<<grid, kSimtThreads, kBytes, a.stream>>>(
         a.T, a.H, a.cu, static_cast<const IO *>(a.q), static_cast<const IO *>(a.k),
         static_cast<const IO *>(a.v), a.gate, a.beta, a.state, a.z, static_cast<IO *>(a.o),
         a.init_state ? 1 : 0, device_error_word(), a.gate_heads);
