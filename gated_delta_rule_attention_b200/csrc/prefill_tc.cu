@@ -125,9 +125,9 @@ struct TcParams {
     // kLocalTrans: CTAs from `split` on run the transition pass and write s_out2
     int split;
     float *s_out2;
-    // Packed variable-length sequences (nullptr: dense).  CTA (s, h) takes tokens
-    // [cu[s], cu[s+1]) of head row h of the packed [H][T][128] tensors; its state is
-    // slot s of the s_in / s_out segment stride.
+    // Packed variable-length sequences (nullptr: dense; nseg = their number).  A CTA of
+    // sequence s and head row h takes tokens [cu[s], cu[s+1]) of head row h of the packed
+    // [H][T][128] tensors; its state is slot s of the s_in / s_out segment stride.
     const int *cu;
 };
 
@@ -137,10 +137,43 @@ struct TcParams {
 struct CtaRange {
     int bh, seg, tb, te;
 };
+// Packed sequences are served longest first: the CTAs of the r-th longest sequence (ties by
+// index) come r-th in launch order, so that the longest ones start in the first wave instead
+// of trailing it.  Every warp ranks the sequences itself (lane s counts the sequences ahead
+// of sequence s), so no shared memory or barrier is involved; with more than 128 sequences
+// they are taken in order.
+__device__ __forceinline__ int packed_sequence_of_rank(const TcParams &p, int r) {
+    if (p.nseg > 128) return r;
+    auto len = [&](int i) -> int {
+        const int a = min(max(p.cu[i], 0), p.T);
+        return min(max(p.cu[i + 1], a), p.T) - a;
+    };
+    const int lane = threadIdx.x & 31;
+    int sel = r;
+    for (int s0 = 0; s0 < p.nseg; s0 += 32) {
+        const int s = s0 + lane;
+        bool hit = false;
+        if (s < p.nseg) {
+            const int ls = len(s);
+            int rank = 0;
+            for (int j = 0; j < p.nseg; ++j) {
+                const int lj = len(j);
+                rank += (lj > ls || (lj == ls && j < s)) ? 1 : 0;
+            }
+            hit = rank == r;
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (m) sel = s0 + __ffs(m) - 1;
+    }
+    return sel;
+}
+// (RANKED = false: packed sequences in launch order.  Only the outputs passes ever run packed;
+// the mode-0 one takes the launch order, its registers having no room for the ranking.)
+template <bool RANKED = true>
 __device__ __forceinline__ CtaRange cta_range(const TcParams &p, int idx) {
     CtaRange r;
     r.bh = idx % p.BH;
-    r.seg = idx / p.BH;
+    r.seg = (RANKED && p.cu) ? packed_sequence_of_rank(p, idx / p.BH) : idx / p.BH;
     if (p.cu) {
         const int a = p.cu[r.seg], b = p.cu[r.seg + 1];
         r.tb = min(max(a, 0), p.T);
@@ -337,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const CtaRange rng = cta_range(p, (int)blockIdx.x - (KIND == kLocalTrans && trans ? p.split : 0));
+    const CtaRange rng = cta_range<KIND == kOutput>(p, (int)blockIdx.x - (KIND == kLocalTrans && trans ? p.split : 0));
     const int bh = rng.bh, seg = rng.seg, tb = rng.tb, te = rng.te;
     if (te <= tb) return;   // an empty packed sequence: nothing to read or write
     const int nch = (te - tb + kC - 1) / kC;
@@ -993,7 +1026,7 @@ __global__ void __launch_bounds__(kThreads01, 1) prefill01_kernel(const __grid_c
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const CtaRange rng = cta_range(p, (int)blockIdx.x);
+    const CtaRange rng = cta_range<KIND == kOutput>(p, (int)blockIdx.x);
     const int bh = rng.bh, seg = rng.seg, tb = rng.tb, te = rng.te;
     if (te <= tb) return;   // an empty packed sequence: nothing to read or write
     const int nch = (te - tb + kC - 1) / kC;
@@ -1423,7 +1456,7 @@ __global__ void __launch_bounds__(kThreadsE, 1) prefill_elu_kernel(const __grid_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const CtaRange rng = cta_range(p, (int)blockIdx.x);
+    const CtaRange rng = cta_range<false>(p, (int)blockIdx.x);
     const int bh = rng.bh, seg = rng.seg, tb = rng.tb, te = rng.te;
     if (te <= tb) return;   // an empty packed sequence: nothing to read or write
     const int nch = (te - tb + kC - 1) / kC;
