@@ -6,7 +6,8 @@ head) slice with the tolerance of the dense prefill (2e-2 bf16, 2e-3 fp32 I/O). 
 length mixes put sequence ends inside, at, and just past chunk boundaries, with empty
 and one-token sequences; the tensor-core path (bf16, d = 128, modes 0-2) and the
 CUDA-core path (fp32, d = 64, and mode 3) are both covered, with and without start
-states, plus a bad offsets table (clamped and reported, nothing out of bounds) and the
+states, plus a bad offsets table (clamped and reported, nothing out of bounds), the
+longest-first schedule of the outputs passes (ties, more than 128 sequences) and the
 serving-batch workload the benchmark times, on sampled sequences.
 """
 import numpy as np
@@ -89,6 +90,45 @@ def test_varlen_equals_separate_dense_calls(la):
         torch.cuda.synchronize()
         assert torch.equal(o[:, a:b], od[0]), f"sequence {s}: outputs differ"
         assert torch.equal(S[s], Sd[0])
+
+
+@pytest.mark.parametrize("lengths", [
+    [64] * 5 + [1] * 3 + [200, 65] + [64] * 4,          # ties: equal lengths keep index order
+    [(37 * i) % 150 for i in range(130)],               # more than 128 sequences: launch order
+])
+def test_varlen_longest_first_schedule(la, lengths):
+    """The outputs passes take packed sequences longest first (ties by index), ranking them in
+    every warp, up to 128 sequences, and in launch order beyond: each sequence's outputs and
+    final state are still its own (bit for bit against the call on the sequences in reverse
+    order, whose schedule differs), and match the oracle on sampled sequences."""
+    w = base(2, torch.bfloat16, 128, seed=302)
+    inp = W.varlen_inputs(w, lengths, device="cuda")
+    cu = [int(x) for x in inp["cu"].tolist()]
+    o, S, _ = la.prefill_varlen(inp["q"], inp["k"], inp["v"], inp["cu"], mode=2, gate=inp["gate"],
+                                beta=inp["beta"])
+    la.check_status()
+    # the same sequences packed in reverse order
+    N = len(lengths)
+    rev = list(range(N))[::-1]
+    cat = lambda t: torch.cat([t[:, cu[s]:cu[s + 1]] for s in rev], dim=1).contiguous()
+    rcu = torch.tensor(np.concatenate([[0], np.cumsum([lengths[s] for s in rev])]), dtype=torch.int32,
+                       device="cuda")
+    o2, S2, _ = la.prefill_varlen(cat(inp["q"]), cat(inp["k"]), cat(inp["v"]), rcu, mode=2,
+                                  gate=cat(inp["gate"]), beta=cat(inp["beta"]))
+    la.check_status()
+    rc = [int(x) for x in rcu.tolist()]
+    for j, s in enumerate(rev):
+        assert torch.equal(o[:, cu[s]:cu[s + 1]], o2[:, rc[j]:rc[j + 1]]), f"sequence {s}"
+        assert torch.equal(S[s], S2[j]), f"state {s}"
+    g = lambda t: f64(t)
+    pick = [s for s in (0, 5, 8, N - 1) if lengths[s] > 0][:3]
+    for s in pick:
+        a, b = cu[s], cu[s + 1]
+        sub = lambda t: t[:, a:b]
+        ro, rS, _ = oracle.prefill_packed(2, g(sub(inp["q"])), g(sub(inp["k"])), g(sub(inp["v"])), [0, b - a],
+                                          g(sub(inp["gate"])), g(sub(inp["beta"])), None, None)
+        assert seq_err(f64(o[:, a:b]), ro, [0, b - a]) < TOL[torch.bfloat16], f"sequence {s}"
+        assert slice_rel_err(f64(S[s:s + 1]), rS) < TOL[torch.bfloat16], f"state {s}"
 
 
 def test_varlen_bad_offsets_are_reported(la):
